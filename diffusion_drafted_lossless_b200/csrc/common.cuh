@@ -1,0 +1,88 @@
+// common.cuh — shared helpers of the Uno B200 library (device status word, error plumbing,
+// order-preserving keys, small warp utilities).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#include "../../include/uno.h"
+
+namespace uno {
+
+constexpr unsigned kFullMask = 0xFFFFFFFFu;
+
+// ------------------------------------------------------------------------------------
+// host-side error reporting (thread-local last error)
+// ------------------------------------------------------------------------------------
+uno_status set_error(uno_status s, const char* fmt, ...);
+uno_status check_cuda(cudaError_t e, const char* what);
+
+// Device status word: kernels record UNO_ERR_TIMEOUT there when a bounded wait gives up.
+// device_status_ptr() is its device address on the current device (defined in api.cu).
+uint32_t* device_status_ptr();
+
+__device__ __forceinline__ void record_device_status(uint32_t* status, uint32_t code) {
+    atomicCAS(status, 0u, code);
+}
+
+// ------------------------------------------------------------------------------------
+// order-preserving 32-bit keys of float values (bf16 values are widened first).
+// -0.0 is mapped to +0.0 so that the two compare equal, as they do as numbers.
+// ------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t float_key(float f) {
+    uint32_t x = __float_as_uint(f);
+    if (x == 0x80000000u) x = 0u;
+    return (x & 0x80000000u) ? ~x : (x | 0x80000000u);
+}
+
+__device__ __forceinline__ float key_float(uint32_t k) {
+    uint32_t x = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
+    return __uint_as_float(x);
+}
+
+// packed candidate: larger = higher priority = (value desc, token id asc)
+__device__ __forceinline__ uint64_t pack_candidate(uint32_t key, uint32_t id) {
+    return ((uint64_t)key << 32) | (uint64_t)(0xFFFFFFFFu - id);
+}
+__device__ __forceinline__ uint32_t candidate_id(uint64_t c) { return 0xFFFFFFFFu - (uint32_t)(c & 0xFFFFFFFFu); }
+__device__ __forceinline__ uint32_t candidate_key(uint64_t c) { return (uint32_t)(c >> 32); }
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// streaming 16-byte load: read once, do not keep in L1
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+    return r;
+}
+
+template <typename T>
+__device__ __forceinline__ T warp_sum(T v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFullMask, v, o);
+    return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFullMask, v, o));
+    return v;
+}
+
+// inclusive scan over the 32 lanes of a warp
+template <typename T>
+__device__ __forceinline__ T warp_inclusive_scan(T v, int lane) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        T t = __shfl_up_sync(kFullMask, v, o);
+        if (lane >= o) v += t;
+    }
+    return v;
+}
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace uno

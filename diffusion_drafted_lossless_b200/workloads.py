@@ -230,14 +230,38 @@ def verify_uniforms(w: VerifyWorkload) -> np.ndarray:
     return uniforms(w.seed + 1000, (w.B, w.K, 3))
 
 
+def _block_rows(seed: int, tag: int, blk: int, n_rows: int, n_cols: int, need: int) -> np.ndarray:
+    """The first `need` standard-normal rows of block `blk` of an [n_rows, n_cols] tensor."""
+    return _rng(seed, tag, blk).standard_normal((min(need, n_rows - blk * ROW_BLOCK), n_cols), dtype=np.float32)
+
+
 def tv_logits(w: TVWorkload, rows: np.ndarray | None = None) -> tuple[np.ndarray, np.ndarray]:
     """Teacher ~ N(0, 3^2) and student = teacher + N(0, 1), both bf16 bits [n, V].
 
-    The noise is added to the teacher draw before rounding; each is rounded once.
+    The noise is added to the teacher draw before rounding; each is rounded once. Each
+    block of rows is generated and rounded by one worker thread, so only the bf16 outputs
+    are ever held in full. Row r equals normal_rows(...)[r] of the same streams.
     """
-    t = normal_rows(w.seed, TAG_TEACHER, w.N, w.V, w.teacher_sigma, rows)
-    e = normal_rows(w.seed, TAG_STUDENT_NOISE, w.N, w.V, w.noise_sigma, rows)
-    return bf16_bits(t), bf16_bits(t + e)
+    rows = np.arange(w.N) if rows is None else np.asarray(rows, dtype=np.int64)
+    T = np.empty((len(rows), w.V), dtype=np.uint16)
+    S = np.empty((len(rows), w.V), dtype=np.uint16)
+
+    def work(item):
+        blk, idx = item
+        need = int(rows[idx].max() % ROW_BLOCK) + 1
+        sel = rows[idx] % ROW_BLOCK
+        t = _block_rows(w.seed, TAG_TEACHER, blk, w.N, w.V, need)[sel]
+        t *= np.float32(w.teacher_sigma)
+        e = _block_rows(w.seed, TAG_STUDENT_NOISE, blk, w.N, w.V, need)[sel]
+        e *= np.float32(w.noise_sigma)
+        T[idx] = bf16_bits(t)
+        e += t
+        S[idx] = bf16_bits(e)
+
+    items = list(_blocks_for(rows).items())
+    with ThreadPoolExecutor(_threads()) as ex:
+        list(ex.map(work, items))
+    return T, S
 
 
 def to_f64(a: np.ndarray, dtype: str) -> np.ndarray:

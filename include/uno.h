@@ -1,0 +1,207 @@
+/*
+ * uno.h — C ABI of the Uno draft-and-verify hot path on NVIDIA B200 (sm_100a).
+ *
+ * Three operations, each stated by the Uno pages:
+ *   uno_gated_lora_linear  the row-gated LoRA projection (LoopUno project page, "How it
+ *                          works" and "Setup / Recipe"; uno-qwen3-8B model card intro)
+ *   uno_block_verify       lossless verification of a drafted block (LoopUno project page,
+ *                          "How it works", "Training is self-distillation"; model card,
+ *                          "Evaluation protocol")
+ *   uno_tv_loss            the TV self-distillation loss and its gradient (LoopUno project
+ *                          page, "Training is self-distillation")
+ *
+ * Conventions shared by every entry point
+ *   - Pointers named as tensors are DEVICE pointers owned by the caller, row-major and
+ *     contiguous, unless a comment says "host". The library never allocates, frees or
+ *     keeps caller memory, and never synchronises the stream.
+ *   - Scratch memory is a caller-supplied device `workspace` of at least the size the
+ *     matching uno_*_workspace_size() reports (256-byte aligned). A workspace may be reused
+ *     by later calls on the same stream, but two calls that may run at the same time need
+ *     two workspaces.
+ *   - Every call validates its arguments on the host before any launch and returns a
+ *     uno_status; on error nothing is launched and no output is written. Errors are never
+ *     signalled by a device trap. A call that returns UNO_OK has only been enqueued on
+ *     `stream` (asynchronous); results are ready after the stream reaches that point.
+ *   - uno_last_error_string() gives a readable reason for the calling thread's last
+ *     failing call.
+ *   - Device pointers must be 16-byte aligned.
+ *   - bf16 is IEEE-754 binary32 truncated to its upper 16 bits (1-8-7), stored as uint16.
+ */
+#ifndef UNO_H
+#define UNO_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream (cudaStream_t / CUstream). NULL is the legacy default stream. */
+typedef struct CUstream_st* uno_stream_t;
+
+typedef enum {
+    UNO_OK = 0,
+    UNO_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad scalar parameter */
+    UNO_ERR_UNSUPPORTED = 2,   /* shape / dtype / alignment outside the supported limits */
+    UNO_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed (see last error) */
+    UNO_ERR_TIMEOUT = 4,       /* a bounded device-side wait gave up (device status word) */
+    UNO_ERR_WORKSPACE = 5      /* workspace missing, too small or misaligned */
+} uno_status;
+
+typedef enum {
+    UNO_BF16 = 0,
+    UNO_F32 = 1
+} uno_dtype;
+
+/* Readable name of a status code (static storage). */
+const char* uno_status_string(uno_status status);
+
+/* Detail of the calling thread's last failing call ("" if none; thread-local storage). */
+const char* uno_last_error_string(void);
+
+/* ABI version of this library: major * 10000 + minor * 100 + patch. */
+int uno_version(void);
+
+/*
+ * Device status word: kernels whose bounded waits time out record UNO_ERR_TIMEOUT there
+ * instead of trapping. This call synchronises the current device, returns the word in
+ * *code (UNO_OK if no kernel recorded anything since the last read) and clears it.
+ */
+uno_status uno_read_device_status(uint32_t* code);
+
+/* ======================================================================================
+ * Row-gated LoRA linear
+ *
+ *   Y = X W0^T + scale * diag(g) (X A^T) B^T
+ *
+ * The frozen base weight W0 serves every row; the rank-r adapter (A, B) is added only on
+ * rows whose gate is non-zero (draft-noise rows; the seed / prefill / verify / AR rows
+ * have gate 0). Source: LoopUno project page, "How it works" (one LoRA switched on only for
+ * noise positions) and "Setup / Recipe" (gated LoRA, r=128, alpha=2048, all seven
+ * projections, noise rows only); uno-qwen3-8B model card introduction (adapter applied
+ * selectively on draft-noise rows).
+ *
+ *   x       [M, d_in]      activations, dtype
+ *   w0      [d_out, d_in]  frozen base weight (nn.Linear layout), dtype
+ *   lora_a  [rank, d_in]   adapter down-projection, dtype
+ *   lora_b  [d_out, rank]  adapter up-projection, dtype
+ *   row_gate[M] float32    per-row gate; NULL means all zeros (base layer only)
+ *   scale                  adapter scale (alpha / r under the standard LoRA reading)
+ *   y       [M, d_out]     output, dtype; must not overlap any input
+ *
+ * Arithmetic: bf16 tensor-core products with fp32 accumulation. The adapter's
+ * intermediate T = scale * g * (X A^T) is accumulated in fp32 and rounded once to bf16
+ * before the up-projection, which accumulates into the same fp32 accumulator as X W0^T;
+ * Y is rounded once to the output dtype. With dtype UNO_F32 the inputs are rounded to
+ * bf16 (round-to-nearest-even) on the device first and Y is written as float32.
+ *
+ * Limits (else UNO_ERR_UNSUPPORTED): d_in and d_out multiples of 64; rank a multiple of 8
+ * with 8 <= rank <= 256; 1 <= M <= 2^20; d_in, d_out <= 65536.
+ * Workspace: uno_gated_lora_linear_workspace_size(M, d_in, d_out, rank, dtype) bytes.
+ * ====================================================================================== */
+size_t uno_gated_lora_linear_workspace_size(int64_t M, int64_t d_in, int64_t d_out,
+                                            int64_t rank, uno_dtype dtype);
+
+uno_status uno_gated_lora_linear(const void* x, const void* w0, const void* lora_a,
+                                 const void* lora_b, const float* row_gate, float scale,
+                                 int64_t M, int64_t d_in, int64_t d_out, int64_t rank,
+                                 uno_dtype dtype, void* y, void* workspace,
+                                 size_t workspace_bytes, uno_stream_t stream);
+
+/* ======================================================================================
+ * Lossless block verify
+ *
+ * For each sequence b of a batch, a block of K positions was drafted in one forward.
+ * verifier_logits[b, i] gives the verifier's (frozen base model's) next-token logits at
+ * block position i, drafter_logits[b, i] the drafter's (model + gated LoRA). Both rows
+ * are warped the same way: z = logit / temperature; top-k (exactly k kept, ties to the
+ * lower token id); softmax; top-p (shortest prefix of the (probability desc, id asc)
+ * order whose cumulative mass is >= top_p, the crossing token included); renormalise.
+ * Call the results p_i and q_i.
+ *
+ *   x_0 = pos0_tokens[b], or the inverse-CDF draw of p_0 with uniforms[b,0,0]
+ *   d_i = draft_tokens[b,i], or the inverse-CDF draw of q_i with uniforms[b,i,0], i >= 1
+ *   draft i is accepted iff uniforms[b,i,1] * q_i(d_i) < p_i(d_i)  (prob. min(1, p/q))
+ *   n = 1 + number of leading accepted drafts (position 0 is always emitted)
+ *   at the first rejection j: next = inverse-CDF draw of normalise(max(0, p_j - q_j))
+ *   with uniforms[b,j,2] (p_j itself if that has no mass); next = -1 if all accepted.
+ *
+ * The inverse-CDF draw of a distribution w with uniform u returns the smallest token id t
+ * (ascending) whose cumulative mass sum_{s<=t} w_s exceeds u * sum(w).
+ * The acceptance probability is 1 - TV(p_i, q_i) and every emitted token is distributed
+ * as p_i: the verify is lossless. Source: LoopUno project page, "How it works" (the
+ * unmodified model verifies the block and keeps the longest correct prefix; the first
+ * position is always the exact AR token) and "Training is self-distillation" (acceptance
+ * probability is exactly 1 - TV); uno-qwen3-8B model card, "Evaluation protocol"
+ * (temperature 1.0, top-p 0.95, top-k 50, block 16).
+ *
+ *   verifier_logits [B, K, V]  dtype (bf16 or f32); all K rows used
+ *   drafter_logits  [B, K, V]  dtype; rows i >= 1 used (row 0 is never read)
+ *   temperature     > 0
+ *   top_k           0 = off; else 1 <= top_k <= 1024 (top_k >= V is the same as off)
+ *   top_p           (0, 1) filters; >= 1 = off
+ *   draft_tokens    [B, K] int32 or NULL (column 0 ignored); NULL: drawn from q_i
+ *   pos0_tokens     [B] int32 or NULL; NULL: drawn from p_0
+ *   uniforms        [B, K, 3] float32 in [0, 1): (sample, accept, resample)
+ *   out_tokens      [B, K] int32: x_0, d_1 .. d_{n-1}, then -1
+ *   out_count       [B] int32: n
+ *   out_next_token  [B] int32 or NULL: the correction token, -1 if every draft was accepted
+ *   out_p_tok       [B, K] float32 or NULL: p_i(token_i) (token_0 = x_0, token_i = d_i)
+ *   out_q_tok       [B, K] float32 or NULL: q_i(d_i); 0 at i = 0
+ *   out_tv          [B, K] float32 or NULL: TV(p_i, q_i) for i >= 1, 0 at i = 0
+ *
+ * Logits must be finite. Limits (else UNO_ERR_UNSUPPORTED): 1 <= K <= 32, 1 <= V < 2^31,
+ * B >= 0 (B = 0 does nothing), B * K * V < 2^40.
+ * Workspace: uno_block_verify_workspace_size(B, K, V, top_k, top_p, dtype) bytes.
+ * ====================================================================================== */
+size_t uno_block_verify_workspace_size(int32_t B, int32_t K, int32_t V, int32_t top_k,
+                                       float top_p, uno_dtype dtype);
+
+uno_status uno_block_verify(const void* verifier_logits, const void* drafter_logits,
+                            uno_dtype dtype, int32_t B, int32_t K, int32_t V,
+                            float temperature, int32_t top_k, float top_p,
+                            const int32_t* draft_tokens, const int32_t* pos0_tokens,
+                            const float* uniforms, int32_t* out_tokens, int32_t* out_count,
+                            int32_t* out_next_token, float* out_p_tok, float* out_q_tok,
+                            float* out_tv, void* workspace, size_t workspace_bytes,
+                            uno_stream_t stream);
+
+/* ======================================================================================
+ * TV self-distillation loss and its gradient
+ *
+ *   p_t = softmax(teacher_logits[t]), q_t = softmax(student_logits[t])   (T = 1, no filter)
+ *   tv[t] = 1/2 sum_v |p_t,v - q_t,v|
+ *   mean  = sum over masked tokens of tv[t] / N_mask        (0 when no token is masked in)
+ *   grad_student[t, v] = grad_scale / N_mask * q_t,v * (s_v - sum_w q_t,w s_w)
+ *                        with s = 1/2 sign(q_t - p_t), sign(0) = 0; 0 on unmasked tokens
+ *
+ * The teacher (frozen model on the clean copy) is constant; the student is model + LoRA
+ * on the block-noised copy. Source: LoopUno project page, "Training is
+ * self-distillation" (TV distance between the two next-token distributions on the
+ * response tokens) and "Setup / Recipe" (objective: TV distance to the frozen model's own
+ * distribution).
+ *
+ *   teacher_logits, student_logits [N, V] dtype (bf16 or f32)
+ *   response_mask  [N] uint8 or NULL (NULL: every token counts)
+ *   grad_scale     dL/dmean (1 for the plain mean)
+ *   out_tv         [N] float32
+ *   out_mean       [1] float32
+ *   grad_student   [N, V] dtype or NULL (NULL: loss only)
+ *
+ * Logits must be finite. Limits (else UNO_ERR_UNSUPPORTED): 1 <= V < 2^31, N >= 0,
+ * N * V < 2^40.
+ * Workspace: uno_tv_loss_workspace_size(N, V, dtype) bytes.
+ * ====================================================================================== */
+size_t uno_tv_loss_workspace_size(int64_t N, int64_t V, uno_dtype dtype);
+
+uno_status uno_tv_loss(const void* teacher_logits, const void* student_logits,
+                       uno_dtype dtype, int64_t N, int64_t V, const uint8_t* response_mask,
+                       float grad_scale, float* out_tv, float* out_mean, void* grad_student,
+                       void* workspace, size_t workspace_bytes, uno_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* UNO_H */

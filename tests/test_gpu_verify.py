@@ -1,0 +1,166 @@
+"""GPU parity of uno_block_verify against the fp64 oracle (called through the C ABI).
+
+Sizes span several 256-element tiles with ragged tails (V not a multiple of the tile, and
+V not a multiple of the 16-byte vector so that rows are misaligned), every top-k capacity
+class, both dtypes, heavy ties, adversarial orderings, supplied drafts / position-0
+tokens, K = 1 and K = 32, and the serving-scale workload (B=64, K=16, V=151936) checked on
+sampled sequences.
+"""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from diffusion_drafted_lossless_b200 import workloads as W
+from tests.gpu_util import compare_verify, f32, verify_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+def _inputs(B, K, V, dtype, seed, sigma=3.0, rho=0.8):
+    w = W.VerifyWorkload("t", seed, B=B, K=K, V=V, sigma=sigma, rho=rho, temperature=1.0, top_k=0, top_p=1.0,
+                         dtype=dtype)
+    P, Q = W.verify_logits(w)
+    return P.reshape(B, K, V), Q.reshape(B, K, V), W.verify_uniforms(w)
+
+
+def _oracle(P, Q, u, T, top_k, top_p, dtype, drafts=None, pos0=None):
+    return oracle.block_verify(W.to_f64(P, dtype), W.to_f64(Q, dtype), u.astype(np.float64), f32(T), top_k,
+                               f32(top_p) if top_p < 1 else 1.0, drafts=drafts, pos0=pos0)
+
+
+def _check(P, Q, u, T, top_k, top_p, dtype, drafts=None, pos0=None):
+    gpu = verify_gpu(P, Q, u, T, top_k, top_p, dtype, drafts=drafts, pos0=pos0)
+    ref = _oracle(P, Q, u, T, top_k, top_p, dtype, drafts, pos0)
+    n, near, bad = compare_verify(gpu, ref)
+    assert not bad, bad[:5]
+    assert (gpu["count"] >= 1).all()
+    return gpu, ref, near
+
+
+CASES = [
+    ("bf16", 3, 5, 3000, 1.0, 50, 0.95),
+    ("bf16", 4, 8, 20000, 0.7, 1, 1.0),
+    ("bf16", 2, 16, 4099, 1.3, 64, 0.5),
+    ("bf16", 3, 4, 5000, 1.0, 100, 0.9),
+    ("bf16", 2, 3, 9000, 1.0, 700, 0.99),
+    ("f32", 3, 6, 2500, 1.0, 50, 0.95),
+    ("f32", 2, 5, 777, 2.0, 20, 1.0),
+    ("bf16", 5, 32, 1200, 1.0, 5, 0.8),
+    ("bf16", 3, 1, 500, 1.0, 10, 0.9),
+    ("bf16", 6, 16, 151936, 1.0, 50, 0.95),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[f"{c[0]}-B{c[1]}K{c[2]}V{c[3]}k{c[5]}" for c in CASES])
+def test_topk_parity(case):
+    dtype, B, K, V, T, k, p = case
+    P, Q, u = _inputs(B, K, V, dtype, seed=zlib.crc32(str(case).encode()) % 10007)
+    gpu, ref, near = _check(P, Q, u, T, k, p, dtype)
+    assert near <= max(1, B // 100)
+
+
+def test_heavy_ties():
+    B, K, V = 4, 6, 6000
+    rng = np.random.default_rng(31)
+    Pf = np.round(rng.standard_normal((B, K, V)) * 2) / 2  # values on a 0.5 grid: many ties
+    Qf = np.round((0.7 * Pf + 0.7 * rng.standard_normal((B, K, V))) * 2) / 2
+    P, Q = W.bf16_bits(Pf.astype(np.float32)), W.bf16_bits(Qf.astype(np.float32))
+    u = rng.random((B, K, 3), dtype=np.float32)
+    for k in (1, 7, 50, 200):
+        _check(P, Q, u, 1.0, k, 0.9, "bf16")
+
+
+@pytest.mark.parametrize("order", ["ascending", "descending", "constant", "one_hot"])
+def test_adversarial_orders(order):
+    B, K, V = 2, 4, 5000
+    base = np.linspace(-5, 5, V, dtype=np.float32)
+    if order == "descending":
+        base = base[::-1].copy()
+    elif order == "constant":
+        base = np.zeros(V, np.float32)
+    elif order == "one_hot":
+        base = np.full(V, -3.0, np.float32)
+        base[V // 2] = 4.0
+    P = np.broadcast_to(W.bf16_bits(base), (B, K, V)).copy()
+    Q = np.broadcast_to(W.bf16_bits(base[::-1].copy()), (B, K, V)).copy()
+    u = np.random.default_rng(32).random((B, K, 3), dtype=np.float32)
+    for k in (1, 50, 64, 300):
+        _check(P, Q, u, 1.0, k, 0.95, "bf16")
+
+
+def test_identical_rows_accept_all():
+    P, _, u = _inputs(4, 8, 10000, "bf16", seed=33)
+    gpu, ref, _ = _check(P, P, u, 1.0, 50, 0.95, "bf16")
+    assert (gpu["count"] == 8).all() and (gpu["next"] == -1).all()
+    np.testing.assert_allclose(gpu["tv"], 0.0, atol=1e-6)
+
+
+def test_supplied_drafts_and_pos0():
+    B, K, V = 5, 6, 3000
+    P, Q, u = _inputs(B, K, V, "bf16", seed=34)
+    rng = np.random.default_rng(34)
+    drafts = rng.integers(0, V, (B, K)).astype(np.int32)
+    # make some drafts the verifier's argmax so that acceptances happen
+    drafts[:, 1:3] = W.bf16_to_f32(P).reshape(B, K, V)[:, 1:3].argmax(axis=2)
+    pos0 = rng.integers(0, V, B).astype(np.int32)
+    gpu, ref, _ = _check(P, Q, u, 1.0, 50, 0.95, "bf16", drafts=drafts, pos0=pos0)
+    assert (gpu["tokens"][:, 0] == pos0).all()
+
+
+def test_empty_batch():
+    from diffusion_drafted_lossless_b200 import _lib
+    z = torch.empty((0, 4, 100), dtype=torch.bfloat16, device="cuda")
+    u = torch.empty((0, 4, 3), device="cuda")
+    t = torch.empty((0, 4), dtype=torch.int32, device="cuda")
+    c = torch.empty((0,), dtype=torch.int32, device="cuda")
+    _lib.uno_block_verify(z, z, 1.0, 50, 0.95, u, t, c)
+    torch.cuda.synchronize()
+
+
+def test_repeated_calls_reuse_workspace():
+    """Counters in the workspace are reset by each call: two calls give the same result."""
+    from diffusion_drafted_lossless_b200 import _lib
+    B, K, V = 3, 5, 7000
+    P, Q, u = _inputs(B, K, V, "bf16", seed=35)
+    ws = torch.empty(_lib.uno_block_verify_workspace_size(B, K, V, 50, 0.95), dtype=torch.uint8, device="cuda")
+    outs = []
+    for _ in range(3):
+        from tests.gpu_util import dev
+        t = torch.empty((B, K), dtype=torch.int32, device="cuda")
+        c = torch.empty((B,), dtype=torch.int32, device="cuda")
+        nx = torch.empty((B,), dtype=torch.int32, device="cuda")
+        _lib.uno_block_verify(dev(P, "bf16"), dev(Q, "bf16"), 1.0, 50, 0.95, torch.from_numpy(u).cuda(), t, c,
+                              nx, workspace=ws)
+        torch.cuda.synchronize()
+        outs.append((t.cpu().numpy(), c.cpu().numpy(), nx.cpu().numpy()))
+    for o in outs[1:]:
+        for a, b in zip(o, outs[0]):
+            np.testing.assert_array_equal(a, b)
+
+
+def test_serving_scale_sampled_sequences():
+    """B=64, K=16, V=151936 bf16, T=1, top-k 50, top-p 0.95 (the serving workload): the full
+    batch runs on the GPU; the oracle recomputes 6 sampled sequences one by one."""
+    w = W.SERVING_VERIFY
+    P, Q = W.verify_logits(w)
+    u = W.verify_uniforms(w)
+    B, K, V = w.B, w.K, w.V
+    gpu = verify_gpu(P.reshape(B, K, V), Q.reshape(B, K, V), u, w.temperature, w.top_k, w.top_p)
+    seqs = [0, 13, 27, 38, 51, 63]
+    rows = np.concatenate([np.arange(s * K, (s + 1) * K) for s in seqs])
+    ref = oracle.block_verify(W.to_f64(P[rows], "bf16").reshape(len(seqs), K, V),
+                              W.to_f64(Q[rows], "bf16").reshape(len(seqs), K, V),
+                              u[seqs].astype(np.float64), f32(w.temperature), w.top_k, f32(w.top_p))
+    sub = {k: (v[seqs] if v is not None else None) for k, v in gpu.items()}
+    n, near, bad = compare_verify(sub, ref)
+    assert not bad, bad
+    assert near <= 1
+    assert (gpu["count"] >= 1).all() and (gpu["count"] <= K).all()
+    # every sequence: tokens after the count are -1, next is -1 exactly when all accepted
+    for b in range(B):
+        c = gpu["count"][b]
+        assert (gpu["tokens"][b, c:] == -1).all() and (gpu["tokens"][b, :c] >= 0).all()
+        assert (gpu["next"][b] == -1) == (c == K)
