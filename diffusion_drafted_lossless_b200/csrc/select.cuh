@@ -154,3 +154,98 @@ __device__ void cta_sort_desc(uint64_t* a, int n) {
 }
 
 }  // namespace uno
+
+namespace uno {
+
+// Warp bitonic sort of n (power of two) 64-bit keys in shared memory, descending.
+__device__ __forceinline__ void warp_sort_desc(uint64_t* a, int n, int lane) {
+    for (int size = 2; size <= n; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int t = lane; t < n / 2; t += 32) {
+                int lo = 2 * t - (t & (stride - 1));
+                int hi = lo + stride;
+                bool desc = ((lo & size) == 0);
+                uint64_t x = a[lo], y = a[hi];
+                if ((x < y) == desc) {
+                    a[lo] = y;
+                    a[hi] = x;
+                }
+            }
+            __syncwarp();
+        }
+    }
+}
+
+}  // namespace uno
+
+namespace uno {
+
+// ------------------------------------------------------------------------------------
+// Selection on the value key only, for buffers kept in ascending token-id order.
+// Candidates are packed (key32 << 32 | ~id). KEYBITS = 16 for bf16 values (the low 16
+// bits of a widened bf16 key are fixed by its sign), 32 for fp32.
+// warp_select_key finds the key of the k-th largest entry (tau) and how many entries
+// equal to tau belong to the top-k (need); because the buffer is in id order, those are
+// the first `need` entries equal to tau, which warp_compact_key keeps (stable).
+// ------------------------------------------------------------------------------------
+template <int KEYBITS>
+__device__ __forceinline__ uint32_t radix_of(uint64_t c) {
+    return (uint32_t)(c >> (64 - KEYBITS));
+}
+
+template <int KEYBITS>
+__device__ __forceinline__ uint32_t key32_of_radix(uint32_t r) {
+    if (KEYBITS == 32) return r;
+    return (r << 16) | ((r & 0x8000u) ? 0x0000u : 0xFFFFu);
+}
+
+template <int KEYBITS>
+__device__ __forceinline__ void warp_select_key(const uint64_t* buf, int n, int k, uint32_t* hist, int lane,
+                                                uint32_t& tau_radix, int& need) {
+    uint32_t prefix = 0;
+    uint32_t k_rem = (uint32_t)k;
+#pragma unroll 1
+    for (int shift = KEYBITS - 8; shift >= 0; shift -= 8) {
+        const uint32_t hi_mask = (shift + 8 >= 32) ? 0u : (~0u << (shift + 8));
+#pragma unroll
+        for (int j = 0; j < 8; ++j) hist[lane * 8 + j] = 0u;
+        __syncwarp();
+        for (int i = lane; i < n; i += 32) {
+            uint32_t x = radix_of<KEYBITS>(buf[i]);
+            if ((x & hi_mask) == prefix) atomicAdd(&hist[(x >> shift) & 0xFFu], 1u);
+        }
+        __syncwarp();
+        int bin;
+        uint32_t above, cnt;
+        warp_find_bin(hist, k_rem, lane, bin, above, cnt);
+        __syncwarp();
+        prefix |= (uint32_t)bin << shift;
+        k_rem -= above;
+        (void)cnt;
+    }
+    tau_radix = prefix;
+    need = (int)k_rem;
+}
+
+// keep entries with radix > tau, and the first `need` (in buffer order) equal to tau
+template <int KEYBITS>
+__device__ __forceinline__ int warp_compact_key(uint64_t* buf, int n, uint32_t tau, int need, int lane) {
+    int out = 0, ties = 0;
+    for (int base = 0; base < n; base += 32) {
+        int i = base + lane;
+        uint64_t x = i < n ? buf[i] : 0ull;
+        uint32_t r = radix_of<KEYBITS>(x);
+        bool tie = i < n && r == tau;
+        unsigned tball = __ballot_sync(kFullMask, tie);
+        bool keep = i < n && (r > tau || (tie && ties + __popc(tball & ((1u << lane) - 1u)) < need));
+        unsigned ball = __ballot_sync(kFullMask, keep);
+        __syncwarp();
+        if (keep) buf[out + __popc(ball & ((1u << lane) - 1u))] = x;
+        out += __popc(ball);
+        ties += __popc(tball);
+        __syncwarp();
+    }
+    return out;
+}
+
+}  // namespace uno

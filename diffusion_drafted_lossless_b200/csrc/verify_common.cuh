@@ -116,115 +116,178 @@ __device__ inline RecView rec_view(unsigned char* recs, int kcap, int64_t row) {
     return r;
 }
 
-// probability of token t under the record's distribution (0 if not a survivor)
-__device__ inline double rec_prob(const RecView& R, int t) {
-    int n = __ldcg(R.n);
-    int lo = 0, hi = n - 1;
+// ------------------------------------------------------------------------------------
+// Warp-cooperative use of a record staged in shared memory (ids ascending, fp64 weights).
+// ------------------------------------------------------------------------------------
+struct SRec {
+    double* w;
+    int32_t* id;
+    int n;
+    double Z;
+};
+
+__device__ __forceinline__ double warp_scan_f64(double v, int lane) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        double t = __shfl_up_sync(kFullMask, v, o);
+        if (lane >= o) v += t;
+    }
+    return v;
+}
+
+__device__ __forceinline__ double warp_sum_f64(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFullMask, v, o);
+    return v;
+}
+
+// copy a global record into the warp's slice (w, id arrays of capacity kcap)
+__device__ inline SRec warp_stage_rec(unsigned char* recs, int kcap, int64_t row, double* w, int32_t* id, int lane) {
+    RecView R = rec_view(recs, kcap, row);
+    SRec s;
+    s.w = w;
+    s.id = id;
+    s.n = __ldcg(R.n);
+    s.Z = __ldcg(R.Z);
+    for (int j = lane; j < s.n; j += 32) {
+        w[j] = __ldcg(R.w + j);
+        id[j] = __ldcg(R.id + j);
+    }
+    __syncwarp();
+    return s;
+}
+
+// probability of token t (0 if not a survivor); every lane gets the same answer
+__device__ __forceinline__ double srec_prob(const SRec& R, int t) {
+    int lo = 0, hi = R.n - 1;
     while (lo <= hi) {
         int mid = (lo + hi) >> 1;
-        int v = __ldcg(R.id + mid);
-        if (v == t) return __ldcg(R.w + mid) / __ldcg(R.Z);
+        int v = R.id[mid];
+        if (v == t) return R.w[mid] / R.Z;
         if (v < t) lo = mid + 1;
         else hi = mid - 1;
     }
     return 0.0;
 }
 
-// inverse-CDF draw: smallest id (ascending) whose cumulative weight exceeds u * Z
-__device__ inline int rec_inv_cdf(const RecView& R, double u) {
-    int n = __ldcg(R.n);
-    double target = u * __ldcg(R.Z);
-    double cum = 0.0;
+// inverse-CDF draw over weights x_j (ascending id order): the first j whose cumulative
+// weight exceeds target; the last j with positive weight if rounding leaves no crossing.
+template <typename F>
+__device__ __forceinline__ int warp_inv_cdf_gen(int n, double target, int lane, F weight) {
+    double carry = 0.0;
     int last = -1;
-    for (int j = 0; j < n; ++j) {
-        double w = __ldcg(R.w + j);
-        if (w <= 0.0) continue;
-        cum += w;
-        last = __ldcg(R.id + j);
-        if (cum > target) return last;
+    for (int base = 0; base < n; base += 32) {
+        int j = base + lane;
+        double x = j < n ? weight(j) : 0.0;
+        double incl = warp_scan_f64(x, lane);
+        unsigned hit = __ballot_sync(kFullMask, x > 0.0 && carry + incl > target);
+        if (hit) return base + __ffs(hit) - 1;
+        unsigned pos = __ballot_sync(kFullMask, x > 0.0);
+        if (pos) last = base + 31 - __clz(pos);
+        carry += __shfl_sync(kFullMask, incl, 31);
     }
     return last;
 }
 
-// residual draw: normalise(max(0, p - q)) over p's survivors (q's tokens outside p's
-// survivors have p = 0 and so no residual mass); p itself if the residual is empty
-__device__ inline int rec_residual(const RecView& P, const RecView& Q, double u) {
-    int n = __ldcg(P.n);
-    double Zp = __ldcg(P.Z);
-    double R = 0.0;
-    for (int j = 0; j < n; ++j) {
-        double d = __ldcg(P.w + j) / Zp - rec_prob(Q, __ldcg(P.id + j));
-        R += d > 0.0 ? d : 0.0;
-    }
-    if (!(R > 0.0)) return rec_inv_cdf(P, u);
-    double target = u * R, cum = 0.0;
-    int last = -1;
-    for (int j = 0; j < n; ++j) {
-        int id = __ldcg(P.id + j);
-        double d = __ldcg(P.w + j) / Zp - rec_prob(Q, id);
-        if (!(d > 0.0)) continue;
-        cum += d;
-        last = id;
-        if (cum > target) return id;
-    }
-    return last;
+__device__ __forceinline__ int srec_inv_cdf(const SRec& R, double u, int lane) {
+    int j = warp_inv_cdf_gen(R.n, u * R.Z, lane, [&](int i) { return R.w[i]; });
+    return j >= 0 ? R.id[j] : -1;
 }
 
 // TV(p, q) = 1/2 (sum over p's survivors |p - q| + q's mass outside p's survivors)
-__device__ inline double rec_tv(const RecView& P, const RecView& Q) {
+__device__ __forceinline__ double srec_tv(const SRec& P, const SRec& Q, int lane) {
     double s = 0.0;
-    int np = __ldcg(P.n), nq = __ldcg(Q.n);
-    double Zp = __ldcg(P.Z), Zq = __ldcg(Q.Z);
-    for (int j = 0; j < np; ++j) s += fabs(__ldcg(P.w + j) / Zp - rec_prob(Q, __ldcg(P.id + j)));
-    for (int j = 0; j < nq; ++j)
-        if (rec_prob(P, __ldcg(Q.id + j)) == 0.0) s += __ldcg(Q.w + j) / Zq;
-    return 0.5 * s;
+    for (int j = lane; j < P.n; j += 32) s += fabs(P.w[j] / P.Z - srec_prob(Q, P.id[j]));
+    for (int j = lane; j < Q.n; j += 32)
+        if (srec_prob(P, Q.id[j]) == 0.0) s += Q.w[j] / Q.Z;
+    return 0.5 * warp_sum_f64(s);
 }
 
-// Per-sequence verify, one warp, lane i = block position i (K <= 32). Rows of sequence b:
-// records rbase + i are the verifier rows i = 0..K-1, rbase + K + i - 1 the drafter rows.
-__device__ inline void sequence_verify(const VerifyArgs& a, unsigned char* recs, int kcap, int b,
-                                       int rows_per_seq, int lane) {
+// residual draw: normalise(max(0, p - q)) over p's survivors; p itself if that is empty
+__device__ __forceinline__ int srec_residual(const SRec& P, const SRec& Q, double u, int lane) {
+    auto r = [&](int j) {
+        double d = P.w[j] / P.Z - srec_prob(Q, P.id[j]);
+        return d > 0.0 ? d : 0.0;
+    };
+    double R = 0.0;
+    for (int j = lane; j < P.n; j += 32) R += r(j);
+    R = warp_sum_f64(R);
+    if (!(R > 0.0)) return srec_inv_cdf(P, u, lane);
+    int j = warp_inv_cdf_gen(P.n, u * R, lane, r);
+    return j >= 0 ? P.id[j] : -1;
+}
+
+// Per-sequence verify by the whole CTA (NW warps, the first FW of them with two record
+// slices each in `region`): warp w evaluates block positions w, w + FW, ...; warp 0 then
+// takes the longest accepted prefix, writes the outputs and draws the correction token.
+template <int NW>
+__device__ void sequence_verify(const VerifyArgs& a, unsigned char* recs, int kcap, int b, int rows_per_seq,
+                                unsigned char* region, size_t region_bytes) {
+    __shared__ int s_tok[32];
+    __shared__ double s_p[32], s_q[32], s_tv[32];
+    __shared__ int s_acc[32];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int K = a.K;
+    const size_t slice = (size_t)kcap * 12;
+    int FW = (int)(region_bytes / (2 * slice));
+    FW = FW < NW ? FW : NW;
     const int64_t rbase = (int64_t)b * rows_per_seq;
-    const int i = lane;
-    const bool act = i < K;
-    int tok = -1;
-    bool acc = true;
-    double pi = 0.0, qi = 0.0, tv = 0.0;
-    if (act) {
-        RecView P = rec_view(recs, kcap, rbase + i);
-        const float* u = a.u + ((int64_t)b * K + i) * 3;
-        if (i == 0) {
-            tok = a.pos0 ? a.pos0[b] : rec_inv_cdf(P, (double)u[0]);
-            pi = (tok >= 0 && tok < a.V) ? rec_prob(P, tok) : 0.0;
-        } else {
-            RecView Qr = rec_view(recs, kcap, rbase + K + i - 1);
-            tok = a.drafts ? a.drafts[(int64_t)b * K + i] : rec_inv_cdf(Qr, (double)u[0]);
-            bool in = tok >= 0 && tok < a.V;
-            pi = in ? rec_prob(P, tok) : 0.0;
-            qi = in ? rec_prob(Qr, tok) : 0.0;
-            acc = (double)u[1] * qi < pi;
-            if (a.out_tv) tv = rec_tv(P, Qr);
+    double* w0 = reinterpret_cast<double*>(region + (size_t)warp * 2 * slice);
+    int32_t* i0 = reinterpret_cast<int32_t*>(region + (size_t)warp * 2 * slice + (size_t)kcap * 8);
+    double* w1 = reinterpret_cast<double*>(region + (size_t)warp * 2 * slice + slice);
+    int32_t* i1 = reinterpret_cast<int32_t*>(region + (size_t)warp * 2 * slice + slice + (size_t)kcap * 8);
+    if (warp < FW) {
+        for (int i = warp; i < K; i += FW) {
+            const float* u = a.u + ((int64_t)b * K + i) * 3;
+            SRec P = warp_stage_rec(recs, kcap, rbase + i, w0, i0, lane);
+            int tok;
+            double pi = 0.0, qi = 0.0, tv = 0.0;
+            int acc = 1;
+            if (i == 0) {
+                tok = a.pos0 ? a.pos0[b] : srec_inv_cdf(P, (double)u[0], lane);
+                pi = (tok >= 0 && tok < a.V) ? srec_prob(P, tok) : 0.0;
+            } else {
+                SRec Q = warp_stage_rec(recs, kcap, rbase + K + i - 1, w1, i1, lane);
+                tok = a.drafts ? a.drafts[(int64_t)b * K + i] : srec_inv_cdf(Q, (double)u[0], lane);
+                bool in = tok >= 0 && tok < a.V;
+                pi = in ? srec_prob(P, tok) : 0.0;
+                qi = in ? srec_prob(Q, tok) : 0.0;
+                acc = (double)u[1] * qi < pi;
+                if (a.out_tv) tv = srec_tv(P, Q, lane);
+            }
+            if (lane == 0) {
+                s_tok[i] = tok;
+                s_p[i] = pi;
+                s_q[i] = qi;
+                s_tv[i] = tv;
+                s_acc[i] = acc;
+            }
+            __syncwarp();
         }
     }
-    unsigned rej = __ballot_sync(kFullMask, act && !acc);
-    const int n = rej ? (__ffs(rej) - 1) : K;
-    if (act) {
-        int64_t o = (int64_t)b * K + i;
-        a.out_tokens[o] = i < n ? tok : -1;
-        if (a.out_p) a.out_p[o] = (float)pi;
-        if (a.out_q) a.out_q[o] = (float)qi;
-        if (a.out_tv) a.out_tv[o] = (float)tv;
-    }
-    if (lane == 0) {
-        a.out_count[b] = n;
-        if (a.out_next && n == K) a.out_next[b] = -1;
-    }
-    if (n < K && lane == n && a.out_next) {
-        RecView P = rec_view(recs, kcap, rbase + n);
-        RecView Qr = rec_view(recs, kcap, rbase + K + n - 1);
-        a.out_next[b] = rec_residual(P, Qr, (double)a.u[((int64_t)b * K + n) * 3 + 2]);
+    __syncthreads();
+    if (warp == 0) {
+        const int i = lane;
+        const bool act = i < K;
+        unsigned rej = __ballot_sync(kFullMask, act && !s_acc[act ? i : 0]);
+        const int n = rej ? (__ffs(rej) - 1) : K;
+        if (act) {
+            int64_t o = (int64_t)b * K + i;
+            a.out_tokens[o] = i < n ? s_tok[i] : -1;
+            if (a.out_p) a.out_p[o] = (float)s_p[i];
+            if (a.out_q) a.out_q[o] = (float)s_q[i];
+            if (a.out_tv) a.out_tv[o] = (float)s_tv[i];
+        }
+        if (lane == 0) a.out_count[b] = n;
+        if (a.out_next) {
+            int nxt = -1;
+            if (n < K) {
+                SRec P = warp_stage_rec(recs, kcap, rbase + n, w0, i0, lane);
+                SRec Q = warp_stage_rec(recs, kcap, rbase + K + n - 1, w1, i1, lane);
+                nxt = srec_residual(P, Q, (double)a.u[((int64_t)b * K + n) * 3 + 2], lane);
+            }
+            if (lane == 0) a.out_next[b] = nxt;
+        }
     }
 }
 

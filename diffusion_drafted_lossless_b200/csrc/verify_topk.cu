@@ -6,23 +6,18 @@
 // sampler settings from the uno-qwen3-8B model card, "Evaluation protocol" (temperature
 // 1.0, top-k 50, top-p 0.95, block 16).
 //
-// One launch does the whole step. The logit rows (verifier rows 0..K-1 and drafter rows
-// 1..K-1 of every sequence) are cut into S segments; one CTA streams one segment once
-// with 16-byte coalesced loads and keeps the segment's exact top-k:
-//   - a CTA-wide lower bound tau0 = k-th largest of the per-thread maxima of the first
-//     loads (k distinct elements are >= it, so nothing below it can be in the top-k);
-//   - each warp walks its sub-range in token-id order and appends candidates to its own
-//     shared-memory buffer; once the buffer has been cut to its exact top-k, later (higher
-//     id) elements are appended only when strictly above the k-th value, which keeps the
-//     ties-to-lower-id rule exact;
-//   - the warps' lists are merged with a CTA radix select and written to the workspace.
-// The last CTA to finish a row (atomic counter, no waiting) merges the S lists, applies
-// softmax and top-p in fp64 and stores the survivor list sorted by token id. The last row
-// of a sequence to finish runs the per-sequence verify (draft sampling, acceptance,
-// prefix, residual resample) in one warp, one lane per block position.
+// Three launches, none of which waits on another CTA:
+//   1. stream: the logit rows (verifier rows 0..K-1 and drafter rows 1..K-1 of every
+//      sequence) are read once with 16-byte coalesced loads; every warp keeps the exact
+//      top-k of its own run of the row in shared memory and writes it out;
+//   2. finish: one warp per row merges the row's lists, applies softmax and top-p in fp64
+//      and stores the survivors sorted by token id;
+//   3. sequence: one CTA per sequence runs draft sampling, acceptance, the longest
+//      accepted prefix and the residual resample, one warp per block position.
 #include <cuda_bf16.h>
 
 #include <cstdlib>
+#include <cstring>
 
 #include "select.cuh"
 #include "verify_common.cuh"
@@ -31,301 +26,833 @@ namespace uno {
 namespace vtopk {
 
 constexpr int kUnroll = 4;
+constexpr int kStreamWarps = 8;  // warps per CTA of the streaming kernel
+constexpr int kGuessPerWarp = 8; // sample maxima each warp contributes to the guess
 
 template <int KCAP>
-struct Cfg;
-template <>
-struct Cfg<64> { static constexpr int WARPS = 16, MIN_CTAS = 2; };
-template <>
-struct Cfg<256> { static constexpr int WARPS = 8, MIN_CTAS = 2; };
-template <>
-struct Cfg<1024> { static constexpr int WARPS = 4, MIN_CTAS = 2; };
+constexpr int cap_entries() { return KCAP + 576; }
 
+// warps per CTA of the row-finishing kernel and its shared memory per warp
 template <int KCAP>
-constexpr int cap_entries() { return KCAP + 384; }
-
-template <typename T, int KCAP>
-constexpr size_t smem_bytes() {
-    constexpr int W = Cfg<KCAP>::WARPS;
-    return (size_t)W * cap_entries<KCAP>() * 8 + (size_t)W * KCAP * 8 + (size_t)W * 256 * 4 + 256 * 4;
-}
+struct FinishCfg;
+template <>
+struct FinishCfg<64> { static constexpr int WARPS = 4; };
+template <>
+struct FinishCfg<256> { static constexpr int WARPS = 2; };
+template <>
+struct FinishCfg<1024> { static constexpr int WARPS = 1; };
 
 struct Params {
     VerifyArgs a;
-    int S;
-    int rows_per_seq;
-    uint32_t* row_counter;
-    uint32_t* seq_counter;
-    uint64_t* seg_lists;
+    int S;               // segments per row (one streaming CTA each)
+    int rows_per_seq;    // 2K - 1
+    int lists_per_row;   // S * kStreamWarps
+    uint64_t* lists;     // [rows * lists_per_row][kcap]
+    int32_t* counts;     // [rows * lists_per_row]
+    uint32_t* guesses;   // [rows * lists_per_row] ordered key of the guess each list was taken with
     unsigned char* recs;
     int kcap;
 };
 
-struct WarpState {
-    uint64_t* buf;
-    uint32_t* hist;
-    int count;
-    bool have_k;
-    float thr;
-};
+template <typename T>
+struct KeyBits;
+template <>
+struct KeyBits<__nv_bfloat16> { static constexpr int value = 16; };
+template <>
+struct KeyBits<float> { static constexpr int value = 32; };
 
-__device__ __forceinline__ void warp_shrink(WarpState& s, int k, int lane) {
-    uint64_t T = warp_select(s.buf, s.count, k, s.hist, lane);
-    uint64_t mn;
-    s.count = warp_compact(s.buf, s.count, T, lane, &mn);
-    s.have_k = true;
-    s.thr = key_float(candidate_key(mn));
-    __syncwarp();
-}
-
-// Offer one lane-chunk (raw vector v with nvalid elements, token ids id0..) to the warp's
-// candidate buffer. Only lanes whose maximum passes both thresholds unpack the vector.
-template <typename T, int CAP>
-__device__ __forceinline__ void warp_offer(WarpState& s, const uint4& v, int nvalid, uint32_t id0, float tau0,
-                                           int k, int lane) {
-    constexpr int VEC = Elem<T>::VEC;
-    const float vmax = raw_max<T>(v);
-    bool hit = nvalid > 0 && vmax >= tau0 && (!s.have_k || vmax > s.thr);
-    if (!__any_sync(kFullMask, hit)) return;
-    int c = 0;
-    uint32_t mask = 0;
-    if (hit) {
+// Descending bitonic sort of one 32-bit key per lane across the warp.
+__device__ __forceinline__ uint32_t warp_sort32_desc(uint32_t v, int lane) {
 #pragma unroll
-        for (int j = 0; j < VEC; ++j) {
-            float x = raw_get<T>(v, j);
-            bool t = j < nvalid && x >= tau0 && (!s.have_k || x > s.thr);
-            mask |= (uint32_t)t << j;
-            c += t;
+    for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            uint32_t o = __shfl_xor_sync(kFullMask, v, stride);
+            bool keep_max = ((lane & stride) == 0) == ((lane & size) == 0);
+            v = keep_max ? max(v, o) : min(v, o);
         }
     }
-    int incl = warp_inclusive_scan(c, lane);
-    int total = __shfl_sync(kFullMask, incl, 31);
-    int pos = s.count + incl - c;
-#pragma unroll
-    for (int j = 0; j < VEC; ++j)
-        if ((mask >> j) & 1u) s.buf[pos++] = pack_candidate(float_key(raw_get<T>(v, j)), id0 + (uint32_t)j);
-    s.count += total;
-    __syncwarp();
-    if (s.count > CAP - 32 * VEC) warp_shrink(s, k, lane);
+    return v;
 }
 
-template <typename T, int KCAP>
-__global__ void __launch_bounds__(Cfg<KCAP>::WARPS * 32, Cfg<KCAP>::MIN_CTAS)
-rows_kernel(Params p) {
-    constexpr int VEC = Elem<T>::VEC;
-    constexpr int WARPS = Cfg<KCAP>::WARPS;
-    constexpr int NT = WARPS * 32;
-    constexpr int CAP = cap_entries<KCAP>();
-    constexpr int CH = 32 * VEC;  // elements per warp step (one "chunk")
+// Packed lane-chunk tests. hit(): does any element x satisfy x >= lo and x > thr?
+// mask(): which elements do (bit j = element j), for the nvalid first elements.
+template <typename T>
+struct LaneOps;
 
+template <>
+struct LaneOps<__nv_bfloat16> {
+    using Thr = __nv_bfloat162;
+    __device__ static __forceinline__ Thr thr(float f) { return __float2bfloat162_rn(f); }  // f is a bf16 value
+    __device__ static __forceinline__ __nv_bfloat162 w2(uint32_t w) { return *reinterpret_cast<__nv_bfloat162*>(&w); }
+    __device__ static __forceinline__ bool hit(const uint4& v, Thr lo, Thr th) {
+        __nv_bfloat162 m = __hmax2(__hmax2(w2(v.x), w2(v.y)), __hmax2(w2(v.z), w2(v.w)));
+        return (__hge2_mask(m, lo) & __hgt2_mask(m, th)) != 0u;
+    }
+    __device__ static __forceinline__ uint32_t mask(const uint4& v, int nvalid, Thr lo, Thr th) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t m = 0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            uint32_t t = __hge2_mask(w2(w[q]), lo) & __hgt2_mask(w2(w[q]), th);
+            m |= ((t & 1u) << (2 * q)) | (((t >> 16) & 1u) << (2 * q + 1));
+        }
+        return nvalid >= 8 ? m : (m & ((1u << nvalid) - 1u));
+    }
+};
+
+template <>
+struct LaneOps<float> {
+    using Thr = float;
+    __device__ static __forceinline__ Thr thr(float f) { return f; }
+    __device__ static __forceinline__ bool hit(const uint4& v, Thr lo, Thr th) {
+        float m = raw_max<float>(v);
+        return m >= lo && m > th;
+    }
+    __device__ static __forceinline__ uint32_t mask(const uint4& v, int nvalid, Thr lo, Thr th) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t m = 0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            float x = __uint_as_float(w[q]);
+            m |= (uint32_t)(q < nvalid && x >= lo && x > th) << q;
+        }
+        return m;
+    }
+};
+
+// Per-warp candidate state, in shared memory so that the rare out-of-line paths can
+// update it. The buffer is always in ascending token-id order.
+struct WarpSlot {
+    int count;
+    int have_k;
+    float thr;  // the buffer's k-th value once it has been cut to k (-inf before)
+};
+
+template <int KB>
+__device__ __noinline__ void warp_shrink(uint64_t* buf, uint32_t* hist, WarpSlot* ws, uint32_t* bound, int k,
+                                         int lane) {
+    uint32_t tau;
+    int need;
+    warp_select_key<KB>(buf, ws->count, k, hist, lane, tau, need);
+    const int n = warp_compact_key<KB>(buf, ws->count, tau, need, lane);
+    const uint32_t key = key32_of_radix<KB>(tau);
+    __syncwarp();
+    if (lane == 0) {
+        ws->count = n;
+        ws->have_k = 1;
+        ws->thr = key_float(key);
+        atomicMax(bound, key);
+    }
+    __syncwarp();
+}
+
+// Cut an unordered buffer to its exact top-k by the packed (value desc, id asc) order.
+__device__ __noinline__ void warp_shrink_packed(uint64_t* buf, uint32_t* hist, WarpSlot* ws, int k, int lane) {
+    const int n0 = ws->count;
+    const uint64_t T = warp_select(buf, n0, k, hist, lane);
+    uint64_t mn;
+    const int n = warp_compact(buf, n0, T, lane, &mn);
+    __syncwarp();
+    if (lane == 0) {
+        ws->count = n;
+        ws->have_k = 1;
+        ws->thr = key_float(candidate_key(mn));
+    }
+    __syncwarp();
+}
+
+// Lane-local append (no warp collectives): the lane's elements of chunk v that pass
+// x >= lo and x > th go to the warp's unordered buffer through a shared-memory atomic.
+template <typename T>
+__device__ __forceinline__ void lane_append(const uint4& v, int nvalid, uint32_t id0, typename LaneOps<T>::Thr lo,
+                                            typename LaneOps<T>::Thr th, uint64_t* buf, WarpSlot* ws) {
+    uint32_t m = LaneOps<T>::mask(v, nvalid, lo, th);
+    int pos = atomicAdd(&ws->count, __popc(m));
+    while (m) {
+        const int j = __ffs(m) - 1;
+        buf[pos++] = pack_candidate(float_key(raw_get<T>(v, j)), id0 + (uint32_t)j);
+        m &= m - 1u;
+    }
+}
+
+// Append the elements of this lane's chunk that pass the current bounds (every lane of
+// the warp calls it; lanes with nothing to add pass through).
+template <typename T, int CAP>
+__device__ __noinline__ void warp_append(const uint4 v, int nvalid, uint32_t id0, uint64_t* buf, uint32_t* hist,
+                                         WarpSlot* ws, uint32_t* bound, float guess, int k, int lane) {
+    using Ops = LaneOps<T>;
+    constexpr int VEC = Elem<T>::VEC;
+    const float lo = fmaxf(guess, key_float(*reinterpret_cast<volatile uint32_t*>(bound)));
+    const float th = ws->have_k ? ws->thr : -INFINITY;
+    uint32_t m = nvalid > 0 ? Ops::mask(v, nvalid, Ops::thr(lo), Ops::thr(th)) : 0u;
+    const int c = __popc(m);
+    const int incl = warp_inclusive_scan(c, lane);
+    const int total = __shfl_sync(kFullMask, incl, 31);
+    int pos = ws->count + incl - c;
+    while (m) {
+        const int j = __ffs(m) - 1;
+        buf[pos++] = pack_candidate(float_key(raw_get<T>(v, j)), id0 + (uint32_t)j);
+        m &= m - 1u;
+    }
+    __syncwarp();
+    if (lane == 0) ws->count += total;
+    __syncwarp();
+    if (ws->count > CAP - 32 * VEC) warp_shrink<KeyBits<T>::value>(buf, hist, ws, bound, k, lane);
+}
+
+// ---------------------------------------------------------------------------------------
+// Kernel 1: stream the logit rows once. Every warp walks its own contiguous run of chunks
+// in token-id order and keeps the run's exact top-k (ties to the lower id). Warps share
+// only a lower bound on the segment's k-th value (any warp's k-th value is one), used as
+// a non-strict filter; they never wait for one another.
+//   - first bound: the k-th largest of the warp's first 32 * kUnroll lane-chunk maxima
+//     (distinct elements, so at least k elements are >= it);
+//   - once a warp's buffer has been cut to its exact top-k, later (higher id) elements
+//     are appended only when strictly above its k-th value.
+// ---------------------------------------------------------------------------------------
+template <typename T, int KCAP>
+__global__ void __launch_bounds__(kStreamWarps * 32)
+stream_kernel(Params p) {
+    using Ops = LaneOps<T>;
+    constexpr int VEC = Elem<T>::VEC;
+    constexpr int CAP = cap_entries<KCAP>();
+    constexpr int CH = 32 * VEC;  // elements per warp step (one chunk)
     extern __shared__ __align__(16) unsigned char smem_raw[];
     uint64_t* wbuf = reinterpret_cast<uint64_t*>(smem_raw);
-    uint64_t* merged = wbuf + WARPS * CAP;
-    uint32_t* whist = reinterpret_cast<uint32_t*>(merged + WARPS * KCAP);
-    uint32_t* chist = whist + WARPS * 256;
-    __shared__ uint64_t bc[4];
-    __shared__ int s_cnt[WARPS];
-    __shared__ int s_w;
-    __shared__ int s_last;
+    uint32_t* whist = reinterpret_cast<uint32_t*>(wbuf + kStreamWarps * CAP);
+    __shared__ uint32_t s_bound;
+    __shared__ float s_guess;
+    __shared__ WarpSlot s_slot[kStreamWarps];
+    __shared__ uint64_t s_top[kStreamWarps * kGuessPerWarp];
+    __shared__ int s_nsample[kStreamWarps];
 
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const VerifyArgs& a = p.a;
     const int S = p.S, k = a.top_k, V = a.V;
     const int grow = blockIdx.x / S, seg = blockIdx.x % S;
     const int b = grow / p.rows_per_seq, r = grow % p.rows_per_seq;
     const bool isP = r < a.K;
     const int pos = isP ? r : r - a.K + 1;
-    const int64_t row_elem0 = ((int64_t)b * a.K + pos) * V;
-    const T* row = reinterpret_cast<const T*>(isP ? a.P : a.Q) + row_elem0;
+    const T* row = reinterpret_cast<const T*>(isP ? a.P : a.Q) + ((int64_t)b * a.K + pos) * V;
     const bool aligned = ((reinterpret_cast<uintptr_t>(row) & 15u) == 0);
 
     const int nchunks = (V + CH - 1) / CH;
+    const int full_chunks = aligned ? V / CH : 0;  // chunks read with plain 16-byte loads
     const int sc0 = (int)((int64_t)nchunks * seg / S), sc1 = (int)((int64_t)nchunks * (seg + 1) / S);
-    const int c0 = sc0 + (int)((int64_t)(sc1 - sc0) * warp / WARPS);
-    const int c1 = sc0 + (int)((int64_t)(sc1 - sc0) * (warp + 1) / WARPS);
+    const int c0 = sc0 + (int)((int64_t)(sc1 - sc0) * warp / kStreamWarps);
+    const int c1 = sc0 + (int)((int64_t)(sc1 - sc0) * (warp + 1) / kStreamWarps);
 
-    WarpState st{wbuf + warp * CAP, whist + warp * 256, 0, false, 0.f};
+    uint64_t* buf = wbuf + warp * CAP;
+    uint32_t* hist = whist + warp * 256;
+    WarpSlot* ws = &s_slot[warp];
+    if (threadIdx.x == 0) {
+        s_bound = 0x007FFFFFu;  // ordered key of -inf
+        s_guess = -INFINITY;
+    }
+    if (lane == 0) {
+        ws->count = 0;
+        ws->have_k = 0;
+        ws->thr = -INFINITY;
+    }
+    __syncthreads();
+    volatile uint32_t* vbound = &s_bound;
 
-    // ---- prologue: the first kUnroll chunks of each warp; CTA lower bound tau0 ----
     uint4 raw[kUnroll];
     int nv[kUnroll];
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-        int c = c0 + u;
-        int64_t e0 = (int64_t)c * CH + lane * VEC;
-        nv[u] = (c < c1) ? (int)max((int64_t)0, min((int64_t)VEC, (int64_t)V - e0)) : 0;
-        raw[u] = nv[u] > 0 ? load_raw<T>(row, e0, nv[u], aligned) : make_uint4(0, 0, 0, 0);
-    }
-    float tmax = -INFINITY;
-    bool tany = false;
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-        if (nv[u] > 0) {
-            tmax = fmaxf(tmax, raw_max<T>(raw[u]));
-            tany = true;
-        }
-    }
-    float tau0 = -INFINITY;
-    {
-        int have = __syncthreads_count(tany);
-        if (have >= k) {
-            merged[tid] = tany ? pack_candidate(float_key(tmax), (uint32_t)tid) : 0ull;
-            __syncthreads();
-            uint64_t T0 = cta_select<NT>(merged, NT, k, chist, bc);
-            uint32_t key = candidate_key(T0);
-            tau0 = key_float(key < 0x007FFFFFu ? 0x007FFFFFu : key);
-        }
-    }
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u)
-        warp_offer<T, CAP>(st, raw[u], nv[u], (uint32_t)((c0 + u) * CH + lane * VEC), tau0, k, lane);
-
-    // ---- stream the rest of the warp's range ----
-    for (int cb = c0 + kUnroll; cb < c1; cb += kUnroll) {
+    auto load = [&](int cb) {
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            int c = cb + u;
-            int64_t e0 = (int64_t)c * CH + lane * VEC;
-            nv[u] = (c < c1) ? (int)max((int64_t)0, min((int64_t)VEC, (int64_t)V - e0)) : 0;
-            raw[u] = nv[u] > 0 ? load_raw<T>(row, e0, nv[u], aligned) : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u)
-            warp_offer<T, CAP>(st, raw[u], nv[u], (uint32_t)((cb + u) * CH + lane * VEC), tau0, k, lane);
-    }
-    if (st.count > k) warp_shrink(st, k, lane);
-
-    // ---- merge the warps' lists: the segment's exact top-k ----
-    if (lane == 0) s_cnt[warp] = st.count;
-    __syncthreads();
-    int off = 0, total = 0;
-    for (int w = 0; w < WARPS; ++w) {
-        off += (w < warp) ? s_cnt[w] : 0;
-        total += s_cnt[w];
-    }
-    for (int j = lane; j < st.count; j += 32) merged[off + j] = st.buf[j];
-    if (tid == 0) s_w = 0;
-    __syncthreads();
-    uint64_t T1 = 0;
-    if (total > k) T1 = cta_select<NT>(merged, total, k, chist, bc);
-    uint64_t* out = p.seg_lists + ((int64_t)grow * S + seg) * KCAP;
-    for (int j = tid; j < total; j += NT) {
-        uint64_t v = merged[j];
-        if (v >= T1) out[atomicAdd(&s_w, 1)] = v;
-    }
-    __syncthreads();
-    for (int j = s_w + tid; j < KCAP; j += NT) out[j] = 0ull;
-
-    // ---- last CTA of the row: survivors of the warped row ----
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_last = (atomicAdd(&p.row_counter[grow], 1u) == (unsigned)(S - 1));
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-
-    const int n = S * KCAP;
-    const uint64_t* lists = p.seg_lists + (int64_t)grow * S * KCAP;
-    for (int j = tid; j < n; j += NT) merged[j] = __ldcg(lists + j);
-    __syncthreads();
-    uint64_t T2 = cta_select<NT>(merged, n, k, chist, bc);
-    int np = 1;
-    while (np < k) np <<= 1;
-    uint64_t* sb = wbuf;                                       // [np] selected, sorted
-    double* w = reinterpret_cast<double*>(wbuf + KCAP);        // [KCAP] weights
-    uint64_t* ib = wbuf + 2 * KCAP;                            // [np] id-sort keys
-    if (tid == 0) s_w = 0;
-    __syncthreads();
-    for (int j = tid; j < n; j += NT) {
-        uint64_t v = merged[j];
-        if (v >= T2) sb[atomicAdd(&s_w, 1)] = v;
-    }
-    __syncthreads();
-    for (int j = k + tid; j < np; j += NT) sb[j] = 0ull;
-    __syncthreads();
-    cta_sort_desc<NT>(sb, np);
-    const double Td = (double)a.temperature;
-    const double zmax = (double)key_float(candidate_key(sb[0])) / Td;
-    for (int j = tid; j < k; j += NT) w[j] = exp((double)key_float(candidate_key(sb[j])) / Td - zmax);
-    __syncthreads();
-    if (tid == 0) {
-        int c = k;
-        if (a.top_p < 1.0f) {
-            double Ssum = 0.0;
-            for (int j = 0; j < k; ++j) Ssum += w[j];
-            double cum = 0.0, tp = (double)a.top_p;
-            for (int j = 0; j < k; ++j) {
-                cum += w[j] / Ssum;
-                if (cum >= tp) {
-                    c = j + 1;
-                    break;
-                }
+            const int c = cb + u;
+            const int64_t e0 = (int64_t)c * CH + lane * VEC;
+            if (c < full_chunks && c < c1) {
+                nv[u] = VEC;
+                raw[u] = ld_stream_v4(row + e0);
+            } else {
+                nv[u] = (c < c1) ? (int)max((int64_t)0, min((int64_t)VEC, (int64_t)V - e0)) : 0;
+                raw[u] = nv[u] > 0 ? load_raw<T>(row, e0, nv[u], aligned) : make_uint4(0, 0, 0, 0);
             }
         }
-        s_w = c;
-    }
-    __syncthreads();
-    const int nsurv = s_w;
-    int np2 = 1;
-    while (np2 < nsurv) np2 <<= 1;
-    for (int j = tid; j < np2; j += NT)
-        ib[j] = j < nsurv ? ((uint64_t)(0xFFFFFFFFu - candidate_id(sb[j])) << 32) | (uint64_t)j : 0ull;
-    __syncthreads();
-    cta_sort_desc<NT>(ib, np2);
-    RecView rec = rec_view(p.recs, p.kcap, grow);
-    for (int j = tid; j < nsurv; j += NT) {
-        uint64_t e = ib[j];
-        rec.id[j] = (int32_t)(0xFFFFFFFFu - (uint32_t)(e >> 32));
-        rec.w[j] = w[(uint32_t)(e & 0xFFFFFFFFu)];
-    }
-    __syncthreads();
-    if (tid == 0) {
-        double Z = 0.0;
-        for (int j = 0; j < nsurv; ++j) Z += __ldcg(rec.w + j);
-        *rec.Z = Z;
-        *rec.n = nsurv;
-    }
+    };
+    auto offer = [&](int cb) {
+        const typename Ops::Thr lo = Ops::thr(fmaxf(s_guess, key_float(*vbound)));
+        const typename Ops::Thr th = Ops::thr(ws->have_k ? ws->thr : -INFINITY);
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const bool hit = nv[u] > 0 && Ops::hit(raw[u], lo, th);
+            if (__any_sync(kFullMask, hit))
+                warp_append<T, CAP>(raw[u], hit ? nv[u] : 0, (uint32_t)((cb + u) * CH + lane * VEC), buf, hist, ws,
+                                    &s_bound, s_guess, k, lane);
+        }
+    };
 
-    // ---- last row of the sequence: the verify decisions ----
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_last = (atomicAdd(&p.seq_counter[b], 1u) == (unsigned)(p.rows_per_seq - 1));
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    if (warp == 0) sequence_verify(a, p.recs, p.kcap, b, p.rows_per_seq, lane);
+    // ---- prologue (every warp, also those with an empty run) ----
+    load(c0);
+    {
+        // Sample of the segment: the lane-chunk maxima of every warp's first loads
+        // (key 0 = no element). (a) The k-th largest of a warp's maxima is a lower bound on
+        // the k-th value (they are distinct elements): shared in s_bound. (b) A guess tau_g
+        // from the CTA's whole sample, expected to leave about 3.7k candidates in the row;
+        // rows that end with fewer than k candidates are redone exactly by the finish
+        // kernel, so the guess never changes the result.
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u)
+            buf[u * 32 + lane] =
+                ((uint64_t)(nv[u] > 0 ? float_key(raw_max<T>(raw[u])) : 0u) << 32) | (uint32_t)(u * 32 + lane);
+        __syncwarp();
+        warp_sort_desc(buf, 32 * kUnroll, lane);
+        if (k <= 32 * kUnroll) {
+            const uint32_t key = (uint32_t)(buf[k - 1] >> 32);
+            if (lane == 0) atomicMax(&s_bound, key < 0x007FFFFFu ? 0x007FFFFFu : key);
+        }
+        if (lane < kGuessPerWarp) s_top[warp * kGuessPerWarp + lane] = buf[lane] | ((uint64_t)warp << 16);
+        int nvalid = 0;
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) nvalid += nv[u];
+        nvalid = warp_sum(nvalid);
+        if (lane == 0) s_nsample[warp] = nvalid;
+        __syncthreads();
+        if (warp == 0) {
+            int ns = 0;
+            for (int w = 0; w < kStreamWarps; ++w) ns += s_nsample[w];
+            uint64_t* tb = buf;  // warp 0's buffer is still free
+            for (int j = lane; j < kStreamWarps * kGuessPerWarp; j += 32) tb[j] = s_top[j];
+            __syncwarp();
+            warp_sort_desc(tb, kStreamWarps * kGuessPerWarp, lane);
+            // expected number of sample elements among the row's top-k: k * ns / V
+            const int m = (int)(3.0 * k * (double)ns / (double)V) + 2;
+            uint32_t g = 0u;
+            if (m <= kStreamWarps * kGuessPerWarp && ns < V) g = (uint32_t)(tb[m - 1] >> 32);
+            if (lane == 0) s_guess = key_float(g < 0x007FFFFFu ? 0x007FFFFFu : g);
+            __syncwarp();
+        }
+        __syncthreads();
+    }
+    offer(c0);
+
+    // ---- stream the rest of the warp's run ----
+    for (int cb = c0 + kUnroll; cb < c1; cb += kUnroll) {
+        load(cb);
+        offer(cb);
+    }
+    if (ws->count > k) warp_shrink<KeyBits<T>::value>(buf, hist, ws, &s_bound, k, lane);
+
+    const int64_t list = ((int64_t)grow * S + seg) * kStreamWarps + warp;
+    uint64_t* out = p.lists + list * KCAP;
+    const int cnt = ws->count;
+    for (int j = lane; j < cnt; j += 32) out[j] = buf[j];
+    if (lane == 0) {
+        p.counts[list] = cnt;
+        p.guesses[list] = float_key(s_guess);
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// Kernel 2: one warp per row. Merge the row's lists into its exact top-k, softmax in
+// fp64, top-p, and write the survivor record sorted by token id.
+// ---------------------------------------------------------------------------------------
+// ---------------------------------------------------------------------------------------
+// Kernel 1 (rows whose start is 16-byte aligned): persistent, fed by TMA.
+// One CTA per SM; its warps take the grid's work items (row segments) in turn and each
+// warp keeps the exact top-k of its run of every item (its 1/kTmaWarps share of the
+// segment) among the elements >= its own guess g (see below). Each warp owns a ring of
+// kStages shared-memory stages filled by bulk async copies that one lane issues ahead
+// without regard to item boundaries, so the next item's data is already arriving while
+// the current one finishes. An mbarrier per stage counts the arriving bytes. Warps never
+// wait for one another. Every wait is bounded: on timeout the warp records
+// UNO_ERR_TIMEOUT in the device status word, waits (bounded) for its copies still in
+// flight, and stops.
+// The guess g: from the first stage of its run the warp takes the maxima of its 32 lanes
+// and sets g to the m-th largest, m chosen so that g is very unlikely to exceed the row's
+// k-th value. The row's result is exact whenever its k-th value is >= every
+// warp's g (then every element that can be in the top-k was a candidate); the finish
+// kernel checks that and otherwise redoes the row exactly.
+// ---------------------------------------------------------------------------------------
+constexpr int kTmaWarps = 4;       // warps per CTA; several CTAs share an SM
+constexpr int kTmaCtasPerSm = 4;
+constexpr int kStageChunks = 4;    // 512-byte chunks per stage (2 KB)
+constexpr int kStages = 4;
+constexpr int kChunkBytes = 512;
+constexpr int kTmaGuessPerWarp = 16;
+constexpr int kFlushChunks = 2;             // chunks between flushes of the flagged list
+constexpr int kHitCap = 32 * kFlushChunks;  // lane-chunks that can be flagged between flushes
+
+template <int KCAP>
+constexpr int tma_cap() { return KCAP + 320; }  // 32 flagged lane-chunks (<= 256 elements) fit after a cut to k
+
+template <int KCAP>
+constexpr size_t tma_smem_bytes() {
+    return (size_t)kTmaWarps * kStages * kStageChunks * kChunkBytes   // rings
+           + (size_t)kTmaWarps * tma_cap<KCAP>() * 8                  // candidate buffers
+           + (size_t)kTmaWarps * kHitCap * 16                         // flagged chunks (data)
+           + (size_t)kTmaWarps * kHitCap * 4                          // flagged chunks (first id)
+           + (size_t)kTmaWarps * 256 * 4                              // histograms
+           + (size_t)kTmaWarps * kStages * 8;                         // mbarriers
+}
+
+struct RunGeom {
+    int c0, ct, c1, nst;  // chunks [c0, ct) by TMA in nst stages, [ct, c1) by plain loads
+};
+
+template <int CH>
+__device__ __forceinline__ RunGeom run_geom(int item, int warp, int S, int V) {
+    const int seg = item % S;
+    const int nchunks = (V + CH - 1) / CH, full_chunks = V / CH;
+    const int sc0 = (int)((int64_t)nchunks * seg / S), sc1 = (int)((int64_t)nchunks * (seg + 1) / S);
+    RunGeom g;
+    g.c0 = sc0 + (sc1 - sc0) * warp / kTmaWarps;
+    g.c1 = sc0 + (sc1 - sc0) * (warp + 1) / kTmaWarps;
+    g.ct = max(g.c0, min(g.c1, full_chunks));
+    g.nst = (g.ct - g.c0 + kStageChunks - 1) / kStageChunks;
+    return g;
+}
+
+template <typename T>
+__device__ __forceinline__ const T* item_row(const Params& p, int item) {
+    const VerifyArgs& a = p.a;
+    const int grow = item / p.S;
+    const int b = grow / p.rows_per_seq, r = grow % p.rows_per_seq;
+    const bool isP = r < a.K;
+    const int pos = isP ? r : r - a.K + 1;
+    return reinterpret_cast<const T*>(isP ? a.P : a.Q) + ((int64_t)b * a.K + pos) * a.V;
+}
+
+// Unpack the flagged lane-chunks hv[0..nh) (first token ids hid[]) and append their
+// elements that pass x >= lo and x > th to the warp's buffer, 32 chunks at a time; the
+// buffer is cut to its exact top-k whenever another 32 chunks might not fit.
+template <typename T, int CAP>
+__device__ __noinline__ void warp_flush_hits(const uint4* hv, const uint32_t* hid, int nh, int nvalid, float lo_f,
+                                             uint64_t* buf, uint32_t* hist, WarpSlot* ws, int k, int lane) {
+    using Ops = LaneOps<T>;
+    constexpr int VEC = Elem<T>::VEC;
+    for (int h0 = 0; h0 < nh; h0 += 32) {
+        if (ws->count > CAP - 32 * VEC) warp_shrink_packed(buf, hist, ws, k, lane);
+        const typename Ops::Thr lo = Ops::thr(lo_f);
+        const typename Ops::Thr th = Ops::thr(ws->have_k ? ws->thr : -INFINITY);
+        const int h = h0 + lane;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        uint32_t m = 0, id0 = 0;
+        if (h < nh) {
+            v = hv[h];
+            id0 = hid[h];
+            m = Ops::mask(v, nvalid, lo, th);
+        }
+        const int c = __popc(m);
+        const int incl = warp_inclusive_scan(c, lane);
+        const int total = __shfl_sync(kFullMask, incl, 31);
+        int pos = ws->count + incl - c;
+        while (m) {
+            const int j = __ffs(m) - 1;
+            buf[pos++] = pack_candidate(float_key(raw_get<T>(v, j)), id0 + (uint32_t)j);
+            m &= m - 1u;
+        }
+        __syncwarp();
+        if (lane == 0) ws->count += total;
+        __syncwarp();
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// Kernel 1 (rows whose start is 16-byte aligned): persistent, fed by TMA.
+// kTmaCtasPerSm CTAs per SM, each taking the grid's work items (row segments) in turn;
+// each of a CTA's warps keeps the exact top-k of its run of the item (its 1/kTmaWarps
+// share) among the elements >= the item's guess g. Each warp owns a ring of kStages
+// shared-memory stages filled by bulk async copies that one lane issues ahead without
+// regard to item boundaries, so the next item's data is already arriving while the
+// current one finishes; an mbarrier per stage counts the arriving bytes. Testing a
+// lane-chunk against the thresholds is a few packed bf16x2 operations; a lane whose
+// chunk passes only records it, and after each stage the warp unpacks all recorded chunks
+// together into its candidate buffer. The buffer is cut to its exact top-k (packed
+// value/id order) when more might not fit; after the cut, later (higher id) elements of
+// the warp's run are kept only when strictly above the k-th value.
+// The guess g: the CTA sorts the lane maxima of its warps' first stages and takes the
+// m-th largest, m chosen so that g is very unlikely to exceed the row's k-th value. The
+// result is exact whenever the row's k-th value is >= g (every element that can be in the
+// top-k was then a candidate); the finish kernel checks that and otherwise redoes the row.
+// Every wait is bounded: on timeout the warp records UNO_ERR_TIMEOUT in the device status
+// word, waits (bounded) for its copies still in flight, and stops.
+// ---------------------------------------------------------------------------------------
+template <typename T, int KCAP>
+__global__ void __launch_bounds__(kTmaWarps * 32, kTmaCtasPerSm)
+stream_tma_kernel(Params p, int n_items, uint32_t* status) {
+    using Ops = LaneOps<T>;
+    constexpr int VEC = Elem<T>::VEC;
+    constexpr int CAP = tma_cap<KCAP>();
+    constexpr int CH = 32 * VEC;  // elements per chunk (512 bytes)
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    unsigned char* rings = smem_raw;
+    uint4* hvs = reinterpret_cast<uint4*>(rings + (size_t)kTmaWarps * kStages * kStageChunks * kChunkBytes);
+    uint64_t* wbuf = reinterpret_cast<uint64_t*>(hvs + kTmaWarps * kHitCap);
+    uint32_t* hids = reinterpret_cast<uint32_t*>(wbuf + kTmaWarps * CAP);
+    uint32_t* whist = hids + kTmaWarps * kHitCap;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(whist + kTmaWarps * 256);
+    __shared__ WarpSlot s_slot[kTmaWarps];
+    __shared__ int s_nhit[kTmaWarps];
+    __shared__ uint64_t s_top[kTmaWarps * kTmaGuessPerWarp];
+    __shared__ int s_nsample[kTmaWarps];
+    __shared__ float s_guess;
+
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int S = p.S, k = p.a.top_k, V = p.a.V;
+    unsigned char* ring = rings + (size_t)warp * kStages * kStageChunks * kChunkBytes;
+    uint64_t* bar = bars + warp * kStages;
+    uint64_t* buf = wbuf + warp * CAP;
+    uint4* hv = hvs + warp * kHitCap;
+    uint32_t* hid = hids + warp * kHitCap;
+    uint32_t* hist = whist + warp * 256;
+    WarpSlot* ws = &s_slot[warp];
+    int* nhit = &s_nhit[warp];
+
+    if (lane == 0) {
+        for (int j = 0; j < kStages; ++j) mbar_init(&bar[j], 1);
+        fence_mbar_init();
+        *nhit = 0;
+    }
+    __syncwarp();
+
+    // producer state (lane 0): the next stage to issue, as (item, stage within the run)
+    int pi = blockIdx.x, pt = 0;
+    RunGeom pg = pi < n_items ? run_geom<CH>(pi, warp, S, V) : RunGeom{0, 0, 0, 0};
+    int issued = 0;  // stages issued so far (all items), lane 0's count
+    auto issue_next = [&]() {  // lane 0
+        while (pi < n_items && pt >= pg.nst) {  // skip to the next stage that exists
+            pi += gridDim.x;
+            pt = 0;
+            if (pi < n_items) pg = run_geom<CH>(pi, warp, S, V);
+        }
+        if (pi >= n_items) return;
+        const int slot = issued % kStages;
+        const uint32_t bytes = (uint32_t)min(kStageChunks, pg.ct - (pg.c0 + pt * kStageChunks)) * kChunkBytes;
+        const unsigned char* src = reinterpret_cast<const unsigned char*>(item_row<T>(p, pi)) +
+                                   (int64_t)(pg.c0 + pt * kStageChunks) * kChunkBytes;
+        mbar_arrive_expect_tx(&bar[slot], bytes);
+        bulk_g2s(ring + (size_t)slot * kStageChunks * kChunkBytes, src, bytes, &bar[slot]);
+        ++pt;
+        ++issued;
+    };
+    if (lane == 0)
+        for (int j = 0; j < kStages; ++j) issue_next();
+    __syncwarp();
+
+    int consumed = 0;  // stages consumed so far (all items)
+    bool ok = true;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+        const RunGeom g = run_geom<CH>(item, warp, S, V);
+        const T* row = item_row<T>(p, item);
+        if (lane == 0) {
+            ws->count = 0;
+            ws->have_k = 0;
+            ws->thr = -INFINITY;
+        }
+        // ---- the item's guess from every warp's first stage (two CTA barriers per item) ----
+        int slot = consumed % kStages;
+        if (g.nst > 0) ok = ok && __all_sync(kFullMask, mbar_wait(&bar[slot], (uint32_t)((consumed / kStages) & 1)));
+        {
+            const int nc0 = (g.nst > 0 && ok) ? min(kStageChunks, g.ct - g.c0) : 0;
+            const unsigned char* stg = ring + (size_t)slot * kStageChunks * kChunkBytes;
+            float lm = -INFINITY;
+            for (int j = 0; j < nc0; ++j) lm = fmaxf(lm, raw_max<T>(lds128(stg + j * kChunkBytes + lane * 16)));
+            const uint32_t sorted = warp_sort32_desc(nc0 > 0 ? float_key(lm) : 0u, lane);
+            if (lane < kTmaGuessPerWarp)
+                s_top[warp * kTmaGuessPerWarp + lane] = ((uint64_t)sorted << 32) | (uint32_t)(warp * 32 + lane);
+            if (lane == 0) s_nsample[warp] = nc0 * CH;
+            __syncthreads();
+            if (warp == 0) {
+                int ns = 0;
+                for (int w = 0; w < kTmaWarps; ++w) ns += s_nsample[w];
+                uint64_t* tb = buf;  // warp 0's buffer is empty at an item's start
+                for (int j = lane; j < kTmaWarps * kTmaGuessPerWarp; j += 32) tb[j] = s_top[j];
+                __syncwarp();
+                warp_sort_desc(tb, kTmaWarps * kTmaGuessPerWarp, lane);
+                // lambda = expected number of sample elements among the row's top-k; the
+                // m-th largest lane maximum with m = 3 lambda + 8 exceeds the row's k-th
+                // value only with negligible probability on exchangeable data
+                const int m = (int)(3.0 * k * (double)ns / (double)V) + 8;
+                uint32_t gk = 0u;
+                if (m <= kTmaWarps * kTmaGuessPerWarp && ns < V) gk = (uint32_t)(tb[m - 1] >> 32);
+                if (lane == 0) s_guess = key_float(gk < 0x007FFFFFu ? 0x007FFFFFu : gk);
+                __syncwarp();
+            }
+            __syncthreads();
+        }
+        const float guess = s_guess;
+        const typename Ops::Thr lo = Ops::thr(guess);
+
+        for (int t = 0; t < g.nst && ok; ++t) {
+            slot = consumed % kStages;
+            if (t > 0) ok = __all_sync(kFullMask, mbar_wait(&bar[slot], (uint32_t)((consumed / kStages) & 1)));
+            if (!ok) break;
+            const unsigned char* stg = ring + (size_t)slot * kStageChunks * kChunkBytes;
+            const int nc = min(kStageChunks, g.ct - (g.c0 + t * kStageChunks));
+#pragma unroll
+            for (int j0 = 0; j0 < kStageChunks; j0 += kFlushChunks) {
+                const typename Ops::Thr th = Ops::thr(ws->have_k ? ws->thr : -INFINITY);
+#pragma unroll
+                for (int j = j0; j < j0 + kFlushChunks; ++j) {
+                    if (j < nc) {
+                        const uint4 v = lds128(stg + j * kChunkBytes + lane * 16);
+                        if (Ops::hit(v, lo, th)) {
+                            const int h = atomicAdd(nhit, 1);
+                            hv[h] = v;
+                            hid[h] = (uint32_t)((g.c0 + t * kStageChunks + j) * CH + lane * VEC);
+                        }
+                    }
+                }
+                __syncwarp();
+                const int nh = *nhit;
+                if (nh > 0) {
+                    warp_flush_hits<T, CAP>(hv, hid, nh, VEC, guess, buf, hist, ws, k, lane);
+                    if (lane == 0) *nhit = 0;
+                    __syncwarp();
+                }
+            }
+            // every lane's reads of this slot are complete (their values fed the tests above
+            // and the warp has passed __syncwarp): the slot can be refilled
+            ++consumed;
+            if (lane == 0) issue_next();
+            __syncwarp();
+        }
+        if (!ok) break;
+        // the row's last, partial chunk (not a multiple of 16 bytes long) by plain loads
+        for (int c = g.ct; c < g.c1; ++c) {
+            const int64_t e0 = (int64_t)c * CH + lane * VEC;
+            const int nv = (int)max((int64_t)0, min((int64_t)VEC, (int64_t)V - e0));
+            const uint4 v = nv > 0 ? load_raw<T>(row, e0, nv, nv == VEC) : make_uint4(0, 0, 0, 0);
+            const typename Ops::Thr th = Ops::thr(ws->have_k ? ws->thr : -INFINITY);
+            if (ws->count > CAP - 32 * VEC) warp_shrink_packed(buf, hist, ws, k, lane);
+            if (nv > 0 && Ops::hit(v, lo, th)) lane_append<T>(v, nv, (uint32_t)e0, lo, th, buf, ws);
+            __syncwarp();
+        }
+        if (ws->count > k) warp_shrink_packed(buf, hist, ws, k, lane);
+        const int64_t list = (int64_t)item * kTmaWarps + warp;
+        uint64_t* out = p.lists + list * KCAP;
+        const int cnt = ws->count;
+        for (int j = lane; j < cnt; j += 32) out[j] = buf[j];
+        if (lane == 0) {
+            p.counts[list] = cnt;
+            p.guesses[list] = float_key(guess);
+        }
+        __syncwarp();
+    }
+    if (!ok) {
+        // wait (bounded) for the copies still in flight, then stop
+        const int n_issued = __shfl_sync(kFullMask, issued, 0);
+        for (int t = consumed; t < n_issued; ++t) mbar_wait(&bar[t % kStages], (uint32_t)((t / kStages) & 1), 1u << 16);
+        if (lane == 0) record_device_status(status, (uint32_t)UNO_ERR_TIMEOUT);
+    }
+}
+
+// Exact top-k of a whole row by one warp, with no guess (the finish kernel's fallback).
+// Leaves the k largest (ties to the lower id) in buf[0..return) in ascending id order.
+template <typename T, int CAP>
+__device__ __noinline__ int warp_exact_row(const T* row, int V, uint64_t* buf, uint32_t* hist, WarpSlot* ws,
+                                           uint32_t* bound, int k, int lane) {
+    constexpr int VEC = Elem<T>::VEC;
+    constexpr int CH = 32 * VEC;
+    using Ops = LaneOps<T>;
+    const bool aligned = ((reinterpret_cast<uintptr_t>(row) & 15u) == 0);
+    if (lane == 0) {
+        ws->count = 0;
+        ws->have_k = 0;
+        ws->thr = -INFINITY;
+        *bound = 0x007FFFFFu;
+    }
+    __syncwarp();
+    const int nchunks = (V + CH - 1) / CH;
+    for (int c = 0; c < nchunks; ++c) {
+        const int64_t e0 = (int64_t)c * CH + lane * VEC;
+        const int nv = (int)max((int64_t)0, min((int64_t)VEC, (int64_t)V - e0));
+        const uint4 v = nv > 0 ? load_raw<T>(row, e0, nv, aligned) : make_uint4(0, 0, 0, 0);
+        const bool hit = nv > 0 && Ops::hit(v, Ops::thr(-INFINITY), Ops::thr(ws->have_k ? ws->thr : -INFINITY));
+        if (__any_sync(kFullMask, hit))
+            warp_append<T, CAP>(v, hit ? nv : 0, (uint32_t)(c * CH + lane * VEC), buf, hist, ws, bound, -INFINITY, k,
+                                lane);
+    }
+    if (ws->count > k) warp_shrink<KeyBits<T>::value>(buf, hist, ws, bound, k, lane);
+    return ws->count;
+}
+
+// capacity of the finish kernel's exact fallback buffer (it reuses the row's candidate
+// area of lists_per_row * KCAP >= kStreamWarps * KCAP entries)
+template <int KCAP>
+constexpr int fallback_cap() { return KCAP + 320; }
+static_assert(fallback_cap<64>() <= 8 * 64 && fallback_cap<256>() <= 8 * 256 && fallback_cap<1024>() <= 8 * 1024,
+              "fallback buffer must fit the candidate area");
+static_assert(fallback_cap<64>() - 256 >= 64, "fallback buffer must hold k + one chunk");
+
+template <int KCAP>
+constexpr size_t finish_bytes_per_warp(int lists_per_row) {
+    return (size_t)lists_per_row * KCAP * 8 + 2 * KCAP * 8 + 256 * 4 + 32;
+}
+
+template <typename T, int KCAP>
+__global__ void __launch_bounds__(FinishCfg<KCAP>::WARPS * 32)
+finish_kernel(Params p, int n_rows) {
+    constexpr int FW = FinishCfg<KCAP>::WARPS;
+    constexpr int KB = KeyBits<T>::value;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t grow = (int64_t)blockIdx.x * FW + warp;
+    if (grow >= n_rows) return;
+    const VerifyArgs& a = p.a;
+    const int k = a.top_k, L = p.lists_per_row;
+    unsigned char* base = smem_raw + warp * finish_bytes_per_warp<KCAP>(L);
+    uint64_t* cand = reinterpret_cast<uint64_t*>(base);      // [L * KCAP], ascending id
+    uint64_t* sb = cand + (size_t)L * KCAP;                  // [np] (value desc, id asc)
+    double* w = reinterpret_cast<double*>(sb + KCAP);        // [KCAP]
+    uint32_t* hist = reinterpret_cast<uint32_t*>(sb + 2 * KCAP);
+    WarpSlot* ws = reinterpret_cast<WarpSlot*>(hist + 256);
+    uint32_t* bound = reinterpret_cast<uint32_t*>(ws + 1);
+
+    // gather the row's lists in (segment, warp) order: ascending token id overall
+    int n = 0;
+    uint32_t G = 0u;  // the largest guess any list was taken with
+    for (int l = 0; l < L; ++l) {
+        const int64_t list = grow * L + l;
+        const int cnt = __ldcg(p.counts + list);
+        G = max(G, __ldcg(p.guesses + list));
+        const uint64_t* src = p.lists + list * KCAP;
+        for (int j = lane; j < cnt; j += 32) cand[n + j] = __ldcg(src + j);
+        n += cnt;
+    }
+    __syncwarp();
+    if (n > k) {
+        const uint64_t T2 = warp_select(cand, n, k, hist, lane);
+        uint64_t mn;
+        n = warp_compact(cand, n, T2, lane, &mn);
+    }
+    // exact iff the k-th value is >= every guess: then every element that can be in the
+    // top-k was >= its warp's guess and so was a candidate
+    uint32_t kmin = 0xFFFFFFFFu;
+    for (int j = lane; j < n; j += 32) kmin = min(kmin, candidate_key(cand[j]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) kmin = min(kmin, __shfl_xor_sync(kFullMask, kmin, o));
+    if (n < k || kmin < G) {
+        // the streaming guess left fewer than k candidates: redo this row exactly
+        const int b = (int)(grow / p.rows_per_seq), r = (int)(grow % p.rows_per_seq);
+        const bool isP = r < a.K;
+        const int pos = isP ? r : r - a.K + 1;
+        const T* row = reinterpret_cast<const T*>(isP ? a.P : a.Q) + ((int64_t)b * a.K + pos) * a.V;
+        n = warp_exact_row<T, fallback_cap<KCAP>()>(row, a.V, cand, hist, ws, bound, k, lane);
+    }
+    // cand[0..n): the row's top-k (any order). Sort by (value desc, id asc) for top-p.
+    const double Td = (double)a.temperature;
+    int np = 1;
+    while (np < n) np <<= 1;
+    for (int j = lane; j < np; j += 32) sb[j] = j < n ? cand[j] : 0ull;
+    __syncwarp();
+    warp_sort_desc(sb, np, lane);
+    const double zmax = (double)key_float(candidate_key(sb[0])) / Td;
+    double part = 0.0;
+    for (int j = lane; j < n; j += 32) {
+        w[j] = exp((double)key_float(candidate_key(sb[j])) / Td - zmax);
+        part += w[j];
+    }
+    __syncwarp();
+    int c = n;
+    if (a.top_p < 1.0f) {
+        const double Ssum = warp_sum_f64(part), tp = (double)a.top_p;
+        double carry = 0.0;
+        c = -1;
+        for (int b0 = 0; b0 < n && c < 0; b0 += 32) {
+            int j = b0 + lane;
+            double x = j < n ? w[j] / Ssum : 0.0;
+            double incl = warp_scan_f64(x, lane);
+            unsigned hit = __ballot_sync(kFullMask, j < n && carry + incl >= tp);
+            if (hit) c = b0 + __ffs(hit);
+            carry += __shfl_sync(kFullMask, incl, 31);
+        }
+        if (c < 0) c = n;
+    }
+    // survivors sb[0..c) sorted by id (key: ~id << 32 | position), reusing cand
+    int np2 = 1;
+    while (np2 < c) np2 <<= 1;
+    uint64_t* ib = cand;
+    for (int j = lane; j < np2; j += 32)
+        ib[j] = j < c ? ((uint64_t)(0xFFFFFFFFu - candidate_id(sb[j])) << 32) | (uint64_t)j : 0ull;
+    __syncwarp();
+    warp_sort_desc(ib, np2, lane);
+    RecView rec = rec_view(p.recs, p.kcap, grow);
+    double z = 0.0;
+    for (int j = lane; j < c; j += 32) {
+        const uint64_t e = ib[j];
+        const double wj = w[(uint32_t)(e & 0xFFFFFFFFu)];
+        rec.id[j] = (int32_t)(0xFFFFFFFFu - (uint32_t)(e >> 32));
+        rec.w[j] = wj;
+        z += wj;
+    }
+    z = warp_sum_f64(z);
+    if (lane == 0) {
+        *rec.Z = z;
+        *rec.n = c;
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// Kernel 3: one CTA per sequence: draft sampling, acceptance, longest accepted prefix,
+// residual resample.
+// ---------------------------------------------------------------------------------------
+constexpr int kSeqWarps = 8;
+
+__global__ void __launch_bounds__(kSeqWarps * 32)
+sequence_kernel(Params p, size_t region_bytes) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    sequence_verify<kSeqWarps>(p.a, p.recs, p.kcap, blockIdx.x, p.rows_per_seq, smem_raw, region_bytes);
+}
+
+inline int num_sms() {
+    static int n[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return 148;
+    if (n[dev] == 0) {
+        int v = 0;
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+        n[dev] = v > 0 ? v : 148;
+    }
+    return n[dev];
 }
 
 struct Layout {
-    int kcap, S, rows_per_seq;
-    size_t off_row_cnt, off_seq_cnt, off_lists, off_recs, total;
+    int kcap, S, rows_per_seq, lists_per_row;
+    size_t off_lists, off_counts, off_guesses, off_recs, total;
 };
 
-inline int choose_segments(int V, int warps) {
+inline int choose_segments(int V) {
     static int forced = -1;
     if (forced < 0) {
         const char* e = getenv("UNO_VERIFY_SEGMENTS");
         forced = e ? atoi(e) : 0;
     }
-    int S = forced > 0 ? forced : V / 49152;
-    if (S < 1) S = 1;
-    if (S > warps) S = warps;
-    return S;
+    int S = forced > 0 ? forced : 1;
+    int nchunks = (V + 255) / 256;
+    if (S > nchunks) S = nchunks;
+    if (S > 8) S = 8;
+    return S < 1 ? 1 : S;
 }
 
 inline Layout layout(const VerifyArgs& a) {
     Layout L{};
     L.kcap = a.top_k <= 64 ? 64 : (a.top_k <= 256 ? 256 : 1024);
-    int warps = L.kcap == 64 ? Cfg<64>::WARPS : (L.kcap == 256 ? Cfg<256>::WARPS : Cfg<1024>::WARPS);
-    L.S = choose_segments(a.V, warps);
+    L.S = choose_segments(a.V);
     L.rows_per_seq = 2 * a.K - 1;
+    // sized for the streaming kernel with the most warps; the launch sets the actual count
+    L.lists_per_row = L.S * (kTmaWarps > kStreamWarps ? kTmaWarps : kStreamWarps);
     size_t rows = (size_t)a.B * L.rows_per_seq;
-    L.off_row_cnt = 0;
-    L.off_seq_cnt = align_up(rows * 4, 16);
-    L.off_lists = align_up(L.off_seq_cnt + (size_t)a.B * 4, 256);
-    L.off_recs = align_up(L.off_lists + rows * L.S * L.kcap * 8, 256);
+    L.off_lists = 0;
+    L.off_counts = align_up(rows * L.lists_per_row * L.kcap * 8, 256);
+    L.off_guesses = align_up(L.off_counts + rows * L.lists_per_row * 4, 256);
+    L.off_recs = align_up(L.off_guesses + rows * L.lists_per_row * 4, 256);
     L.total = align_up(L.off_recs + rows * rec_bytes(L.kcap), 256);
     return L;
+}
+
+template <typename F>
+uno_status set_smem(F* fn, size_t bytes, bool& done, const char* what) {
+    if (done) return UNO_OK;
+    uno_status s = check_cuda(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes), what);
+    if (s == UNO_OK) done = true;
+    return s;
 }
 
 template <typename T, int KCAP>
@@ -334,25 +861,48 @@ uno_status launch_t(const VerifyArgs& a, const Layout& L, unsigned char* ws, cud
     p.a = a;
     p.S = L.S;
     p.rows_per_seq = L.rows_per_seq;
-    p.row_counter = reinterpret_cast<uint32_t*>(ws + L.off_row_cnt);
-    p.seq_counter = reinterpret_cast<uint32_t*>(ws + L.off_seq_cnt);
-    p.seg_lists = reinterpret_cast<uint64_t*>(ws + L.off_lists);
+    p.lists_per_row = L.lists_per_row;
+    p.lists = reinterpret_cast<uint64_t*>(ws + L.off_lists);
+    p.counts = reinterpret_cast<int32_t*>(ws + L.off_counts);
+    p.guesses = reinterpret_cast<uint32_t*>(ws + L.off_guesses);
     p.recs = ws + L.off_recs;
     p.kcap = KCAP;
-    constexpr size_t smem = smem_bytes<T, KCAP>();
-    static bool attr = false;
-    if (!attr) {
-        uno_status s = check_cuda(cudaFuncSetAttribute(rows_kernel<T, KCAP>,
-                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
-                                  "cudaFuncSetAttribute(verify top-k)");
-        if (s != UNO_OK) return s;
-        attr = true;
+    const int n_rows = a.B * L.rows_per_seq;
+    const bool rows_aligned = ((reinterpret_cast<uintptr_t>(a.P) | reinterpret_cast<uintptr_t>(a.Q)) & 15u) == 0 &&
+                              ((size_t)a.V * sizeof(T)) % 16 == 0;
+    // The register-load streaming kernel is the default; the TMA-fed persistent kernel is
+    // selected with UNO_VERIFY_STREAM=tma (it needs 16-byte aligned rows).
+    const char* sel = getenv("UNO_VERIFY_STREAM");
+    const bool use_tma = sel && strcmp(sel, "tma") == 0 && rows_aligned && tma_smem_bytes<KCAP>() <= 227 * 1024;
+    p.lists_per_row = L.S * (use_tma ? kTmaWarps : kStreamWarps);
+    static bool a1 = false, a2 = false, a3 = false;
+    const size_t smem1 = (size_t)kStreamWarps * cap_entries<KCAP>() * 8 + (size_t)kStreamWarps * 256 * 4;
+    constexpr int FW = FinishCfg<KCAP>::WARPS;
+    const size_t smem2 = FW * finish_bytes_per_warp<KCAP>(p.lists_per_row);
+    const size_t region3 = (size_t)kSeqWarps * 2 * 12 * KCAP;
+    const size_t smem3 = region3 < 200 * 1024 ? region3 : 200 * 1024;
+    if (smem2 > 227 * 1024) return set_error(UNO_ERR_UNSUPPORTED, "verify: too many segments for top_k %d", a.top_k);
+
+    uno_status s;
+    if ((s = set_smem(stream_kernel<T, KCAP>, smem1, a1, "cudaFuncSetAttribute(verify stream)")) != UNO_OK) return s;
+    if ((s = set_smem(finish_kernel<T, KCAP>, 227 * 1024, a2, "cudaFuncSetAttribute(verify finish)")) != UNO_OK) return s;
+    if ((s = set_smem(sequence_kernel, 200 * 1024, a3, "cudaFuncSetAttribute(verify sequence)")) != UNO_OK) return s;
+    if (use_tma) {
+        static bool a0 = false;
+        const size_t smem0 = tma_smem_bytes<KCAP>();
+        if ((s = set_smem(stream_tma_kernel<T, KCAP>, smem0, a0, "cudaFuncSetAttribute(verify stream tma)")) != UNO_OK)
+            return s;
+        const int n_items = n_rows * L.S;
+        const int grid = n_items < num_sms() * kTmaCtasPerSm ? n_items : num_sms() * kTmaCtasPerSm;
+        stream_tma_kernel<T, KCAP><<<(unsigned)grid, kTmaWarps * 32, smem0, stream>>>(p, n_items, device_status_ptr());
+    } else {
+        stream_kernel<T, KCAP><<<(unsigned)(n_rows * L.S), kStreamWarps * 32, smem1, stream>>>(p);
     }
-    uno_status s = check_cuda(cudaMemsetAsync(ws, 0, L.off_lists, stream), "cudaMemsetAsync(verify counters)");
-    if (s != UNO_OK) return s;
-    int64_t grid = (int64_t)a.B * L.rows_per_seq * L.S;
-    rows_kernel<T, KCAP><<<(unsigned)grid, Cfg<KCAP>::WARPS * 32, smem, stream>>>(p);
-    return check_cuda(cudaGetLastError(), "launch(verify top-k)");
+    if ((s = check_cuda(cudaGetLastError(), "launch(verify stream)")) != UNO_OK) return s;
+    finish_kernel<T, KCAP><<<(unsigned)((n_rows + FW - 1) / FW), FW * 32, smem2, stream>>>(p, n_rows);
+    if ((s = check_cuda(cudaGetLastError(), "launch(verify finish)")) != UNO_OK) return s;
+    sequence_kernel<<<(unsigned)a.B, kSeqWarps * 32, smem3, stream>>>(p, smem3);
+    return check_cuda(cudaGetLastError(), "launch(verify sequence)");
 }
 
 }  // namespace vtopk

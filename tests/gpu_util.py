@@ -16,7 +16,8 @@ import torch
 
 from diffusion_drafted_lossless_b200 import _lib
 
-NEAR = 1e-4
+NEAR = 1e-4          # the stated threshold band
+NEAR_FP64 = 1e-9     # band for decisions both sides take in fp64 (they differ only in summation order)
 PROB_TOL = 1e-5
 
 
@@ -61,12 +62,19 @@ def decision_path_margin(ref, b):
     return float(np.min(m)) if m.size else np.inf
 
 
-def compare_verify(gpu, ref, check_tv=True):
-    """Returns (n_sequences, n_near, list of mismatch descriptions outside near-threshold)."""
+def compare_verify(gpu, ref, check_tv=True, near_eps=NEAR):
+    """Compare GPU and oracle verify outputs sequence by sequence.
+
+    A sequence whose decision path has an oracle margin below `near_eps` is excused (not
+    compared) and counted. Returns (n_sequences, n_excused, mismatch descriptions,
+    n_literal_near) where the last counts sequences with a margin below the stated 1e-4.
+    """
     B, K = ref["tokens"].shape
-    bad, near = [], 0
+    bad, near, literal = [], 0, 0
     for b in range(B):
-        if decision_path_margin(ref, b) < NEAR:
+        m = decision_path_margin(ref, b)
+        literal += m < NEAR
+        if m < near_eps:
             near += 1
             continue
         if gpu["count"][b] != ref["count"][b]:
@@ -83,11 +91,11 @@ def compare_verify(gpu, ref, check_tv=True):
         if ep > PROB_TOL or eq > PROB_TOL:
             bad.append(f"seq {b}: p/q error {ep:.3g} {eq:.3g}")
         if check_tv and gpu.get("tv") is not None:
-            rows_ok = np.min(ref["margins"][b, :, 3:5], axis=1) >= NEAR  # top-p cut of both rows decided
+            rows_ok = np.min(ref["margins"][b, :, 3:5], axis=1) >= near_eps  # top-p cuts decided
             et = np.abs(gpu["tv"][b] - ref["tv"][b])[rows_ok]
             if et.size and et.max() > PROB_TOL:
                 bad.append(f"seq {b}: tv error {et.max():.3g}")
-    return B, near, bad
+    return B, near, bad, literal
 
 
 def bf16_ulp(x: np.ndarray) -> np.ndarray:

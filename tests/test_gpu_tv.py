@@ -13,6 +13,12 @@ from tests.gpu_util import PROB_TOL, bf16_ulp, dev
 pytestmark = pytest.mark.gpu
 
 
+def _psum(Tf, Sf):
+    """p + q per element (scale for the sign-decision band)."""
+    from scipy.special import softmax
+    return softmax(Tf, axis=1) + softmax(Sf, axis=1)
+
+
 def _run(T, S, dtype, mask=None, grad_scale=1.0, want_grad=True):
     N, V = T.shape
     td, sd = dev(T, dtype), dev(S, dtype)
@@ -26,13 +32,16 @@ def _run(T, S, dtype, mask=None, grad_scale=1.0, want_grad=True):
     return tv.cpu().numpy(), float(mean.cpu()[0]), gg
 
 
-def _compare_grad(g_gpu, ref_grad, absdiff):
-    flip = absdiff < 1e-7
+def _compare_grad(g_gpu, ref_grad, absdiff, psum):
+    """Within one bf16 ulp of the fp64 gradient. Mismatches are excused only where
+    sign(q - p) is not decided at fp32 resolution (|p - q| <= 1e-6 (p + q)); those are
+    counted and must stay below 0.1% of the elements."""
+    undecided = absdiff <= 1e-6 * psum
     err = np.abs(g_gpu.astype(np.float64) - ref_grad)
     ok = err <= bf16_ulp(ref_grad) + 1e-38
-    bad = ~ok & ~flip
+    bad = ~ok & ~undecided
     assert not bad.any(), (np.argwhere(bad)[:5], err[bad][:5], ref_grad[bad][:5])
-    assert flip.mean() < 1e-3
+    assert (~ok & undecided).mean() < 1e-3
 
 
 @pytest.mark.parametrize("N,V,dtype", [(7, 1000, "bf16"), (5, 4099, "bf16"), (3, 20000, "f32"), (4, 777, "f32"),
@@ -45,11 +54,11 @@ def test_tv_parity(N, V, dtype):
     mask = np.ones(N, bool)
     mask[1::3] = False
     tv, mean, g = _run(T, S, dtype, mask=mask, grad_scale=1.5)
-    ref = oracle.tv_loss(W.to_f64(T, dtype), W.to_f64(S, dtype), mask=mask, grad_scale=np.float32(1.5),
-                         want_absdiff=True)
+    Tf, Sf = W.to_f64(T, dtype), W.to_f64(S, dtype)
+    ref = oracle.tv_loss(Tf, Sf, mask=mask, grad_scale=np.float32(1.5), want_absdiff=True)
     np.testing.assert_allclose(tv, ref["tv"], atol=PROB_TOL, rtol=0)
     assert abs(mean - ref["mean"]) <= PROB_TOL
-    _compare_grad(g, ref["grad"], ref["absdiff"])
+    _compare_grad(g, ref["grad"], ref["absdiff"], _psum(Tf, Sf))
 
 
 def test_tv_identical_and_no_grad():
@@ -78,8 +87,9 @@ def test_tv_full_size_sampled_rows():
     tv, mean, g = _run(T, S, "bf16")
     rows = np.array([0, 1, 777, 4095, 4096, 8191, 9000, 12000, 15000, 16380, 16382, 16383])
     Tr, Sr = W.tv_logits(w, rows)
-    ref = oracle.tv_loss(W.to_f64(Tr, "bf16"), W.to_f64(Sr, "bf16"), want_absdiff=True)
+    Tf, Sf = W.to_f64(Tr, "bf16"), W.to_f64(Sr, "bf16")
+    ref = oracle.tv_loss(Tf, Sf, want_absdiff=True)
     np.testing.assert_allclose(tv[rows], ref["tv"], atol=PROB_TOL, rtol=0)
     # gradient of the sampled rows: the oracle's per-row gradient carries 1/N_mask = 1/N
-    _compare_grad(g[rows], ref["grad"] * len(rows) / w.N, ref["absdiff"])
+    _compare_grad(g[rows], ref["grad"] * len(rows) / w.N, ref["absdiff"], _psum(Tf, Sf))
     assert abs(mean - tv.astype(np.float64).mean()) < 1e-6
