@@ -218,7 +218,7 @@ stream_kernel(Params p) {
     constexpr int VEC = Elem<T>::VEC;
     constexpr int CAP = cap_entries<KCAP>();
     constexpr int CH = 32 * VEC;  // elements per warp step (one chunk)
-    extern __shared__ __align__(16) unsigned char smem_raw[];
+    extern __shared__ __align__(128) unsigned char smem_raw[];
     uint64_t* wbuf = reinterpret_cast<uint64_t*>(smem_raw);
     uint32_t* whist = reinterpret_cast<uint32_t*>(wbuf + kStreamWarps * CAP);
     __shared__ uint32_t s_bound;
@@ -690,7 +690,7 @@ __global__ void __launch_bounds__(FinishCfg<KCAP>::WARPS * 32)
 finish_kernel(Params p, int n_rows) {
     constexpr int FW = FinishCfg<KCAP>::WARPS;
     constexpr int KB = KeyBits<T>::value;
-    extern __shared__ __align__(16) unsigned char smem_raw[];
+    extern __shared__ __align__(128) unsigned char smem_raw[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t grow = (int64_t)blockIdx.x * FW + warp;
     if (grow >= n_rows) return;
@@ -796,7 +796,7 @@ constexpr int kSeqWarps = 8;
 
 __global__ void __launch_bounds__(kSeqWarps * 32)
 sequence_kernel(Params p, size_t region_bytes) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
+    extern __shared__ __align__(128) unsigned char smem_raw[];
     sequence_verify<kSeqWarps>(p.a, p.recs, p.kcap, blockIdx.x, p.rows_per_seq, smem_raw, region_bytes);
 }
 
