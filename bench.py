@@ -1,0 +1,407 @@
+"""Benchmark of the Uno draft-and-verify hot path on B200.
+
+One step = one pass of the whole hot path over one batch of 64 sequences x block 16
+(V = 151936, Qwen3-8B shapes):
+  1. the seven row-gated LoRA projections of one decoder layer (q, k, v, o, gate, up,
+     down) at M = 64 x 16 = 1024 rows, rank 128, position 0 of each block ungated;
+  2. the lossless block verify over the [64, 16, 151936] verifier / drafter logits
+     (bf16, T = 1, top-k 50, top-p 0.95; drafter correlated with the verifier, rho 0.8);
+  3. the TV self-distillation loss and its gradient over the same 1024 logit rows
+     (teacher = verifier logits, student = drafter logits).
+Metric: verified draft rows per second = 64 * 16 / step time, summed over GPUs.
+
+Inputs are seeded synthetic tensors of those shapes (no weights or datasets); every
+tensor is larger than L2 or read once per step, so no L2 flush is needed.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl uno|reference]
+For N > 1 run under torch.distributed.run (one process per GPU); each rank runs its own
+replica (data parallel, weak scaling) and the time is the maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from diffusion_drafted_lossless_b200 import workloads as W  # noqa: E402
+
+METRIC = "verified draft rows/s (B=64, block 16, V=151936); TFLOP/s & GB/s vs B200 peak"
+UNIT = "rows/s"
+WORKLOAD = "uno_step_b64_k16_v151936_qwen3_8b"
+LINEARS = W.QWEN3_8B
+VERIFY = W.SERVING_VERIFY
+LAUNCHES_PER_STEP = 7 * 3 + 3 + 2  # 7 x (down, gate, main) + verify (stream, finish, sequence) + TV (mask, rows)
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------------------
+# workload
+# ---------------------------------------------------------------------------------------
+def gemm_flops(shape, M, rank, n_gated):
+    return 2 * M * shape.d_in * shape.d_out + 2 * M * shape.d_in * rank + 2 * n_gated * rank * shape.d_out
+
+
+def verify_bytes(w):
+    """Bytes the verify must read: verifier rows 0..K-1 and drafter rows 1..K-1."""
+    return w.B * (2 * w.K - 1) * w.V * 2
+
+
+def tv_bytes(n, v):
+    return n * v * (2 + 2 + 2)  # read teacher and student, write the bf16 gradient
+
+
+class Step:
+    """Device-resident inputs and outputs of one step, and the calls that make it."""
+
+    def __init__(self, torch, dev):
+        from diffusion_drafted_lossless_b200 import _lib
+        self.torch, self.lib, self.dev = torch, _lib, dev
+        bf = torch.bfloat16
+
+        def t(a):
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(bf).to(dev)
+
+        w = LINEARS
+        self.lin = []
+        xs = {}
+        for sh in w.shapes:
+            inp = W.linear_inputs(w, sh)
+            if sh.d_in not in xs:
+                xs[sh.d_in] = t(inp["x"])
+            y = torch.empty((w.M, sh.d_out), dtype=bf, device=dev)
+            ws = torch.empty(_lib.uno_gated_lora_linear_workspace_size(w.M, sh.d_in, sh.d_out, w.rank),
+                             dtype=torch.uint8, device=dev)
+            self.lin.append(dict(shape=sh, x=xs[sh.d_in], w0=t(inp["w0"]), a=t(inp["a"]), b=t(inp["b"]),
+                                 g=torch.from_numpy(inp["gate"]).to(dev), y=y, ws=ws))
+        self.n_gated = int((W.row_gate(w.M, w.block) > 0).sum())
+        self.x_host = {k: v.cpu() for k, v in xs.items()}
+        v = VERIFY
+        P, Q = W.verify_logits(v)
+        self.P, self.Q = t(P).view(v.B, v.K, v.V), t(Q).view(v.B, v.K, v.V)
+        self.P_host, self.Q_host = self.P.cpu(), self.Q.cpu()
+        self.u = torch.from_numpy(W.verify_uniforms(v)).to(dev)
+        self.tokens = torch.empty((v.B, v.K), dtype=torch.int32, device=dev)
+        self.count = torch.empty((v.B,), dtype=torch.int32, device=dev)
+        self.next = torch.empty((v.B,), dtype=torch.int32, device=dev)
+        self.vws = torch.empty(_lib.uno_block_verify_workspace_size(v.B, v.K, v.V, v.top_k, v.top_p),
+                               dtype=torch.uint8, device=dev)
+        n = v.B * v.K
+        self.tv = torch.empty((n,), device=dev)
+        self.mean = torch.empty((1,), device=dev)
+        self.grad = torch.empty((n, v.V), dtype=bf, device=dev)
+        self.tws = torch.empty(_lib.uno_tv_loss_workspace_size(n, v.V), dtype=torch.uint8, device=dev)
+
+    def linears(self):
+        for L in self.lin:
+            self.lib.uno_gated_lora_linear(L["x"], L["w0"], L["a"], L["b"], L["g"], LINEARS.scale, L["y"],
+                                           workspace=L["ws"])
+
+    def verify(self):
+        v = VERIFY
+        self.lib.uno_block_verify(self.P, self.Q, v.temperature, v.top_k, v.top_p, self.u, self.tokens,
+                                  self.count, self.next, workspace=self.vws)
+
+    def tv_loss(self):
+        v = VERIFY
+        n = v.B * v.K
+        self.lib.uno_tv_loss(self.P.view(n, v.V), self.Q.view(n, v.V), self.tv, self.mean, self.grad,
+                             workspace=self.tws)
+
+    def run(self):
+        self.linears()
+        self.verify()
+        self.tv_loss()
+
+    # end to end: host inputs in pinned memory, copied in every step; results copied back
+    def setup_host(self):
+        torch = self.torch
+        self.hx = {k: v.pin_memory() for k, v in self.x_host.items()}
+        self.hP, self.hQ = self.P_host.pin_memory(), self.Q_host.pin_memory()
+        self.hu = self.u.cpu().pin_memory()
+        self.out_tokens = torch.empty_like(self.tokens, device="cpu").pin_memory()
+        self.out_count = torch.empty_like(self.count, device="cpu").pin_memory()
+        self.out_next = torch.empty_like(self.next, device="cpu").pin_memory()
+        self.out_mean = torch.empty_like(self.mean, device="cpu").pin_memory()
+        self.h2d = sum(t.numel() * t.element_size() for t in list(self.hx.values()) + [self.hP, self.hQ, self.hu])
+        self.d2h = sum(t.numel() * t.element_size() for t in
+                       (self.out_tokens, self.out_count, self.out_next, self.out_mean))
+
+    def run_e2e(self):
+        for k, h in self.hx.items():
+            next(L["x"] for L in self.lin if L["shape"].d_in == k).copy_(h, non_blocking=True)
+        self.P.copy_(self.hP, non_blocking=True)
+        self.Q.copy_(self.hQ, non_blocking=True)
+        self.u.copy_(self.hu, non_blocking=True)
+        self.run()
+        self.out_tokens.copy_(self.tokens, non_blocking=True)
+        self.out_count.copy_(self.count, non_blocking=True)
+        self.out_next.copy_(self.next, non_blocking=True)
+        self.out_mean.copy_(self.mean, non_blocking=True)
+
+
+# ---------------------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------------------
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.f = None
+
+    def __enter__(self):
+        try:
+            self.f = tempfile.NamedTemporaryFile("w+", delete=False, suffix=".csv")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.f.flush()
+        rows = [r.split(",") for r in open(self.f.name).read().strip().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [c.strip() for c in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------------
+# CPU oracle baseline (bounded sample)
+# ---------------------------------------------------------------------------------------
+def oracle_sample(n_seq=2):
+    """Time the fp64 oracle on a bounded sample of the step: n_seq sequences through the
+    verify, the same n_seq * 16 rows through the seven linears and the TV loss."""
+    import oracle
+    v = VERIFY
+    rows = np.arange(n_seq * v.K)
+    P, Q = W.verify_logits(v, rows)
+    u = W.verify_uniforms(v)[:n_seq]
+    lin = [W.linear_inputs(LINEARS, sh, rows=rows) for sh in LINEARS.shapes]
+    Pf, Qf = W.to_f64(P, "bf16"), W.to_f64(Q, "bf16")
+    t0 = time.perf_counter()
+    for inp in lin:
+        oracle.gated_lora(W.to_f64(inp["x"], "bf16"), W.to_f64(inp["w0"], "bf16"), W.to_f64(inp["a"], "bf16"),
+                          W.to_f64(inp["b"], "bf16"), inp["gate"].astype(np.float64), inp["scale"])
+    oracle.block_verify(Pf.reshape(n_seq, v.K, v.V), Qf.reshape(n_seq, v.K, v.V), u.astype(np.float64),
+                        v.temperature, v.top_k, float(np.float32(v.top_p)))
+    oracle.tv_loss(Pf, Qf, want_grad=True)
+    dt = time.perf_counter() - t0
+    n_rows = n_seq * v.K
+    return {"value": n_rows / dt, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n_seq} of 64 sequences ({n_rows} rows) through all three parts of the step; "
+                      f"{dt:.1f} s of fp64 CPU work"}
+
+
+# ---------------------------------------------------------------------------------------
+def time_phase(torch, fn, reps=5):
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ts = []
+    for _ in range(reps):
+        torch.cuda.synchronize()
+        s.record()
+        fn()
+        e.record()
+        torch.cuda.synchronize()
+        ts.append(s.elapsed_time(e))
+    return float(np.median(ts))
+
+
+def run_uno(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    st = Step(torch, dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x):
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        st.run()
+    barrier()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier()
+        s.record()
+        for _ in range(args.steps):
+            st.run()
+        e.record()
+        barrier()
+    ms = max_over_ranks(s.elapsed_time(e) / args.steps)
+    clocks = clk.summary()
+
+    # per-phase times (same stream, CUDA events, after the timed region)
+    ph = {"gated_lora_linears": time_phase(torch, st.linears), "block_verify": time_phase(torch, st.verify),
+          "tv_loss": time_phase(torch, st.tv_loss)}
+    # end to end through the C ABI with host buffers
+    st.setup_host()
+    for _ in range(2):
+        st.run_e2e()
+    barrier()
+    with_e2e = max(1, min(args.steps, 5))
+    s.record()
+    for _ in range(with_e2e):
+        st.run_e2e()
+    e.record()
+    barrier()
+    e2e_ms = max_over_ranks(s.elapsed_time(e) / with_e2e)
+
+    v, pk = VERIFY, peaks()
+    rows = v.B * v.K
+    value = world * rows / (ms * 1e-3)
+    gemm_fl = sum(gemm_flops(L["shape"], LINEARS.M, LINEARS.rank, st.n_gated) for L in st.lin)
+    dominant = max(ph, key=ph.get)
+    if dominant == "gated_lora_linears":
+        ach = gemm_fl / (ph[dominant] * 1e-3) / 1e12
+        roof = {"kernel": "gated_lora_linears (7 projections)", "bound": "tensor", "achieved": ach,
+                "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops"],
+                "traffic": None, "algorithmic_per_launch": gemm_fl / 7}
+    elif dominant == "block_verify":
+        ach = verify_bytes(v) / (ph[dominant] * 1e-3) / 1e9
+        roof = {"kernel": "block_verify", "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / pk["hbm_gbs"], "traffic": None, "algorithmic_per_launch": verify_bytes(v)}
+    else:
+        ach = tv_bytes(rows, v.V) / (ph[dominant] * 1e-3) / 1e9
+        roof = {"kernel": "tv_loss", "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / pk["hbm_gbs"], "traffic": None, "algorithmic_per_launch": tv_bytes(rows, v.V)}
+    roof["peak_source"] = pk["source"]
+    phases = {
+        "gated_lora_linears": {"ms": ph["gated_lora_linears"],
+                               "tflops": gemm_fl / (ph["gated_lora_linears"] * 1e-3) / 1e12},
+        "block_verify": {"ms": ph["block_verify"],
+                         "gbs": verify_bytes(v) / (ph["block_verify"] * 1e-3) / 1e9,
+                         "rows_per_s": rows / (ph["block_verify"] * 1e-3)},
+        "tv_loss": {"ms": ph["tv_loss"], "gbs": tv_bytes(rows, v.V) / (ph["tv_loss"] * 1e-3) / 1e9},
+    }
+    cpu = oracle_sample() if (rank == 0 and world == 1 and not args.no_cpu) else None
+    mean_count = float(st.count.float().mean().item())
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "B": v.B, "K": v.K, "V": v.V, "global_batch": world * rows,
+                       "seq_len": v.K, "parallelism": f"dp{world}",
+                       "linears": "Qwen3-8B layer: q,k,v,o,gate,up,down at M=1024, rank 128, scale 2",
+                       "verify": "T=1, top-k 50, top-p 0.95, drafts sampled in-kernel",
+                       "tv": "1024 rows x 151936, teacher=verifier, student=drafter logits",
+                       "l2": "no flush: every input (logits 622 MB, weights 380 MB) exceeds L2 or is read once"},
+            "roofline": roof, "phases": phases, "cpu_baseline": cpu,
+            "e2e": {"value": world * rows / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": st.h2d,
+                    "d2h_bytes_per_step": st.d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps, "clocks": clocks,
+            "diagnostics": {"mean_tokens_per_step": mean_count},
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    """The reference arm: the fp64 CPU oracle on the host cores, on bounded samples."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    for _ in range(args.warmup):
+        oracle_sample(n_seq=1)
+    vals = [oracle_sample(n_seq=1)["value"] for _ in range(args.steps)]
+    base = oracle_sample(n_seq=1)
+    value = float(np.median(vals))
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 16 / value * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "B": 64, "K": 16, "V": 151936, "sample": "1 sequence per step"},
+            "cpu_baseline": dict(base, value=value),
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["uno", "reference"], default="uno")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "uno":
+        args.warmup = 3
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+               "--master-addr=127.0.0.1", "--master-port=29511", __file__] + sys.argv[1:]
+        sys.exit(subprocess.call(cmd))
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_uno(args)
+
+
+if __name__ == "__main__":
+    main()

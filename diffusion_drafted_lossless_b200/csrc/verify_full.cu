@@ -1,13 +1,697 @@
-// verify_full.cu — block verify without top-k (full-vocabulary softmax, optional top-p).
+// verify_full.cu — lossless block verify without top-k: softmax over the whole
+// vocabulary, optionally followed by top-p.
+//
+// Same verify rule as the top-k path (LoopUno project page, "How it works" and "Training
+// is self-distillation"; uno-qwen3-8B model card, "Evaluation protocol"); this path serves
+// the unfiltered and the top-p-only sampler settings (the LoopUno runs use temperature 1.0
+// and top-p 0.95 without top-k).
+//
+// One CTA per sequence. For each of its rows (verifier rows 0..K-1, drafter rows
+// 1..K-1) the CTA
+//   1. streams the row once and keeps, per chunk of CH elements, the maximum and the sum
+//      of exp(z - max) (z = logit / T); from them the row's max M and sum S;
+//   2. with top-p: finds the exact cut by radix histograms of the probability mass over
+//      the order-preserving key of the logits (bits 31..24, then 23..16, ...: 2 levels
+//      for bf16 logits, 4 for fp32), restricted at each level to the crossing bin. That
+//      gives the cut value tau, the mass above it and how many of the tokens equal to tau
+//      are kept (the lowest ids: ties are ordered by id);
+//   3. stores per chunk the surviving mass and the number of tokens equal to tau.
+// Draws (inverse CDF over ascending ids) walk the chunk table and then scan one chunk in
+// id order; probabilities of single tokens need the token's rank among the tau-ties, from
+// the table and a scan of its chunk. The correction token's residual max(0, p - q) and the
+// optional TV take one more pass over the two rows involved.
+// Sums are fp32 within a chunk and fp64 across chunks.
+#include <cuda_bf16.h>
+
 #include "verify_common.cuh"
 
 namespace uno {
+namespace vfull {
 
-size_t verify_full_workspace_bytes(const VerifyArgs& a) { (void)a; return 256; }
+constexpr int kWarps = 16;
+constexpr int kThreads = kWarps * 32;
+constexpr int kVecPerLane = 8;  // 16-byte vectors per lane per chunk
+
+struct RowInfo {
+    float M;        // max of z = logit / T
+    int c_tie;      // number of tokens equal to tau that survive (top-p)
+    uint32_t tau;   // key of the cut value (0: no cut, every token survives)
+    int pad;
+    double S;       // sum exp(z - M) over the row
+    double Z;       // surviving mass (sum over survivors of exp(z - M))
+    double w_tau;   // exp(z_tau - M)
+};
+
+struct Params {
+    VerifyArgs a;
+    int rows_per_seq;
+    int nchunks;
+    double* cmass;    // [B * rows_per_seq * nchunks] surviving mass per chunk (rel. to M)
+    int* cties;       // [B * rows_per_seq * nchunks] tokens equal to tau per chunk
+    double* cres;     // [B * nchunks] scratch: residual mass per chunk
+    RowInfo* infos;   // [B * rows_per_seq]
+};
+
+template <typename T>
+struct Chunk {
+    static constexpr int VEC = Elem<T>::VEC;
+    static constexpr int CH = 32 * VEC * kVecPerLane;  // elements per chunk
+};
+
+// element (vector j, lane, slot e) of chunk c in id order: c*CH + j*32*VEC + lane*VEC + e
+template <typename T>
+__device__ __forceinline__ uint4 load_vec(const T* row, int V, int c, int j, int lane, int& nv) {
+    constexpr int VEC = Elem<T>::VEC;
+    const int64_t e0 = (int64_t)c * Chunk<T>::CH + (int64_t)j * 32 * VEC + lane * VEC;
+    nv = (int)max((int64_t)0, min((int64_t)VEC, (int64_t)V - e0));
+    const bool aligned = ((reinterpret_cast<uintptr_t>(row + e0) & 15u) == 0);
+    return nv > 0 ? load_raw<T>(row, e0, nv, aligned && nv == VEC) : make_uint4(0, 0, 0, 0);
+}
+
+__device__ __forceinline__ double cta_sum_f64(double v, double* red) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    v = warp_sum_f64(v);
+    __syncthreads();
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    double t = 0.0;
+    for (int w = 0; w < kWarps; ++w) t += red[w];
+    __syncthreads();
+    return t;
+}
+
+__device__ __forceinline__ float cta_max_f32(float v, float* red) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    v = warp_max(v);
+    __syncthreads();
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    float t = -INFINITY;
+    for (int w = 0; w < kWarps; ++w) t = fmaxf(t, red[w]);
+    __syncthreads();
+    return t;
+}
+
+// ---------------------------------------------------------------------------------------
+// per row: statistics, top-p cut, per-chunk survivor table (whole CTA)
+// ---------------------------------------------------------------------------------------
+template <typename T>
+__device__ void prepare_row(const T* row, const VerifyArgs& a, int nchunks, double* cmass, int* cties, RowInfo* info,
+                            float* hist_f, uint32_t* hist_n, double* dred, float* fred) {
+    constexpr int VEC = Elem<T>::VEC;
+    constexpr int NLEVELS = sizeof(T) == 2 ? 2 : 4;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int V = a.V;
+    const float invT = 1.0f / a.temperature;
+
+    // 1. per chunk max and sum; row max and sum
+    float lmax = -INFINITY;
+    for (int c = warp; c < nchunks; c += kWarps) {
+        float cm = -INFINITY;
+        for (int j = 0; j < kVecPerLane; ++j) {
+            int nv;
+            uint4 v = load_vec<T>(row, V, c, j, lane, nv);
+            for (int e = 0; e < nv; ++e) cm = fmaxf(cm, raw_get<T>(v, e) * invT);
+        }
+        cm = warp_max(cm);
+        float cs = 0.f;
+        for (int j = 0; j < kVecPerLane; ++j) {
+            int nv;
+            uint4 v = load_vec<T>(row, V, c, j, lane, nv);
+            for (int e = 0; e < nv; ++e) cs += __expf(raw_get<T>(v, e) * invT - cm);
+        }
+        cs = warp_sum(cs);
+        if (lane == 0) {
+            cmass[c] = (double)cs;               // relative to the chunk max for now
+            reinterpret_cast<float*>(cties)[c] = cm;  // chunk max parked in the ties slot
+        }
+        lmax = fmaxf(lmax, cm);
+    }
+    const float M = cta_max_f32(lmax, fred);
+    double part = 0.0;
+    for (int c = threadIdx.x; c < nchunks; c += kThreads) {
+        const float cm = reinterpret_cast<float*>(cties)[c];
+        const double m = cmass[c] * exp((double)cm - (double)M);
+        cmass[c] = m;
+        cties[c] = 0;
+        part += m;
+    }
+    const double S = cta_sum_f64(part, dred);
+    RowInfo ri{};
+    ri.M = M;
+    ri.S = S;
+    ri.Z = S;
+    ri.tau = 0u;
+    ri.c_tie = 0;
+    ri.w_tau = 0.0;
+    if (a.top_p < 1.0f) {
+        // 2. exact top-p cut by radix histograms of the mass over the logit keys
+        const double target = (double)a.top_p * S;
+        uint32_t prefix = 0;     // key bits fixed so far
+        double above = 0.0;      // mass of keys above the current prefix bin
+        uint32_t count_at = 0;
+        for (int level = 0; level < NLEVELS; ++level) {
+            const int shift = 24 - 8 * level;
+            const uint32_t hi_mask = level == 0 ? 0u : (~0u << (shift + 8));
+            for (int i = threadIdx.x; i < 256 * kWarps; i += kThreads) {
+                hist_f[i] = 0.f;
+                hist_n[i] = 0u;
+            }
+            __syncthreads();
+            float* hf = hist_f + warp * 256;
+            uint32_t* hn = hist_n + warp * 256;
+            for (int c = warp; c < nchunks; c += kWarps) {
+                for (int j = 0; j < kVecPerLane; ++j) {
+                    int nv;
+                    uint4 v = load_vec<T>(row, V, c, j, lane, nv);
+                    for (int e = 0; e < nv; ++e) {
+                        const float x = raw_get<T>(v, e);
+                        const uint32_t key = float_key(x);
+                        if ((key & hi_mask) == prefix) {
+                            const uint32_t bin = (key >> shift) & 0xFFu;
+                            atomicAdd(&hf[bin], __expf(x * invT - M));
+                            atomicAdd(&hn[bin], 1u);
+                        }
+                    }
+                }
+            }
+            __syncthreads();
+            // combine the warps' histograms; walk bins from the top
+            if (warp == 0) {
+                double cum = above;
+                int chosen = -1;
+                double chosen_above = above;
+                uint32_t chosen_n = 0;
+                for (int b0 = 255; b0 >= 0 && chosen < 0; b0 -= 32) {
+                    const int bin = b0 - lane;
+                    double m = 0.0;
+                    uint32_t n = 0;
+                    for (int w = 0; w < kWarps; ++w) {
+                        m += (double)hist_f[w * 256 + bin];
+                        n += hist_n[w * 256 + bin];
+                    }
+                    const double incl = warp_scan_f64(m, lane);
+                    const unsigned hit = __ballot_sync(kFullMask, cum + incl >= target && n > 0);
+                    if (hit) {
+                        const int src = __ffs(hit) - 1;
+                        chosen = b0 - src;
+                        chosen_above = cum + __shfl_sync(kFullMask, incl - m, src);
+                        chosen_n = __shfl_sync(kFullMask, n, src);
+                    }
+                    cum += __shfl_sync(kFullMask, incl, 31);
+                }
+                if (chosen < 0) {  // rounding: the whole mass falls short of the target; keep everything
+                    chosen = -2;
+                }
+                if (lane == 0) {
+                    dred[0] = chosen_above;
+                    dred[1] = (double)chosen;
+                    dred[2] = (double)chosen_n;
+                }
+            }
+            __syncthreads();
+            const int chosen = (int)dred[1];
+            if (chosen == -2) {
+                prefix = 0;
+                above = 0.0;
+                count_at = 0;
+                break;
+            }
+            above = dred[0];
+            count_at = (uint32_t)dred[2];
+            prefix |= (uint32_t)chosen << shift;
+            __syncthreads();
+        }
+        if (count_at > 0) {
+            // the cut value; for bf16 logits the low 16 key bits follow from the sign
+            uint32_t tau = prefix;
+            if (NLEVELS == 2) tau |= (tau & 0x80000000u) ? 0x0000u : 0xFFFFu;
+            const double w_tau = exp((double)key_float(tau) / (double)a.temperature - (double)M);
+            double need = (target - above) / w_tau;
+            int c_tie = (int)ceil(need - 1e-12);
+            c_tie = c_tie < 1 ? 1 : (c_tie > (int)count_at ? (int)count_at : c_tie);
+            ri.tau = tau;
+            ri.c_tie = c_tie;
+            ri.w_tau = w_tau;
+            ri.Z = above + (double)c_tie * w_tau;
+            // 3. per chunk: mass of keys above tau, and the number of tokens equal to tau
+            for (int c = warp; c < nchunks; c += kWarps) {
+                float mg = 0.f;
+                int nt = 0;
+                for (int j = 0; j < kVecPerLane; ++j) {
+                    int nv;
+                    uint4 v = load_vec<T>(row, V, c, j, lane, nv);
+                    for (int e = 0; e < nv; ++e) {
+                        const float x = raw_get<T>(v, e);
+                        const uint32_t key = float_key(x);
+                        if (key > tau) mg += __expf(x * invT - M);
+                        nt += key == tau;
+                    }
+                }
+                mg = warp_sum(mg);
+                nt = warp_sum(nt);
+                if (lane == 0) {
+                    cmass[c] = (double)mg;
+                    cties[c] = nt;
+                }
+            }
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) *info = ri;
+    __syncthreads();
+}
+
+// ---------------------------------------------------------------------------------------
+// warp-level walks over one row
+// ---------------------------------------------------------------------------------------
+// surviving mass of chunk c given the ties that precede it
+__device__ __forceinline__ double chunk_surv(const RowInfo& ri, const double* cmass, const int* cties, int c,
+                                             int ties_before) {
+    if (ri.tau == 0u) return cmass[c];
+    const int kept = max(0, min(ri.c_tie - ties_before, cties[c]));
+    return cmass[c] + (double)kept * ri.w_tau;
+}
+
+// Scan chunk c of the row in id order; for every element calls f(id, z, survivor weight,
+// lane) — all lanes call f for their elements of each 32-lane vector in turn.
+template <typename T, typename F>
+__device__ __forceinline__ void scan_chunk(const T* row, const VerifyArgs& a, const RowInfo& ri, int c,
+                                           int ties_before, int lane, F f) {
+    constexpr int VEC = Elem<T>::VEC;
+    const float invT = 1.0f / a.temperature;
+    int carry = ties_before;
+    for (int j = 0; j < kVecPerLane; ++j) {
+        int nv;
+        const uint4 v = load_vec<T>(row, a.V, c, j, lane, nv);
+        int nt = 0;
+        for (int e = 0; e < nv; ++e) nt += float_key(raw_get<T>(v, e)) == ri.tau;
+        const int incl = warp_inclusive_scan(nt, lane);
+        int rank = carry + incl - nt;
+        const int64_t id0 = (int64_t)c * Chunk<T>::CH + (int64_t)j * 32 * VEC + lane * VEC;
+        double wv[Elem<T>::VEC];
+        for (int e = 0; e < VEC; ++e) {
+            wv[e] = 0.0;
+            if (e < nv) {
+                const float x = raw_get<T>(v, e);
+                const uint32_t key = float_key(x);
+                bool surv = ri.tau == 0u || key > ri.tau;
+                if (ri.tau != 0u && key == ri.tau) surv = rank++ < ri.c_tie;
+                if (surv) wv[e] = (double)__expf(x * invT - ri.M);
+            }
+        }
+        f(id0, wv, nv, j);
+        carry += __shfl_sync(kFullMask, incl, 31);
+    }
+}
+
+// inverse-CDF draw over the row's survivors with uniform u (one warp)
+template <typename T>
+__device__ int warp_row_draw(const T* row, const VerifyArgs& a, const RowInfo& ri, const double* cmass,
+                             const int* cties, int nchunks, double u, int lane) {
+    const double target = u * ri.Z;
+    double carry = 0.0;
+    int tcarry = 0;
+    int cstar = -1, tstar = 0;
+    double before = 0.0;
+    for (int c0 = 0; c0 < nchunks && cstar < 0; c0 += 32) {
+        const int c = c0 + lane;
+        const int nt = c < nchunks ? cties[c] : 0;
+        const int tincl = warp_inclusive_scan(nt, lane);
+        const double m = c < nchunks ? chunk_surv(ri, cmass, cties, c, tcarry + tincl - nt) : 0.0;
+        const double incl = warp_scan_f64(m, lane);
+        const unsigned hit = __ballot_sync(kFullMask, c < nchunks && m > 0.0 && carry + incl > target);
+        if (hit) {
+            const int src = __ffs(hit) - 1;
+            cstar = c0 + src;
+            tstar = tcarry + __shfl_sync(kFullMask, tincl - nt, src);
+            before = carry + __shfl_sync(kFullMask, incl - m, src);
+        }
+        carry += __shfl_sync(kFullMask, incl, 31);
+        tcarry += __shfl_sync(kFullMask, tincl, 31);
+    }
+    double tgt = target;
+    if (cstar < 0) {  // rounding left no crossing: the answer is the row's last survivor
+        for (int c = nchunks - 1; c >= 0; --c) {
+            int tb = 0;
+            for (int q = 0; q < c; ++q) tb += cties[q];
+            if (chunk_surv(ri, cmass, cties, c, tb) > 0.0) {
+                cstar = c;
+                tstar = tb;
+                break;
+            }
+        }
+        if (cstar < 0) return -1;
+        tgt = INFINITY;  // no element crosses: the scan below reports the chunk's last survivor
+    }
+    const double target2 = tgt;
+    int found = -1, last = -1;
+    double cum = before;
+    scan_chunk<T>(row, a, ri, cstar, tstar, lane, [&](int64_t id0, const double* wv, int nv, int) {
+        double s = 0.0;
+        for (int e = 0; e < nv; ++e) s += wv[e];
+        const double incl = warp_scan_f64(s, lane);
+        if (found < 0) {
+            const unsigned hit = __ballot_sync(kFullMask, s > 0.0 && cum + incl > target2);
+            if (hit) {
+                const int src = __ffs(hit) - 1;
+                int tok = -1;
+                if (lane == src) {
+                    double cc = cum + incl - s;
+                    for (int e = 0; e < nv; ++e) {
+                        if (wv[e] <= 0.0) continue;
+                        cc += wv[e];
+                        tok = (int)(id0 + e);
+                        if (cc > target2) break;
+                    }
+                }
+                found = __shfl_sync(kFullMask, tok, src);
+            }
+            const unsigned pos = __ballot_sync(kFullMask, s > 0.0);
+            if (pos) {
+                const int src = 31 - __clz(pos);
+                int tl = -1;
+                if (lane == src)
+                    for (int e = 0; e < nv; ++e)
+                        if (wv[e] > 0.0) tl = (int)(id0 + e);
+                last = __shfl_sync(kFullMask, tl, src);
+            }
+        }
+        cum += __shfl_sync(kFullMask, incl, 31);
+    });
+    return found >= 0 ? found : last;
+}
+
+// probability of token t under the row's distribution (one warp)
+template <typename T>
+__device__ double warp_row_prob(const T* row, const VerifyArgs& a, const RowInfo& ri, const int* cties, int t,
+                                int lane) {
+    if (t < 0 || t >= a.V) return 0.0;
+    constexpr int CH = Chunk<T>::CH;
+    const int c = t / CH;
+    int tb = 0;
+    if (ri.tau != 0u) {
+        for (int q = lane; q < c; q += 32) tb += cties[q];
+        tb = warp_sum(tb);
+    }
+    double w = 0.0;
+    scan_chunk<T>(row, a, ri, c, tb, lane, [&](int64_t id0, const double* wv, int nv, int) {
+        if (t >= id0 && t < id0 + nv) w = wv[t - id0];
+    });
+    // the owning lane holds w; share it
+    unsigned own = __ballot_sync(kFullMask, w != 0.0);
+    if (own) w = __shfl_sync(kFullMask, w, __ffs(own) - 1);
+    return w / ri.Z;
+}
+
+// ---------------------------------------------------------------------------------------
+// CTA-level passes over a pair of rows: residual mass per chunk, or TV
+// ---------------------------------------------------------------------------------------
+template <typename T, typename F>
+__device__ void pair_pass(const T* prow, const T* qrow, const VerifyArgs& a, const RowInfo& rp, const RowInfo& rq,
+                          const int* ctp, const int* ctq, int nchunks, F per_chunk) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int c = warp; c < nchunks; c += kWarps) {
+        int tbp = 0, tbq = 0;
+        if (rp.tau != 0u || rq.tau != 0u) {
+            for (int q = lane; q < c; q += 32) {
+                tbp += ctp[q];
+                tbq += ctq[q];
+            }
+            tbp = warp_sum(tbp);
+            tbq = warp_sum(tbq);
+        }
+        double wp[kVecPerLane][Elem<T>::VEC];
+        scan_chunk<T>(prow, a, rp, c, tbp, lane, [&](int64_t, const double* wv, int nv, int j) {
+            for (int e = 0; e < Elem<T>::VEC; ++e) wp[j][e] = e < nv ? wv[e] / rp.Z : 0.0;
+        });
+        double acc = 0.0;
+        scan_chunk<T>(qrow, a, rq, c, tbq, lane, [&](int64_t, const double* wv, int nv, int j) {
+            for (int e = 0; e < nv; ++e) acc += per_chunk(wp[j][e], wv[e] / rq.Z);
+        });
+        acc = warp_sum_f64(acc);
+        (void)acc;
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// the kernel: one CTA per sequence
+// ---------------------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(kThreads) seq_kernel(Params p) {
+    __shared__ float hist_f[256 * kWarps];
+    __shared__ uint32_t hist_n[256 * kWarps];
+    __shared__ double dred[kWarps];
+    __shared__ float fred[kWarps];
+    __shared__ int s_tok[32];
+    __shared__ double s_p[32], s_q[32], s_tv[32];
+    __shared__ int s_acc[32];
+    const VerifyArgs& a = p.a;
+    const int b = blockIdx.x, K = a.K, V = a.V, NC = p.nchunks;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int R = p.rows_per_seq;
+    const int64_t rbase = (int64_t)b * R;
+    auto rowp = [&](int r) -> const T* {
+        const bool isP = r < K;
+        const int pos = isP ? r : r - K + 1;
+        return reinterpret_cast<const T*>(isP ? a.P : a.Q) + ((int64_t)b * K + pos) * V;
+    };
+    for (int r = 0; r < R; ++r)
+        prepare_row<T>(rowp(r), a, NC, p.cmass + (rbase + r) * NC, p.cties + (rbase + r) * NC, p.infos + rbase + r,
+                       hist_f, hist_n, dred, fred);
+    __syncthreads();
+
+    // per position: draws, probabilities, acceptance (warp per position)
+    for (int i = warp; i < K; i += kWarps) {
+        const RowInfo rp = p.infos[rbase + i];
+        const double* cmp = p.cmass + (rbase + i) * NC;
+        const int* ctp = p.cties + (rbase + i) * NC;
+        const float* u = a.u + ((int64_t)b * K + i) * 3;
+        int tok;
+        double pi = 0.0, qi = 0.0;
+        int acc = 1;
+        if (i == 0) {
+            tok = a.pos0 ? a.pos0[b] : warp_row_draw<T>(rowp(0), a, rp, cmp, ctp, NC, (double)u[0], lane);
+            pi = warp_row_prob<T>(rowp(0), a, rp, ctp, tok, lane);
+        } else {
+            const int rq_i = K + i - 1;
+            const RowInfo rq = p.infos[rbase + rq_i];
+            const double* cmq = p.cmass + (rbase + rq_i) * NC;
+            const int* ctq = p.cties + (rbase + rq_i) * NC;
+            tok = a.drafts ? a.drafts[(int64_t)b * K + i] : warp_row_draw<T>(rowp(rq_i), a, rq, cmq, ctq, NC, (double)u[0], lane);
+            pi = warp_row_prob<T>(rowp(i), a, rp, ctp, tok, lane);
+            qi = warp_row_prob<T>(rowp(rq_i), a, rq, ctq, tok, lane);
+            acc = (double)u[1] * qi < pi;
+        }
+        if (lane == 0) {
+            s_tok[i] = tok;
+            s_p[i] = pi;
+            s_q[i] = qi;
+            s_acc[i] = acc;
+            s_tv[i] = 0.0;
+        }
+    }
+    __syncthreads();
+    int n = K;
+    for (int i = 1; i < K; ++i)
+        if (!s_acc[i]) {
+            n = i;
+            break;
+        }
+
+    // optional TV per position (i >= 1): 1/2 sum |p - q| over the whole vocabulary
+    if (a.out_tv) {
+        for (int i = 1; i < K; ++i) {
+            const int rq_i = K + i - 1;
+            double part = 0.0;
+            const RowInfo rp = p.infos[rbase + i], rq = p.infos[rbase + rq_i];
+            const int* ctp = p.cties + (rbase + i) * NC;
+            const int* ctq = p.cties + (rbase + rq_i) * NC;
+            pair_pass<T>(rowp(i), rowp(rq_i), a, rp, rq, ctp, ctq, NC, [&](double pv, double qv) {
+                part += fabs(pv - qv);
+                return 0.0;
+            });
+            const double tv = 0.5 * cta_sum_f64(part, dred);
+            if (threadIdx.x == 0) s_tv[i] = tv;
+            __syncthreads();
+        }
+    }
+
+    // the correction token: residual max(0, p_n - q_n) (whole CTA for the per-chunk table)
+    int nxt = -1;
+    if (n < K) {
+        const int rq_n = K + n - 1;
+        const RowInfo rp = p.infos[rbase + n], rq = p.infos[rbase + rq_n];
+        const double* cmp = p.cmass + (rbase + n) * NC;
+        const int* ctp = p.cties + (rbase + n) * NC;
+        const int* ctq = p.cties + (rbase + rq_n) * NC;
+        double* cres = p.cres + (int64_t)b * NC;
+        const T* prow = rowp(n);
+        const T* qrow = rowp(rq_n);
+        // residual mass per chunk (warp per chunk)
+        for (int c = warp; c < NC; c += kWarps) {
+            int tbp = 0, tbq = 0;
+            for (int q = lane; q < c; q += 32) {
+                tbp += ctp[q];
+                tbq += ctq[q];
+            }
+            tbp = warp_sum(tbp);
+            tbq = warp_sum(tbq);
+            double wp[kVecPerLane][Elem<T>::VEC];
+            scan_chunk<T>(prow, a, rp, c, tbp, lane, [&](int64_t, const double* wv, int nv, int j) {
+                for (int e = 0; e < Elem<T>::VEC; ++e) wp[j][e] = e < nv ? wv[e] / rp.Z : 0.0;
+            });
+            double acc = 0.0;
+            scan_chunk<T>(qrow, a, rq, c, tbq, lane, [&](int64_t, const double* wv, int nv, int j) {
+                for (int e = 0; e < nv; ++e) {
+                    const double d = wp[j][e] - wv[e] / rq.Z;
+                    acc += d > 0.0 ? d : 0.0;
+                }
+            });
+            acc = warp_sum_f64(acc);
+            if (lane == 0) cres[c] = acc;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            const double uu = (double)a.u[((int64_t)b * K + n) * 3 + 2];
+            double Rtot = 0.0;
+            for (int c = lane; c < NC; c += 32) Rtot += cres[c];
+            Rtot = warp_sum_f64(Rtot);
+            if (!(Rtot > 0.0)) {
+                nxt = warp_row_draw<T>(prow, a, rp, cmp, ctp, NC, uu, lane);
+            } else {
+                // walk the residual table, then scan the crossing chunk
+                const double target = uu * Rtot;
+                double carry = 0.0, before = 0.0;
+                int cstar = -1;
+                for (int c0 = 0; c0 < NC && cstar < 0; c0 += 32) {
+                    const int c = c0 + lane;
+                    const double m = c < NC ? cres[c] : 0.0;
+                    const double incl = warp_scan_f64(m, lane);
+                    const unsigned hit = __ballot_sync(kFullMask, c < NC && m > 0.0 && carry + incl > target);
+                    if (hit) {
+                        const int src = __ffs(hit) - 1;
+                        cstar = c0 + src;
+                        before = carry + __shfl_sync(kFullMask, incl - m, src);
+                    }
+                    carry += __shfl_sync(kFullMask, incl, 31);
+                }
+                if (cstar < 0)
+                    for (int c = NC - 1; c >= 0 && cstar < 0; --c)
+                        if (cres[c] > 0.0) {
+                            cstar = c;
+                            before = target;
+                        }
+                int tbp = 0, tbq = 0;
+                for (int q = lane; q < cstar; q += 32) {
+                    tbp += ctp[q];
+                    tbq += ctq[q];
+                }
+                tbp = warp_sum(tbp);
+                tbq = warp_sum(tbq);
+                double wp[kVecPerLane][Elem<T>::VEC];
+                scan_chunk<T>(prow, a, rp, cstar, tbp, lane, [&](int64_t, const double* wv, int nv, int j) {
+                    for (int e = 0; e < Elem<T>::VEC; ++e) wp[j][e] = e < nv ? wv[e] / rp.Z : 0.0;
+                });
+                int found = -1, last = -1;
+                double cum = before;
+                scan_chunk<T>(qrow, a, rq, cstar, tbq, lane, [&](int64_t id0, const double* wv, int nv, int j) {
+                    double r[Elem<T>::VEC];
+                    double s = 0.0;
+                    for (int e = 0; e < Elem<T>::VEC; ++e) {
+                        const double d = e < nv ? wp[j][e] - wv[e] / rq.Z : 0.0;
+                        r[e] = d > 0.0 ? d : 0.0;
+                        s += r[e];
+                    }
+                    const double incl = warp_scan_f64(s, lane);
+                    if (found < 0) {
+                        const unsigned hit = __ballot_sync(kFullMask, s > 0.0 && cum + incl > target);
+                        if (hit) {
+                            const int src = __ffs(hit) - 1;
+                            int tk = -1;
+                            if (lane == src) {
+                                double cc = cum + incl - s;
+                                for (int e = 0; e < nv; ++e) {
+                                    if (r[e] <= 0.0) continue;
+                                    cc += r[e];
+                                    tk = (int)(id0 + e);
+                                    if (cc > target) break;
+                                }
+                            }
+                            found = __shfl_sync(kFullMask, tk, src);
+                        }
+                        const unsigned pos = __ballot_sync(kFullMask, s > 0.0);
+                        if (pos) {
+                            const int src = 31 - __clz(pos);
+                            int tl = -1;
+                            if (lane == src)
+                                for (int e = 0; e < nv; ++e)
+                                    if (r[e] > 0.0) tl = (int)(id0 + e);
+                            last = __shfl_sync(kFullMask, tl, src);
+                        }
+                    }
+                    cum += __shfl_sync(kFullMask, incl, 31);
+                });
+                nxt = found >= 0 ? found : last;
+            }
+        }
+    }
+
+    if (warp == 0) {
+        const int i = lane;
+        if (i < K) {
+            const int64_t o = (int64_t)b * K + i;
+            a.out_tokens[o] = i < n ? s_tok[i] : -1;
+            if (a.out_p) a.out_p[o] = (float)s_p[i];
+            if (a.out_q) a.out_q[o] = (float)s_q[i];
+            if (a.out_tv) a.out_tv[o] = (float)s_tv[i];
+        }
+        if (lane == 0) {
+            a.out_count[b] = n;
+            if (a.out_next) a.out_next[b] = n < K ? nxt : -1;
+        }
+    }
+}
+
+struct Layout {
+    int nchunks, rows_per_seq;
+    size_t off_cmass, off_cties, off_cres, off_infos, total;
+};
+
+inline Layout layout(const VerifyArgs& a) {
+    Layout L{};
+    const int CH = a.dtype == UNO_BF16 ? Chunk<__nv_bfloat16>::CH : Chunk<float>::CH;
+    L.nchunks = (a.V + CH - 1) / CH;
+    L.rows_per_seq = 2 * a.K - 1;
+    const size_t rows = (size_t)a.B * L.rows_per_seq;
+    L.off_cmass = 0;
+    L.off_cties = align_up(rows * L.nchunks * 8, 256);
+    L.off_cres = align_up(L.off_cties + rows * L.nchunks * 4, 256);
+    L.off_infos = align_up(L.off_cres + (size_t)a.B * L.nchunks * 8, 256);
+    L.total = align_up(L.off_infos + rows * sizeof(RowInfo), 256);
+    return L;
+}
+
+}  // namespace vfull
+
+size_t verify_full_workspace_bytes(const VerifyArgs& a) { return vfull::layout(a).total; }
 
 uno_status verify_full_launch(const VerifyArgs& a, void* workspace, cudaStream_t stream) {
-    (void)a; (void)workspace; (void)stream;
-    return set_error(UNO_ERR_UNSUPPORTED, "verify without top-k is not built yet");
+    const vfull::Layout L = vfull::layout(a);
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    vfull::Params p{};
+    p.a = a;
+    p.rows_per_seq = L.rows_per_seq;
+    p.nchunks = L.nchunks;
+    p.cmass = reinterpret_cast<double*>(ws + L.off_cmass);
+    p.cties = reinterpret_cast<int*>(ws + L.off_cties);
+    p.cres = reinterpret_cast<double*>(ws + L.off_cres);
+    p.infos = reinterpret_cast<vfull::RowInfo*>(ws + L.off_infos);
+    if (a.dtype == UNO_BF16)
+        vfull::seq_kernel<__nv_bfloat16><<<(unsigned)a.B, vfull::kThreads, 0, stream>>>(p);
+    else
+        vfull::seq_kernel<float><<<(unsigned)a.B, vfull::kThreads, 0, stream>>>(p);
+    return check_cuda(cudaGetLastError(), "launch(verify full)");
 }
 
 }  // namespace uno
