@@ -174,7 +174,7 @@ class ClockSampler:
         try:
             self.f = tempfile.NamedTemporaryFile("w+", delete=False, suffix=".csv")
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.QUERY}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -286,6 +286,7 @@ def run_uno(args):
     barrier()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
+        time.sleep(0.3)  # let the sampler start before the timed region
         barrier()
         s.record()
         for _ in range(args.steps):
@@ -386,7 +387,7 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["uno", "reference"], default="uno")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
