@@ -23,7 +23,7 @@ UNO_BF16, UNO_F32 = 0, 1
 EXPORTED = (
     "uno_status_string", "uno_last_error_string", "uno_version", "uno_read_device_status",
     "uno_gated_lora_linear_workspace_size", "uno_gated_lora_linear",
-    "uno_block_verify_workspace_size", "uno_block_verify",
+    "uno_block_verify_workspace_size", "uno_block_verify", "uno_block_verify_noalloc",
     "uno_tv_loss_workspace_size", "uno_tv_loss",
 )
 
@@ -61,6 +61,9 @@ def load(path: str | os.PathLike | None = None) -> ctypes.CDLL:
     lib.uno_block_verify_workspace_size.argtypes = [_i32, _i32, _i32, _i32, _f32, ctypes.c_int]
     lib.uno_block_verify.argtypes = [_vp, _vp, ctypes.c_int, _i32, _i32, _i32, _f32, _i32, _f32,
                                      _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+    lib.uno_block_verify_noalloc.argtypes = [_vp, _vp, ctypes.c_int, _i32, _i32, _i32, _f32, _i32, _f32,
+                                             _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+    lib.uno_block_verify_noalloc.restype = ctypes.c_int
     lib.uno_tv_loss_workspace_size.restype = _sz
     lib.uno_tv_loss_workspace_size.argtypes = [_i64, _i64, ctypes.c_int]
     lib.uno_tv_loss.argtypes = [_vp, _vp, ctypes.c_int, _i64, _i64, _vp, _f32, _vp, _vp, _vp, _vp, _sz, _vp]
@@ -149,6 +152,19 @@ def uno_block_verify(verifier_logits, drafter_logits, temperature, top_k, top_p,
         _ptr(verifier_logits), _ptr(drafter_logits), code, B, K, V, float(temperature), int(top_k), float(top_p),
         _ptr(draft_tokens), _ptr(pos0_tokens), _ptr(uniforms), _ptr(out_tokens), _ptr(out_count),
         _ptr(out_next_token), _ptr(out_p_tok), _ptr(out_q_tok), _ptr(out_tv), _ptr(ws), nb, _stream(stream)))
+
+
+def uno_block_verify_noalloc(verifier_logits, drafter_logits, temperature, top_k, top_p, uniforms,
+                             out_tokens, out_count, out_next_token=None, out_p_tok=None, out_q_tok=None,
+                             out_tv=None, draft_tokens=None, pos0_tokens=None, stream=None):
+    """uno_block_verify with the library's fixed scratch array instead of a workspace, for
+    callers that cannot allocate device memory (see include/uno.h)."""
+    B, K, V = verifier_logits.shape
+    code = _dtype_code(verifier_logits)
+    _check(load().uno_block_verify_noalloc(
+        _ptr(verifier_logits), _ptr(drafter_logits), code, B, K, V, float(temperature), int(top_k), float(top_p),
+        _ptr(draft_tokens), _ptr(pos0_tokens), _ptr(uniforms), _ptr(out_tokens), _ptr(out_count),
+        _ptr(out_next_token), _ptr(out_p_tok), _ptr(out_q_tok), _ptr(out_tv), _stream(stream)))
 
 
 # ---------------------------------------------------------------------------------------

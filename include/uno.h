@@ -168,6 +168,39 @@ uno_status uno_block_verify(const void* verifier_logits, const void* drafter_log
                             uno_stream_t stream);
 
 /* ======================================================================================
+ * Block verify without a caller-supplied workspace
+ *
+ * The Uno pages have no counterpart to this call: it is a convenience of this library.
+ * It takes the arguments of uno_block_verify except the workspace and gives the same
+ * results. It serves callers that cannot allocate device memory where they call the
+ * verify: a plugin or embedded runtime that receives device pointers and a stream from
+ * its host application but has no allocator of its own, or a latency-bound serving loop
+ * that may not call cudaMalloc (which can synchronise the whole device).
+ *
+ * Its scratch is a fixed array of UNO_NOALLOC_SCRATCH_BYTES compiled into the library; every
+ * device that loads the library holds it until the process exits. The call allocates and
+ * frees nothing. The first call on a device looks up the array's device address (with that
+ * device current); make that first call before any stream capture. All calls on a device
+ * share the array, which keeps the last call's contents (nothing in it needs to start at
+ * zero); calls that can overlap on the GPU race on it, so order them on one stream or
+ * synchronise between them.
+ *
+ * Errors: as uno_block_verify, plus UNO_ERR_UNSUPPORTED when the batch needs more scratch
+ * than the array holds (uno_block_verify_workspace_size(...) > UNO_NOALLOC_SCRATCH_BYTES;
+ * the 64 x 16 x 151936 top-k 50 batch needs about 9.4 MiB).
+ * ====================================================================================== */
+#define UNO_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+uno_status uno_block_verify_noalloc(const void* verifier_logits, const void* drafter_logits,
+                                    uno_dtype dtype, int32_t B, int32_t K, int32_t V,
+                                    float temperature, int32_t top_k, float top_p,
+                                    const int32_t* draft_tokens, const int32_t* pos0_tokens,
+                                    const float* uniforms, int32_t* out_tokens,
+                                    int32_t* out_count, int32_t* out_next_token,
+                                    float* out_p_tok, float* out_q_tok, float* out_tv,
+                                    uno_stream_t stream);
+
+/* ======================================================================================
  * TV self-distillation loss and its gradient
  *
  *   p_t = softmax(teacher_logits[t]), q_t = softmax(student_logits[t])   (T = 1, no filter)
