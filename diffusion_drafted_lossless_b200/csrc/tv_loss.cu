@@ -7,11 +7,34 @@
 //   mean = sum_{masked} TV / N_mask
 //   dmean/dstudent_v = q_v (s_v - sum_w q_w s_w) / N_mask,  s = 1/2 sign(q - p)
 //
-// One CTA per token row. Pass 1 streams both rows from HBM once and keeps per-thread
+// Two kernels compute the same thing.
+//
+// cluster_kernel (bf16 rows whose length is a multiple of 8 elements, the common case):
+// a thread-block cluster of CL CTAs owns one (teacher, student) row pair at a time, each
+// CTA holding a 1/CL slice of both rows in shared memory, so every logit is read from HBM
+// exactly once. The slices arrive by bulk copies (mbarrier completion) issued one row
+// ahead, so the next row streams in while this one is computed. Per row: slice maxima ->
+// cluster max; exp of both rows, keeping exp(student) in shared memory -> cluster sums;
+// p, q, sum |p - q| and sum q s, overwriting the kept exp with sign(q - p) folded into its
+// spare bits -> cluster sums; gradient from the kept values. Cluster-wide reductions read
+// every CTA's per-warp partials through distributed shared memory after a cluster barrier.
+// That is 3 exponentials per element pair and 6 bytes of HBM traffic per element pair.
+//
+// rows_kernel (fp32 rows, unaligned rows, rows too long for the cluster's shared memory):
+// one CTA per token row. Pass 1 streams both rows from HBM once and keeps per-thread
 // online (max, sum); pass 2 re-reads them (L2) for sum |p - q| and c = sum q s; pass 3
-// re-reads them and writes the bf16 gradient. A tiny pre-kernel counts the mask; the last
-// CTA to finish (atomic counter, no waiting) writes the mean.
+// re-reads them and writes the gradient.
+//
+// A tiny pre-kernel counts the mask; the CTA that finishes the last row (atomic counter,
+// no waiting) writes the mean.
 #include <cuda_bf16.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <algorithm>
+#include <map>
+#include <mutex>
+#include <utility>
 
 #include "tv_loss.cuh"
 #include "verify_common.cuh"
@@ -30,6 +53,7 @@ struct Work {
 struct Params {
     TVArgs a;
     Work* work;
+    uint32_t* status;
 };
 
 __global__ void count_mask_kernel(const uint8_t* mask, int64_t N, Work* work) {
@@ -235,6 +259,360 @@ __global__ void __launch_bounds__(kThreads, 1) rows_kernel(Params p) {
 
 __global__ void empty_mean_kernel(float* out_mean) { *out_mean = 0.f; }
 
+// =====================================================================================
+// cluster kernel
+// =====================================================================================
+namespace cl {
+
+constexpr int kWarps = 16;                   // compute warps
+constexpr int kThreads = (kWarps + 1) * 32;  // + one producer warp
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Shared memory: a header of mbarriers and reduction slots, two input buffers of
+// (teacher, student) bf16 row slices, and exp(student) of the current row in fp32.
+//   mbarriers: full[2] (an input buffer has landed), empty[2] (every compute warp is done
+//   with an input buffer), red[3] (every warp of the cluster has sent its partial of
+//   reduction 0 / 1 / 2); then three arrays of per-warp partials, [ncta][kWarps] float2 each.
+constexpr int kReductions = 3;
+__host__ __device__ inline size_t header_bytes(int ncta) {
+    return ((size_t)64 + (size_t)kReductions * ncta * kWarps * 8 + 127) / 128 * 128;
+}
+// Elements of a row slice: a multiple of 8 (16-byte bulk copies and 8-element units).
+inline int64_t slice_elems(int64_t V, int cl) { return ((V + cl - 1) / cl + 7) / 8 * 8; }
+inline size_t smem_bytes(int64_t n, int ncta) { return header_bytes(ncta) + (size_t)n * (2 * 2 * 2 + 4); }
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_size() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_id() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t num_clusters() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    __syncwarp();
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t map_rank(const void* local, uint32_t rank) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+    return remote;
+}
+// 8-byte store into another CTA's shared memory, counted in bytes on that CTA's mbarrier
+__device__ __forceinline__ void st_async_v2(uint32_t dst, uint32_t bar, float a, float b) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(dst),
+                 "f"(a), "f"(b), "r"(bar)
+                 : "memory");
+}
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// bulk copy shared -> global (16-byte aligned addresses, size a multiple of 16), tracked
+// by this thread's bulk groups
+__device__ __forceinline__ void bulk_s2g(void* dst, const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_u32(src)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// every committed group has finished reading its shared-memory source
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// every committed group has completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// packed pairs of fp32 (Blackwell's two-wide fp32 pipe)
+typedef unsigned long long f2;
+__device__ __forceinline__ f2 pk(float lo, float hi) {
+    f2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float lo_of(f2 v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float hi_of(f2 v) { return __uint_as_float((uint32_t)(v >> 32)); }
+__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
+    f2 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ f2 add2(f2 a, f2 b) {
+    f2 d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ f2 sub2(f2 a, f2 b) {
+    f2 d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ f2 mul2(f2 a, f2 b) {
+    f2 d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// the two bf16 values of a 32-bit word, widened (exact)
+__device__ __forceinline__ f2 widen(uint32_t w) { return pk(bf16_lo(w), bf16_hi(w)); }
+
+__global__ void __launch_bounds__(kThreads, 1) cluster_kernel(Params p, int64_t n) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    const TVArgs& a = p.a;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const uint32_t rank = cluster_rank(), ncta = cluster_size();
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = full + 2;
+    uint64_t* red = full + 4;  // [kReductions]
+    float2* slots = reinterpret_cast<float2*>(smem + 64);  // [kReductions][ncta][kWarps]
+    const size_t hdr = header_bytes((int)ncta);
+    uint16_t* inbuf = reinterpret_cast<uint16_t*>(smem + hdr);  // [2][teacher, student][n]
+    float* es = reinterpret_cast<float*>(smem + hdr + (size_t)n * 8);
+    const int half = (int)(n / 2);  // unit u keeps its 8 exps at es[u*4 ..+4) and es[half + u*4 ..+4)
+    const int64_t N = a.N, V = a.V;
+    const int64_t lo = (int64_t)rank * n;
+    const int cnt = (int)max((int64_t)0, min(n, V - lo));  // elements of this CTA's slice
+    const uint32_t bytes = (uint32_t)cnt * 2u;
+    const int units = cnt / 8;
+    const uint32_t red_bytes = ncta * kWarps * 8u;
+    const __nv_bfloat16* T = reinterpret_cast<const __nv_bfloat16*>(a.teacher);
+    const __nv_bfloat16* S = reinterpret_cast<const __nv_bfloat16*>(a.student);
+    __nv_bfloat16* G = reinterpret_cast<__nv_bfloat16*>(a.grad);
+    const uint32_t n_mask = p.work->n_mask;
+    uint32_t* status = p.status;
+    const int64_t first = cluster_id(), step = num_clusters();
+    bool failed = false;
+    auto wait = [&](uint64_t* bar, uint32_t parity) {
+        if (!mbar_wait(bar, parity)) {
+            failed = true;
+            record_device_status(status, UNO_ERR_TIMEOUT);
+        }
+    };
+
+    bool more_rows = false;  // the current row is not this cluster's last
+    // Cluster-wide reduction i of this row's per-warp float2 partials (every lane of the
+    // warp passes the same value): each warp stores it into slot [rank][warp] of every CTA
+    // of the cluster; once all have landed, every warp combines them (max or sum).
+    auto reduce = [&](float2 part, int i, uint32_t parity, bool is_max) -> float2 {
+        float2* slot = slots + (size_t)i * ncta * kWarps;
+        if ((uint32_t)lane < ncta)
+            st_async_v2(map_rank(&slot[rank * kWarps + warp], lane), map_rank(&red[i], lane), part.x, part.y);
+        wait(&red[i], parity);
+        float x = is_max ? -INFINITY : 0.f, y = x;
+        for (uint32_t j = lane; j < ncta * kWarps; j += 32) {
+            const float2 w = slot[j];
+            x = is_max ? fmaxf(x, w.x) : x + w.x;
+            y = is_max ? fmaxf(y, w.y) : y + w.y;
+        }
+        // the next row's phase of this reduction is armed before this CTA sends anything
+        // that lets another CTA reach it
+        if (tid == 0 && more_rows) mbar_arrive_expect_tx(&red[i], red_bytes);
+        return is_max ? make_float2(warp_max(x), warp_max(y)) : make_float2(warp_sum(x), warp_sum(y));
+    };
+
+    if (tid == 0) {
+        mbar_init(&full[0], 1);
+        mbar_init(&full[1], 1);
+        mbar_init(&empty[0], kWarps);
+        mbar_init(&empty[1], kWarps);
+        for (int i = 0; i < kReductions; ++i) mbar_init(&red[i], 1);
+        fence_mbar_init();
+        // armed one row ahead, so that no partial can arrive before its phase is armed
+        if (first < N)
+            for (int i = 0; i < kReductions; ++i) mbar_arrive_expect_tx(&red[i], red_bytes);
+    }
+    // every CTA's mbarriers are initialised and armed before any CTA sends to them
+    cluster_sync();
+
+    if (warp == kWarps) {
+        // ---------------- producer: one row ahead, each buffer refilled once released ----
+        // A released buffer holds the gradient of its row in place of the teacher slice:
+        // stream that out first, then refill the buffer.
+        if (lane == 0 && cnt > 0) {
+            uint32_t k = 0;
+            for (int64_t r = first; r < N; r += step, ++k) {
+                const int b = k & 1;
+                uint16_t* dst = inbuf + (size_t)b * 2 * n;
+                if (k >= 2) {
+                    wait(&empty[b], ((k >> 1) - 1) & 1);
+                    if (G != nullptr) {
+                        bulk_s2g(G + (r - 2 * step) * V + lo, dst, bytes);
+                        bulk_commit();
+                        bulk_wait_read();  // the slice has been read out before it is refilled
+                    }
+                }
+                fence_proxy_async_smem();
+                mbar_arrive_expect_tx(&full[b], 2u * bytes);
+                bulk_g2s(dst, T + r * V + lo, bytes, &full[b]);
+                bulk_g2s(dst + n, S + r * V + lo, bytes, &full[b]);
+            }
+            // the last two rows' gradients
+            for (uint32_t j = (k >= 2 ? k - 2 : 0); j < k; ++j) {
+                const int b = j & 1;
+                wait(&empty[b], (j >> 1) & 1);
+                if (G != nullptr) {
+                    bulk_s2g(G + (first + (int64_t)j * step) * V + lo, inbuf + (size_t)b * 2 * n, bytes);
+                    bulk_commit();
+                }
+            }
+            bulk_wait_all();  // every gradient store has completed
+        }
+        __syncwarp();
+    } else {
+        // ---------------- compute warps ----------------
+        double tv_sum = 0.0;  // this cluster's masked TV (rank 0, thread 0)
+        uint32_t rows_done = 0, it = 0;
+        for (int64_t r = first; r < N; r += step, ++it) {
+            const int b = it & 1;
+            const uint32_t par = it & 1;
+            more_rows = r + step < N;
+            if (cnt > 0) wait(&full[b], (it >> 1) & 1);
+            const uint16_t* tin = inbuf + (size_t)b * 2 * n;
+            const uint16_t* sin = tin + n;
+
+            // ---- row maxima over the cluster ----
+            __nv_bfloat162 mt2 = __floats2bfloat162_rn(-INFINITY, -INFINITY), ms2 = mt2;
+            for (int u = tid; u < units; u += kWarps * 32) {
+                const uint4 wt = lds128(tin + u * 8), ws = lds128(sin + u * 8);
+                const uint32_t at4[4] = {wt.x, wt.y, wt.z, wt.w}, as4[4] = {ws.x, ws.y, ws.z, ws.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    mt2 = __hmax2(mt2, *reinterpret_cast<const __nv_bfloat162*>(&at4[j]));
+                    ms2 = __hmax2(ms2, *reinterpret_cast<const __nv_bfloat162*>(&as4[j]));
+                }
+            }
+            float2 v = make_float2(warp_max(fmaxf(__low2float(mt2), __high2float(mt2))),
+                                   warp_max(fmaxf(__low2float(ms2), __high2float(ms2))));
+            v = reduce(v, 0, par, true);
+            const float Mt = v.x, Ms = v.y;
+            const float lt = Mt * kLog2e, ls = Ms * kLog2e;
+            const f2 L2E = pk(kLog2e, kLog2e), NLT = pk(-lt, -lt), NLS = pk(-ls, -ls);
+
+            // ---- sums of exp(x - max); exp(s - Ms) kept ----
+            f2 zt2 = pk(0.f, 0.f), zs2 = zt2;
+            for (int u = tid; u < units; u += kWarps * 32) {
+                const uint4 wt = lds128(tin + u * 8), ws = lds128(sin + u * 8);
+                const uint32_t at4[4] = {wt.x, wt.y, wt.z, wt.w}, as4[4] = {ws.x, ws.y, ws.z, ws.w};
+                float e[8];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const f2 xt = fma2(widen(at4[j]), L2E, NLT), xs = fma2(widen(as4[j]), L2E, NLS);
+                    zt2 = add2(zt2, pk(ex2(lo_of(xt)), ex2(hi_of(xt))));
+                    e[2 * j] = ex2(lo_of(xs));
+                    e[2 * j + 1] = ex2(hi_of(xs));
+                    zs2 = add2(zs2, pk(e[2 * j], e[2 * j + 1]));
+                }
+                *reinterpret_cast<float4*>(es + u * 4) = make_float4(e[0], e[1], e[2], e[3]);
+                *reinterpret_cast<float4*>(es + half + u * 4) = make_float4(e[4], e[5], e[6], e[7]);
+            }
+            v = reduce(make_float2(warp_sum(lo_of(zt2) + hi_of(zt2)), warp_sum(lo_of(zs2) + hi_of(zs2))), 1, par,
+                       false);
+            const float Zt = v.x, Zs = v.y;
+            // p = exp(t - Mt) / Zt, q = kept exp(s - Ms) / Zs. q > p is decided in the log
+            // domain, exact up to the rounding of one threshold:
+            //   q > p  <=>  s - t > K = (Ms + ln Zs) - (Mt + ln Zt)
+            // (Ms - Mt is exact; Zs / Zt is near 1 in practice, so its log is accurate to ~1e-7)
+            const float at = 1.f / Zt, as = 1.f / Zs;
+            const float K = (Ms - Mt) + logf(Zs / Zt);
+
+            // ---- A = sum of q over q > p, P = sum of p over q > p ----
+            // TV = A - P and sum_v q_v sign(q_v - p_v) / 2 = A - 1/2 (both rows sum to 1)
+            float Araw = 0.f, Praw = 0.f;
+            for (int u = tid; u < units; u += kWarps * 32) {
+                const uint4 wt = lds128(tin + u * 8), ws = lds128(sin + u * 8);
+                const float4 k0 = *reinterpret_cast<const float4*>(es + u * 4);
+                const float4 k1 = *reinterpret_cast<const float4*>(es + half + u * 4);
+                const uint32_t at4[4] = {wt.x, wt.y, wt.z, wt.w}, as4[4] = {ws.x, ws.y, ws.z, ws.w};
+                const float qe[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const f2 t2 = widen(at4[j]);
+                    const f2 dl = sub2(widen(as4[j]), t2);
+                    const f2 xt = fma2(t2, L2E, NLT);
+                    if (lo_of(dl) > K) {
+                        Araw += qe[2 * j];
+                        Praw += ex2(lo_of(xt));
+                    }
+                    if (hi_of(dl) > K) {
+                        Araw += qe[2 * j + 1];
+                        Praw += ex2(hi_of(xt));
+                    }
+                }
+            }
+            v = reduce(make_float2(warp_sum(Araw * as), warp_sum(Praw * at)), 2, par, false);
+            const float Af = v.x, Pf = v.y;
+            const bool on = a.mask == nullptr || a.mask[r] != 0;
+
+            // ---- gradient: f q (s - c) = f q (1 - A) where q > p, -f q A elsewhere ----
+            // written as bf16 in place of the teacher slice (each unit by the thread that read
+            // it); the producer warp streams the slice out once every warp is done
+            if (G != nullptr) {
+                const bool grad_on = on && n_mask > 0;
+                const float f = grad_on ? a.grad_scale / (float)n_mask : 0.f;
+                const float kp = f * (1.f - Af) * as, kn = -f * Af * as;
+                uint16_t* gout = const_cast<uint16_t*>(tin);
+                for (int u = tid; u < units; u += kWarps * 32) {
+                    uint4 o = make_uint4(0u, 0u, 0u, 0u);
+                    if (grad_on) {
+                        const uint4 wt = lds128(tin + u * 8), ws = lds128(sin + u * 8);
+                        const float4 k0 = *reinterpret_cast<const float4*>(es + u * 4);
+                        const float4 k1 = *reinterpret_cast<const float4*>(es + half + u * 4);
+                        const uint32_t at4[4] = {wt.x, wt.y, wt.z, wt.w}, as4[4] = {ws.x, ws.y, ws.z, ws.w};
+                        const f2 qe[4] = {pk(k0.x, k0.y), pk(k0.z, k0.w), pk(k1.x, k1.y), pk(k1.z, k1.w)};
+                        uint32_t ow[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const f2 dl = sub2(widen(as4[j]), widen(at4[j]));
+                            const f2 fac = pk(lo_of(dl) > K ? kp : kn, hi_of(dl) > K ? kp : kn);
+                            const f2 g = mul2(qe[j], fac);
+                            __nv_bfloat162 hv = __floats2bfloat162_rn(lo_of(g), hi_of(g));
+                            ow[j] = *reinterpret_cast<uint32_t*>(&hv);
+                        }
+                        o = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                    }
+                    *reinterpret_cast<uint4*>(gout + u * 8) = o;
+                }
+                fence_proxy_async_smem();  // the bulk store reads these through the async proxy
+            }
+            // this warp is done with the input buffer
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[b]);
+            if (rank == 0 && tid == 0) {
+                const double tv = (double)Af - (double)Pf;
+                a.out_tv[r] = (float)tv;
+                if (on) tv_sum += tv;
+                ++rows_done;
+            }
+        }
+        // this cluster's share of the masked mean; the cluster that completes the last row
+        // writes it
+        if (rank == 0 && tid == 0 && rows_done > 0) {
+            atomicAdd(&p.work->sum_tv, tv_sum);
+            __threadfence();
+            const uint32_t prev = atomicAdd(&p.work->done, rows_done);
+            if (prev + rows_done == (uint32_t)N) {
+                __threadfence();
+                const double s = atomicAdd(&p.work->sum_tv, 0.0);
+                *a.out_mean = n_mask > 0 ? (float)(s / (double)n_mask) : 0.f;
+            }
+        }
+    }
+    // no CTA leaves while a store into its shared memory may be in flight
+    cluster_sync();
+}
+
+}  // namespace cl
+
 }  // namespace tvk
 
 size_t tv_loss_workspace_bytes(int64_t N, int64_t V, uno_dtype dtype) {
@@ -244,15 +622,102 @@ size_t tv_loss_workspace_bytes(int64_t N, int64_t V, uno_dtype dtype) {
     return 256;
 }
 
+namespace {
+
+struct DeviceInfo {
+    bool ready = false;
+    int smem_optin = 0;
+    std::map<std::pair<int, size_t>, int> max_clusters;  // (cluster size, smem) -> co-resident clusters
+};
+std::mutex g_mu;
+DeviceInfo g_dev[64];
+
+// Cluster size for rows of V bf16 elements: UNO_TV_CLUSTER if set (1, 2, 4, 8 or 16) and
+// its slices fit, else the smallest whose slices fit in one CTA's shared memory; 0 when none
+// fits.
+int choose_cluster(int64_t V, int smem_optin) {
+    auto need = [&](int c) { return tvk::cl::smem_bytes(tvk::cl::slice_elems(V, c), c); };
+    if (const char* e = getenv("UNO_TV_CLUSTER")) {
+        const int c = atoi(e);
+        if ((c == 1 || c == 2 || c == 4 || c == 8 || c == 16) && need(c) <= (size_t)smem_optin) return c;
+    }
+    for (int c = 1; c <= 16; c *= 2)
+        if (need(c) <= (size_t)smem_optin) return c;
+    return 0;
+}
+
+// Launch the cluster kernel; returns false (nothing launched) when it cannot run here.
+bool launch_cluster(const tvk::Params& p, cudaStream_t stream, uno_status& st) {
+    const TVArgs& a = p.a;
+    if (a.dtype != UNO_BF16 || a.V % 8 != 0) return false;
+    const uintptr_t al = reinterpret_cast<uintptr_t>(a.teacher) | reinterpret_cast<uintptr_t>(a.student) |
+                         reinterpret_cast<uintptr_t>(a.grad);
+    if (al & 15u) return false;
+    if (const char* e = getenv("UNO_TV_KERNEL"))
+        if (strcmp(e, "rows") == 0) return false;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceInfo& di = g_dev[dev];
+    if (!di.ready) {
+        if (cudaDeviceGetAttribute(&di.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+            return false;
+        if (cudaFuncSetAttribute(tvk::cl::cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 di.smem_optin) != cudaSuccess ||
+            cudaFuncSetAttribute(tvk::cl::cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+                cudaSuccess) {
+            cudaGetLastError();
+            return false;
+        }
+        di.ready = true;
+    }
+    const int c = choose_cluster(a.V, di.smem_optin);
+    if (c == 0) return false;
+    const int64_t n = tvk::cl::slice_elems(a.V, c);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)c;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(tvk::cl::kThreads);
+    cfg.dynamicSmemBytes = tvk::cl::smem_bytes(n, c);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    auto key = std::make_pair(c, cfg.dynamicSmemBytes);
+    auto found = di.max_clusters.find(key);
+    int maxc = 0;
+    if (found != di.max_clusters.end()) {
+        maxc = found->second;
+    } else {
+        cudaLaunchConfig_t q = cfg;
+        q.gridDim = dim3((unsigned)c);
+        if (cudaOccupancyMaxActiveClusters(&maxc, tvk::cl::cluster_kernel, &q) != cudaSuccess) {
+            cudaGetLastError();
+            maxc = 0;
+        }
+        di.max_clusters[key] = maxc;
+    }
+    if (maxc <= 0) return false;
+    const int64_t clusters = std::min<int64_t>(a.N, (int64_t)maxc);
+    cfg.gridDim = dim3((unsigned)(clusters * c));
+    st = check_cuda(cudaLaunchKernelEx(&cfg, tvk::cl::cluster_kernel, p, n), "launch(tv cluster)");
+    return true;
+}
+
+}  // namespace
+
 uno_status tv_loss_launch(const TVArgs& a, void* workspace, cudaStream_t stream) {
     if (a.N == 0) {
         tvk::empty_mean_kernel<<<1, 1, 0, stream>>>(a.out_mean);
         return check_cuda(cudaGetLastError(), "launch(tv mean)");
     }
-    tvk::Params p{a, static_cast<tvk::Work*>(workspace)};
+    tvk::Params p{a, static_cast<tvk::Work*>(workspace), device_status_ptr()};
     tvk::count_mask_kernel<<<1, 1024, 0, stream>>>(a.mask, a.N, p.work);
     uno_status s = check_cuda(cudaGetLastError(), "launch(tv mask count)");
     if (s != UNO_OK) return s;
+    if (launch_cluster(p, stream, s)) return s;
     if (a.dtype == UNO_BF16) tvk::rows_kernel<__nv_bfloat16><<<(unsigned)a.N, tvk::kThreads, 0, stream>>>(p);
     else tvk::rows_kernel<float><<<(unsigned)a.N, tvk::kThreads, 0, stream>>>(p);
     return check_cuda(cudaGetLastError(), "launch(tv rows)");

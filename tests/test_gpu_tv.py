@@ -44,8 +44,13 @@ def _compare_grad(g_gpu, ref_grad, absdiff, psum):
     assert (~ok & undecided).mean() < 1e-3
 
 
+# bf16 rows whose length is a multiple of 8 run on the cluster kernel (on B200: cluster size 1
+# for V = 1000 and 12000, 2 for 20000, 4 for 40000, 8 for 151936 and 16 for 166144); the
+# others on the per-row kernel
 @pytest.mark.parametrize("N,V,dtype", [(7, 1000, "bf16"), (5, 4099, "bf16"), (3, 20000, "f32"), (4, 777, "f32"),
-                                       (2, 1, "bf16"), (9, 151936, "bf16")])
+                                       (2, 1, "bf16"), (9, 151936, "bf16"), (5, 20000, "bf16"),
+                                       (5, 12000, "bf16"), (3, 40000, "bf16"), (4, 166144, "bf16"), (600, 2048, "bf16"),
+                                       (1, 8, "bf16")])
 def test_tv_parity(N, V, dtype):
     w = W.TVWorkload("t", 40 + N + V, N=N, V=V)
     T, S = W.tv_logits(w)
@@ -59,6 +64,39 @@ def test_tv_parity(N, V, dtype):
     np.testing.assert_allclose(tv, ref["tv"], atol=PROB_TOL, rtol=0)
     assert abs(mean - ref["mean"]) <= PROB_TOL
     _compare_grad(g, ref["grad"], ref["absdiff"], _psum(Tf, Sf))
+
+
+@pytest.mark.parametrize("env,N,V", [
+    ({"UNO_TV_CLUSTER": "16"}, 5, 151936),   # a larger cluster than needed
+    ({"UNO_TV_CLUSTER": "16"}, 3, 64),       # half of the CTAs hold an empty slice
+    ({"UNO_TV_CLUSTER": "16"}, 4, 1000),     # ragged last slice
+    ({"UNO_TV_CLUSTER": "2"}, 300, 151936),  # does not fit: falls back to the default size
+    ({"UNO_TV_KERNEL": "rows"}, 6, 151936),  # the per-row kernel on bf16 rows
+])
+def test_tv_kernel_variants(monkeypatch, env, N, V):
+    """Every kernel variant and cluster size gives the oracle's result."""
+    for k, v in env.items():
+        monkeypatch.setenv(k, v)
+    w = W.TVWorkload("t", 7 + N + V, N=N, V=V)
+    T, S = W.tv_logits(w)
+    mask = np.ones(N, bool)
+    mask[::4] = False
+    tv, mean, g = _run(T, S, "bf16", mask=mask, grad_scale=0.75)
+    Tf, Sf = W.to_f64(T, "bf16"), W.to_f64(S, "bf16")
+    ref = oracle.tv_loss(Tf, Sf, mask=mask, grad_scale=np.float32(0.75), want_absdiff=True)
+    np.testing.assert_allclose(tv, ref["tv"], atol=PROB_TOL, rtol=0)
+    assert abs(mean - ref["mean"]) <= PROB_TOL
+    _compare_grad(g, ref["grad"], ref["absdiff"], _psum(Tf, Sf))
+
+
+def test_tv_identical_rows_zero_gradient():
+    """p == q: TV 0 and a gradient of exactly 0 (sign(q - p) = 0 everywhere), on both kernels."""
+    T, _ = W.tv_logits(W.TVWorkload("t", 43, N=5, V=151936))
+    tv, mean, g = _run(T, T, "bf16")
+    assert np.abs(tv).max() == 0.0 and mean == 0.0 and (g == 0).all()
+    T, _ = W.tv_logits(W.TVWorkload("t", 44, N=3, V=4099))
+    tv, mean, g = _run(T, T, "bf16")
+    assert np.abs(tv).max() == 0.0 and mean == 0.0 and (g == 0).all()
 
 
 def test_tv_identical_and_no_grad():
