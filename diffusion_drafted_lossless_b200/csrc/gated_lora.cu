@@ -8,8 +8,8 @@
 // weights).
 //
 // Three steps on the caller's stream:
-//   1. down:  Tacc = X A^T (fp32), split over K across CTAs, reduced with fp32 atomics;
-//   2. gate:  T = bf16(scale * g[m] * Tacc[m, :])   (rows with g = 0 give T = 0);
+//   1. down:  X A^T split over K across CTAs, each split's fp32 partial in its own slice;
+//   2. gate:  T = bf16(scale * g[m] * sum of the partials[m, :])   (rows with g = 0 give 0);
 //   3. main:  Y = [X | T] [W0 | B]^T — the K loop runs over d_in columns of (X, W0) and then
 //             over the r columns of (T, B), accumulating both into one TMEM accumulator.
 // Steps 1 and 3 use one warp-specialised kernel: warp 0 issues TMA tile loads into a
@@ -43,7 +43,7 @@ struct Params {
     void* out;              // bf16 or fp32 [M, ldo]
     int ldo;
     int out_f32;
-    float* red;             // if set: fp32 atomic accumulation into red[M, ldo] instead of out
+    float* red;             // if set: this split's fp32 partial into red[blockIdx.z][M, ldo] instead of out
     uint32_t* status;
 };
 
@@ -248,8 +248,17 @@ gemm_kernel(const __grid_constant__ CUtensorMap tA0, const __grid_constant__ CUt
                 if (row >= p.M || col0 >= p.N) continue;
                 const int ncol = min(32, p.N - col0);
                 if (p.red) {
-                    float* dst = p.red + (size_t)row * p.ldo + col0;
-                    for (int j = 0; j < ncol; ++j) atomicAdd(dst + j, __uint_as_float(r[j]));
+                    // split-K partial: this z-slice's own [M, ldo] fp32 slice, plain stores
+                    float* dst = p.red + ((size_t)blockIdx.z * p.M + row) * p.ldo + col0;
+                    if (ncol == 32) {
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4)
+                            *reinterpret_cast<float4*>(dst + j) = make_float4(
+                                __uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
+                                __uint_as_float(r[j + 3]));
+                    } else {
+                        for (int j = 0; j < ncol; ++j) dst[j] = __uint_as_float(r[j]);
+                    }
                 } else if (p.out_f32) {
                     float* dst = reinterpret_cast<float*>(p.out) + (size_t)row * p.ldo + col0;
                     if (ncol == 32) {
@@ -282,10 +291,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tA0, const __grid_constant__ CUt
                     }
                 }
             }
-        } else if (row < p.M && !p.red) {
-            // no K tiles: the product is zero
+        } else if (row < p.M) {
+            // no K tiles: the product (or this split's partial) is zero
             for (int col = n0; col < min(n0 + BN, p.N); ++col) {
-                if (p.out_f32) reinterpret_cast<float*>(p.out)[(size_t)row * p.ldo + col] = 0.f;
+                if (p.red) p.red[((size_t)blockIdx.z * p.M + row) * p.ldo + col] = 0.f;
+                else if (p.out_f32) reinterpret_cast<float*>(p.out)[(size_t)row * p.ldo + col] = 0.f;
                 else reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)row * p.ldo + col] = __float2bfloat16_rn(0.f);
             }
         }
@@ -303,14 +313,24 @@ gemm_kernel(const __grid_constant__ CUtensorMap tA0, const __grid_constant__ CUt
 // ---------------------------------------------------------------------------------------
 // small element-wise kernels
 // ---------------------------------------------------------------------------------------
-// T[m, j] = bf16(scale * g[m] * Tacc[m, j])
-__global__ void gate_kernel(const float* __restrict__ tacc, const float* __restrict__ gate, float scale, int M, int r,
-                            __nv_bfloat16* __restrict__ t) {
-    const int64_t n = (int64_t)M * r;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-        const int m = (int)(i / r);
-        const float g = gate ? gate[m] : 0.f;
-        t[i] = __float2bfloat16_rn(scale * g * tacc[i]);
+// T[m, j] = bf16(scale * g[m] * sum_s Tpart[s, m, j])   (r a multiple of 8)
+__global__ void gate_kernel(const float* __restrict__ tpart, int splits, const float* __restrict__ gate, float scale,
+                            int M, int r, __nv_bfloat16* __restrict__ t) {
+    const int64_t n4 = (int64_t)M * r / 4, slice = (int64_t)M * r;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
+        const int m = (int)(i * 4 / r);
+        const float g = gate ? scale * gate[m] : 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (g != 0.f)
+            for (int s = 0; s < splits; ++s) {
+                const float4 v = reinterpret_cast<const float4*>(tpart + s * slice)[i];
+                acc.x += v.x;
+                acc.y += v.y;
+                acc.z += v.z;
+                acc.w += v.w;
+            }
+        __nv_bfloat162 h0 = __floats2bfloat162_rn(g * acc.x, g * acc.y), h1 = __floats2bfloat162_rn(g * acc.z, g * acc.w);
+        reinterpret_cast<uint2*>(t)[i] = make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
     }
 }
 
@@ -381,6 +401,19 @@ int down_bn(int64_t rank) {
     return r16 <= 16 ? 16 : (r16 <= 32 ? 32 : (r16 <= 64 ? 64 : (r16 <= 128 ? 128 : 256)));
 }
 
+// split-K of the down-projection: about one wave of CTAs over the M tiles, each split
+// at least one K tile
+struct DownSplit {
+    int splits, per;
+};
+DownSplit down_split(int64_t M, int64_t d_in) {
+    const int m_tiles = (int)((M + BM - 1) / BM), kt0 = (int)(d_in / BK);
+    int splits = 148 / m_tiles;
+    splits = splits < 1 ? 1 : (splits > kt0 ? kt0 : splits);
+    const int per = (kt0 + splits - 1) / splits;
+    return {(kt0 + per - 1) / per, per};
+}
+
 struct WsLayout {
     size_t tacc, t, x, w0, a, b, total;
 };
@@ -393,7 +426,7 @@ WsLayout ws_layout(int64_t M, int64_t d_in, int64_t d_out, int64_t rank, uno_dty
         off = align_up(off + bytes, 256);
         return o;
     };
-    L.tacc = take((size_t)M * rank * 4);
+    L.tacc = take((size_t)down_split(M, d_in).splits * M * rank * 4);  // per-split partials
     L.t = take((size_t)M * rank * 2);
     if (dtype == UNO_F32) {
         L.x = take((size_t)M * d_in * 2);
@@ -436,33 +469,31 @@ uno_status gated_lora_launch(const GatedLoraArgs& g, void* workspace, cudaStream
     const int m_tiles = (M + BM - 1) / BM;
     uint32_t* status = device_status_ptr();
 
-    // ---- 1. down: Tacc = X A^T, split-K with fp32 atomics ----
+    // ---- 1. down: per-split partials of X A^T (fp32, plain stores) ----
     CUtensorMap tX, tA, tW0, tT, tBl;
     const int bnd = down_bn(r);
     if ((s = make_tmap(&tX, x, M, din, BM)) != UNO_OK) return s;
     if ((s = make_tmap(&tA, a, r, din, bnd)) != UNO_OK) return s;
-    if ((s = check_cuda(cudaMemsetAsync(tacc, 0, (size_t)M * r * 4, stream), "cudaMemsetAsync(Tacc)")) != UNO_OK)
-        return s;
     const int kt0 = din / BK;
-    int splits = 148 / m_tiles;
-    splits = splits < 1 ? 1 : (splits > kt0 ? kt0 : splits);
-    const int per = (kt0 + splits - 1) / splits;
-    splits = (kt0 + per - 1) / per;
+    const DownSplit ds = down_split(M, din);
     Params pd{};
     pd.M = M;
     pd.N = r;
     pd.kt0 = kt0;
     pd.kt1 = 0;
-    pd.kt_per_split = per;
+    pd.kt_per_split = ds.per;
     pd.red = tacc;
     pd.ldo = r;
     pd.status = status;
-    if ((s = launch_bn(bnd, tX, tA, tX, tA, pd, dim3(1, m_tiles, splits), stream)) != UNO_OK) return s;
+    if ((s = launch_bn(bnd, tX, tA, tX, tA, pd, dim3(1, m_tiles, ds.splits), stream)) != UNO_OK) return s;
 
-    // ---- 2. gate: T = bf16(scale * g * Tacc) ----
-    gate_kernel<<<(M * r + 255) / 256 < 1184 ? (M * r + 255) / 256 : 1184, 256, 0, stream>>>(tacc, g.gate, g.scale, M,
-                                                                                            r, t);
-    if ((s = check_cuda(cudaGetLastError(), "launch(gate)")) != UNO_OK) return s;
+    // ---- 2. gate: T = bf16(scale * g * sum of the partials) ----
+    {
+        const int64_t n4 = (int64_t)M * r / 4;
+        const int blocks = (int)((n4 + 255) / 256 < 1184 ? (n4 + 255) / 256 : 1184);
+        gate_kernel<<<blocks, 256, 0, stream>>>(tacc, ds.splits, g.gate, g.scale, M, r, t);
+        if ((s = check_cuda(cudaGetLastError(), "launch(gate)")) != UNO_OK) return s;
+    }
 
     // ---- 3. main: Y = [X | T] [W0 | B]^T ----
     int BN = 256;
