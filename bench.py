@@ -40,7 +40,7 @@ UNIT = "rows/s"
 WORKLOAD = "uno_step_b64_k16_v151936_qwen3_8b"
 LINEARS = W.QWEN3_8B
 VERIFY = W.SERVING_VERIFY
-LAUNCHES_PER_STEP = 7 * 3 + 3 + 2  # 7 x (down, gate, main) + verify (stream, finish, sequence) + TV (mask, rows)
+LAUNCHES_PER_STEP = 7 + 3 + 2  # 7 projections (one kernel each) + verify (stream, finish, sequence) + TV (mask, rows)
 
 
 def peaks():
@@ -332,7 +332,7 @@ def run_uno(args):
     value = world * rows / (ms * 1e-3)
     gemm_fl = sum(gemm_flops(L["shape"], LINEARS.M, LINEARS.rank, st.n_gated) for L in st.lin)
     # the dominant kernel: the TV kernel is one launch per step (plus a 1-block mask count);
-    # the linears are 21 launches (7 projections x 3 kernels), the verify 3
+    # the linears are 7 launches (one per projection), the verify 3
     per_launch = {"gated_lora_linears": ph["gated_lora_linears"] / 7, "block_verify": ph["block_verify"],
                   "tv_loss": ph["tv_loss"]}
     dominant = max(per_launch, key=per_launch.get)

@@ -7,22 +7,36 @@
 // model card introduction (seed, prefill, verification and AR rows use the frozen base
 // weights).
 //
-// Three steps on the caller's stream:
-//   1. down:  X A^T split over K across CTAs, each split's fp32 partial in its own slice;
-//   2. gate:  T = bf16(scale * g[m] * sum of the partials[m, :])   (rows with g = 0 give 0);
-//   3. main:  Y = [X | T] [W0 | B]^T — the K loop runs over d_in columns of (X, W0) and then
-//             over the r columns of (T, B), accumulating both into one TMEM accumulator.
-// Steps 1 and 3 use one warp-specialised kernel: warp 0 issues TMA tile loads into a
-// ring of shared-memory stages, warp 1 owns the TMEM accumulator and issues
-// tcgen05.mma (kind::f16, bf16 x bf16 -> fp32, 128 x BN x 16 per instruction) from one
-// thread, and warps 2-5 read the accumulator back with tcgen05.ld for the epilogue.
-// Every mbarrier wait is bounded; on timeout the kernel records UNO_ERR_TIMEOUT in the
-// device status word, lets its in-flight copies and MMAs drain (bounded), frees its TMEM
-// and returns.
+// One persistent kernel per call, one CTA per SM, as many CTAs as can be resident at once
+// (a cooperative launch where the runtime takes it). CTA c takes the work items
+// c, c + G, c + 2G, ... (G CTAs):
+//   1. adapter items (m, s), first in the list: the fp32 product X A^T of row tile m over
+//      the s-th range of K. With one range it is written at once as
+//      T = bf16(scale * g * (X A^T)); with several, each stores an fp32 partial and the item
+//      that completes row tile m last (a ticket) sums the partials into T. Row tile m's T is
+//      then published with a release flag carrying this call's epoch.
+//   2. output tiles (m, n): Y[m, n] = [X | T] [W0 | B]^T. The K loop runs over the d_in
+//      columns of (X, W0) and then over the r columns of (T, B), all into one TMEM
+//      accumulator; the loads of (T, B) wait (bounded) for row tile m's flag, by which
+//      time the adapter items, scheduled first everywhere, have normally long finished.
+// Warp roles: warp 0 issues TMA tile loads into a ring of shared-memory stages that runs on
+// across items; warp 1 owns TMEM (two accumulators) and issues tcgen05.mma (kind::f16,
+// bf16 x bf16 -> fp32, 128 x N x 16) from one thread; warps 2-5 drain one accumulator to
+// global memory while the next item accumulates into the other.
+// A second form (UNO_LORA_CG=2) runs each item on a cluster of two CTAs: one tcgen05.mma
+// stream with cta_group::2 issued by the leader computes a 256 x N tile, each CTA holding
+// its 128 rows of A and half of B, the TMA loads of both completing on the leader's
+// mbarriers (plain loads, no multicast).
+// Every wait is bounded; on timeout the kernel records UNO_ERR_TIMEOUT in the device status
+// word, stops issuing work, lets in-flight copies drain (bounded), frees its TMEM and
+// returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
+#include <chrono>
+#include <cstdlib>
 #include <cstring>
 
 #include "gated_lora.cuh"
@@ -30,20 +44,36 @@
 namespace uno {
 namespace glora {
 
-constexpr int BM = 128;         // rows per tile (UMMA M)
-constexpr int BK = 64;          // K elements per stage: one 128-byte swizzle row of bf16
+constexpr int BM = 128;          // rows per tile (UMMA M)
+constexpr int BK = 64;           // K elements per stage: one 128-byte swizzle row of bf16
 constexpr int UMMA_K = 16;
-constexpr int kThreads = 192;   // warp 0: TMA, warp 1: MMA + TMEM, warps 2-5: epilogue
-constexpr int kSmemBudget = 200 * 1024;
+constexpr int kThreads = 192;    // warp 0: TMA, warp 1: MMA + TMEM, warps 2-5: epilogue
+constexpr int kEpiThreads = 128;
+constexpr int kMaxStages = 8;
+constexpr int kSmemBudget = 220 * 1024;
+constexpr uint32_t A_BYTES = BM * BK * 2;
+constexpr uint32_t kFlagPolls = 1u << 22;  // polls of a T flag, each after a short sleep
 
 struct Params {
-    int M, N;               // output extent
-    int kt0, kt1;           // K tiles of segment 0 (X, W0) and segment 1 (T, B)
-    int kt_per_split;       // split-K: K tiles per z-slice of the grid (segment 0 only)
-    void* out;              // bf16 or fp32 [M, ldo]
-    int ldo;
+    int M, N, r;                  // rows, d_out, rank
+    int kt0, kt1;                 // K tiles of (X, W0) and of (T, B)
+    int m_tiles;                  // 128-row tiles (T flags, tickets)
+    int m_units;                  // row units of the work items: 128 x CG rows
+    int splits, per;              // adapter items: m_tiles x splits, `per` K tiles each
+    int n_adapter, n_items;       // adapter items, all items
+    int rb;                       // adapter accumulator width: r rounded up to 16 x CG
+    int stages;                   // shared-memory ring depth
+    uint32_t b_bytes;             // bytes of one B-operand stage (max(BN, rb) rows)
+    uint32_t cb;                  // TMEM columns of one accumulator
+    void* y;                      // [M, N] bf16 or fp32
     int out_f32;
-    float* red;             // if set: this split's fp32 partial into red[blockIdx.z][M, ldo] instead of out
+    float* tpart;                 // [splits][M][r] fp32 partials (splits > 1)
+    __nv_bfloat16* t;             // [M][r] bf16 T
+    const float* gate;            // [M] or NULL (all zero)
+    float scale;
+    unsigned long long* flags;    // [m_tiles]: the epoch once row tile m's T is written
+    unsigned long long* tickets;  // [m_tiles]: (epoch << 16) | partials stored
+    unsigned long long epoch;     // this call's tag, < 2^48, never 0
     uint32_t* status;
 };
 
@@ -113,231 +143,400 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-template <int BN>
-constexpr int tmem_cols() { return BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256)); }
 
-template <int BN>
-constexpr int stages() {
-    return (kSmemBudget - 1024) / (BM * BK * 2 + BN * BK * 2) < 8 ? (kSmemBudget - 1024) / (BM * BK * 2 + BN * BK * 2) : 8;
+__device__ __forceinline__ void named_sync_epilogue() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory"); }
+
+__device__ __forceinline__ bool wait_flag(const unsigned long long* f, unsigned long long epoch) {
+    for (uint32_t i = 0; i < kFlagPolls; ++i) {
+        unsigned long long v;
+        asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(f) : "memory");
+        if (v == epoch) {
+            // T was written through the generic proxy; the TMA loads read it through the async one
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            return true;
+        }
+        __nanosleep(64);
+    }
+    return false;
 }
 
-template <int BN>
-constexpr size_t smem_bytes() { return (size_t)stages<BN>() * (BM * BK * 2 + BN * BK * 2) + 1024; }
+// one more partial of row tile m stored; true for the one that completes the tile
+__device__ __forceinline__ bool take_ticket(unsigned long long* t, unsigned long long epoch, int splits) {
+    unsigned long long old = *reinterpret_cast<volatile unsigned long long*>(t), now = 0;
+    for (int i = 0; i < 1 << 20; ++i) {
+        now = (old >> 16) == epoch ? old + 1 : ((epoch << 16) | 1ull);
+        const unsigned long long seen = atomicCAS(t, old, now);
+        if (seen == old) break;
+        old = seen;
+    }
+    __threadfence();
+    return (int)(now & 0xFFFFull) == splits;
+}
 
-// ---------------------------------------------------------------------------------------
-// the GEMM kernel: C[m0:m0+128, n0:n0+BN] over K tiles of segment 0 then segment 1
-// ---------------------------------------------------------------------------------------
-template <int BN>
+struct Item {
+    bool adapter;
+    int m, j;    // row unit (128 x CG rows); split (adapter) or column tile (output)
+    int kb, ke;  // K tiles [kb, ke)
+};
+
+__device__ __forceinline__ Item decode(const Params& p, int item) {
+    Item it;
+    if (item < p.n_adapter) {
+        it.adapter = true;
+        it.m = item % p.m_units;
+        it.j = item / p.m_units;
+        it.kb = it.j * p.per;
+        it.ke = min(p.kt0, it.kb + p.per);
+    } else {
+        const int q = item - p.n_adapter;
+        it.adapter = false;
+        it.m = q % p.m_units;  // row units fastest: concurrent tiles share W0's column block
+        it.j = q / p.m_units;
+        it.kb = 0;
+        it.ke = p.kt0 + p.kt1;
+    }
+    return it;
+}
+
+// ---- pair (cta_group::2) forms: one MMA over the two CTAs of a cluster ----
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t map_to_rank(const void* local, uint32_t rank) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+    return remote;
+}
+__device__ __forceinline__ void pair_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// TMA load into this CTA's shared memory whose completed bytes count on the leader CTA's
+// mbarrier (cluster address `bar`)
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+}
+__device__ __forceinline__ void umma_bf16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8, %9, %10, %11, %12}, p;\n\t}\n" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u), "r"(0u), "r"(0u),
+        "r"(0u), "r"(0u));
+}
+// arrive on the mbarrier at this offset in both CTAs of the pair once the MMAs complete
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"((unsigned short)3)
+        : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// CG = 1: one CTA computes a 128 x N tile. CG = 2: the two CTAs of a cluster compute a
+// 256 x N tile with one MMA stream issued by the leader (rank 0): each CTA holds its 128
+// rows of A and half of the N rows of B, and its own 128-lane accumulator.
+template <int BN, int CG>
 __global__ void __launch_bounds__(kThreads, 1)
-gemm_kernel(const __grid_constant__ CUtensorMap tA0, const __grid_constant__ CUtensorMap tB0,
-            const __grid_constant__ CUtensorMap tA1, const __grid_constant__ CUtensorMap tB1, Params p) {
-    constexpr int ST = stages<BN>();
-    constexpr uint32_t A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2;
-    constexpr uint32_t TCOLS = tmem_cols<BN>();
+lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__ CUtensorMap tW0,
+                 const __grid_constant__ CUtensorMap tA, const __grid_constant__ CUtensorMap tT,
+                 const __grid_constant__ CUtensorMap tB, Params p) {
     extern __shared__ unsigned char smem_dyn[];
-    __shared__ __align__(8) uint64_t full[ST], empty[ST], accum;
+    __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages], tfull[2], tempty[2];
     __shared__ uint32_t tmem_holder;
-    __shared__ int s_abort;
+    __shared__ int s_abort, s_last;
 
     // 128-byte swizzled tiles need 1024-byte aligned shared-memory addresses
     unsigned char* smem = smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u);
+    const int ST = p.stages;
     unsigned char* sA = smem;
     unsigned char* sB = smem + (size_t)ST * A_BYTES;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
-    // K tiles of this CTA: split-K slices cover segment 0 only
-    int kb = 0, ke = p.kt0 + p.kt1;
-    if (p.kt_per_split > 0) {
-        kb = blockIdx.z * p.kt_per_split;
-        ke = min(p.kt0, kb + p.kt_per_split);
-    }
-    const int nk = max(0, ke - kb);
+    volatile int* abort_flag = &s_abort;
+    const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
+    const bool leader = rank == 0;
+    const int unit0 = blockIdx.x / CG, units = gridDim.x / CG;  // this CTA's pair and the pair count
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < ST; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(&accum, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], CG * kEpiThreads / 32);
+        }
         s_abort = 0;
         fence_mbar_init();
     }
-    if (warp == 1) {  // TMEM accumulator: TCOLS fp32 columns x 128 lanes
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_holder)),
-                     "r"(TCOLS)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    if (warp == 1) {  // two accumulators of cb fp32 columns x 128 lanes (in each CTA of a pair)
+        if constexpr (CG == 2) {
+            asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                             smem_u32(&tmem_holder)),
+                         "r"(2 * p.cb)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+        } else {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                             smem_u32(&tmem_holder)),
+                         "r"(2 * p.cb)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        }
     }
     if (warp == 0 && lane == 0) {
-        prefetch_tmap(&tA0);
-        prefetch_tmap(&tB0);
-        if (p.kt1 > 0) {
-            prefetch_tmap(&tA1);
-            prefetch_tmap(&tB1);
-        }
+        prefetch_tmap(&tX);
+        prefetch_tmap(&tW0);
+        prefetch_tmap(&tA);
+        prefetch_tmap(&tT);
+        prefetch_tmap(&tB);
     }
     tmem_fence_before();
     __syncthreads();
+    if constexpr (CG == 2) pair_sync();  // the peer's mbarriers exist before any remote arrive
     tmem_fence_after();
     const uint32_t tmem = tmem_holder;
 
     if (warp == 0) {
         if (lane == 0) {
-            // ---- TMA producer ----
-            int it = 0;
-            for (; it < nk; ++it) {
-                const int s = it % ST;
-                if (it >= ST && !mbar_wait(&empty[s], (uint32_t)(((it / ST) & 1) ^ 1))) {
-                    s_abort = 1;
-                    break;
-                }
-                if (*reinterpret_cast<volatile int*>(&s_abort)) break;
-                const int kt = kb + it;
-                mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES);
-                if (kt < p.kt0) {
-                    tma_load_2d(sA + (size_t)s * A_BYTES, &tA0, kt * BK, m0, &full[s]);
-                    tma_load_2d(sB + (size_t)s * B_BYTES, &tB0, kt * BK, n0, &full[s]);
-                } else {
-                    tma_load_2d(sA + (size_t)s * A_BYTES, &tA1, (kt - p.kt0) * BK, m0, &full[s]);
-                    tma_load_2d(sB + (size_t)s * B_BYTES, &tB1, (kt - p.kt0) * BK, n0, &full[s]);
+            // ---- TMA producer (each CTA loads its own rows of A and its half of B) ----
+            const uint32_t lead_full0 = CG == 2 ? map_to_rank(&full[0], 0) : 0u;
+            uint32_t g = 0;  // K steps issued by this CTA, across items
+            for (int item = unit0; item < p.n_items && !*abort_flag; item += units) {
+                const Item w = decode(p, item);
+                const int m0 = w.m * BM * CG + (int)rank * BM;
+                const int nrows = w.adapter ? p.rb : BN;  // B rows of the whole (pair) tile
+                const int n0 = w.adapter ? (int)rank * (nrows / CG) : w.j * BN + (int)rank * (BN / CG);
+                for (int kt = w.kb; kt < w.ke; ++kt, ++g) {
+                    const int s = (int)(g % ST);
+                    if (g >= (uint32_t)ST && !mbar_wait(&empty[s], ((g / ST) & 1) ^ 1)) {
+                        *abort_flag = 1;
+                        break;
+                    }
+                    // rows past M have no T (their loads are zero-filled): nothing to wait for
+                    if (!w.adapter && kt == p.kt0 && m0 < p.M && !wait_flag(&p.flags[m0 / BM], p.epoch)) {
+                        *abort_flag = 1;
+                        break;
+                    }
+                    if (*abort_flag) break;
+                    unsigned char* a = sA + (size_t)s * A_BYTES;
+                    unsigned char* b = sB + (size_t)s * p.b_bytes;
+                    const CUtensorMap* ma = w.adapter || kt < p.kt0 ? &tX : &tT;
+                    const CUtensorMap* mb = w.adapter ? &tA : (kt < p.kt0 ? &tW0 : &tB);
+                    const int kx = (w.adapter || kt < p.kt0 ? kt : kt - p.kt0) * BK;
+                    if (leader) mbar_arrive_expect_tx(&full[s], CG * A_BYTES + (uint32_t)nrows * 128u);
+                    if constexpr (CG == 2) {
+                        const uint32_t bar = lead_full0 + (uint32_t)s * 8u;
+                        tma_load_2d_pair(a, ma, kx, m0, bar);
+                        tma_load_2d_pair(b, mb, kx, n0, bar);
+                    } else {
+                        tma_load_2d(a, ma, kx, m0, &full[s]);
+                        tma_load_2d(b, mb, kx, n0, &full[s]);
+                    }
                 }
             }
-            // drain: wait (bounded) for the loads that no MMA will consume
-            if (*reinterpret_cast<volatile int*>(&s_abort))
-                for (int j = max(0, it - ST); j < it; ++j) mbar_wait(&full[j % ST], (uint32_t)((j / ST) & 1), 1u << 16);
+            // on abort: wait (bounded) for the loads that no MMA will consume
+            if (*abort_flag && leader) {
+                const uint32_t lo = g > (uint32_t)ST ? g - ST : 0;
+                for (uint32_t j = lo; j < g; ++j) mbar_wait(&full[j % ST], (j / ST) & 1, 1u << 16);
+            }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            // ---- MMA issuer (one thread) ----
-            constexpr uint32_t idesc = instr_desc_bf16(BM, BN);
-            int it = 0;
-            for (; it < nk; ++it) {
-                const int s = it % ST;
-                if (!mbar_wait(&full[s], (uint32_t)((it / ST) & 1))) {
-                    s_abort = 1;
+        if (lane == 0 && leader) {
+            // ---- MMA issuer (one thread of the leader CTA) ----
+            uint32_t g = 0, li = 0;
+            for (int item = unit0; item < p.n_items && !*abort_flag; item += units, ++li) {
+                const Item w = decode(p, item);
+                const int buf = li & 1;
+                if (li >= 2 && !mbar_wait(&tempty[buf], ((li >> 1) & 1) ^ 1)) {
+                    *abort_flag = 1;
                     break;
                 }
                 tmem_fence_after();
-                const uint32_t a0 = smem_u32(sA + (size_t)s * A_BYTES), b0 = smem_u32(sB + (size_t)s * B_BYTES);
+                const uint32_t d = tmem + (uint32_t)buf * p.cb;
+                const uint32_t idesc = instr_desc_bf16(BM * CG, w.adapter ? p.rb : BN);
+                bool ok = true;
+                for (int kt = w.kb; kt < w.ke; ++kt, ++g) {
+                    const int s = (int)(g % ST);
+                    if (!mbar_wait(&full[s], (g / ST) & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    tmem_fence_after();
+                    const uint32_t a0 = smem_u32(sA + (size_t)s * A_BYTES), b0 = smem_u32(sB + (size_t)s * p.b_bytes);
 #pragma unroll
-                for (int kk = 0; kk < BK / UMMA_K; ++kk) {
-                    const uint32_t off = kk * UMMA_K * 2;  // bytes along K within the 128-byte row
-                    umma_bf16(tmem, smem_desc_sw128(a0 + off), smem_desc_sw128(b0 + off), idesc,
-                              (it > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+                        const uint32_t off = kk * UMMA_K * 2;  // bytes along K within the 128-byte row
+                        const uint32_t acc = (kt > w.kb || kk > 0) ? 1u : 0u;
+                        if constexpr (CG == 2)
+                            umma_bf16_pair(d, smem_desc_sw128(a0 + off), smem_desc_sw128(b0 + off), idesc, acc);
+                        else
+                            umma_bf16(d, smem_desc_sw128(a0 + off), smem_desc_sw128(b0 + off), idesc, acc);
+                    }
+                    // the stage is free (in both CTAs) once these MMAs have read it
+                    if constexpr (CG == 2) umma_commit_pair(&empty[s]);
+                    else umma_commit(&empty[s]);
                 }
-                umma_commit(&empty[s]);  // the stage is free once these MMAs have read it
+                if (!ok) {
+                    *abort_flag = 1;
+                    break;
+                }
+                // the accumulator is final once every MMA has completed
+                if constexpr (CG == 2) umma_commit_pair(&tfull[buf]);
+                else umma_commit(&tfull[buf]);
             }
-            umma_commit(&accum);  // the accumulator is final once every MMA has completed
         }
     } else {
-        // ---- epilogue: TMEM -> registers -> global ----
-        const int q = warp & 3;  // TMEM lane quarter this warp may access
-        const int row = m0 + q * 32 + lane;
-        const bool okw = mbar_wait(&accum, 0);
-        tmem_fence_after();
-        if (!okw) {
-            if (lane == 0) s_abort = 1;
-        } else if (nk > 0) {
-#pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 32) {
-                uint32_t r[32];
-                __syncwarp();  // tcgen05.ld is .sync.aligned: the whole warp, converged
-                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, r);
-                const int col0 = n0 + c0;
-                if (row >= p.M || col0 >= p.N) continue;
-                const int ncol = min(32, p.N - col0);
-                if (p.red) {
-                    // split-K partial: this z-slice's own [M, ldo] fp32 slice, plain stores
-                    float* dst = p.red + ((size_t)blockIdx.z * p.M + row) * p.ldo + col0;
-                    if (ncol == 32) {
-#pragma unroll
-                        for (int j = 0; j < 32; j += 4)
-                            *reinterpret_cast<float4*>(dst + j) = make_float4(
-                                __uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
-                                __uint_as_float(r[j + 3]));
+        // ---- epilogue: TMEM -> registers -> global, four warps, one TMEM lane quarter each ----
+        const int q = warp & 3;
+        const int et = threadIdx.x - 64;  // 0..127 across the epilogue warps
+        const uint32_t lead_tempty0 = CG == 2 ? map_to_rank(&tempty[0], 0) : 0u;
+        uint32_t li = 0;
+        for (int item = unit0; item < p.n_items; item += units, ++li) {
+            const Item w = decode(p, item);
+            const int buf = li & 1;
+            const int m0 = w.m * BM * CG + (int)rank * BM;
+            const int row = m0 + q * 32 + lane;
+            bool ok = !*abort_flag && mbar_wait(&tfull[buf], (li >> 1) & 1);
+            tmem_fence_after();
+            if (!ok) *abort_flag = 1;
+            const uint32_t taddr = tmem + (uint32_t)buf * p.cb + ((uint32_t)(q * 32) << 16);
+            if (ok && w.adapter) {
+                const float gs = (row < p.M && p.gate) ? p.scale * p.gate[row] : 0.f;
+                for (int c0 = 0; c0 < p.rb; c0 += 32) {
+                    uint32_t r[32];
+                    __syncwarp();
+                    tmem_ld32(taddr + (uint32_t)c0, r);
+                    if (row >= p.M || c0 >= p.r) continue;
+                    const int ncol = min(32, p.r - c0);  // a multiple of 8
+                    if (p.splits == 1) {
+                        __nv_bfloat16* dst = p.t + (size_t)row * p.r + c0;
+                        for (int j = 0; j < ncol; j += 8) {
+                            __nv_bfloat162 h0 = __floats2bfloat162_rn(gs * __uint_as_float(r[j]), gs * __uint_as_float(r[j + 1]));
+                            __nv_bfloat162 h1 = __floats2bfloat162_rn(gs * __uint_as_float(r[j + 2]), gs * __uint_as_float(r[j + 3]));
+                            __nv_bfloat162 h2 = __floats2bfloat162_rn(gs * __uint_as_float(r[j + 4]), gs * __uint_as_float(r[j + 5]));
+                            __nv_bfloat162 h3 = __floats2bfloat162_rn(gs * __uint_as_float(r[j + 6]), gs * __uint_as_float(r[j + 7]));
+                            *reinterpret_cast<uint4*>(dst + j) =
+                                make_uint4(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),
+                                           *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
+                        }
                     } else {
-                        for (int j = 0; j < ncol; ++j) dst[j] = __uint_as_float(r[j]);
+                        float* dst = p.tpart + ((size_t)w.j * p.M + row) * p.r + c0;
+                        for (int j = 0; j < ncol; j += 4)
+                            *reinterpret_cast<float4*>(dst + j) =
+                                make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
+                                            __uint_as_float(r[j + 3]));
                     }
-                } else if (p.out_f32) {
-                    float* dst = reinterpret_cast<float*>(p.out) + (size_t)row * p.ldo + col0;
-                    if (ncol == 32) {
-#pragma unroll
-                        for (int j = 0; j < 32; j += 4)
-                            *reinterpret_cast<float4*>(dst + j) = make_float4(
-                                __uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
-                                __uint_as_float(r[j + 3]));
+                }
+            } else if (ok) {
+                for (int c0 = 0; c0 < BN; c0 += 32) {
+                    uint32_t r[32];
+                    __syncwarp();
+                    tmem_ld32(taddr + (uint32_t)c0, r);
+                    const int col0 = w.j * BN + c0;
+                    if (row >= p.M || col0 >= p.N) continue;
+                    const int ncol = min(32, p.N - col0);  // a multiple of 32: N is a multiple of 64
+                    if (p.out_f32) {
+                        float* dst = reinterpret_cast<float*>(p.y) + (size_t)row * p.N + col0;
+                        for (int j = 0; j < ncol; j += 4)
+                            *reinterpret_cast<float4*>(dst + j) =
+                                make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
+                                            __uint_as_float(r[j + 3]));
                     } else {
-                        for (int j = 0; j < ncol; ++j) dst[j] = __uint_as_float(r[j]);
-                    }
-                } else {
-                    __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.ldo + col0;
-                    if (ncol == 32) {
+                        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.y) + (size_t)row * p.N + col0;
 #pragma unroll
                         for (int j = 0; j < 32; j += 8) {
-                            uint4 o;
                             __nv_bfloat162 h0 = __floats2bfloat162_rn(__uint_as_float(r[j]), __uint_as_float(r[j + 1]));
                             __nv_bfloat162 h1 = __floats2bfloat162_rn(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
                             __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[j + 4]), __uint_as_float(r[j + 5]));
                             __nv_bfloat162 h3 = __floats2bfloat162_rn(__uint_as_float(r[j + 6]), __uint_as_float(r[j + 7]));
-                            o.x = *reinterpret_cast<uint32_t*>(&h0);
-                            o.y = *reinterpret_cast<uint32_t*>(&h1);
-                            o.z = *reinterpret_cast<uint32_t*>(&h2);
-                            o.w = *reinterpret_cast<uint32_t*>(&h3);
-                            *reinterpret_cast<uint4*>(dst + j) = o;
+                            *reinterpret_cast<uint4*>(dst + j) =
+                                make_uint4(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),
+                                           *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
                         }
-                    } else {
-                        for (int j = 0; j < ncol; ++j) dst[j] = __float2bfloat16_rn(__uint_as_float(r[j]));
                     }
                 }
             }
-        } else if (row < p.M) {
-            // no K tiles: the product (or this split's partial) is zero
-            for (int col = n0; col < min(n0 + BN, p.N); ++col) {
-                if (p.red) p.red[((size_t)blockIdx.z * p.M + row) * p.ldo + col] = 0.f;
-                else if (p.out_f32) reinterpret_cast<float*>(p.out)[(size_t)row * p.ldo + col] = 0.f;
-                else reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)row * p.ldo + col] = __float2bfloat16_rn(0.f);
+            // the accumulator may be refilled (the leader's MMA waits for both CTAs' warps)
+            tmem_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if constexpr (CG == 2) mbar_arrive_remote(lead_tempty0 + (uint32_t)buf * 8u);
+                else mbar_arrive(&tempty[buf]);
+            }
+
+            if (w.adapter) {
+                // publish this CTA's 128 rows of T (all four warps take every barrier)
+                const int tile = m0 / BM;
+                asm volatile("fence.proxy.async.global;" ::: "memory");
+                __threadfence();
+                named_sync_epilogue();
+                if (p.splits > 1) {
+                    if (et == 0)
+                        s_last = (ok && !*abort_flag && m0 < p.M) ? take_ticket(&p.tickets[tile], p.epoch, p.splits) : 0;
+                    named_sync_epilogue();
+                    if (s_last) {
+                        // sum the partials of these 128 rows into T
+                        const int r4 = p.r / 4;
+                        for (int idx = et; idx < BM * r4; idx += kEpiThreads) {
+                            const int rr = m0 + idx / r4, c = (idx % r4) * 4;
+                            if (rr >= p.M) continue;
+                            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                            for (int s = 0; s < p.splits; ++s) {
+                                const float4 v = __ldcg(reinterpret_cast<const float4*>(
+                                    p.tpart + ((size_t)s * p.M + rr) * p.r + c));
+                                acc.x += v.x;
+                                acc.y += v.y;
+                                acc.z += v.z;
+                                acc.w += v.w;
+                            }
+                            const float gs = p.gate ? p.scale * p.gate[rr] : 0.f;
+                            __nv_bfloat162 h0 = __floats2bfloat162_rn(gs * acc.x, gs * acc.y);
+                            __nv_bfloat162 h1 = __floats2bfloat162_rn(gs * acc.z, gs * acc.w);
+                            *reinterpret_cast<uint2*>(p.t + (size_t)rr * p.r + c) =
+                                make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
+                        }
+                        asm volatile("fence.proxy.async.global;" ::: "memory");
+                        __threadfence();
+                    }
+                    named_sync_epilogue();
+                    if (et == 0 && s_last)
+                        asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(&p.flags[tile]), "l"(p.epoch) : "memory");
+                } else if (et == 0 && ok && m0 < p.M) {
+                    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(&p.flags[tile]), "l"(p.epoch) : "memory");
+                }
             }
         }
     }
 
     tmem_fence_before();
     __syncthreads();
+    if constexpr (CG == 2) pair_sync();  // nothing of the pair still reaches this CTA
     if (warp == 1) {
         tmem_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TCOLS) : "memory");
+        if constexpr (CG == 2)
+            asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * p.cb) : "memory");
+        else
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * p.cb) : "memory");
     }
     if (threadIdx.x == 0 && s_abort) record_device_status(p.status, (uint32_t)UNO_ERR_TIMEOUT);
-}
-
-// ---------------------------------------------------------------------------------------
-// small element-wise kernels
-// ---------------------------------------------------------------------------------------
-// T[m, j] = bf16(scale * g[m] * sum_s Tpart[s, m, j])   (r a multiple of 8)
-__global__ void gate_kernel(const float* __restrict__ tpart, int splits, const float* __restrict__ gate, float scale,
-                            int M, int r, __nv_bfloat16* __restrict__ t) {
-    const int64_t n4 = (int64_t)M * r / 4, slice = (int64_t)M * r;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
-        const int m = (int)(i * 4 / r);
-        const float g = gate ? scale * gate[m] : 0.f;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (g != 0.f)
-            for (int s = 0; s < splits; ++s) {
-                const float4 v = reinterpret_cast<const float4*>(tpart + s * slice)[i];
-                acc.x += v.x;
-                acc.y += v.y;
-                acc.z += v.z;
-                acc.w += v.w;
-            }
-        __nv_bfloat162 h0 = __floats2bfloat162_rn(g * acc.x, g * acc.y), h1 = __floats2bfloat162_rn(g * acc.z, g * acc.w);
-        reinterpret_cast<uint2*>(t)[i] = make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
-    }
 }
 
 __global__ void f32_to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst, int64_t n) {
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
         dst[i] = __float2bfloat16_rn(src[i]);
 }
+
 
 // ---------------------------------------------------------------------------------------
 // host side
@@ -369,150 +568,217 @@ uno_status make_tmap(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols
     return UNO_OK;
 }
 
-template <int BN>
-uno_status launch_gemm(const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& a1, const CUtensorMap& b1,
-                       const Params& p, dim3 grid, cudaStream_t stream) {
-    static bool attr = false;
-    if (!attr) {
-        uno_status s = check_cuda(cudaFuncSetAttribute(gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                       (int)smem_bytes<BN>()),
-                                  "cudaFuncSetAttribute(gemm)");
-        if (s != UNO_OK) return s;
-        attr = true;
-    }
-    gemm_kernel<BN><<<grid, kThreads, smem_bytes<BN>(), stream>>>(a0, b0, a1, b1, p);
-    return check_cuda(cudaGetLastError(), "launch(gated lora gemm)");
-}
 
-uno_status launch_bn(int BN, const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& a1,
-                     const CUtensorMap& b1, const Params& p, dim3 grid, cudaStream_t stream) {
-    switch (BN) {
-        case 16: return launch_gemm<16>(a0, b0, a1, b1, p, grid, stream);
-        case 32: return launch_gemm<32>(a0, b0, a1, b1, p, grid, stream);
-        case 64: return launch_gemm<64>(a0, b0, a1, b1, p, grid, stream);
-        case 128: return launch_gemm<128>(a0, b0, a1, b1, p, grid, stream);
-        case 256: return launch_gemm<256>(a0, b0, a1, b1, p, grid, stream);
-    }
-    return set_error(UNO_ERR_UNSUPPORTED, "tile width %d", BN);
-}
-
-int down_bn(int64_t rank) {
-    int r16 = (int)((rank + 15) / 16 * 16);
-    return r16 <= 16 ? 16 : (r16 <= 32 ? 32 : (r16 <= 64 ? 64 : (r16 <= 128 ? 128 : 256)));
-}
-
-// split-K of the down-projection: about one wave of CTAs over the M tiles, each split
-// at least one K tile
-struct DownSplit {
-    int splits, per;
-};
-DownSplit down_split(int64_t M, int64_t d_in) {
-    const int m_tiles = (int)((M + BM - 1) / BM), kt0 = (int)(d_in / BK);
-    int splits = 148 / m_tiles;
-    splits = splits < 1 ? 1 : (splits > kt0 ? kt0 : splits);
-    const int per = (kt0 + splits - 1) / splits;
-    return {(kt0 + per - 1) / per, per};
-}
-
-struct WsLayout {
-    size_t tacc, t, x, w0, a, b, total;
+// The launch plan of one call (also sizes the workspace).
+struct Plan {
+    int CG, BN, rb, cb, m_tiles, m_units, n_tiles, kt0, kt1, splits, per, n_adapter, n_items, stages;
+    uint32_t b_bytes;
+    size_t smem;
+    // workspace offsets
+    size_t flags, tickets, t, tpart, x, w0, a, b, total;
 };
 
-WsLayout ws_layout(int64_t M, int64_t d_in, int64_t d_out, int64_t rank, uno_dtype dtype) {
-    WsLayout L{};
+Plan make_plan(int64_t M, int64_t d_in, int64_t d_out, int64_t rank, uno_dtype dtype) {
+    Plan P{};
+    P.m_tiles = (int)((M + BM - 1) / BM);
+    // Single-CTA 128 x BN tiles. The CTA-pair form (256 x 256 tiles, one MMA stream over two
+    // SMs, each loading half of B) is selected with UNO_LORA_CG=2; on the Qwen3-8B and
+    // looped-3B shapes it measured no faster, so it is not the default.
+    P.CG = 1;
+    if (const char* e = getenv("UNO_LORA_CG")) {
+        const int c = atoi(e);
+        if (c == 1 || (c == 2 && M >= 2 * BM && d_out % 256 == 0)) P.CG = c;
+    }
+    P.m_units = (int)((M + (int64_t)BM * P.CG - 1) / ((int64_t)BM * P.CG));
+    if (P.CG == 2) {
+        P.BN = 256;
+    } else {
+        P.BN = 256;
+        while (P.BN > 64 && (int64_t)P.m_tiles * ((d_out + P.BN - 1) / P.BN) < 120) P.BN >>= 1;
+    }
+    P.n_tiles = (int)((d_out + P.BN - 1) / P.BN);
+    const int rq = 16 * P.CG;  // each CTA of a pair holds rb / 2 rows of A: a multiple of 16
+    P.rb = (int)((rank + rq - 1) / rq * rq);
+    const int w = P.BN > P.rb ? P.BN : P.rb;  // N of the widest MMA
+    P.cb = 32;
+    while (P.cb < w) P.cb <<= 1;
+    P.kt0 = (int)(d_in / BK);
+    P.kt1 = (int)((rank + BK - 1) / BK);
+    // One adapter item per row unit: its time is set by streaming the unit's rows of X and
+    // all of A through the SM, not by its MMAs, and summing split partials back in one CTA
+    // costs more than it saves (the split path stays for UNO_LORA_SPLITS=n).
+    int splits = 1;
+    if (const char* e = getenv("UNO_LORA_SPLITS")) splits = atoi(e);
+    splits = splits < 1 ? 1 : (splits > P.kt0 ? P.kt0 : splits);
+    P.per = (P.kt0 + splits - 1) / splits;
+    P.splits = (P.kt0 + P.per - 1) / P.per;
+    P.n_adapter = P.m_units * P.splits;
+    P.n_items = P.n_adapter + P.m_units * P.n_tiles;
+    P.b_bytes = (uint32_t)(w / P.CG) * 128u;
+    P.stages = (int)((kSmemBudget - 1024) / (A_BYTES + P.b_bytes));
+    if (P.stages > kMaxStages) P.stages = kMaxStages;
+    P.smem = (size_t)P.stages * (A_BYTES + P.b_bytes) + 1024;
     size_t off = 0;
     auto take = [&](size_t bytes) {
         size_t o = off;
         off = align_up(off + bytes, 256);
         return o;
     };
-    L.tacc = take((size_t)down_split(M, d_in).splits * M * rank * 4);  // per-split partials
-    L.t = take((size_t)M * rank * 2);
+    P.flags = take((size_t)P.m_tiles * 8);
+    P.tickets = take((size_t)P.m_tiles * 8);
+    P.t = take((size_t)M * rank * 2);
+    P.tpart = P.splits > 1 ? take((size_t)P.splits * M * rank * 4) : 0;
     if (dtype == UNO_F32) {
-        L.x = take((size_t)M * d_in * 2);
-        L.w0 = take((size_t)d_out * d_in * 2);
-        L.a = take((size_t)rank * d_in * 2);
-        L.b = take((size_t)d_out * rank * 2);
+        P.x = take((size_t)M * d_in * 2);
+        P.w0 = take((size_t)d_out * d_in * 2);
+        P.a = take((size_t)rank * d_in * 2);
+        P.b = take((size_t)d_out * rank * 2);
     }
-    L.total = off;
-    return L;
+    P.total = off;
+    return P;
+}
+
+// A fresh tag per call (48 bits, never 0), starting from a time-derived value so that flags
+// left in a reused workspace by another process are not mistaken for this call's.
+unsigned long long next_epoch() {
+    static std::atomic<unsigned long long> counter{
+        (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count() * 2654435761ull};
+    unsigned long long e;
+    do {
+        e = counter.fetch_add(1) & 0xFFFFFFFFFFFFull;
+    } while (e == 0);
+    return e;
+}
+
+int num_sms_cached() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 1;
+    }
+    return n;
+}
+
+template <int BN, int CG>
+uno_status launch_t(const CUtensorMap (&maps)[5], Params& p, const Plan& P, cudaStream_t stream) {
+    static bool attr = false;
+    if (!attr) {
+        uno_status s = check_cuda(cudaFuncSetAttribute(lora_gemm_kernel<BN, CG>,
+                                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                       (int)(kSmemBudget + 1024)),
+                                  "cudaFuncSetAttribute(gated lora)");
+        if (s != UNO_OK) return s;
+        attr = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attrs[2];
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = P.smem;
+    cfg.stream = stream;
+    cfg.attrs = attrs;
+    int n_attr = 0;
+    attrs[n_attr].id = cudaLaunchAttributeClusterDimension;
+    attrs[n_attr].val.clusterDim.x = CG;
+    attrs[n_attr].val.clusterDim.y = 1;
+    attrs[n_attr].val.clusterDim.z = 1;
+    ++n_attr;
+    cfg.numAttrs = n_attr;
+    // resident units (CTAs or CTA pairs): an output tile may wait for its row unit's T
+    int resident = 0;
+    {
+        cudaLaunchConfig_t q = cfg;
+        q.gridDim = dim3(CG);
+        uno_status s = check_cuda(cudaOccupancyMaxActiveClusters(&resident, lora_gemm_kernel<BN, CG>, &q),
+                                  "cudaOccupancyMaxActiveClusters(gated lora)");
+        if (s != UNO_OK) return s;
+    }
+    if (resident < 1) return set_error(UNO_ERR_CUDA, "gated lora kernel does not fit on the GPU");
+    const int units = p.n_items < resident ? p.n_items : resident;
+    cfg.gridDim = dim3((unsigned)(units * CG));
+    // Ask for a cooperative launch (every CTA resident, as the waits on T assume); where the
+    // runtime does not take it together with clusters, the grid is sized to what is
+    // resident at once, which an otherwise idle GPU runs in full.
+    attrs[n_attr].id = cudaLaunchAttributeCooperative;
+    attrs[n_attr].val.cooperative = 1;
+    cfg.numAttrs = n_attr + 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, lora_gemm_kernel<BN, CG>, maps[0], maps[1], maps[2], maps[3], maps[4], p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        cfg.numAttrs = n_attr;
+        e = cudaLaunchKernelEx(&cfg, lora_gemm_kernel<BN, CG>, maps[0], maps[1], maps[2], maps[3], maps[4], p);
+    }
+    return check_cuda(e, "launch(gated lora)");
 }
 
 }  // namespace glora
 
 size_t gated_lora_workspace_bytes(int64_t M, int64_t d_in, int64_t d_out, int64_t rank, uno_dtype dtype) {
-    return glora::ws_layout(M, d_in, d_out, rank, dtype).total;
+    return glora::make_plan(M, d_in, d_out, rank, dtype).total;
 }
 
 uno_status gated_lora_launch(const GatedLoraArgs& g, void* workspace, cudaStream_t stream) {
     using namespace glora;
-    const WsLayout L = ws_layout(g.M, g.d_in, g.d_out, g.rank, g.dtype);
+    const Plan P = make_plan(g.M, g.d_in, g.d_out, g.rank, g.dtype);
     unsigned char* ws = static_cast<unsigned char*>(workspace);
-    float* tacc = reinterpret_cast<float*>(ws + L.tacc);
-    __nv_bfloat16* t = reinterpret_cast<__nv_bfloat16*>(ws + L.t);
     const void *x = g.x, *w0 = g.w0, *a = g.a, *b = g.b;
     uno_status s;
     if (g.dtype == UNO_F32) {  // round the fp32 operands to bf16 once
         struct { const void* src; size_t off; int64_t n; } cv[4] = {
-            {g.x, L.x, g.M * g.d_in}, {g.w0, L.w0, g.d_out * g.d_in}, {g.a, L.a, g.rank * g.d_in}, {g.b, L.b, g.d_out * g.rank}};
+            {g.x, P.x, g.M * g.d_in}, {g.w0, P.w0, g.d_out * g.d_in}, {g.a, P.a, g.rank * g.d_in}, {g.b, P.b, g.d_out * g.rank}};
         for (auto& c : cv) {
             f32_to_bf16_kernel<<<592, 256, 0, stream>>>(static_cast<const float*>(c.src),
                                                       reinterpret_cast<__nv_bfloat16*>(ws + c.off), c.n);
             if ((s = check_cuda(cudaGetLastError(), "launch(f32->bf16)")) != UNO_OK) return s;
         }
-        x = ws + L.x;
-        w0 = ws + L.w0;
-        a = ws + L.a;
-        b = ws + L.b;
+        x = ws + P.x;
+        w0 = ws + P.w0;
+        a = ws + P.a;
+        b = ws + P.b;
     }
     const int M = (int)g.M, din = (int)g.d_in, dout = (int)g.d_out, r = (int)g.rank;
-    const int m_tiles = (M + BM - 1) / BM;
-    uint32_t* status = device_status_ptr();
-
-    // ---- 1. down: per-split partials of X A^T (fp32, plain stores) ----
-    CUtensorMap tX, tA, tW0, tT, tBl;
-    const int bnd = down_bn(r);
-    if ((s = make_tmap(&tX, x, M, din, BM)) != UNO_OK) return s;
-    if ((s = make_tmap(&tA, a, r, din, bnd)) != UNO_OK) return s;
-    const int kt0 = din / BK;
-    const DownSplit ds = down_split(M, din);
-    Params pd{};
-    pd.M = M;
-    pd.N = r;
-    pd.kt0 = kt0;
-    pd.kt1 = 0;
-    pd.kt_per_split = ds.per;
-    pd.red = tacc;
-    pd.ldo = r;
-    pd.status = status;
-    if ((s = launch_bn(bnd, tX, tA, tX, tA, pd, dim3(1, m_tiles, ds.splits), stream)) != UNO_OK) return s;
-
-    // ---- 2. gate: T = bf16(scale * g * sum of the partials) ----
-    {
-        const int64_t n4 = (int64_t)M * r / 4;
-        const int blocks = (int)((n4 + 255) / 256 < 1184 ? (n4 + 255) / 256 : 1184);
-        gate_kernel<<<blocks, 256, 0, stream>>>(tacc, ds.splits, g.gate, g.scale, M, r, t);
-        if ((s = check_cuda(cudaGetLastError(), "launch(gate)")) != UNO_OK) return s;
+    __nv_bfloat16* t = reinterpret_cast<__nv_bfloat16*>(ws + P.t);
+    CUtensorMap maps[5];
+    const int cg = P.CG;
+    if ((s = make_tmap(&maps[0], x, M, din, BM)) != UNO_OK) return s;              // X
+    if ((s = make_tmap(&maps[1], w0, dout, din, P.BN / cg)) != UNO_OK) return s;   // W0
+    if ((s = make_tmap(&maps[2], a, r, din, P.rb / cg)) != UNO_OK) return s;       // A
+    if ((s = make_tmap(&maps[3], t, M, r, BM)) != UNO_OK) return s;                // T
+    if ((s = make_tmap(&maps[4], b, dout, r, P.BN / cg)) != UNO_OK) return s;      // B
+    Params p{};
+    p.M = M;
+    p.N = dout;
+    p.r = r;
+    p.kt0 = P.kt0;
+    p.kt1 = P.kt1;
+    p.m_tiles = P.m_tiles;
+    p.m_units = P.m_units;
+    p.splits = P.splits;
+    p.per = P.per;
+    p.n_adapter = P.n_adapter;
+    p.n_items = P.n_items;
+    p.rb = P.rb;
+    p.stages = P.stages;
+    p.b_bytes = P.b_bytes;
+    p.cb = (uint32_t)P.cb;
+    p.y = g.y;
+    p.out_f32 = g.dtype == UNO_F32;
+    p.tpart = P.splits > 1 ? reinterpret_cast<float*>(ws + P.tpart) : nullptr;
+    p.t = t;
+    p.gate = g.gate;
+    p.scale = g.scale;
+    p.flags = reinterpret_cast<unsigned long long*>(ws + P.flags);
+    p.tickets = reinterpret_cast<unsigned long long*>(ws + P.tickets);
+    p.epoch = next_epoch();
+    p.status = device_status_ptr();
+    if (P.CG == 2) return launch_t<256, 2>(maps, p, P, stream);
+    switch (P.BN) {
+        case 64: return launch_t<64, 1>(maps, p, P, stream);
+        case 128: return launch_t<128, 1>(maps, p, P, stream);
+        case 256: return launch_t<256, 1>(maps, p, P, stream);
     }
-
-    // ---- 3. main: Y = [X | T] [W0 | B]^T ----
-    int BN = 256;
-    while (BN > 64 && (int64_t)m_tiles * ((dout + BN - 1) / BN) < 120) BN >>= 1;
-    if ((s = make_tmap(&tW0, w0, dout, din, BN)) != UNO_OK) return s;
-    if ((s = make_tmap(&tT, t, M, r, BM)) != UNO_OK) return s;
-    if ((s = make_tmap(&tBl, b, dout, r, BN)) != UNO_OK) return s;
-    Params pm{};
-    pm.M = M;
-    pm.N = dout;
-    pm.kt0 = kt0;
-    pm.kt1 = (r + BK - 1) / BK;
-    pm.kt_per_split = 0;
-    pm.out = g.y;
-    pm.ldo = dout;
-    pm.out_f32 = g.dtype == UNO_F32;
-    pm.red = nullptr;
-    pm.status = status;
-    return launch_bn(BN, tX, tW0, tT, tBl, pm, dim3((dout + BN - 1) / BN, m_tiles, 1), stream);
+    return set_error(UNO_ERR_UNSUPPORTED, "tile width %d", P.BN);
 }
 
 }  // namespace uno

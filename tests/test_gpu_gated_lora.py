@@ -89,3 +89,55 @@ def test_full_shapes_sampled_rows(wl, name):
     ref = _ref(inp, rows)
     assert _rel(y[rows], ref) <= TOL
     assert np.isfinite(y).all()
+
+
+def test_calls_back_to_back_on_one_workspace():
+    """Two calls with different gates on the same workspace: the second call's output
+    tiles must use its own adapter rows, not the ones the first call left behind."""
+    M, d_in, d_out, r = 512, 1024, 1024, 64
+    w = W.GatedLoraWorkload("t", 93, M=M, block=8, rank=r, scale=2.0, shapes=(W.LinearShape("t", d_in, d_out),))
+    inp = W.linear_inputs(w, w.shapes[0])
+    import torch
+    from diffusion_drafted_lossless_b200 import _lib
+    dv = {k: torch.from_numpy(inp[k].view(np.int16)).view(torch.bfloat16).cuda() for k in ("x", "w0", "a", "b")}
+    ws = torch.empty(_lib.uno_gated_lora_linear_workspace_size(M, d_in, d_out, r), dtype=torch.uint8, device="cuda")
+    outs = []
+    gates = [inp["gate"], (1.0 - inp["gate"]).astype(np.float32)]
+    for gt in gates:
+        y = torch.empty((M, d_out), dtype=torch.bfloat16, device="cuda")
+        _lib.uno_gated_lora_linear(dv["x"], dv["w0"], dv["a"], dv["b"], torch.from_numpy(gt).cuda(), 2.0, y,
+                                   workspace=ws)
+        outs.append(y)
+    torch.cuda.synchronize()
+    for y, gt in zip(outs, gates):
+        ref = _ref(dict(inp, gate=gt))
+        assert _rel(y.float().cpu().numpy(), ref) <= TOL
+
+
+@pytest.mark.parametrize("splits", ["3", "64"])
+def test_split_adapter_path(monkeypatch, splits):
+    """The adapter product split over K (partials summed by the item that completes a row
+    tile) gives the same result; 64 splits exceed the K tiles and are clamped."""
+    monkeypatch.setenv("UNO_LORA_SPLITS", splits)
+    for M, d_in, d_out, r in [(300, 1024, 256, 64), (1000, 768, 1024, 256), (129, 256, 640, 128)]:
+        w = W.GatedLoraWorkload("t", 5 + M, M=M, block=8, rank=r, scale=2.0,
+                                shapes=(W.LinearShape("t", d_in, d_out),))
+        inp = W.linear_inputs(w, w.shapes[0])
+        y = _run(inp, M, d_in, d_out, r)
+        assert _rel(y, _ref(inp)) <= TOL
+
+
+@pytest.mark.parametrize("env", [{"UNO_LORA_CG": "2"}, {"UNO_LORA_CG": "2", "UNO_LORA_SPLITS": "3"},
+                                 {"UNO_LORA_CG": "1"}])
+def test_cta_pair_and_single_forms(monkeypatch, env):
+    """The CTA-pair form (256-row tiles, one MMA stream over two SMs) and the single-CTA
+    form give the oracle's result on ragged shapes (M not a multiple of 256, rank 8/24/256)."""
+    for k, v in env.items():
+        monkeypatch.setenv(k, v)
+    for M, d_in, d_out, r in [(300, 1024, 512, 64), (1000, 768, 1024, 256), (257, 256, 768, 8),
+                              (512, 512, 256, 24), (1024, 4096, 4096, 128)]:
+        w = W.GatedLoraWorkload("t", 11 + M + r, M=M, block=8, rank=r, scale=2.0,
+                                shapes=(W.LinearShape("t", d_in, d_out),))
+        inp = W.linear_inputs(w, w.shapes[0])
+        y = _run(inp, M, d_in, d_out, r)
+        assert _rel(y, _ref(inp)) <= TOL, (M, d_in, d_out, r)
