@@ -271,11 +271,11 @@ constexpr float kLog2e = 1.4426950408889634f;
 // Shared memory: a header of mbarriers and reduction slots, two input buffers of
 // (teacher, student) bf16 row slices, and exp(student) of the current row in fp32.
 //   mbarriers: full[2] (an input buffer has landed), empty[2] (every compute warp is done
-//   with an input buffer), red[3] (every warp of the cluster has sent its partial of
-//   reduction 0 / 1 / 2); then three arrays of per-warp partials, [ncta][kWarps] float2 each.
-constexpr int kReductions = 3;
+//   with an input buffer), red[2] (every warp of the cluster has sent its partial of
+//   reduction 0 / 1); then the per-warp partials, [ncta][kWarps] float4 (reduction 0:
+//   max and sum of exp for both rows) and [ncta][kWarps] float2 (reduction 1).
 __host__ __device__ inline size_t header_bytes(int ncta) {
-    return ((size_t)64 + (size_t)kReductions * ncta * kWarps * 8 + 127) / 128 * 128;
+    return ((size_t)64 + (size_t)ncta * kWarps * (16 + 8) + 127) / 128 * 128;
 }
 // Elements of a row slice: a multiple of 8 (16-byte bulk copies and 8-element units).
 inline int64_t slice_elems(int64_t V, int cl) { return ((V + cl - 1) / cl + 7) / 8 * 8; }
@@ -310,7 +310,13 @@ __device__ __forceinline__ uint32_t map_rank(const void* local, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
     return remote;
 }
-// 8-byte store into another CTA's shared memory, counted in bytes on that CTA's mbarrier
+// stores into another CTA's shared memory, counted in bytes on that CTA's mbarrier
+__device__ __forceinline__ void st_async_v4(uint32_t dst, uint32_t bar, float a, float b, float c, float d) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                     dst),
+                 "f"(a), "f"(b), "f"(c), "f"(d), "r"(bar)
+                 : "memory");
+}
 __device__ __forceinline__ void st_async_v2(uint32_t dst, uint32_t bar, float a, float b) {
     asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(dst),
                  "f"(a), "f"(b), "r"(bar)
@@ -373,8 +379,9 @@ __global__ void __launch_bounds__(kThreads, 1) cluster_kernel(Params p, int64_t 
     const uint32_t rank = cluster_rank(), ncta = cluster_size();
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + 2;
-    uint64_t* red = full + 4;  // [kReductions]
-    float2* slots = reinterpret_cast<float2*>(smem + 64);  // [kReductions][ncta][kWarps]
+    uint64_t* red = full + 4;  // [2]
+    float4* slots0 = reinterpret_cast<float4*>(smem + 64);                              // [ncta][kWarps]
+    float2* slots1 = reinterpret_cast<float2*>(smem + 64 + (size_t)ncta * kWarps * 16);  // [ncta][kWarps]
     const size_t hdr = header_bytes((int)ncta);
     uint16_t* inbuf = reinterpret_cast<uint16_t*>(smem + hdr);  // [2][teacher, student][n]
     float* es = reinterpret_cast<float*>(smem + hdr + (size_t)n * 8);
@@ -384,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1) cluster_kernel(Params p, int64_t 
     const int cnt = (int)max((int64_t)0, min(n, V - lo));  // elements of this CTA's slice
     const uint32_t bytes = (uint32_t)cnt * 2u;
     const int units = cnt / 8;
-    const uint32_t red_bytes = ncta * kWarps * 8u;
+    const uint32_t red0_bytes = ncta * kWarps * 16u, red1_bytes = ncta * kWarps * 8u;
     const __nv_bfloat16* T = reinterpret_cast<const __nv_bfloat16*>(a.teacher);
     const __nv_bfloat16* S = reinterpret_cast<const __nv_bfloat16*>(a.student);
     __nv_bfloat16* G = reinterpret_cast<__nv_bfloat16*>(a.grad);
@@ -400,24 +407,47 @@ __global__ void __launch_bounds__(kThreads, 1) cluster_kernel(Params p, int64_t 
     };
 
     bool more_rows = false;  // the current row is not this cluster's last
-    // Cluster-wide reduction i of this row's per-warp float2 partials (every lane of the
-    // warp passes the same value): each warp stores it into slot [rank][warp] of every CTA
-    // of the cluster; once all have landed, every warp combines them (max or sum).
-    auto reduce = [&](float2 part, int i, uint32_t parity, bool is_max) -> float2 {
-        float2* slot = slots + (size_t)i * ncta * kWarps;
+    // Cluster-wide reductions of this row's per-warp partials (every lane of the warp
+    // passes the same value): each warp stores its partial into slot [rank][warp] of every
+    // CTA of the cluster; once all have landed, every warp combines them. The next row's
+    // phase of a reduction is armed before this CTA sends anything that lets another CTA
+    // reach it.
+    // 0: (max t, sum exp(t - max t), max s, sum exp(s - max s)) -> row maxima and sums
+    auto reduce0 = [&](float4 part, uint32_t parity) -> float4 {
         if ((uint32_t)lane < ncta)
-            st_async_v2(map_rank(&slot[rank * kWarps + warp], lane), map_rank(&red[i], lane), part.x, part.y);
-        wait(&red[i], parity);
-        float x = is_max ? -INFINITY : 0.f, y = x;
+            st_async_v4(map_rank(&slots0[rank * kWarps + warp], lane), map_rank(&red[0], lane), part.x, part.y,
+                        part.z, part.w);
+        wait(&red[0], parity);
+        float Mt = -INFINITY, Ms = -INFINITY;
         for (uint32_t j = lane; j < ncta * kWarps; j += 32) {
-            const float2 w = slot[j];
-            x = is_max ? fmaxf(x, w.x) : x + w.x;
-            y = is_max ? fmaxf(y, w.y) : y + w.y;
+            const float4 w = slots0[j];
+            Mt = fmaxf(Mt, w.x);
+            Ms = fmaxf(Ms, w.z);
         }
-        // the next row's phase of this reduction is armed before this CTA sends anything
-        // that lets another CTA reach it
-        if (tid == 0 && more_rows) mbar_arrive_expect_tx(&red[i], red_bytes);
-        return is_max ? make_float2(warp_max(x), warp_max(y)) : make_float2(warp_sum(x), warp_sum(y));
+        Mt = warp_max(Mt);
+        Ms = warp_max(Ms);
+        float Zt = 0.f, Zs = 0.f;
+        for (uint32_t j = lane; j < ncta * kWarps; j += 32) {
+            const float4 w = slots0[j];
+            if (w.y > 0.f) Zt += w.y * ex2((w.x - Mt) * kLog2e);
+            if (w.w > 0.f) Zs += w.w * ex2((w.z - Ms) * kLog2e);
+        }
+        if (tid == 0 && more_rows) mbar_arrive_expect_tx(&red[0], red0_bytes);
+        return make_float4(Mt, warp_sum(Zt), Ms, warp_sum(Zs));
+    };
+    // 1: (A, P) sums
+    auto reduce1 = [&](float2 part, uint32_t parity) -> float2 {
+        if ((uint32_t)lane < ncta)
+            st_async_v2(map_rank(&slots1[rank * kWarps + warp], lane), map_rank(&red[1], lane), part.x, part.y);
+        wait(&red[1], parity);
+        float x = 0.f, y = 0.f;
+        for (uint32_t j = lane; j < ncta * kWarps; j += 32) {
+            const float2 w = slots1[j];
+            x += w.x;
+            y += w.y;
+        }
+        if (tid == 0 && more_rows) mbar_arrive_expect_tx(&red[1], red1_bytes);
+        return make_float2(warp_sum(x), warp_sum(y));
     };
 
     if (tid == 0) {
@@ -425,11 +455,14 @@ __global__ void __launch_bounds__(kThreads, 1) cluster_kernel(Params p, int64_t 
         mbar_init(&full[1], 1);
         mbar_init(&empty[0], kWarps);
         mbar_init(&empty[1], kWarps);
-        for (int i = 0; i < kReductions; ++i) mbar_init(&red[i], 1);
+        mbar_init(&red[0], 1);
+        mbar_init(&red[1], 1);
         fence_mbar_init();
         // armed one row ahead, so that no partial can arrive before its phase is armed
-        if (first < N)
-            for (int i = 0; i < kReductions; ++i) mbar_arrive_expect_tx(&red[i], red_bytes);
+        if (first < N) {
+            mbar_arrive_expect_tx(&red[0], red0_bytes);
+            mbar_arrive_expect_tx(&red[1], red1_bytes);
+        }
     }
     // every CTA's mbarriers are initialised and armed before any CTA sends to them
     cluster_sync();
@@ -480,7 +513,7 @@ __global__ void __launch_bounds__(kThreads, 1) cluster_kernel(Params p, int64_t 
             const uint16_t* tin = inbuf + (size_t)b * 2 * n;
             const uint16_t* sin = tin + n;
 
-            // ---- row maxima over the cluster ----
+            // ---- this warp's maxima (exps are taken relative to them) ----
             __nv_bfloat162 mt2 = __floats2bfloat162_rn(-INFINITY, -INFINITY), ms2 = mt2;
             for (int u = tid; u < units; u += kWarps * 32) {
                 const uint4 wt = lds128(tin + u * 8), ws = lds128(sin + u * 8);
@@ -491,14 +524,13 @@ __global__ void __launch_bounds__(kThreads, 1) cluster_kernel(Params p, int64_t 
                     ms2 = __hmax2(ms2, *reinterpret_cast<const __nv_bfloat162*>(&as4[j]));
                 }
             }
-            float2 v = make_float2(warp_max(fmaxf(__low2float(mt2), __high2float(mt2))),
-                                   warp_max(fmaxf(__low2float(ms2), __high2float(ms2))));
-            v = reduce(v, 0, par, true);
-            const float Mt = v.x, Ms = v.y;
-            const float lt = Mt * kLog2e, ls = Ms * kLog2e;
+            const float mt = warp_max(fmaxf(__low2float(mt2), __high2float(mt2)));
+            const float ms = warp_max(fmaxf(__low2float(ms2), __high2float(ms2)));
+            // a warp with no elements uses 0 (its sums are 0 and it never reads its factors)
+            const float lt = (mt == -INFINITY ? 0.f : mt) * kLog2e, ls = (ms == -INFINITY ? 0.f : ms) * kLog2e;
             const f2 L2E = pk(kLog2e, kLog2e), NLT = pk(-lt, -lt), NLS = pk(-ls, -ls);
 
-            // ---- sums of exp(x - max); exp(s - Ms) kept ----
+            // ---- sums of exp(x - warp max); exp(s - warp max) kept ----
             f2 zt2 = pk(0.f, 0.f), zs2 = zt2;
             for (int u = tid; u < units; u += kWarps * 32) {
                 const uint4 wt = lds128(tin + u * 8), ws = lds128(sin + u * 8);
@@ -515,14 +547,16 @@ __global__ void __launch_bounds__(kThreads, 1) cluster_kernel(Params p, int64_t 
                 *reinterpret_cast<float4*>(es + u * 4) = make_float4(e[0], e[1], e[2], e[3]);
                 *reinterpret_cast<float4*>(es + half + u * 4) = make_float4(e[4], e[5], e[6], e[7]);
             }
-            v = reduce(make_float2(warp_sum(lo_of(zt2) + hi_of(zt2)), warp_sum(lo_of(zs2) + hi_of(zs2))), 1, par,
-                       false);
-            const float Zt = v.x, Zs = v.y;
-            // p = exp(t - Mt) / Zt, q = kept exp(s - Ms) / Zs. q > p is decided in the log
-            // domain, exact up to the rounding of one threshold:
+            const float4 st = reduce0(make_float4(mt, warp_sum(lo_of(zt2) + hi_of(zt2)), ms,
+                                                  warp_sum(lo_of(zs2) + hi_of(zs2))), par);
+            const float Mt = st.x, Zt = st.y, Ms = st.z, Zs = st.w;
+            // p = exp(t - wmt) * at, q = kept exp(s - wms) * as: this warp's maxima folded
+            // into at, as (the same arithmetic for both rows: identical rows give p == q).
+            // q > p is decided in the log domain, exact up to the rounding of one threshold:
             //   q > p  <=>  s - t > K = (Ms + ln Zs) - (Mt + ln Zt)
             // (Ms - Mt is exact; Zs / Zt is near 1 in practice, so its log is accurate to ~1e-7)
-            const float at = 1.f / Zt, as = 1.f / Zs;
+            const float at = mt == -INFINITY ? 0.f : ex2(lt - Mt * kLog2e) / Zt;
+            const float as = ms == -INFINITY ? 0.f : ex2(ls - Ms * kLog2e) / Zs;
             const float K = (Ms - Mt) + logf(Zs / Zt);
 
             // ---- A = sum of q over q > p, P = sum of p over q > p ----
@@ -549,8 +583,8 @@ __global__ void __launch_bounds__(kThreads, 1) cluster_kernel(Params p, int64_t 
                     }
                 }
             }
-            v = reduce(make_float2(warp_sum(Araw * as), warp_sum(Praw * at)), 2, par, false);
-            const float Af = v.x, Pf = v.y;
+            const float2 ap = reduce1(make_float2(warp_sum(Araw * as), warp_sum(Praw * at)), par);
+            const float Af = ap.x, Pf = ap.y;
             const bool on = a.mask == nullptr || a.mask[r] != 0;
 
             // ---- gradient: f q (s - c) = f q (1 - A) where q > p, -f q A elsewhere ----
