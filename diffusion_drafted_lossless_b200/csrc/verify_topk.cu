@@ -201,6 +201,74 @@ __device__ __noinline__ void warp_append(const uint4 v, int nvalid, uint32_t id0
     if (ws->count > CAP - 32 * VEC) warp_shrink<KeyBits<T>::value>(buf, hist, ws, bound, k, lane);
 }
 
+// One chunk of the bulk loop: lanes whose part of the chunk passes the bounds append
+// their candidates (every lane of the warp calls it; the buffer is cut first when it may
+// not have room for the whole chunk).
+template <int CAP>
+__device__ __forceinline__ void handle_chunk(const uint4 v, uint32_t id0, uint64_t* buf, uint32_t* hist, WarpSlot* ws,
+                                             uint32_t* bound, const float* guess, int k, int lane,
+                                             __nv_bfloat162& lo, __nv_bfloat162& th) {
+    using Ops = LaneOps<__nv_bfloat16>;
+    bool h = Ops::hit(v, lo, th);
+    if (!__any_sync(kFullMask, h)) return;
+    if (ws->count > CAP - 256) {  // room for a whole chunk (uniform)
+        warp_shrink<16>(buf, hist, ws, bound, k, lane);
+        lo = Ops::thr(fmaxf(*guess, key_float(*reinterpret_cast<volatile uint32_t*>(bound))));
+        th = Ops::thr(ws->have_k ? ws->thr : -INFINITY);
+        h = Ops::hit(v, lo, th);
+    }
+    if (h) lane_append<__nv_bfloat16>(v, 8, id0, lo, th, buf, ws);
+    __syncwarp();
+}
+
+// The bulk of a warp's run over an aligned bf16 row: full chunks [cb, cf) (at least two
+// groups of kUnroll), 16-byte loads two groups ahead, one test of each lane's maximum per
+// group, lane-local appends for the rare lanes that hold a candidate. The thresholds are
+// kept in registers and refreshed after appends (a stale, lower threshold only admits
+// more candidates). Returns the first chunk not processed.
+template <int CAP>
+__device__ __noinline__ int stream_full_bf16(const uint4* lp, int cb, int cf, uint64_t* buf, uint32_t* hist,
+                                             WarpSlot* ws, uint32_t* bound, const float* guess, int k, int lane) {
+    using Ops = LaneOps<__nv_bfloat16>;
+    constexpr int CH = 256;  // elements per warp chunk
+    const volatile uint32_t* vb = bound;
+    __nv_bfloat162 lo = Ops::thr(fmaxf(*guess, key_float(*vb))), th = Ops::thr(ws->have_k ? ws->thr : -INFINITY);
+    uint4 a0 = ld_stream_v4(lp), a1 = ld_stream_v4(lp + 32), a2 = ld_stream_v4(lp + 64), a3 = ld_stream_v4(lp + 96);
+    for (; cb + kUnroll <= cf; cb += kUnroll) {
+        const bool more = cb + 2 * kUnroll <= cf;
+        uint4 b0, b1, b2, b3;
+        if (more) {
+            b0 = ld_stream_v4(lp + 128);
+            b1 = ld_stream_v4(lp + 160);
+            b2 = ld_stream_v4(lp + 192);
+            b3 = ld_stream_v4(lp + 224);
+        }
+        const __nv_bfloat162 m01 = __hmax2(__hmax2(__hmax2(Ops::w2(a0.x), Ops::w2(a0.y)), __hmax2(Ops::w2(a0.z), Ops::w2(a0.w))),
+                                           __hmax2(__hmax2(Ops::w2(a1.x), Ops::w2(a1.y)), __hmax2(Ops::w2(a1.z), Ops::w2(a1.w))));
+        const __nv_bfloat162 m23 = __hmax2(__hmax2(__hmax2(Ops::w2(a2.x), Ops::w2(a2.y)), __hmax2(Ops::w2(a2.z), Ops::w2(a2.w))),
+                                           __hmax2(__hmax2(Ops::w2(a3.x), Ops::w2(a3.y)), __hmax2(Ops::w2(a3.z), Ops::w2(a3.w))));
+        const __nv_bfloat162 mall = __hmax2(m01, m23);
+        if (__any_sync(kFullMask, (__hge2_mask(mall, lo) & __hgt2_mask(mall, th)) != 0u)) {
+            handle_chunk<CAP>(a0, (uint32_t)(cb * CH + lane * 8), buf, hist, ws, bound, guess, k, lane, lo, th);
+            handle_chunk<CAP>(a1, (uint32_t)((cb + 1) * CH + lane * 8), buf, hist, ws, bound, guess, k, lane, lo, th);
+            handle_chunk<CAP>(a2, (uint32_t)((cb + 2) * CH + lane * 8), buf, hist, ws, bound, guess, k, lane, lo, th);
+            handle_chunk<CAP>(a3, (uint32_t)((cb + 3) * CH + lane * 8), buf, hist, ws, bound, guess, k, lane, lo, th);
+            // another warp's cut may have raised the shared bound
+            lo = Ops::thr(fmaxf(*guess, key_float(*vb)));
+        }
+        if (!more) {
+            cb += kUnroll;
+            break;
+        }
+        a0 = b0;
+        a1 = b1;
+        a2 = b2;
+        a3 = b3;
+        lp += 128;
+    }
+    return cb;
+}
+
 // ---------------------------------------------------------------------------------------
 // Kernel 1: stream the logit rows once. Every warp walks its own contiguous run of chunks
 // in token-id order and keeps the run's exact top-k (ties to the lower id). Warps share
@@ -212,7 +280,7 @@ __device__ __noinline__ void warp_append(const uint4 v, int nvalid, uint32_t id0
 //     are appended only when strictly above its k-th value.
 // ---------------------------------------------------------------------------------------
 template <typename T, int KCAP>
-__global__ void __launch_bounds__(kStreamWarps * 32)
+__global__ void __launch_bounds__(kStreamWarps * 32, 3)
 stream_kernel(Params p) {
     using Ops = LaneOps<T>;
     constexpr int VEC = Elem<T>::VEC;
@@ -331,7 +399,14 @@ stream_kernel(Params p) {
     offer(c0);
 
     // ---- stream the rest of the warp's run ----
-    for (int cb = c0 + kUnroll; cb < c1; cb += kUnroll) {
+    int cb = c0 + kUnroll;
+    if constexpr (VEC == 8) {
+        const int cf = max(cb, min(c1, full_chunks));
+        if (cb + 2 * kUnroll <= cf)
+            cb = stream_full_bf16<CAP>(reinterpret_cast<const uint4*>(row) + (int64_t)cb * 32 + lane, cb, cf, buf,
+                                       hist, ws, &s_bound, &s_guess, k, lane);
+    }
+    for (; cb < c1; cb += kUnroll) {
         load(cb);
         offer(cb);
     }
