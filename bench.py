@@ -260,6 +260,23 @@ def oracle_sample(n_seq=2):
 
 
 # ---------------------------------------------------------------------------------------
+def reduce_max(x, dist, device):
+    """The maximum of x over all ranks (x itself without a process group): every rank's
+    time is the slowest rank's, as the job finishes when the last replica does."""
+    if dist is None:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(rows_per_rank, world, ms_per_step):
+    """Rows per second of the whole job: every rank runs its own replica of the step (weak
+    scaling), and the step time is the maximum over ranks."""
+    return world * rows_per_rank / (ms_per_step * 1e-3)
+
+
 def run_uno(args):
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -281,11 +298,7 @@ def run_uno(args):
         torch.cuda.synchronize()
 
     def max_over_ranks(x):
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, dist, dev)
 
     for _ in range(args.warmup):
         st.run()
@@ -329,7 +342,7 @@ def run_uno(args):
 
     v, pk = VERIFY, peaks()
     rows = v.B * v.K
-    value = world * rows / (ms * 1e-3)
+    value = whole_job_rate(rows, world, ms)
     gemm_fl = sum(gemm_flops(L["shape"], LINEARS.M, LINEARS.rank, st.n_gated) for L in st.lin)
     # the dominant kernel: the TV kernel is one launch per step (plus a 1-block mask count);
     # the linears are 7 launches (one per projection), the verify 3
