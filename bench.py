@@ -260,6 +260,98 @@ def oracle_sample(n_seq=2):
 
 
 # ---------------------------------------------------------------------------------------
+def measure_configs(torch, dev, lib, pk, reduce):
+    """The other single-GPU configurations of the path, each timed with CUDA events after
+    warm-up (inputs resident in HBM, larger than L2): the looped 3B-class step (7 gated
+    projections x 22 layers x 2 loops at M = 2048, then the verify at B = 256, K = 8,
+    V = 166144, top-p 0.95) and the TV loss at 16384 x 151936. Inputs are drawn on the
+    device from a seeded generator with the configurations' distributions."""
+    gen = torch.Generator(device=dev)
+    bf = torch.bfloat16
+
+    def normal(shape, sigma, seed):
+        gen.manual_seed(seed)
+        t = torch.randn(shape, generator=gen, device=dev, dtype=torch.float32)
+        return (t * sigma).to(bf)
+
+    def timed(fn, reps):
+        fn()
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(reps):
+            fn()
+        e.record()
+        torch.cuda.synchronize()
+        return reduce(s.elapsed_time(e) / reps)
+
+    out = {}
+    # ---- looped 3B-class step: 7 projections x 22 layers x 2 loops, shared across loops ----
+    w = W.LOOPED_3B
+    M = w.M
+    gate = torch.from_numpy(W.row_gate(M, w.block)).to(dev)
+    n_gated = int((gate > 0).sum().item())
+    xs = {d: normal((M, d), w.x_sigma, 7000 + d) for d in sorted({sh.d_in for sh in w.shapes})}
+    layers = []
+    for l in range(W.LOOPED_3B_LAYERS):
+        lw = []
+        for i, sh in enumerate(w.shapes):
+            seed = 8000 + 10 * l + i
+            lw.append((sh, normal((sh.d_out, sh.d_in), w.w_sigma, seed), normal((w.rank, sh.d_in), w.w_sigma, seed + 3000),
+                       normal((sh.d_out, w.rank), w.w_sigma, seed + 6000)))
+        layers.append(lw)
+    ys = {sh.name: torch.empty((M, sh.d_out), dtype=bf, device=dev) for sh in w.shapes}
+    wss = {sh.name: torch.empty(lib.uno_gated_lora_linear_workspace_size(M, sh.d_in, sh.d_out, w.rank),
+                                dtype=torch.uint8, device=dev) for sh in w.shapes}
+
+    def looped():
+        for _ in range(W.LOOPED_3B_LOOPS):
+            for lw in layers:
+                for sh, w0, a, b in lw:
+                    lib.uno_gated_lora_linear(xs[sh.d_in], w0, a, b, gate, w.scale, ys[sh.name], workspace=wss[sh.name])
+
+    ms = timed(looped, 3)
+    fl = W.LOOPED_3B_LAYERS * W.LOOPED_3B_LOOPS * sum(gemm_flops(sh, M, w.rank, n_gated) for sh in w.shapes)
+    out["looped_3b_linears_m2048_x44"] = {"ms": ms, "tflops": fl / (ms * 1e-3) / 1e12,
+                                          "frac": fl / (ms * 1e-3) / 1e12 / pk["bf16_tflops_sustained"],
+                                          "peak": "bf16_tflops_sustained (a seconds-long loop)",
+                                          "launches": 7 * W.LOOPED_3B_LAYERS * W.LOOPED_3B_LOOPS}
+    del layers, xs, ys, wss
+    v = W.LOOPED_VERIFY
+    P = normal((v.B, v.K, v.V), v.sigma, 9001)
+    Q = (v.rho * P.float() + (1 - v.rho ** 2) ** 0.5 * normal((v.B, v.K, v.V), v.sigma, 9002).float()).to(bf)
+    gen.manual_seed(9003)
+    u = torch.rand((v.B, v.K, 3), generator=gen, device=dev, dtype=torch.float32)
+    tok = torch.empty((v.B, v.K), dtype=torch.int32, device=dev)
+    cnt = torch.empty((v.B,), dtype=torch.int32, device=dev)
+    nxt = torch.empty((v.B,), dtype=torch.int32, device=dev)
+    vws = torch.empty(lib.uno_block_verify_workspace_size(v.B, v.K, v.V, v.top_k, v.top_p), dtype=torch.uint8,
+                      device=dev)
+    ms = timed(lambda: lib.uno_block_verify(P, Q, v.temperature, v.top_k, v.top_p, u, tok, cnt, nxt, workspace=vws), 5)
+    vb = verify_bytes(v)
+    out["looped_3b_verify_b256_k8_v166144"] = {"ms": ms, "gbs": vb / (ms * 1e-3) / 1e9,
+                                               "frac": vb / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                                               "rows_per_s": v.B * v.K / (ms * 1e-3),
+                                               "mean_tokens_per_step": float(cnt.float().mean().item())}
+    del P, Q, u, vws
+    # ---- TV loss at 8 x 2048 response tokens ----
+    t = W.TV_LOSS
+    T_ = normal((t.N, t.V), t.teacher_sigma, 9101)
+    S_ = torch.empty_like(T_)
+    for i in range(0, t.N, 2048):  # student = teacher + N(0, 1), in slices to bound the fp32 temporaries
+        S_[i:i + 2048] = (T_[i:i + 2048].float() + normal((min(2048, t.N - i), t.V), t.noise_sigma, 9102 + i).float()).to(bf)
+    tv = torch.empty((t.N,), device=dev)
+    mean = torch.empty((1,), device=dev)
+    grad = torch.empty((t.N, t.V), dtype=bf, device=dev)
+    tws = torch.empty(lib.uno_tv_loss_workspace_size(t.N, t.V), dtype=torch.uint8, device=dev)
+    ms = timed(lambda: lib.uno_tv_loss(T_, S_, tv, mean, grad, workspace=tws), 3)
+    tb = tv_bytes(t.N, t.V)
+    out["tv_loss_n16384_v151936"] = {"ms": ms, "gbs": tb / (ms * 1e-3) / 1e9, "frac": tb / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
+    del T_, S_, grad
+    torch.cuda.empty_cache()
+    return out
+
+
 def reduce_max(x, dist, device):
     """The maximum of x over all ranks (x itself without a process group): every rank's
     time is the slowest rank's, as the job finishes when the last replica does."""
@@ -341,6 +433,7 @@ def run_uno(args):
     e2e_ms = max_over_ranks(s.elapsed_time(e) / with_e2e)
 
     v, pk = VERIFY, peaks()
+    configs = None if args.no_configs else measure_configs(torch, dev, st.lib, pk, max_over_ranks)
     rows = v.B * v.K
     value = whole_job_rate(rows, world, ms)
     gemm_fl = sum(gemm_flops(L["shape"], LINEARS.M, LINEARS.rank, st.n_gated) for L in st.lin)
@@ -385,7 +478,7 @@ def run_uno(args):
                        "verify": "T=1, top-k 50, top-p 0.95, drafts sampled in-kernel",
                        "tv": "1024 rows x 151936, teacher=verifier, student=drafter logits",
                        "l2": "no flush: every input (logits 622 MB, weights 380 MB) exceeds L2 or is read once"},
-            "roofline": roof, "phases": phases, "cpu_baseline": cpu,
+            "roofline": roof, "phases": phases, "configs": configs, "cpu_baseline": cpu,
             "e2e": {"value": world * rows / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": st.h2d,
                     "d2h_bytes_per_step": st.d2h, "ms_per_step": e2e_ms},
             "gpu_launches": LAUNCHES_PER_STEP * args.steps, "clocks": clocks,
@@ -424,6 +517,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["uno", "reference"], default="uno")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--no-configs", action="store_true", help="skip the other configurations' measurements")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "uno":
         args.warmup = 3

@@ -6,8 +6,8 @@
 // the unfiltered and the top-p-only sampler settings (the LoopUno runs use temperature 1.0
 // and top-p 0.95 without top-k).
 //
-// One CTA per sequence. For each of its rows (verifier rows 0..K-1, drafter rows
-// 1..K-1) the CTA
+// Two launches. rows_kernel: one CTA per row (verifier rows 0..K-1 and drafter rows 1..K-1
+// of every sequence), which
 //   1. streams the row once and keeps, per chunk of CH elements, the maximum and the sum
 //      of exp(z - max) (z = logit / T); from them the row's max M and sum S;
 //   2. with top-p: finds the exact cut by radix histograms of the probability mass over
@@ -16,6 +16,8 @@
 //      gives the cut value tau, the mass above it and how many of the tokens equal to tau
 //      are kept (the lowest ids: ties are ordered by id);
 //   3. stores per chunk the surviving mass and the number of tokens equal to tau.
+// seq_kernel: one CTA per sequence, one warp per block position for the draws, the
+// probabilities and the acceptance, then the whole CTA for the residual and the TV.
 // Draws (inverse CDF over ascending ids) walk the chunk table and then scan one chunk in
 // id order; probabilities of single tokens need the token's rank among the tau-ties, from
 // the table and a scan of its chunk. The correction token's residual max(0, p - q) and the
@@ -98,7 +100,6 @@ __device__ __forceinline__ float cta_max_f32(float v, float* red) {
 template <typename T>
 __device__ void prepare_row(const T* row, const VerifyArgs& a, int nchunks, double* cmass, int* cties, RowInfo* info,
                             float* hist_f, uint32_t* hist_n, double* dred, float* fred) {
-    constexpr int VEC = Elem<T>::VEC;
     constexpr int NLEVELS = sizeof(T) == 2 ? 2 : 4;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int V = a.V;
@@ -147,10 +148,71 @@ __device__ void prepare_row(const T* row, const VerifyArgs& a, int nchunks, doub
     if (a.top_p < 1.0f) {
         // 2. exact top-p cut by radix histograms of the mass over the logit keys
         const double target = (double)a.top_p * S;
+        // level A: mass by distance below the max, 1/8-nat bins (the radix levels below,
+        // restricted to the crossing bin, then fix the exact cut). Binning by value spreads
+        // the elements over many bins, where the first radix level over the key's top bits
+        // would put most of them in a few.
+        auto vbin = [&](float x) {
+            const float d = M - x * invT;
+            return d < 31.875f ? (int)(d * 8.f) : 255;
+        };
+        // Only elements within D nats of the max are binned: those further down weigh at
+        // most V e^-D together, which is below the mass top-p leaves out when
+        // D >= ln(V / ((1 - top_p) S)), so the cut lies within D (a full pass is the
+        // fallback for rounding).
+        // (D is a whole number of bins, so that a bin is either binned in full or not at all)
+        const double dcut = log((double)V / ((1.0 - (double)a.top_p) * S)) + 0.5;
+        float D = dcut > 31.875 ? 31.875f : (dcut < 0.125 ? 0.125f : ceilf((float)dcut * 8.f) * 0.125f);
+        int vchosen = -1;
+        double vabove = 0.0;
+        for (int attempt = 0; attempt < 2 && vchosen < 0; ++attempt) {
+            if (attempt == 1) D = INFINITY;  // every element
+            for (int i = threadIdx.x; i < 256 * kWarps; i += kThreads) hist_f[i] = 0.f;
+            __syncthreads();
+            float* hf = hist_f + warp * 256;
+            for (int c = warp; c < nchunks; c += kWarps) {
+                for (int j = 0; j < kVecPerLane; ++j) {
+                    int nv;
+                    uint4 v = load_vec<T>(row, V, c, j, lane, nv);
+                    for (int e = 0; e < nv; ++e) {
+                        const float x = raw_get<T>(v, e);
+                        if (M - x * invT < D) atomicAdd(&hf[vbin(x)], __expf(x * invT - M));
+                    }
+                }
+            }
+            __syncthreads();
+            if (warp == 0) {
+            double cum = 0.0;
+            int chosen = -1;
+            double chosen_above = 0.0;
+            for (int b0 = 0; b0 < 256 && chosen < 0; b0 += 32) {
+                const int bin = b0 + lane;
+                double m = 0.0;
+                for (int w = 0; w < kWarps; ++w) m += (double)hist_f[w * 256 + bin];
+                const double incl = warp_scan_f64(m, lane);
+                // (a bin whose elements all underflow to 0 cannot be where the mass crosses)
+                const unsigned hit = __ballot_sync(kFullMask, cum + incl >= target && m > 0.0);
+                if (hit) {
+                    const int src = __ffs(hit) - 1;
+                    chosen = b0 + src;
+                    chosen_above = cum + __shfl_sync(kFullMask, incl - m, src);
+                }
+                cum += __shfl_sync(kFullMask, incl, 31);
+            }
+            if (lane == 0) {
+                dred[0] = chosen_above;
+                dred[1] = (double)chosen;
+            }
+            }
+            __syncthreads();
+            vchosen = (int)dred[1];  // -1: the binned mass falls short of the target
+            vabove = dred[0];
+            __syncthreads();
+        }
         uint32_t prefix = 0;     // key bits fixed so far
-        double above = 0.0;      // mass of keys above the current prefix bin
+        double above = vchosen >= 0 ? vabove : 0.0;  // mass of keys above the current prefix bin
         uint32_t count_at = 0;
-        for (int level = 0; level < NLEVELS; ++level) {
+        for (int level = 0; level < NLEVELS && vchosen >= 0; ++level) {
             const int shift = 24 - 8 * level;
             const uint32_t hi_mask = level == 0 ? 0u : (~0u << (shift + 8));
             for (int i = threadIdx.x; i < 256 * kWarps; i += kThreads) {
@@ -167,7 +229,7 @@ __device__ void prepare_row(const T* row, const VerifyArgs& a, int nchunks, doub
                     for (int e = 0; e < nv; ++e) {
                         const float x = raw_get<T>(v, e);
                         const uint32_t key = float_key(x);
-                        if ((key & hi_mask) == prefix) {
+                        if ((key & hi_mask) == prefix && vbin(x) == vchosen) {
                             const uint32_t bin = (key >> shift) & 0xFFu;
                             atomicAdd(&hf[bin], __expf(x * invT - M));
                             atomicAdd(&hn[bin], 1u);
@@ -305,6 +367,49 @@ __device__ __forceinline__ void scan_chunk(const T* row, const VerifyArgs& a, co
     }
 }
 
+// Scan chunk c of two rows (verifier p, drafter q) together in id order; for every vector
+// of 32 lanes calls f(id0, wp, wq, nv) with the lane's normalised survivor probabilities
+// of both rows (reciprocals of the rows' surviving masses taken once).
+template <typename T, typename F>
+__device__ __forceinline__ void scan_pair_chunk(const T* prow, const T* qrow, const VerifyArgs& a, const RowInfo& rp,
+                                                const RowInfo& rq, int c, int tbp, int tbq, int lane, F f) {
+    constexpr int VEC = Elem<T>::VEC;
+    const float invT = 1.0f / a.temperature;
+    const double izp = 1.0 / rp.Z, izq = 1.0 / rq.Z;
+    int carp = tbp, carq = tbq;
+    for (int j = 0; j < kVecPerLane; ++j) {
+        int nv;
+        const uint4 vp = load_vec<T>(prow, a.V, c, j, lane, nv);
+        const uint4 vq = load_vec<T>(qrow, a.V, c, j, lane, nv);
+        int ntp = 0, ntq = 0;
+        for (int e = 0; e < nv; ++e) {
+            ntp += float_key(raw_get<T>(vp, e)) == rp.tau;
+            ntq += float_key(raw_get<T>(vq, e)) == rq.tau;
+        }
+        const int ip = warp_inclusive_scan(ntp, lane), iq = warp_inclusive_scan(ntq, lane);
+        int rkp = carp + ip - ntp, rkq = carq + iq - ntq;
+        const int64_t id0 = (int64_t)c * Chunk<T>::CH + (int64_t)j * 32 * VEC + lane * VEC;
+        double wp[VEC], wq[VEC];
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+            wp[e] = 0.0;
+            wq[e] = 0.0;
+            if (e < nv) {
+                const float xp = raw_get<T>(vp, e), xq = raw_get<T>(vq, e);
+                const uint32_t kp = float_key(xp), kq = float_key(xq);
+                bool sp = rp.tau == 0u || kp > rp.tau, sq = rq.tau == 0u || kq > rq.tau;
+                if (rp.tau != 0u && kp == rp.tau) sp = rkp++ < rp.c_tie;
+                if (rq.tau != 0u && kq == rq.tau) sq = rkq++ < rq.c_tie;
+                if (sp) wp[e] = (double)__expf(xp * invT - rp.M) * izp;
+                if (sq) wq[e] = (double)__expf(xq * invT - rq.M) * izq;
+            }
+        }
+        f(id0, wp, wq, nv);
+        carp += __shfl_sync(kFullMask, ip, 31);
+        carq += __shfl_sync(kFullMask, iq, 31);
+    }
+}
+
 // inverse-CDF draw over the row's survivors with uniform u (one warp)
 template <typename T>
 __device__ int warp_row_draw(const T* row, const VerifyArgs& a, const RowInfo& ri, const double* cmass,
@@ -421,14 +526,11 @@ __device__ void pair_pass(const T* prow, const T* qrow, const VerifyArgs& a, con
             tbp = warp_sum(tbp);
             tbq = warp_sum(tbq);
         }
-        double wp[kVecPerLane][Elem<T>::VEC];
-        scan_chunk<T>(prow, a, rp, c, tbp, lane, [&](int64_t, const double* wv, int nv, int j) {
-            for (int e = 0; e < Elem<T>::VEC; ++e) wp[j][e] = e < nv ? wv[e] / rp.Z : 0.0;
-        });
         double acc = 0.0;
-        scan_chunk<T>(qrow, a, rq, c, tbq, lane, [&](int64_t, const double* wv, int nv, int j) {
-            for (int e = 0; e < nv; ++e) acc += per_chunk(wp[j][e], wv[e] / rq.Z);
-        });
+        scan_pair_chunk<T>(prow, qrow, a, rp, rq, c, tbp, tbq, lane,
+                           [&](int64_t, const double* wp, const double* wq, int nv) {
+                               for (int e = 0; e < nv; ++e) acc += per_chunk(wp[e], wq[e]);
+                           });
         acc = warp_sum_f64(acc);
         (void)acc;
     }
@@ -437,12 +539,26 @@ __device__ void pair_pass(const T* prow, const T* qrow, const VerifyArgs& a, con
 // ---------------------------------------------------------------------------------------
 // the kernel: one CTA per sequence
 // ---------------------------------------------------------------------------------------
+// One CTA per row (every row of every sequence): the row's chunk table and RowInfo.
 template <typename T>
-__global__ void __launch_bounds__(kThreads) seq_kernel(Params p) {
+__global__ void __launch_bounds__(kThreads) rows_kernel(Params p) {
     __shared__ float hist_f[256 * kWarps];
     __shared__ uint32_t hist_n[256 * kWarps];
     __shared__ double dred[kWarps];
     __shared__ float fred[kWarps];
+    const VerifyArgs& a = p.a;
+    const int K = a.K, V = a.V, NC = p.nchunks, R = p.rows_per_seq;
+    const int64_t g = blockIdx.x;  // b * R + r
+    const int b = (int)(g / R), r = (int)(g % R);
+    const bool isP = r < K;
+    const int pos = isP ? r : r - K + 1;
+    const T* row = reinterpret_cast<const T*>(isP ? a.P : a.Q) + ((int64_t)b * K + pos) * V;
+    prepare_row<T>(row, a, NC, p.cmass + g * NC, p.cties + g * NC, p.infos + g, hist_f, hist_n, dred, fred);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) seq_kernel(Params p) {
+    __shared__ double dred[kWarps];
     __shared__ int s_tok[32];
     __shared__ double s_p[32], s_q[32], s_tv[32];
     __shared__ int s_acc[32];
@@ -456,10 +572,7 @@ __global__ void __launch_bounds__(kThreads) seq_kernel(Params p) {
         const int pos = isP ? r : r - K + 1;
         return reinterpret_cast<const T*>(isP ? a.P : a.Q) + ((int64_t)b * K + pos) * V;
     };
-    for (int r = 0; r < R; ++r)
-        prepare_row<T>(rowp(r), a, NC, p.cmass + (rbase + r) * NC, p.cties + (rbase + r) * NC, p.infos + rbase + r,
-                       hist_f, hist_n, dred, fred);
-    __syncthreads();
+    // the rows' tables come from rows_kernel (earlier on the stream)
 
     // per position: draws, probabilities, acceptance (warp per position)
     for (int i = warp; i < K; i += kWarps) {
@@ -537,17 +650,14 @@ __global__ void __launch_bounds__(kThreads) seq_kernel(Params p) {
             }
             tbp = warp_sum(tbp);
             tbq = warp_sum(tbq);
-            double wp[kVecPerLane][Elem<T>::VEC];
-            scan_chunk<T>(prow, a, rp, c, tbp, lane, [&](int64_t, const double* wv, int nv, int j) {
-                for (int e = 0; e < Elem<T>::VEC; ++e) wp[j][e] = e < nv ? wv[e] / rp.Z : 0.0;
-            });
             double acc = 0.0;
-            scan_chunk<T>(qrow, a, rq, c, tbq, lane, [&](int64_t, const double* wv, int nv, int j) {
-                for (int e = 0; e < nv; ++e) {
-                    const double d = wp[j][e] - wv[e] / rq.Z;
-                    acc += d > 0.0 ? d : 0.0;
-                }
-            });
+            scan_pair_chunk<T>(prow, qrow, a, rp, rq, c, tbp, tbq, lane,
+                               [&](int64_t, const double* wp, const double* wq, int nv) {
+                                   for (int e = 0; e < nv; ++e) {
+                                       const double d = wp[e] - wq[e];
+                                       acc += d > 0.0 ? d : 0.0;
+                                   }
+                               });
             acc = warp_sum_f64(acc);
             if (lane == 0) cres[c] = acc;
         }
@@ -589,17 +699,14 @@ __global__ void __launch_bounds__(kThreads) seq_kernel(Params p) {
                 }
                 tbp = warp_sum(tbp);
                 tbq = warp_sum(tbq);
-                double wp[kVecPerLane][Elem<T>::VEC];
-                scan_chunk<T>(prow, a, rp, cstar, tbp, lane, [&](int64_t, const double* wv, int nv, int j) {
-                    for (int e = 0; e < Elem<T>::VEC; ++e) wp[j][e] = e < nv ? wv[e] / rp.Z : 0.0;
-                });
                 int found = -1, last = -1;
                 double cum = before;
-                scan_chunk<T>(qrow, a, rq, cstar, tbq, lane, [&](int64_t id0, const double* wv, int nv, int j) {
+                scan_pair_chunk<T>(prow, qrow, a, rp, rq, cstar, tbp, tbq, lane,
+                                   [&](int64_t id0, const double* wp, const double* wq, int nv) {
                     double r[Elem<T>::VEC];
                     double s = 0.0;
                     for (int e = 0; e < Elem<T>::VEC; ++e) {
-                        const double d = e < nv ? wp[j][e] - wv[e] / rq.Z : 0.0;
+                        const double d = e < nv ? wp[e] - wq[e] : 0.0;
                         r[e] = d > 0.0 ? d : 0.0;
                         s += r[e];
                     }
@@ -687,10 +794,14 @@ uno_status verify_full_launch(const VerifyArgs& a, void* workspace, cudaStream_t
     p.cties = reinterpret_cast<int*>(ws + L.off_cties);
     p.cres = reinterpret_cast<double*>(ws + L.off_cres);
     p.infos = reinterpret_cast<vfull::RowInfo*>(ws + L.off_infos);
-    if (a.dtype == UNO_BF16)
+    const unsigned rows = (unsigned)((int64_t)a.B * L.rows_per_seq);
+    if (a.dtype == UNO_BF16) {
+        vfull::rows_kernel<__nv_bfloat16><<<rows, vfull::kThreads, 0, stream>>>(p);
         vfull::seq_kernel<__nv_bfloat16><<<(unsigned)a.B, vfull::kThreads, 0, stream>>>(p);
-    else
+    } else {
+        vfull::rows_kernel<float><<<rows, vfull::kThreads, 0, stream>>>(p);
         vfull::seq_kernel<float><<<(unsigned)a.B, vfull::kThreads, 0, stream>>>(p);
+    }
     return check_cuda(cudaGetLastError(), "launch(verify full)");
 }
 
