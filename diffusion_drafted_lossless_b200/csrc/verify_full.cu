@@ -70,6 +70,30 @@ __device__ __forceinline__ uint4 load_vec(const T* row, int V, int c, int j, int
     return nv > 0 ? load_raw<T>(row, e0, nv, aligned && nv == VEC) : make_uint4(0, 0, 0, 0);
 }
 
+// Full bf16 vectors: the 8 elements in id order, and packed tests that let a vector whose
+// elements cannot pass a pass's test skip the per-element work (the exact test still
+// decides every element of a vector that is not skipped).
+__device__ __forceinline__ void unpack8(const uint4& v, float (&x)[8]) {
+    x[0] = bf16_lo(v.x); x[1] = bf16_hi(v.x); x[2] = bf16_lo(v.y); x[3] = bf16_hi(v.y);
+    x[4] = bf16_lo(v.z); x[5] = bf16_hi(v.z); x[6] = bf16_lo(v.w); x[7] = bf16_hi(v.w);
+}
+__device__ __forceinline__ __nv_bfloat162 as_b2(uint32_t w) { return *reinterpret_cast<__nv_bfloat162*>(&w); }
+// some element >= lo
+__device__ __forceinline__ bool any_ge(const uint4& v, __nv_bfloat162 lo) {
+    const __nv_bfloat162 m = __hmax2(__hmax2(as_b2(v.x), as_b2(v.y)), __hmax2(as_b2(v.z), as_b2(v.w)));
+    return __hge2_mask(m, lo) != 0u;
+}
+// some element in [lo, hi]
+__device__ __forceinline__ bool any_in(const uint4& v, __nv_bfloat162 lo, __nv_bfloat162 hi) {
+    const uint32_t m = (__hge2_mask(as_b2(v.x), lo) & __hle2_mask(as_b2(v.x), hi)) |
+                       (__hge2_mask(as_b2(v.y), lo) & __hle2_mask(as_b2(v.y), hi)) |
+                       (__hge2_mask(as_b2(v.z), lo) & __hle2_mask(as_b2(v.z), hi)) |
+                       (__hge2_mask(as_b2(v.w), lo) & __hle2_mask(as_b2(v.w), hi));
+    return m != 0u;
+}
+template <typename T>
+constexpr bool kIsBf16 = sizeof(T) == 2;
+
 __device__ __forceinline__ double cta_sum_f64(double v, double* red) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     v = warp_sum_f64(v);
@@ -112,6 +136,13 @@ __device__ void prepare_row(const T* row, const VerifyArgs& a, int nchunks, doub
         for (int j = 0; j < kVecPerLane; ++j) {
             int nv;
             uint4 v = load_vec<T>(row, V, c, j, lane, nv);
+            if constexpr (kIsBf16<T>) {
+                if (nv == 8) {
+                    const __nv_bfloat162 m2 = __hmax2(__hmax2(as_b2(v.x), as_b2(v.y)), __hmax2(as_b2(v.z), as_b2(v.w)));
+                    cm = fmaxf(cm, fmaxf(__low2float(m2), __high2float(m2)) * invT);
+                    continue;
+                }
+            }
             for (int e = 0; e < nv; ++e) cm = fmaxf(cm, raw_get<T>(v, e) * invT);
         }
         cm = warp_max(cm);
@@ -119,6 +150,15 @@ __device__ void prepare_row(const T* row, const VerifyArgs& a, int nchunks, doub
         for (int j = 0; j < kVecPerLane; ++j) {
             int nv;
             uint4 v = load_vec<T>(row, V, c, j, lane, nv);
+            if constexpr (kIsBf16<T>) {
+                if (nv == 8) {
+                    float x[8];
+                    unpack8(v, x);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) cs += __expf(x[e] * invT - cm);
+                    continue;
+                }
+            }
             for (int e = 0; e < nv; ++e) cs += __expf(raw_get<T>(v, e) * invT - cm);
         }
         cs = warp_sum(cs);
@@ -170,10 +210,25 @@ __device__ void prepare_row(const T* row, const VerifyArgs& a, int nchunks, doub
             for (int i = threadIdx.x; i < 256 * kWarps; i += kThreads) hist_f[i] = 0.f;
             __syncthreads();
             float* hf = hist_f + warp * 256;
+            // packed prefilter: a logit below (M - D) T - 1/16 (rounded down) cannot pass
+            const __nv_bfloat162 alo = D == INFINITY
+                                           ? __float2bfloat162_rn(-INFINITY)
+                                           : __bfloat162bfloat162(__float2bfloat16_rd(((M - D) - 0.0625f) * a.temperature));
             for (int c = warp; c < nchunks; c += kWarps) {
                 for (int j = 0; j < kVecPerLane; ++j) {
                     int nv;
                     uint4 v = load_vec<T>(row, V, c, j, lane, nv);
+                    if constexpr (kIsBf16<T>) {
+                        if (nv == 8) {
+                            if (!any_ge(v, alo)) continue;
+                            float x[8];
+                            unpack8(v, x);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                if (M - x[e] * invT < D) atomicAdd(&hf[vbin(x[e])], __expf(x[e] * invT - M));
+                            continue;
+                        }
+                    }
                     for (int e = 0; e < nv; ++e) {
                         const float x = raw_get<T>(v, e);
                         if (M - x * invT < D) atomicAdd(&hf[vbin(x)], __expf(x * invT - M));
@@ -212,6 +267,13 @@ __device__ void prepare_row(const T* row, const VerifyArgs& a, int nchunks, doub
         uint32_t prefix = 0;     // key bits fixed so far
         double above = vchosen >= 0 ? vabove : 0.0;  // mass of keys above the current prefix bin
         uint32_t count_at = 0;
+        // packed prefilter of the radix levels: the logits of the chosen bin lie within
+        // [(M - (b + 1) / 8) T, (M - b / 8) T], widened by 1/16 and rounded outwards
+        const float vlo = (M - (vchosen + 1) * 0.125f - 0.0625f) * a.temperature;
+        const float vhi = (M - vchosen * 0.125f + 0.0625f) * a.temperature;
+        const __nv_bfloat162 rlo = vchosen == 255 ? __float2bfloat162_rn(-INFINITY)
+                                                  : __bfloat162bfloat162(__float2bfloat16_rd(vlo));
+        const __nv_bfloat162 rhi = __bfloat162bfloat162(__float2bfloat16_ru(vhi));
         for (int level = 0; level < NLEVELS && vchosen >= 0; ++level) {
             const int shift = 24 - 8 * level;
             const uint32_t hi_mask = level == 0 ? 0u : (~0u << (shift + 8));
@@ -226,6 +288,23 @@ __device__ void prepare_row(const T* row, const VerifyArgs& a, int nchunks, doub
                 for (int j = 0; j < kVecPerLane; ++j) {
                     int nv;
                     uint4 v = load_vec<T>(row, V, c, j, lane, nv);
+                    if constexpr (kIsBf16<T>) {
+                        if (nv == 8) {
+                            if (!any_in(v, rlo, rhi)) continue;
+                            float x[8];
+                            unpack8(v, x);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                const uint32_t key = float_key(x[e]);
+                                if ((key & hi_mask) == prefix && vbin(x[e]) == vchosen) {
+                                    const uint32_t bin = (key >> shift) & 0xFFu;
+                                    atomicAdd(&hf[bin], __expf(x[e] * invT - M));
+                                    atomicAdd(&hn[bin], 1u);
+                                }
+                            }
+                            continue;
+                        }
+                    }
                     for (int e = 0; e < nv; ++e) {
                         const float x = raw_get<T>(v, e);
                         const uint32_t key = float_key(x);
@@ -300,9 +379,24 @@ __device__ void prepare_row(const T* row, const VerifyArgs& a, int nchunks, doub
             for (int c = warp; c < nchunks; c += kWarps) {
                 float mg = 0.f;
                 int nt = 0;
+                const __nv_bfloat162 tlo = __float2bfloat162_rn(key_float(tau));  // tau is a bf16 value here
                 for (int j = 0; j < kVecPerLane; ++j) {
                     int nv;
                     uint4 v = load_vec<T>(row, V, c, j, lane, nv);
+                    if constexpr (kIsBf16<T>) {
+                        if (nv == 8) {
+                            if (!any_ge(v, tlo)) continue;
+                            float x[8];
+                            unpack8(v, x);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                const uint32_t key = float_key(x[e]);
+                                if (key > tau) mg += __expf(x[e] * invT - M);
+                                nt += key == tau;
+                            }
+                            continue;
+                        }
+                    }
                     for (int e = 0; e < nv; ++e) {
                         const float x = raw_get<T>(v, e);
                         const uint32_t key = float_key(x);
