@@ -84,6 +84,8 @@ def _bind(lib):
                                         _i32p, _i32p, _f64p, _i32p, _i32p, _i32p,
                                         _f64p, _f64p, _f64p, _f64p]
     lib.oracle_tv_loss.argtypes = [_f64p, _f64p, _i64, _i64, _u8p, _f64, _f64p, _f64p, _f64p, _f64p]
+    lib.oracle_block_noise.argtypes = [_i32p, ctypes.POINTER(ctypes.c_float), _i64, _i64, _i64, _i32p, _f64p]
+    lib.oracle_block_noise.restype = ctypes.c_int
     lib.oracle_num_threads.restype = ctypes.c_int
     lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
     return lib
@@ -177,3 +179,17 @@ def tv_loss(teacher, student, mask=None, grad_scale=1.0, want_grad=True, want_ab
                                 _p(tv, _f64p), ctypes.byref(mean), _p(g, _f64p), _p(ad, _f64p))
     assert rc == 0
     return {"tv": tv, "mean": mean.value, "grad": g, "absdiff": ad}
+
+
+def block_noise(clean, uniforms, V):
+    """Block-noised copy, random_uniform mode: dict tokens [B, K] int32, gate [B*K] (see
+    oracle_block_noise)."""
+    c = np.ascontiguousarray(clean, dtype=np.int32)
+    B, K = c.shape
+    u = np.ascontiguousarray(uniforms, dtype=np.float32).reshape(B, K)
+    out = np.empty((B, K), np.int32)
+    gate = np.empty(B * K)
+    rc = _load().oracle_block_noise(_p(c, _i32p), u.ctypes.data_as(ctypes.POINTER(ctypes.c_float)), B, K, int(V),
+                                    _p(out, _i32p), _p(gate, _f64p))
+    assert rc == 0
+    return {"tokens": out, "gate": gate}

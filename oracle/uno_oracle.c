@@ -387,3 +387,33 @@ int oracle_tv_loss(const double* teacher, const double* student, int64_t N, int6
     *mean = n_mask > 0 ? s / (double)n_mask : 0.0;
     return 0;
 }
+
+/* ------------------------------------------------------------------------------------
+ * Block noising, noise mode random_uniform [LU-train: the student reads a block-noised
+ * copy of each sequence; MC-proto: noise mode random_uniform].
+ * Readings: position 0 of every block keeps its token (it is the exact AR token, [LU-how])
+ * and each draft position 1..K-1 gets a token drawn uniformly from the vocabulary from a
+ * supplied uniform u in [0, 1):
+ *   out[b, 0] = clean[b, 0];   out[b, i] = min(V - 1, floor(u[b, i] * V))   (i >= 1)
+ * (u is a float32 and V < 2^24, so u * V is exact in fp64 and the floor is exact).
+ * gate[b*K + i] (optional) is the row gate of the adapter: 0 at i = 0, 1 at the noise rows.
+ * ------------------------------------------------------------------------------------ */
+int oracle_block_noise(const int32_t* clean, const float* u, int64_t B, int64_t K, int64_t V, int32_t* out,
+                       double* gate)
+{
+    if (B < 0 || K < 1 || V < 1 || V >= (1 << 24)) return 1;
+    for (int64_t b = 0; b < B; ++b) {
+        for (int64_t i = 0; i < K; ++i) {
+            const int64_t o = b * K + i;
+            if (i == 0) {
+                out[o] = clean[o];
+            } else {
+                double t = floor((double)u[o] * (double)V);
+                if (t > (double)(V - 1)) t = (double)(V - 1);
+                out[o] = (int32_t)t;
+            }
+            if (gate) gate[o] = i == 0 ? 0.0 : 1.0;
+        }
+    }
+    return 0;
+}

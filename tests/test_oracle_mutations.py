@@ -12,6 +12,7 @@ import pytest
 
 import oracle
 from tests import test_oracle_gated_lora as pins_lora
+from tests import test_oracle_noise as pins_noise
 from tests import test_oracle_tv as pins_tv
 from tests import test_oracle_verify as pins_verify
 
@@ -29,6 +30,8 @@ PINS = [
     pins_tv.test_identical_is_zero, pins_tv.test_range_symmetry_and_overlap_identity,
     pins_tv.test_two_token_closed_form, pins_tv.test_mean_over_mask_and_masked_gradient,
     pins_tv.test_gradient_rows_sum_to_zero, pins_tv.test_gradient_finite_differences,
+    pins_noise.test_hand_example, pins_noise.test_extremes_of_the_uniform, pins_noise.test_block_of_one_keeps_the_block,
+    pins_noise.test_noised_tokens_are_uniform,
 ]
 PINS_EXACT = [lambda c=c: pins_verify.test_exact_losslessness(c) for c in range(6)]
 
@@ -56,6 +59,12 @@ MUTATIONS = {
     "lora_scale_dropped": ("y[m * d_out + o] = base + scale * gm * lora;", "y[m * d_out + o] = base + gm * lora;"),
     "w0_transposed": ("base += xm[k] * w0[o * d_in + k];", "base += xm[k] * w0[(k * d_out + o) % (d_in * d_out)];"),
     "lora_b_index_swapped": ("lora += t[j] * b[o * rank + j];", "lora += t[j] * b[(j * d_out + o) % (d_out * rank)];"),
+    "noise_position0_noised": ("            if (i == 0) {\n                out[o] = clean[o];",
+                               "            if (i < 0) {\n                out[o] = clean[o];"),
+    "noise_rounds_up": ("double t = floor((double)u[o] * (double)V);", "double t = ceil((double)u[o] * (double)V);"),
+    "noise_not_clamped": ("if (t > (double)(V - 1)) t = (double)(V - 1);", "if (t > (double)V) t = (double)V;"),
+    "noise_skips_last_token": ("double t = floor((double)u[o] * (double)V);",
+                               "double t = floor((double)u[o] * (double)(V - 1));"),
 }
 
 
