@@ -24,7 +24,7 @@ EXPORTED = (
     "uno_status_string", "uno_last_error_string", "uno_version", "uno_read_device_status",
     "uno_gated_lora_linear_workspace_size", "uno_gated_lora_linear",
     "uno_block_verify_workspace_size", "uno_block_verify", "uno_block_verify_noalloc",
-    "uno_tv_loss_workspace_size", "uno_tv_loss",
+    "uno_tv_loss_workspace_size", "uno_tv_loss", "uno_block_noise",
 )
 
 
@@ -67,6 +67,8 @@ def load(path: str | os.PathLike | None = None) -> ctypes.CDLL:
     lib.uno_tv_loss_workspace_size.restype = _sz
     lib.uno_tv_loss_workspace_size.argtypes = [_i64, _i64, ctypes.c_int]
     lib.uno_tv_loss.argtypes = [_vp, _vp, ctypes.c_int, _i64, _i64, _vp, _f32, _vp, _vp, _vp, _vp, _sz, _vp]
+    lib.uno_block_noise.argtypes = [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp]
+    lib.uno_block_noise.restype = ctypes.c_int
     for fn in ("uno_gated_lora_linear", "uno_block_verify", "uno_tv_loss"):
         getattr(lib, fn).restype = ctypes.c_int
     lib.uno_read_device_status.restype = ctypes.c_int
@@ -181,3 +183,13 @@ def uno_tv_loss(teacher_logits, student_logits, out_tv, out_mean, grad_student=N
     _check(load().uno_tv_loss(_ptr(teacher_logits), _ptr(student_logits), code, N, V, _ptr(response_mask),
                               float(grad_scale), _ptr(out_tv), _ptr(out_mean), _ptr(grad_student), _ptr(ws), nb,
                               _stream(stream)))
+
+
+# ---------------------------------------------------------------------------------------
+def uno_block_noise(clean_tokens, uniforms, V, noised_tokens, row_gate=None, stream=None):
+    """Block-noised copy, noise mode random_uniform: position 0 kept, draft positions
+    min(V - 1, floor(u V)); optional row gate (see include/uno.h)."""
+    B, K = clean_tokens.shape
+    _check(load().uno_block_noise(_ptr(clean_tokens), _ptr(uniforms), B, K, int(V), _ptr(noised_tokens),
+                                  _ptr(row_gate), _stream(stream)))
+    return noised_tokens

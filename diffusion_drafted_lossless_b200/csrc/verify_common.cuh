@@ -244,7 +244,7 @@ __device__ void sequence_verify(const VerifyArgs& a, unsigned char* recs, int kc
             double pi = 0.0, qi = 0.0, tv = 0.0;
             int acc = 1;
             if (i == 0) {
-                tok = a.pos0 ? a.pos0[b] : srec_inv_cdf(P, (double)u[0], lane);
+                tok = a.pos0 && a.pos0[b] >= 0 ? a.pos0[b] : srec_inv_cdf(P, (double)u[0], lane);
                 pi = (tok >= 0 && tok < a.V) ? srec_prob(P, tok) : 0.0;
             } else {
                 SRec Q = warp_stage_rec(recs, kcap, rbase + K + i - 1, w1, i1, lane);

@@ -678,7 +678,8 @@ __global__ void __launch_bounds__(kThreads) seq_kernel(Params p) {
         double pi = 0.0, qi = 0.0;
         int acc = 1;
         if (i == 0) {
-            tok = a.pos0 ? a.pos0[b] : warp_row_draw<T>(rowp(0), a, rp, cmp, ctp, NC, (double)u[0], lane);
+            tok = a.pos0 && a.pos0[b] >= 0 ? a.pos0[b]
+                                           : warp_row_draw<T>(rowp(0), a, rp, cmp, ctp, NC, (double)u[0], lane);
             pi = warp_row_prob<T>(rowp(0), a, rp, ctp, tok, lane);
         } else {
             const int rq_i = K + i - 1;

@@ -9,6 +9,9 @@
  *                          "Evaluation protocol")
  *   uno_tv_loss            the TV self-distillation loss and its gradient (LoopUno project
  *                          page, "Training is self-distillation")
+ * and the block-noised copy that feeds the drafter and the student:
+ *   uno_block_noise        noise mode random_uniform (LoopUno project page, "Training is
+ *                          self-distillation"; model card, "Evaluation protocol")
  *
  * Conventions shared by every entry point
  *   - Pointers named as tensors are DEVICE pointers owned by the caller, row-major and
@@ -24,7 +27,7 @@
  *     `stream` (asynchronous); results are ready after the stream reaches that point.
  *   - uno_last_error_string() gives a readable reason for the calling thread's last
  *     failing call.
- *   - Device pointers must be 16-byte aligned.
+ *   - Device pointers must be 16-byte aligned (uno_block_noise: 4-byte aligned).
  *   - bf16 is IEEE-754 binary32 truncated to its upper 16 bits (1-8-7), stored as uint16.
  */
 #ifndef UNO_H
@@ -120,7 +123,8 @@ uno_status uno_gated_lora_linear(const void* x, const void* w0, const void* lora
  * order whose cumulative mass is >= top_p, the crossing token included); renormalise.
  * Call the results p_i and q_i.
  *
- *   x_0 = pos0_tokens[b], or the inverse-CDF draw of p_0 with uniforms[b,0,0]
+ *   x_0 = pos0_tokens[b] if given and >= 0, else the inverse-CDF draw of p_0 with
+ *         uniforms[b,0,0]
  *   d_i = draft_tokens[b,i], or the inverse-CDF draw of q_i with uniforms[b,i,0], i >= 1
  *   draft i is accepted iff uniforms[b,i,1] * q_i(d_i) < p_i(d_i)  (prob. min(1, p/q))
  *   n = 1 + number of leading accepted drafts (position 0 is always emitted)
@@ -142,7 +146,9 @@ uno_status uno_gated_lora_linear(const void* x, const void* w0, const void* lora
  *   top_k           0 = off; else 1 <= top_k <= 1024 (top_k >= V is the same as off)
  *   top_p           (0, 1) filters; >= 1 = off
  *   draft_tokens    [B, K] int32 or NULL (column 0 ignored); NULL: drawn from q_i
- *   pos0_tokens     [B] int32 or NULL; NULL: drawn from p_0
+ *   pos0_tokens     [B] int32 or NULL; NULL or an entry < 0: drawn from p_0 (so a
+ *                   previous step's out_next_token can be passed as is: -1 when all of
+ *                   its drafts were accepted)
  *   uniforms        [B, K, 3] float32 in [0, 1): (sample, accept, resample)
  *   out_tokens      [B, K] int32: x_0, d_1 .. d_{n-1}, then -1
  *   out_count       [B] int32: n
@@ -199,6 +205,32 @@ uno_status uno_block_verify_noalloc(const void* verifier_logits, const void* dra
                                     int32_t* out_count, int32_t* out_next_token,
                                     float* out_p_tok, float* out_q_tok, float* out_tv,
                                     uno_stream_t stream);
+
+/* ======================================================================================
+ * Block noising, noise mode random_uniform
+ *
+ * The block-noised copy that the student (training) and the drafter (decode) read: in
+ * every block, position 0 keeps its token and each draft position i = 1..K-1 gets a token
+ * drawn uniformly from the vocabulary by the supplied uniform:
+ *   noised[b, 0] = clean[b, 0]
+ *   noised[b, i] = min(V - 1, floor(uniforms[b, i] * V))          (i >= 1, fp64, exact)
+ *   row_gate[b * K + i] = 0 at i = 0, 1 at i >= 1  (the adapter's gate for these rows)
+ * Source: LoopUno project page, "Training is self-distillation" (the student is the model
+ * with its LoRA on a block-noised copy of each sequence) and "How it works" (position 0 is
+ * the exact AR token; the adapter is on only for noise positions); uno-qwen3-8B model
+ * card, "Evaluation protocol" (noise mode random_uniform).
+ *
+ *   clean_tokens  [B, K] int32
+ *   uniforms      [B, K] float32 in [0, 1) (uniforms[b, 0] is not read; 1.0 maps to V - 1)
+ *   noised_tokens [B, K] int32; may be clean_tokens itself (each output element depends
+ *                 only on the same input element)
+ *   row_gate      [B * K] float32 or NULL
+ *
+ * Device pointers, 4-byte aligned. Limits (else UNO_ERR_INVALID_ARG): B >= 0, K >= 1,
+ * 1 <= V < 2^24. B = 0 launches nothing. No workspace.
+ * ====================================================================================== */
+uno_status uno_block_noise(const int32_t* clean_tokens, const float* uniforms, int32_t B, int32_t K,
+                           int32_t V, int32_t* noised_tokens, float* row_gate, uno_stream_t stream);
 
 /* ======================================================================================
  * TV self-distillation loss and its gradient

@@ -225,9 +225,9 @@ int64_t oracle_inv_cdf(const double* w, int64_t V, double Z, double u, double* m
  *
  * Inputs (row-major): P, Q logits [B, K, V] (verifier, drafter); u [B, K, 3] uniforms
  * (sample, accept, resample); drafts [B, K] (NULL: d_i drawn from Q_i with u[b,i,0]);
- * pos0 [B] (NULL: x_0 drawn from P_0 with u[b,0,0]).
+ * pos0 [B] (NULL, or an entry < 0: x_0 drawn from P_0 with u[b,0,0]).
  * For each sequence b:
- *   x_0 = pos0[b] or invCDF(P_0, u[b,0,0])                     (always emitted)
+ *   x_0 = pos0[b] if given and >= 0, else invCDF(P_0, u[b,0,0])   (always emitted)
  *   for i = 1..K-1: d_i = drafts[b,i] or invCDF(Q_i, u[b,i,0])
  *                   accept iff u[b,i,1] * Q_i(d_i) < P_i(d_i); stop at the first reject j
  *   out_tokens = [x_0, d_1, ..., d_{n-1}, -1, ...], out_count = n (= j, or K if none)
@@ -266,7 +266,7 @@ int oracle_block_verify(const double* P, const double* Q, int64_t B, int64_t K, 
             double Zp = oracle_warp_row(prow, V, T, top_k, top_p, wp, &mg[3], NULL);
             if (i == 0) {
                 int64_t x0;
-                if (pos0) x0 = pos0[b];
+                if (pos0 && pos0[b] >= 0) x0 = pos0[b];
                 else x0 = oracle_inv_cdf(wp, V, Zp, ui[0], &mg[0]);
                 tok[0] = (int32_t)x0;
                 acc[0] = 1;

@@ -28,7 +28,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported(lib):
     names = declared_functions()
-    assert len(names) == 11, names
+    assert len(names) == 12, names
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(_lib.EXPORTED)
@@ -118,3 +118,14 @@ def test_product_path_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(_lib, "_lib", None)
     with pytest.raises(RuntimeError, match="no fallback"):
         _lib.load(tmp_path / "missing.so")
+
+
+def test_noise_validation(lib):
+    f = lib.uno_block_noise
+    assert f(FAKE, FAKE, -1, 4, 100, FAKE, None, None) == _lib.UNO_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, 2, 0, 100, FAKE, None, None) == _lib.UNO_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, 2, 4, 0, FAKE, None, None) == _lib.UNO_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, 2, 4, 1 << 24, FAKE, None, None) == _lib.UNO_ERR_INVALID_ARG
+    assert f(None, FAKE, 2, 4, 100, FAKE, None, None) == _lib.UNO_ERR_INVALID_ARG
+    assert f(FAKE + 2, FAKE, 2, 4, 100, FAKE, None, None) == _lib.UNO_ERR_UNSUPPORTED
+    assert f(None, None, 0, 4, 100, None, None, None) == _lib.UNO_OK  # B = 0: nothing to do

@@ -1,0 +1,70 @@
+"""The linear draft/verify step driver on the GPU: each step's block noising, gated
+projection and verify agree with the oracle chained the same way (the carried token feeds
+the next step's position 0), and the CUDA-graph replay gives the eager results."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from diffusion_drafted_lossless_b200 import workloads as W
+from diffusion_drafted_lossless_b200.driver import DraftVerifyDriver
+from tests.gpu_util import NEAR_FP64, decision_path_margin
+
+pytestmark = pytest.mark.gpu
+
+V = W.VerifyWorkload("drv", 4242, B=8, K=16, V=32000, sigma=3.0, rho=0.8, temperature=1.0, top_k=50, top_p=0.95)
+L = W.GatedLoraWorkload("drv", 4243, M=8 * 16, block=16, rank=16, scale=2.0,
+                        shapes=(W.LinearShape("q", 512, 512), W.LinearShape("k", 512, 128), W.LinearShape("v", 512, 128),
+                                W.LinearShape("o", 512, 512), W.LinearShape("gate", 512, 1024),
+                                W.LinearShape("up", 512, 1024), W.LinearShape("down", 1024, 512)))
+
+
+def _run(steps, graph):
+    d = DraftVerifyDriver(L, V)
+    out = []
+    for s in range(steps):
+        if graph and s == 1:
+            d.capture()
+        tok, cnt, nxt = d.step()
+        torch.cuda.synchronize()
+        out.append((tok.cpu().numpy().copy(), cnt.cpu().numpy().copy(), nxt.cpu().numpy().copy(),
+                    d.noised.cpu().numpy().copy(), d.gate.cpu().numpy().copy(), d.lin[0]["y"].float().cpu().numpy()))
+    return d, out
+
+
+def test_steps_match_the_chained_oracle():
+    d, out = _run(4, graph=False)
+    Pf = W.to_f64(d.P_host, "bf16").reshape(V.B, V.K, V.V)
+    Qf = W.to_f64(d.Q_host, "bf16").reshape(V.B, V.K, V.V)
+    carry = np.full(V.B, -1, np.int32)
+    counts = []
+    for s, (tok, cnt, nxt, noised, gate, y0) in enumerate(out):
+        u, un = d.pool_inputs(s)
+        clean = np.zeros((V.B, V.K), np.int32)
+        clean[:, 0] = carry
+        nz = oracle.block_noise(clean, un, V.V)
+        assert (noised == nz["tokens"]).all() and (gate == nz["gate"]).all()
+        ref = oracle.block_verify(Pf, Qf, u.astype(np.float64), V.temperature, V.top_k,
+                                  float(np.float32(V.top_p)), pos0=nz["tokens"][:, 0])
+        for b in range(V.B):
+            if decision_path_margin(ref, b) < NEAR_FP64:
+                continue  # a decision within rounding of its threshold
+            assert cnt[b] == ref["count"][b] and nxt[b] == ref["next"][b], (s, b)
+            assert (tok[b] == ref["tokens"][b]).all(), (s, b)
+        # the gated projection uses the noise kernel's gate
+        inp = W.linear_inputs(L, L.shapes[0])
+        yref = oracle.gated_lora(W.to_f64(inp["x"], "bf16"), W.to_f64(inp["w0"], "bf16"), W.to_f64(inp["a"], "bf16"),
+                                 W.to_f64(inp["b"], "bf16"), nz["gate"], float(np.float32(L.scale)))
+        assert np.abs(y0 - yref).max() / np.abs(yref).max() <= 5e-3
+        carry = nxt.copy()
+        counts.append(cnt)
+    tpf = DraftVerifyDriver.tokens_per_forward(counts)
+    assert 1.0 <= tpf <= V.K
+
+
+def test_graph_replay_equals_eager():
+    _, eager = _run(4, graph=False)
+    _, graph = _run(4, graph=True)
+    for a, b in zip(eager, graph):
+        for x, y in zip(a[:5], b[:5]):
+            assert (x == y).all()

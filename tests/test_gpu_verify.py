@@ -275,3 +275,19 @@ def test_looped_verify_sampled_sequences():
     n, near, bad, literal = compare_verify(sub, ref, check_tv=False, near_eps=FULL_BAND)
     assert not bad, bad
     assert (gpu["count"] >= 1).all() and (gpu["count"] <= K).all()
+
+
+@pytest.mark.parametrize("top_k", [50, 0])
+def test_pos0_entries_below_zero_draw_from_p0(top_k):
+    """pos0_tokens[b] < 0 (a previous step's next token when all its drafts were accepted)
+    draws x_0 from p_0, on both paths; the other entries are taken as given."""
+    B, K, V = 6, 5, 4000
+    P, Q, u = _inputs(B, K, V, "bf16", seed=91 + top_k)
+    pos0 = np.random.default_rng(91).integers(0, V, B).astype(np.int32)
+    pos0[::2] = -1
+    if top_k:
+        gpu, ref, _ = _check(P, Q, u, 1.0, top_k, 0.95, "bf16", pos0=pos0)
+    else:
+        gpu, ref, _ = _check_full(P, Q, u, 1.0, 0.95, "bf16", pos0=pos0)
+    assert (gpu["tokens"][1::2, 0] == pos0[1::2]).all()
+    assert (gpu["tokens"][::2, 0] >= 0).all()

@@ -277,6 +277,14 @@ def test_position0_is_the_ar_token():
     out2 = oracle.block_verify(P, Q, u, 0.8, 7, 0.93, pos0=pos0)
     np.testing.assert_array_equal(out2["tokens"][:, 0], pos0)
     assert (out2["count"] >= 1).all()
+    # an entry < 0 (a previous step's next token when all its drafts were accepted) means
+    # "draw from p_0": those sequences equal the run without pos0
+    pos0[::3] = -1
+    out3 = oracle.block_verify(P, Q, u, 0.8, 7, 0.93, pos0=pos0)
+    for b in range(B):
+        ref = out if pos0[b] < 0 else out2
+        np.testing.assert_array_equal(out3["tokens"][b], ref["tokens"][b])
+        assert out3["count"][b] == ref["count"][b] and out3["next"][b] == ref["next"][b]
 
 
 def test_supplied_drafts_zero_probabilities():
