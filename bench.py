@@ -349,6 +349,27 @@ def measure_configs(torch, dev, lib, pk, reduce):
     out["tv_loss_n16384_v151936"] = {"ms": ms, "gbs": tb / (ms * 1e-3) / 1e9, "frac": tb / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
     del T_, S_, grad
     torch.cuda.empty_cache()
+    # ---- the draft/verify step driver at the serving shapes: noising, the seven gated
+    #      projections, the verify, the carried token; eager and replayed from a CUDA graph ----
+    try:
+        from diffusion_drafted_lossless_b200.driver import DraftVerifyDriver
+        d = DraftVerifyDriver(LINEARS, VERIFY)
+        counts = []
+        for _ in range(3):
+            counts.append(d.step()[1].cpu().numpy())
+        ms_eager = timed(lambda: d.step(), 10)
+        d.capture()
+        ms_graph = timed(lambda: d.step(), 20)
+        for _ in range(5):
+            counts.append(d.step()[1].cpu().numpy())
+        out["draft_verify_driver_b64_k16"] = {"ms_eager": ms_eager, "ms_graph": ms_graph,
+                                              "tokens_per_forward": DraftVerifyDriver.tokens_per_forward(counts),
+                                              "library_launches_per_step": 1 + 7 + 3,
+                                              "torch_copies_per_step": 2}
+        del d
+    except Exception as e:  # reported, never fatal to the bench line
+        out["draft_verify_driver_b64_k16"] = {"error": f"{type(e).__name__}: {e}"[:300]}
+    torch.cuda.empty_cache()
     return out
 
 
