@@ -25,6 +25,12 @@
 // Sums are fp32 within a chunk and fp64 across chunks.
 #include <cuda_bf16.h>
 
+#include <cstdlib>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <type_traits>
+
 #include "verify_common.cuh"
 
 namespace uno {
@@ -52,6 +58,7 @@ struct Params {
     int* cties;       // [B * rows_per_seq * nchunks] tokens equal to tau per chunk
     double* cres;     // [B * nchunks] scratch: residual mass per chunk
     RowInfo* infos;   // [B * rows_per_seq]
+    uint32_t* status; // device status word (bounded waits that give up)
 };
 
 template <typename T>
@@ -119,23 +126,180 @@ __device__ __forceinline__ float cta_max_f32(float v, float* red) {
 }
 
 // ---------------------------------------------------------------------------------------
-// per row: statistics, top-p cut, per-chunk survivor table (whole CTA)
+// where a row's elements come from, and which CTAs share the work of a row
 // ---------------------------------------------------------------------------------------
+// The whole row in global memory (per-row kernel).
 template <typename T>
-__device__ void prepare_row(const T* row, const VerifyArgs& a, int nchunks, double* cmass, int* cties, RowInfo* info,
-                            float* hist_f, uint32_t* hist_n, double* dred, float* fred) {
+struct GlobalRow {
+    const T* row;
+    int V;
+    __device__ __forceinline__ uint4 load(int c, int j, int lane, int& nv) const {
+        return load_vec<T>(row, V, c, j, lane, nv);
+    }
+};
+
+// This CTA's slice of a bf16 row in shared memory, starting at chunk c0 (cluster kernel;
+// V is a multiple of 8, so every 8-element vector is either whole or past the end).
+struct SharedSlice {
+    const uint16_t* slice;
+    int c0, V;
+    __device__ __forceinline__ uint4 load(int c, int j, int lane, int& nv) const {
+        constexpr int CH = Chunk<__nv_bfloat16>::CH;
+        const int e0 = c * CH + j * 256 + lane * 8;
+        nv = e0 < V ? 8 : 0;
+        return nv ? lds128(slice + (e0 - c0 * CH)) : make_uint4(0u, 0u, 0u, 0u);
+    }
+};
+
+__device__ __forceinline__ uint32_t cl_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cl_size() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cl_index() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cl_count() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+    return r;
+}
+
+// One CTA per row: the group is the CTA.
+struct CtaGroup {
+    __device__ __forceinline__ int size() const { return 1; }
+    __device__ __forceinline__ void sync() const { __syncthreads(); }
+    template <class X>
+    __device__ __forceinline__ const X* peer(const X* p, int) const { return p; }
+};
+
+// A thread-block cluster per row: barriers are cluster barriers (release / acquire), and
+// peer(p, r) is the generic address of p's counterpart in the shared memory of CTA r.
+struct ClusterGroup {
+    int n;
+    __device__ __forceinline__ int size() const { return n; }
+    __device__ __forceinline__ void sync() const {
+        asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+    }
+    template <class X>
+    __device__ __forceinline__ const X* peer(const X* p, int r) const {
+        uint64_t q;
+        asm volatile("mapa.u64 %0, %1, %2;" : "=l"(q) : "l"(reinterpret_cast<uint64_t>(p)), "r"(r));
+        return reinterpret_cast<const X*>(q);
+    }
+};
+
+// What each CTA of a group publishes for a row-wide reduction: its partials, read by every
+// CTA of the group after a group barrier. Two areas are used in turn, so that one barrier
+// per exchange suffices (area e is rewritten at exchange e + 2, after every CTA has passed
+// the barrier of exchange e + 1 and so has finished reading it).
+struct Xchg {
+    double mass[256];
+    uint32_t cnt[256];
+    double s;
+    float m;
+    int pad;
+};
+
+// Units of the cluster kernel's balanced passes: vector row j of a chunk, one 16-byte vector
+// per lane (a CTA's slice has at most kMaxUnits of them).
+constexpr int kMaxUnits = 192;
+// Keys of the exact cut histogram (bf16 values: 16-bit keys; 16 per thread of the first 256).
+constexpr int kKeyBins = 4096;
+
+struct RowShared {
+    float hist_f[256 * kWarps];   // per-warp histograms; the group's key counts (as uint32)
+    uint32_t hist_n[256 * kWarps];  // per-warp histograms; this CTA's key counts
+    double comb_m[256];           // the group's histogram; key-mass partial sums
+    uint32_t comb_n[256];
+    double dred[kWarps];
+    float fred[kWarps];
+    float ustat[kMaxUnits];       // per unit: max (then survivor mass)
+    float usum[kMaxUnits];        // per unit: sum of exps
+    int uties[kMaxUnits];         // per unit: tokens equal to the cut
+    Xchg x[2];
+};
+static_assert(kKeyBins <= 256 * kWarps, "key counts live in the histogram arrays");
+
+// ---------------------------------------------------------------------------------------
+// per row: statistics, top-p cut, per-chunk survivor table (a CTA, or a cluster of CTAs each
+// holding a slice of the row)
+// ---------------------------------------------------------------------------------------
+// Chunks [c0, c1) of the row are this CTA's; cmass and cties are indexed by the row's chunk
+// index; info (written if not null) receives the row's RowInfo, which every CTA of the group
+// computes identically (every CTA combines the same partials in the same order). xe counts
+// the exchanges made so far.
+template <typename T, typename Src, typename Grp>
+__device__ void prepare_row(const Src& src, const VerifyArgs& a, int c0, int c1, double* cmass, int* cties,
+                            RowInfo* info, RowShared& sh, const Grp& grp, int& xe) {
     constexpr int NLEVELS = sizeof(T) == 2 ? 2 : 4;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int V = a.V;
     const float invT = 1.0f / a.temperature;
 
+    constexpr bool kSlice = std::is_same<Src, SharedSlice>::value;
+    constexpr int CH = Chunk<T>::CH;
+    const int U = (c1 - c0) * kVecPerLane;  // units of this CTA (slice form)
+
     // 1. per chunk max and sum; row max and sum
     float lmax = -INFINITY;
-    for (int c = warp; c < nchunks; c += kWarps) {
+    if constexpr (kSlice) {
+        // balanced over the warps: unit u = vector row u % 8 of chunk c0 + u / 8
+        for (int u = warp; u < U; u += kWarps) {
+            int nv;
+            const uint4 v = src.load(c0 + u / kVecPerLane, u % kVecPerLane, lane, nv);
+            float m = -INFINITY;
+            if (nv == 8) {
+                const __nv_bfloat162 m2 = __hmax2(__hmax2(as_b2(v.x), as_b2(v.y)), __hmax2(as_b2(v.z), as_b2(v.w)));
+                m = fmaxf(__low2float(m2), __high2float(m2)) * invT;
+            }
+            m = warp_max(m);
+            if (lane == 0) sh.ustat[u] = m;
+        }
+        __syncthreads();
+        for (int u = warp; u < U; u += kWarps) {
+            const float* um = sh.ustat + (u / kVecPerLane) * kVecPerLane;
+            float cm = um[0];
+#pragma unroll
+            for (int k = 1; k < kVecPerLane; ++k) cm = fmaxf(cm, um[k]);
+            int nv;
+            const uint4 v = src.load(c0 + u / kVecPerLane, u % kVecPerLane, lane, nv);
+            float cs = 0.f;
+            if (nv == 8) {
+                float x[8];
+                unpack8(v, x);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) cs += __expf(x[e] * invT - cm);
+            }
+            cs = warp_sum(cs);
+            if (lane == 0) sh.usum[u] = cs;
+        }
+        __syncthreads();
+        for (int c = c0 + threadIdx.x; c < c1; c += kThreads) {
+            const int u0 = (c - c0) * kVecPerLane;
+            float cm = -INFINITY;
+            double cs = 0.0;
+            for (int k = 0; k < kVecPerLane; ++k) {
+                cm = fmaxf(cm, sh.ustat[u0 + k]);
+                cs += (double)sh.usum[u0 + k];
+            }
+            cmass[c] = cs;                             // relative to the chunk max for now
+            reinterpret_cast<float*>(cties)[c] = cm;  // chunk max parked in the ties slot
+            lmax = fmaxf(lmax, cm);
+        }
+    } else
+    for (int c = c0 + warp; c < c1; c += kWarps) {
         float cm = -INFINITY;
         for (int j = 0; j < kVecPerLane; ++j) {
             int nv;
-            uint4 v = load_vec<T>(row, V, c, j, lane, nv);
+            uint4 v = src.load(c, j, lane, nv);
             if constexpr (kIsBf16<T>) {
                 if (nv == 8) {
                     const __nv_bfloat162 m2 = __hmax2(__hmax2(as_b2(v.x), as_b2(v.y)), __hmax2(as_b2(v.z), as_b2(v.w)));
@@ -149,7 +313,7 @@ __device__ void prepare_row(const T* row, const VerifyArgs& a, int nchunks, doub
         float cs = 0.f;
         for (int j = 0; j < kVecPerLane; ++j) {
             int nv;
-            uint4 v = load_vec<T>(row, V, c, j, lane, nv);
+            uint4 v = src.load(c, j, lane, nv);
             if constexpr (kIsBf16<T>) {
                 if (nv == 8) {
                     float x[8];
@@ -168,16 +332,32 @@ __device__ void prepare_row(const T* row, const VerifyArgs& a, int nchunks, doub
         }
         lmax = fmaxf(lmax, cm);
     }
-    const float M = cta_max_f32(lmax, fred);
+    // this CTA's max and its sum relative to it; then the group's M and S
+    const float mc = cta_max_f32(lmax, sh.fred);
     double part = 0.0;
-    for (int c = threadIdx.x; c < nchunks; c += kThreads) {
-        const float cm = reinterpret_cast<float*>(cties)[c];
-        const double m = cmass[c] * exp((double)cm - (double)M);
-        cmass[c] = m;
-        cties[c] = 0;
-        part += m;
+    for (int c = c0 + threadIdx.x; c < c1; c += kThreads)
+        part += cmass[c] * exp((double)reinterpret_cast<float*>(cties)[c] - (double)mc);
+    const double sc = cta_sum_f64(part, sh.dred);
+    float M;
+    double S = 0.0;
+    {
+        Xchg& xo = sh.x[xe++ & 1];
+        if (threadIdx.x == 0) {
+            xo.m = mc;
+            xo.s = sc;
+        }
+        grp.sync();
+        M = -INFINITY;
+        for (int r = 0; r < grp.size(); ++r) M = fmaxf(M, grp.peer(&xo, r)->m);
+        for (int r = 0; r < grp.size(); ++r) {
+            const Xchg* xr = grp.peer(&xo, r);
+            S += xr->s * exp((double)xr->m - (double)M);  // (a CTA without chunks sends 0 and -inf)
+        }
     }
-    const double S = cta_sum_f64(part, dred);
+    for (int c = c0 + threadIdx.x; c < c1; c += kThreads) {
+        cmass[c] = cmass[c] * exp((double)reinterpret_cast<float*>(cties)[c] - (double)M);
+        cties[c] = 0;
+    }
     RowInfo ri{};
     ri.M = M;
     ri.S = S;
@@ -203,21 +383,124 @@ __device__ void prepare_row(const T* row, const VerifyArgs& a, int nchunks, doub
         // (D is a whole number of bins, so that a bin is either binned in full or not at all)
         const double dcut = log((double)V / ((1.0 - (double)a.top_p) * S)) + 0.5;
         float D = dcut > 31.875 ? 31.875f : (dcut < 0.125 ? 0.125f : ceilf((float)dcut * 8.f) * 0.125f);
+        uint32_t tau = 0u;      // key of the cut value
+        double above = 0.0;     // mass of the keys above it
+        uint32_t count_at = 0;  // tokens equal to it (0: no cut, every token survives)
+        bool have_cut = false;
+        if constexpr (kSlice) {
+            // Exact cut from counts per bf16 value: every token with the same value has the same
+            // weight, so the mass of a value is its count times one exp (fp64). The values within
+            // D of the max span at most kKeyBins 16-bit keys unless the range reaches close to 0;
+            // otherwise (or if rounding leaves the target unmet) the histograms below decide.
+            const float hiv = __bfloat162float(__float2bfloat16_ru(M * a.temperature));  // >= the max logit
+            const float lov = __bfloat162float(__float2bfloat16_rd((M - D) * a.temperature));
+            const uint32_t hi16 = float_key(hiv) >> 16, lo16 = float_key(lov) >> 16;
+            const uint32_t R = hi16 >= lo16 ? hi16 - lo16 + 1u : 0u;
+            if (R > 0u && R <= (uint32_t)kKeyBins) {
+                uint32_t* kc = sh.hist_n;                                // this CTA's counts (read by the group)
+                uint32_t* tot = reinterpret_cast<uint32_t*>(sh.hist_f);  // the group's counts
+                auto key_weight = [&](uint32_t k16) {  // exp(value / T - M) of a bf16 key
+                    const uint32_t k = (k16 << 16) | ((k16 & 0x8000u) ? 0x0000u : 0xFFFFu);
+                    return exp((double)key_float(k) / (double)a.temperature - (double)M);
+                };
+                for (int i = threadIdx.x; i < (int)R; i += kThreads) kc[i] = 0u;
+                __syncthreads();
+                const __nv_bfloat162 lo2 = __float2bfloat162_rn(lov);  // lov is a bf16 value
+                const int nvec = c1 > c0 ? (int)((min((int64_t)V, (int64_t)c1 * CH) - (int64_t)c0 * CH) / 8) : 0;
+                for (int i = threadIdx.x; i < nvec; i += kThreads) {
+                    const uint4 v = lds128(src.slice + (size_t)i * 8);
+                    if (!any_ge(v, lo2)) continue;
+                    float x[8];
+                    unpack8(v, x);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const uint32_t k = (float_key(x[e]) >> 16) - lo16;
+                        if (k < R) atomicAdd(&kc[k], 1u);
+                    }
+                }
+                grp.sync();  // every CTA's counts are complete
+                for (int i = threadIdx.x; i < (int)R; i += kThreads) {
+                    uint32_t n = 0;
+                    for (int r = 0; r < grp.size(); ++r) n += grp.peer(kc, r)[i];
+                    tot[i] = n;
+                }
+                __syncthreads();
+                // mass of 16 keys per thread (threads 0..255), from the top key down
+                constexpr int KPT = kKeyBins / 256;
+                if (threadIdx.x < 256) {
+                    double msum = 0.0;
+                    for (int q = 0; q < KPT; ++q) {
+                        const int idx = (int)R - 1 - ((int)threadIdx.x * KPT + q);
+                        if (idx >= 0 && tot[idx]) msum += (double)tot[idx] * key_weight(lo16 + (uint32_t)idx);
+                    }
+                    sh.comb_m[threadIdx.x] = msum;
+                }
+                __syncthreads();
+                if (warp == 0) {
+                    double cum = 0.0, t_excl = 0.0;
+                    int t_hit = -1;
+                    for (int t0 = 0; t0 < 256 && t_hit < 0; t0 += 32) {
+                        const double m = sh.comb_m[t0 + lane];
+                        const double incl = warp_scan_f64(m, lane);
+                        const unsigned hit = __ballot_sync(kFullMask, cum + incl >= target && m > 0.0);
+                        if (hit) {
+                            const int hl = __ffs(hit) - 1;
+                            t_hit = t0 + hl;
+                            t_excl = cum + __shfl_sync(kFullMask, incl - m, hl);
+                        }
+                        cum += __shfl_sync(kFullMask, incl, 31);
+                    }
+                    if (lane == 0) {
+                        // the key within that thread's range where the mass reaches the target
+                        // (the last non-empty one if rounding leaves it a hair short)
+                        int idx_hit = -1;
+                        double ab = 0.0, c = t_excl;
+                        uint32_t n_hit = 0;
+                        for (int q = 0; t_hit >= 0 && q < KPT; ++q) {
+                            const int idx = (int)R - 1 - (t_hit * KPT + q);
+                            if (idx < 0) break;
+                            const uint32_t n = tot[idx];
+                            if (!n) continue;
+                            const double w = (double)n * key_weight(lo16 + (uint32_t)idx);
+                            idx_hit = idx;
+                            ab = c;
+                            n_hit = n;
+                            if (c + w >= target) break;
+                            c += w;
+                        }
+                        sh.dred[0] = ab;
+                        sh.dred[1] = (double)idx_hit;
+                        sh.dred[2] = (double)n_hit;
+                    }
+                }
+                __syncthreads();
+                const int idx_hit = (int)sh.dred[1];
+                if (idx_hit >= 0) {
+                    have_cut = true;
+                    const uint32_t k16 = lo16 + (uint32_t)idx_hit;
+                    tau = (k16 << 16) | ((k16 & 0x8000u) ? 0x0000u : 0xFFFFu);
+                    above = sh.dred[0];
+                    count_at = (uint32_t)sh.dred[2];
+                }
+                __syncthreads();
+            }
+        }
+        if (!have_cut) {
         int vchosen = -1;
         double vabove = 0.0;
         for (int attempt = 0; attempt < 2 && vchosen < 0; ++attempt) {
             if (attempt == 1) D = INFINITY;  // every element
-            for (int i = threadIdx.x; i < 256 * kWarps; i += kThreads) hist_f[i] = 0.f;
+            for (int i = threadIdx.x; i < 256 * kWarps; i += kThreads) sh.hist_f[i] = 0.f;
             __syncthreads();
-            float* hf = hist_f + warp * 256;
+            float* hf = sh.hist_f + warp * 256;
             // packed prefilter: a logit below (M - D) T - 1/16 (rounded down) cannot pass
             const __nv_bfloat162 alo = D == INFINITY
                                            ? __float2bfloat162_rn(-INFINITY)
                                            : __bfloat162bfloat162(__float2bfloat16_rd(((M - D) - 0.0625f) * a.temperature));
-            for (int c = warp; c < nchunks; c += kWarps) {
+            for (int c = c0 + warp; c < c1; c += kWarps) {
                 for (int j = 0; j < kVecPerLane; ++j) {
                     int nv;
-                    uint4 v = load_vec<T>(row, V, c, j, lane, nv);
+                    uint4 v = src.load(c, j, lane, nv);
                     if constexpr (kIsBf16<T>) {
                         if (nv == 8) {
                             if (!any_ge(v, alo)) continue;
@@ -236,37 +519,51 @@ __device__ void prepare_row(const T* row, const VerifyArgs& a, int nchunks, doub
                 }
             }
             __syncthreads();
+            {
+                Xchg& xo = sh.x[xe++ & 1];
+                for (int bin = threadIdx.x; bin < 256; bin += kThreads) {
+                    double m = 0.0;
+                    for (int w = 0; w < kWarps; ++w) m += (double)sh.hist_f[w * 256 + bin];
+                    xo.mass[bin] = m;
+                }
+                grp.sync();
+                for (int bin = threadIdx.x; bin < 256; bin += kThreads) {
+                    double m = 0.0;
+                    for (int r = 0; r < grp.size(); ++r) m += grp.peer(&xo, r)->mass[bin];
+                    sh.comb_m[bin] = m;
+                }
+                __syncthreads();
+            }
             if (warp == 0) {
             double cum = 0.0;
             int chosen = -1;
             double chosen_above = 0.0;
             for (int b0 = 0; b0 < 256 && chosen < 0; b0 += 32) {
                 const int bin = b0 + lane;
-                double m = 0.0;
-                for (int w = 0; w < kWarps; ++w) m += (double)hist_f[w * 256 + bin];
+                const double m = sh.comb_m[bin];
                 const double incl = warp_scan_f64(m, lane);
                 // (a bin whose elements all underflow to 0 cannot be where the mass crosses)
                 const unsigned hit = __ballot_sync(kFullMask, cum + incl >= target && m > 0.0);
                 if (hit) {
-                    const int src = __ffs(hit) - 1;
-                    chosen = b0 + src;
-                    chosen_above = cum + __shfl_sync(kFullMask, incl - m, src);
+                    const int hl = __ffs(hit) - 1;
+                    chosen = b0 + hl;
+                    chosen_above = cum + __shfl_sync(kFullMask, incl - m, hl);
                 }
                 cum += __shfl_sync(kFullMask, incl, 31);
             }
             if (lane == 0) {
-                dred[0] = chosen_above;
-                dred[1] = (double)chosen;
+                sh.dred[0] = chosen_above;
+                sh.dred[1] = (double)chosen;
             }
             }
             __syncthreads();
-            vchosen = (int)dred[1];  // -1: the binned mass falls short of the target
-            vabove = dred[0];
+            vchosen = (int)sh.dred[1];  // -1: the binned mass falls short of the target
+            vabove = sh.dred[0];
             __syncthreads();
         }
         uint32_t prefix = 0;     // key bits fixed so far
-        double above = vchosen >= 0 ? vabove : 0.0;  // mass of keys above the current prefix bin
-        uint32_t count_at = 0;
+        above = vchosen >= 0 ? vabove : 0.0;  // mass of keys above the current prefix bin
+        count_at = 0;
         // packed prefilter of the radix levels: the logits of the chosen bin lie within
         // [(M - (b + 1) / 8) T, (M - b / 8) T], widened by 1/16 and rounded outwards
         const float vlo = (M - (vchosen + 1) * 0.125f - 0.0625f) * a.temperature;
@@ -278,16 +575,16 @@ __device__ void prepare_row(const T* row, const VerifyArgs& a, int nchunks, doub
             const int shift = 24 - 8 * level;
             const uint32_t hi_mask = level == 0 ? 0u : (~0u << (shift + 8));
             for (int i = threadIdx.x; i < 256 * kWarps; i += kThreads) {
-                hist_f[i] = 0.f;
-                hist_n[i] = 0u;
+                sh.hist_f[i] = 0.f;
+                sh.hist_n[i] = 0u;
             }
             __syncthreads();
-            float* hf = hist_f + warp * 256;
-            uint32_t* hn = hist_n + warp * 256;
-            for (int c = warp; c < nchunks; c += kWarps) {
+            float* hf = sh.hist_f + warp * 256;
+            uint32_t* hn = sh.hist_n + warp * 256;
+            for (int c = c0 + warp; c < c1; c += kWarps) {
                 for (int j = 0; j < kVecPerLane; ++j) {
                     int nv;
-                    uint4 v = load_vec<T>(row, V, c, j, lane, nv);
+                    uint4 v = src.load(c, j, lane, nv);
                     if constexpr (kIsBf16<T>) {
                         if (nv == 8) {
                             if (!any_in(v, rlo, rhi)) continue;
@@ -317,7 +614,33 @@ __device__ void prepare_row(const T* row, const VerifyArgs& a, int nchunks, doub
                 }
             }
             __syncthreads();
-            // combine the warps' histograms; walk bins from the top
+            // combine the warps' histograms, then the group's; walk bins from the top
+            {
+                Xchg& xo = sh.x[xe++ & 1];
+                for (int bin = threadIdx.x; bin < 256; bin += kThreads) {
+                    double m = 0.0;
+                    uint32_t n = 0;
+                    for (int w = 0; w < kWarps; ++w) {
+                        m += (double)sh.hist_f[w * 256 + bin];
+                        n += sh.hist_n[w * 256 + bin];
+                    }
+                    xo.mass[bin] = m;
+                    xo.cnt[bin] = n;
+                }
+                grp.sync();
+                for (int bin = threadIdx.x; bin < 256; bin += kThreads) {
+                    double m = 0.0;
+                    uint32_t n = 0;
+                    for (int r = 0; r < grp.size(); ++r) {
+                        const Xchg* xr = grp.peer(&xo, r);
+                        m += xr->mass[bin];
+                        n += xr->cnt[bin];
+                    }
+                    sh.comb_m[bin] = m;
+                    sh.comb_n[bin] = n;
+                }
+                __syncthreads();
+            }
             if (warp == 0) {
                 double cum = above;
                 int chosen = -1;
@@ -325,19 +648,15 @@ __device__ void prepare_row(const T* row, const VerifyArgs& a, int nchunks, doub
                 uint32_t chosen_n = 0;
                 for (int b0 = 255; b0 >= 0 && chosen < 0; b0 -= 32) {
                     const int bin = b0 - lane;
-                    double m = 0.0;
-                    uint32_t n = 0;
-                    for (int w = 0; w < kWarps; ++w) {
-                        m += (double)hist_f[w * 256 + bin];
-                        n += hist_n[w * 256 + bin];
-                    }
+                    const double m = sh.comb_m[bin];
+                    const uint32_t n = sh.comb_n[bin];
                     const double incl = warp_scan_f64(m, lane);
                     const unsigned hit = __ballot_sync(kFullMask, cum + incl >= target && n > 0);
                     if (hit) {
-                        const int src = __ffs(hit) - 1;
-                        chosen = b0 - src;
-                        chosen_above = cum + __shfl_sync(kFullMask, incl - m, src);
-                        chosen_n = __shfl_sync(kFullMask, n, src);
+                        const int hl = __ffs(hit) - 1;
+                        chosen = b0 - hl;
+                        chosen_above = cum + __shfl_sync(kFullMask, incl - m, hl);
+                        chosen_n = __shfl_sync(kFullMask, n, hl);
                     }
                     cum += __shfl_sync(kFullMask, incl, 31);
                 }
@@ -345,28 +664,31 @@ __device__ void prepare_row(const T* row, const VerifyArgs& a, int nchunks, doub
                     chosen = -2;
                 }
                 if (lane == 0) {
-                    dred[0] = chosen_above;
-                    dred[1] = (double)chosen;
-                    dred[2] = (double)chosen_n;
+                    sh.dred[0] = chosen_above;
+                    sh.dred[1] = (double)chosen;
+                    sh.dred[2] = (double)chosen_n;
                 }
             }
             __syncthreads();
-            const int chosen = (int)dred[1];
+            const int chosen = (int)sh.dred[1];
             if (chosen == -2) {
                 prefix = 0;
                 above = 0.0;
                 count_at = 0;
                 break;
             }
-            above = dred[0];
-            count_at = (uint32_t)dred[2];
+            above = sh.dred[0];
+            count_at = (uint32_t)sh.dred[2];
             prefix |= (uint32_t)chosen << shift;
             __syncthreads();
         }
         if (count_at > 0) {
             // the cut value; for bf16 logits the low 16 key bits follow from the sign
-            uint32_t tau = prefix;
+            tau = prefix;
             if (NLEVELS == 2) tau |= (tau & 0x80000000u) ? 0x0000u : 0xFFFFu;
+        }
+        }  // !have_cut
+        if (count_at > 0) {
             const double w_tau = exp((double)key_float(tau) / (double)a.temperature - (double)M);
             double need = (target - above) / w_tau;
             int c_tie = (int)ceil(need - 1e-12);
@@ -376,13 +698,50 @@ __device__ void prepare_row(const T* row, const VerifyArgs& a, int nchunks, doub
             ri.w_tau = w_tau;
             ri.Z = above + (double)c_tie * w_tau;
             // 3. per chunk: mass of keys above tau, and the number of tokens equal to tau
-            for (int c = warp; c < nchunks; c += kWarps) {
+            if constexpr (kSlice) {
+                const __nv_bfloat162 tlo = __float2bfloat162_rn(key_float(tau));  // tau is a bf16 value here
+                for (int u = warp; u < U; u += kWarps) {
+                    int nv;
+                    const uint4 v = src.load(c0 + u / kVecPerLane, u % kVecPerLane, lane, nv);
+                    float mg = 0.f;
+                    int nt = 0;
+                    if (nv == 8 && any_ge(v, tlo)) {
+                        float x[8];
+                        unpack8(v, x);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const uint32_t key = float_key(x[e]);
+                            if (key > tau) mg += __expf(x[e] * invT - M);
+                            nt += key == tau;
+                        }
+                    }
+                    mg = warp_sum(mg);
+                    nt = warp_sum(nt);
+                    if (lane == 0) {
+                        sh.ustat[u] = mg;
+                        sh.uties[u] = nt;
+                    }
+                }
+                __syncthreads();
+                for (int c = c0 + threadIdx.x; c < c1; c += kThreads) {
+                    const int u0 = (c - c0) * kVecPerLane;
+                    double m = 0.0;
+                    int n = 0;
+                    for (int k = 0; k < kVecPerLane; ++k) {
+                        m += (double)sh.ustat[u0 + k];
+                        n += sh.uties[u0 + k];
+                    }
+                    cmass[c] = m;
+                    cties[c] = n;
+                }
+            } else
+            for (int c = c0 + warp; c < c1; c += kWarps) {
                 float mg = 0.f;
                 int nt = 0;
                 const __nv_bfloat162 tlo = __float2bfloat162_rn(key_float(tau));  // tau is a bf16 value here
                 for (int j = 0; j < kVecPerLane; ++j) {
                     int nv;
-                    uint4 v = load_vec<T>(row, V, c, j, lane, nv);
+                    uint4 v = src.load(c, j, lane, nv);
                     if constexpr (kIsBf16<T>) {
                         if (nv == 8) {
                             if (!any_ge(v, tlo)) continue;
@@ -414,7 +773,7 @@ __device__ void prepare_row(const T* row, const VerifyArgs& a, int nchunks, doub
         }
     }
     __syncthreads();
-    if (threadIdx.x == 0) *info = ri;
+    if (threadIdx.x == 0 && info) *info = ri;
     __syncthreads();
 }
 
@@ -633,21 +992,101 @@ __device__ void pair_pass(const T* prow, const T* qrow, const VerifyArgs& a, con
 // ---------------------------------------------------------------------------------------
 // the kernel: one CTA per sequence
 // ---------------------------------------------------------------------------------------
-// One CTA per row (every row of every sequence): the row's chunk table and RowInfo.
+// Row g = b * R + r of the work: verifier rows r < K, then drafter rows 1..K-1.
+template <typename T>
+__device__ __forceinline__ const T* work_row(const VerifyArgs& a, int R, int64_t g) {
+    const int b = (int)(g / R), r = (int)(g % R);
+    const bool isP = r < a.K;
+    const int pos = isP ? r : r - a.K + 1;
+    return reinterpret_cast<const T*>(isP ? a.P : a.Q) + ((int64_t)b * a.K + pos) * a.V;
+}
+
+// One CTA per row (every row of every sequence): the row's chunk table and RowInfo, the
+// row read from global memory (HBM once, then L2) by every pass.
 template <typename T>
 __global__ void __launch_bounds__(kThreads) rows_kernel(Params p) {
-    __shared__ float hist_f[256 * kWarps];
-    __shared__ uint32_t hist_n[256 * kWarps];
-    __shared__ double dred[kWarps];
-    __shared__ float fred[kWarps];
+    __shared__ RowShared sh;
+    const int NC = p.nchunks;
+    const int64_t g = blockIdx.x;
+    int xe = 0;
+    const GlobalRow<T> src{work_row<T>(p.a, p.rows_per_seq, g), p.a.V};
+    prepare_row<T>(src, p.a, 0, NC, p.cmass + g * NC, p.cties + g * NC, p.infos + g, sh, CtaGroup{}, xe);
+}
+
+// Cluster form for bf16 rows whose length is a multiple of 8 (16-byte aligned rows): a
+// cluster of CL CTAs owns one row at a time, CTA r holding chunks [r cpc, (r + 1) cpc) of
+// it in shared memory, so the row is read from HBM exactly once and every pass runs from
+// shared memory; the row-wide reductions go through distributed shared memory (ClusterGroup).
+// Persistent: cluster i takes rows i, i + #clusters, ...; the next row's slice is copied in
+// (one bulk copy per CTA, completion counted on an mbarrier) while this row is processed.
+constexpr int kBulkAlign = 128;
+inline size_t cluster_dyn_smem(int cpc) {
+    return kBulkAlign + 2 * (size_t)cpc * Chunk<__nv_bfloat16>::CH * sizeof(uint16_t);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) rows_cluster_kernel(Params p, int cpc) {
+    extern __shared__ __align__(128) unsigned char dsm[];
+    __shared__ RowShared sh;
+    constexpr int CH = Chunk<__nv_bfloat16>::CH;
     const VerifyArgs& a = p.a;
-    const int K = a.K, V = a.V, NC = p.nchunks, R = p.rows_per_seq;
-    const int64_t g = blockIdx.x;  // b * R + r
-    const int b = (int)(g / R), r = (int)(g % R);
-    const bool isP = r < K;
-    const int pos = isP ? r : r - K + 1;
-    const T* row = reinterpret_cast<const T*>(isP ? a.P : a.Q) + ((int64_t)b * K + pos) * V;
-    prepare_row<T>(row, a, NC, p.cmass + g * NC, p.cties + g * NC, p.infos + g, hist_f, hist_n, dred, fred);
+    const int tid = threadIdx.x;
+    const int rank = (int)cl_rank();
+    const ClusterGroup grp{(int)cl_size()};
+    uint64_t* full = reinterpret_cast<uint64_t*>(dsm);  // [2]: a buffer's slice has landed
+    uint16_t* buf = reinterpret_cast<uint16_t*>(dsm + kBulkAlign);
+    const int64_t buf_elems = (int64_t)cpc * CH;
+    const int V = a.V, NC = p.nchunks, R = p.rows_per_seq;
+    const int c0 = min(NC, rank * cpc), c1 = min(NC, c0 + cpc);
+    const int64_t e_lo = min((int64_t)V, (int64_t)c0 * CH), e_hi = min((int64_t)V, (int64_t)c1 * CH);
+    const uint32_t bytes = (uint32_t)((e_hi - e_lo) * 2);  // a multiple of 16; 0 without chunks
+    const int64_t rows = (int64_t)a.B * R;
+    const int64_t first = cl_index(), step = cl_count();
+    uint32_t issued[2] = {0u, 0u}, done[2] = {0u, 0u};  // copies per buffer (thread 0)
+    if (tid == 0) {
+        mbar_init(&full[0], 1);
+        mbar_init(&full[1], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    auto issue = [&](int64_t g, int bi) {
+        ++issued[bi];
+        if (bytes == 0) {
+            mbar_arrive(&full[bi]);
+            return;
+        }
+        mbar_arrive_expect_tx(&full[bi], bytes);
+        bulk_g2s(buf + bi * buf_elems, work_row<__nv_bfloat16>(a, R, g) + e_lo, bytes, &full[bi]);
+    };
+    bool failed = false;
+    if (tid == 0 && first < rows) issue(first, 0);
+    int xe = 0;
+    int it = 0;
+    for (int64_t g = first; g < rows; g += step, ++it) {
+        const int bi = it & 1;
+        __syncthreads();  // every warp is done with the other buffer (the previous row)
+        if (tid == 0 && !failed && g + step < rows) {
+            fence_proxy_async_smem();
+            issue(g + step, bi ^ 1);
+        }
+        if (!failed) {
+            if (mbar_wait(&full[bi], (uint32_t)(it >> 1) & 1u)) {
+                if (tid == 0) ++done[bi];
+            } else {
+                failed = true;
+                record_device_status(p.status, UNO_ERR_TIMEOUT);
+            }
+        }
+        // (after a timeout the CTA keeps taking part in the cluster's barriers; its results
+        // are not valid, and the status word says so)
+        const SharedSlice src{buf + bi * buf_elems, c0, V};
+        prepare_row<__nv_bfloat16>(src, a, c0, c1, p.cmass + g * NC, p.cties + g * NC,
+                                   rank == 0 ? p.infos + g : nullptr, sh, grp, xe);
+    }
+    // no CTA leaves while another may still read its exchange areas
+    grp.sync();
+    if (tid == 0)  // copies still in flight after a timeout: wait for them (bounded)
+        for (int bi = 0; bi < 2; ++bi)
+            while (done[bi] < issued[bi] && mbar_wait(&full[bi], done[bi] & 1u)) ++done[bi];
 }
 
 template <typename T>
@@ -874,6 +1313,105 @@ inline Layout layout(const VerifyArgs& a) {
     return L;
 }
 
+// Cluster size for the rows: UNO_VERIFY_FULL_CLUSTER (1, 2, 4, 8 or 16) if set, else the
+// smallest size whose two slice buffers fit in shared memory next to RowShared.
+inline bool cluster_fits(int nchunks, int c, size_t room) {
+    const int cpc = (nchunks + c - 1) / c;
+    return cpc * kVecPerLane <= kMaxUnits && cluster_dyn_smem(cpc) <= room;
+}
+inline int choose_cluster(int nchunks, size_t room) {
+    if (const char* e = getenv("UNO_VERIFY_FULL_CLUSTER")) {
+        const int c = atoi(e);
+        if (c == 1 || c == 2 || c == 4 || c == 8 || c == 16) return cluster_fits(nchunks, c, room) ? c : 0;
+    }
+    for (int c = 1; c <= 16; c *= 2)
+        if (cluster_fits(nchunks, c, room)) return c;
+    return 0;
+}
+
+struct ClusterDevice {
+    bool ready = false;
+    size_t dyn_max = 0;  // dynamic shared memory a CTA may use beside the kernel's static part
+    std::map<std::pair<int, size_t>, int> max_clusters;  // (cluster size, dynamic smem) -> co-resident clusters
+};
+std::mutex g_cluster_mu;
+ClusterDevice g_cluster_dev[64];
+
+// Launch rows_cluster_kernel when it applies (bf16, V a multiple of 8, 16-byte aligned
+// logits, a cluster that fits) and UNO_VERIFY_FULL is not "rows"; returns false to fall back
+// to the per-row kernel. UNO_VERIFY_FULL=cluster makes a case that cannot take the cluster
+// form an error (UNO_ERR_UNSUPPORTED) instead of a fallback.
+bool launch_rows_cluster(const Params& p, cudaStream_t stream, uno_status& st) {
+    const VerifyArgs& a = p.a;
+    const char* mode = getenv("UNO_VERIFY_FULL");
+    if (mode && strcmp(mode, "rows") == 0) return false;
+    const bool required = mode && strcmp(mode, "cluster") == 0;
+    auto no = [&](const char* why) {
+        if (required) st = set_error(UNO_ERR_UNSUPPORTED, "verify (full vocabulary): no cluster form: %s", why);
+        return required;
+    };
+    if (a.dtype != UNO_BF16 || a.V % 8 != 0) return no("bf16 rows whose length is a multiple of 8 only");
+    if ((reinterpret_cast<uintptr_t>(a.P) | reinterpret_cast<uintptr_t>(a.Q)) & 15u)
+        return no("logits must be 16-byte aligned");
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return no("no current device");
+    std::lock_guard<std::mutex> lock(g_cluster_mu);
+    ClusterDevice& di = g_cluster_dev[dev];
+    if (!di.ready) {
+        int optin = 0;
+        cudaFuncAttributes fa{};
+        if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+            cudaFuncGetAttributes(&fa, rows_cluster_kernel) != cudaSuccess || optin <= (int)fa.sharedSizeBytes) {
+            cudaGetLastError();
+            return no("shared memory attributes unavailable");
+        }
+        const int dyn_max = optin - (int)fa.sharedSizeBytes;
+        if (cudaFuncSetAttribute(rows_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_max) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(rows_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+                cudaSuccess) {
+            cudaGetLastError();
+            return no("kernel attributes refused");
+        }
+        di.dyn_max = (size_t)dyn_max;
+        di.ready = true;
+    }
+    const int c = choose_cluster(p.nchunks, di.dyn_max);
+    if (c == 0) return no("the row slices do not fit in the shared memory of this cluster size");
+    const int cpc = (p.nchunks + c - 1) / c;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)c;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = cluster_dyn_smem(cpc);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const auto key = std::make_pair(c, cfg.dynamicSmemBytes);
+    int maxc = 0;
+    const auto found = di.max_clusters.find(key);
+    if (found != di.max_clusters.end()) {
+        maxc = found->second;
+    } else {
+        cudaLaunchConfig_t q = cfg;
+        q.gridDim = dim3((unsigned)c);
+        if (cudaOccupancyMaxActiveClusters(&maxc, rows_cluster_kernel, &q) != cudaSuccess) {
+            cudaGetLastError();
+            maxc = 0;
+        }
+        di.max_clusters[key] = maxc;
+    }
+    if (maxc <= 0) return no("no cluster of this size can be resident");
+    const int64_t rows = (int64_t)a.B * p.rows_per_seq;
+    const int64_t clusters = std::min<int64_t>(rows, (int64_t)maxc);
+    cfg.gridDim = dim3((unsigned)(clusters * c));
+    st = check_cuda(cudaLaunchKernelEx(&cfg, rows_cluster_kernel, p, cpc), "launch(verify full rows, cluster)");
+    return true;
+}
+
 }  // namespace vfull
 
 size_t verify_full_workspace_bytes(const VerifyArgs& a) { return vfull::layout(a).total; }
@@ -889,9 +1427,14 @@ uno_status verify_full_launch(const VerifyArgs& a, void* workspace, cudaStream_t
     p.cties = reinterpret_cast<int*>(ws + L.off_cties);
     p.cres = reinterpret_cast<double*>(ws + L.off_cres);
     p.infos = reinterpret_cast<vfull::RowInfo*>(ws + L.off_infos);
+    p.status = device_status_ptr();
     const unsigned rows = (unsigned)((int64_t)a.B * L.rows_per_seq);
     if (a.dtype == UNO_BF16) {
-        vfull::rows_kernel<__nv_bfloat16><<<rows, vfull::kThreads, 0, stream>>>(p);
+        uno_status st = UNO_OK;
+        if (!vfull::launch_rows_cluster(p, stream, st))
+            vfull::rows_kernel<__nv_bfloat16><<<rows, vfull::kThreads, 0, stream>>>(p);
+        else if (st != UNO_OK)
+            return st;
         vfull::seq_kernel<__nv_bfloat16><<<(unsigned)a.B, vfull::kThreads, 0, stream>>>(p);
     } else {
         vfull::rows_kernel<float><<<rows, vfull::kThreads, 0, stream>>>(p);

@@ -258,6 +258,63 @@ def test_full_vocab_ties_and_supplied_tokens():
     assert (gpu["tokens"][:, 0] == pos0).all()
 
 
+CLUSTER_CASES = [
+    (16, 16, 5000, 1.0, 0.95),   # 3 chunks: clusters of 4 and 8 hold CTAs without chunks
+    (16, 16, 5000, 0.8, 1.0),
+    (4, 8, 20000, 1.2, 0.5),     # 10 chunks, a ragged last one
+    (3, 5, 2048, 1.0, 0.9),      # exactly one chunk
+]
+
+
+@pytest.mark.parametrize("cl", [1, 2, 4, 8])
+@pytest.mark.parametrize("case", CLUSTER_CASES, ids=[f"B{c[0]}K{c[1]}V{c[2]}T{c[3]}p{c[4]}" for c in CLUSTER_CASES])
+def test_full_vocab_cluster_kernel(case, cl, monkeypatch):
+    """The cluster form of the full-vocabulary rows pass (each row's slices resident in the
+    shared memory of a CL-CTA cluster, persistent over the rows with the next row copied in
+    while this one is processed) against the oracle, for every cluster size. With
+    UNO_VERIFY_FULL=cluster a case that could not take the cluster form is an error, so
+    these runs cannot pass on the per-row kernel. B (2K - 1) = 496 rows for the first cases:
+    several rows per cluster, so both buffers are reused and their mbarrier phases wrap."""
+    monkeypatch.setenv("UNO_VERIFY_FULL", "cluster")
+    monkeypatch.setenv("UNO_VERIFY_FULL_CLUSTER", str(cl))
+    B, K, V, T, p = case
+    P, Q, u = _inputs(B, K, V, "bf16", seed=zlib.crc32(str((case, cl)).encode()) % 10007)
+    _check_full(P, Q, u, T, p, "bf16")
+
+
+def test_full_vocab_cluster_ties_and_repeatability(monkeypatch):
+    """Heavy ties at the top-p cut (logits on a 1/2 grid) through the cluster form, and the
+    same call twice gives identical outputs (every CTA of a cluster combines the same
+    partials in the same order)."""
+    monkeypatch.setenv("UNO_VERIFY_FULL", "cluster")
+    monkeypatch.setenv("UNO_VERIFY_FULL_CLUSTER", "4")
+    B, K, V = 6, 7, 12000
+    rng = np.random.default_rng(43)
+    Pf = np.round(rng.standard_normal((B, K, V)) * 2) / 2
+    Qf = np.round((0.7 * Pf + 0.7 * rng.standard_normal((B, K, V))) * 2) / 2
+    P, Q = W.bf16_bits(Pf.astype(np.float32)), W.bf16_bits(Qf.astype(np.float32))
+    u = rng.random((B, K, 3), dtype=np.float32)
+    for top_p in (0.9, 0.3):
+        a, _, _ = _check_full(P, Q, u, 1.0, top_p, "bf16")
+        b = verify_gpu(P, Q, u, 1.0, 0, top_p, "bf16")
+        for k in ("tokens", "count", "next"):
+            assert (a[k] == b[k]).all(), k
+
+
+def test_full_vocab_cluster_required_rejects_unaligned(monkeypatch):
+    """V not a multiple of 8 cannot take the cluster form: with UNO_VERIFY_FULL=cluster the
+    call fails with UNO_ERR_UNSUPPORTED (no kernel runs); by default it takes the per-row
+    kernel."""
+    from diffusion_drafted_lossless_b200._lib import UnoError
+    B, K, V = 2, 3, 4099
+    P, Q, u = _inputs(B, K, V, "bf16", seed=5)
+    monkeypatch.setenv("UNO_VERIFY_FULL", "cluster")
+    with pytest.raises(UnoError, match="UNSUPPORTED"):
+        verify_gpu(P, Q, u, 1.0, 0, 0.9, "bf16")
+    monkeypatch.delenv("UNO_VERIFY_FULL")
+    _check_full(P, Q, u, 1.0, 0.9, "bf16")
+
+
 def test_looped_verify_sampled_sequences():
     """B=256, K=8, V=166144 bf16, T=1, top-p 0.95, no top-k (the looped-3B step's verify):
     the whole batch on the GPU, 4 sampled sequences recomputed by the oracle."""
