@@ -264,7 +264,8 @@ def measure_configs(torch, dev, lib, pk, reduce):
     """The other single-GPU configurations of the path, each timed with CUDA events after
     warm-up (inputs resident in HBM, larger than L2): the looped 3B-class step (7 gated
     projections x 22 layers x 2 loops at M = 2048, then the verify at B = 256, K = 8,
-    V = 166144, top-p 0.95) and the TV loss at 16384 x 151936. Inputs are drawn on the
+    V = 166144, top-p 0.95), its one-loop drafting variant (second loop over the 256 verify
+    rows only) and the TV loss at 16384 x 151936. Inputs are drawn on the
     device from a seeded generator with the configurations' distributions."""
     gen = torch.Generator(device=dev)
     bf = torch.bfloat16
@@ -316,7 +317,33 @@ def measure_configs(torch, dev, lib, pk, reduce):
                                           "frac": fl / (ms * 1e-3) / 1e12 / pk["bf16_tflops_sustained"],
                                           "peak": "bf16_tflops_sustained (a seconds-long loop)",
                                           "launches": 7 * W.LOOPED_3B_LAYERS * W.LOOPED_3B_LOOPS}
-    del layers, xs, ys, wss
+    # ---- one-loop drafting: the draft rows leave after the first loop; the verify rows (the
+    # gate-0 rows, laid out first) go through the second loop alone, a prefix of the batch ----
+    n_verify = M - n_gated
+    gate_vf = torch.cat([torch.zeros(n_verify), torch.ones(n_gated)]).to(dev)
+    gate_v = torch.zeros(n_verify, device=dev)
+    ys_v = {sh.name: torch.empty((n_verify, sh.d_out), dtype=bf, device=dev) for sh in w.shapes}
+    wss_v = {sh.name: torch.empty(lib.uno_gated_lora_linear_workspace_size(n_verify, sh.d_in, sh.d_out, w.rank),
+                                  dtype=torch.uint8, device=dev) for sh in w.shapes}
+
+    def one_loop():
+        for lw in layers:
+            for sh, w0, a, b in lw:
+                lib.uno_gated_lora_linear(xs[sh.d_in], w0, a, b, gate_vf, w.scale, ys[sh.name], workspace=wss[sh.name])
+        for lw in layers:
+            for sh, w0, a, b in lw:
+                lib.uno_gated_lora_linear(xs[sh.d_in][:n_verify], w0, a, b, gate_v, w.scale, ys_v[sh.name],
+                                          workspace=wss_v[sh.name])
+
+    ms1 = timed(one_loop, 3)
+    fl1 = W.LOOPED_3B_LAYERS * sum(gemm_flops(sh, M, w.rank, n_gated) + gemm_flops(sh, n_verify, w.rank, 0)
+                                   for sh in w.shapes)
+    out["looped_3b_linears_one_loop_drafting"] = {
+        "ms": ms1, "tflops": fl1 / (ms1 * 1e-3) / 1e12,
+        "frac": fl1 / (ms1 * 1e-3) / 1e12 / pk["bf16_tflops_sustained"],
+        "saving_vs_two_loops": 1.0 - ms1 / ms, "verify_rows": n_verify,
+        "launches": 7 * W.LOOPED_3B_LAYERS * 2}
+    del layers, xs, ys, wss, ys_v, wss_v
     v = W.LOOPED_VERIFY
     P = normal((v.B, v.K, v.V), v.sigma, 9001)
     Q = (v.rho * P.float() + (1 - v.rho ** 2) ** 0.5 * normal((v.B, v.K, v.V), v.sigma, 9002).float()).to(bf)

@@ -101,6 +101,13 @@ __device__ __forceinline__ bool any_in(const uint4& v, __nv_bfloat162 lo, __nv_b
 template <typename T>
 constexpr bool kIsBf16 = sizeof(T) == 2;
 
+// Order-preserving 16-bit keys of the two bf16 values of w (the top 16 bits of float_key of
+// each): h ^ 0x8000 for a value >= +0, ~h for a negative one; -0 is taken as +0 first.
+__device__ __forceinline__ uint32_t bf16x2_keys(uint32_t w) {
+    w &= ~__vcmpeq2(w, 0x80008000u);
+    return w ^ 0x80008000u ^ (((w >> 15) & 0x00010001u) * 0x7FFFu);
+}
+
 __device__ __forceinline__ double cta_sum_f64(double v, double* red) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     v = warp_sum_f64(v);
@@ -211,6 +218,7 @@ struct Xchg {
 // Units of the cluster kernel's balanced passes: vector row j of a chunk, one 16-byte vector
 // per lane (a CTA's slice has at most kMaxUnits of them).
 constexpr int kMaxUnits = 192;
+constexpr int kUB = 4;  // units (or vectors) a warp (thread) works on at a time in the slice passes
 // Keys of the exact cut histogram (bf16 values: 16-bit keys; 16 per thread of the first 256).
 constexpr int kKeyBins = 4096;
 
@@ -224,6 +232,7 @@ struct RowShared {
     float ustat[kMaxUnits];       // per unit: max (then survivor mass)
     float usum[kMaxUnits];        // per unit: sum of exps
     int uties[kMaxUnits];         // per unit: tokens equal to the cut
+    float cmx[kMaxUnits / kVecPerLane];  // per chunk of the slice: max
     Xchg x[2];
 };
 static_assert(kKeyBins <= 256 * kWarps, "key counts live in the histogram arrays");
@@ -251,45 +260,74 @@ __device__ void prepare_row(const Src& src, const VerifyArgs& a, int c0, int c1,
     // 1. per chunk max and sum; row max and sum
     float lmax = -INFINITY;
     if constexpr (kSlice) {
-        // balanced over the warps: unit u = vector row u % 8 of chunk c0 + u / 8
-        for (int u = warp; u < U; u += kWarps) {
-            int nv;
-            const uint4 v = src.load(c0 + u / kVecPerLane, u % kVecPerLane, lane, nv);
-            float m = -INFINITY;
-            if (nv == 8) {
-                const __nv_bfloat162 m2 = __hmax2(__hmax2(as_b2(v.x), as_b2(v.y)), __hmax2(as_b2(v.z), as_b2(v.w)));
-                m = fmaxf(__low2float(m2), __high2float(m2)) * invT;
+        // balanced over the warps: unit u = vector row u % 8 of chunk c0 + u / 8; each warp
+        // takes UB of its units at a time, so that their loads and reductions overlap
+        for (int ub = warp; ub < U; ub += kUB * kWarps) {
+            float m[kUB];
+#pragma unroll
+            for (int k = 0; k < kUB; ++k) {
+                const int u = ub + k * kWarps;
+                m[k] = -INFINITY;
+                if (u < U) {
+                    int nv;
+                    const uint4 v = src.load(c0 + u / kVecPerLane, u % kVecPerLane, lane, nv);
+                    if (nv == 8) {
+                        const __nv_bfloat162 m2 =
+                            __hmax2(__hmax2(as_b2(v.x), as_b2(v.y)), __hmax2(as_b2(v.z), as_b2(v.w)));
+                        m[k] = fmaxf(__low2float(m2), __high2float(m2)) * invT;
+                    }
+                }
             }
-            m = warp_max(m);
-            if (lane == 0) sh.ustat[u] = m;
+#pragma unroll
+            for (int off = 16; off; off >>= 1)
+#pragma unroll
+                for (int k = 0; k < kUB; ++k) m[k] = fmaxf(m[k], __shfl_xor_sync(kFullMask, m[k], off));
+            if (lane == 0)
+#pragma unroll
+                for (int k = 0; k < kUB; ++k)
+                    if (ub + k * kWarps < U) sh.ustat[ub + k * kWarps] = m[k];
         }
         __syncthreads();
-        for (int u = warp; u < U; u += kWarps) {
-            const float* um = sh.ustat + (u / kVecPerLane) * kVecPerLane;
+        for (int c = c0 + threadIdx.x; c < c1; c += kThreads) {
+            const float* um = sh.ustat + (c - c0) * kVecPerLane;
             float cm = um[0];
-#pragma unroll
             for (int k = 1; k < kVecPerLane; ++k) cm = fmaxf(cm, um[k]);
-            int nv;
-            const uint4 v = src.load(c0 + u / kVecPerLane, u % kVecPerLane, lane, nv);
-            float cs = 0.f;
-            if (nv == 8) {
-                float x[8];
-                unpack8(v, x);
+            sh.cmx[c - c0] = cm;
+        }
+        __syncthreads();
+        for (int ub = warp; ub < U; ub += kUB * kWarps) {
+            float cs[kUB];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) cs += __expf(x[e] * invT - cm);
+            for (int k = 0; k < kUB; ++k) {
+                const int u = ub + k * kWarps;
+                cs[k] = 0.f;
+                if (u < U) {
+                    int nv;
+                    const uint4 v = src.load(c0 + u / kVecPerLane, u % kVecPerLane, lane, nv);
+                    if (nv == 8) {
+                        const float cm = sh.cmx[u / kVecPerLane];
+                        float x[8];
+                        unpack8(v, x);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) cs[k] += __expf(x[e] * invT - cm);
+                    }
+                }
             }
-            cs = warp_sum(cs);
-            if (lane == 0) sh.usum[u] = cs;
+#pragma unroll
+            for (int off = 16; off; off >>= 1)
+#pragma unroll
+                for (int k = 0; k < kUB; ++k) cs[k] += __shfl_xor_sync(kFullMask, cs[k], off);
+            if (lane == 0)
+#pragma unroll
+                for (int k = 0; k < kUB; ++k)
+                    if (ub + k * kWarps < U) sh.usum[ub + k * kWarps] = cs[k];
         }
         __syncthreads();
         for (int c = c0 + threadIdx.x; c < c1; c += kThreads) {
             const int u0 = (c - c0) * kVecPerLane;
-            float cm = -INFINITY;
+            const float cm = sh.cmx[c - c0];
             double cs = 0.0;
-            for (int k = 0; k < kVecPerLane; ++k) {
-                cm = fmaxf(cm, sh.ustat[u0 + k]);
-                cs += (double)sh.usum[u0 + k];
-            }
+            for (int k = 0; k < kVecPerLane; ++k) cs += (double)sh.usum[u0 + k];
             cmass[c] = cs;                             // relative to the chunk max for now
             reinterpret_cast<float*>(cties)[c] = cm;  // chunk max parked in the ties slot
             lmax = fmaxf(lmax, cm);
@@ -347,12 +385,17 @@ __device__ void prepare_row(const Src& src, const VerifyArgs& a, int c0, int c1,
             xo.s = sc;
         }
         grp.sync();
-        M = -INFINITY;
-        for (int r = 0; r < grp.size(); ++r) M = fmaxf(M, grp.peer(&xo, r)->m);
-        for (int r = 0; r < grp.size(); ++r) {
-            const Xchg* xr = grp.peer(&xo, r);
-            S += xr->s * exp((double)xr->m - (double)M);  // (a CTA without chunks sends 0 and -inf)
+        // every warp combines the group's partials, lane r taking CTA r's (a CTA without
+        // chunks sends 0 and -inf); the fixed lane order makes the sums identical everywhere
+        float mr = -INFINITY;
+        double sr = 0.0;
+        if (lane < grp.size()) {
+            const Xchg* xr = grp.peer(&xo, lane);
+            mr = xr->m;
+            sr = xr->s;
         }
+        M = warp_max(mr);
+        S = warp_sum_f64(lane < grp.size() ? sr * exp((double)mr - (double)M) : 0.0);
     }
     for (int c = c0 + threadIdx.x; c < c1; c += kThreads) {
         cmass[c] = cmass[c] * exp((double)reinterpret_cast<float*>(cties)[c] - (double)M);
@@ -399,23 +442,32 @@ __device__ void prepare_row(const Src& src, const VerifyArgs& a, int c0, int c1,
             if (R > 0u && R <= (uint32_t)kKeyBins) {
                 uint32_t* kc = sh.hist_n;                                // this CTA's counts (read by the group)
                 uint32_t* tot = reinterpret_cast<uint32_t*>(sh.hist_f);  // the group's counts
-                auto key_weight = [&](uint32_t k16) {  // exp(value / T - M) of a bf16 key
+                auto key_weight = [&](uint32_t k16) {  // a token's weight exp(z - M), for a bf16 key
                     const uint32_t k = (k16 << 16) | ((k16 & 0x8000u) ? 0x0000u : 0xFFFFu);
-                    return exp((double)key_float(k) / (double)a.temperature - (double)M);
+                    return (double)__expf(key_float(k) * invT - M);
                 };
                 for (int i = threadIdx.x; i < (int)R; i += kThreads) kc[i] = 0u;
                 __syncthreads();
                 const __nv_bfloat162 lo2 = __float2bfloat162_rn(lov);  // lov is a bf16 value
                 const int nvec = c1 > c0 ? (int)((min((int64_t)V, (int64_t)c1 * CH) - (int64_t)c0 * CH) / 8) : 0;
-                for (int i = threadIdx.x; i < nvec; i += kThreads) {
-                    const uint4 v = lds128(src.slice + (size_t)i * 8);
-                    if (!any_ge(v, lo2)) continue;
-                    float x[8];
-                    unpack8(v, x);
+                for (int i0 = threadIdx.x; i0 < nvec; i0 += kUB * kThreads) {
+                    uint4 vb[kUB];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const uint32_t k = (float_key(x[e]) >> 16) - lo16;
-                        if (k < R) atomicAdd(&kc[k], 1u);
+                    for (int k = 0; k < kUB; ++k) {
+                        const int i = i0 + k * kThreads;
+                        vb[k] = i < nvec ? lds128(src.slice + (size_t)i * 8) : make_uint4(0u, 0u, 0u, 0u);
+                    }
+#pragma unroll
+                    for (int k = 0; k < kUB; ++k) {
+                        if (i0 + k * kThreads >= nvec || !any_ge(vb[k], lo2)) continue;
+                        const uint32_t w4[4] = {vb[k].x, vb[k].y, vb[k].z, vb[k].w};
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const uint32_t k2 = bf16x2_keys(w4[q]);
+                            const uint32_t ka = (k2 & 0xFFFFu) - lo16, kb = (k2 >> 16) - lo16;
+                            if (ka < R) atomicAdd(&kc[ka], 1u);
+                            if (kb < R) atomicAdd(&kc[kb], 1u);
+                        }
                     }
                 }
                 grp.sync();  // every CTA's counts are complete
@@ -700,27 +752,46 @@ __device__ void prepare_row(const Src& src, const VerifyArgs& a, int c0, int c1,
             // 3. per chunk: mass of keys above tau, and the number of tokens equal to tau
             if constexpr (kSlice) {
                 const __nv_bfloat162 tlo = __float2bfloat162_rn(key_float(tau));  // tau is a bf16 value here
-                for (int u = warp; u < U; u += kWarps) {
-                    int nv;
-                    const uint4 v = src.load(c0 + u / kVecPerLane, u % kVecPerLane, lane, nv);
-                    float mg = 0.f;
-                    int nt = 0;
-                    if (nv == 8 && any_ge(v, tlo)) {
-                        float x[8];
-                        unpack8(v, x);
+                for (int ub = warp; ub < U; ub += kUB * kWarps) {
+                    float mg[kUB];
+                    int nt[kUB];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const uint32_t key = float_key(x[e]);
-                            if (key > tau) mg += __expf(x[e] * invT - M);
-                            nt += key == tau;
+                    for (int k = 0; k < kUB; ++k) {
+                        const int u = ub + k * kWarps;
+                        mg[k] = 0.f;
+                        nt[k] = 0;
+                        if (u < U) {
+                            int nv;
+                            const uint4 v = src.load(c0 + u / kVecPerLane, u % kVecPerLane, lane, nv);
+                            if (nv == 8 && any_ge(v, tlo)) {
+                                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) {
+                                    // IEEE comparisons of bf16 values order them as their keys
+                                    // do (-0 equal to +0)
+                                    const uint32_t gt = __hgt2_mask(as_b2(w4[q]), tlo);
+                                    const uint32_t eq = __heq2_mask(as_b2(w4[q]), tlo);
+                                    if (gt & 0xFFFFu) mg[k] += __expf(bf16_lo(w4[q]) * invT - M);
+                                    if (gt >> 16) mg[k] += __expf(bf16_hi(w4[q]) * invT - M);
+                                    nt[k] += (int)((eq & 1u) + (eq >> 31));
+                                }
+                            }
                         }
                     }
-                    mg = warp_sum(mg);
-                    nt = warp_sum(nt);
-                    if (lane == 0) {
-                        sh.ustat[u] = mg;
-                        sh.uties[u] = nt;
-                    }
+#pragma unroll
+                    for (int off = 16; off; off >>= 1)
+#pragma unroll
+                        for (int k = 0; k < kUB; ++k) {
+                            mg[k] += __shfl_xor_sync(kFullMask, mg[k], off);
+                            nt[k] += __shfl_xor_sync(kFullMask, nt[k], off);
+                        }
+                    if (lane == 0)
+#pragma unroll
+                        for (int k = 0; k < kUB; ++k)
+                            if (ub + k * kWarps < U) {
+                                sh.ustat[ub + k * kWarps] = mg[k];
+                                sh.uties[ub + k * kWarps] = nt[k];
+                            }
                 }
                 __syncthreads();
                 for (int c = c0 + threadIdx.x; c < c1; c += kThreads) {

@@ -91,6 +91,26 @@ def test_full_shapes_sampled_rows(wl, name):
     assert np.isfinite(y).all()
 
 
+@pytest.mark.parametrize("name", ["k", "down"])
+def test_one_loop_drafting_verify_prefix(name):
+    """One-loop drafting's second loop: the looped-3B projections over the 256 verify rows
+    only (gate 0), passed as the first rows of the 2048-row activations (a prefix view),
+    against the oracle's base layer on every row."""
+    wl = W.LOOPED_3B
+    sh = [s for s in wl.shapes if s.name == name][0]
+    inp = W.linear_inputs(wl, sh)
+    n_verify = wl.M // wl.block
+    x = dev(inp["x"], "bf16")[:n_verify]
+    w0, a, b = (dev(inp[k], "bf16") for k in ("w0", "a", "b"))
+    g = torch.zeros(n_verify, device="cuda")
+    y = torch.empty((n_verify, sh.d_out), dtype=torch.bfloat16, device="cuda")
+    _lib.uno_gated_lora_linear(x, w0, a, b, g, wl.scale, y)
+    torch.cuda.synchronize()
+    ref = oracle.gated_lora(W.to_f64(inp["x"], "bf16")[:n_verify], W.to_f64(inp["w0"], "bf16"),
+                            W.to_f64(inp["a"], "bf16"), W.to_f64(inp["b"], "bf16"), np.zeros(n_verify), 2.0)
+    assert _rel(y.float().cpu().numpy(), ref) <= TOL
+
+
 def test_calls_back_to_back_on_one_workspace():
     """Two calls with different gates on the same workspace: the second call's output
     tiles must use its own adapter rows, not the ones the first call left behind."""
