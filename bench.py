@@ -558,6 +558,48 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_kernel_case(args):
+    """One workload alone, for profiling a kernel: `--kernel-case looped_verify` is the
+    looped 3B-class verify (block 8, V = 166144, top-p 0.95, no top-k) at `--case-batch`
+    sequences, called W times as warm-up and then K times; prints the mean time per call
+    as a JSON line (a profiling aid, not a bench line)."""
+    import torch
+    from diffusion_drafted_lossless_b200 import _lib as lib
+    dev = torch.device("cuda", 0)
+    v = W.LOOPED_VERIFY
+    B = args.case_batch
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(9001)
+    P = (torch.randn((B, v.K, v.V), generator=gen, device=dev) * v.sigma).to(torch.bfloat16)
+    gen.manual_seed(9002)
+    noise = torch.randn((B, v.K, v.V), generator=gen, device=dev) * v.sigma
+    Q = (v.rho * P.float() + (1 - v.rho ** 2) ** 0.5 * noise).to(torch.bfloat16)
+    del noise
+    gen.manual_seed(9003)
+    u = torch.rand((B, v.K, 3), generator=gen, device=dev)
+    tok = torch.empty((B, v.K), dtype=torch.int32, device=dev)
+    cnt = torch.empty((B,), dtype=torch.int32, device=dev)
+    nxt = torch.empty((B,), dtype=torch.int32, device=dev)
+    ws = torch.empty(lib.uno_block_verify_workspace_size(B, v.K, v.V, v.top_k, v.top_p), dtype=torch.uint8,
+                     device=dev)
+
+    def call():
+        lib.uno_block_verify(P, Q, v.temperature, v.top_k, v.top_p, u, tok, cnt, nxt, workspace=ws)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(args.steps):
+        call()
+    e.record()
+    torch.cuda.synchronize()
+    print(json.dumps({"kernel_case": args.kernel_case, "batch": B, "calls": args.steps,
+                      "ms_per_call": s.elapsed_time(e) / args.steps,
+                      "device_status": lib.uno_read_device_status()}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -566,7 +608,13 @@ def main():
     ap.add_argument("--impl", choices=["uno", "reference"], default="uno")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-configs", action="store_true", help="skip the other configurations' measurements")
+    ap.add_argument("--kernel-case", choices=["looped_verify"], default=None,
+                    help="run one workload alone (for kernel profiling) instead of the bench")
+    ap.add_argument("--case-batch", type=int, default=32, help="sequences of the --kernel-case workload")
     args = ap.parse_args()
+    if args.kernel_case:
+        run_kernel_case(args)
+        return
     if args.warmup < 3 and args.impl == "uno":
         args.warmup = 3
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:

@@ -61,6 +61,8 @@ struct Params {
     int m_units;                  // row units of the work items: 128 x CG rows
     int splits, per;              // adapter items: m_tiles x splits, `per` K tiles each
     int n_adapter, n_items;       // adapter items, all items
+    int n_tiles;                  // column tiles of the output
+    int ksplit, kper;             // output items per tile (split over K), K tiles of (X, W0) each
     int rb;                       // adapter accumulator width: r rounded up to 16 x CG
     int stages;                   // shared-memory ring depth
     uint32_t b_bytes;             // bytes of one B-operand stage (max(BN, rb) rows)
@@ -68,6 +70,8 @@ struct Params {
     void* y;                      // [M, N] bf16 or fp32
     int out_f32;
     float* tpart;                 // [splits][M][r] fp32 partials (splits > 1)
+    float* ypart;                 // [ksplit][M][N] fp32 partials of the output (ksplit > 1)
+    unsigned long long* otickets; // [m_tiles * n_tiles]: (epoch << 16) | output partials stored
     __nv_bfloat16* t;             // [M][r] bf16 T
     const float* gate;            // [M] or NULL (all zero)
     float scale;
@@ -176,6 +180,7 @@ __device__ __forceinline__ bool take_ticket(unsigned long long* t, unsigned long
 struct Item {
     bool adapter;
     int m, j;    // row unit (128 x CG rows); split (adapter) or column tile (output)
+    int s;       // output: K split (the last one also runs the (T, B) columns)
     int kb, ke;  // K tiles [kb, ke)
 };
 
@@ -185,15 +190,18 @@ __device__ __forceinline__ Item decode(const Params& p, int item) {
         it.adapter = true;
         it.m = item % p.m_units;
         it.j = item / p.m_units;
+        it.s = 0;
         it.kb = it.j * p.per;
         it.ke = min(p.kt0, it.kb + p.per);
     } else {
         const int q = item - p.n_adapter;
         it.adapter = false;
         it.m = q % p.m_units;  // row units fastest: concurrent tiles share W0's column block
-        it.j = q / p.m_units;
-        it.kb = 0;
-        it.ke = p.kt0 + p.kt1;
+        const int js = q / p.m_units;
+        it.s = js % p.ksplit;
+        it.j = js / p.ksplit;
+        it.kb = it.s * p.kper;
+        it.ke = it.s == p.ksplit - 1 ? p.kt0 + p.kt1 : it.kb + p.kper;
     }
     return it;
 }
@@ -446,7 +454,13 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
                     const int col0 = w.j * BN + c0;
                     if (row >= p.M || col0 >= p.N) continue;
                     const int ncol = min(32, p.N - col0);  // a multiple of 32: N is a multiple of 64
-                    if (p.out_f32) {
+                    if (p.ksplit > 1) {  // this split's fp32 partial
+                        float* dst = p.ypart + ((size_t)w.s * p.M + row) * p.N + col0;
+                        for (int j = 0; j < ncol; j += 4)
+                            *reinterpret_cast<float4*>(dst + j) =
+                                make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
+                                            __uint_as_float(r[j + 3]));
+                    } else if (p.out_f32) {
                         float* dst = reinterpret_cast<float*>(p.y) + (size_t)row * p.N + col0;
                         for (int j = 0; j < ncol; j += 4)
                             *reinterpret_cast<float4*>(dst + j) =
@@ -475,6 +489,61 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
                 else mbar_arrive(&tempty[buf]);
             }
 
+            if (!w.adapter && p.ksplit > 1) {
+                // the split that stores a tile's partials last (a ticket) sums them into Y
+                // (all four warps take every barrier)
+                const int tile = (m0 / BM) * p.n_tiles + w.j;
+                __threadfence();
+                named_sync_epilogue();
+                if (et == 0)
+                    s_last = (ok && !*abort_flag && m0 < p.M) ? take_ticket(&p.otickets[tile], p.epoch, p.ksplit) : 0;
+                named_sync_epilogue();
+                if (s_last) {
+                    // four float4 per thread at a time, every split's loads issued together
+                    constexpr int n4 = BN / 4;
+                    const size_t plane = (size_t)p.M * p.N;
+                    for (int idx0 = et; idx0 < BM * n4; idx0 += 4 * kEpiThreads) {
+                        float4 acc[4];
+                        size_t off[4];
+                        bool valid[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int idx = idx0 + u * kEpiThreads;
+                            const int rr = m0 + idx / n4, c = w.j * BN + (idx % n4) * 4;
+                            valid[u] = idx < BM * n4 && rr < p.M && c < p.N;
+                            off[u] = valid[u] ? (size_t)rr * p.N + c : 0;
+                            acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        }
+                        for (int k = 0; k < p.ksplit; ++k) {
+                            float4 v[4];
+#pragma unroll
+                            for (int u = 0; u < 4; ++u)
+                                v[u] = valid[u] ? __ldcg(reinterpret_cast<const float4*>(p.ypart + k * plane + off[u]))
+                                                : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                acc[u].x += v[u].x;
+                                acc[u].y += v[u].y;
+                                acc[u].z += v[u].z;
+                                acc[u].w += v[u].w;
+                            }
+                        }
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            if (!valid[u]) continue;
+                            if (p.out_f32) {
+                                *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.y) + off[u]) = acc[u];
+                            } else {
+                                __nv_bfloat162 h0 = __floats2bfloat162_rn(acc[u].x, acc[u].y);
+                                __nv_bfloat162 h1 = __floats2bfloat162_rn(acc[u].z, acc[u].w);
+                                *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.y) + off[u]) =
+                                    make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
+                            }
+                        }
+                    }
+                }
+                named_sync_epilogue();
+            }
             if (w.adapter) {
                 // publish this CTA's 128 rows of T (all four warps take every barrier)
                 const int tile = m0 / BM;
@@ -572,10 +641,11 @@ uno_status make_tmap(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols
 // The launch plan of one call (also sizes the workspace).
 struct Plan {
     int CG, BN, rb, cb, m_tiles, m_units, n_tiles, kt0, kt1, splits, per, n_adapter, n_items, stages;
+    int ksplit, kper;
     uint32_t b_bytes;
     size_t smem;
     // workspace offsets
-    size_t flags, tickets, t, tpart, x, w0, a, b, total;
+    size_t flags, tickets, t, tpart, ypart, otickets, x, w0, a, b, total;
 };
 
 Plan make_plan(int64_t M, int64_t d_in, int64_t d_out, int64_t rank, uno_dtype dtype) {
@@ -613,7 +683,18 @@ Plan make_plan(int64_t M, int64_t d_in, int64_t d_out, int64_t rank, uno_dtype d
     P.per = (P.kt0 + splits - 1) / splits;
     P.splits = (P.kt0 + P.per - 1) / P.per;
     P.n_adapter = P.m_units * P.splits;
-    P.n_items = P.n_adapter + P.m_units * P.n_tiles;
+    // Output tiles split over K (UNO_LORA_KSPLIT=n, single-CTA tiles only): each split stores
+    // an fp32 partial and the split that finishes a tile last sums them. Meant for small M,
+    // where few tiles leave SMs idle; on the looped-3B shapes at M = 256 it measured slower
+    // (the summing of the partials costs more than the shorter K loops save), so it is off
+    // by default.
+    int ks = 1;
+    if (const char* e = getenv("UNO_LORA_KSPLIT"))
+        if (P.CG == 1) ks = atoi(e);
+    ks = ks < 1 ? 1 : (ks > P.kt0 ? P.kt0 : ks);
+    P.kper = (P.kt0 + ks - 1) / ks;
+    P.ksplit = (P.kt0 + P.kper - 1) / P.kper;  // every split has K tiles of (X, W0); the last also (T, B)
+    P.n_items = P.n_adapter + P.m_units * P.n_tiles * P.ksplit;
     P.b_bytes = (uint32_t)(w / P.CG) * 128u;
     P.stages = (int)((kSmemBudget - 1024) / (A_BYTES + P.b_bytes));
     if (P.stages > kMaxStages) P.stages = kMaxStages;
@@ -628,6 +709,8 @@ Plan make_plan(int64_t M, int64_t d_in, int64_t d_out, int64_t rank, uno_dtype d
     P.tickets = take((size_t)P.m_tiles * 8);
     P.t = take((size_t)M * rank * 2);
     P.tpart = P.splits > 1 ? take((size_t)P.splits * M * rank * 4) : 0;
+    P.ypart = P.ksplit > 1 ? take((size_t)P.ksplit * M * d_out * 4) : 0;
+    P.otickets = P.ksplit > 1 ? take((size_t)P.m_tiles * P.n_tiles * 8) : 0;
     if (dtype == UNO_F32) {
         P.x = take((size_t)M * d_in * 2);
         P.w0 = take((size_t)d_out * d_in * 2);
@@ -758,6 +841,11 @@ uno_status gated_lora_launch(const GatedLoraArgs& g, void* workspace, cudaStream
     p.per = P.per;
     p.n_adapter = P.n_adapter;
     p.n_items = P.n_items;
+    p.n_tiles = P.n_tiles;
+    p.ksplit = P.ksplit;
+    p.kper = P.kper;
+    p.ypart = P.ksplit > 1 ? reinterpret_cast<float*>(ws + P.ypart) : nullptr;
+    p.otickets = P.ksplit > 1 ? reinterpret_cast<unsigned long long*>(ws + P.otickets) : nullptr;
     p.rb = P.rb;
     p.stages = P.stages;
     p.b_bytes = P.b_bytes;

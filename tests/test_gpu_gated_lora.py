@@ -111,6 +111,26 @@ def test_one_loop_drafting_verify_prefix(name):
     assert _rel(y.float().cpu().numpy(), ref) <= TOL
 
 
+@pytest.mark.parametrize("ks", [2, 3, 7])
+def test_output_split_k(monkeypatch, ks):
+    """Output tiles split over K (selected with UNO_LORA_KSPLIT): the fp32 partials are
+    summed by the split that finishes a tile last. Ragged M and N, every rank class, fp32 storage, and
+    two calls in a row (the tickets of the second call must not count the first's)."""
+    monkeypatch.setenv("UNO_LORA_KSPLIT", str(ks))
+    for M, d_in, d_out, r in [(200, 512, 384, 16), (300, 1024, 256, 64), (129, 256, 640, 128)]:
+        w = W.GatedLoraWorkload("t", 177 + M + ks, M=M, block=8, rank=r, scale=2.0,
+                                shapes=(W.LinearShape("t", d_in, d_out),))
+        inp = W.linear_inputs(w, w.shapes[0])
+        ref = _ref(inp)
+        for _ in range(2):
+            assert _rel(_run(inp, M, d_in, d_out, r), ref) <= TOL
+    w = W.TINY_LINEAR
+    sh = w.shapes[0]
+    inp = W.linear_inputs(w, sh)
+    inp16 = dict(inp, dtype="bf16", **{k: W.bf16_bits(inp[k]) for k in ("x", "w0", "a", "b")})
+    assert _rel(_run(inp, w.M, sh.d_in, sh.d_out, w.rank), _ref(inp16)) <= TOL
+
+
 def test_calls_back_to_back_on_one_workspace():
     """Two calls with different gates on the same workspace: the second call's output
     tiles must use its own adapter rows, not the ones the first call left behind."""
