@@ -6,16 +6,22 @@
 // the unfiltered and the top-p-only sampler settings (the LoopUno runs use temperature 1.0
 // and top-p 0.95 without top-k).
 //
-// Two launches. rows_kernel: one CTA per row (verifier rows 0..K-1 and drafter rows 1..K-1
-// of every sequence), which
-//   1. streams the row once and keeps, per chunk of CH elements, the maximum and the sum
-//      of exp(z - max) (z = logit / T); from them the row's max M and sum S;
-//   2. with top-p: finds the exact cut by radix histograms of the probability mass over
-//      the order-preserving key of the logits (bits 31..24, then 23..16, ...: 2 levels
-//      for bf16 logits, 4 for fp32), restricted at each level to the crossing bin. That
-//      gives the cut value tau, the mass above it and how many of the tokens equal to tau
-//      are kept (the lowest ids: ties are ordered by id);
-//   3. stores per chunk the surviving mass and the number of tokens equal to tau.
+// Two launches. The rows pass handles every row (verifier rows 0..K-1 and drafter rows
+// 1..K-1 of every sequence):
+//   1. per chunk of CH elements, the maximum and the sum of exp(z - max) (z = logit / T);
+//      from them the row's max M and sum S;
+//   2. with top-p, the exact cut: the cut value tau, the mass above it and how many of the
+//      tokens equal to tau are kept (the lowest ids: ties are ordered by id);
+//   3. per chunk, the surviving mass and the number of tokens equal to tau.
+// It has two forms. rows_cluster_kernel (bf16 rows, V a multiple of 8): a thread-block
+// cluster per row, each CTA holding a slice of whole chunks in shared memory (one bulk copy,
+// the next row's copied in meanwhile), row-wide reductions through distributed shared
+// memory; the cut comes from counts per bf16 value (one exp per distinct value) where the
+// values near the max span few keys. rows_kernel (any row): one CTA per row reading the row
+// from global memory in every pass; the cut comes from a histogram of the mass over 1/8-nat
+// bins below the max, then radix histograms over the order-preserving logit key (bits
+// 31..24, then 23..16, ...: 2 levels for bf16 logits, 4 for fp32) restricted at each level
+// to the crossing bin.
 // seq_kernel: one CTA per sequence, one warp per block position for the draws, the
 // probabilities and the acceptance, then the whole CTA for the residual and the TV.
 // Draws (inverse CDF over ascending ids) walk the chunk table and then scan one chunk in
