@@ -86,7 +86,14 @@ def _check(status: int) -> None:
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    """Device address of a tensor argument (None passes NULL). The C ABI takes row-major
+    contiguous device memory, so anything else is refused here rather than misread there."""
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or not t.is_contiguous():
+        raise ValueError("tensor arguments must be contiguous CUDA tensors "
+                         f"(got {type(t).__name__}{'' if not isinstance(t, torch.Tensor) else f' on {t.device}, contiguous={t.is_contiguous()}'})")
+    return ctypes.c_void_p(t.data_ptr())
 
 
 def _stream(stream):

@@ -129,3 +129,17 @@ def test_noise_validation(lib):
     assert f(None, FAKE, 2, 4, 100, FAKE, None, None) == _lib.UNO_ERR_INVALID_ARG
     assert f(FAKE + 2, FAKE, 2, 4, 100, FAKE, None, None) == _lib.UNO_ERR_UNSUPPORTED
     assert f(None, None, 0, 4, 100, None, None, None) == _lib.UNO_OK  # B = 0: nothing to do
+
+
+def test_binding_refuses_host_and_strided_tensors(lib):
+    """The binding passes only contiguous CUDA tensors to the C ABI: a host tensor (or a
+    strided view) is refused with ValueError before any library call."""
+    import torch
+    clean = torch.zeros((2, 4), dtype=torch.int32)
+    u = torch.zeros((2, 4), dtype=torch.float32)
+    out = torch.zeros((2, 4), dtype=torch.int32)
+    with pytest.raises(ValueError, match="contiguous CUDA"):
+        _lib.uno_block_noise(clean, u, 100, out)
+    with pytest.raises(ValueError, match="contiguous CUDA"):
+        _lib._ptr(torch.zeros((4, 4))[:, 1])
+    assert _lib._ptr(None) is None
