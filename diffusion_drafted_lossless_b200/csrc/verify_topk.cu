@@ -764,7 +764,6 @@ template <typename T, int KCAP>
 __global__ void __launch_bounds__(FinishCfg<KCAP>::WARPS * 32)
 finish_kernel(Params p, int n_rows) {
     constexpr int FW = FinishCfg<KCAP>::WARPS;
-    constexpr int KB = KeyBits<T>::value;
     extern __shared__ __align__(128) unsigned char smem_raw[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t grow = (int64_t)blockIdx.x * FW + warp;
