@@ -8,7 +8,10 @@ One step = one pass of the whole hot path over one batch of 64 sequences x block
      (bf16, T = 1, top-k 50, top-p 0.95; drafter correlated with the verifier, rho 0.8);
   3. the TV self-distillation loss and its gradient over the same 1024 logit rows
      (teacher = verifier logits, student = drafter logits).
-Metric: verified draft rows per second = 64 * 16 / step time, summed over GPUs.
+Metric: verified draft rows per second = B * K / t_verify, with t_verify the mean time of
+the verify inside the timed steps (CUDA events on the library's stream), summed over GPUs;
+the whole step's rate is reported beside it ("step"), and "e2e" is the whole step through
+the C ABI with every input copied in from pinned host memory and every result copied back.
 
 Inputs are seeded synthetic tensors of those shapes (no weights or datasets); every
 tensor is larger than L2 or read once per step, so no L2 flush is needed.
@@ -40,7 +43,7 @@ UNIT = "rows/s"
 WORKLOAD = "uno_step_b64_k16_v151936_qwen3_8b"
 LINEARS = W.QWEN3_8B
 VERIFY = W.SERVING_VERIFY
-LAUNCHES_PER_STEP = 7 + 3 + 2  # 7 projections (one kernel each) + verify (stream, finish, sequence) + TV (mask, rows)
+LAUNCHES_PER_STEP = 7 + 3 + 2  # 7 projections (one kernel each) + verify (cluster items, generic items, assembly) + TV (mask, rows)
 
 
 def peaks():
@@ -152,16 +155,19 @@ class Step:
     # end to end: host inputs in pinned memory, copied in every step; results copied back
     def setup_host(self):
         torch = self.torch
+
+        def pinned_like(t):
+            return torch.empty(t.shape, dtype=t.dtype, device="cpu").pin_memory()
+
         self.hx = {k: v.pin_memory() for k, v in self.x_host.items()}
         self.hP, self.hQ = self.P_host.pin_memory(), self.Q_host.pin_memory()
         self.hu = self.u.cpu().pin_memory()
-        self.out_tokens = torch.empty_like(self.tokens, device="cpu").pin_memory()
-        self.out_count = torch.empty_like(self.count, device="cpu").pin_memory()
-        self.out_next = torch.empty_like(self.next, device="cpu").pin_memory()
-        self.out_mean = torch.empty_like(self.mean, device="cpu").pin_memory()
+        # every result of the step: the seven projection outputs, the verify's tokens, counts
+        # and correction tokens, the per-token TV, the mean TV and the TV gradient
+        self.d_out = [L["y"] for L in self.lin] + [self.tokens, self.count, self.next, self.tv, self.mean, self.grad]
+        self.h_out = [pinned_like(t) for t in self.d_out]
         self.h2d = sum(t.numel() * t.element_size() for t in list(self.hx.values()) + [self.hP, self.hQ, self.hu])
-        self.d2h = sum(t.numel() * t.element_size() for t in
-                       (self.out_tokens, self.out_count, self.out_next, self.out_mean))
+        self.d2h = sum(t.numel() * t.element_size() for t in self.h_out)
 
     def run_e2e(self):
         for k, h in self.hx.items():
@@ -170,10 +176,8 @@ class Step:
         self.Q.copy_(self.hQ, non_blocking=True)
         self.u.copy_(self.hu, non_blocking=True)
         self.run()
-        self.out_tokens.copy_(self.tokens, non_blocking=True)
-        self.out_count.copy_(self.count, non_blocking=True)
-        self.out_next.copy_(self.next, non_blocking=True)
-        self.out_mean.copy_(self.mean, non_blocking=True)
+        for h, d in zip(self.h_out, self.d_out):
+            h.copy_(d, non_blocking=True)
 
 
 # ---------------------------------------------------------------------------------------
@@ -235,9 +239,11 @@ class ClockSampler:
 # ---------------------------------------------------------------------------------------
 # CPU oracle baseline (bounded sample)
 # ---------------------------------------------------------------------------------------
-def oracle_sample(n_seq=2):
+def oracle_sample(n_seq=2, threads=None):
     """Time the fp64 oracle on a bounded sample of the step: n_seq sequences through the
-    verify, the same n_seq * 16 rows through the seven linears and the TV loss."""
+    verify, the same n_seq * 16 rows through the seven linears and through the TV loss.
+    Returns the headline metric (verify rows per second of the oracle's verify) and the
+    whole-step rate. `threads` sets the oracle's OpenMP thread count for the call."""
     import oracle
     v = VERIFY
     rows = np.arange(n_seq * v.K)
@@ -245,18 +251,28 @@ def oracle_sample(n_seq=2):
     u = W.verify_uniforms(v)[:n_seq]
     lin = [W.linear_inputs(LINEARS, sh, rows=rows) for sh in LINEARS.shapes]
     Pf, Qf = W.to_f64(P, "bf16"), W.to_f64(Q, "bf16")
-    t0 = time.perf_counter()
-    for inp in lin:
-        oracle.gated_lora(W.to_f64(inp["x"], "bf16"), W.to_f64(inp["w0"], "bf16"), W.to_f64(inp["a"], "bf16"),
-                          W.to_f64(inp["b"], "bf16"), inp["gate"].astype(np.float64), inp["scale"])
-    oracle.block_verify(Pf.reshape(n_seq, v.K, v.V), Qf.reshape(n_seq, v.K, v.V), u.astype(np.float64),
-                        v.temperature, v.top_k, float(np.float32(v.top_p)))
-    oracle.tv_loss(Pf, Qf, want_grad=True)
-    dt = time.perf_counter() - t0
+    before = oracle.num_threads()
+    if threads:
+        oracle.set_num_threads(threads)
+    try:
+        t0 = time.perf_counter()
+        oracle.block_verify(Pf.reshape(n_seq, v.K, v.V), Qf.reshape(n_seq, v.K, v.V), u.astype(np.float64),
+                            v.temperature, v.top_k, float(np.float32(v.top_p)))
+        t1 = time.perf_counter()
+        for inp in lin:
+            oracle.gated_lora(W.to_f64(inp["x"], "bf16"), W.to_f64(inp["w0"], "bf16"), W.to_f64(inp["a"], "bf16"),
+                              W.to_f64(inp["b"], "bf16"), inp["gate"].astype(np.float64), inp["scale"])
+        oracle.tv_loss(Pf, Qf, want_grad=True)
+        t2 = time.perf_counter()
+        cores = oracle.num_threads()
+    finally:
+        oracle.set_num_threads(before)
     n_rows = n_seq * v.K
-    return {"value": n_rows / dt, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{n_seq} of 64 sequences ({n_rows} rows) through all three parts of the step; "
-                      f"{dt:.1f} s of fp64 CPU work"}
+    return {"value": n_rows / (t1 - t0), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{n_seq} of 64 sequences ({n_rows} rows): the verify alone gives the value "
+                      f"({t1 - t0:.2f} s); the same rows through the seven linears and the TV loss too "
+                      f"({t2 - t0:.1f} s of fp64 CPU work in all)",
+            "step_rows_per_s": n_rows / (t2 - t0)}
 
 
 # ---------------------------------------------------------------------------------------
@@ -483,7 +499,8 @@ def run_uno(args):
     v, pk = VERIFY, peaks()
     configs = None if args.no_configs else measure_configs(torch, dev, st.lib, pk, max_over_ranks)
     rows = v.B * v.K
-    value = whole_job_rate(rows, world, ms)
+    # the headline: B * K / t_verify (the verify's mean time inside the timed steps)
+    value = whole_job_rate(rows, world, ph["block_verify"])
     gemm_fl = sum(gemm_flops(L["shape"], LINEARS.M, LINEARS.rank, st.n_gated) for L in st.lin)
     # the dominant kernel: the TV kernel is one launch per step (plus a 1-block mask count);
     # the linears are 7 launches (one per projection), the verify 3
@@ -513,7 +530,12 @@ def run_uno(args):
                          "rows_per_s": rows / (ph["block_verify"] * 1e-3)},
         "tv_loss": {"ms": ph["tv_loss"], "gbs": tv_bytes(rows, v.V) / (ph["tv_loss"] * 1e-3) / 1e9},
     }
-    cpu = oracle_sample() if (rank == 0 and world == 1 and not args.no_cpu) else None
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = oracle_sample()
+        one = oracle_sample(n_seq=1, threads=1)
+        cpu["single_thread"] = {"value": one["value"], "cores": one["cores"], "sample": one["sample"],
+                                "step_rows_per_s": one["step_rows_per_s"]}
     mean_count = float(st.count.float().mean().item())
     if rank == 0:
         line = {
@@ -522,13 +544,20 @@ def run_uno(args):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": WORKLOAD, "B": v.B, "K": v.K, "V": v.V, "global_batch": world * rows,
                        "seq_len": v.K, "parallelism": f"dp{world}",
+                       "value": "B*K / mean verify time inside the timed steps (each step: 7 projections, "
+                                "verify, TV loss)",
                        "linears": "Qwen3-8B layer: q,k,v,o,gate,up,down at M=1024, rank 128, scale 2",
                        "verify": "T=1, top-k 50, top-p 0.95, drafts sampled in-kernel",
                        "tv": "1024 rows x 151936, teacher=verifier, student=drafter logits",
                        "l2": "no flush: every input (logits 622 MB, weights 380 MB) exceeds L2 or is read once"},
             "roofline": roof, "phases": phases, "configs": configs, "cpu_baseline": cpu,
+            "step": {"ms": ms, "rows_per_s": whole_job_rate(rows, world, ms),
+                     "what": "the whole step (7 projections + verify + TV loss), device time"},
             "e2e": {"value": world * rows / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": st.h2d,
-                    "d2h_bytes_per_step": st.d2h, "ms_per_step": e2e_ms},
+                    "d2h_bytes_per_step": st.d2h, "ms_per_step": e2e_ms,
+                    "what": "the whole step through the C ABI: activations, logits and uniforms copied in "
+                            "from pinned host memory, every result (projection outputs, tokens, counts, "
+                            "correction tokens, per-token TV, mean TV, TV gradient) copied back"},
             "gpu_launches": LAUNCHES_PER_STEP * args.steps, "clocks": clocks,
             "diagnostics": {"mean_tokens_per_step": mean_count},
         }
@@ -539,52 +568,86 @@ def run_uno(args):
 
 
 def run_reference(args):
-    """The reference arm: the fp64 CPU oracle on the host cores, on bounded samples."""
+    """The reference arm: the fp64 CPU oracle on the host cores, on bounded samples (one
+    sequence per step), measured on this arm's metric: verify rows per second."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     for _ in range(args.warmup):
         oracle_sample(n_seq=1)
-    vals = [oracle_sample(n_seq=1)["value"] for _ in range(args.steps)]
-    base = oracle_sample(n_seq=1)
-    value = float(np.median(vals))
+    runs = [oracle_sample(n_seq=1) for _ in range(args.steps)]
+    value = float(np.median([r["value"] for r in runs]))
+    base = runs[-1]
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 16 / value * 1e3,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": VERIFY.K / value * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "B": 64, "K": 16, "V": 151936, "sample": "1 sequence per step"},
+            "config": {"workload": WORKLOAD, "B": 64, "K": 16, "V": 151936,
+                       "sample": "1 of the 64 sequences per step (16 rows)"},
             "cpu_baseline": dict(base, value=value),
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
 def run_kernel_case(args):
-    """One workload alone, for profiling a kernel: `--kernel-case looped_verify` is the
-    looped 3B-class verify (block 8, V = 166144, top-p 0.95, no top-k) at `--case-batch`
-    sequences, called W times as warm-up and then K times; prints the mean time per call
-    as a JSON line (a profiling aid, not a bench line)."""
+    """One workload alone, for profiling its kernels (a profiling aid, not a bench line):
+      looped_verify   the looped 3B-class verify (block 8, V = 166144, top-p 0.95, no top-k)
+                      at --case-batch sequences;
+      serving_verify  the serving verify (block 16, V = 151936, top-k 50, top-p 0.95) at
+                      --case-batch sequences;
+      qwen3_linears   the seven Qwen3-8B gated projections at M = 1024 (one call = 7 launches);
+      tv_rows         the TV loss and gradient over --case-batch x 16 rows of V = 151936.
+    Runs W warm-up calls and then K calls and prints the mean time per call as JSON."""
     import torch
     from diffusion_drafted_lossless_b200 import _lib as lib
     dev = torch.device("cuda", 0)
-    v = W.LOOPED_VERIFY
-    B = args.case_batch
     gen = torch.Generator(device=dev)
-    gen.manual_seed(9001)
-    P = (torch.randn((B, v.K, v.V), generator=gen, device=dev) * v.sigma).to(torch.bfloat16)
-    gen.manual_seed(9002)
-    noise = torch.randn((B, v.K, v.V), generator=gen, device=dev) * v.sigma
-    Q = (v.rho * P.float() + (1 - v.rho ** 2) ** 0.5 * noise).to(torch.bfloat16)
-    del noise
-    gen.manual_seed(9003)
-    u = torch.rand((B, v.K, 3), generator=gen, device=dev)
-    tok = torch.empty((B, v.K), dtype=torch.int32, device=dev)
-    cnt = torch.empty((B,), dtype=torch.int32, device=dev)
-    nxt = torch.empty((B,), dtype=torch.int32, device=dev)
-    ws = torch.empty(lib.uno_block_verify_workspace_size(B, v.K, v.V, v.top_k, v.top_p), dtype=torch.uint8,
-                     device=dev)
+    bf = torch.bfloat16
 
-    def call():
-        lib.uno_block_verify(P, Q, v.temperature, v.top_k, v.top_p, u, tok, cnt, nxt, workspace=ws)
+    def normal(shape, sigma, seed):
+        gen.manual_seed(seed)
+        return (torch.randn(shape, generator=gen, device=dev) * sigma).to(bf)
+
+    B = args.case_batch
+    if args.kernel_case in ("looped_verify", "serving_verify"):
+        v = W.LOOPED_VERIFY if args.kernel_case == "looped_verify" else W.SERVING_VERIFY
+        P = normal((B, v.K, v.V), v.sigma, 9001)
+        Q = (v.rho * P.float() + (1 - v.rho ** 2) ** 0.5 * normal((B, v.K, v.V), v.sigma, 9002).float()).to(bf)
+        gen.manual_seed(9003)
+        u = torch.rand((B, v.K, 3), generator=gen, device=dev)
+        tok = torch.empty((B, v.K), dtype=torch.int32, device=dev)
+        cnt = torch.empty((B,), dtype=torch.int32, device=dev)
+        nxt = torch.empty((B,), dtype=torch.int32, device=dev)
+        ws = torch.empty(lib.uno_block_verify_workspace_size(B, v.K, v.V, v.top_k, v.top_p), dtype=torch.uint8,
+                         device=dev)
+
+        def call():
+            lib.uno_block_verify(P, Q, v.temperature, v.top_k, v.top_p, u, tok, cnt, nxt, workspace=ws)
+    elif args.kernel_case == "qwen3_linears":
+        w = LINEARS
+        gate = torch.from_numpy(W.row_gate(w.M, w.block)).to(dev)
+        lin = []
+        for i, sh in enumerate(w.shapes):
+            lin.append((normal((w.M, sh.d_in), w.x_sigma, 100 + i), normal((sh.d_out, sh.d_in), w.w_sigma, 200 + i),
+                        normal((w.rank, sh.d_in), w.w_sigma, 300 + i), normal((sh.d_out, w.rank), w.w_sigma, 400 + i),
+                        torch.empty((w.M, sh.d_out), dtype=bf, device=dev),
+                        torch.empty(lib.uno_gated_lora_linear_workspace_size(w.M, sh.d_in, sh.d_out, w.rank),
+                                    dtype=torch.uint8, device=dev)))
+
+        def call():
+            for x, w0, a, b, y, ws in lin:
+                lib.uno_gated_lora_linear(x, w0, a, b, gate, w.scale, y, workspace=ws)
+    else:
+        n, V = B * 16, W.TV_LOSS.V
+        T_ = normal((n, V), 3.0, 9101)
+        S_ = (T_.float() + normal((n, V), 1.0, 9102).float()).to(bf)
+        tv = torch.empty((n,), device=dev)
+        mean = torch.empty((1,), device=dev)
+        grad = torch.empty((n, V), dtype=bf, device=dev)
+        ws = torch.empty(lib.uno_tv_loss_workspace_size(n, V), dtype=torch.uint8, device=dev)
+
+        def call():
+            lib.uno_tv_loss(T_, S_, tv, mean, grad, workspace=ws)
 
     for _ in range(args.warmup):
         call()
@@ -608,7 +671,8 @@ def main():
     ap.add_argument("--impl", choices=["uno", "reference"], default="uno")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-configs", action="store_true", help="skip the other configurations' measurements")
-    ap.add_argument("--kernel-case", choices=["looped_verify"], default=None,
+    ap.add_argument("--kernel-case", choices=["looped_verify", "serving_verify", "qwen3_linears", "tv_rows"],
+                    default=None,
                     help="run one workload alone (for kernel profiling) instead of the bench")
     ap.add_argument("--case-batch", type=int, default=32, help="sequences of the --kernel-case workload")
     args = ap.parse_args()

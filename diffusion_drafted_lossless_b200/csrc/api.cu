@@ -3,6 +3,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "gated_lora.cuh"
@@ -16,12 +17,16 @@ __device__ uint32_t g_device_status = 0u;
 namespace {
 thread_local char t_last_error[512] = "";
 constexpr int kMaxDevices = 64;
+std::mutex g_status_mu;
 uint32_t* g_status_ptr[kMaxDevices] = {};
 }
 
+// The device address of the status word on the current device, looked up once per device
+// (the cache is shared by all host threads, so it is filled under a lock).
 uint32_t* device_status_ptr() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_status_mu);
     if (!g_status_ptr[dev]) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;

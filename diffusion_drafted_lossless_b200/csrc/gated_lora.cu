@@ -77,7 +77,10 @@ struct Params {
     float scale;
     unsigned long long* flags;    // [m_tiles]: the epoch once row tile m's T is written
     unsigned long long* tickets;  // [m_tiles]: (epoch << 16) | partials stored
-    unsigned long long epoch;     // this call's tag, < 2^48, never 0
+    unsigned long long* header;   // [4]: epoch of the next execution, its complement, CTA-exit ticket
+    unsigned long long host_tag;  // lower bound for this execution's epoch (fresh per host call), < 2^48
+    uint32_t flag_polls;          // polls of a T flag before the wait gives up
+    int withhold_flags;           // test switch: adapter items do not publish T (every wait on it runs out)
     uint32_t* status;
 };
 
@@ -150,8 +153,8 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 
 __device__ __forceinline__ void named_sync_epilogue() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory"); }
 
-__device__ __forceinline__ bool wait_flag(const unsigned long long* f, unsigned long long epoch) {
-    for (uint32_t i = 0; i < kFlagPolls; ++i) {
+__device__ __forceinline__ bool wait_flag(const unsigned long long* f, unsigned long long epoch, uint32_t polls) {
+    for (uint32_t i = 0; i < polls; ++i) {
         unsigned long long v;
         asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(f) : "memory");
         if (v == epoch) {
@@ -160,6 +163,16 @@ __device__ __forceinline__ bool wait_flag(const unsigned long long* f, unsigned 
             return true;
         }
         __nanosleep(64);
+    }
+    return false;
+}
+
+// Wait for an mbarrier phase (bounded), giving up early once another role of this CTA has
+// aborted: a role that waits for work the aborted one will never deliver stops at once.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    for (uint32_t i = 0; i < kWaitLimit; i += 256) {
+        if (mbar_wait(bar, parity, 256)) return true;
+        if (*abort_flag) return false;
     }
     return false;
 }
@@ -175,6 +188,34 @@ __device__ __forceinline__ bool take_ticket(unsigned long long* t, unsigned long
     }
     __threadfence();
     return (int)(now & 0xFFFFull) == splits;
+}
+
+constexpr unsigned long long kEpochMask = 0xFFFFFFFFFFFFull;
+
+// This execution's epoch. Each CTA reads the workspace header when it starts, and only the
+// last CTA of the grid to finish advances it (retire_epoch), so all CTAs see the same
+// value. It is the larger of the header's stored value (when its check word matches) and
+// the host's tag, so it is above every epoch this workspace has seen: a CUDA-graph replay, whose host tag is frozen at
+// capture, still gets a fresh epoch, and no flag or ticket left by an earlier execution
+// (or by unrelated data in a fresh workspace, which fails the check) can match it.
+__device__ __forceinline__ unsigned long long read_epoch(const unsigned long long* hdr, unsigned long long host_tag) {
+    const unsigned long long e = __ldcg(hdr), chk = __ldcg(hdr + 1);
+    unsigned long long stored = (chk == ~e) ? (e & kEpochMask) : 0ull;
+    unsigned long long ep = stored > host_tag ? stored : host_tag;
+    return ep == 0 ? 1ull : ep;
+}
+
+// Called once per CTA after all of its work: the last CTA to finish stores epoch + 1 (and
+// its complement) for the next execution on this workspace.
+__device__ __forceinline__ void retire_epoch(unsigned long long* hdr, unsigned long long epoch, int ctas) {
+    __threadfence();
+    if (take_ticket(hdr + 2, epoch, ctas)) {
+        unsigned long long nx = (epoch + 1) & kEpochMask;
+        if (nx == 0) nx = 1;
+        hdr[0] = nx;
+        hdr[1] = ~nx;
+        __threadfence();
+    }
 }
 
 struct Item {
@@ -246,6 +287,11 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
         "h"((unsigned short)3)
         : "memory");
 }
+// arrive on this CTA's mbarrier once the pair's MMAs issued so far complete
+__device__ __forceinline__ void umma_commit_pair_local(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t bar) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
 }
@@ -259,9 +305,10 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
                  const __grid_constant__ CUtensorMap tA, const __grid_constant__ CUtensorMap tT,
                  const __grid_constant__ CUtensorMap tB, Params p) {
     extern __shared__ unsigned char smem_dyn[];
-    __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages], tfull[2], tempty[2];
+    __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages], tfull[2], tempty[2], drain;
     __shared__ uint32_t tmem_holder;
     __shared__ int s_abort, s_last;
+    __shared__ unsigned long long s_epoch;
 
     // 128-byte swizzled tiles need 1024-byte aligned shared-memory addresses
     unsigned char* smem = smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u);
@@ -284,7 +331,9 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
             mbar_init(&tfull[b], 1);
             mbar_init(&tempty[b], CG * kEpiThreads / 32);
         }
+        mbar_init(&drain, 1);
         s_abort = 0;
+        s_epoch = read_epoch(p.header, p.host_tag);
         fence_mbar_init();
     }
     if (warp == 1) {  // two accumulators of cb fp32 columns x 128 lanes (in each CTA of a pair)
@@ -314,6 +363,7 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
     if constexpr (CG == 2) pair_sync();  // the peer's mbarriers exist before any remote arrive
     tmem_fence_after();
     const uint32_t tmem = tmem_holder;
+    const unsigned long long epoch = s_epoch;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -332,7 +382,7 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
                         break;
                     }
                     // rows past M have no T (their loads are zero-filled): nothing to wait for
-                    if (!w.adapter && kt == p.kt0 && m0 < p.M && !wait_flag(&p.flags[m0 / BM], p.epoch)) {
+                    if (!w.adapter && kt == p.kt0 && m0 < p.M && !wait_flag(&p.flags[m0 / BM], epoch, p.flag_polls)) {
                         *abort_flag = 1;
                         break;
                     }
@@ -366,7 +416,7 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
             for (int item = unit0; item < p.n_items && !*abort_flag; item += units, ++li) {
                 const Item w = decode(p, item);
                 const int buf = li & 1;
-                if (li >= 2 && !mbar_wait(&tempty[buf], ((li >> 1) & 1) ^ 1)) {
+                if (li >= 2 && !wait_or_abort(&tempty[buf], ((li >> 1) & 1) ^ 1, abort_flag)) {
                     *abort_flag = 1;
                     break;
                 }
@@ -376,7 +426,7 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
                 bool ok = true;
                 for (int kt = w.kb; kt < w.ke; ++kt, ++g) {
                     const int s = (int)(g % ST);
-                    if (!mbar_wait(&full[s], (g / ST) & 1)) {
+                    if (!wait_or_abort(&full[s], (g / ST) & 1, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -403,6 +453,12 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
                 if constexpr (CG == 2) umma_commit_pair(&tfull[buf]);
                 else umma_commit(&tfull[buf]);
             }
+            if (*abort_flag) {
+                // let every MMA issued so far complete before the accumulators are freed
+                if constexpr (CG == 2) umma_commit_pair_local(&drain);
+                else umma_commit(&drain);
+                mbar_wait(&drain, 0, 1u << 16);
+            }
         }
     } else {
         // ---- epilogue: TMEM -> registers -> global, four warps, one TMEM lane quarter each ----
@@ -415,7 +471,7 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
             const int buf = li & 1;
             const int m0 = w.m * BM * CG + (int)rank * BM;
             const int row = m0 + q * 32 + lane;
-            bool ok = !*abort_flag && mbar_wait(&tfull[buf], (li >> 1) & 1);
+            bool ok = !*abort_flag && wait_or_abort(&tfull[buf], (li >> 1) & 1, abort_flag);
             tmem_fence_after();
             if (!ok) *abort_flag = 1;
             const uint32_t taddr = tmem + (uint32_t)buf * p.cb + ((uint32_t)(q * 32) << 16);
@@ -496,7 +552,7 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
                 __threadfence();
                 named_sync_epilogue();
                 if (et == 0)
-                    s_last = (ok && !*abort_flag && m0 < p.M) ? take_ticket(&p.otickets[tile], p.epoch, p.ksplit) : 0;
+                    s_last = (ok && !*abort_flag && m0 < p.M) ? take_ticket(&p.otickets[tile], epoch, p.ksplit) : 0;
                 named_sync_epilogue();
                 if (s_last) {
                     // four float4 per thread at a time, every split's loads issued together
@@ -552,7 +608,7 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
                 named_sync_epilogue();
                 if (p.splits > 1) {
                     if (et == 0)
-                        s_last = (ok && !*abort_flag && m0 < p.M) ? take_ticket(&p.tickets[tile], p.epoch, p.splits) : 0;
+                        s_last = (ok && !*abort_flag && m0 < p.M) ? take_ticket(&p.tickets[tile], epoch, p.splits) : 0;
                     named_sync_epilogue();
                     if (s_last) {
                         // sum the partials of these 128 rows into T
@@ -579,10 +635,10 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
                         __threadfence();
                     }
                     named_sync_epilogue();
-                    if (et == 0 && s_last)
-                        asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(&p.flags[tile]), "l"(p.epoch) : "memory");
-                } else if (et == 0 && ok && m0 < p.M) {
-                    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(&p.flags[tile]), "l"(p.epoch) : "memory");
+                    if (et == 0 && s_last && !p.withhold_flags)
+                        asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(&p.flags[tile]), "l"(epoch) : "memory");
+                } else if (et == 0 && ok && m0 < p.M && !p.withhold_flags) {
+                    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(&p.flags[tile]), "l"(epoch) : "memory");
                 }
             }
         }
@@ -598,7 +654,10 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
         else
             asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * p.cb) : "memory");
     }
-    if (threadIdx.x == 0 && s_abort) record_device_status(p.status, (uint32_t)UNO_ERR_TIMEOUT);
+    if (threadIdx.x == 0) {
+        if (s_abort) record_device_status(p.status, (uint32_t)UNO_ERR_TIMEOUT);
+        retire_epoch(p.header, epoch, (int)gridDim.x);
+    }
 }
 
 __global__ void f32_to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst, int64_t n) {
@@ -645,7 +704,7 @@ struct Plan {
     uint32_t b_bytes;
     size_t smem;
     // workspace offsets
-    size_t flags, tickets, t, tpart, ypart, otickets, x, w0, a, b, total;
+    size_t header, flags, tickets, t, tpart, ypart, otickets, x, w0, a, b, total;
 };
 
 Plan make_plan(int64_t M, int64_t d_in, int64_t d_out, int64_t rank, uno_dtype dtype) {
@@ -705,6 +764,7 @@ Plan make_plan(int64_t M, int64_t d_in, int64_t d_out, int64_t rank, uno_dtype d
         off = align_up(off + bytes, 256);
         return o;
     };
+    P.header = take(32);
     P.flags = take((size_t)P.m_tiles * 8);
     P.tickets = take((size_t)P.m_tiles * 8);
     P.t = take((size_t)M * rank * 2);
@@ -721,8 +781,8 @@ Plan make_plan(int64_t M, int64_t d_in, int64_t d_out, int64_t rank, uno_dtype d
     return P;
 }
 
-// A fresh tag per call (48 bits, never 0), starting from a time-derived value so that flags
-// left in a reused workspace by another process are not mistaken for this call's.
+// A fresh host tag per call (48 bits, never 0), starting from a time-derived value; the
+// kernel takes the larger of it and the workspace header's stored epoch (read_epoch).
 unsigned long long next_epoch() {
     static std::atomic<unsigned long long> counter{
         (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count() * 2654435761ull};
@@ -858,7 +918,18 @@ uno_status gated_lora_launch(const GatedLoraArgs& g, void* workspace, cudaStream
     p.scale = g.scale;
     p.flags = reinterpret_cast<unsigned long long*>(ws + P.flags);
     p.tickets = reinterpret_cast<unsigned long long*>(ws + P.tickets);
-    p.epoch = next_epoch();
+    p.header = reinterpret_cast<unsigned long long*>(ws + P.header);
+    p.host_tag = next_epoch();
+    // UNO_LORA_TEST_WITHHOLD_FLAGS=1 (tests of the failure path only): the adapter items keep
+    // T to themselves and the output tiles' waits for it give up after a few thousand polls;
+    // the call must then end with UNO_ERR_TIMEOUT in the device status word
+    p.withhold_flags = 0;
+    p.flag_polls = kFlagPolls;
+    if (const char* e = getenv("UNO_LORA_TEST_WITHHOLD_FLAGS"))
+        if (atoi(e) == 1) {
+            p.withhold_flags = 1;
+            p.flag_polls = 4096;
+        }
     p.status = device_status_ptr();
     if (P.CG == 2) return launch_t<256, 2>(maps, p, P, stream);
     switch (P.BN) {

@@ -45,7 +45,7 @@ __device__ __forceinline__ void warp_find_bin(const uint32_t* hist, uint32_t k_r
 
 // Warp scope: returns T such that exactly k of buf[0..n) are >= T (1 <= k <= n).
 // `hist` is 256 words of this warp's shared memory.
-__device__ __noinline__ uint64_t warp_select(const uint64_t* buf, int n, int k, uint32_t* hist, int lane) {
+static __device__ __noinline__ uint64_t warp_select(const uint64_t* buf, int n, int k, uint32_t* hist, int lane) {
     uint64_t prefix = 0;
     uint32_t k_rem = (uint32_t)k;
     for (int shift = 56; shift >= 0; shift -= 8) {
@@ -99,7 +99,7 @@ __device__ __forceinline__ int warp_compact(uint64_t* buf, int n, uint64_t T, in
 // CTA scope (all NT threads call): returns T such that exactly k of v[0..n) are >= T.
 // `hist` is 256 words of shared memory; `bc` is 4 words of shared memory.
 template <int NT>
-__device__ __noinline__ uint64_t cta_select(const uint64_t* v, int n, int k, uint32_t* hist, uint64_t* bc) {
+static __device__ __noinline__ uint64_t cta_select(const uint64_t* v, int n, int k, uint32_t* hist, uint64_t* bc) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint64_t prefix = 0;
     uint32_t k_rem = (uint32_t)k;

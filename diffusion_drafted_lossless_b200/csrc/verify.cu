@@ -1,17 +1,37 @@
-// verify.cu — dispatch of the block verify to the top-k path or the full-vocabulary path.
+// verify.cu — dispatch of the block verify. The item path (verify_full.cu: one thread-block
+// cluster per block position, rows resident in shared memory) takes every top-k-off batch and
+// the top-k batches it supports (bf16 rows whose length is a multiple of 8, 16-byte aligned,
+// k <= 256); the streaming path (verify_topk.cu) takes the other top-k batches.
+// UNO_VERIFY_TOPK=stream sends every top-k batch to the streaming path.
+#include <algorithm>
+#include <cstdlib>
+#include <cstring>
+
 #include "verify_common.cuh"
 
 namespace uno {
 
+static bool topk_stream_forced() {
+    const char* e = getenv("UNO_VERIFY_TOPK");
+    return e && strcmp(e, "stream") == 0;
+}
+
 size_t verify_workspace_bytes(const VerifyArgs& a) {
     if (a.B == 0) return 0;
-    return a.top_k > 0 ? verify_topk_workspace_bytes(a) : verify_full_workspace_bytes(a);
+    if (a.top_k == 0) return verify_full_workspace_bytes(a);
+    return std::max(verify_topk_workspace_bytes(a), verify_full_workspace_bytes(a));
 }
 
 uno_status verify_launch(const VerifyArgs& a, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
     (void)workspace_bytes;
     if (a.B == 0) return UNO_OK;
-    return a.top_k > 0 ? verify_topk_launch(a, workspace, stream) : verify_full_launch(a, workspace, stream);
+    bool taken = false;
+    if (a.top_k == 0) return verify_full_launch(a, workspace, stream, true, &taken);
+    if (!topk_stream_forced()) {
+        const uno_status s = verify_full_launch(a, workspace, stream, false, &taken);
+        if (s != UNO_OK || taken) return s;
+    }
+    return verify_topk_launch(a, workspace, stream);
 }
 
 }  // namespace uno

@@ -1,1523 +1,1731 @@
-// verify_full.cu — lossless block verify without top-k: softmax over the whole
-// vocabulary, optionally followed by top-p.
+// verify_full.cu — lossless block verify without top-k: softmax over the whole vocabulary,
+// optionally followed by top-p, with the top-p cut decided exactly.
 //
-// Same verify rule as the top-k path (LoopUno project page, "How it works" and "Training
-// is self-distillation"; uno-qwen3-8B model card, "Evaluation protocol"); this path serves
-// the unfiltered and the top-p-only sampler settings (the LoopUno runs use temperature 1.0
-// and top-p 0.95 without top-k).
+// The verify rule is the top-k path's (LoopUno project page, "How it works" and "Training is
+// self-distillation"; uno-qwen3-8B model card, "Evaluation protocol"); this path serves the
+// unfiltered and the top-p-only sampler settings (the LoopUno runs use temperature 1.0 and
+// top-p 0.95 without top-k).
 //
-// Two launches. The rows pass handles every row (verifier rows 0..K-1 and drafter rows
-// 1..K-1 of every sequence):
-//   1. per chunk of CH elements, the maximum and the sum of exp(z - max) (z = logit / T);
-//      from them the row's max M and sum S;
-//   2. with top-p, the exact cut: the cut value tau, the mass above it and how many of the
-//      tokens equal to tau are kept (the lowest ids: ties are ordered by id);
-//   3. per chunk, the surviving mass and the number of tokens equal to tau.
-// It has two forms. rows_cluster_kernel (bf16 rows, V a multiple of 8): a thread-block
-// cluster per row, each CTA holding a slice of whole chunks in shared memory (one bulk copy,
-// the next row's copied in meanwhile), row-wide reductions through distributed shared
-// memory; the cut comes from counts per bf16 value (one exp per distinct value) where the
-// values near the max span few keys. rows_kernel (any row): one CTA per row reading the row
-// from global memory in every pass; the cut comes from a histogram of the mass over 1/8-nat
-// bins below the max, then radix histograms over the order-preserving logit key (bits
-// 31..24, then 23..16, ...: 2 levels for bf16 logits, 4 for fp32) restricted at each level
-// to the crossing bin.
-// seq_kernel: one CTA per sequence, one warp per block position for the draws, the
-// probabilities and the acceptance, then the whole CTA for the residual and the TV.
-// Draws (inverse CDF over ascending ids) walk the chunk table and then scan one chunk in
-// id order; probabilities of single tokens need the token's rank among the tau-ties, from
-// the table and a scan of its chunk. The correction token's residual max(0, p - q) and the
-// optional TV take one more pass over the two rows involved.
-// Sums are fp32 within a chunk and fp64 across chunks.
+// Work is split by block position. Item (b, i) owns the verifier row P_i and, for i >= 1, the
+// drafter row Q_i of sequence b, and everything it decides depends on those rows alone:
+//   i = 0:  x_0 (drawn from P_0 unless supplied) and P_0(x_0);
+//   i >= 1: d_i (drawn from Q_i unless supplied), P_i(d_i), Q_i(d_i), the acceptance test
+//           u * Q_i(d_i) < P_i(d_i), TV(P_i, Q_i), and a draw from the residual
+//           normalise(max(0, P_i - Q_i)) with the position's resample uniform, which is the
+//           correction token if i turns out to be the first rejection.
+// Items write small records; assemble_kernel then takes each sequence's longest accepted
+// prefix. Nothing waits on another item.
+//
+// Exact cut. With bf16 logits a row is fixed by how many tokens hold each 16-bit value, so
+// every mass the verify needs is a sum over distinct values of count * exp(value / T - max),
+// one fp64 exp per distinct value rather than one per token. pair_kernel counts the values
+// whose magnitude lies within 2048 bf16 steps of the row's largest magnitude (both signs: all
+// but tiny magnitudes); the few tokens below that band have their fp64 weights summed one by
+// one. The cut is then the value at which the mass from the top first reaches top_p * S, and
+// the ties at that value are kept lowest id first, as the sorted order (probability desc, id
+// asc) keeps them. Sums run in fp64 in a different order from a sequential sum, so results
+// agree with an exact evaluation up to fp64 rounding.
+//
+// pair_kernel (bf16, V a multiple of 8, 16-byte aligned logits): a thread-block cluster of CL
+// CTAs owns an item at a time, CTA r holding elements [r L, (r + 1) L) of both rows in shared
+// memory (one bulk copy per row, so each row crosses HBM once). Each CTA runs two teams of
+// eight warps on alternate items, so one team computes while the other waits for its copy or
+// for a cluster exchange. Per item and team: (1) the largest value and magnitude of each row;
+// (2) the per-value counts; (3) each CTA sums the cluster's counts for its share of the values
+// and their masses; (4) every CTA finds the same cut from the exchanged masses; (5) the CTA
+// holding the boundary among the tied tokens finds it; (6) one pass over the rows sums, per
+// warp part, the masses the draws walk (drafter survivors, verifier survivors, residual);
+// (7) the CTAs that hold the drawn tokens find them. Exchanges are one-sided: each CTA stores
+// its partials into every CTA's shared memory and arrives on that CTA's mbarrier.
+// item_generic_kernel (any dtype and layout, and any item pair_kernel could not decide, e.g.
+// a cut among the tiny-magnitude tokens): one CTA per item reading the rows from global
+// memory in every pass, an fp64 exp per token, the cut by radix selection over the
+// order-preserving 32-bit keys with fp64 masses per bin.
+// Every wait is bounded; on timeout a kernel records UNO_ERR_TIMEOUT and stops.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+#include <climits>
 #include <cstdlib>
 #include <cstring>
 #include <map>
+#include <tuple>
 #include <mutex>
-#include <type_traits>
 
+#include "select.cuh"
 #include "verify_common.cuh"
 
 namespace uno {
 namespace vfull {
 
-constexpr int kWarps = 16;
-constexpr int kThreads = kWarps * 32;
-constexpr int kVecPerLane = 8;  // 16-byte vectors per lane per chunk
-
-struct RowInfo {
-    float M;        // max of z = logit / T
-    int c_tie;      // number of tokens equal to tau that survive (top-p)
-    uint32_t tau;   // key of the cut value (0: no cut, every token survives)
-    int pad;
-    double S;       // sum exp(z - M) over the row
-    double Z;       // surviving mass (sum over survivors of exp(z - M))
-    double w_tau;   // exp(z_tau - M)
+// One record per item (b, i).
+struct Rec {
+    int32_t tok;    // x_0 (i = 0) or d_i
+    int32_t res;    // residual draw (i >= 1), -1 at i = 0
+    int32_t acc;    // acceptance of d_i (1 at i = 0)
+    int32_t state;  // kDone, or kRedo for the generic kernel
+    double p, q;    // P_i(tok), Q_i(tok) (q = 0 at i = 0)
+    double tv;      // TV(P_i, Q_i) (0 at i = 0)
+    double pad;
 };
+static_assert(sizeof(Rec) == 48, "record layout");
+constexpr int32_t kDone = 1, kRedo = 2;
 
 struct Params {
-    VerifyArgs a;
-    int rows_per_seq;
-    int nchunks;
-    double* cmass;    // [B * rows_per_seq * nchunks] surviving mass per chunk (rel. to M)
-    int* cties;       // [B * rows_per_seq * nchunks] tokens equal to tau per chunk
-    double* cres;     // [B * nchunks] scratch: residual mass per chunk
-    RowInfo* infos;   // [B * rows_per_seq]
-    uint32_t* status; // device status word (bounded waits that give up)
+    const void* P;
+    const void* Q;
+    int B, K, V;
+    double T;       // temperature
+    double top_p;   // used when cut != 0
+    int cut;        // top-p < 1
+    int top_k;      // 0: off
+    int need_p0;    // P_0(x_0) is an output: P_0 is needed even when x_0 is supplied
+    const int32_t* drafts;
+    const int32_t* pos0;
+    const float* u;
+    Rec* recs;
+    uint32_t* status;
 };
 
-template <typename T>
-struct Chunk {
-    static constexpr int VEC = Elem<T>::VEC;
-    static constexpr int CH = 32 * VEC * kVecPerLane;  // elements per chunk
+__device__ __forceinline__ bool pos0_given(const Params& p, int b) { return p.pos0 && p.pos0[b] >= 0; }
+// an item with nothing to compute: x_0 supplied and P_0(x_0) not wanted
+__device__ __forceinline__ bool trivial_item(const Params& p, int b, int i) {
+    return i == 0 && pos0_given(p, b) && !p.need_p0;
+}
+__device__ __forceinline__ void write_trivial(const Params& p, int item, int b) {
+    Rec r;
+    r.tok = p.pos0[b];
+    r.res = -1;
+    r.acc = 1;
+    r.state = kDone;
+    r.p = 0.0;
+    r.q = 0.0;
+    r.tv = 0.0;
+    r.pad = 0.0;
+    p.recs[item] = r;
+}
+
+// =======================================================================================
+// generic kernel: one CTA per item, rows read from global memory in every pass
+// =======================================================================================
+namespace gen {
+
+constexpr int kThreads = 1024;
+constexpr int kWarps = kThreads / 32;
+
+template <typename TL>
+__device__ __forceinline__ float val(const TL* row, int v);
+template <>
+__device__ __forceinline__ float val<__nv_bfloat16>(const __nv_bfloat16* row, int v) {
+    return __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(row)[v] << 16);
+}
+template <>
+__device__ __forceinline__ float val<float>(const float* row, int v) {
+    return row[v];
+}
+
+struct Row {
+    double zmax;     // max of logit / T
+    double Sk;       // surviving mass: sum over survivors of exp(logit / T - zmax)
+    uint32_t kap_k;  // top-k: tokens with a larger order key survive it, and those with this key
+    int th_k;        //   and an id below th_k (kap_k = 0: top-k off)
+    uint32_t kap_p;  // top-p within the top-k survivors, the same way (kap_p = 0: top-p off)
+    int th_p;
 };
 
-// element (vector j, lane, slot e) of chunk c in id order: c*CH + j*32*VEC + lane*VEC + e
-template <typename T>
-__device__ __forceinline__ uint4 load_vec(const T* row, int V, int c, int j, int lane, int& nv) {
-    constexpr int VEC = Elem<T>::VEC;
-    const int64_t e0 = (int64_t)c * Chunk<T>::CH + (int64_t)j * 32 * VEC + lane * VEC;
-    nv = (int)max((int64_t)0, min((int64_t)VEC, (int64_t)V - e0));
-    const bool aligned = ((reinterpret_cast<uintptr_t>(row + e0) & 15u) == 0);
-    return nv > 0 ? load_raw<T>(row, e0, nv, aligned && nv == VEC) : make_uint4(0, 0, 0, 0);
-}
+struct Shared {
+    double red[kWarps];
+    float fred[kWarps];
+    int ired[kWarps];
+    double binm[256];
+    unsigned binc[256];
+    int sel, sel2, mode;
+    double dsel;
+};
 
-// Full bf16 vectors: the 8 elements in id order, and packed tests that let a vector whose
-// elements cannot pass a pass's test skip the per-element work (the exact test still
-// decides every element of a vector that is not skipped).
-__device__ __forceinline__ void unpack8(const uint4& v, float (&x)[8]) {
-    x[0] = bf16_lo(v.x); x[1] = bf16_hi(v.x); x[2] = bf16_lo(v.y); x[3] = bf16_hi(v.y);
-    x[4] = bf16_lo(v.z); x[5] = bf16_hi(v.z); x[6] = bf16_lo(v.w); x[7] = bf16_hi(v.w);
-}
-__device__ __forceinline__ __nv_bfloat162 as_b2(uint32_t w) { return *reinterpret_cast<__nv_bfloat162*>(&w); }
-// some element >= lo
-__device__ __forceinline__ bool any_ge(const uint4& v, __nv_bfloat162 lo) {
-    const __nv_bfloat162 m = __hmax2(__hmax2(as_b2(v.x), as_b2(v.y)), __hmax2(as_b2(v.z), as_b2(v.w)));
-    return __hge2_mask(m, lo) != 0u;
-}
-// some element in [lo, hi]
-__device__ __forceinline__ bool any_in(const uint4& v, __nv_bfloat162 lo, __nv_bfloat162 hi) {
-    const uint32_t m = (__hge2_mask(as_b2(v.x), lo) & __hle2_mask(as_b2(v.x), hi)) |
-                       (__hge2_mask(as_b2(v.y), lo) & __hle2_mask(as_b2(v.y), hi)) |
-                       (__hge2_mask(as_b2(v.z), lo) & __hle2_mask(as_b2(v.z), hi)) |
-                       (__hge2_mask(as_b2(v.w), lo) & __hle2_mask(as_b2(v.w), hi));
-    return m != 0u;
-}
-template <typename T>
-constexpr bool kIsBf16 = sizeof(T) == 2;
-
-// Order-preserving 16-bit keys of the two bf16 values of w (the top 16 bits of float_key of
-// each): h ^ 0x8000 for a value >= +0, ~h for a negative one; -0 is taken as +0 first.
-__device__ __forceinline__ uint32_t bf16x2_keys(uint32_t w) {
-    w &= ~__vcmpeq2(w, 0x80008000u);
-    return w ^ 0x80008000u ^ (((w >> 15) & 0x00010001u) * 0x7FFFu);
-}
-
-__device__ __forceinline__ double cta_sum_f64(double v, double* red) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+__device__ double block_sum(double v, Shared& s) {
     v = warp_sum_f64(v);
     __syncthreads();
-    if (lane == 0) red[warp] = v;
+    if ((threadIdx.x & 31) == 0) s.red[threadIdx.x >> 5] = v;
     __syncthreads();
     double t = 0.0;
-    for (int w = 0; w < kWarps; ++w) t += red[w];
-    __syncthreads();
+    for (int w = 0; w < kWarps; ++w) t += s.red[w];  // same order in every thread
     return t;
 }
 
-__device__ __forceinline__ float cta_max_f32(float v, float* red) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+__device__ float block_max(float v, Shared& s) {
     v = warp_max(v);
     __syncthreads();
-    if (lane == 0) red[warp] = v;
+    if ((threadIdx.x & 31) == 0) s.fred[threadIdx.x >> 5] = v;
     __syncthreads();
     float t = -INFINITY;
-    for (int w = 0; w < kWarps; ++w) t = fmaxf(t, red[w]);
-    __syncthreads();
+    for (int w = 0; w < kWarps; ++w) t = fmaxf(t, s.fred[w]);
     return t;
 }
 
-// ---------------------------------------------------------------------------------------
-// where a row's elements come from, and which CTAs share the work of a row
-// ---------------------------------------------------------------------------------------
-// The whole row in global memory (per-row kernel).
-template <typename T>
-struct GlobalRow {
-    const T* row;
-    int V;
-    __device__ __forceinline__ uint4 load(int c, int j, int lane, int& nv) const {
-        return load_vec<T>(row, V, c, j, lane, nv);
+__device__ __forceinline__ bool in_topk(const Row& r, uint32_t key, int v) {
+    return key > r.kap_k || (key == r.kap_k && v < r.th_k);
+}
+__device__ __forceinline__ bool survives(const Row& r, uint32_t key, int v) {
+    return in_topk(r, key, v) && (key > r.kap_p || (key == r.kap_p && v < r.th_p));
+}
+
+// Radix selection over the order-preserving 32-bit keys of the tokens `in(v, key)`, 8 bits at
+// a time from the top: the largest key at which the running total of amount(v, x) from the
+// top reaches `target`. Returns the key, the total of the tokens strictly above it and how
+// many tokens hold it. If rounding leaves the target unmet, the smallest key present.
+template <typename TL, typename In, typename Amt>
+__device__ void radix_select(const TL* row, int V, In in, Amt amount, double target, Shared& s, uint32_t& key,
+                             double& above, unsigned& count) {
+    const int tid = threadIdx.x;
+    uint32_t prefix = 0u, mask = 0u;
+    double cb = 0.0;
+    unsigned cnt = 0;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int j = tid; j < 256; j += kThreads) {
+            s.binm[j] = 0.0;
+            s.binc[j] = 0u;
+        }
+        __syncthreads();
+        for (int v = tid; v < V; v += kThreads) {
+            const float x = val(row, v);
+            const uint32_t k = float_key(x);
+            if ((k & mask) == prefix && in(v, k)) {
+                const int bin = (int)((k >> shift) & 0xFFu);
+                atomicAdd(&s.binm[bin], amount(v, x));
+                atomicAdd(&s.binc[bin], 1u);
+            }
+        }
+        __syncthreads();
+        if (tid == 0) {
+            double c = cb;
+            int bin = -1;
+            for (int j = 255; j >= 0; --j) {
+                if (s.binc[j] == 0u) continue;
+                if (c + s.binm[j] >= target) {
+                    bin = j;
+                    break;
+                }
+                c += s.binm[j];
+            }
+            if (bin < 0) {
+                for (int j = 0; j < 256 && bin < 0; ++j)
+                    if (s.binc[j]) bin = j;
+                c = cb;
+                for (int j = 255; j > bin; --j) c += s.binm[j];
+            }
+            s.sel = bin;
+            s.dsel = c;
+        }
+        __syncthreads();
+        const int bin = s.sel;
+        cb = s.dsel;
+        cnt = s.binc[bin];
+        prefix |= (uint32_t)bin << shift;
+        mask |= 0xFFu << shift;
+        __syncthreads();
     }
+    key = prefix;
+    above = cb;
+    count = cnt;
+}
+
+// The id of the t-th (1-based, id order) token with `in(v, key)` and this key.
+template <typename TL, typename In>
+__device__ int tie_id(const TL* row, int V, In in, uint32_t key, long long t, Shared& s) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int seg = (V + kWarps - 1) / kWarps;
+    const int v0 = warp * seg, v1 = min(V, v0 + seg);
+    int c = 0;
+    for (int v = v0 + lane; v < v1; v += 32) {
+        const uint32_t k = float_key(val(row, v));
+        c += (k == key && in(v, k));
+    }
+    c = warp_sum(c);
+    __syncthreads();
+    if (lane == 0) s.ired[warp] = c;
+    __syncthreads();
+    if (tid == 0) {
+        long long before = 0;
+        int w = 0;
+        for (; w < kWarps; ++w) {
+            if (before + s.ired[w] >= t) break;
+            before += s.ired[w];
+        }
+        s.sel = w;
+        s.sel2 = (int)(t - before);  // rank within that warp's part (1-based)
+    }
+    __syncthreads();
+    if (warp == s.sel) {
+        int need = s.sel2, found = -1;
+        for (int base = v0; base < v1 && found < 0; base += 32) {
+            const int v = base + lane;
+            bool hit = false;
+            if (v < v1) {
+                const uint32_t k = float_key(val(row, v));
+                hit = k == key && in(v, k);
+            }
+            const unsigned bal = __ballot_sync(kFullMask, hit);
+            const int nb = __popc(bal);
+            if (nb >= need) {
+                unsigned b = bal;
+                for (int q = 1; q < need; ++q) b &= b - 1;
+                found = base + __ffs(b) - 1;
+            }
+            need -= nb;
+        }
+        if (lane == 0) s.sel = found;
+    }
+    __syncthreads();
+    const int id = s.sel;
+    __syncthreads();
+    return id;
+}
+
+// Row statistics, the top-k cut and the top-p cut of one row.
+template <typename TL>
+__device__ void row_stats(const TL* row, const Params& p, Shared& s, Row& out) {
+    const int V = p.V, tid = threadIdx.x;
+    float m = -INFINITY;
+    for (int v = tid; v < V; v += kThreads) m = fmaxf(m, val(row, v));
+    m = block_max(m, s);
+    Row r;
+    r.zmax = (double)m / p.T;  // the largest logit survives both cuts
+    r.kap_k = 0u;
+    r.th_k = INT_MAX;
+    r.kap_p = 0u;
+    r.th_p = INT_MAX;
+    const double zmax = r.zmax, T = p.T;
+    auto all = [&](int, uint32_t) { return true; };
+    if (p.top_k > 0) {
+        // the k largest values, ties to the lower id
+        uint32_t key;
+        double above;
+        unsigned cnt;
+        radix_select(row, V, all, [](int, float) { return 1.0; }, (double)p.top_k, s, key, above, cnt);
+        long long t = (long long)p.top_k - (long long)above;
+        if (t < 1) t = 1;
+        if (t > (long long)cnt) t = cnt;
+        r.kap_k = key;
+        if (t < (long long)cnt) r.th_k = tie_id(row, V, all, key, t, s) + 1;
+    }
+    const Row rk = r;
+    auto in_k = [&](int v, uint32_t k) { return in_topk(rk, k, v); };
+    double acc = 0.0;
+    for (int v = tid; v < V; v += kThreads) {
+        const float x = val(row, v);
+        if (in_topk(r, float_key(x), v)) acc += exp((double)x / T - zmax);
+    }
+    const double S = block_sum(acc, s);
+    r.Sk = S;
+    if (p.cut) {
+        // the mass from the top first reaches top_p * S: the fewest (at least one) of the
+        // tokens at that value, lowest ids first, that bring it there
+        const double target = p.top_p * S;
+        uint32_t key;
+        double cb;
+        unsigned cnt;
+        radix_select(row, V, in_k, [&](int, float x) { return exp((double)x / T - zmax); }, target, s, key, cb, cnt);
+        const double wk = exp((double)key_float(key) / T - zmax);
+        long long t = (long long)ceil((target - cb) / wk);
+        if (t < 1) t = 1;
+        if (t > (long long)cnt) t = cnt;
+        while (t > 1 && cb + (double)(t - 1) * wk >= target) --t;
+        while (t < (long long)cnt && cb + (double)t * wk < target) ++t;
+        r.kap_p = key;
+        r.Sk = cb + (double)t * wk;
+        if (t < (long long)cnt) r.th_p = tie_id(row, V, in_k, key, t, s) + 1;
+    }
+    out = r;
+}
+
+template <typename TL>
+__device__ __forceinline__ double kept_weight(const TL* row, const Row& r, const Params& p, int v) {
+    const float x = val(row, v);
+    return survives(r, float_key(x), v) ? exp((double)x / p.T - r.zmax) : 0.0;
+}
+
+// Inverse-CDF draw over ascending ids: the first id whose cumulative weight exceeds target;
+// if rounding leaves no crossing, the last id with positive weight. -1 if no weight at all.
+template <typename F>
+__device__ int draw(int V, double target, F wfn, Shared& s) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int seg = (V + kWarps - 1) / kWarps;
+    const int v0 = warp * seg, v1 = min(V, v0 + seg);
+    double part = 0.0;
+    for (int v = v0 + lane; v < v1; v += 32) part += wfn(v);
+    part = warp_sum_f64(part);
+    __syncthreads();
+    if (lane == 0) s.red[warp] = part;
+    __syncthreads();
+    if (tid == 0) {
+        double c = 0.0, clast = 0.0;
+        int wd = -1, last = -1;
+        for (int w = 0; w < kWarps; ++w) {
+            if (!(s.red[w] > 0.0)) continue;
+            last = w;
+            clast = c;
+            if (c + s.red[w] > target) {
+                wd = w;
+                break;
+            }
+            c += s.red[w];
+        }
+        s.mode = wd < 0;
+        s.sel = wd < 0 ? last : wd;
+        s.dsel = wd < 0 ? clast : c;
+    }
+    __syncthreads();
+    const int wsel = s.sel;
+    if (wsel < 0) return -1;
+    if (warp == wsel) {
+        const bool last_mode = s.mode;
+        double carry = s.dsel;
+        int res = -1, lastpos = -1;
+        const int stop = last_mode ? v1 : V;
+        for (int base = v0; base < stop; base += 32) {
+            const int v = base + lane;
+            const double x = v < stop ? wfn(v) : 0.0;
+            const double incl = warp_scan_f64(x, lane);
+            const unsigned hit = last_mode ? 0u : __ballot_sync(kFullMask, x > 0.0 && carry + incl > target);
+            if (hit) {
+                res = base + __ffs(hit) - 1;
+                break;
+            }
+            const unsigned pos = __ballot_sync(kFullMask, x > 0.0);
+            if (pos) lastpos = base + 31 - __clz(pos);
+            carry += __shfl_sync(kFullMask, incl, 31);
+        }
+        if (lane == 0) s.sel2 = res >= 0 ? res : lastpos;
+    }
+    __syncthreads();
+    const int out = s.sel2;
+    __syncthreads();
+    return out;
+}
+
+template <typename TL>
+__global__ void __launch_bounds__(kThreads) item_kernel(Params p, int only_redo) {
+    __shared__ Shared s;
+    const int n_items = p.B * p.K;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+        if (only_redo && p.recs[item].state == kDone) continue;
+        const int b = item / p.K, i = item % p.K;
+        if (trivial_item(p, b, i)) {
+            if (threadIdx.x == 0) write_trivial(p, item, b);
+            continue;
+        }
+        const TL* P = static_cast<const TL*>(p.P) + (int64_t)item * p.V;
+        const float* u = p.u + (int64_t)item * 3;
+        Row rp;
+        row_stats(P, p, s, rp);
+        auto wP = [&](int v) { return kept_weight(P, rp, p, v); };
+        if (i == 0) {
+            const int x0 = pos0_given(p, b) ? p.pos0[b] : draw(p.V, (double)u[0] * rp.Sk, wP, s);
+            const double px = (x0 >= 0 && x0 < p.V) ? wP(x0) / rp.Sk : 0.0;
+            if (threadIdx.x == 0) {
+                Rec r;
+                r.tok = x0;
+                r.res = -1;
+                r.acc = 1;
+                r.state = kDone;
+                r.p = px;
+                r.q = 0.0;
+                r.tv = 0.0;
+                r.pad = 0.0;
+                p.recs[item] = r;
+            }
+            __syncthreads();
+            continue;
+        }
+        const TL* Q = static_cast<const TL*>(p.Q) + (int64_t)item * p.V;
+        Row rq;
+        row_stats(Q, p, s, rq);
+        auto wQ = [&](int v) { return kept_weight(Q, rq, p, v); };
+        const int d = p.drafts ? p.drafts[item] : draw(p.V, (double)u[0] * rq.Sk, wQ, s);
+        const bool in = d >= 0 && d < p.V;
+        const double pd = in ? wP(d) / rp.Sk : 0.0, qd = in ? wQ(d) / rq.Sk : 0.0;
+        const int acc = (double)u[1] * qd < pd;
+        auto resid = [&](int v) {
+            const double dl = wP(v) / rp.Sk - wQ(v) / rq.Sk;
+            return dl > 0.0 ? dl : 0.0;
+        };
+        double rs = 0.0, ts = 0.0;
+        for (int v = threadIdx.x; v < p.V; v += kThreads) {
+            const double dl = wP(v) / rp.Sk - wQ(v) / rq.Sk;
+            if (dl > 0.0) rs += dl;
+            ts += fabs(dl);
+        }
+        const double R = block_sum(rs, s);
+        const double tv = 0.5 * block_sum(ts, s);
+        const int res = R > 0.0 ? draw(p.V, (double)u[2] * R, resid, s) : draw(p.V, (double)u[2] * rp.Sk, wP, s);
+        if (threadIdx.x == 0) {
+            Rec r;
+            r.tok = d;
+            r.res = res;
+            r.acc = acc;
+            r.state = kDone;
+            r.p = pd;
+            r.q = qd;
+            r.tv = tv;
+            r.pad = 0.0;
+            p.recs[item] = r;
+        }
+        __syncthreads();
+    }
+}
+
+}  // namespace gen
+
+// =======================================================================================
+// pair_kernel: one cluster per item, the rows' slices resident in shared memory
+// =======================================================================================
+namespace pk {
+
+constexpr int kTeams = 2;
+constexpr int kTeamWarps = 8;
+constexpr int kTeamThreads = kTeamWarps * 32;
+constexpr int kThreads = kTeams * kTeamThreads;
+constexpr int kWords = 2048;   // full mode: counted magnitudes per row, a_top - d for d < kWords
+constexpr int kWinK = 256;     // top-k mode: counted values per row, the 256 largest bf16 values from the max down
+constexpr int kLut = 512;      // tabulated survivor weights per row (positive values, d < kLut)
+constexpr int kMaxCL = 16;
+constexpr int kMaxTopK = 256;  // top-k mode: largest k
+
+// shared-memory layout of one team (byte offsets from the team's base); host and device
+struct Layout {
+    int CL;          // CTAs per cluster
+    int L;           // slice length in elements (a multiple of 8)
+    int hw;          // histogram words per row (kWords, or kWinK in top-k mode)
+    int OW;          // histogram words owned by each CTA: hw / CL
+    int KL;          // top-k mode: survivor list capacity per row (a power of two >= k)
+    uint32_t off_hist, off_own, off_lut, off_list, off_x1, off_x2, off_x3, off_misc, team_bytes;
 };
 
-// This CTA's slice of a bf16 row in shared memory, starting at chunk c0 (cluster kernel;
-// V is a multiple of 8, so every 8-element vector is either whole or past the end).
-struct SharedSlice {
-    const uint16_t* slice;
-    int c0, V;
-    __device__ __forceinline__ uint4 load(int c, int j, int lane, int& nv) const {
-        constexpr int CH = Chunk<__nv_bfloat16>::CH;
-        const int e0 = c * CH + j * 256 + lane * 8;
-        nv = e0 < V ? 8 : 0;
-        return nv ? lds128(slice + (e0 - c0 * CH)) : make_uint4(0u, 0u, 0u, 0u);
-    }
+struct RowStat {
+    double zmax;      // max of logit / T
+    double S;         // total mass
+    double Sk;        // surviving mass
+    double wk;        // weight of the cut value
+    float M;          // max value
+    uint32_t atop;    // largest magnitude (bf16 bits without the sign)
+    uint32_t kM;      // order key of the max value (top-k mode)
+    uint32_t kbits;   // bf16 bits of the cut value
+    int kd, kneg;     // cut value as (word d, sign)
+    int tkeep;        // ties kept, cluster-wide
+    int theta;        // ties with id < theta survive (this CTA's slice)
+    int lut_n;        // lut holds the weights of positive values with d < lut_n
 };
 
-__device__ __forceinline__ uint32_t cl_rank() {
+struct TeamShared {
+    RowStat rs[2];
+    double wpart[kTeamWarps][3];  // per-warp part masses: draw row, verifier survivors, residual
+    double dred[kTeamWarps][6];
+    uint32_t ured[kTeamWarps][4];
+    int ipart[kTeamWarps];
+    int redo, abort_;
+    int sel, sel2, mode;
+    double dsel;
+    unsigned lcnt[2];   // top-k mode: survivors appended to this CTA's lists (when it is the head)
+    int np[2];          // top-k mode: survivors of the top-p cut
+    double Z[2];        // top-k mode: their mass
+};
+
+// ---- PTX wrappers for the cluster ----
+__device__ __forceinline__ uint32_t ctarank() {
     uint32_t r;
     asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
     return r;
 }
-__device__ __forceinline__ uint32_t cl_size() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
-    return r;
+__device__ __forceinline__ uint32_t mapa(const void* local, uint32_t rank) {
+    uint32_t a;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(local)), "r"(rank));
+    return a;
 }
-__device__ __forceinline__ uint32_t cl_index() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
-    return r;
+__device__ __forceinline__ void st_remote_f64(uint32_t addr, double v) {
+    asm volatile("st.shared::cluster.f64 [%0], %1;" ::"r"(addr), "d"(v) : "memory");
 }
-__device__ __forceinline__ uint32_t cl_count() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
-    return r;
+__device__ __forceinline__ void st_remote_u64(uint32_t addr, unsigned long long v) {
+    asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(addr), "l"(v) : "memory");
 }
-
-// One CTA per row: the group is the CTA.
-struct CtaGroup {
-    __device__ __forceinline__ int size() const { return 1; }
-    __device__ __forceinline__ void sync() const { __syncthreads(); }
-    template <class X>
-    __device__ __forceinline__ const X* peer(const X* p, int) const { return p; }
-};
-
-// A thread-block cluster per row: barriers are cluster barriers (release / acquire), and
-// peer(p, r) is the generic address of p's counterpart in the shared memory of CTA r.
-struct ClusterGroup {
-    int n;
-    __device__ __forceinline__ int size() const { return n; }
-    __device__ __forceinline__ void sync() const {
-        asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+__device__ __forceinline__ uint32_t ld_remote_u32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint32_t atom_remote_add(uint32_t addr, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.shared::cluster.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(addr), "r"(v) : "memory");
+    return old;
+}
+__device__ __forceinline__ uint2 ld_remote_v2(uint32_t addr) {
+    uint2 v;
+    asm volatile("ld.shared::cluster.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr) : "memory");
+    return v;
+}
+__device__ __forceinline__ void arrive_remote(uint32_t bar) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void fence_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
+__device__ __forceinline__ bool wait_cluster(uint64_t* bar, uint32_t parity) {
+    for (uint32_t k = 0; k < kWaitLimit; ++k) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred q;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 q, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, q;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+        if (ok) return true;
     }
-    template <class X>
-    __device__ __forceinline__ const X* peer(const X* p, int r) const {
-        uint64_t q;
-        asm volatile("mapa.u64 %0, %1, %2;" : "=l"(q) : "l"(reinterpret_cast<uint64_t>(p)), "r"(r));
-        return reinterpret_cast<const X*>(q);
-    }
-};
-
-// What each CTA of a group publishes for a row-wide reduction: its partials, read by every
-// CTA of the group after a group barrier. Two areas are used in turn, so that one barrier
-// per exchange suffices (area e is rewritten at exchange e + 2, after every CTA has passed
-// the barrier of exchange e + 1 and so has finished reading it).
-struct Xchg {
-    double mass[256];
-    uint32_t cnt[256];
-    double s;
-    float m;
-    int pad;
-};
-
-// Units of the cluster kernel's balanced passes: vector row j of a chunk, one 16-byte vector
-// per lane (a CTA's slice has at most kMaxUnits of them).
-constexpr int kMaxUnits = 192;
-constexpr int kUB = 4;  // units (or vectors) a warp (thread) works on at a time in the slice passes
-// Keys of the exact cut histogram (bf16 values: 16-bit keys; 16 per thread of the first 256).
-constexpr int kKeyBins = 4096;
-
-struct RowShared {
-    float hist_f[256 * kWarps];   // per-warp histograms; the group's key counts (as uint32)
-    uint32_t hist_n[256 * kWarps];  // per-warp histograms; this CTA's key counts
-    double comb_m[256];           // the group's histogram; key-mass partial sums
-    uint32_t comb_n[256];
-    double dred[kWarps];
-    float fred[kWarps];
-    float ustat[kMaxUnits];       // per unit: max (then survivor mass)
-    float usum[kMaxUnits];        // per unit: sum of exps
-    int uties[kMaxUnits];         // per unit: tokens equal to the cut
-    float cmx[kMaxUnits / kVecPerLane];  // per chunk of the slice: max
-    Xchg x[2];
-};
-static_assert(kKeyBins <= 256 * kWarps, "key counts live in the histogram arrays");
-
-// ---------------------------------------------------------------------------------------
-// per row: statistics, top-p cut, per-chunk survivor table (a CTA, or a cluster of CTAs each
-// holding a slice of the row)
-// ---------------------------------------------------------------------------------------
-// Chunks [c0, c1) of the row are this CTA's; cmass and cties are indexed by the row's chunk
-// index; info (written if not null) receives the row's RowInfo, which every CTA of the group
-// computes identically (every CTA combines the same partials in the same order). xe counts
-// the exchanges made so far.
-template <typename T, typename Src, typename Grp>
-__device__ void prepare_row(const Src& src, const VerifyArgs& a, int c0, int c1, double* cmass, int* cties,
-                            RowInfo* info, RowShared& sh, const Grp& grp, int& xe) {
-    constexpr int NLEVELS = sizeof(T) == 2 ? 2 : 4;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int V = a.V;
-    const float invT = 1.0f / a.temperature;
-
-    constexpr bool kSlice = std::is_same<Src, SharedSlice>::value;
-    constexpr int CH = Chunk<T>::CH;
-    const int U = (c1 - c0) * kVecPerLane;  // units of this CTA (slice form)
-
-    // 1. per chunk max and sum; row max and sum
-    float lmax = -INFINITY;
-    if constexpr (kSlice) {
-        // balanced over the warps: unit u = vector row u % 8 of chunk c0 + u / 8; each warp
-        // takes UB of its units at a time, so that their loads and reductions overlap
-        for (int ub = warp; ub < U; ub += kUB * kWarps) {
-            float m[kUB];
-#pragma unroll
-            for (int k = 0; k < kUB; ++k) {
-                const int u = ub + k * kWarps;
-                m[k] = -INFINITY;
-                if (u < U) {
-                    int nv;
-                    const uint4 v = src.load(c0 + u / kVecPerLane, u % kVecPerLane, lane, nv);
-                    if (nv == 8) {
-                        const __nv_bfloat162 m2 =
-                            __hmax2(__hmax2(as_b2(v.x), as_b2(v.y)), __hmax2(as_b2(v.z), as_b2(v.w)));
-                        m[k] = fmaxf(__low2float(m2), __high2float(m2)) * invT;
-                    }
-                }
-            }
-#pragma unroll
-            for (int off = 16; off; off >>= 1)
-#pragma unroll
-                for (int k = 0; k < kUB; ++k) m[k] = fmaxf(m[k], __shfl_xor_sync(kFullMask, m[k], off));
-            if (lane == 0)
-#pragma unroll
-                for (int k = 0; k < kUB; ++k)
-                    if (ub + k * kWarps < U) sh.ustat[ub + k * kWarps] = m[k];
-        }
-        __syncthreads();
-        for (int c = c0 + threadIdx.x; c < c1; c += kThreads) {
-            const float* um = sh.ustat + (c - c0) * kVecPerLane;
-            float cm = um[0];
-            for (int k = 1; k < kVecPerLane; ++k) cm = fmaxf(cm, um[k]);
-            sh.cmx[c - c0] = cm;
-        }
-        __syncthreads();
-        for (int ub = warp; ub < U; ub += kUB * kWarps) {
-            float cs[kUB];
-#pragma unroll
-            for (int k = 0; k < kUB; ++k) {
-                const int u = ub + k * kWarps;
-                cs[k] = 0.f;
-                if (u < U) {
-                    int nv;
-                    const uint4 v = src.load(c0 + u / kVecPerLane, u % kVecPerLane, lane, nv);
-                    if (nv == 8) {
-                        const float cm = sh.cmx[u / kVecPerLane];
-                        float x[8];
-                        unpack8(v, x);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) cs[k] += __expf(x[e] * invT - cm);
-                    }
-                }
-            }
-#pragma unroll
-            for (int off = 16; off; off >>= 1)
-#pragma unroll
-                for (int k = 0; k < kUB; ++k) cs[k] += __shfl_xor_sync(kFullMask, cs[k], off);
-            if (lane == 0)
-#pragma unroll
-                for (int k = 0; k < kUB; ++k)
-                    if (ub + k * kWarps < U) sh.usum[ub + k * kWarps] = cs[k];
-        }
-        __syncthreads();
-        for (int c = c0 + threadIdx.x; c < c1; c += kThreads) {
-            const int u0 = (c - c0) * kVecPerLane;
-            const float cm = sh.cmx[c - c0];
-            double cs = 0.0;
-            for (int k = 0; k < kVecPerLane; ++k) cs += (double)sh.usum[u0 + k];
-            cmass[c] = cs;                             // relative to the chunk max for now
-            reinterpret_cast<float*>(cties)[c] = cm;  // chunk max parked in the ties slot
-            lmax = fmaxf(lmax, cm);
-        }
-    } else
-    for (int c = c0 + warp; c < c1; c += kWarps) {
-        float cm = -INFINITY;
-        for (int j = 0; j < kVecPerLane; ++j) {
-            int nv;
-            uint4 v = src.load(c, j, lane, nv);
-            if constexpr (kIsBf16<T>) {
-                if (nv == 8) {
-                    const __nv_bfloat162 m2 = __hmax2(__hmax2(as_b2(v.x), as_b2(v.y)), __hmax2(as_b2(v.z), as_b2(v.w)));
-                    cm = fmaxf(cm, fmaxf(__low2float(m2), __high2float(m2)) * invT);
-                    continue;
-                }
-            }
-            for (int e = 0; e < nv; ++e) cm = fmaxf(cm, raw_get<T>(v, e) * invT);
-        }
-        cm = warp_max(cm);
-        float cs = 0.f;
-        for (int j = 0; j < kVecPerLane; ++j) {
-            int nv;
-            uint4 v = src.load(c, j, lane, nv);
-            if constexpr (kIsBf16<T>) {
-                if (nv == 8) {
-                    float x[8];
-                    unpack8(v, x);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) cs += __expf(x[e] * invT - cm);
-                    continue;
-                }
-            }
-            for (int e = 0; e < nv; ++e) cs += __expf(raw_get<T>(v, e) * invT - cm);
-        }
-        cs = warp_sum(cs);
-        if (lane == 0) {
-            cmass[c] = (double)cs;               // relative to the chunk max for now
-            reinterpret_cast<float*>(cties)[c] = cm;  // chunk max parked in the ties slot
-        }
-        lmax = fmaxf(lmax, cm);
-    }
-    // this CTA's max and its sum relative to it; then the group's M and S
-    const float mc = cta_max_f32(lmax, sh.fred);
-    double part = 0.0;
-    for (int c = c0 + threadIdx.x; c < c1; c += kThreads)
-        part += cmass[c] * exp((double)reinterpret_cast<float*>(cties)[c] - (double)mc);
-    const double sc = cta_sum_f64(part, sh.dred);
-    float M;
-    double S = 0.0;
-    {
-        Xchg& xo = sh.x[xe++ & 1];
-        if (threadIdx.x == 0) {
-            xo.m = mc;
-            xo.s = sc;
-        }
-        grp.sync();
-        // every warp combines the group's partials, lane r taking CTA r's (a CTA without
-        // chunks sends 0 and -inf); the fixed lane order makes the sums identical everywhere
-        float mr = -INFINITY;
-        double sr = 0.0;
-        if (lane < grp.size()) {
-            const Xchg* xr = grp.peer(&xo, lane);
-            mr = xr->m;
-            sr = xr->s;
-        }
-        M = warp_max(mr);
-        S = warp_sum_f64(lane < grp.size() ? sr * exp((double)mr - (double)M) : 0.0);
-    }
-    for (int c = c0 + threadIdx.x; c < c1; c += kThreads) {
-        cmass[c] = cmass[c] * exp((double)reinterpret_cast<float*>(cties)[c] - (double)M);
-        cties[c] = 0;
-    }
-    RowInfo ri{};
-    ri.M = M;
-    ri.S = S;
-    ri.Z = S;
-    ri.tau = 0u;
-    ri.c_tie = 0;
-    ri.w_tau = 0.0;
-    if (a.top_p < 1.0f) {
-        // 2. exact top-p cut by radix histograms of the mass over the logit keys
-        const double target = (double)a.top_p * S;
-        // level A: mass by distance below the max, 1/8-nat bins (the radix levels below,
-        // restricted to the crossing bin, then fix the exact cut). Binning by value spreads
-        // the elements over many bins, where the first radix level over the key's top bits
-        // would put most of them in a few.
-        auto vbin = [&](float x) {
-            const float d = M - x * invT;
-            return d < 31.875f ? (int)(d * 8.f) : 255;
-        };
-        // Only elements within D nats of the max are binned: those further down weigh at
-        // most V e^-D together, which is below the mass top-p leaves out when
-        // D >= ln(V / ((1 - top_p) S)), so the cut lies within D (a full pass is the
-        // fallback for rounding).
-        // (D is a whole number of bins, so that a bin is either binned in full or not at all)
-        const double dcut = log((double)V / ((1.0 - (double)a.top_p) * S)) + 0.5;
-        float D = dcut > 31.875 ? 31.875f : (dcut < 0.125 ? 0.125f : ceilf((float)dcut * 8.f) * 0.125f);
-        uint32_t tau = 0u;      // key of the cut value
-        double above = 0.0;     // mass of the keys above it
-        uint32_t count_at = 0;  // tokens equal to it (0: no cut, every token survives)
-        bool have_cut = false;
-        if constexpr (kSlice) {
-            // Exact cut from counts per bf16 value: every token with the same value has the same
-            // weight, so the mass of a value is its count times one exp (fp64). The values within
-            // D of the max span at most kKeyBins 16-bit keys unless the range reaches close to 0;
-            // otherwise (or if rounding leaves the target unmet) the histograms below decide.
-            const float hiv = __bfloat162float(__float2bfloat16_ru(M * a.temperature));  // >= the max logit
-            const float lov = __bfloat162float(__float2bfloat16_rd((M - D) * a.temperature));
-            const uint32_t hi16 = float_key(hiv) >> 16, lo16 = float_key(lov) >> 16;
-            const uint32_t R = hi16 >= lo16 ? hi16 - lo16 + 1u : 0u;
-            if (R > 0u && R <= (uint32_t)kKeyBins) {
-                uint32_t* kc = sh.hist_n;                                // this CTA's counts (read by the group)
-                uint32_t* tot = reinterpret_cast<uint32_t*>(sh.hist_f);  // the group's counts
-                auto key_weight = [&](uint32_t k16) {  // a token's weight exp(z - M), for a bf16 key
-                    const uint32_t k = (k16 << 16) | ((k16 & 0x8000u) ? 0x0000u : 0xFFFFu);
-                    return (double)__expf(key_float(k) * invT - M);
-                };
-                for (int i = threadIdx.x; i < (int)R; i += kThreads) kc[i] = 0u;
-                __syncthreads();
-                const __nv_bfloat162 lo2 = __float2bfloat162_rn(lov);  // lov is a bf16 value
-                const int nvec = c1 > c0 ? (int)((min((int64_t)V, (int64_t)c1 * CH) - (int64_t)c0 * CH) / 8) : 0;
-                for (int i0 = threadIdx.x; i0 < nvec; i0 += kUB * kThreads) {
-                    uint4 vb[kUB];
-#pragma unroll
-                    for (int k = 0; k < kUB; ++k) {
-                        const int i = i0 + k * kThreads;
-                        vb[k] = i < nvec ? lds128(src.slice + (size_t)i * 8) : make_uint4(0u, 0u, 0u, 0u);
-                    }
-#pragma unroll
-                    for (int k = 0; k < kUB; ++k) {
-                        if (i0 + k * kThreads >= nvec || !any_ge(vb[k], lo2)) continue;
-                        const uint32_t w4[4] = {vb[k].x, vb[k].y, vb[k].z, vb[k].w};
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const uint32_t k2 = bf16x2_keys(w4[q]);
-                            const uint32_t ka = (k2 & 0xFFFFu) - lo16, kb = (k2 >> 16) - lo16;
-                            if (ka < R) atomicAdd(&kc[ka], 1u);
-                            if (kb < R) atomicAdd(&kc[kb], 1u);
-                        }
-                    }
-                }
-                grp.sync();  // every CTA's counts are complete
-                for (int i = threadIdx.x; i < (int)R; i += kThreads) {
-                    uint32_t n = 0;
-                    for (int r = 0; r < grp.size(); ++r) n += grp.peer(kc, r)[i];
-                    tot[i] = n;
-                }
-                __syncthreads();
-                // mass of 16 keys per thread (threads 0..255), from the top key down
-                constexpr int KPT = kKeyBins / 256;
-                if (threadIdx.x < 256) {
-                    double msum = 0.0;
-                    for (int q = 0; q < KPT; ++q) {
-                        const int idx = (int)R - 1 - ((int)threadIdx.x * KPT + q);
-                        if (idx >= 0 && tot[idx]) msum += (double)tot[idx] * key_weight(lo16 + (uint32_t)idx);
-                    }
-                    sh.comb_m[threadIdx.x] = msum;
-                }
-                __syncthreads();
-                if (warp == 0) {
-                    double cum = 0.0, t_excl = 0.0;
-                    int t_hit = -1;
-                    for (int t0 = 0; t0 < 256 && t_hit < 0; t0 += 32) {
-                        const double m = sh.comb_m[t0 + lane];
-                        const double incl = warp_scan_f64(m, lane);
-                        const unsigned hit = __ballot_sync(kFullMask, cum + incl >= target && m > 0.0);
-                        if (hit) {
-                            const int hl = __ffs(hit) - 1;
-                            t_hit = t0 + hl;
-                            t_excl = cum + __shfl_sync(kFullMask, incl - m, hl);
-                        }
-                        cum += __shfl_sync(kFullMask, incl, 31);
-                    }
-                    if (lane == 0) {
-                        // the key within that thread's range where the mass reaches the target
-                        // (the last non-empty one if rounding leaves it a hair short)
-                        int idx_hit = -1;
-                        double ab = 0.0, c = t_excl;
-                        uint32_t n_hit = 0;
-                        for (int q = 0; t_hit >= 0 && q < KPT; ++q) {
-                            const int idx = (int)R - 1 - (t_hit * KPT + q);
-                            if (idx < 0) break;
-                            const uint32_t n = tot[idx];
-                            if (!n) continue;
-                            const double w = (double)n * key_weight(lo16 + (uint32_t)idx);
-                            idx_hit = idx;
-                            ab = c;
-                            n_hit = n;
-                            if (c + w >= target) break;
-                            c += w;
-                        }
-                        sh.dred[0] = ab;
-                        sh.dred[1] = (double)idx_hit;
-                        sh.dred[2] = (double)n_hit;
-                    }
-                }
-                __syncthreads();
-                const int idx_hit = (int)sh.dred[1];
-                if (idx_hit >= 0) {
-                    have_cut = true;
-                    const uint32_t k16 = lo16 + (uint32_t)idx_hit;
-                    tau = (k16 << 16) | ((k16 & 0x8000u) ? 0x0000u : 0xFFFFu);
-                    above = sh.dred[0];
-                    count_at = (uint32_t)sh.dred[2];
-                }
-                __syncthreads();
-            }
-        }
-        if (!have_cut) {
-        int vchosen = -1;
-        double vabove = 0.0;
-        for (int attempt = 0; attempt < 2 && vchosen < 0; ++attempt) {
-            if (attempt == 1) D = INFINITY;  // every element
-            for (int i = threadIdx.x; i < 256 * kWarps; i += kThreads) sh.hist_f[i] = 0.f;
-            __syncthreads();
-            float* hf = sh.hist_f + warp * 256;
-            // packed prefilter: a logit below (M - D) T - 1/16 (rounded down) cannot pass
-            const __nv_bfloat162 alo = D == INFINITY
-                                           ? __float2bfloat162_rn(-INFINITY)
-                                           : __bfloat162bfloat162(__float2bfloat16_rd(((M - D) - 0.0625f) * a.temperature));
-            for (int c = c0 + warp; c < c1; c += kWarps) {
-                for (int j = 0; j < kVecPerLane; ++j) {
-                    int nv;
-                    uint4 v = src.load(c, j, lane, nv);
-                    if constexpr (kIsBf16<T>) {
-                        if (nv == 8) {
-                            if (!any_ge(v, alo)) continue;
-                            float x[8];
-                            unpack8(v, x);
-#pragma unroll
-                            for (int e = 0; e < 8; ++e)
-                                if (M - x[e] * invT < D) atomicAdd(&hf[vbin(x[e])], __expf(x[e] * invT - M));
-                            continue;
-                        }
-                    }
-                    for (int e = 0; e < nv; ++e) {
-                        const float x = raw_get<T>(v, e);
-                        if (M - x * invT < D) atomicAdd(&hf[vbin(x)], __expf(x * invT - M));
-                    }
-                }
-            }
-            __syncthreads();
-            {
-                Xchg& xo = sh.x[xe++ & 1];
-                for (int bin = threadIdx.x; bin < 256; bin += kThreads) {
-                    double m = 0.0;
-                    for (int w = 0; w < kWarps; ++w) m += (double)sh.hist_f[w * 256 + bin];
-                    xo.mass[bin] = m;
-                }
-                grp.sync();
-                for (int bin = threadIdx.x; bin < 256; bin += kThreads) {
-                    double m = 0.0;
-                    for (int r = 0; r < grp.size(); ++r) m += grp.peer(&xo, r)->mass[bin];
-                    sh.comb_m[bin] = m;
-                }
-                __syncthreads();
-            }
-            if (warp == 0) {
-            double cum = 0.0;
-            int chosen = -1;
-            double chosen_above = 0.0;
-            for (int b0 = 0; b0 < 256 && chosen < 0; b0 += 32) {
-                const int bin = b0 + lane;
-                const double m = sh.comb_m[bin];
-                const double incl = warp_scan_f64(m, lane);
-                // (a bin whose elements all underflow to 0 cannot be where the mass crosses)
-                const unsigned hit = __ballot_sync(kFullMask, cum + incl >= target && m > 0.0);
-                if (hit) {
-                    const int hl = __ffs(hit) - 1;
-                    chosen = b0 + hl;
-                    chosen_above = cum + __shfl_sync(kFullMask, incl - m, hl);
-                }
-                cum += __shfl_sync(kFullMask, incl, 31);
-            }
-            if (lane == 0) {
-                sh.dred[0] = chosen_above;
-                sh.dred[1] = (double)chosen;
-            }
-            }
-            __syncthreads();
-            vchosen = (int)sh.dred[1];  // -1: the binned mass falls short of the target
-            vabove = sh.dred[0];
-            __syncthreads();
-        }
-        uint32_t prefix = 0;     // key bits fixed so far
-        above = vchosen >= 0 ? vabove : 0.0;  // mass of keys above the current prefix bin
-        count_at = 0;
-        // packed prefilter of the radix levels: the logits of the chosen bin lie within
-        // [(M - (b + 1) / 8) T, (M - b / 8) T], widened by 1/16 and rounded outwards
-        const float vlo = (M - (vchosen + 1) * 0.125f - 0.0625f) * a.temperature;
-        const float vhi = (M - vchosen * 0.125f + 0.0625f) * a.temperature;
-        const __nv_bfloat162 rlo = vchosen == 255 ? __float2bfloat162_rn(-INFINITY)
-                                                  : __bfloat162bfloat162(__float2bfloat16_rd(vlo));
-        const __nv_bfloat162 rhi = __bfloat162bfloat162(__float2bfloat16_ru(vhi));
-        for (int level = 0; level < NLEVELS && vchosen >= 0; ++level) {
-            const int shift = 24 - 8 * level;
-            const uint32_t hi_mask = level == 0 ? 0u : (~0u << (shift + 8));
-            for (int i = threadIdx.x; i < 256 * kWarps; i += kThreads) {
-                sh.hist_f[i] = 0.f;
-                sh.hist_n[i] = 0u;
-            }
-            __syncthreads();
-            float* hf = sh.hist_f + warp * 256;
-            uint32_t* hn = sh.hist_n + warp * 256;
-            for (int c = c0 + warp; c < c1; c += kWarps) {
-                for (int j = 0; j < kVecPerLane; ++j) {
-                    int nv;
-                    uint4 v = src.load(c, j, lane, nv);
-                    if constexpr (kIsBf16<T>) {
-                        if (nv == 8) {
-                            if (!any_in(v, rlo, rhi)) continue;
-                            float x[8];
-                            unpack8(v, x);
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) {
-                                const uint32_t key = float_key(x[e]);
-                                if ((key & hi_mask) == prefix && vbin(x[e]) == vchosen) {
-                                    const uint32_t bin = (key >> shift) & 0xFFu;
-                                    atomicAdd(&hf[bin], __expf(x[e] * invT - M));
-                                    atomicAdd(&hn[bin], 1u);
-                                }
-                            }
-                            continue;
-                        }
-                    }
-                    for (int e = 0; e < nv; ++e) {
-                        const float x = raw_get<T>(v, e);
-                        const uint32_t key = float_key(x);
-                        if ((key & hi_mask) == prefix && vbin(x) == vchosen) {
-                            const uint32_t bin = (key >> shift) & 0xFFu;
-                            atomicAdd(&hf[bin], __expf(x * invT - M));
-                            atomicAdd(&hn[bin], 1u);
-                        }
-                    }
-                }
-            }
-            __syncthreads();
-            // combine the warps' histograms, then the group's; walk bins from the top
-            {
-                Xchg& xo = sh.x[xe++ & 1];
-                for (int bin = threadIdx.x; bin < 256; bin += kThreads) {
-                    double m = 0.0;
-                    uint32_t n = 0;
-                    for (int w = 0; w < kWarps; ++w) {
-                        m += (double)sh.hist_f[w * 256 + bin];
-                        n += sh.hist_n[w * 256 + bin];
-                    }
-                    xo.mass[bin] = m;
-                    xo.cnt[bin] = n;
-                }
-                grp.sync();
-                for (int bin = threadIdx.x; bin < 256; bin += kThreads) {
-                    double m = 0.0;
-                    uint32_t n = 0;
-                    for (int r = 0; r < grp.size(); ++r) {
-                        const Xchg* xr = grp.peer(&xo, r);
-                        m += xr->mass[bin];
-                        n += xr->cnt[bin];
-                    }
-                    sh.comb_m[bin] = m;
-                    sh.comb_n[bin] = n;
-                }
-                __syncthreads();
-            }
-            if (warp == 0) {
-                double cum = above;
-                int chosen = -1;
-                double chosen_above = above;
-                uint32_t chosen_n = 0;
-                for (int b0 = 255; b0 >= 0 && chosen < 0; b0 -= 32) {
-                    const int bin = b0 - lane;
-                    const double m = sh.comb_m[bin];
-                    const uint32_t n = sh.comb_n[bin];
-                    const double incl = warp_scan_f64(m, lane);
-                    const unsigned hit = __ballot_sync(kFullMask, cum + incl >= target && n > 0);
-                    if (hit) {
-                        const int hl = __ffs(hit) - 1;
-                        chosen = b0 - hl;
-                        chosen_above = cum + __shfl_sync(kFullMask, incl - m, hl);
-                        chosen_n = __shfl_sync(kFullMask, n, hl);
-                    }
-                    cum += __shfl_sync(kFullMask, incl, 31);
-                }
-                if (chosen < 0) {  // rounding: the whole mass falls short of the target; keep everything
-                    chosen = -2;
-                }
-                if (lane == 0) {
-                    sh.dred[0] = chosen_above;
-                    sh.dred[1] = (double)chosen;
-                    sh.dred[2] = (double)chosen_n;
-                }
-            }
-            __syncthreads();
-            const int chosen = (int)sh.dred[1];
-            if (chosen == -2) {
-                prefix = 0;
-                above = 0.0;
-                count_at = 0;
-                break;
-            }
-            above = sh.dred[0];
-            count_at = (uint32_t)sh.dred[2];
-            prefix |= (uint32_t)chosen << shift;
-            __syncthreads();
-        }
-        if (count_at > 0) {
-            // the cut value; for bf16 logits the low 16 key bits follow from the sign
-            tau = prefix;
-            if (NLEVELS == 2) tau |= (tau & 0x80000000u) ? 0x0000u : 0xFFFFu;
-        }
-        }  // !have_cut
-        if (count_at > 0) {
-            const double w_tau = exp((double)key_float(tau) / (double)a.temperature - (double)M);
-            double need = (target - above) / w_tau;
-            int c_tie = (int)ceil(need - 1e-12);
-            c_tie = c_tie < 1 ? 1 : (c_tie > (int)count_at ? (int)count_at : c_tie);
-            ri.tau = tau;
-            ri.c_tie = c_tie;
-            ri.w_tau = w_tau;
-            ri.Z = above + (double)c_tie * w_tau;
-            // 3. per chunk: mass of keys above tau, and the number of tokens equal to tau
-            if constexpr (kSlice) {
-                const __nv_bfloat162 tlo = __float2bfloat162_rn(key_float(tau));  // tau is a bf16 value here
-                for (int ub = warp; ub < U; ub += kUB * kWarps) {
-                    float mg[kUB];
-                    int nt[kUB];
-#pragma unroll
-                    for (int k = 0; k < kUB; ++k) {
-                        const int u = ub + k * kWarps;
-                        mg[k] = 0.f;
-                        nt[k] = 0;
-                        if (u < U) {
-                            int nv;
-                            const uint4 v = src.load(c0 + u / kVecPerLane, u % kVecPerLane, lane, nv);
-                            if (nv == 8 && any_ge(v, tlo)) {
-                                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                                for (int q = 0; q < 4; ++q) {
-                                    // IEEE comparisons of bf16 values order them as their keys
-                                    // do (-0 equal to +0)
-                                    const uint32_t gt = __hgt2_mask(as_b2(w4[q]), tlo);
-                                    const uint32_t eq = __heq2_mask(as_b2(w4[q]), tlo);
-                                    if (gt & 0xFFFFu) mg[k] += __expf(bf16_lo(w4[q]) * invT - M);
-                                    if (gt >> 16) mg[k] += __expf(bf16_hi(w4[q]) * invT - M);
-                                    nt[k] += (int)((eq & 1u) + (eq >> 31));
-                                }
-                            }
-                        }
-                    }
-#pragma unroll
-                    for (int off = 16; off; off >>= 1)
-#pragma unroll
-                        for (int k = 0; k < kUB; ++k) {
-                            mg[k] += __shfl_xor_sync(kFullMask, mg[k], off);
-                            nt[k] += __shfl_xor_sync(kFullMask, nt[k], off);
-                        }
-                    if (lane == 0)
-#pragma unroll
-                        for (int k = 0; k < kUB; ++k)
-                            if (ub + k * kWarps < U) {
-                                sh.ustat[ub + k * kWarps] = mg[k];
-                                sh.uties[ub + k * kWarps] = nt[k];
-                            }
-                }
-                __syncthreads();
-                for (int c = c0 + threadIdx.x; c < c1; c += kThreads) {
-                    const int u0 = (c - c0) * kVecPerLane;
-                    double m = 0.0;
-                    int n = 0;
-                    for (int k = 0; k < kVecPerLane; ++k) {
-                        m += (double)sh.ustat[u0 + k];
-                        n += sh.uties[u0 + k];
-                    }
-                    cmass[c] = m;
-                    cties[c] = n;
-                }
-            } else
-            for (int c = c0 + warp; c < c1; c += kWarps) {
-                float mg = 0.f;
-                int nt = 0;
-                const __nv_bfloat162 tlo = __float2bfloat162_rn(key_float(tau));  // tau is a bf16 value here
-                for (int j = 0; j < kVecPerLane; ++j) {
-                    int nv;
-                    uint4 v = src.load(c, j, lane, nv);
-                    if constexpr (kIsBf16<T>) {
-                        if (nv == 8) {
-                            if (!any_ge(v, tlo)) continue;
-                            float x[8];
-                            unpack8(v, x);
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) {
-                                const uint32_t key = float_key(x[e]);
-                                if (key > tau) mg += __expf(x[e] * invT - M);
-                                nt += key == tau;
-                            }
-                            continue;
-                        }
-                    }
-                    for (int e = 0; e < nv; ++e) {
-                        const float x = raw_get<T>(v, e);
-                        const uint32_t key = float_key(x);
-                        if (key > tau) mg += __expf(x * invT - M);
-                        nt += key == tau;
-                    }
-                }
-                mg = warp_sum(mg);
-                nt = warp_sum(nt);
-                if (lane == 0) {
-                    cmass[c] = (double)mg;
-                    cties[c] = nt;
-                }
-            }
-        }
-    }
-    __syncthreads();
-    if (threadIdx.x == 0 && info) *info = ri;
-    __syncthreads();
+    return false;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void team_sync(int team) {
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "n"(kTeamThreads) : "memory");
 }
 
-// ---------------------------------------------------------------------------------------
-// warp-level walks over one row
-// ---------------------------------------------------------------------------------------
-// surviving mass of chunk c given the ties that precede it
-__device__ __forceinline__ double chunk_surv(const RowInfo& ri, const double* cmass, const int* cties, int c,
-                                             int ties_before) {
-    if (ri.tau == 0u) return cmass[c];
-    const int kept = max(0, min(ri.c_tie - ties_before, cties[c]));
-    return cmass[c] + (double)kept * ri.w_tau;
+__device__ __forceinline__ float bf(uint32_t h16) { return __uint_as_float(h16 << 16); }
+
+// weight of a bf16 value relative to the row's max: exp(v / T - zmax)
+__device__ __forceinline__ double wexp(uint32_t h16, const RowStat& r, double T) {
+    return exp((double)bf(h16) / T - r.zmax);
 }
 
-// Scan chunk c of the row in id order; for every element calls f(id, z, survivor weight,
-// lane) — all lanes call f for their elements of each 32-lane vector in turn.
-template <typename T, typename F>
-__device__ __forceinline__ void scan_chunk(const T* row, const VerifyArgs& a, const RowInfo& ri, int c,
-                                           int ties_before, int lane, F f) {
-    constexpr int VEC = Elem<T>::VEC;
-    const float invT = 1.0f / a.temperature;
-    int carry = ties_before;
-    for (int j = 0; j < kVecPerLane; ++j) {
-        int nv;
-        const uint4 v = load_vec<T>(row, a.V, c, j, lane, nv);
-        int nt = 0;
-        for (int e = 0; e < nv; ++e) nt += float_key(raw_get<T>(v, e)) == ri.tau;
-        const int incl = warp_inclusive_scan(nt, lane);
-        int rank = carry + incl - nt;
-        const int64_t id0 = (int64_t)c * Chunk<T>::CH + (int64_t)j * 32 * VEC + lane * VEC;
-        double wv[Elem<T>::VEC];
-        for (int e = 0; e < VEC; ++e) {
-            wv[e] = 0.0;
-            if (e < nv) {
-                const float x = raw_get<T>(v, e);
-                const uint32_t key = float_key(x);
-                bool surv = ri.tau == 0u || key > ri.tau;
-                if (ri.tau != 0u && key == ri.tau) surv = rank++ < ri.c_tie;
-                if (surv) wv[e] = (double)__expf(x * invT - ri.M);
-            }
-        }
-        f(id0, wv, nv, j);
-        carry += __shfl_sync(kFullMask, incl, 31);
+// value of histogram word d with the given sign
+__device__ __forceinline__ uint32_t word_bits(const RowStat& r, int d, int neg) {
+    return (r.atop - (uint32_t)d) | (neg ? 0x8000u : 0u);
+}
+
+// survivor weight of one element (value bits h16, token id v), 0 if it does not survive
+__device__ __forceinline__ double surv_weight(uint32_t h16, int v, const RowStat& r, const double* lut, double T,
+                                              int cut) {
+    const float x = bf(h16);
+    if (cut) {
+        const float kx = bf(r.kbits);
+        if (x < kx || (x == kx && v >= r.theta) || x != x) return 0.0;
     }
+    const uint32_t d = r.atop - h16;  // positive values only (sign bit clear)
+    if (!(h16 & 0x8000u) && d < (uint32_t)r.lut_n) return lut[d];
+    if (!(fabsf(x) < INFINITY)) return 0.0;
+    return exp((double)x / T - r.zmax);
 }
 
-// Scan chunk c of two rows (verifier p, drafter q) together in id order; for every vector
-// of 32 lanes calls f(id0, wp, wq, nv) with the lane's normalised survivor probabilities
-// of both rows (reciprocals of the rows' surviving masses taken once).
-template <typename T, typename F>
-__device__ __forceinline__ void scan_pair_chunk(const T* prow, const T* qrow, const VerifyArgs& a, const RowInfo& rp,
-                                                const RowInfo& rq, int c, int tbp, int tbq, int lane, F f) {
-    constexpr int VEC = Elem<T>::VEC;
-    const float invT = 1.0f / a.temperature;
-    const double izp = 1.0 / rp.Z, izq = 1.0 / rq.Z;
-    int carp = tbp, carq = tbq;
-    for (int j = 0; j < kVecPerLane; ++j) {
-        int nv;
-        const uint4 vp = load_vec<T>(prow, a.V, c, j, lane, nv);
-        const uint4 vq = load_vec<T>(qrow, a.V, c, j, lane, nv);
-        int ntp = 0, ntq = 0;
-        for (int e = 0; e < nv; ++e) {
-            ntp += float_key(raw_get<T>(vp, e)) == rp.tau;
-            ntq += float_key(raw_get<T>(vq, e)) == rq.tau;
-        }
-        const int ip = warp_inclusive_scan(ntp, lane), iq = warp_inclusive_scan(ntq, lane);
-        int rkp = carp + ip - ntp, rkq = carq + iq - ntq;
-        const int64_t id0 = (int64_t)c * Chunk<T>::CH + (int64_t)j * 32 * VEC + lane * VEC;
-        double wp[VEC], wq[VEC];
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) {
-            wp[e] = 0.0;
-            wq[e] = 0.0;
-            if (e < nv) {
-                const float xp = raw_get<T>(vp, e), xq = raw_get<T>(vq, e);
-                const uint32_t kp = float_key(xp), kq = float_key(xq);
-                bool sp = rp.tau == 0u || kp > rp.tau, sq = rq.tau == 0u || kq > rq.tau;
-                if (rp.tau != 0u && kp == rp.tau) sp = rkp++ < rp.c_tie;
-                if (rq.tau != 0u && kq == rq.tau) sq = rkq++ < rq.c_tie;
-                if (sp) wp[e] = (double)__expf(xp * invT - rp.M) * izp;
-                if (sq) wq[e] = (double)__expf(xq * invT - rq.M) * izq;
-            }
-        }
-        f(id0, wp, wq, nv);
-        carp += __shfl_sync(kFullMask, ip, 31);
-        carq += __shfl_sync(kFullMask, iq, 31);
-    }
-}
+// the element's 16 bits from a shared-memory slice
+__device__ __forceinline__ uint32_t elem(const uint16_t* buf, int e) { return buf[e]; }
 
-// inverse-CDF draw over the row's survivors with uniform u (one warp)
-template <typename T>
-__device__ int warp_row_draw(const T* row, const VerifyArgs& a, const RowInfo& ri, const double* cmass,
-                             const int* cties, int nchunks, double u, int lane) {
-    const double target = u * ri.Z;
-    double carry = 0.0;
-    int tcarry = 0;
-    int cstar = -1, tstar = 0;
-    double before = 0.0;
-    for (int c0 = 0; c0 < nchunks && cstar < 0; c0 += 32) {
-        const int c = c0 + lane;
-        const int nt = c < nchunks ? cties[c] : 0;
-        const int tincl = warp_inclusive_scan(nt, lane);
-        const double m = c < nchunks ? chunk_surv(ri, cmass, cties, c, tcarry + tincl - nt) : 0.0;
-        const double incl = warp_scan_f64(m, lane);
-        const unsigned hit = __ballot_sync(kFullMask, c < nchunks && m > 0.0 && carry + incl > target);
-        if (hit) {
-            const int src = __ffs(hit) - 1;
-            cstar = c0 + src;
-            tstar = tcarry + __shfl_sync(kFullMask, tincl - nt, src);
-            before = carry + __shfl_sync(kFullMask, incl - m, src);
-        }
-        carry += __shfl_sync(kFullMask, incl, 31);
-        tcarry += __shfl_sync(kFullMask, tincl, 31);
-    }
-    double tgt = target;
-    if (cstar < 0) {  // rounding left no crossing: the answer is the row's last survivor
-        for (int c = nchunks - 1; c >= 0; --c) {
-            int tb = 0;
-            for (int q = 0; q < c; ++q) tb += cties[q];
-            if (chunk_surv(ri, cmass, cties, c, tb) > 0.0) {
-                cstar = c;
-                tstar = tb;
-                break;
-            }
-        }
-        if (cstar < 0) return -1;
-        tgt = INFINITY;  // no element crosses: the scan below reports the chunk's last survivor
-    }
-    const double target2 = tgt;
-    int found = -1, last = -1;
-    double cum = before;
-    scan_chunk<T>(row, a, ri, cstar, tstar, lane, [&](int64_t id0, const double* wv, int nv, int) {
-        double s = 0.0;
-        for (int e = 0; e < nv; ++e) s += wv[e];
-        const double incl = warp_scan_f64(s, lane);
-        if (found < 0) {
-            const unsigned hit = __ballot_sync(kFullMask, s > 0.0 && cum + incl > target2);
-            if (hit) {
-                const int src = __ffs(hit) - 1;
-                int tok = -1;
-                if (lane == src) {
-                    double cc = cum + incl - s;
-                    for (int e = 0; e < nv; ++e) {
-                        if (wv[e] <= 0.0) continue;
-                        cc += wv[e];
-                        tok = (int)(id0 + e);
-                        if (cc > target2) break;
-                    }
-                }
-                found = __shfl_sync(kFullMask, tok, src);
-            }
-            const unsigned pos = __ballot_sync(kFullMask, s > 0.0);
-            if (pos) {
-                const int src = 31 - __clz(pos);
-                int tl = -1;
-                if (lane == src)
-                    for (int e = 0; e < nv; ++e)
-                        if (wv[e] > 0.0) tl = (int)(id0 + e);
-                last = __shfl_sync(kFullMask, tl, src);
-            }
-        }
-        cum += __shfl_sync(kFullMask, incl, 31);
-    });
-    return found >= 0 ? found : last;
-}
+// 16-bit order key of a bf16 value (larger value, larger key) and back
+__device__ __forceinline__ uint32_t key16(uint32_t h) { return (h & 0x8000u) ? (~h & 0xFFFFu) : (h | 0x8000u); }
+__device__ __forceinline__ uint32_t bits16(uint32_t k) { return (k & 0x8000u) ? (k & 0x7FFFu) : (~k & 0xFFFFu); }
+__device__ __forceinline__ __nv_bfloat162 as_bf2(uint32_t w) { return *reinterpret_cast<const __nv_bfloat162*>(&w); }
 
-// probability of token t under the row's distribution (one warp)
-template <typename T>
-__device__ double warp_row_prob(const T* row, const VerifyArgs& a, const RowInfo& ri, const int* cties, int t,
-                                int lane) {
-    if (t < 0 || t >= a.V) return 0.0;
-    constexpr int CH = Chunk<T>::CH;
-    const int c = t / CH;
-    int tb = 0;
-    if (ri.tau != 0u) {
-        for (int q = lane; q < c; q += 32) tb += cties[q];
-        tb = warp_sum(tb);
-    }
-    double w = 0.0;
-    scan_chunk<T>(row, a, ri, c, tb, lane, [&](int64_t id0, const double* wv, int nv, int) {
-        if (t >= id0 && t < id0 + nv) w = wv[t - id0];
-    });
-    // the owning lane holds w; share it
-    unsigned own = __ballot_sync(kFullMask, w != 0.0);
-    if (own) w = __shfl_sync(kFullMask, w, __ffs(own) - 1);
-    return w / ri.Z;
-}
+// TOPK = false: full-vocabulary mode (top-p over the whole row, or no cut). TOPK = true:
+// top-k (k <= kMaxTopK), then top-p over the k survivors.
+template <bool TOPK>
+__global__ void __launch_bounds__(kThreads, 1) pair_kernel(Params p, Layout Ly) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ __align__(8) uint64_t bars[kTeams][5];
 
-// ---------------------------------------------------------------------------------------
-// CTA-level passes over a pair of rows: residual mass per chunk, or TV
-// ---------------------------------------------------------------------------------------
-template <typename T, typename F>
-__device__ void pair_pass(const T* prow, const T* qrow, const VerifyArgs& a, const RowInfo& rp, const RowInfo& rq,
-                          const int* ctp, const int* ctq, int nchunks, F per_chunk) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int c = warp; c < nchunks; c += kWarps) {
-        int tbp = 0, tbq = 0;
-        if (rp.tau != 0u || rq.tau != 0u) {
-            for (int q = lane; q < c; q += 32) {
-                tbp += ctp[q];
-                tbq += ctq[q];
-            }
-            tbp = warp_sum(tbp);
-            tbq = warp_sum(tbq);
-        }
-        double acc = 0.0;
-        scan_pair_chunk<T>(prow, qrow, a, rp, rq, c, tbp, tbq, lane,
-                           [&](int64_t, const double* wp, const double* wq, int nv) {
-                               for (int e = 0; e < nv; ++e) acc += per_chunk(wp[e], wq[e]);
-                           });
-        acc = warp_sum_f64(acc);
-        (void)acc;
-    }
-}
+    const int team = threadIdx.x / kTeamThreads, tt = threadIdx.x % kTeamThreads;
+    const int tw = tt >> 5, lane = tt & 31;
+    const int CL = Ly.CL;
+    const uint32_t crank = ctarank();
+    const int cid = blockIdx.x / CL, NC = gridDim.x / CL;
+    const int n_items = p.B * p.K;
+    const double T = p.T;
 
-// ---------------------------------------------------------------------------------------
-// the kernel: one CTA per sequence
-// ---------------------------------------------------------------------------------------
-// Row g = b * R + r of the work: verifier rows r < K, then drafter rows 1..K-1.
-template <typename T>
-__device__ __forceinline__ const T* work_row(const VerifyArgs& a, int R, int64_t g) {
-    const int b = (int)(g / R), r = (int)(g % R);
-    const bool isP = r < a.K;
-    const int pos = isP ? r : r - a.K + 1;
-    return reinterpret_cast<const T*>(isP ? a.P : a.Q) + ((int64_t)b * a.K + pos) * a.V;
-}
+    unsigned char* base = smem + (size_t)team * Ly.team_bytes;
+    uint16_t* bufs[2] = {reinterpret_cast<uint16_t*>(base), reinterpret_cast<uint16_t*>(base) + Ly.L};
+    uint32_t* hist = reinterpret_cast<uint32_t*>(base + Ly.off_hist);      // [2][hw]
+    uint2* own = reinterpret_cast<uint2*>(base + Ly.off_own);              // [2][OW]: (+count, -count)
+    double* lut = reinterpret_cast<double*>(base + Ly.off_lut);            // [2][kLut] (full mode)
+    uint64_t* list = reinterpret_cast<uint64_t*>(base + Ly.off_list);      // top-k mode: [2][KL] survivors,
+    uint64_t* ltmp = list + 2 * Ly.KL;                                     //   [2][KL] scratch,
+    double* lw = reinterpret_cast<double*>(ltmp + 2 * Ly.KL);              //   [2][KL] weights,
+    int32_t* lid = reinterpret_cast<int32_t*>(lw + 2 * Ly.KL);             //   [2][KL] ids
+    unsigned long long* x1 = reinterpret_cast<unsigned long long*>(base + Ly.off_x1);  // [kMaxCL]
+    double* x2 = reinterpret_cast<double*>(base + Ly.off_x2);              // [kMaxCL][6]
+    double* x3 = reinterpret_cast<double*>(base + Ly.off_x3);              // [kMaxCL][3]
+    TeamShared& ts = *reinterpret_cast<TeamShared*>(base + Ly.off_misc);
+    uint64_t* full = &bars[team][0];
+    uint64_t* xb1 = &bars[team][1];
+    uint64_t* xb2a = &bars[team][2];
+    uint64_t* xb2b = &bars[team][3];
+    uint64_t* xb3 = &bars[team][4];
 
-// One CTA per row (every row of every sequence): the row's chunk table and RowInfo, the
-// row read from global memory (HBM once, then L2) by every pass.
-template <typename T>
-__global__ void __launch_bounds__(kThreads) rows_kernel(Params p) {
-    __shared__ RowShared sh;
-    const int NC = p.nchunks;
-    const int64_t g = blockIdx.x;
-    int xe = 0;
-    const GlobalRow<T> src{work_row<T>(p.a, p.rows_per_seq, g), p.a.V};
-    prepare_row<T>(src, p.a, 0, NC, p.cmass + g * NC, p.cties + g * NC, p.infos + g, sh, CtaGroup{}, xe);
-}
-
-// Cluster form for bf16 rows whose length is a multiple of 8 (16-byte aligned rows): a
-// cluster of CL CTAs owns one row at a time, CTA r holding chunks [r cpc, (r + 1) cpc) of
-// it in shared memory, so the row is read from HBM exactly once and every pass runs from
-// shared memory; the row-wide reductions go through distributed shared memory (ClusterGroup).
-// Persistent: cluster i takes rows i, i + #clusters, ...; the next row's slice is copied in
-// (one bulk copy per CTA, completion counted on an mbarrier) while this row is processed.
-constexpr int kBulkAlign = 128;
-inline size_t cluster_dyn_smem(int cpc) {
-    return kBulkAlign + 2 * (size_t)cpc * Chunk<__nv_bfloat16>::CH * sizeof(uint16_t);
-}
-
-__global__ void __launch_bounds__(kThreads, 1) rows_cluster_kernel(Params p, int cpc) {
-    extern __shared__ __align__(128) unsigned char dsm[];
-    __shared__ RowShared sh;
-    constexpr int CH = Chunk<__nv_bfloat16>::CH;
-    const VerifyArgs& a = p.a;
-    const int tid = threadIdx.x;
-    const int rank = (int)cl_rank();
-    const ClusterGroup grp{(int)cl_size()};
-    uint64_t* full = reinterpret_cast<uint64_t*>(dsm);  // [2]: a buffer's slice has landed
-    uint16_t* buf = reinterpret_cast<uint16_t*>(dsm + kBulkAlign);
-    const int64_t buf_elems = (int64_t)cpc * CH;
-    const int V = a.V, NC = p.nchunks, R = p.rows_per_seq;
-    const int c0 = min(NC, rank * cpc), c1 = min(NC, c0 + cpc);
-    const int64_t e_lo = min((int64_t)V, (int64_t)c0 * CH), e_hi = min((int64_t)V, (int64_t)c1 * CH);
-    const uint32_t bytes = (uint32_t)((e_hi - e_lo) * 2);  // a multiple of 16; 0 without chunks
-    const int64_t rows = (int64_t)a.B * R;
-    const int64_t first = cl_index(), step = cl_count();
-    uint32_t issued[2] = {0u, 0u}, done[2] = {0u, 0u};  // copies per buffer (thread 0)
-    if (tid == 0) {
-        mbar_init(&full[0], 1);
-        mbar_init(&full[1], 1);
+    if (tt == 0) {
+        mbar_init(full, 1);
+        mbar_init(xb1, CL);
+        mbar_init(xb2a, CL);
+        mbar_init(xb2b, CL);
+        mbar_init(xb3, CL);
+        ts.abort_ = 0;
         fence_mbar_init();
     }
     __syncthreads();
-    auto issue = [&](int64_t g, int bi) {
-        ++issued[bi];
-        if (bytes == 0) {
-            mbar_arrive(&full[bi]);
-            return;
-        }
-        mbar_arrive_expect_tx(&full[bi], bytes);
-        bulk_g2s(buf + bi * buf_elems, work_row<__nv_bfloat16>(a, R, g) + e_lo, bytes, &full[bi]);
-    };
-    bool failed = false;
-    if (tid == 0 && first < rows) issue(first, 0);
-    int xe = 0;
-    int it = 0;
-    for (int64_t g = first; g < rows; g += step, ++it) {
-        const int bi = it & 1;
-        __syncthreads();  // every warp is done with the other buffer (the previous row)
-        if (tid == 0 && !failed && g + step < rows) {
-            fence_proxy_async_smem();
-            issue(g + step, bi ^ 1);
-        }
-        if (!failed) {
-            if (mbar_wait(&full[bi], (uint32_t)(it >> 1) & 1u)) {
-                if (tid == 0) ++done[bi];
-            } else {
-                failed = true;
-                record_device_status(p.status, UNO_ERR_TIMEOUT);
+    cluster_sync_all();  // every CTA's barriers exist before any remote arrive
+
+    const int lo = (int)crank * Ly.L;
+    const int n = max(0, min(Ly.L, p.V - lo));
+    const int nvec = n >> 3;
+    const int pv = (nvec + kTeamWarps - 1) / kTeamWarps;  // vectors per warp part
+    const int wv0 = min(nvec, tw * pv), wv1 = min(nvec, wv0 + pv);
+    const int step = kTeams * NC;
+
+    // the leader (tt == 0) issues the bulk copies of the team's next item
+    int issued = -1, inflight = 0;
+    auto needs_rows = [&](int it) { return !trivial_item(p, it / p.K, it % p.K); };
+    auto issue = [&](int it) {
+        const int i = it % p.K;
+        const int nrows = i > 0 ? 2 : 1;
+        if (n > 0) {
+            mbar_arrive_expect_tx(full, (uint32_t)(n * 2 * nrows));
+            const __nv_bfloat16* Prow = static_cast<const __nv_bfloat16*>(p.P) + (int64_t)it * p.V + lo;
+            bulk_g2s(bufs[0], Prow, (uint32_t)(n * 2), full);
+            if (i > 0) {
+                const __nv_bfloat16* Qrow = static_cast<const __nv_bfloat16*>(p.Q) + (int64_t)it * p.V + lo;
+                bulk_g2s(bufs[1], Qrow, (uint32_t)(n * 2), full);
             }
-        }
-        // (after a timeout the CTA keeps taking part in the cluster's barriers; its results
-        // are not valid, and the status word says so)
-        const SharedSlice src{buf + bi * buf_elems, c0, V};
-        prepare_row<__nv_bfloat16>(src, a, c0, c1, p.cmass + g * NC, p.cties + g * NC,
-                                   rank == 0 ? p.infos + g : nullptr, sh, grp, xe);
-    }
-    // no CTA leaves while another may still read its exchange areas
-    grp.sync();
-    if (tid == 0)  // copies still in flight after a timeout: wait for them (bounded)
-        for (int bi = 0; bi < 2; ++bi)
-            while (done[bi] < issued[bi] && mbar_wait(&full[bi], done[bi] & 1u)) ++done[bi];
-}
-
-template <typename T>
-__global__ void __launch_bounds__(kThreads) seq_kernel(Params p) {
-    __shared__ double dred[kWarps];
-    __shared__ int s_tok[32];
-    __shared__ double s_p[32], s_q[32], s_tv[32];
-    __shared__ int s_acc[32];
-    const VerifyArgs& a = p.a;
-    const int b = blockIdx.x, K = a.K, V = a.V, NC = p.nchunks;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int R = p.rows_per_seq;
-    const int64_t rbase = (int64_t)b * R;
-    auto rowp = [&](int r) -> const T* {
-        const bool isP = r < K;
-        const int pos = isP ? r : r - K + 1;
-        return reinterpret_cast<const T*>(isP ? a.P : a.Q) + ((int64_t)b * K + pos) * V;
-    };
-    // the rows' tables come from rows_kernel (earlier on the stream)
-
-    // per position: draws, probabilities, acceptance (warp per position)
-    for (int i = warp; i < K; i += kWarps) {
-        const RowInfo rp = p.infos[rbase + i];
-        const double* cmp = p.cmass + (rbase + i) * NC;
-        const int* ctp = p.cties + (rbase + i) * NC;
-        const float* u = a.u + ((int64_t)b * K + i) * 3;
-        int tok;
-        double pi = 0.0, qi = 0.0;
-        int acc = 1;
-        if (i == 0) {
-            tok = a.pos0 && a.pos0[b] >= 0 ? a.pos0[b]
-                                           : warp_row_draw<T>(rowp(0), a, rp, cmp, ctp, NC, (double)u[0], lane);
-            pi = warp_row_prob<T>(rowp(0), a, rp, ctp, tok, lane);
         } else {
-            const int rq_i = K + i - 1;
-            const RowInfo rq = p.infos[rbase + rq_i];
-            const double* cmq = p.cmass + (rbase + rq_i) * NC;
-            const int* ctq = p.cties + (rbase + rq_i) * NC;
-            tok = a.drafts ? a.drafts[(int64_t)b * K + i] : warp_row_draw<T>(rowp(rq_i), a, rq, cmq, ctq, NC, (double)u[0], lane);
-            pi = warp_row_prob<T>(rowp(i), a, rp, ctp, tok, lane);
-            qi = warp_row_prob<T>(rowp(rq_i), a, rq, ctq, tok, lane);
-            acc = (double)u[1] * qi < pi;
+            mbar_arrive(full);
         }
-        if (lane == 0) {
-            s_tok[i] = tok;
-            s_p[i] = pi;
-            s_q[i] = qi;
-            s_acc[i] = acc;
-            s_tv[i] = 0.0;
-        }
-    }
-    __syncthreads();
-    int n = K;
-    for (int i = 1; i < K; ++i)
-        if (!s_acc[i]) {
-            n = i;
-            break;
-        }
+        issued = it;
+        inflight = 1;
+    };
 
-    // optional TV per position (i >= 1): 1/2 sum |p - q| over the whole vocabulary
-    if (a.out_tv) {
-        for (int i = 1; i < K; ++i) {
-            const int rq_i = K + i - 1;
-            double part = 0.0;
-            const RowInfo rp = p.infos[rbase + i], rq = p.infos[rbase + rq_i];
-            const int* ctp = p.cties + (rbase + i) * NC;
-            const int* ctq = p.cties + (rbase + rq_i) * NC;
-            pair_pass<T>(rowp(i), rowp(rq_i), a, rp, rq, ctp, ctq, NC, [&](double pv, double qv) {
-                part += fabs(pv - qv);
-                return 0.0;
-            });
-            const double tv = 0.5 * cta_sum_f64(part, dred);
-            if (threadIdx.x == 0) s_tv[i] = tv;
-            __syncthreads();
+    uint32_t xph = 0, lph = 0;  // phases of the exchange barriers and of the buffer barrier
+    uint32_t hph = 0;           // top-k mode: items this CTA has been the head of (its xb3 phase)
+    for (int item = cid + team * NC; item < n_items; item += step) {
+        const int b = item / p.K, i = item % p.K;
+        if (!needs_rows(item)) {
+            if (crank == 0 && tt == 0) write_trivial(p, item, b);
+            continue;
         }
-    }
+        const int nrows = i > 0 ? 2 : 1;
+        if (tt == 0 && issued != item) issue(item);
+        if (tw == 0) {
+            const bool ok = mbar_wait(full, lph & 1);
+            if (!ok && lane == 0) ts.abort_ = 1;
+        }
+        ++lph;
+        if (tt == 0) inflight = 0;
+        team_sync(team);
+        if (ts.abort_) break;
 
-    // the correction token: residual max(0, p_n - q_n) (whole CTA for the per-chunk table)
-    int nxt = -1;
-    if (n < K) {
-        const int rq_n = K + n - 1;
-        const RowInfo rp = p.infos[rbase + n], rq = p.infos[rbase + rq_n];
-        const double* cmp = p.cmass + (rbase + n) * NC;
-        const int* ctp = p.cties + (rbase + n) * NC;
-        const int* ctq = p.cties + (rbase + rq_n) * NC;
-        double* cres = p.cres + (int64_t)b * NC;
-        const T* prow = rowp(n);
-        const T* qrow = rowp(rq_n);
-        // residual mass per chunk (warp per chunk)
-        for (int c = warp; c < NC; c += kWarps) {
-            int tbp = 0, tbq = 0;
-            for (int q = lane; q < c; q += 32) {
-                tbp += ctp[q];
-                tbq += ctq[q];
+        // ---- (1) largest value and magnitude of each row slice ----
+        {
+            __nv_bfloat162 mx[2], mg[2];
+            for (int r = 0; r < 2; ++r) {
+                mx[r] = __floats2bfloat162_rn(-INFINITY, -INFINITY);
+                mg[r] = __floats2bfloat162_rn(0.f, 0.f);
             }
-            tbp = warp_sum(tbp);
-            tbq = warp_sum(tbq);
-            double acc = 0.0;
-            scan_pair_chunk<T>(prow, qrow, a, rp, rq, c, tbp, tbq, lane,
-                               [&](int64_t, const double* wp, const double* wq, int nv) {
-                                   for (int e = 0; e < nv; ++e) {
-                                       const double d = wp[e] - wq[e];
-                                       acc += d > 0.0 ? d : 0.0;
-                                   }
-                               });
-            acc = warp_sum_f64(acc);
-            if (lane == 0) cres[c] = acc;
+            for (int r = 0; r < nrows; ++r) {
+                const uint4* v4 = reinterpret_cast<const uint4*>(bufs[r]);
+                for (int j = tt; j < nvec; j += kTeamThreads) {
+                    const uint4 v = v4[j];
+                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t a = w[q] & 0x7FFF7FFFu;
+                        mx[r] = __hmax2(mx[r], *reinterpret_cast<const __nv_bfloat162*>(&w[q]));
+                        mg[r] = __hmax2(mg[r], *reinterpret_cast<const __nv_bfloat162*>(&a));
+                    }
+                }
+            }
+            float fm[2], fa[2];
+            for (int r = 0; r < 2; ++r) {
+                fm[r] = warp_max(fmaxf(__low2float(mx[r]), __high2float(mx[r])));
+                fa[r] = warp_max(fmaxf(__low2float(mg[r]), __high2float(mg[r])));
+            }
+            if (lane == 0) {
+                ts.dred[tw][0] = fm[0];
+                ts.dred[tw][1] = fa[0];
+                ts.dred[tw][2] = fm[1];
+                ts.dred[tw][3] = fa[1];
+            }
+            // clear the counts (nobody reads them before the exchange below)
+            for (int j = tt; j < 2 * Ly.hw; j += kTeamThreads) hist[j] = 0u;
+            if (TOPK && tt < 2 && (int)crank == item % CL) ts.lcnt[tt] = 0u;
+            team_sync(team);
+            if (tw == 0) {
+                float m0 = -INFINITY, a0 = 0.f, m1 = -INFINITY, a1 = 0.f;
+                for (int w = 0; w < kTeamWarps; ++w) {
+                    m0 = fmaxf(m0, (float)ts.dred[w][0]);
+                    a0 = fmaxf(a0, (float)ts.dred[w][1]);
+                    m1 = fmaxf(m1, (float)ts.dred[w][2]);
+                    a1 = fmaxf(a1, (float)ts.dred[w][3]);
+                }
+                const unsigned long long pk = (unsigned long long)(__float_as_uint(m0) >> 16) |
+                                              ((unsigned long long)(__float_as_uint(a0) >> 16) << 16) |
+                                              ((unsigned long long)(__float_as_uint(m1) >> 16) << 32) |
+                                              ((unsigned long long)(__float_as_uint(a1) >> 16) << 48);
+                if (lane < CL) {
+                    st_remote_u64(mapa(&x1[crank], (uint32_t)lane), pk);
+                    arrive_remote(mapa(xb1, (uint32_t)lane));
+                }
+                const bool ok = wait_cluster(xb1, xph & 1);
+                if (!ok && lane == 0) ts.abort_ = 1;
+                if (lane < 2) {
+                    float M = -INFINITY;
+                    uint32_t A = 0;
+                    for (int r = 0; r < CL; ++r) {
+                        const unsigned long long v = x1[r] >> (32 * lane);
+                        M = fmaxf(M, bf((uint32_t)(v & 0xFFFFu)));
+                        A = max(A, (uint32_t)((v >> 16) & 0xFFFFu));
+                    }
+                    RowStat& rs = ts.rs[lane];
+                    rs.M = M;
+                    rs.atop = A;
+                    rs.kM = key16(__float_as_uint(M) >> 16);
+                    rs.zmax = (double)M / T;
+                }
+            }
+            team_sync(team);
+            if (ts.abort_) break;
         }
-        __syncthreads();
-        if (warp == 0) {
-            const double uu = (double)a.u[((int64_t)b * K + n) * 3 + 2];
-            double Rtot = 0.0;
-            for (int c = lane; c < NC; c += 32) Rtot += cres[c];
-            Rtot = warp_sum_f64(Rtot);
-            if (!(Rtot > 0.0)) {
-                nxt = warp_row_draw<T>(prow, a, rp, cmp, ctp, NC, uu, lane);
-            } else {
-                // walk the residual table, then scan the crossing chunk
-                const double target = uu * Rtot;
-                double carry = 0.0, before = 0.0;
-                int cstar = -1;
-                for (int c0 = 0; c0 < NC && cstar < 0; c0 += 32) {
-                    const int c = c0 + lane;
-                    const double m = c < NC ? cres[c] : 0.0;
+
+        // ---- (2) counts per value: full mode, every magnitude within kWords steps of the
+        //      largest (the rest weighed one by one); top-k mode, the kWinK largest values ----
+        if constexpr (TOPK) {
+            for (int r = 0; r < nrows; ++r) {
+                const uint32_t kM = ts.rs[r].kM;
+                const uint32_t kf = kM >= (uint32_t)(kWinK - 1) ? kM - (uint32_t)(kWinK - 1) : 0u;
+                const uint32_t hf = bits16(kf);
+                const __nv_bfloat162 f2 = as_bf2(hf | (hf << 16));
+                uint32_t* h = hist + r * Ly.hw;
+                const uint4* v4 = reinterpret_cast<const uint4*>(bufs[r]);
+                for (int j = tt; j < nvec; j += kTeamThreads) {
+                    const uint4 v = v4[j];
+                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t m = __hge2_mask(as_bf2(w[q]), f2);
+                        if (m) {
+                            // (-0 passes a +0 floor but lies below it in key order: d checked)
+                            const uint32_t dl = kM - key16(w[q] & 0xFFFFu), dh = kM - key16(w[q] >> 16);
+                            if ((m & 0xFFFFu) && dl < (uint32_t)kWinK) atomicAdd(&h[dl], 1u);
+                            if ((m >> 16) && dh < (uint32_t)kWinK) atomicAdd(&h[dh], 1u);
+                        }
+                    }
+                }
+            }
+            if (lane == 0) {
+                ts.dred[tw][4] = 0.0;
+                ts.dred[tw][5] = 0.0;
+            }
+            team_sync(team);
+            if (tw == 0) {
+                fence_cluster();
+                if (lane < CL) arrive_remote(mapa(xb2a, (uint32_t)lane));
+                const bool ok = wait_cluster(xb2a, xph & 1);
+                if (!ok && lane == 0) ts.abort_ = 1;
+            }
+            team_sync(team);
+            if (ts.abort_) break;
+        } else {
+            double below[2] = {0.0, 0.0};  // fp64 weights of the tokens under the counted band
+            for (int r = 0; r < nrows; ++r) {
+                const RowStat rs = ts.rs[r];
+                uint32_t* h = hist + r * Ly.hw;
+                const uint4* v4 = reinterpret_cast<const uint4*>(bufs[r]);
+                for (int j = tt; j < nvec; j += kTeamThreads) {
+                    const uint4 v = v4[j];
+                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t hl = w[q] & 0xFFFFu, hh = w[q] >> 16;
+                        const uint32_t dl = rs.atop - (hl & 0x7FFFu), dh = rs.atop - (hh & 0x7FFFu);
+                        if (dl < (uint32_t)kWords) atomicAdd(&h[dl], (hl & 0x8000u) ? 0x10000u : 1u);
+                        else if (fabsf(bf(hl)) < INFINITY) below[r] += wexp(hl, rs, T);
+                        if (dh < (uint32_t)kWords) atomicAdd(&h[dh], (hh & 0x8000u) ? 0x10000u : 1u);
+                        else if (fabsf(bf(hh)) < INFINITY) below[r] += wexp(hh, rs, T);
+                    }
+                }
+            }
+            below[0] = warp_sum_f64(below[0]);
+            below[1] = warp_sum_f64(below[1]);
+            if (lane == 0) {
+                ts.dred[tw][4] = below[0];
+                ts.dred[tw][5] = below[1];
+            }
+            team_sync(team);
+            if (tw == 0) {
+                fence_cluster();
+                if (lane < CL) arrive_remote(mapa(xb2a, (uint32_t)lane));
+                const bool ok = wait_cluster(xb2a, xph & 1);
+                if (!ok && lane == 0) ts.abort_ = 1;
+            }
+            team_sync(team);
+            if (ts.abort_) break;
+        }
+
+        // ---- (3) this CTA's share of the values: cluster-wide counts, and (full mode) their
+        //      masses ----
+        {
+            const int w0 = (int)crank * Ly.OW;
+            double pm[2] = {0.0, 0.0}, nm[2] = {0.0, 0.0};
+            for (int r = 0; r < nrows; ++r) {
+                const RowStat rs = ts.rs[r];
+                for (int k = tt; k < Ly.OW; k += kTeamThreads) {
+                    const int d = w0 + k;
+                    uint32_t cp = 0, cn = 0;
+                    for (int q = 0; q < CL; ++q) {
+                        const uint32_t c = ld_remote_u32(mapa(&hist[r * Ly.hw + d], (uint32_t)q));
+                        if constexpr (TOPK) {
+                            cp += c;
+                        } else {
+                            cp += c & 0xFFFFu;
+                            cn += c >> 16;
+                        }
+                    }
+                    own[r * Ly.OW + k] = make_uint2(cp, cn);
+                    if constexpr (TOPK) {
+                        pm[r] += (double)cp;
+                    } else {
+                        if (cp) pm[r] += (double)cp * wexp(word_bits(rs, d, 0), rs, T);
+                        if (cn) nm[r] += (double)cn * wexp(word_bits(rs, d, 1), rs, T);
+                    }
+                }
+            }
+            for (int r = 0; r < 2; ++r) {
+                pm[r] = warp_sum_f64(pm[r]);
+                nm[r] = warp_sum_f64(nm[r]);
+            }
+            team_sync(team);  // dred[.][0..3] of step (1) are no longer read
+            if (lane == 0) {
+                ts.dred[tw][0] = pm[0];
+                ts.dred[tw][1] = nm[0];
+                ts.dred[tw][2] = pm[1];
+                ts.dred[tw][3] = nm[1];
+            }
+            team_sync(team);
+            if (tw == 0) {
+                double v6[6] = {0, 0, 0, 0, 0, 0};
+                for (int w = 0; w < kTeamWarps; ++w) {
+                    v6[0] += ts.dred[w][0];
+                    v6[1] += ts.dred[w][1];
+                    v6[2] += ts.dred[w][4];
+                    v6[3] += ts.dred[w][2];
+                    v6[4] += ts.dred[w][3];
+                    v6[5] += ts.dred[w][5];
+                }
+                if (lane < CL) {
+                    const uint32_t slot = mapa(&x2[crank * 6], (uint32_t)lane);
+                    for (int k = 0; k < 6; ++k) st_remote_f64(slot + 8u * k, v6[k]);
+                    arrive_remote(mapa(xb2b, (uint32_t)lane));
+                }
+                const bool ok = wait_cluster(xb2b, xph & 1);
+                if (!ok && lane == 0) ts.abort_ = 1;
+            }
+            team_sync(team);
+            if (ts.abort_) break;
+        }
+
+        // ---- (4) the cut of each row, identical in every CTA ----
+        if (TOPK && tw < nrows) {  // warp r finds the k-th largest value of row r
+            const int r = tw;
+            RowStat& rs = ts.rs[r];
+            rs.S = 0.0;
+            rs.Sk = 0.0;
+            rs.kbits = 0xFF80u;
+            rs.kd = -1;
+            rs.kneg = 0;
+            rs.tkeep = 0;
+            rs.theta = INT_MAX;
+            const double target = (double)p.top_k;
+            double c = 0.0;
+            int part = -1;
+            for (int q = 0; q < CL && part < 0; ++q) {
+                const double m = x2[q * 6 + 3 * r];
+                if (m > 0.0 && c + m >= target) part = q;
+                else c += m;
+            }
+            int redo = part < 0;  // fewer than k tokens among the counted values
+            if (!redo) {
+                const int w0 = part * Ly.OW;
+                int kd = -1;
+                double cb = 0.0;
+                for (int k0 = 0; k0 < Ly.OW && kd < 0; k0 += 32) {
+                    const int k = k0 + lane;
+                    const uint32_t cnt = k < Ly.OW ? ld_remote_v2(mapa(&own[r * Ly.OW + k], (uint32_t)part)).x : 0u;
+                    const double m = (double)cnt;
                     const double incl = warp_scan_f64(m, lane);
-                    const unsigned hit = __ballot_sync(kFullMask, c < NC && m > 0.0 && carry + incl > target);
+                    const unsigned hit = __ballot_sync(kFullMask, cnt > 0 && c + incl >= target);
                     if (hit) {
                         const int src = __ffs(hit) - 1;
-                        cstar = c0 + src;
-                        before = carry + __shfl_sync(kFullMask, incl - m, src);
+                        kd = w0 + k0 + src;
+                        cb = c + __shfl_sync(kFullMask, incl - m, src);
                     }
-                    carry += __shfl_sync(kFullMask, incl, 31);
+                    c += __shfl_sync(kFullMask, incl, 31);
                 }
-                if (cstar < 0)
-                    for (int c = NC - 1; c >= 0 && cstar < 0; --c)
-                        if (cres[c] > 0.0) {
-                            cstar = c;
-                            before = target;
+                if (kd < 0) {
+                    redo = 1;
+                } else {
+                    rs.kd = kd;
+                    rs.kbits = bits16(rs.kM - (uint32_t)kd);
+                    rs.tkeep = (int)(target - cb);  // the tokens at the k-th value that are kept
+                    // +0 and -0 are one value but two keys: leave such a cut to the generic kernel
+                    if ((rs.kbits & 0x7FFFu) == 0u) redo = 1;
+                }
+            }
+            if (lane == 0) ts.dred[r][0] = redo;
+        }
+        if (!TOPK && tw < nrows) {  // warp r decides row r
+            const int r = tw;
+            RowStat& rs = ts.rs[r];
+            double S = 0.0;
+            for (int q = 0; q < CL; ++q) S += x2[q * 6 + 3 * r + 0];
+            for (int q = 0; q < CL; ++q) S += x2[q * 6 + 3 * r + 2];
+            for (int q = 0; q < CL; ++q) S += x2[q * 6 + 3 * r + 1];
+            rs.S = S;
+            rs.Sk = S;
+            rs.kbits = 0xFF80u;  // -inf: no cut
+            rs.kd = -1;
+            rs.kneg = 0;
+            rs.tkeep = 0;
+            rs.theta = INT_MAX;
+            int redo = !(S > 0.0) || !(S < INFINITY);
+            if (p.cut && !redo) {
+                const double target = p.top_p * S;
+                // value order: positive parts of CTAs 0..CL-1, the uncounted band, negative
+                // parts of CTAs CL-1..0
+                double c = 0.0;
+                int part = -1, neg = 0;
+                for (int q = 0; q < CL && part < 0; ++q) {
+                    const double m = x2[q * 6 + 3 * r + 0];
+                    if (m > 0.0 && c + m >= target) part = q;
+                    else c += m;
+                }
+                if (part < 0) {
+                    double zb = 0.0;
+                    for (int q = 0; q < CL; ++q) zb += x2[q * 6 + 3 * r + 2];
+                    if (zb > 0.0 && c + zb >= target) redo = 1;  // the cut lies among uncounted tokens
+                    c += zb;
+                    for (int q = CL - 1; q >= 0 && part < 0 && !redo; --q) {
+                        const double m = x2[q * 6 + 3 * r + 1];
+                        if (m > 0.0 && c + m >= target) {
+                            part = q;
+                            neg = 1;
+                        } else {
+                            c += m;
                         }
-                int tbp = 0, tbq = 0;
-                for (int q = lane; q < cstar; q += 32) {
-                    tbp += ctp[q];
-                    tbq += ctq[q];
-                }
-                tbp = warp_sum(tbp);
-                tbq = warp_sum(tbq);
-                int found = -1, last = -1;
-                double cum = before;
-                scan_pair_chunk<T>(prow, qrow, a, rp, rq, cstar, tbp, tbq, lane,
-                                   [&](int64_t id0, const double* wp, const double* wq, int nv) {
-                    double r[Elem<T>::VEC];
-                    double s = 0.0;
-                    for (int e = 0; e < Elem<T>::VEC; ++e) {
-                        const double d = e < nv ? wp[e] - wq[e] : 0.0;
-                        r[e] = d > 0.0 ? d : 0.0;
-                        s += r[e];
                     }
-                    const double incl = warp_scan_f64(s, lane);
-                    if (found < 0) {
-                        const unsigned hit = __ballot_sync(kFullMask, s > 0.0 && cum + incl > target);
+                    if (part < 0) redo = 1;  // rounding left the target unmet
+                }
+                if (!redo) {
+                    // scan the owner's words in value order
+                    const int w0 = part * Ly.OW;
+                    int kd = -1;
+                    uint32_t kc = 0;
+                    double cb = 0.0, wk = 0.0;
+                    for (int k0 = 0; k0 < Ly.OW && kd < 0; k0 += 32) {
+                        const int k = k0 + lane;
+                        const int kk = neg ? Ly.OW - 1 - k : k;
+                        uint32_t cnt = 0;
+                        double w = 0.0;
+                        if (k < Ly.OW) {
+                            const uint2 c2 = ld_remote_v2(mapa(&own[r * Ly.OW + kk], (uint32_t)part));
+                            cnt = neg ? c2.y : c2.x;
+                            if (cnt) w = wexp(word_bits(rs, w0 + kk, neg), rs, T);
+                        }
+                        const double m = (double)cnt * w;
+                        const double incl = warp_scan_f64(m, lane);
+                        const unsigned hit = __ballot_sync(kFullMask, cnt > 0 && c + incl >= target);
                         if (hit) {
                             const int src = __ffs(hit) - 1;
-                            int tk = -1;
-                            if (lane == src) {
-                                double cc = cum + incl - s;
-                                for (int e = 0; e < nv; ++e) {
-                                    if (r[e] <= 0.0) continue;
-                                    cc += r[e];
-                                    tk = (int)(id0 + e);
-                                    if (cc > target) break;
+                            kd = w0 + (neg ? Ly.OW - 1 - (k0 + src) : k0 + src);
+                            kc = __shfl_sync(kFullMask, cnt, src);
+                            wk = __shfl_sync(kFullMask, w, src);
+                            cb = c + __shfl_sync(kFullMask, incl - m, src);
+                        }
+                        c += __shfl_sync(kFullMask, incl, 31);
+                    }
+                    if (kd < 0) {
+                        redo = 1;
+                    } else {
+                        long long t = (long long)ceil((target - cb) / wk);
+                        if (t < 1) t = 1;
+                        if (t > (long long)kc) t = kc;
+                        while (t > 1 && cb + (double)(t - 1) * wk >= target) --t;
+                        while (t < (long long)kc && cb + (double)t * wk < target) ++t;
+                        rs.kd = kd;
+                        rs.kneg = neg;
+                        rs.kbits = word_bits(rs, kd, neg);
+                        rs.wk = wk;
+                        rs.tkeep = (int)t;
+                        rs.Sk = cb + (double)t * wk;
+                        // +0 and -0 are one value but two counts: leave such a cut to the
+                        // generic kernel
+                        if ((rs.kbits & 0x7FFFu) == 0u) redo = 1;
+                    }
+                }
+            }
+            if (lane == 0) ts.dred[r][0] = redo;  // dred[0..1][0] are free here
+        }
+        team_sync(team);
+        {
+            const int redo = (int)ts.dred[0][0] | (nrows > 1 ? (int)ts.dred[1][0] : 0);
+            team_sync(team);
+            if (redo) {
+                if (crank == 0 && tt == 0) p.recs[item].state = kRedo;
+                // full mode: the exchange of step (6) still runs so that every barrier keeps its
+                // phase; top-k mode: every CTA skips steps (5) to (7) alike
+            }
+            const bool cutting = TOPK || p.cut;
+            // survivor weights of the top positive values (full mode)
+            for (int r = 0; r < nrows && !TOPK; ++r) {
+                RowStat& rs = ts.rs[r];
+                int ln = kLut;
+                if (p.cut && rs.kd >= 0 && !rs.kneg) ln = min(kLut, rs.kd + 1);
+                for (int d = tt; d < ln; d += kTeamThreads)
+                    lut[r * kLut + d] = ((int)rs.atop - d >= 0) ? wexp(word_bits(rs, d, 0), rs, T) : 0.0;
+                if (tt == 0) rs.lut_n = (int)min((uint32_t)ln, rs.atop + 1u);
+            }
+
+            // ---- (5) where the kept ties end: counts of the tie value in lower-ranked CTAs ----
+            if (cutting && !redo && tw < nrows) {
+                const int r = tw;
+                RowStat& rs = ts.rs[r];
+                long long before = 0;
+                uint32_t mine = 0;
+                for (int q = 0; q < CL; ++q) {
+                    uint32_t c = 0;
+                    if (lane == 0) c = ld_remote_u32(mapa(&hist[r * Ly.hw + rs.kd], (uint32_t)q));
+                    if (!TOPK) c = rs.kneg ? (c >> 16) : (c & 0xFFFFu);
+                    if (q < (int)crank) before += c;
+                    if (q == (int)crank) mine = c;
+                }
+                if (lane == 0) {
+                    const long long keep = min((long long)mine, max(0LL, (long long)rs.tkeep - before));
+                    ts.ured[r][0] = (uint32_t)keep;
+                    ts.ured[r][1] = mine;
+                }
+            }
+            team_sync(team);
+            for (int r = 0; r < nrows && cutting && !redo; ++r) {
+                RowStat& rs = ts.rs[r];
+                const uint32_t keep = ts.ured[r][0], mine = ts.ured[r][1];
+                if (keep == mine) {
+                    if (tt == 0) rs.theta = INT_MAX;
+                } else if (keep == 0) {
+                    if (tt == 0) rs.theta = 0;
+                } else {
+                    // this CTA holds the boundary: find its keep-th tie in id order
+                    const uint16_t* buf = bufs[r];
+                    int c = 0;
+                    for (int e = wv0 * 8 + lane; e < wv1 * 8; e += 32) c += elem(buf, e) == rs.kbits;
+                    c = warp_sum(c);
+                    if (lane == 0) ts.ipart[tw] = c;
+                    team_sync(team);
+                    int before = 0, wt = 0;
+                    for (; wt < kTeamWarps; ++wt) {
+                        if (before + ts.ipart[wt] >= (int)keep) break;
+                        before += ts.ipart[wt];
+                    }
+                    if (tw == wt) {
+                        int need = (int)keep - before, found = -1;
+                        for (int e0 = wv0 * 8; e0 < wv1 * 8 && found < 0; e0 += 32) {
+                            const int e = e0 + lane;
+                            const unsigned bal = __ballot_sync(kFullMask, e < wv1 * 8 && elem(buf, e) == rs.kbits);
+                            const int nb = __popc(bal);
+                            if (nb >= need) {
+                                unsigned bb = bal;
+                                for (int q = 1; q < need; ++q) bb &= bb - 1;
+                                found = e0 + __ffs(bb) - 1;
+                            }
+                            need -= nb;
+                        }
+                        if (lane == 0) rs.theta = lo + found + 1;
+                    }
+                }
+                team_sync(team);
+            }
+            team_sync(team);
+
+            if constexpr (TOPK) {
+                if (!redo) {
+                    const int head = item % CL;
+                    // ---- (6) the top-k survivors, appended to the head CTA's lists ----
+                    for (int r = 0; r < nrows; ++r) {
+                        const RowStat rs = ts.rs[r];
+                        const __nv_bfloat162 k2 = as_bf2(rs.kbits | (rs.kbits << 16));
+                        const float kx = bf(rs.kbits);
+                        const uint32_t cnt_addr = mapa(&ts.lcnt[r], (uint32_t)head);
+                        const uint32_t list_addr = mapa(&list[r * Ly.KL], (uint32_t)head);
+                        const uint4* v4 = reinterpret_cast<const uint4*>(bufs[r]);
+                        for (int j = tt; j < nvec; j += kTeamThreads) {
+                            const uint4 v = v4[j];
+                            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                const uint32_t m = __hge2_mask(as_bf2(w[q]), k2);
+                                if (!m) continue;
+#pragma unroll
+                                for (int hh = 0; hh < 2; ++hh) {
+                                    if (!((m >> (16 * hh)) & 1u)) continue;
+                                    const uint32_t h16 = (w[q] >> (16 * hh)) & 0xFFFFu;
+                                    const float x = bf(h16);
+                                    const int id = lo + j * 8 + 2 * q + hh;
+                                    if (x == kx && id >= rs.theta) continue;  // a tie past the kept ones
+                                    const uint32_t slot = atom_remote_add(cnt_addr, 1u);
+                                    if (slot < (uint32_t)Ly.KL)
+                                        st_remote_u64(list_addr + 8u * slot, pack_candidate(float_key(x), (uint32_t)id));
                                 }
                             }
-                            found = __shfl_sync(kFullMask, tk, src);
-                        }
-                        const unsigned pos = __ballot_sync(kFullMask, s > 0.0);
-                        if (pos) {
-                            const int src = 31 - __clz(pos);
-                            int tl = -1;
-                            if (lane == src)
-                                for (int e = 0; e < nv; ++e)
-                                    if (r[e] > 0.0) tl = (int)(id0 + e);
-                            last = __shfl_sync(kFullMask, tl, src);
                         }
                     }
-                    cum += __shfl_sync(kFullMask, incl, 31);
-                });
-                nxt = found >= 0 ? found : last;
+                    team_sync(team);
+                    if (tt == 0) {
+                        fence_cluster();
+                        arrive_remote(mapa(xb3, (uint32_t)head));
+                    }
+                    // ---- (7) the head: softmax and top-p over the survivors, the draws, the tests ----
+                    if ((int)crank == head) {
+                        if (tw == 0) {
+                            const bool ok = wait_cluster(xb3, hph & 1);
+                            if (!ok && lane == 0) ts.abort_ = 1;
+                        }
+                        ++hph;
+                        team_sync(team);
+                        if (ts.abort_) break;
+                        if (tw < nrows) {  // warp r: row r's survivor record
+                            const int r = tw;
+                            const int nk = (int)min(ts.lcnt[r], (unsigned)Ly.KL);
+                            uint64_t* Lr = list + r * Ly.KL;
+                            uint64_t* Tr = ltmp + r * Ly.KL;
+                            double* Wr = lw + r * Ly.KL;
+                            int32_t* Ir = lid + r * Ly.KL;
+                            int n2 = 32;
+                            while (n2 < nk) n2 <<= 1;
+                            for (int j = nk + lane; j < n2; j += 32) Lr[j] = 0ull;
+                            __syncwarp();
+                            warp_sort_desc(Lr, n2, lane);  // (value desc, id asc)
+                            const double zmax = ts.rs[r].zmax;
+                            double S1 = 0.0;
+                            for (int j = lane; j < nk; j += 32) {
+                                const double w = exp((double)key_float(candidate_key(Lr[j])) / T - zmax);
+                                Tr[j] = __double_as_longlong(w);
+                                S1 += w;
+                            }
+                            S1 = warp_sum_f64(S1);
+                            __syncwarp();
+                            // top-p: the shortest prefix of that order whose mass reaches top_p
+                            int np = nk;
+                            if (p.cut) {
+                                double carry = 0.0;
+                                for (int j0 = 0; j0 < nk; j0 += 32) {
+                                    const int j = j0 + lane;
+                                    const double x = j < nk ? __longlong_as_double(Tr[j]) / S1 : 0.0;
+                                    const double incl = warp_scan_f64(x, lane);
+                                    const unsigned hit = __ballot_sync(kFullMask, j < nk && carry + incl >= p.top_p);
+                                    if (hit) {
+                                        np = j0 + __ffs(hit);
+                                        break;
+                                    }
+                                    carry += __shfl_sync(kFullMask, incl, 31);
+                                }
+                            }
+                            // the survivors in id order, with their weights
+                            int sid[kMaxTopK / 32];
+                            double sw[kMaxTopK / 32];
+                            for (int j = lane, t = 0; j < n2; j += 32, ++t) {
+                                const uint32_t id = j < np ? candidate_id(Lr[j]) : 0xFFFFFFFFu;
+                                sid[t] = (int)id;
+                                sw[t] = j < np ? __longlong_as_double(Tr[j]) : 0.0;
+                            }
+                            __syncwarp();
+                            for (int j = lane, t = 0; j < n2; j += 32, ++t)
+                                Lr[j] = j < np ? (((uint64_t)(0xFFFFFFFFu - (uint32_t)sid[t]) << 32) | (uint32_t)j) : 0ull;
+                            for (int j = lane, t = 0; j < n2; j += 32, ++t) Tr[j] = __double_as_longlong(sw[t]);
+                            __syncwarp();
+                            warp_sort_desc(Lr, n2, lane);  // ascending id
+                            double Z = 0.0;
+                            for (int j = lane; j < np; j += 32) {
+                                const uint32_t src = (uint32_t)(Lr[j] & 0xFFFFFFFFu);
+                                Ir[j] = (int32_t)(0xFFFFFFFFu - (uint32_t)(Lr[j] >> 32));
+                                Wr[j] = __longlong_as_double(Tr[src]);
+                                Z += Wr[j];
+                            }
+                            Z = warp_sum_f64(Z);
+                            if (lane == 0) {
+                                ts.np[r] = np;
+                                ts.Z[r] = Z;
+                            }
+                        }
+                        team_sync(team);
+                        if (tw == 0) {
+                            const float* u = p.u + (int64_t)item * 3;
+                            SRec P;
+                            P.w = lw;
+                            P.id = lid;
+                            P.n = ts.np[0];
+                            P.Z = ts.Z[0];
+                            Rec rec;
+                            rec.state = kDone;
+                            rec.pad = 0.0;
+                            if (i == 0) {
+                                const int x0 = pos0_given(p, b) ? p.pos0[b] : srec_inv_cdf(P, (double)u[0], lane);
+                                rec.tok = x0;
+                                rec.res = -1;
+                                rec.acc = 1;
+                                rec.p = (x0 >= 0 && x0 < p.V) ? srec_prob(P, x0) : 0.0;
+                                rec.q = 0.0;
+                                rec.tv = 0.0;
+                            } else {
+                                SRec Q;
+                                Q.w = lw + Ly.KL;
+                                Q.id = lid + Ly.KL;
+                                Q.n = ts.np[1];
+                                Q.Z = ts.Z[1];
+                                const int d = p.drafts ? p.drafts[item] : srec_inv_cdf(Q, (double)u[0], lane);
+                                const bool in = d >= 0 && d < p.V;
+                                rec.tok = d;
+                                rec.p = in ? srec_prob(P, d) : 0.0;
+                                rec.q = in ? srec_prob(Q, d) : 0.0;
+                                rec.acc = (double)u[1] * rec.q < rec.p;
+                                rec.tv = srec_tv(P, Q, lane);
+                                rec.res = srec_residual(P, Q, (double)u[2], lane);
+                            }
+                            if (lane == 0) p.recs[item] = rec;
+                        }
+                    }
+                }
+            } else {
+            // ---- (6) masses per warp part: draw row, verifier survivors, residual ----
+            const int draw_row = i > 0 ? 1 : 0;
+            const RowStat rp = ts.rs[0];
+            const RowStat rq = ts.rs[nrows > 1 ? 1 : 0];
+            const double iSp = 1.0 / rp.Sk, iSq = 1.0 / rq.Sk;
+            double sd = 0.0, sp = 0.0, sr = 0.0;
+            if (!redo) {
+                const uint32_t kp = rp.kbits | (rp.kbits << 16), kq = rq.kbits | (rq.kbits << 16);
+                const uint4* vp = reinterpret_cast<const uint4*>(bufs[0]);
+                const uint4* vq = reinterpret_cast<const uint4*>(bufs[1]);
+                for (int j = wv0 + lane; j < wv1; j += 32) {
+                    const uint4 a = vp[j];
+                    const uint32_t wa[4] = {a.x, a.y, a.z, a.w};
+                    uint32_t ma = 0, mb = 0;
+                    uint32_t wb[4] = {0, 0, 0, 0};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        ma |= __hge2_mask(*reinterpret_cast<const __nv_bfloat162*>(&wa[q]),
+                                          *reinterpret_cast<const __nv_bfloat162*>(&kp));
+                    if (nrows > 1) {
+                        const uint4 bq = vq[j];
+                        wb[0] = bq.x;
+                        wb[1] = bq.y;
+                        wb[2] = bq.z;
+                        wb[3] = bq.w;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            mb |= __hge2_mask(*reinterpret_cast<const __nv_bfloat162*>(&wb[q]),
+                                              *reinterpret_cast<const __nv_bfloat162*>(&kq));
+                    }
+                    if (!(ma | mb)) continue;
+                    const int e0 = lo + j * 8;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const uint32_t hp = (wa[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
+                        const double wp = surv_weight(hp, e0 + e, rp, lut, T, p.cut);
+                        double wq = 0.0;
+                        if (nrows > 1) {
+                            const uint32_t hq = (wb[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
+                            wq = surv_weight(hq, e0 + e, rq, lut + kLut, T, p.cut);
+                        }
+                        sd += draw_row ? wq : wp;
+                        sp += wp;
+                        if (wp > 0.0) {
+                            const double dl = wp * iSp - wq * iSq;
+                            if (dl > 0.0) sr += dl;
+                        }
+                    }
+                }
             }
+            sd = warp_sum_f64(sd);
+            sp = warp_sum_f64(sp);
+            sr = warp_sum_f64(sr);
+            if (lane == 0) {
+                ts.wpart[tw][0] = sd;
+                ts.wpart[tw][1] = sp;
+                ts.wpart[tw][2] = sr;
+            }
+            team_sync(team);
+            if (tw == 0) {
+                double v3[3] = {0, 0, 0};
+                for (int w = 0; w < kTeamWarps; ++w)
+                    for (int k = 0; k < 3; ++k) v3[k] += ts.wpart[w][k];
+                if (lane < CL) {
+                    const uint32_t slot = mapa(&x3[crank * 3], (uint32_t)lane);
+                    for (int k = 0; k < 3; ++k) st_remote_f64(slot + 8u * k, v3[k]);
+                    arrive_remote(mapa(xb3, (uint32_t)lane));
+                }
+                const bool ok = wait_cluster(xb3, xph & 1);
+                if (!ok && lane == 0) ts.abort_ = 1;
+            }
+            team_sync(team);
+            if (ts.abort_) break;
+
+            // ---- (7) the draws: the CTA and warp part holding each target, then its token ----
+            if (!redo) {
+                const float* u = p.u + (int64_t)item * 3;
+                // mode 0: the draw row's survivors, 1: verifier survivors, 2: residual
+                auto weight_at = [&](int mode, int e) -> double {  // e: element of this slice
+                    const uint32_t hp = elem(bufs[0], e);
+                    const double wp = surv_weight(hp, lo + e, rp, lut, T, p.cut);
+                    if (mode == 1 || (mode == 0 && !draw_row)) return wp;
+                    const double wq = surv_weight(elem(bufs[1], e), lo + e, rq, lut + kLut, T, p.cut);
+                    if (mode == 0) return wq;
+                    if (!(wp > 0.0)) return 0.0;
+                    const double dl = wp * iSp - wq * iSq;
+                    return dl > 0.0 ? dl : 0.0;
+                };
+                // returns the token id (only meaningful in the owning CTA), or -1 elsewhere;
+                // identical owner choice in every CTA from the exchanged totals
+                auto find = [&](int mode, double target) -> int {
+                    double c = 0.0, clast = 0.0;
+                    int owner = -1, last = -1;
+                    for (int q = 0; q < CL; ++q) {
+                        const double m = x3[q * 3 + mode];
+                        if (!(m > 0.0)) continue;
+                        last = q;
+                        clast = c;
+                        if (c + m > target) {
+                            owner = q;
+                            break;
+                        }
+                        c += m;
+                    }
+                    const bool last_mode = owner < 0;
+                    if (last_mode) {
+                        owner = last;
+                        c = clast;
+                    }
+                    if (owner != (int)crank) return -1;
+                    double c2 = c, c2last = c;
+                    int wsel = -1, wlast = -1;
+                    for (int w = 0; w < kTeamWarps; ++w) {
+                        const double m = ts.wpart[w][mode];
+                        if (!(m > 0.0)) continue;
+                        wlast = w;
+                        c2last = c2;
+                        if (!last_mode && c2 + m > target) {
+                            wsel = w;
+                            break;
+                        }
+                        c2 += m;
+                    }
+                    const bool lm = last_mode || wsel < 0;
+                    if (wsel < 0) {
+                        wsel = wlast;
+                        c2 = c2last;
+                    }
+                    int res = -1;
+                    if (tw == wsel) {
+                        const int v0 = min(nvec, wsel * pv) * 8, v1 = min(nvec, wsel * pv + pv) * 8;
+                        double carry = c2;
+                        int lastpos = -1;
+                        for (int base = v0; base < v1 && res < 0; base += 32) {
+                            const int e = base + lane;
+                            const double x = e < v1 ? weight_at(mode, e) : 0.0;
+                            const double incl = warp_scan_f64(x, lane);
+                            const unsigned hit = lm ? 0u : __ballot_sync(kFullMask, x > 0.0 && carry + incl > target);
+                            if (hit) res = lo + base + __ffs(hit) - 1;
+                            const unsigned pos = __ballot_sync(kFullMask, x > 0.0);
+                            if (pos) lastpos = lo + base + 31 - __clz(pos);
+                            carry += __shfl_sync(kFullMask, incl, 31);
+                        }
+                        if (res < 0) res = lastpos;
+                    }
+                    return res;
+                };
+                // the item's token: drawn, or supplied
+                int tok = -1;
+                bool tok_here = false;
+                if (i == 0 ? !pos0_given(p, b) : !p.drafts) {
+                    const double target = (double)u[0] * (draw_row ? rq.Sk : rp.Sk);
+                    tok = find(0, target);
+                    tok_here = tok >= 0;
+                } else {
+                    tok = i == 0 ? p.pos0[b] : p.drafts[item];
+                    const bool in = tok >= 0 && tok < p.V;
+                    tok_here = in ? (tok >= lo && tok < lo + n) : crank == 0;
+                    tok_here = tok_here && tw == 0;
+                }
+                if (tok_here && lane == 0) {
+                    const bool in = tok >= 0 && tok < p.V;
+                    double pd = 0.0, qd = 0.0;
+                    if (in) {
+                        pd = surv_weight(elem(bufs[0], tok - lo), tok, rp, lut, T, p.cut) * iSp;
+                        if (i > 0) qd = surv_weight(elem(bufs[1], tok - lo), tok, rq, lut + kLut, T, p.cut) * iSq;
+                    }
+                    Rec& rec = p.recs[item];
+                    rec.tok = tok;
+                    rec.p = pd;
+                    rec.q = qd;
+                    rec.acc = i == 0 ? 1 : ((double)u[1] * qd < pd);
+                }
+                if (i > 0) {
+                    double R = 0.0;
+                    for (int q = 0; q < CL; ++q) R += x3[q * 3 + 2];
+                    const int mode = R > 0.0 ? 2 : 1;
+                    const int res = find(mode, (double)u[2] * (R > 0.0 ? R : rp.Sk));
+                    if (res >= 0 && lane == 0) p.recs[item].res = res;
+                    if (crank == 0 && tt == 0) {
+                        p.recs[item].tv = R;
+                        p.recs[item].state = kDone;
+                    }
+                } else if (crank == 0 && tt == 0) {
+                    p.recs[item].res = -1;
+                    p.recs[item].tv = 0.0;
+                    p.recs[item].state = kDone;
+                }
+            }
+            }  // full mode
+        }
+        ++xph;
+        team_sync(team);  // the buffer is free
+        if (tt == 0) {
+            int nx = item + step;
+            while (nx < n_items && !needs_rows(nx)) nx += step;
+            if (nx < n_items) issue(nx);
         }
     }
+    // a copy issued for an item this team will not process (after an abort): let it land
+    if (tt == 0 && inflight) mbar_wait(full, lph & 1, 1u << 16);
+    __syncthreads();
+    cluster_sync_all();  // no CTA leaves while another may still read its shared memory
+    if (tt == 0 && ts.abort_) record_device_status(p.status, (uint32_t)UNO_ERR_TIMEOUT);
+}
 
-    if (warp == 0) {
-        const int i = lane;
-        if (i < K) {
-            const int64_t o = (int64_t)b * K + i;
-            a.out_tokens[o] = i < n ? s_tok[i] : -1;
-            if (a.out_p) a.out_p[o] = (float)s_p[i];
-            if (a.out_q) a.out_q[o] = (float)s_q[i];
-            if (a.out_tv) a.out_tv[o] = (float)s_tv[i];
-        }
-        if (lane == 0) {
-            a.out_count[b] = n;
-            if (a.out_next) a.out_next[b] = n < K ? nxt : -1;
-        }
+}  // namespace pk
+
+// =======================================================================================
+// per sequence: the longest accepted prefix and the outputs
+// =======================================================================================
+__global__ void assemble_kernel(Params p, int32_t* out_tokens, int32_t* out_count, int32_t* out_next, float* out_p,
+                                float* out_q, float* out_tv) {
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= p.B) return;
+    const int K = p.K;
+    const Rec* r = p.recs + (int64_t)b * K;
+    int n = 1;
+    while (n < K && r[n].acc) ++n;
+    for (int i = 0; i < K; ++i) {
+        const int64_t o = (int64_t)b * K + i;
+        out_tokens[o] = i < n ? r[i].tok : -1;
+        if (out_p) out_p[o] = (float)r[i].p;
+        if (out_q) out_q[o] = (float)r[i].q;
+        if (out_tv) out_tv[o] = (float)r[i].tv;
     }
+    out_count[b] = n;
+    if (out_next) out_next[b] = n < K ? r[n].res : -1;
 }
 
-struct Layout {
-    int nchunks, rows_per_seq;
-    size_t off_cmass, off_cties, off_cres, off_infos, total;
-};
+// =======================================================================================
+// host side
+// =======================================================================================
+inline size_t recs_bytes(const VerifyArgs& a) { return align_up((size_t)a.B * a.K * sizeof(Rec), 256); }
 
-inline Layout layout(const VerifyArgs& a) {
-    Layout L{};
-    const int CH = a.dtype == UNO_BF16 ? Chunk<__nv_bfloat16>::CH : Chunk<float>::CH;
-    L.nchunks = (a.V + CH - 1) / CH;
-    L.rows_per_seq = 2 * a.K - 1;
-    const size_t rows = (size_t)a.B * L.rows_per_seq;
-    L.off_cmass = 0;
-    L.off_cties = align_up(rows * L.nchunks * 8, 256);
-    L.off_cres = align_up(L.off_cties + rows * L.nchunks * 4, 256);
-    L.off_infos = align_up(L.off_cres + (size_t)a.B * L.nchunks * 8, 256);
-    L.total = align_up(L.off_infos + rows * sizeof(RowInfo), 256);
-    return L;
-}
-
-// Cluster size for the rows: UNO_VERIFY_FULL_CLUSTER (1, 2, 4, 8 or 16) if set, else the
-// smallest size whose two slice buffers fit in shared memory next to RowShared.
-inline bool cluster_fits(int nchunks, int c, size_t room) {
-    const int cpc = (nchunks + c - 1) / c;
-    return cpc * kVecPerLane <= kMaxUnits && cluster_dyn_smem(cpc) <= room;
-}
-inline int choose_cluster(int nchunks, size_t room) {
-    if (const char* e = getenv("UNO_VERIFY_FULL_CLUSTER")) {
-        const int c = atoi(e);
-        if (c == 1 || c == 2 || c == 4 || c == 8 || c == 16) return cluster_fits(nchunks, c, room) ? c : 0;
+// the team layout for cluster size CL; top_k > 0 selects the top-k mode
+pk::Layout make_layout(int V, int CL, int top_k) {
+    pk::Layout Ly{};
+    Ly.CL = CL;
+    Ly.L = (int)(((int64_t)V + (int64_t)CL * 8 - 1) / ((int64_t)CL * 8) * 8);
+    Ly.hw = top_k > 0 ? pk::kWinK : pk::kWords;
+    Ly.OW = Ly.hw / CL;
+    Ly.KL = 0;
+    if (top_k > 0) {
+        Ly.KL = 32;
+        while (Ly.KL < top_k) Ly.KL <<= 1;
     }
-    for (int c = 1; c <= 16; c *= 2)
-        if (cluster_fits(nchunks, c, room)) return c;
-    return 0;
+    uint32_t off = (uint32_t)align_up((size_t)Ly.L * 2 * 2, 16);
+    Ly.off_hist = off;
+    off += (uint32_t)(2 * Ly.hw * 4);
+    Ly.off_own = off;
+    off += (uint32_t)(2 * Ly.OW * 8);
+    Ly.off_lut = off;
+    off += top_k > 0 ? 0u : 2u * pk::kLut * 8u;
+    Ly.off_list = off;
+    off += (uint32_t)(2 * Ly.KL * (8 + 8 + 8 + 4));
+    off = (uint32_t)align_up(off, 16);
+    Ly.off_x1 = off;
+    off += pk::kMaxCL * 8;
+    Ly.off_x2 = off;
+    off += pk::kMaxCL * 6 * 8;
+    Ly.off_x3 = off;
+    off += pk::kMaxCL * 3 * 8;
+    Ly.off_misc = off;
+    off += (uint32_t)align_up(sizeof(pk::TeamShared), 16);
+    Ly.team_bytes = (uint32_t)align_up(off, 128);
+    return Ly;
 }
 
-struct ClusterDevice {
+struct DeviceInfo {
     bool ready = false;
-    size_t dyn_max = 0;  // dynamic shared memory a CTA may use beside the kernel's static part
-    std::map<std::pair<int, size_t>, int> max_clusters;  // (cluster size, dynamic smem) -> co-resident clusters
+    size_t dyn_max = 0;
+    std::map<std::tuple<int, int, size_t>, int> max_clusters;  // (mode, cluster size, smem) -> resident clusters
 };
-std::mutex g_cluster_mu;
-ClusterDevice g_cluster_dev[64];
+std::mutex g_mu;
+DeviceInfo g_dev[64];
 
-// Launch rows_cluster_kernel when it applies (bf16, V a multiple of 8, 16-byte aligned
-// logits, a cluster that fits) and UNO_VERIFY_FULL is not "rows"; returns false to fall back
-// to the per-row kernel. UNO_VERIFY_FULL=cluster makes a case that cannot take the cluster
-// form an error (UNO_ERR_UNSUPPORTED) instead of a fallback.
-bool launch_rows_cluster(const Params& p, cudaStream_t stream, uno_status& st) {
-    const VerifyArgs& a = p.a;
+template <bool TOPK>
+bool set_attributes(int dyn_max) {
+    return cudaFuncSetAttribute(pk::pair_kernel<TOPK>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_max) ==
+               cudaSuccess &&
+           cudaFuncSetAttribute(pk::pair_kernel<TOPK>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+               cudaSuccess;
+}
+
+// Launch pair_kernel where it applies; false (with st untouched) to leave every item to the
+// generic kernel. UNO_VERIFY_FULL=generic always leaves them; UNO_VERIFY_FULL=cluster makes a
+// case the pair kernel cannot take an error. UNO_VERIFY_FULL_CLUSTER=c forces the cluster size.
+bool launch_pairs(const VerifyArgs& a, const Params& p, cudaStream_t stream, uno_status& st) {
     const char* mode = getenv("UNO_VERIFY_FULL");
-    if (mode && strcmp(mode, "rows") == 0) return false;
+    if (mode && strcmp(mode, "generic") == 0) return false;
     const bool required = mode && strcmp(mode, "cluster") == 0;
     auto no = [&](const char* why) {
-        if (required) st = set_error(UNO_ERR_UNSUPPORTED, "verify (full vocabulary): no cluster form: %s", why);
+        if (required) st = set_error(UNO_ERR_UNSUPPORTED, "verify: no cluster form: %s", why);
         return required;
     };
     if (a.dtype != UNO_BF16 || a.V % 8 != 0) return no("bf16 rows whose length is a multiple of 8 only");
+    if (a.top_k > pk::kMaxTopK) return no("top-k above 256");
     if ((reinterpret_cast<uintptr_t>(a.P) | reinterpret_cast<uintptr_t>(a.Q)) & 15u)
         return no("logits must be 16-byte aligned");
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return no("no current device");
-    std::lock_guard<std::mutex> lock(g_cluster_mu);
-    ClusterDevice& di = g_cluster_dev[dev];
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceInfo& di = g_dev[dev];
     if (!di.ready) {
         int optin = 0;
-        cudaFuncAttributes fa{};
+        cudaFuncAttributes fa{}, fb{};
         if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
-            cudaFuncGetAttributes(&fa, rows_cluster_kernel) != cudaSuccess || optin <= (int)fa.sharedSizeBytes) {
+            cudaFuncGetAttributes(&fa, pk::pair_kernel<false>) != cudaSuccess ||
+            cudaFuncGetAttributes(&fb, pk::pair_kernel<true>) != cudaSuccess) {
             cudaGetLastError();
             return no("shared memory attributes unavailable");
         }
-        const int dyn_max = optin - (int)fa.sharedSizeBytes;
-        if (cudaFuncSetAttribute(rows_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_max) !=
-                cudaSuccess ||
-            cudaFuncSetAttribute(rows_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
-                cudaSuccess) {
+        const int stat = (int)std::max(fa.sharedSizeBytes, fb.sharedSizeBytes);
+        if (optin <= stat) return no("shared memory attributes unavailable");
+        const int dyn_max = optin - stat;
+        if (!set_attributes<false>(dyn_max) || !set_attributes<true>(dyn_max)) {
             cudaGetLastError();
             return no("kernel attributes refused");
         }
         di.dyn_max = (size_t)dyn_max;
         di.ready = true;
     }
-    const int c = choose_cluster(p.nchunks, di.dyn_max);
-    if (c == 0) return no("the row slices do not fit in the shared memory of this cluster size");
-    const int cpc = (p.nchunks + c - 1) / c;
+    int forced = 0;
+    if (const char* e = getenv("UNO_VERIFY_FULL_CLUSTER")) forced = atoi(e);
+    int CL = 0;
+    pk::Layout Ly{};
+    for (int c = 1; c <= pk::kMaxCL; c *= 2) {
+        if (forced && c != forced) continue;
+        const pk::Layout t = make_layout(a.V, c, a.top_k);
+        if (t.L >= 65536) continue;  // per-CTA counts are 16-bit
+        if ((size_t)t.team_bytes * pk::kTeams <= di.dyn_max) {
+            CL = c;
+            Ly = t;
+            break;
+        }
+    }
+    if (CL == 0) return no("the row slices do not fit in the shared memory of any cluster size");
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)c;
+    attr[0].val.clusterDim.x = (unsigned)CL;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = cluster_dyn_smem(cpc);
+    cfg.blockDim = dim3(pk::kThreads);
+    cfg.dynamicSmemBytes = (size_t)Ly.team_bytes * pk::kTeams;
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const auto key = std::make_pair(c, cfg.dynamicSmemBytes);
+    const bool topk = a.top_k > 0;
+    const auto key = std::make_tuple((int)topk, CL, cfg.dynamicSmemBytes);
     int maxc = 0;
     const auto found = di.max_clusters.find(key);
     if (found != di.max_clusters.end()) {
         maxc = found->second;
     } else {
         cudaLaunchConfig_t q = cfg;
-        q.gridDim = dim3((unsigned)c);
-        if (cudaOccupancyMaxActiveClusters(&maxc, rows_cluster_kernel, &q) != cudaSuccess) {
+        q.gridDim = dim3((unsigned)CL);
+        const cudaError_t e = topk ? cudaOccupancyMaxActiveClusters(&maxc, pk::pair_kernel<true>, &q)
+                                   : cudaOccupancyMaxActiveClusters(&maxc, pk::pair_kernel<false>, &q);
+        if (e != cudaSuccess) {
             cudaGetLastError();
             maxc = 0;
         }
         di.max_clusters[key] = maxc;
     }
     if (maxc <= 0) return no("no cluster of this size can be resident");
-    const int64_t rows = (int64_t)a.B * p.rows_per_seq;
-    const int64_t clusters = std::min<int64_t>(rows, (int64_t)maxc);
-    cfg.gridDim = dim3((unsigned)(clusters * c));
-    st = check_cuda(cudaLaunchKernelEx(&cfg, rows_cluster_kernel, p, cpc), "launch(verify full rows, cluster)");
+    const int64_t items = (int64_t)a.B * a.K;
+    const int64_t clusters = std::min<int64_t>((items + pk::kTeams - 1) / pk::kTeams, (int64_t)maxc);
+    cfg.gridDim = dim3((unsigned)(clusters * CL));
+    const cudaError_t e = topk ? cudaLaunchKernelEx(&cfg, pk::pair_kernel<true>, p, Ly)
+                               : cudaLaunchKernelEx(&cfg, pk::pair_kernel<false>, p, Ly);
+    st = check_cuda(e, "launch(verify, pairs)");
     return true;
+}
+
+int num_sms() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 1;
+    }
+    return n;
 }
 
 }  // namespace vfull
 
-size_t verify_full_workspace_bytes(const VerifyArgs& a) { return vfull::layout(a).total; }
+size_t verify_full_workspace_bytes(const VerifyArgs& a) { return vfull::recs_bytes(a); }
 
-uno_status verify_full_launch(const VerifyArgs& a, void* workspace, cudaStream_t stream) {
-    const vfull::Layout L = vfull::layout(a);
-    unsigned char* ws = static_cast<unsigned char*>(workspace);
+// The item path: pair_kernel where it applies, the generic kernel for the rest, then the
+// per-sequence assembly. With allow_generic false (top-k on: the streaming path serves the
+// cases pair_kernel does not take) nothing is launched unless pair_kernel takes the batch.
+uno_status verify_full_launch(const VerifyArgs& a, void* workspace, cudaStream_t stream, bool allow_generic,
+                              bool* taken) {
     vfull::Params p{};
-    p.a = a;
-    p.rows_per_seq = L.rows_per_seq;
-    p.nchunks = L.nchunks;
-    p.cmass = reinterpret_cast<double*>(ws + L.off_cmass);
-    p.cties = reinterpret_cast<int*>(ws + L.off_cties);
-    p.cres = reinterpret_cast<double*>(ws + L.off_cres);
-    p.infos = reinterpret_cast<vfull::RowInfo*>(ws + L.off_infos);
+    p.P = a.P;
+    p.Q = a.Q;
+    p.B = a.B;
+    p.K = a.K;
+    p.V = a.V;
+    p.T = (double)a.temperature;
+    p.cut = a.top_p < 1.0f;
+    p.top_p = (double)a.top_p;
+    p.top_k = a.top_k;
+    p.need_p0 = a.out_p != nullptr;
+    p.drafts = a.drafts;
+    p.pos0 = a.pos0;
+    p.u = a.u;
+    p.recs = static_cast<vfull::Rec*>(workspace);
     p.status = device_status_ptr();
-    const unsigned rows = (unsigned)((int64_t)a.B * L.rows_per_seq);
-    if (a.dtype == UNO_BF16) {
-        uno_status st = UNO_OK;
-        if (!vfull::launch_rows_cluster(p, stream, st))
-            vfull::rows_kernel<__nv_bfloat16><<<rows, vfull::kThreads, 0, stream>>>(p);
-        else if (st != UNO_OK)
-            return st;
-        vfull::seq_kernel<__nv_bfloat16><<<(unsigned)a.B, vfull::kThreads, 0, stream>>>(p);
-    } else {
-        vfull::rows_kernel<float><<<rows, vfull::kThreads, 0, stream>>>(p);
-        vfull::seq_kernel<float><<<(unsigned)a.B, vfull::kThreads, 0, stream>>>(p);
+    uno_status st = UNO_OK;
+    int only_redo = 0;
+    if (vfull::launch_pairs(a, p, stream, st)) {
+        if (st != UNO_OK) return st;
+        only_redo = 1;
+    } else if (!allow_generic) {
+        *taken = false;
+        return UNO_OK;
     }
-    return check_cuda(cudaGetLastError(), "launch(verify full)");
+    *taken = true;
+    const int items = a.B * a.K;
+    const unsigned grid = (unsigned)std::min(items, 2 * vfull::num_sms());
+    if (a.dtype == UNO_BF16)
+        vfull::gen::item_kernel<__nv_bfloat16><<<grid, vfull::gen::kThreads, 0, stream>>>(p, only_redo);
+    else
+        vfull::gen::item_kernel<float><<<grid, vfull::gen::kThreads, 0, stream>>>(p, only_redo);
+    if ((st = check_cuda(cudaGetLastError(), "launch(verify, generic)")) != UNO_OK) return st;
+    vfull::assemble_kernel<<<(unsigned)((a.B + 127) / 128), 128, 0, stream>>>(p, a.out_tokens, a.out_count, a.out_next,
+                                                                             a.out_p, a.out_q, a.out_tv);
+    return check_cuda(cudaGetLastError(), "launch(verify, assemble)");
 }
 
 }  // namespace uno

@@ -14,11 +14,15 @@ prefix is kept and the first position is the exact AR token):
   4. the correction token becomes the next step's carried token.
 There is no model: the projections' activations and the verifier / drafter logits are
 seeded synthetic inputs of the right shapes (a model's forward would compute them from the
-noised tokens); each step's uniforms come from a small pool. Every step is the same
-sequence of launches, so it can be captured once in a CUDA graph and replayed.
+noised tokens). Each step's activations and uniforms come from a small pool and are copied
+into the step's input buffers before its launches, so consecutive steps compute on
+different data. Every step is the same sequence of launches, so it can be captured once in
+a CUDA graph and replayed.
 tokens_per_forward() is the mean accepted count per sequence and step.
 """
 from __future__ import annotations
+
+import dataclasses
 
 import numpy as np
 import torch
@@ -38,12 +42,22 @@ class DraftVerifyDriver:
             return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(bf).to(self.dev)
 
         self.lin = []
+        self.x = {}  # the step's activations, one buffer per input width (read by the captured launches)
         for sh in linears.shapes:
             inp = W.linear_inputs(linears, sh)
             ws = torch.empty(_lib.uno_gated_lora_linear_workspace_size(linears.M, sh.d_in, sh.d_out, linears.rank),
                              dtype=torch.uint8, device=self.dev)
-            self.lin.append(dict(shape=sh, x=t(inp["x"]), w0=t(inp["w0"]), a=t(inp["a"]), b=t(inp["b"]), ws=ws,
+            if sh.d_in not in self.x:
+                self.x[sh.d_in] = torch.empty((linears.M, sh.d_in), dtype=bf, device=self.dev)
+            self.lin.append(dict(shape=sh, x=self.x[sh.d_in], w0=t(inp["w0"]), a=t(inp["a"]), b=t(inp["b"]), ws=ws,
                                  y=torch.empty((linears.M, sh.d_out), dtype=bf, device=self.dev)))
+        # pool entry s draws its activations from the workload's seed + s (entry 0 is the
+        # workload's own X); they stay on the device and are copied in per step
+        self.pool_x = []
+        for s in range(pool):
+            lw = dataclasses.replace(linears, seed=linears.seed + s)
+            self.pool_x.append({d: t(W.linear_inputs(lw, next(sh for sh in linears.shapes if sh.d_in == d))["x"])
+                                for d in self.x})
         P, Q = W.verify_logits(v)
         self.P_host, self.Q_host = P, Q
         self.P = t(P).view(v.B, v.K, v.V)
@@ -68,6 +82,10 @@ class DraftVerifyDriver:
         """The uniforms of step s (verify [B, K, 3], noise [B, K])."""
         return self.pool_u[s % len(self.pool_u)], self.pool_noise[s % len(self.pool_noise)]
 
+    def pool_linear_workload(self, s: int) -> W.GatedLoraWorkload:
+        """The workload whose X (W.linear_inputs) step s's projections read."""
+        return dataclasses.replace(self.lw, seed=self.lw.seed + s % len(self.pool_x))
+
     def _ops(self):
         v, lw = self.v, self.lw
         _lib.uno_block_noise(self.carry, self.u_noise, v.V, self.noised, self.gate)
@@ -91,6 +109,8 @@ class DraftVerifyDriver:
         u, un = self.pool_inputs(self.steps)
         self.u.copy_(torch.from_numpy(u))
         self.u_noise.copy_(torch.from_numpy(un))
+        for d, x in self.pool_x[self.steps % len(self.pool_x)].items():
+            self.x[d].copy_(x)
         if self.graph is not None:
             self.graph.replay()
         else:

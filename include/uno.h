@@ -85,6 +85,10 @@ int uno_version(void);
  * Device status word: kernels whose bounded waits time out record UNO_ERR_TIMEOUT there
  * instead of trapping. This call synchronises the current device, returns the word in
  * *code (UNO_OK if no kernel recorded anything since the last read) and clears it.
+ * There is one word per device, shared by every stream and host thread that uses the
+ * library on that device: a timeout recorded by any call since the last read is reported
+ * to whichever caller reads first. Callers that run calls concurrently on several streams
+ * learn that some call timed out, not which.
  */
 uno_status uno_read_device_status(uint32_t* code);
 

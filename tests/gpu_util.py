@@ -62,40 +62,95 @@ def decision_path_margin(ref, b):
     return float(np.min(m)) if m.size else np.inf
 
 
-def compare_verify(gpu, ref, check_tv=True, near_eps=NEAR):
-    """Compare GPU and oracle verify outputs sequence by sequence.
+def _path(ref, b):
+    """The oracle's decisions for sequence b in the order they are taken, as
+    (position, margin) pairs: per reached position the top-p cuts of P_i and Q_i, the draw
+    and the acceptance test; at the first rejection the residual draw. A margin of inf is a
+    decision that was not taken (a supplied token, top-p off, i = 0 for the drafter)."""
+    K = ref["tokens"].shape[1]
+    n = int(ref["count"][b])
+    out = []
+    for i in range(min(n, K - 1) + 1):
+        m = ref["margins"][b, i]
+        for c in (3, 4, 0, 1):
+            if np.isfinite(m[c]):
+                out.append((i, float(m[c])))
+        if i == n and n < K and np.isfinite(m[2]):
+            out.append((i, float(m[2])))
+    return out
 
-    A sequence whose decision path has an oracle margin below `near_eps` is excused (not
-    compared) and counted. Returns (n_sequences, n_excused, mismatch descriptions,
-    n_literal_near) where the last counts sequences with a margin below the stated 1e-4.
+
+class Comparison:
+    """Result of comparing GPU and oracle verify outputs (see compare_verify)."""
+
+    def __init__(self):
+        self.n = 0               # sequences
+        self.matched = 0         # sequences whose outputs all agree
+        self.excused = 0         # sequences with a difference explained by a decision in the band
+        self.decisions = 0       # decisions taken on the oracle's paths
+        self.near = 0            # of them within the band
+        self.literal_near = 0    # of them within the stated 1e-4
+        self.bad = []
+
+    def check(self, min_matched=0.9, max_excused_frac=1e-3):
+        """No unexplained difference; at least `min_matched` of the sequences compared in
+        full; excused decisions below `max_excused_frac` of all decisions."""
+        assert not self.bad, self.bad[:5]
+        assert self.matched >= min_matched * self.n, f"only {self.matched} of {self.n} sequences compared"
+        assert self.excused <= max_excused_frac * self.decisions, \
+            f"{self.excused} excused of {self.decisions} decisions"
+        return self
+
+
+def compare_verify(gpu, ref, check_tv=True, band=NEAR_FP64):
+    """Compare GPU and oracle verify outputs sequence by sequence, every output.
+
+    A difference is excused only if a decision taken before it on the oracle's path (or the
+    differing decision itself) has an oracle margin below `band`: that decision may go the
+    other way when both sides evaluate it in fp64 with different summation orders. Every
+    other difference is a failure. Outputs after the first difference depend on it and are
+    not compared further.
     """
     B, K = ref["tokens"].shape
-    bad, near, literal = [], 0, 0
+    c = Comparison()
+    c.n = B
     for b in range(B):
-        m = decision_path_margin(ref, b)
-        literal += m < NEAR
-        if m < near_eps:
-            near += 1
+        path = _path(ref, b)
+        c.decisions += len(path)
+        c.near += sum(m < band for _, m in path)
+        c.literal_near += sum(m < NEAR for _, m in path)
+        n_ref, n_gpu = int(ref["count"][b]), int(gpu["count"][b])
+        first = None   # first differing position (K for a difference in the correction token only)
+        why = None
+        for i in range(K):
+            if gpu["tokens"][b, i] != ref["tokens"][b, i]:
+                first, why = i, f"token {i}: {gpu['tokens'][b, i]} vs {ref['tokens'][b, i]}"
+                break
+        if first is None and n_gpu != n_ref:
+            first, why = min(n_gpu, n_ref), f"count {n_gpu} vs {n_ref}"
+        if first is None and gpu["next"][b] != ref["next"][b]:
+            first, why = K, f"next {gpu['next'][b]} vs {ref['next'][b]}"
+        if first is None:
+            upto = min(n_ref + 1, K)
+            ep = np.abs(gpu["p_tok"][b, :upto] - ref["p_tok"][b, :upto]).max()
+            eq = np.abs(gpu["q_tok"][b, :upto] - ref["q_tok"][b, :upto]).max()
+            if ep > PROB_TOL or eq > PROB_TOL:
+                c.bad.append(f"seq {b}: p/q error {ep:.3g} {eq:.3g}")
+                continue
+            if check_tv and gpu.get("tv") is not None:
+                rows_ok = np.min(ref["margins"][b, :, 3:5], axis=1) >= band  # top-p cuts decided
+                et = np.abs(gpu["tv"][b] - ref["tv"][b])[rows_ok]
+                if et.size and et.max() > PROB_TOL:
+                    c.bad.append(f"seq {b}: tv error {et.max():.3g}")
+                    continue
+            c.matched += 1
             continue
-        if gpu["count"][b] != ref["count"][b]:
-            bad.append(f"seq {b}: count {gpu['count'][b]} vs {ref['count'][b]}")
-            continue
-        if not np.array_equal(gpu["tokens"][b], ref["tokens"][b]):
-            bad.append(f"seq {b}: tokens {gpu['tokens'][b]} vs {ref['tokens'][b]}")
-        if gpu["next"][b] != ref["next"][b]:
-            bad.append(f"seq {b}: next {gpu['next'][b]} vs {ref['next'][b]}")
-        n = int(ref["count"][b])
-        upto = min(n + 1, K)
-        ep = np.abs(gpu["p_tok"][b, :upto] - ref["p_tok"][b, :upto]).max()
-        eq = np.abs(gpu["q_tok"][b, :upto] - ref["q_tok"][b, :upto]).max()
-        if ep > PROB_TOL or eq > PROB_TOL:
-            bad.append(f"seq {b}: p/q error {ep:.3g} {eq:.3g}")
-        if check_tv and gpu.get("tv") is not None:
-            rows_ok = np.min(ref["margins"][b, :, 3:5], axis=1) >= near_eps  # top-p cuts decided
-            et = np.abs(gpu["tv"][b] - ref["tv"][b])[rows_ok]
-            if et.size and et.max() > PROB_TOL:
-                bad.append(f"seq {b}: tv error {et.max():.3g}")
-    return B, near, bad, literal
+        before = [m for i, m in path if i <= first]
+        if before and min(before) < band:
+            c.excused += 1
+        else:
+            c.bad.append(f"seq {b}: {why} (smallest margin on the path {min(before) if before else np.inf:.3g})")
+    return c
 
 
 def bf16_ulp(x: np.ndarray) -> np.ndarray:

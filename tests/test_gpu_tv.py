@@ -117,17 +117,23 @@ def test_tv_empty_mask_and_empty_batch():
     assert float(mean_t.cpu()[0]) == 0.0
 
 
-def test_tv_full_size_sampled_rows():
-    """N = 16384 tokens, V = 151936, bf16: the whole batch runs on the GPU; the oracle
-    recomputes 12 sampled rows; the mean is checked against the GPU's own per-token TV."""
+def test_tv_full_size_rows_and_mean():
+    """N = 16384 tokens, V = 151936, bf16: the whole batch runs on the GPU. The oracle
+    recomputes the TV of every row (in blocks of rows, without the gradient) and so the mean,
+    and the gradient of 288 rows spread over the batch (every residue of the row index modulo
+    any cluster count up to 16 is among them, so every cluster's share is checked)."""
     w = W.TV_LOSS
     T, S = W.tv_logits(w)
     tv, mean, g = _run(T, S, "bf16")
-    rows = np.array([0, 1, 777, 4095, 4096, 8191, 9000, 12000, 15000, 16380, 16382, 16383])
-    Tr, Sr = W.tv_logits(w, rows)
-    Tf, Sf = W.to_f64(Tr, "bf16"), W.to_f64(Sr, "bf16")
+    ref_tv = np.empty(w.N)
+    for r0 in range(0, w.N, 1024):
+        Tf, Sf = W.to_f64(T[r0:r0 + 1024], "bf16"), W.to_f64(S[r0:r0 + 1024], "bf16")
+        ref_tv[r0:r0 + 1024] = oracle.tv_loss(Tf, Sf, want_grad=False)["tv"]
+    np.testing.assert_allclose(tv, ref_tv, atol=PROB_TOL, rtol=0)
+    assert abs(mean - ref_tv.mean()) <= PROB_TOL
+    rows = np.unique(np.concatenate([np.arange(0, w.N, 57), [1, 4095, 4096, 8191, 16382, 16383]]))
+    assert len(rows) >= 256
+    Tf, Sf = W.to_f64(T[rows], "bf16"), W.to_f64(S[rows], "bf16")
     ref = oracle.tv_loss(Tf, Sf, want_absdiff=True)
-    np.testing.assert_allclose(tv[rows], ref["tv"], atol=PROB_TOL, rtol=0)
-    # gradient of the sampled rows: the oracle's per-row gradient carries 1/N_mask = 1/N
+    # the oracle's per-row gradient carries 1/N_mask = 1/len(rows); the batch's is 1/N
     _compare_grad(g[rows], ref["grad"] * len(rows) / w.N, ref["absdiff"], _psum(Tf, Sf))
-    assert abs(mean - tv.astype(np.float64).mean()) < 1e-6

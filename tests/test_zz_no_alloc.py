@@ -30,25 +30,34 @@ def _host(outs):
     return [o.cpu().numpy() for o in outs]
 
 
-@pytest.mark.parametrize("top_k,top_p", [(50, 0.95), (0, 0.95)])
-def test_noalloc_matches_workspace_entry_point(top_k, top_p):
-    w = W.VerifyWorkload("noalloc", 4242 + top_k, B=64, K=16, V=151936, sigma=3.0, rho=0.8, temperature=1.0,
+def _batch(top_k, top_p, seed):
+    w = W.VerifyWorkload("noalloc", seed, B=64, K=16, V=151936, sigma=3.0, rho=0.8, temperature=1.0,
                          top_k=top_k, top_p=top_p)
     P, Q = W.verify_logits(w)
     u = W.verify_uniforms(w)
-    Pd, Qd = dev(P, "bf16").view(64, 16, -1), dev(Q, "bf16").view(64, 16, -1)
-    ud = torch.from_numpy(u).cuda()
-    ref = _outs(64, 16)
-    _lib.uno_block_verify(Pd, Qd, 1.0, top_k, top_p, ud, *ref)
-    ref = _host(ref)
-    for _ in range(2):  # two calls in a row on the shared array
+    return (dev(P, "bf16").view(64, 16, -1), dev(Q, "bf16").view(64, 16, -1), 1.0, top_k, top_p,
+            torch.from_numpy(u).cuda())
+
+
+def test_noalloc_matches_workspace_entry_point():
+    # two batches that use the shared array differently: the top-k path (top-k 50) and the
+    # full-vocabulary path (top-k off), with different logits and uniforms
+    batches = [_batch(50, 0.95, 4292), _batch(0, 0.95, 4242)]
+    refs = []
+    for args in batches:
+        ref = _outs(64, 16)
+        _lib.uno_block_verify(*args, *ref)
+        refs.append(_host(ref))
+    # the no-alloc calls alternate between the batches, so each call finds the array as the
+    # other batch left it; every call must still give the workspace entry point's results
+    for call, which in enumerate((0, 0, 1, 0, 1, 1)):
         got = _outs(64, 16)
-        _lib.uno_block_verify_noalloc(Pd, Qd, 1.0, top_k, top_p, ud, *got)
+        _lib.uno_block_verify_noalloc(*batches[which], *got)
         got = _host(got)
-        for a, b in zip(got[:3], ref[:3]):
-            np.testing.assert_array_equal(a, b)
-        for a, b in zip(got[3:], ref[3:]):
-            np.testing.assert_allclose(a, b, atol=PROB_TOL, rtol=0)
+        for a, b in zip(got[:3], refs[which][:3]):
+            np.testing.assert_array_equal(a, b, err_msg=f"call {call}")
+        for a, b in zip(got[3:], refs[which][3:]):
+            np.testing.assert_allclose(a, b, atol=PROB_TOL, rtol=0, err_msg=f"call {call}")
     assert _lib.uno_read_device_status() == 0
 
 
