@@ -645,6 +645,272 @@ __global__ void __launch_bounds__(kThreads, 1) cluster_kernel(Params p, int64_t 
     cluster_sync();
 }
 
+// ---------------------------------------------------------------------------------------
+// team_kernel: the same computation with two teams of eight warps per CTA on alternate rows.
+// A team waits for its cluster reductions and its copies while the other team computes, so
+// those latencies overlap instead of adding up. Each team holds one (teacher, student) slice
+// pair (the gradient replaces the teacher slice and is streamed out by the team's leader,
+// who then brings in the team's next row); exp(student) is recomputed where it is needed
+// rather than kept (5 exponentials per element pair instead of 3), which is what lets two
+// row pairs fit in shared memory. Reductions: each warp stores its partial into slot
+// [rank][warp] of every CTA of the cluster and arrives on that CTA's barrier.
+// ---------------------------------------------------------------------------------------
+constexpr int kTeams = 2;
+constexpr int kTeamWarps = 8;
+constexpr int kTeamThreads = kTeamWarps * 32;
+constexpr int kTeamKernelThreads = kTeams * kTeamThreads;
+constexpr int kMaxCL = 16;
+
+__host__ __device__ inline size_t team_slice_bytes(int64_t n) { return ((size_t)n * 4 + 127) / 128 * 128; }
+__host__ __device__ inline size_t team_bytes(int64_t n) {
+    return team_slice_bytes(n) + (size_t)kMaxCL * kTeamWarps * (16 + 8);
+}
+
+__device__ __forceinline__ void team_sync(int team) {
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "n"(kTeamThreads) : "memory");
+}
+__device__ __forceinline__ void st_remote_v4(uint32_t addr, float a, float b, float c, float d) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+__device__ __forceinline__ void st_remote_v2(uint32_t addr, float a, float b) {
+    asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a), "f"(b) : "memory");
+}
+__device__ __forceinline__ void arrive_remote(uint32_t bar) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool wait_cluster(uint64_t* bar, uint32_t parity) {
+    for (uint32_t k = 0; k < kWaitLimit; ++k) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred q;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 q, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, q;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+        if (ok) return true;
+    }
+    return false;
+}
+
+__global__ void __launch_bounds__(kTeamKernelThreads, 1) team_kernel(Params p, int64_t n) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ __align__(8) uint64_t bars[kTeams][3];  // slices landed, reduction 0, reduction 1
+    __shared__ double s_tv[kTeams];
+    __shared__ uint32_t s_rows[kTeams];
+    __shared__ int s_abort[kTeams];
+    const TVArgs& a = p.a;
+    const int team = threadIdx.x / kTeamThreads, tt = threadIdx.x % kTeamThreads;
+    const int tw = tt >> 5, lane = tt & 31;
+    const uint32_t rank = cluster_rank(), ncta = cluster_size();
+    unsigned char* base = smem + (size_t)team * team_bytes(n);
+    uint16_t* tin = reinterpret_cast<uint16_t*>(base);  // teacher slice, then the gradient
+    uint16_t* sin = tin + n;                            // student slice
+    float4* s0 = reinterpret_cast<float4*>(base + team_slice_bytes(n));  // [kMaxCL][kTeamWarps]
+    float2* s1 = reinterpret_cast<float2*>(s0 + kMaxCL * kTeamWarps);     // [kMaxCL][kTeamWarps]
+    uint64_t* full = &bars[team][0];
+    uint64_t* red0 = &bars[team][1];
+    uint64_t* red1 = &bars[team][2];
+    const int64_t N = a.N, V = a.V;
+    const int64_t lo = (int64_t)rank * n;
+    const int cnt = (int)max((int64_t)0, min(n, V - lo));
+    const uint32_t bytes = (uint32_t)cnt * 2u;
+    const int units = cnt / 8;
+    const __nv_bfloat16* T = reinterpret_cast<const __nv_bfloat16*>(a.teacher);
+    const __nv_bfloat16* S = reinterpret_cast<const __nv_bfloat16*>(a.student);
+    __nv_bfloat16* G = reinterpret_cast<__nv_bfloat16*>(a.grad);
+    const uint32_t n_mask = p.work->n_mask;
+    const int64_t NC = num_clusters();
+    const int64_t step = kTeams * NC;
+    const int64_t r0 = (int64_t)cluster_id() + team * NC;
+
+    if (tt == 0) {
+        mbar_init(full, 1);
+        mbar_init(red0, ncta * kTeamWarps);
+        mbar_init(red1, ncta * kTeamWarps);
+        s_tv[team] = 0.0;
+        s_rows[team] = 0u;
+        s_abort[team] = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    cluster_sync();  // every CTA's barriers exist before any remote arrive
+
+    auto issue = [&](int64_t r) {  // the leader brings in row r's slices
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(full, 2u * bytes);
+        bulk_g2s(tin, T + r * V + lo, bytes, full);
+        bulk_g2s(sin, S + r * V + lo, bytes, full);
+    };
+    if (tt == 0 && cnt > 0 && r0 < N) issue(r0);
+
+    uint32_t k = 0;
+    for (int64_t r = r0; r < N; r += step, ++k) {
+        const uint32_t par = k & 1;
+        if (cnt > 0 && tw == 0) {
+            const bool ok = mbar_wait(full, par);
+            if (!ok && lane == 0) s_abort[team] = 1;
+        }
+        team_sync(team);
+        if (s_abort[team]) break;
+
+        // ---- this warp's maxima, then its sums of exp(x - warp max) ----
+        __nv_bfloat162 mt2 = __floats2bfloat162_rn(-INFINITY, -INFINITY), ms2 = mt2;
+        for (int u = tt; u < units; u += kTeamThreads) {
+            const uint4 wt = lds128(tin + u * 8), ws = lds128(sin + u * 8);
+            const uint32_t at4[4] = {wt.x, wt.y, wt.z, wt.w}, as4[4] = {ws.x, ws.y, ws.z, ws.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                mt2 = __hmax2(mt2, *reinterpret_cast<const __nv_bfloat162*>(&at4[j]));
+                ms2 = __hmax2(ms2, *reinterpret_cast<const __nv_bfloat162*>(&as4[j]));
+            }
+        }
+        const float mt = warp_max(fmaxf(__low2float(mt2), __high2float(mt2)));
+        const float ms = warp_max(fmaxf(__low2float(ms2), __high2float(ms2)));
+        const float lt = (mt == -INFINITY ? 0.f : mt) * kLog2e, ls = (ms == -INFINITY ? 0.f : ms) * kLog2e;
+        const f2 L2E = pk(kLog2e, kLog2e), NLT = pk(-lt, -lt), NLS = pk(-ls, -ls);
+        f2 zt2 = pk(0.f, 0.f), zs2 = zt2;
+        for (int u = tt; u < units; u += kTeamThreads) {
+            const uint4 wt = lds128(tin + u * 8), ws = lds128(sin + u * 8);
+            const uint32_t at4[4] = {wt.x, wt.y, wt.z, wt.w}, as4[4] = {ws.x, ws.y, ws.z, ws.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const f2 xt = fma2(widen(at4[j]), L2E, NLT), xs = fma2(widen(as4[j]), L2E, NLS);
+                zt2 = add2(zt2, pk(ex2(lo_of(xt)), ex2(hi_of(xt))));
+                zs2 = add2(zs2, pk(ex2(lo_of(xs)), ex2(hi_of(xs))));
+            }
+        }
+        const float zt = warp_sum(lo_of(zt2) + hi_of(zt2)), zs = warp_sum(lo_of(zs2) + hi_of(zs2));
+        // ---- reduction 0: row maxima and sums ----
+        if ((uint32_t)lane < ncta) {
+            st_remote_v4(map_rank(&s0[rank * kTeamWarps + tw], lane), mt, zt, ms, zs);
+            arrive_remote(map_rank(red0, lane));
+        }
+        if (!wait_cluster(red0, par) && lane == 0) s_abort[team] = 1;
+        float Mt = -INFINITY, Ms = -INFINITY;
+        for (uint32_t j = lane; j < ncta * kTeamWarps; j += 32) {
+            const float4 w = s0[j];
+            Mt = fmaxf(Mt, w.x);
+            Ms = fmaxf(Ms, w.z);
+        }
+        Mt = warp_max(Mt);
+        Ms = warp_max(Ms);
+        float Zt = 0.f, Zs = 0.f;
+        for (uint32_t j = lane; j < ncta * kTeamWarps; j += 32) {
+            const float4 w = s0[j];
+            if (w.y > 0.f) Zt += w.y * ex2((w.x - Mt) * kLog2e);
+            if (w.w > 0.f) Zs += w.w * ex2((w.z - Ms) * kLog2e);
+        }
+        Zt = warp_sum(Zt);
+        Zs = warp_sum(Zs);
+        // p = exp(t - wmt) at, q = exp(s - wms) as; q > p  <=>  s - t > K (see cluster_kernel)
+        const float at = mt == -INFINITY ? 0.f : ex2(lt - Mt * kLog2e) / Zt;
+        const float as = ms == -INFINITY ? 0.f : ex2(ls - Ms * kLog2e) / Zs;
+        const float K = (Ms - Mt) + logf(Zs / Zt);
+
+        // ---- A = sum of q over q > p, P = sum of p over q > p ----
+        float Araw = 0.f, Praw = 0.f;
+        for (int u = tt; u < units; u += kTeamThreads) {
+            const uint4 wt = lds128(tin + u * 8), ws = lds128(sin + u * 8);
+            const uint32_t at4[4] = {wt.x, wt.y, wt.z, wt.w}, as4[4] = {ws.x, ws.y, ws.z, ws.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const f2 t2 = widen(at4[j]), s2 = widen(as4[j]);
+                const f2 dl = sub2(s2, t2);
+                const f2 xt = fma2(t2, L2E, NLT), xs = fma2(s2, L2E, NLS);
+                if (lo_of(dl) > K) {
+                    Araw += ex2(lo_of(xs));
+                    Praw += ex2(lo_of(xt));
+                }
+                if (hi_of(dl) > K) {
+                    Araw += ex2(hi_of(xs));
+                    Praw += ex2(hi_of(xt));
+                }
+            }
+        }
+        const float Aw = warp_sum(Araw * as), Pw = warp_sum(Praw * at);
+        if ((uint32_t)lane < ncta) {
+            st_remote_v2(map_rank(&s1[rank * kTeamWarps + tw], lane), Aw, Pw);
+            arrive_remote(map_rank(red1, lane));
+        }
+        if (!wait_cluster(red1, par) && lane == 0) s_abort[team] = 1;
+        float Af = 0.f, Pf = 0.f;
+        for (uint32_t j = lane; j < ncta * kTeamWarps; j += 32) {
+            const float2 w = s1[j];
+            Af += w.x;
+            Pf += w.y;
+        }
+        Af = warp_sum(Af);
+        Pf = warp_sum(Pf);
+        const bool on = a.mask == nullptr || a.mask[r] != 0;
+
+        // ---- gradient f q (1 - A) where q > p, -f q A elsewhere, over the teacher slice ----
+        if (G != nullptr) {
+            const bool grad_on = on && n_mask > 0;
+            const float f = grad_on ? a.grad_scale / (float)n_mask : 0.f;
+            const float kp = f * (1.f - Af) * as, kn = -f * Af * as;
+            for (int u = tt; u < units; u += kTeamThreads) {
+                uint4 o = make_uint4(0u, 0u, 0u, 0u);
+                if (grad_on) {
+                    const uint4 wt = lds128(tin + u * 8), ws = lds128(sin + u * 8);
+                    const uint32_t at4[4] = {wt.x, wt.y, wt.z, wt.w}, as4[4] = {ws.x, ws.y, ws.z, ws.w};
+                    uint32_t ow[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const f2 s2 = widen(as4[j]);
+                        const f2 dl = sub2(s2, widen(at4[j]));
+                        const f2 xs = fma2(s2, L2E, NLS);
+                        const f2 fac = pk(lo_of(dl) > K ? kp : kn, hi_of(dl) > K ? kp : kn);
+                        const f2 g = mul2(pk(ex2(lo_of(xs)), ex2(hi_of(xs))), fac);
+                        __nv_bfloat162 hv = __floats2bfloat162_rn(lo_of(g), hi_of(g));
+                        ow[j] = *reinterpret_cast<uint32_t*>(&hv);
+                    }
+                    o = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                }
+                *reinterpret_cast<uint4*>(tin + u * 8) = o;
+            }
+            fence_proxy_async_smem();  // the bulk store reads these through the async proxy
+        }
+        team_sync(team);  // the slices are no longer read; the gradient is complete
+        if (rank == 0 && tt == 0) {
+            const double tv = (double)Af - (double)Pf;
+            a.out_tv[r] = (float)tv;
+            if (on) s_tv[team] += tv;
+            s_rows[team] += 1u;
+        }
+        if (tt == 0 && cnt > 0) {
+            if (G != nullptr) {
+                bulk_s2g(G + r * V + lo, tin, bytes);
+                bulk_commit();
+                bulk_wait_read();  // the slice has been read out before it is refilled
+            }
+            if (r + step < N) issue(r + step);
+        }
+    }
+    if (tt == 0) {
+        if (s_abort[team]) {
+            // a copy issued for a row this team will not process: let it land
+            mbar_wait(full, k & 1, 1u << 16);
+            record_device_status(p.status, UNO_ERR_TIMEOUT);
+        }
+        bulk_wait_all();  // every gradient store has completed
+        // this team's share of the masked mean; whoever completes the last row writes it
+        if (rank == 0 && s_rows[team] > 0) {
+            atomicAdd(&p.work->sum_tv, s_tv[team]);
+            __threadfence();
+            const uint32_t prev = atomicAdd(&p.work->done, s_rows[team]);
+            if (prev + s_rows[team] == (uint32_t)N) {
+                __threadfence();
+                const double sum = atomicAdd(&p.work->sum_tv, 0.0);
+                *a.out_mean = n_mask > 0 ? (float)(sum / (double)n_mask) : 0.f;
+            }
+        }
+    }
+    __syncthreads();
+    cluster_sync();  // no CTA leaves while a store into its shared memory may be in flight
+}
+
 }  // namespace cl
 
 }  // namespace tvk
@@ -680,6 +946,53 @@ int choose_cluster(int64_t V, int smem_optin) {
     return 0;
 }
 
+// The two-team kernel: the smallest cluster size whose two slice pairs per CTA fit
+// (UNO_TV_CLUSTER forces one that fits).
+bool launch_teams(const tvk::Params& p, cudaStream_t stream, uno_status& st, DeviceInfo& di) {
+    const TVArgs& a = p.a;
+    const size_t room = (size_t)di.smem_optin - 256;  // the kernel's static shared memory
+    auto fits = [&](int c) { return 2 * tvk::cl::team_bytes(tvk::cl::slice_elems(a.V, c)) <= room; };
+    int c = 0;
+    if (const char* e = getenv("UNO_TV_CLUSTER")) {
+        const int f = atoi(e);
+        if ((f == 1 || f == 2 || f == 4 || f == 8 || f == 16) && fits(f)) c = f;
+    }
+    for (int t = 1; t <= 16 && c == 0; t *= 2)
+        if (fits(t)) c = t;
+    if (c == 0) return false;
+    const int64_t n = tvk::cl::slice_elems(a.V, c);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)c;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(tvk::cl::kTeamKernelThreads);
+    cfg.dynamicSmemBytes = 2 * tvk::cl::team_bytes(n);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    auto key = std::make_pair(-c, cfg.dynamicSmemBytes);
+    auto found = di.max_clusters.find(key);
+    int maxc = 0;
+    if (found != di.max_clusters.end()) {
+        maxc = found->second;
+    } else {
+        cudaLaunchConfig_t q = cfg;
+        q.gridDim = dim3((unsigned)c);
+        if (cudaOccupancyMaxActiveClusters(&maxc, tvk::cl::team_kernel, &q) != cudaSuccess) {
+            cudaGetLastError();
+            maxc = 0;
+        }
+        di.max_clusters[key] = maxc;
+    }
+    if (maxc <= 0) return false;
+    const int64_t clusters = std::min<int64_t>((a.N + 1) / 2, (int64_t)maxc);
+    cfg.gridDim = dim3((unsigned)(clusters * c));
+    st = check_cuda(cudaLaunchKernelEx(&cfg, tvk::cl::team_kernel, p, n), "launch(tv teams)");
+    return true;
+}
+
 // Launch the cluster kernel; returns false (nothing launched) when it cannot run here.
 bool launch_cluster(const tvk::Params& p, cudaStream_t stream, uno_status& st) {
     const TVArgs& a = p.a;
@@ -687,8 +1000,11 @@ bool launch_cluster(const tvk::Params& p, cudaStream_t stream, uno_status& st) {
     const uintptr_t al = reinterpret_cast<uintptr_t>(a.teacher) | reinterpret_cast<uintptr_t>(a.student) |
                          reinterpret_cast<uintptr_t>(a.grad);
     if (al & 15u) return false;
-    if (const char* e = getenv("UNO_TV_KERNEL"))
+    bool teams = false;
+    if (const char* e = getenv("UNO_TV_KERNEL")) {
         if (strcmp(e, "rows") == 0) return false;
+        teams = strcmp(e, "teams") == 0;
+    }
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
     std::lock_guard<std::mutex> lock(g_mu);
@@ -699,12 +1015,17 @@ bool launch_cluster(const tvk::Params& p, cudaStream_t stream, uno_status& st) {
         if (cudaFuncSetAttribute(tvk::cl::cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  di.smem_optin) != cudaSuccess ||
             cudaFuncSetAttribute(tvk::cl::cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(tvk::cl::team_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 di.smem_optin - 256) != cudaSuccess ||
+            cudaFuncSetAttribute(tvk::cl::team_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
                 cudaSuccess) {
             cudaGetLastError();
             return false;
         }
         di.ready = true;
     }
+    if (teams) return launch_teams(p, stream, st, di);
     const int c = choose_cluster(a.V, di.smem_optin);
     if (c == 0) return false;
     const int64_t n = tvk::cl::slice_elems(a.V, c);

@@ -729,9 +729,11 @@ __global__ void __launch_bounds__(kThreads, 1) pair_kernel(Params p, Layout Ly) 
                     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const uint32_t a = w[q] & 0x7FFF7FFFu;
                         mx[r] = __hmax2(mx[r], *reinterpret_cast<const __nv_bfloat162*>(&w[q]));
-                        mg[r] = __hmax2(mg[r], *reinterpret_cast<const __nv_bfloat162*>(&a));
+                        if (!TOPK) {  // the largest magnitude sets the counted band (full mode)
+                            const uint32_t a = w[q] & 0x7FFF7FFFu;
+                            mg[r] = __hmax2(mg[r], *reinterpret_cast<const __nv_bfloat162*>(&a));
+                        }
                     }
                 }
             }

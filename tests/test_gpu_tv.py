@@ -72,6 +72,10 @@ def test_tv_parity(N, V, dtype):
     ({"UNO_TV_CLUSTER": "16"}, 4, 1000),     # ragged last slice
     ({"UNO_TV_CLUSTER": "2"}, 300, 151936),  # does not fit: falls back to the default size
     ({"UNO_TV_KERNEL": "rows"}, 6, 151936),  # the per-row kernel on bf16 rows
+    ({"UNO_TV_KERNEL": "teams"}, 37, 151936),  # the two-team kernel: many rows per team
+    ({"UNO_TV_KERNEL": "teams"}, 5, 1000),
+    ({"UNO_TV_KERNEL": "teams", "UNO_TV_CLUSTER": "16"}, 9, 4000),  # CTAs with empty slices
+    ({"UNO_TV_KERNEL": "teams"}, 3, 166144),
 ])
 def test_tv_kernel_variants(monkeypatch, env, N, V):
     """Every kernel variant and cluster size gives the oracle's result."""
