@@ -724,6 +724,11 @@ Plan make_plan(int64_t M, int64_t d_in, int64_t d_out, int64_t rank, uno_dtype d
     } else {
         P.BN = 256;
         while (P.BN > 64 && (int64_t)P.m_tiles * ((d_out + P.BN - 1) / P.BN) < 120) P.BN >>= 1;
+        // UNO_LORA_BN (64, 128 or 256) fixes the tile width, for measurements
+        if (const char* e = getenv("UNO_LORA_BN")) {
+            const int bn = atoi(e);
+            if (bn == 64 || bn == 128 || bn == 256) P.BN = bn;
+        }
     }
     P.n_tiles = (int)((d_out + P.BN - 1) / P.BN);
     const int rq = 16 * P.CG;  // each CTA of a pair holds rb / 2 rows of A: a multiple of 16
@@ -757,6 +762,11 @@ Plan make_plan(int64_t M, int64_t d_in, int64_t d_out, int64_t rank, uno_dtype d
     P.b_bytes = (uint32_t)(w / P.CG) * 128u;
     P.stages = (int)((kSmemBudget - 1024) / (A_BYTES + P.b_bytes));
     if (P.stages > kMaxStages) P.stages = kMaxStages;
+    // UNO_LORA_STAGES=n (2 up to what fits) shortens the ring, for measurements
+    if (const char* e = getenv("UNO_LORA_STAGES")) {
+        const int st = atoi(e);
+        if (st >= 2 && st < P.stages) P.stages = st;
+    }
     P.smem = (size_t)P.stages * (A_BYTES + P.b_bytes) + 1024;
     size_t off = 0;
     auto take = [&](size_t bytes) {

@@ -1502,6 +1502,456 @@ __global__ void __launch_bounds__(kThreads, 1) pair_kernel(Params p, Layout Ly) 
     if (tt == 0 && ts.abort_) record_device_status(p.status, (uint32_t)UNO_ERR_TIMEOUT);
 }
 
+
+// ---------------------------------------------------------------------------------------
+// topk_local_kernel: top-k (k <= kMaxLocalK) with no cluster-wide cut. Each CTA takes the
+// exact top-k of its own slice of each row (the k largest values, ties to the lower id):
+// the row's top-k is among those CL lists, since a token outside its slice's top-k has k
+// better tokens in that slice alone. A head CTA, rotating over the cluster from item to
+// item, merges the lists, then applies softmax and top-p and takes the draws and the tests.
+// Per item the only cluster traffic is each CTA's sorted list stored into the head's shared
+// memory and one arrive on the head's barrier; the head acknowledges once it has read the
+// lists, and a CTA waits for that only before its next push to the same head, CL items
+// later, by when it is normally long done. Items whose slice top-k lies outside the 256
+// largest values of the slice are left to the generic kernel.
+// ---------------------------------------------------------------------------------------
+constexpr int kMaxLocalK = 128;
+
+struct LLayout {
+    int CL;   // CTAs per cluster
+    int L;    // slice length in elements (a multiple of 8)
+    int KL;   // list capacity: a power of two >= k, >= 32
+    uint32_t off_hist, off_loc, off_cand, off_cnt, off_merged, off_w, off_id, off_tmp, off_misc, team_bytes;
+};
+
+struct LShared {
+    float fred[kTeamWarps][2];
+    float M[2];
+    int kd[2], tkeep[2], theta[2], take_all[2], redo[2], mine[2];
+    uint32_t kbits[2];
+    unsigned loc_n[2];
+    int ipart[kTeamWarps];
+    int np[2];
+    double Z[2];
+    int abort_, any_redo;
+};
+
+__global__ void __launch_bounds__(kThreads, 1) topk_local_kernel(Params p, LLayout Ly) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ __align__(8) uint64_t bars[kTeams][2 + kMaxCL];
+
+    const int team = threadIdx.x / kTeamThreads, tt = threadIdx.x % kTeamThreads;
+    const int tw = tt >> 5, lane = tt & 31;
+    const int CL = Ly.CL, KL = Ly.KL;
+    const uint32_t crank = ctarank();
+    const int cid = blockIdx.x / CL, NC = gridDim.x / CL;
+    const int n_items = p.B * p.K;
+    const double T = p.T;
+
+    unsigned char* base = smem + (size_t)team * Ly.team_bytes;
+    uint16_t* bufs[2] = {reinterpret_cast<uint16_t*>(base), reinterpret_cast<uint16_t*>(base) + Ly.L};
+    uint32_t* hist = reinterpret_cast<uint32_t*>(base + Ly.off_hist);      // [2][kWinK]
+    uint64_t* loc = reinterpret_cast<uint64_t*>(base + Ly.off_loc);        // [2][KL] this slice's top-k
+    uint64_t* cand = reinterpret_cast<uint64_t*>(base + Ly.off_cand);      // [2][CL][KL] lists (as head)
+    int* cnt = reinterpret_cast<int*>(base + Ly.off_cnt);                  // [2][kMaxCL] list lengths, -1: redo
+    uint64_t* merged = reinterpret_cast<uint64_t*>(base + Ly.off_merged);  // [2][KL] the row's top-k
+    double* lw = reinterpret_cast<double*>(base + Ly.off_w);               // [2][KL] survivor weights, id order
+    int32_t* lid = reinterpret_cast<int32_t*>(base + Ly.off_id);           // [2][KL] survivor ids
+    uint64_t* ltmp = reinterpret_cast<uint64_t*>(base + Ly.off_tmp);       // [2][KL] scratch
+    LShared& ls = *reinterpret_cast<LShared*>(base + Ly.off_misc);
+    uint64_t* full = &bars[team][0];
+    uint64_t* ein = &bars[team][1];     // the lists of an item this CTA heads have landed
+    uint64_t* freeb = &bars[team][2];   // [kMaxCL]: head q has read the lists this CTA pushed to it
+
+    if (tt == 0) {
+        mbar_init(full, 1);
+        mbar_init(ein, CL);
+        for (int q = 0; q < CL; ++q) mbar_init(&freeb[q], 1);
+        ls.abort_ = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    cluster_sync_all();
+
+    const int lo = (int)crank * Ly.L;
+    const int n = max(0, min(Ly.L, p.V - lo));
+    const int nvec = n >> 3;
+    const int pv = (nvec + kTeamWarps - 1) / kTeamWarps;
+    const int wv0 = min(nvec, tw * pv), wv1 = min(nvec, wv0 + pv);
+    const int step = kTeams * NC;
+    const int kk = min(p.top_k, n);  // this slice's share of the list
+
+    int issued = -1, inflight = 0;
+    auto needs_rows = [&](int it) { return !trivial_item(p, it / p.K, it % p.K); };
+    auto issue = [&](int it) {
+        const int i = it % p.K;
+        const int nrows = i > 0 ? 2 : 1;
+        if (n > 0) {
+            mbar_arrive_expect_tx(full, (uint32_t)(n * 2 * nrows));
+            bulk_g2s(bufs[0], static_cast<const __nv_bfloat16*>(p.P) + (int64_t)it * p.V + lo, (uint32_t)(n * 2), full);
+            if (i > 0)
+                bulk_g2s(bufs[1], static_cast<const __nv_bfloat16*>(p.Q) + (int64_t)it * p.V + lo, (uint32_t)(n * 2),
+                         full);
+        } else {
+            mbar_arrive(full);
+        }
+        issued = it;
+        inflight = 1;
+    };
+
+    uint32_t lph = 0, hph = 0, jitem = 0;
+    uint32_t pushes = 0;  // bit q, per head q: parity of this CTA's completed pushes there (see below)
+    uint32_t pushed_once = 0;
+    for (int item = cid + team * NC; item < n_items; item += step) {
+        const int b = item / p.K, i = item % p.K;
+        if (!needs_rows(item)) {
+            if (crank == 0 && tt == 0) write_trivial(p, item, b);
+            continue;
+        }
+        const int nrows = i > 0 ? 2 : 1;
+        const int head = (int)(jitem % (uint32_t)CL);
+        ++jitem;
+        if (tt == 0 && issued != item) issue(item);
+        if (tw == 0) {
+            const bool ok = mbar_wait(full, lph & 1);
+            if (!ok && lane == 0) ls.abort_ = 1;
+        }
+        ++lph;
+        if (tt == 0) inflight = 0;
+        team_sync(team);
+        if (ls.abort_) break;
+
+        // ---- (1) this slice's largest value per row ----
+        {
+            __nv_bfloat162 mx[2] = {__floats2bfloat162_rn(-INFINITY, -INFINITY), __floats2bfloat162_rn(-INFINITY, -INFINITY)};
+            for (int r = 0; r < nrows; ++r) {
+                const uint4* v4 = reinterpret_cast<const uint4*>(bufs[r]);
+                for (int j = tt; j < nvec; j += kTeamThreads) {
+                    const uint4 v = v4[j];
+                    mx[r] = __hmax2(mx[r], __hmax2(__hmax2(as_bf2(v.x), as_bf2(v.y)), __hmax2(as_bf2(v.z), as_bf2(v.w))));
+                }
+            }
+            const float m0 = warp_max(fmaxf(__low2float(mx[0]), __high2float(mx[0])));
+            const float m1 = warp_max(fmaxf(__low2float(mx[1]), __high2float(mx[1])));
+            if (lane == 0) {
+                ls.fred[tw][0] = m0;
+                ls.fred[tw][1] = m1;
+            }
+            for (int j = tt; j < 2 * kWinK; j += kTeamThreads) hist[j] = 0u;
+            if (tt < 2) ls.loc_n[tt] = 0u;
+            team_sync(team);
+            if (tt < 2) {
+                float M = -INFINITY;
+                for (int w = 0; w < kTeamWarps; ++w) M = fmaxf(M, ls.fred[w][tt]);
+                ls.M[tt] = M;
+            }
+            team_sync(team);
+        }
+        // ---- (2) counts of the slice's 256 largest values ----
+        for (int r = 0; r < nrows; ++r) {
+            const uint32_t kM = key16(__float_as_uint(ls.M[r]) >> 16);
+            const uint32_t kf = kM >= (uint32_t)(kWinK - 1) ? kM - (uint32_t)(kWinK - 1) : 0u;
+            const uint32_t hf = bits16(kf);
+            const __nv_bfloat162 f2 = as_bf2(hf | (hf << 16));
+            uint32_t* h = hist + r * kWinK;
+            const uint4* v4 = reinterpret_cast<const uint4*>(bufs[r]);
+            for (int j = tt; j < nvec; j += kTeamThreads) {
+                const uint4 v = v4[j];
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t m = __hge2_mask(as_bf2(w[q]), f2);
+                    if (m) {
+                        const uint32_t dl = kM - key16(w[q] & 0xFFFFu), dh = kM - key16(w[q] >> 16);
+                        if ((m & 0xFFFFu) && dl < (uint32_t)kWinK) atomicAdd(&h[dl], 1u);
+                        if ((m >> 16) && dh < (uint32_t)kWinK) atomicAdd(&h[dh], 1u);
+                    }
+                }
+            }
+        }
+        team_sync(team);
+        // ---- (3) warp r: the slice's k-th largest value of row r, and how many of its ties count ----
+        if (tw < nrows) {
+            const int r = tw;
+            const uint32_t kM = key16(__float_as_uint(ls.M[r]) >> 16);
+            int take_all = kk >= n, redo = 0, kd = -1, tkeep = 0, mine = 0;
+            if (!take_all && kk > 0) {
+                int c = 0;
+                for (int d0 = 0; d0 < kWinK && kd < 0; d0 += 32) {
+                    const int cn = (int)hist[r * kWinK + d0 + lane];
+                    const int incl = warp_inclusive_scan(cn, lane);
+                    const unsigned hit = __ballot_sync(kFullMask, cn > 0 && c + incl >= kk);
+                    if (hit) {
+                        const int src = __ffs(hit) - 1;
+                        kd = d0 + src;
+                        mine = __shfl_sync(kFullMask, cn, src);
+                        tkeep = kk - (c + __shfl_sync(kFullMask, incl - cn, src));
+                    }
+                    c += __shfl_sync(kFullMask, incl, 31);
+                }
+                if (kd < 0) redo = 1;  // fewer than k of the slice's tokens among its 256 largest values
+            }
+            const uint32_t kb = kd >= 0 ? bits16(kM - (uint32_t)kd) : 0xFF80u;
+            // +0 and -0 are one value under two keys: leave such a cut to the generic kernel
+            if (kd >= 0 && (kb & 0x7FFFu) == 0u) redo = 1;
+            if (lane == 0) {
+                ls.take_all[r] = take_all || kk == 0;
+                ls.redo[r] = redo;
+                ls.kd[r] = kd;
+                ls.kbits[r] = kb;
+                ls.tkeep[r] = tkeep;
+                ls.mine[r] = mine;
+                ls.theta[r] = INT_MAX;
+            }
+        }
+        team_sync(team);
+        // ---- (4) the last tie that counts, in id order (when only some ties count) ----
+        for (int r = 0; r < nrows; ++r) {
+            if (ls.take_all[r] || ls.redo[r] || ls.tkeep[r] >= ls.mine[r]) continue;
+            const uint16_t* buf = bufs[r];
+            const uint32_t kb = ls.kbits[r];
+            const int keep = ls.tkeep[r];
+            int c = 0;
+            for (int e = wv0 * 8 + lane; e < wv1 * 8; e += 32) c += elem(buf, e) == kb;
+            c = warp_sum(c);
+            if (lane == 0) ls.ipart[tw] = c;
+            team_sync(team);
+            int before = 0, wt = 0;
+            for (; wt < kTeamWarps; ++wt) {
+                if (before + ls.ipart[wt] >= keep) break;
+                before += ls.ipart[wt];
+            }
+            if (tw == wt) {
+                int need = keep - before, found = -1;
+                for (int e0 = wv0 * 8; e0 < wv1 * 8 && found < 0; e0 += 32) {
+                    const int e = e0 + lane;
+                    const unsigned bal = __ballot_sync(kFullMask, e < wv1 * 8 && elem(buf, e) == kb);
+                    const int nb = __popc(bal);
+                    if (nb >= need) {
+                        unsigned bb = bal;
+                        for (int q = 1; q < need; ++q) bb &= bb - 1;
+                        found = e0 + __ffs(bb) - 1;
+                    }
+                    need -= nb;
+                }
+                if (lane == 0) ls.theta[r] = lo + found + 1;
+            }
+            team_sync(team);
+        }
+        // ---- (5) the slice's top-k of each row, gathered locally ----
+        for (int r = 0; r < nrows; ++r) {
+            if (ls.redo[r]) continue;
+            const bool all = ls.take_all[r];
+            const uint32_t kb = ls.kbits[r];
+            const __nv_bfloat162 k2 = as_bf2(kb | (kb << 16));
+            const float kx = bf(kb);
+            const int theta = ls.theta[r];
+            uint64_t* Lr = loc + r * KL;
+            const uint4* v4 = reinterpret_cast<const uint4*>(bufs[r]);
+            for (int j = tt; j < nvec; j += kTeamThreads) {
+                const uint4 v = v4[j];
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t m = all ? 0xFFFFFFFFu : __hge2_mask(as_bf2(w[q]), k2);
+                    if (!m) continue;
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        if (!((m >> (16 * hh)) & 1u)) continue;
+                        const uint32_t h16 = (w[q] >> (16 * hh)) & 0xFFFFu;
+                        const float x = bf(h16);
+                        const int id = lo + j * 8 + 2 * q + hh;
+                        if (!all && x == kx && id >= theta) continue;
+                        const unsigned slot = atomicAdd(&ls.loc_n[r], 1u);
+                        if (slot < (unsigned)KL) Lr[slot] = pack_candidate(float_key(x), (uint32_t)id);
+                    }
+                }
+            }
+        }
+        team_sync(team);
+        // ---- (6) warp r sorts row r's list (value desc, id asc) ----
+        if (tw < nrows) {
+            const int r = tw;
+            uint64_t* Lr = loc + r * KL;
+            const int c = ls.redo[r] ? 0 : (int)min(ls.loc_n[r], (unsigned)KL);
+            for (int j = c + lane; j < KL; j += 32) Lr[j] = 0ull;
+            __syncwarp();
+            warp_sort_desc(Lr, KL, lane);
+        }
+        team_sync(team);
+        // ---- (7) push the lists into the head's shared memory ----
+        if (tw == 0) {
+            const uint32_t hbit = 1u << head;
+            if (pushed_once & hbit) {  // the head has read what this CTA pushed there last time
+                const bool ok = wait_cluster(&freeb[head], (pushes >> head) & 1u);
+                if (!ok && lane == 0) ls.abort_ = 1;
+                pushes ^= hbit;
+            }
+            pushed_once |= hbit;
+            for (int r = 0; r < nrows; ++r) {
+                const uint32_t dst = mapa(&cand[(r * CL + (int)crank) * KL], (uint32_t)head);
+                for (int j = lane; j < KL; j += 32) st_remote_u64(dst + 8u * j, loc[r * KL + j]);
+                if (lane == 0) {
+                    const int c = ls.redo[r] ? -1 : (int)min(ls.loc_n[r], (unsigned)KL);
+                    asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(mapa(&cnt[r * kMaxCL + (int)crank], (uint32_t)head)),
+                                 "r"(c)
+                                 : "memory");
+                }
+            }
+            __syncwarp();
+            if (lane == 0) {
+                fence_cluster();
+                arrive_remote(mapa(ein, (uint32_t)head));
+            }
+        }
+        // ---- (8) the head merges the lists, cuts, draws and tests ----
+        if ((int)crank == head) {
+            if (tw == 0) {
+                const bool ok = wait_cluster(ein, hph & 1);
+                if (!ok && lane == 0) ls.abort_ = 1;
+            }
+            ++hph;
+            team_sync(team);
+            if (ls.abort_) break;
+            if (tt == 0) {
+                int rd = 0;
+                for (int r = 0; r < nrows; ++r)
+                    for (int q = 0; q < CL; ++q) rd |= cnt[r * kMaxCL + q] < 0;
+                ls.any_redo = rd;
+            }
+            team_sync(team);
+            const bool redo = ls.any_redo;
+            if (!redo && tw < nrows) {  // warp r: merge, softmax, top-p, survivors by id
+                const int r = tw;
+                const uint64_t* C = cand + r * CL * KL;
+                const int cq = lane < CL ? cnt[r * kMaxCL + lane] : 0;
+                int total = 0;
+                for (int q = 0; q < CL; ++q) total += cnt[r * kMaxCL + q];
+                const int nk = min(p.top_k, total);
+                int ptr = 0;
+                uint64_t hv = (lane < CL && cq > 0) ? C[lane * KL] : 0ull;
+                uint64_t* Mr = merged + r * KL;
+                for (int s2 = 0; s2 < nk; ++s2) {
+                    uint64_t best = hv;
+                    int bl = lane;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) {
+                        const uint64_t ov = __shfl_xor_sync(kFullMask, best, o);
+                        const int ol = __shfl_xor_sync(kFullMask, bl, o);
+                        if (ov > best || (ov == best && ol < bl)) {
+                            best = ov;
+                            bl = ol;
+                        }
+                    }
+                    if (lane == 0) Mr[s2] = best;
+                    if (lane == bl) {
+                        ++ptr;
+                        hv = ptr < cq ? C[lane * KL + ptr] : 0ull;
+                    }
+                }
+                __syncwarp();
+                uint64_t* Tr = ltmp + r * KL;
+                double* Wr = lw + r * KL;
+                int32_t* Ir = lid + r * KL;
+                // the row's largest value is the first of the merged list
+                const double zm = (double)key_float(candidate_key(Mr[0])) / T;
+                double S1 = 0.0;
+                for (int j = lane; j < nk; j += 32) {
+                    const double w = exp((double)key_float(candidate_key(Mr[j])) / T - zm);
+                    Tr[j] = __double_as_longlong(w);
+                    S1 += w;
+                }
+                S1 = warp_sum_f64(S1);
+                __syncwarp();
+                int np = nk;
+                if (p.cut) {
+                    double carry = 0.0;
+                    for (int j0 = 0; j0 < nk; j0 += 32) {
+                        const int j = j0 + lane;
+                        const double x = j < nk ? __longlong_as_double(Tr[j]) / S1 : 0.0;
+                        const double incl = warp_scan_f64(x, lane);
+                        const unsigned hit = __ballot_sync(kFullMask, j < nk && carry + incl >= p.top_p);
+                        if (hit) {
+                            np = j0 + __ffs(hit);
+                            break;
+                        }
+                        carry += __shfl_sync(kFullMask, incl, 31);
+                    }
+                }
+                // the survivors in id order: sort (id asc) the first np entries
+                for (int j = lane; j < KL; j += 32)
+                    Mr[j] = j < np ? (((uint64_t)(0xFFFFFFFFu - candidate_id(Mr[j])) << 32) | (uint32_t)j) : 0ull;
+                __syncwarp();
+                warp_sort_desc(Mr, KL, lane);
+                double Z = 0.0;
+                for (int j = lane; j < np; j += 32) {
+                    const uint32_t src = (uint32_t)(Mr[j] & 0xFFFFFFFFu);
+                    Ir[j] = (int32_t)(0xFFFFFFFFu - (uint32_t)(Mr[j] >> 32));
+                    Wr[j] = __longlong_as_double(Tr[src]);
+                    Z += Wr[j];
+                }
+                Z = warp_sum_f64(Z);
+                if (lane == 0) {
+                    ls.np[r] = np;
+                    ls.Z[r] = Z;
+                }
+            }
+            team_sync(team);
+            // the lists are read: acknowledge to every CTA
+            if (tw == 1 && lane < CL) arrive_remote(mapa(&freeb[crank], (uint32_t)lane));
+            if (tw == 0) {
+                if (redo) {
+                    if (lane == 0) p.recs[item].state = kRedo;
+                } else {
+                    const float* u = p.u + (int64_t)item * 3;
+                    SRec P;
+                    P.w = lw;
+                    P.id = lid;
+                    P.n = ls.np[0];
+                    P.Z = ls.Z[0];
+                    Rec rec;
+                    rec.state = kDone;
+                    rec.pad = 0.0;
+                    if (i == 0) {
+                        const int x0 = pos0_given(p, b) ? p.pos0[b] : srec_inv_cdf(P, (double)u[0], lane);
+                        rec.tok = x0;
+                        rec.res = -1;
+                        rec.acc = 1;
+                        rec.p = (x0 >= 0 && x0 < p.V) ? srec_prob(P, x0) : 0.0;
+                        rec.q = 0.0;
+                        rec.tv = 0.0;
+                    } else {
+                        SRec Q;
+                        Q.w = lw + KL;
+                        Q.id = lid + KL;
+                        Q.n = ls.np[1];
+                        Q.Z = ls.Z[1];
+                        const int d = p.drafts ? p.drafts[item] : srec_inv_cdf(Q, (double)u[0], lane);
+                        const bool in = d >= 0 && d < p.V;
+                        rec.tok = d;
+                        rec.p = in ? srec_prob(P, d) : 0.0;
+                        rec.q = in ? srec_prob(Q, d) : 0.0;
+                        rec.acc = (double)u[1] * rec.q < rec.p;
+                        rec.tv = srec_tv(P, Q, lane);
+                        rec.res = srec_residual(P, Q, (double)u[2], lane);
+                    }
+                    if (lane == 0) p.recs[item] = rec;
+                }
+            }
+        }
+        team_sync(team);  // the buffer and the local lists are free
+        if (tt == 0) {
+            int nx = item + step;
+            while (nx < n_items && !needs_rows(nx)) nx += step;
+            if (nx < n_items) issue(nx);
+        }
+    }
+    if (tt == 0 && inflight) mbar_wait(full, lph & 1, 1u << 16);
+    __syncthreads();
+    cluster_sync_all();
+    if (tt == 0 && ls.abort_) record_device_status(p.status, (uint32_t)UNO_ERR_TIMEOUT);
+}
+
 }  // namespace pk
 
 // =======================================================================================
@@ -1565,6 +2015,38 @@ pk::Layout make_layout(int V, int CL, int top_k) {
     return Ly;
 }
 
+// the team layout of topk_local_kernel for cluster size CL
+pk::LLayout make_llayout(int V, int CL, int top_k) {
+    pk::LLayout Ly{};
+    Ly.CL = CL;
+    Ly.L = (int)(((int64_t)V + (int64_t)CL * 8 - 1) / ((int64_t)CL * 8) * 8);
+    Ly.KL = 32;
+    while (Ly.KL < top_k) Ly.KL <<= 1;
+    const uint32_t KL = (uint32_t)Ly.KL;
+    uint32_t off = (uint32_t)align_up((size_t)Ly.L * 2 * 2, 16);
+    Ly.off_hist = off;
+    off += 2 * pk::kWinK * 4;
+    Ly.off_loc = off;
+    off += 2 * KL * 8;
+    Ly.off_cand = off;
+    off += 2 * (uint32_t)CL * KL * 8;
+    Ly.off_cnt = off;
+    off += 2 * pk::kMaxCL * 4;
+    Ly.off_merged = off;
+    off += 2 * KL * 8;
+    Ly.off_w = off;
+    off += 2 * KL * 8;
+    Ly.off_id = off;
+    off += 2 * KL * 4;
+    off = (uint32_t)align_up(off, 16);
+    Ly.off_tmp = off;
+    off += 2 * KL * 8;
+    Ly.off_misc = off;
+    off += (uint32_t)align_up(sizeof(pk::LShared), 16);
+    Ly.team_bytes = (uint32_t)align_up(off, 128);
+    return Ly;
+}
+
 struct DeviceInfo {
     bool ready = false;
     size_t dyn_max = 0;
@@ -1572,6 +2054,10 @@ struct DeviceInfo {
 };
 std::mutex g_mu;
 DeviceInfo g_dev[64];
+
+struct DeviceInfo;
+bool launch_local(const VerifyArgs& a, const Params& p, cudaStream_t stream, uno_status& st, DeviceInfo& di,
+                  int forced, bool required);
 
 template <bool TOPK>
 bool set_attributes(int dyn_max) {
@@ -1609,10 +2095,19 @@ bool launch_pairs(const VerifyArgs& a, const Params& p, cudaStream_t stream, uno
             cudaGetLastError();
             return no("shared memory attributes unavailable");
         }
-        const int stat = (int)std::max(fa.sharedSizeBytes, fb.sharedSizeBytes);
+        cudaFuncAttributes fc{};
+        if (cudaFuncGetAttributes(&fc, pk::topk_local_kernel) != cudaSuccess) {
+            cudaGetLastError();
+            return no("shared memory attributes unavailable");
+        }
+        const int stat = (int)std::max(std::max(fa.sharedSizeBytes, fb.sharedSizeBytes), fc.sharedSizeBytes);
         if (optin <= stat) return no("shared memory attributes unavailable");
         const int dyn_max = optin - stat;
-        if (!set_attributes<false>(dyn_max) || !set_attributes<true>(dyn_max)) {
+        if (!set_attributes<false>(dyn_max) || !set_attributes<true>(dyn_max) ||
+            cudaFuncSetAttribute(pk::topk_local_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_max) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(pk::topk_local_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+                cudaSuccess) {
             cudaGetLastError();
             return no("kernel attributes refused");
         }
@@ -1621,6 +2116,11 @@ bool launch_pairs(const VerifyArgs& a, const Params& p, cudaStream_t stream, uno
     }
     int forced = 0;
     if (const char* e = getenv("UNO_VERIFY_FULL_CLUSTER")) forced = atoi(e);
+    // top-k up to kMaxLocalK: per-CTA top-k lists merged by a head CTA (UNO_VERIFY_TOPK=window
+    // selects the cluster-wide cut of pair_kernel instead)
+    const char* tmode = getenv("UNO_VERIFY_TOPK");
+    if (a.top_k > 0 && a.top_k <= pk::kMaxLocalK && !(tmode && strcmp(tmode, "window") == 0))
+        return launch_local(a, p, stream, st, di, forced, required);
     int CL = 0;
     pk::Layout Ly{};
     for (int c = 1; c <= pk::kMaxCL; c *= 2) {
@@ -1669,6 +2169,58 @@ bool launch_pairs(const VerifyArgs& a, const Params& p, cudaStream_t stream, uno
     const cudaError_t e = topk ? cudaLaunchKernelEx(&cfg, pk::pair_kernel<true>, p, Ly)
                                : cudaLaunchKernelEx(&cfg, pk::pair_kernel<false>, p, Ly);
     st = check_cuda(e, "launch(verify, pairs)");
+    return true;
+}
+
+// topk_local_kernel: the smallest cluster size whose two team layouts fit
+bool launch_local(const VerifyArgs& a, const Params& p, cudaStream_t stream, uno_status& st, DeviceInfo& di,
+                  int forced, bool required) {
+    auto no = [&](const char* why) {
+        if (required) st = set_error(UNO_ERR_UNSUPPORTED, "verify: no cluster form: %s", why);
+        return required;
+    };
+    int CL = 0;
+    pk::LLayout Ly{};
+    for (int c = 1; c <= pk::kMaxCL; c *= 2) {
+        if (forced && c != forced) continue;
+        const pk::LLayout t = make_llayout(a.V, c, a.top_k);
+        if ((size_t)t.team_bytes * pk::kTeams <= di.dyn_max) {
+            CL = c;
+            Ly = t;
+            break;
+        }
+    }
+    if (CL == 0) return no("the row slices do not fit in the shared memory of any cluster size");
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)CL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(pk::kThreads);
+    cfg.dynamicSmemBytes = (size_t)Ly.team_bytes * pk::kTeams;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const auto key = std::make_tuple(2, CL, cfg.dynamicSmemBytes);
+    int maxc = 0;
+    const auto found = di.max_clusters.find(key);
+    if (found != di.max_clusters.end()) {
+        maxc = found->second;
+    } else {
+        cudaLaunchConfig_t q = cfg;
+        q.gridDim = dim3((unsigned)CL);
+        if (cudaOccupancyMaxActiveClusters(&maxc, pk::topk_local_kernel, &q) != cudaSuccess) {
+            cudaGetLastError();
+            maxc = 0;
+        }
+        di.max_clusters[key] = maxc;
+    }
+    if (maxc <= 0) return no("no cluster of this size can be resident");
+    const int64_t items = (int64_t)a.B * a.K;
+    const int64_t clusters = std::min<int64_t>((items + pk::kTeams - 1) / pk::kTeams, (int64_t)maxc);
+    cfg.gridDim = dim3((unsigned)(clusters * CL));
+    st = check_cuda(cudaLaunchKernelEx(&cfg, pk::topk_local_kernel, p, Ly), "launch(verify, local top-k)");
     return true;
 }
 

@@ -205,16 +205,21 @@ TOPK_CLUSTER_CASES = [
 ]
 
 
+@pytest.mark.parametrize("mode", ["local", "window"])
 @pytest.mark.parametrize("cl", [1, 2, 4, 8, 16])
 @pytest.mark.parametrize("case", TOPK_CLUSTER_CASES, ids=[f"B{c[0]}K{c[1]}V{c[2]}k{c[4]}p{c[5]}" for c in TOPK_CLUSTER_CASES])
-def test_topk_cluster_kernel(case, cl, monkeypatch):
-    """The cluster kernel's top-k mode (the k-th value from per-value counts over the 256
-    largest values, the survivors collected in one CTA of the cluster) against the oracle,
-    for every cluster size that fits; UNO_VERIFY_FULL=cluster makes any other path an error."""
+def test_topk_cluster_kernel(case, cl, mode, monkeypatch):
+    """The cluster kernels' top-k modes against the oracle, for every cluster size that fits:
+    "local" (k <= 128: every CTA takes its slice's exact top-k, a head CTA merges the lists)
+    and "window" (the row's k-th value from per-value counts over its 256 largest values,
+    selected by UNO_VERIFY_TOPK=window; it also serves 128 < k <= 256). UNO_VERIFY_FULL=cluster
+    makes any other path an error."""
     B, K, V, T, k, p = case
     from diffusion_drafted_lossless_b200._lib import UnoError
     monkeypatch.setenv("UNO_VERIFY_FULL", "cluster")
     monkeypatch.setenv("UNO_VERIFY_FULL_CLUSTER", str(cl))
+    if mode == "window":
+        monkeypatch.setenv("UNO_VERIFY_TOPK", "window")
     P, Q, u = _inputs(B, K, V, "bf16", seed=zlib.crc32(str((case, cl)).encode()) % 10007)
     try:
         _check(P, Q, u, T, k, p, "bf16")
