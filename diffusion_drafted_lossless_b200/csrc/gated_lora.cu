@@ -80,6 +80,8 @@ struct Params {
     unsigned long long* header;   // [4]: epoch of the next execution, its complement, CTA-exit ticket
     unsigned long long host_tag;  // lower bound for this execution's epoch (fresh per host call), < 2^48
     uint32_t flag_polls;          // polls of a T flag before the wait gives up
+    int epi_tma;                  // bf16 output tiles leave through shared memory and TMA stores
+    uint32_t epi_off;             // byte offset of the epilogue staging buffers in dynamic smem
     int withhold_flags;           // test switch: adapter items do not publish T (every wait on it runs out)
     uint32_t* status;
 };
@@ -94,6 +96,21 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
         : "memory");
 }
+
+// TMA store of a 2-D box from shared memory (bulk group of this thread)
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int x, int y, const void* src) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(smem_u32(src))
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// at most N of this thread's bulk groups still read their shared-memory source
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -303,7 +320,7 @@ template <int BN, int CG>
 __global__ void __launch_bounds__(kThreads, 1)
 lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__ CUtensorMap tW0,
                  const __grid_constant__ CUtensorMap tA, const __grid_constant__ CUtensorMap tT,
-                 const __grid_constant__ CUtensorMap tB, Params p) {
+                 const __grid_constant__ CUtensorMap tB, const __grid_constant__ CUtensorMap tY, Params p) {
     extern __shared__ unsigned char smem_dyn[];
     __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages], tfull[2], tempty[2], drain;
     __shared__ uint32_t tmem_holder;
@@ -357,6 +374,7 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
         prefetch_tmap(&tA);
         prefetch_tmap(&tT);
         prefetch_tmap(&tB);
+        if (p.epi_tma) prefetch_tmap(&tY);
     }
     tmem_fence_before();
     __syncthreads();
@@ -465,6 +483,9 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
         const int q = warp & 3;
         const int et = threadIdx.x - 64;  // 0..127 across the epilogue warps
         const uint32_t lead_tempty0 = CG == 2 ? map_to_rank(&tempty[0], 0) : 0u;
+        // TMA-store epilogue: two 32 x 32 bf16 staging boxes per warp (64-byte swizzle)
+        unsigned char* stage_box = smem + p.epi_off + (size_t)q * 4096;
+        uint32_t chunk = 0;  // boxes this warp has stored
         uint32_t li = 0;
         for (int item = unit0; item < p.n_items; item += units, ++li) {
             const Item w = decode(p, item);
@@ -508,7 +529,8 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
                     __syncwarp();
                     tmem_ld32(taddr + (uint32_t)c0, r);
                     const int col0 = w.j * BN + c0;
-                    if (row >= p.M || col0 >= p.N) continue;
+                    // (the TMA-store path keeps every lane: the store leaves rows past M out)
+                    if (col0 >= p.N || (row >= p.M && !p.epi_tma)) continue;
                     const int ncol = min(32, p.N - col0);  // a multiple of 32: N is a multiple of 64
                     if (p.ksplit > 1) {  // this split's fp32 partial
                         float* dst = p.ypart + ((size_t)w.s * p.M + row) * p.N + col0;
@@ -522,6 +544,32 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
                             *reinterpret_cast<float4*>(dst + j) =
                                 make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
                                             __uint_as_float(r[j + 3]));
+                    } else if (p.epi_tma) {
+                        // row `lane` of this warp's 32-row box: four 16-byte chunks, chunk c at
+                        // c ^ ((lane >> 1) & 3) (the 64-byte swizzle the tensor map names)
+                        unsigned char* box = stage_box + (chunk & 1) * 2048;
+                        if (chunk >= 2) {  // the store issued from this box two chunks ago has read it
+                            if (lane == 0) bulk_wait_read<1>();
+                            __syncwarp();
+                        }
+#pragma unroll
+                        for (int j = 0; j < 32; j += 8) {
+                            __nv_bfloat162 h0 = __floats2bfloat162_rn(__uint_as_float(r[j]), __uint_as_float(r[j + 1]));
+                            __nv_bfloat162 h1 = __floats2bfloat162_rn(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+                            __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[j + 4]), __uint_as_float(r[j + 5]));
+                            __nv_bfloat162 h3 = __floats2bfloat162_rn(__uint_as_float(r[j + 6]), __uint_as_float(r[j + 7]));
+                            const int c = (j >> 3) ^ ((lane >> 1) & 3);
+                            *reinterpret_cast<uint4*>(box + lane * 64 + c * 16) =
+                                make_uint4(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),
+                                           *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&tY, col0, m0 + q * 32, box);
+                            bulk_commit_group();
+                        }
+                        ++chunk;
                     } else {
                         __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.y) + (size_t)row * p.N + col0;
 #pragma unroll
@@ -642,6 +690,7 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
                 }
             }
         }
+        if (p.epi_tma && lane == 0) bulk_wait_all();  // this warp's output stores have completed
     }
 
     tmem_fence_before();
@@ -696,12 +745,29 @@ uno_status make_tmap(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols
     return UNO_OK;
 }
 
+// row-major [rows, cols] bf16 output, 32 x 32 boxes with 64-byte swizzle (the epilogue's
+// staging layout)
+uno_status make_tmap_store(CUtensorMap* m, void* ptr, int64_t rows, int64_t cols) {
+    auto fn = encode_fn();
+    if (!fn) return set_error(UNO_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t gstride[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {32u, 32u};
+    cuuint32_t estride[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, gdim, gstride, box, estride,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return set_error(UNO_ERR_CUDA, "cuTensorMapEncodeTiled (output) failed (%d)", (int)r);
+    return UNO_OK;
+}
+
 
 // The launch plan of one call (also sizes the workspace).
 struct Plan {
     int CG, BN, rb, cb, m_tiles, m_units, n_tiles, kt0, kt1, splits, per, n_adapter, n_items, stages;
     int ksplit, kper;
-    uint32_t b_bytes;
+    int epi_tma;
+    uint32_t b_bytes, epi_off;
     size_t smem;
     // workspace offsets
     size_t header, flags, tickets, t, tpart, ypart, otickets, x, w0, a, b, total;
@@ -760,14 +826,21 @@ Plan make_plan(int64_t M, int64_t d_in, int64_t d_out, int64_t rank, uno_dtype d
     P.ksplit = (P.kt0 + P.kper - 1) / P.kper;  // every split has K tiles of (X, W0); the last also (T, B)
     P.n_items = P.n_adapter + P.m_units * P.n_tiles * P.ksplit;
     P.b_bytes = (uint32_t)(w / P.CG) * 128u;
-    P.stages = (int)((kSmemBudget - 1024) / (A_BYTES + P.b_bytes));
+    // UNO_LORA_EPI=tma: bf16 output tiles leave through 16 KB of shared-memory staging boxes
+    // and TMA stores instead of per-lane row stores
+    P.epi_tma = 0;
+    if (const char* e = getenv("UNO_LORA_EPI"))
+        if (strcmp(e, "tma") == 0 && dtype == UNO_BF16 && P.ksplit == 1 && P.CG == 1) P.epi_tma = 1;
+    const uint32_t epi_bytes = P.epi_tma ? 4u * 4096u : 0u;
+    P.stages = (int)((kSmemBudget - 1024 - epi_bytes) / (A_BYTES + P.b_bytes));
     if (P.stages > kMaxStages) P.stages = kMaxStages;
     // UNO_LORA_STAGES=n (2 up to what fits) shortens the ring, for measurements
     if (const char* e = getenv("UNO_LORA_STAGES")) {
         const int st = atoi(e);
         if (st >= 2 && st < P.stages) P.stages = st;
     }
-    P.smem = (size_t)P.stages * (A_BYTES + P.b_bytes) + 1024;
+    P.epi_off = (uint32_t)align_up((size_t)P.stages * (A_BYTES + P.b_bytes), 1024);
+    P.smem = (size_t)P.epi_off + epi_bytes + 1024;
     size_t off = 0;
     auto take = [&](size_t bytes) {
         size_t o = off;
@@ -815,7 +888,7 @@ int num_sms_cached() {
 }
 
 template <int BN, int CG>
-uno_status launch_t(const CUtensorMap (&maps)[5], Params& p, const Plan& P, cudaStream_t stream) {
+uno_status launch_t(const CUtensorMap (&maps)[6], Params& p, const Plan& P, cudaStream_t stream) {
     static bool attr = false;
     if (!attr) {
         uno_status s = check_cuda(cudaFuncSetAttribute(lora_gemm_kernel<BN, CG>,
@@ -856,11 +929,11 @@ uno_status launch_t(const CUtensorMap (&maps)[5], Params& p, const Plan& P, cuda
     attrs[n_attr].id = cudaLaunchAttributeCooperative;
     attrs[n_attr].val.cooperative = 1;
     cfg.numAttrs = n_attr + 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, lora_gemm_kernel<BN, CG>, maps[0], maps[1], maps[2], maps[3], maps[4], p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, lora_gemm_kernel<BN, CG>, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], p);
     if (e != cudaSuccess) {
         cudaGetLastError();
         cfg.numAttrs = n_attr;
-        e = cudaLaunchKernelEx(&cfg, lora_gemm_kernel<BN, CG>, maps[0], maps[1], maps[2], maps[3], maps[4], p);
+        e = cudaLaunchKernelEx(&cfg, lora_gemm_kernel<BN, CG>, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], p);
     }
     return check_cuda(e, "launch(gated lora)");
 }
@@ -892,13 +965,18 @@ uno_status gated_lora_launch(const GatedLoraArgs& g, void* workspace, cudaStream
     }
     const int M = (int)g.M, din = (int)g.d_in, dout = (int)g.d_out, r = (int)g.rank;
     __nv_bfloat16* t = reinterpret_cast<__nv_bfloat16*>(ws + P.t);
-    CUtensorMap maps[5];
+    CUtensorMap maps[6];
     const int cg = P.CG;
     if ((s = make_tmap(&maps[0], x, M, din, BM)) != UNO_OK) return s;              // X
     if ((s = make_tmap(&maps[1], w0, dout, din, P.BN / cg)) != UNO_OK) return s;   // W0
     if ((s = make_tmap(&maps[2], a, r, din, P.rb / cg)) != UNO_OK) return s;       // A
     if ((s = make_tmap(&maps[3], t, M, r, BM)) != UNO_OK) return s;                // T
     if ((s = make_tmap(&maps[4], b, dout, r, P.BN / cg)) != UNO_OK) return s;      // B
+    if (P.epi_tma) {
+        if ((s = make_tmap_store(&maps[5], g.y, M, dout)) != UNO_OK) return s;     // Y (stores)
+    } else {
+        maps[5] = maps[0];  // not read
+    }
     Params p{};
     p.M = M;
     p.N = dout;
@@ -933,6 +1011,8 @@ uno_status gated_lora_launch(const GatedLoraArgs& g, void* workspace, cudaStream
     // UNO_LORA_TEST_WITHHOLD_FLAGS=1 (tests of the failure path only): the adapter items keep
     // T to themselves and the output tiles' waits for it give up after a few thousand polls;
     // the call must then end with UNO_ERR_TIMEOUT in the device status word
+    p.epi_tma = P.epi_tma;
+    p.epi_off = P.epi_off;
     p.withhold_flags = 0;
     p.flag_polls = kFlagPolls;
     if (const char* e = getenv("UNO_LORA_TEST_WITHHOLD_FLAGS"))

@@ -214,3 +214,18 @@ def test_withheld_adapter_flags_time_out(monkeypatch):
     monkeypatch.delenv("UNO_LORA_TEST_WITHHOLD_FLAGS")
     assert _rel(_run(inp, M, d_in, d_out, r), _ref(inp)) <= TOL
     assert _lib.uno_read_device_status() == _lib.UNO_OK
+
+
+def test_tma_store_epilogue(monkeypatch):
+    """UNO_LORA_EPI=tma: bf16 output tiles staged in shared memory (64-byte swizzle) and
+    written by TMA stores. Ragged M (the stores leave rows past M out), every tile width,
+    several tiles per CTA, and two calls in a row."""
+    monkeypatch.setenv("UNO_LORA_EPI", "tma")
+    for M, d_in, d_out, r in [(300, 1024, 512, 64), (1000, 768, 1024, 256), (129, 256, 640, 128),
+                              (1024, 4096, 4096, 128), (2048, 2560, 640, 64), (5, 128, 64, 24)]:
+        w = W.GatedLoraWorkload("t", 23 + M + r, M=M, block=8, rank=r, scale=2.0,
+                                shapes=(W.LinearShape("t", d_in, d_out),))
+        inp = W.linear_inputs(w, w.shapes[0])
+        ref = _ref(inp)
+        for _ in range(2):
+            assert _rel(_run(inp, M, d_in, d_out, r), ref) <= TOL, (M, d_in, d_out, r)
