@@ -779,6 +779,7 @@ __global__ void __launch_bounds__(kThreads, 1) pair_kernel(Params p, Layout Ly) 
                         A = max(A, (uint32_t)((v >> 16) & 0xFFFFu));
                     }
                     RowStat& rs = ts.rs[lane];
+                    if (M == 0.f) M = 0.f;  // +0, at or above every zero in key order
                     rs.M = M;
                     rs.atop = A;
                     rs.kM = key16(__float_as_uint(M) >> 16);
@@ -1643,6 +1644,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_local_kernel(Params p, LLayo
             if (tt < 2) {
                 float M = -INFINITY;
                 for (int w = 0; w < kTeamWarps; ++w) M = fmaxf(M, ls.fred[w][tt]);
+                if (M == 0.f) M = 0.f;  // +0, at or above every zero in key order
                 ls.M[tt] = M;
             }
             team_sync(team);
@@ -1789,8 +1791,12 @@ __global__ void __launch_bounds__(kThreads, 1) topk_local_kernel(Params p, LLayo
             }
             pushed_once |= hbit;
             for (int r = 0; r < nrows; ++r) {
+                // odd ranks store their list reversed (ascending), so that the head's lists
+                // alternate in direction, as a bitonic merge network takes them
                 const uint32_t dst = mapa(&cand[(r * CL + (int)crank) * KL], (uint32_t)head);
-                for (int j = lane; j < KL; j += 32) st_remote_u64(dst + 8u * j, loc[r * KL + j]);
+                const bool rev = (crank & 1u) != 0u;
+                for (int j = lane; j < KL; j += 32)
+                    st_remote_u64(dst + 8u * (uint32_t)(rev ? KL - 1 - j : j), loc[r * KL + j]);
                 if (lane == 0) {
                     const int c = ls.redo[r] ? -1 : (int)min(ls.loc_n[r], (unsigned)KL);
                     asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(mapa(&cnt[r * kMaxCL + (int)crank], (uint32_t)head)),
@@ -1821,34 +1827,36 @@ __global__ void __launch_bounds__(kThreads, 1) topk_local_kernel(Params p, LLayo
             }
             team_sync(team);
             const bool redo = ls.any_redo;
-            if (!redo && tw < nrows) {  // warp r: merge, softmax, top-p, survivors by id
+            if (!redo) {
+                // the CL sorted lists of each row (alternately descending and ascending) form
+                // bitonic runs: the merge phases of a bitonic sort (run lengths 2 KL ... CL KL)
+                // leave each row's CL KL entries in descending order
+                const int nall = CL * KL;
+                for (int size = 2 * KL; size <= nall; size <<= 1) {
+                    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+                        for (int t = tt; t < nrows * (nall >> 1); t += kTeamThreads) {
+                            const int r = t / (nall >> 1), tr = t % (nall >> 1);
+                            uint64_t* A = cand + r * nall;
+                            const int lo2 = 2 * tr - (tr & (stride - 1));
+                            const int hi2 = lo2 + stride;
+                            const bool desc = (lo2 & size) == 0;
+                            const uint64_t x = A[lo2], y = A[hi2];
+                            if ((x < y) == desc) {
+                                A[lo2] = y;
+                                A[hi2] = x;
+                            }
+                        }
+                        team_sync(team);
+                    }
+                }
+            }
+            if (!redo && tw < nrows) {  // warp r: softmax, top-p, survivors by id
                 const int r = tw;
-                const uint64_t* C = cand + r * CL * KL;
-                const int cq = lane < CL ? cnt[r * kMaxCL + lane] : 0;
                 int total = 0;
                 for (int q = 0; q < CL; ++q) total += cnt[r * kMaxCL + q];
                 const int nk = min(p.top_k, total);
-                int ptr = 0;
-                uint64_t hv = (lane < CL && cq > 0) ? C[lane * KL] : 0ull;
                 uint64_t* Mr = merged + r * KL;
-                for (int s2 = 0; s2 < nk; ++s2) {
-                    uint64_t best = hv;
-                    int bl = lane;
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) {
-                        const uint64_t ov = __shfl_xor_sync(kFullMask, best, o);
-                        const int ol = __shfl_xor_sync(kFullMask, bl, o);
-                        if (ov > best || (ov == best && ol < bl)) {
-                            best = ov;
-                            bl = ol;
-                        }
-                    }
-                    if (lane == 0) Mr[s2] = best;
-                    if (lane == bl) {
-                        ++ptr;
-                        hv = ptr < cq ? C[lane * KL + ptr] : 0ull;
-                    }
-                }
+                for (int j = lane; j < KL; j += 32) Mr[j] = j < nk ? cand[r * CL * KL + j] : 0ull;
                 __syncwarp();
                 uint64_t* Tr = ltmp + r * KL;
                 double* Wr = lw + r * KL;
