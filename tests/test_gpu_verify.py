@@ -407,3 +407,19 @@ def test_pos0_entries_below_zero_draw_from_p0(top_k):
         gpu, ref, _ = _check_full(P, Q, u, 1.0, 0.95, "bf16", pos0=pos0)
     assert (gpu["tokens"][1::2, 0] == pos0[1::2]).all()
     assert (gpu["tokens"][::2, 0] >= 0).all()
+
+
+@pytest.mark.parametrize("k", [1, 50, 128])
+def test_topk_outlier_slices_go_to_the_generic_kernel(k):
+    """A few huge logits put the largest values of their slice far above the rest, so that
+    slice holds fewer than k tokens among its 256 largest values: the cluster kernel hands
+    those items to the generic kernel, and every result must still be the oracle's."""
+    B, K, V = 3, 4, 40000
+    rng = np.random.default_rng(46 + k)
+    base = rng.standard_normal((B, K, V)).astype(np.float32)
+    base[:, :, 5] = 4000.0
+    base[:, ::2, 20011] = -3000.0
+    P = W.bf16_bits(base)
+    Q = W.bf16_bits((0.8 * base + 0.6 * rng.standard_normal((B, K, V))).astype(np.float32))
+    u = rng.random((B, K, 3), dtype=np.float32)
+    _check(P, Q, u, 1.0, k, 0.9, "bf16")
