@@ -77,7 +77,7 @@ struct Params {
     float scale;
     unsigned long long* flags;    // [m_tiles]: the epoch once row tile m's T is written
     unsigned long long* tickets;  // [m_tiles]: (epoch << 16) | partials stored
-    unsigned long long* header;   // [4]: epoch of the next execution, its complement, CTA-exit ticket
+    unsigned long long* header;   // [5]: the next execution's epoch and exit counter (see Header)
     unsigned long long host_tag;  // lower bound for this execution's epoch (fresh per host call), < 2^48
     uint32_t flag_polls;          // polls of a T flag before the wait gives up
     int epi_tma;                  // bf16 output tiles leave through shared memory and TMA stores
@@ -209,28 +209,52 @@ __device__ __forceinline__ bool take_ticket(unsigned long long* t, unsigned long
 
 constexpr unsigned long long kEpochMask = 0xFFFFFFFFFFFFull;
 
-// This execution's epoch. Each CTA reads the workspace header when it starts, and only the
-// last CTA of the grid to finish advances it (retire_epoch), so all CTAs see the same
-// value. It is the larger of the header's stored value (when its check word matches) and
-// the host's tag, so it is above every epoch this workspace has seen: a CUDA-graph replay, whose host tag is frozen at
-// capture, still gets a fresh epoch, and no flag or ticket left by an earlier execution
-// (or by unrelated data in a fresh workspace, which fails the check) can match it.
-__device__ __forceinline__ unsigned long long read_epoch(const unsigned long long* hdr, unsigned long long host_tag) {
-    const unsigned long long e = __ldcg(hdr), chk = __ldcg(hdr + 1);
-    unsigned long long stored = (chk == ~e) ? (e & kEpochMask) : 0ull;
-    unsigned long long ep = stored > host_tag ? stored : host_tag;
+// The workspace header: [0] the next execution's epoch, [1] its complement (the header is
+// valid only when they match), [2] which exit counter the next execution uses (0 or 1),
+// [3..4] the two exit counters. The counter a valid header names is zero when the execution
+// starts: the previous execution's last CTA cleared it.
+struct Header {
+    unsigned long long epoch, check, slot, count[2];
+};
+
+// This execution's epoch and exit counter. Each CTA reads the header when it starts, and
+// only the last CTA of the grid to finish rewrites it (retire_epoch), so all CTAs see the
+// same values. The epoch is the larger of the header's stored one and the host's tag, so
+// it is above every epoch this workspace has seen: a CUDA-graph replay, whose host tag is
+// frozen at capture, still gets a fresh epoch, and no flag or ticket left by an earlier
+// execution (or unrelated data in a fresh workspace, which fails the check) can match it.
+// slot = -1: the header was not valid; the CTAs then count their exits with a tagged
+// compare-and-swap ticket instead (contended, but only on a workspace's first use).
+__device__ __forceinline__ unsigned long long read_epoch(const unsigned long long* hdr, unsigned long long host_tag,
+                                                         int* slot) {
+    const Header* h = reinterpret_cast<const Header*>(hdr);
+    const unsigned long long e = __ldcg(&h->epoch), chk = __ldcg(&h->check), sl = __ldcg(&h->slot);
+    const bool valid = chk == ~e && sl <= 1ull;
+    *slot = valid ? (int)sl : -1;
+    const unsigned long long stored = valid ? (e & kEpochMask) : 0ull;
+    const unsigned long long ep = stored > host_tag ? stored : host_tag;
     return ep == 0 ? 1ull : ep;
 }
 
-// Called once per CTA after all of its work: the last CTA to finish stores epoch + 1 (and
-// its complement) for the next execution on this workspace.
-__device__ __forceinline__ void retire_epoch(unsigned long long* hdr, unsigned long long epoch, int ctas) {
+// Called once per CTA after all of its work: the last CTA to finish stores epoch + 1 and the
+// other exit counter, cleared, for the next execution on this workspace.
+__device__ __forceinline__ void retire_epoch(unsigned long long* hdr, unsigned long long epoch, int slot, int ctas) {
+    Header* h = reinterpret_cast<Header*>(hdr);
     __threadfence();
-    if (take_ticket(hdr + 2, epoch, ctas)) {
+    bool last;
+    if (slot >= 0) {
+        last = atomicAdd(&h->count[slot], 1ull) + 1ull == (unsigned long long)ctas;
+    } else {
+        last = take_ticket(&h->count[0], epoch, ctas);
+    }
+    if (last) {
+        const int next = slot == 0 ? 1 : 0;
         unsigned long long nx = (epoch + 1) & kEpochMask;
         if (nx == 0) nx = 1;
-        hdr[0] = nx;
-        hdr[1] = ~nx;
+        h->count[next] = 0ull;
+        h->slot = (unsigned long long)next;
+        h->epoch = nx;
+        h->check = ~nx;
         __threadfence();
     }
 }
@@ -326,6 +350,7 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
     __shared__ uint32_t tmem_holder;
     __shared__ int s_abort, s_last;
     __shared__ unsigned long long s_epoch;
+    __shared__ int s_slot;
 
     // 128-byte swizzled tiles need 1024-byte aligned shared-memory addresses
     unsigned char* smem = smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u);
@@ -350,7 +375,7 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
         }
         mbar_init(&drain, 1);
         s_abort = 0;
-        s_epoch = read_epoch(p.header, p.host_tag);
+        s_epoch = read_epoch(p.header, p.host_tag, &s_slot);
         fence_mbar_init();
     }
     if (warp == 1) {  // two accumulators of cb fp32 columns x 128 lanes (in each CTA of a pair)
@@ -705,7 +730,7 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
     }
     if (threadIdx.x == 0) {
         if (s_abort) record_device_status(p.status, (uint32_t)UNO_ERR_TIMEOUT);
-        retire_epoch(p.header, epoch, (int)gridDim.x);
+        retire_epoch(p.header, epoch, s_slot, (int)gridDim.x);
     }
 }
 
@@ -847,7 +872,7 @@ Plan make_plan(int64_t M, int64_t d_in, int64_t d_out, int64_t rank, uno_dtype d
         off = align_up(off + bytes, 256);
         return o;
     };
-    P.header = take(32);
+    P.header = take(sizeof(unsigned long long) * 5);
     P.flags = take((size_t)P.m_tiles * 8);
     P.tickets = take((size_t)P.m_tiles * 8);
     P.t = take((size_t)M * rank * 2);

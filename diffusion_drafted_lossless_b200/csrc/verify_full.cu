@@ -85,7 +85,18 @@ struct Params {
     const float* u;
     Rec* recs;
     uint32_t* status;
+    unsigned long long* trace;  // UNO_VERIFY_TRACE: phase timestamps of cluster 0 (profiling aid), or NULL
 };
+
+// trace slot of (cluster rank, team, item number j < 32, event e < 16) in cluster 0
+__device__ __forceinline__ void trace_mark(const Params& p, int cid, uint32_t crank, int team, uint32_t j, int e) {
+    if (p.trace != nullptr && cid == 0 && j < 32u) {
+        unsigned long long t;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        p.trace[((crank * 2u + (uint32_t)team) * 32u + j) * 16u + (uint32_t)e] = t;
+    }
+}
+constexpr size_t kTraceBytes = 16 * 2 * 32 * 16 * 8;
 
 __device__ __forceinline__ bool pos0_given(const Params& p, int b) { return p.pos0 && p.pos0[b] >= 0; }
 // an item with nothing to compute: x_0 supplied and P_0(x_0) not wanted
@@ -705,6 +716,7 @@ __global__ void __launch_bounds__(kThreads, 1) pair_kernel(Params p, Layout Ly) 
             continue;
         }
         const int nrows = i > 0 ? 2 : 1;
+        if (tt == 0) trace_mark(p, cid, crank, team, xph, 0);
         if (tt == 0 && issued != item) issue(item);
         if (tw == 0) {
             const bool ok = mbar_wait(full, lph & 1);
@@ -714,6 +726,7 @@ __global__ void __launch_bounds__(kThreads, 1) pair_kernel(Params p, Layout Ly) 
         if (tt == 0) inflight = 0;
         team_sync(team);
         if (ts.abort_) break;
+        if (tt == 0) trace_mark(p, cid, crank, team, xph, 1);
 
         // ---- (1) largest value and magnitude of each row slice ----
         {
@@ -790,6 +803,7 @@ __global__ void __launch_bounds__(kThreads, 1) pair_kernel(Params p, Layout Ly) 
             if (ts.abort_) break;
         }
 
+        if (tt == 0) trace_mark(p, cid, crank, team, xph, 2);
         // ---- (2) counts per value: full mode, every magnitude within kWords steps of the
         //      largest (the rest weighed one by one); top-k mode, the kWinK largest values ----
         if constexpr (TOPK) {
@@ -865,6 +879,7 @@ __global__ void __launch_bounds__(kThreads, 1) pair_kernel(Params p, Layout Ly) 
             if (ts.abort_) break;
         }
 
+        if (tt == 0) trace_mark(p, cid, crank, team, xph, 3);
         // ---- (3) this CTA's share of the values: cluster-wide counts, and (full mode) their
         //      masses ----
         {
@@ -927,6 +942,7 @@ __global__ void __launch_bounds__(kThreads, 1) pair_kernel(Params p, Layout Ly) 
             if (ts.abort_) break;
         }
 
+        if (tt == 0) trace_mark(p, cid, crank, team, xph, 4);
         // ---- (4) the cut of each row, identical in every CTA ----
         if (TOPK && tw < nrows) {  // warp r finds the k-th largest value of row r
             const int r = tw;
@@ -1088,6 +1104,7 @@ __global__ void __launch_bounds__(kThreads, 1) pair_kernel(Params p, Layout Ly) 
                 if (tt == 0) rs.lut_n = (int)min((uint32_t)ln, rs.atop + 1u);
             }
 
+            if (tt == 0) trace_mark(p, cid, crank, team, xph, 5);
             // ---- (5) where the kept ties end: counts of the tie value in lower-ranked CTAs ----
             if (cutting && !redo && tw < nrows) {
                 const int r = tw;
@@ -1297,6 +1314,7 @@ __global__ void __launch_bounds__(kThreads, 1) pair_kernel(Params p, Layout Ly) 
                     }
                 }
             } else {
+            if (tt == 0) trace_mark(p, cid, crank, team, xph, 6);
             // ---- (6) masses per warp part: draw row, verifier survivors, residual ----
             const int draw_row = i > 0 ? 1 : 0;
             const RowStat rp = ts.rs[0];
@@ -1371,6 +1389,7 @@ __global__ void __launch_bounds__(kThreads, 1) pair_kernel(Params p, Layout Ly) 
             team_sync(team);
             if (ts.abort_) break;
 
+            if (tt == 0) trace_mark(p, cid, crank, team, xph, 7);
             // ---- (7) the draws: the CTA and warp part holding each target, then its token ----
             if (!redo) {
                 const float* u = p.u + (int64_t)item * 3;
@@ -1488,6 +1507,7 @@ __global__ void __launch_bounds__(kThreads, 1) pair_kernel(Params p, Layout Ly) 
             }
             }  // full mode
         }
+        if (tt == 0) trace_mark(p, cid, crank, team, xph, 8);
         ++xph;
         team_sync(team);  // the buffer is free
         if (tt == 0) {
@@ -1611,7 +1631,8 @@ __global__ void __launch_bounds__(kThreads, 1) topk_local_kernel(Params p, LLayo
         }
         const int nrows = i > 0 ? 2 : 1;
         const int head = (int)(jitem % (uint32_t)CL);
-        ++jitem;
+        const uint32_t jm = jitem++;
+        if (tt == 0) trace_mark(p, cid, crank, team, jm, 0);
         if (tt == 0 && issued != item) issue(item);
         if (tw == 0) {
             const bool ok = mbar_wait(full, lph & 1);
@@ -1622,6 +1643,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_local_kernel(Params p, LLayo
         team_sync(team);
         if (ls.abort_) break;
 
+        if (tt == 0) trace_mark(p, cid, crank, team, jm, 1);
         // ---- (1) this slice's largest value per row ----
         {
             __nv_bfloat162 mx[2] = {__floats2bfloat162_rn(-INFINITY, -INFINITY), __floats2bfloat162_rn(-INFINITY, -INFINITY)};
@@ -1649,6 +1671,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_local_kernel(Params p, LLayo
             }
             team_sync(team);
         }
+        if (tt == 0) trace_mark(p, cid, crank, team, jm, 2);
         // ---- (2) counts of the slice's 256 largest values ----
         for (int r = 0; r < nrows; ++r) {
             const uint32_t kM = key16(__float_as_uint(ls.M[r]) >> 16);
@@ -1672,6 +1695,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_local_kernel(Params p, LLayo
             }
         }
         team_sync(team);
+        if (tt == 0) trace_mark(p, cid, crank, team, jm, 3);
         // ---- (3) warp r: the slice's k-th largest value of row r, and how many of its ties count ----
         if (tw < nrows) {
             const int r = tw;
@@ -1707,6 +1731,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_local_kernel(Params p, LLayo
             }
         }
         team_sync(team);
+        if (tt == 0) trace_mark(p, cid, crank, team, jm, 4);
         // ---- (4) the last tie that counts, in id order (when only some ties count) ----
         for (int r = 0; r < nrows; ++r) {
             if (ls.take_all[r] || ls.redo[r] || ls.tkeep[r] >= ls.mine[r]) continue;
@@ -1740,6 +1765,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_local_kernel(Params p, LLayo
             }
             team_sync(team);
         }
+        if (tt == 0) trace_mark(p, cid, crank, team, jm, 5);
         // ---- (5) the slice's top-k of each row, gathered locally ----
         for (int r = 0; r < nrows; ++r) {
             if (ls.redo[r]) continue;
@@ -1771,6 +1797,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_local_kernel(Params p, LLayo
             }
         }
         team_sync(team);
+        if (tt == 0) trace_mark(p, cid, crank, team, jm, 6);
         // ---- (6) warp r sorts row r's list (value desc, id asc) ----
         if (tw < nrows) {
             const int r = tw;
@@ -1781,6 +1808,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_local_kernel(Params p, LLayo
             warp_sort_desc(Lr, KL, lane);
         }
         team_sync(team);
+        if (tt == 0) trace_mark(p, cid, crank, team, jm, 7);
         // ---- (7) push the lists into the head's shared memory ----
         if (tw == 0) {
             const uint32_t hbit = 1u << head;
@@ -1809,6 +1837,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_local_kernel(Params p, LLayo
                 fence_cluster();
                 arrive_remote(mapa(ein, (uint32_t)head));
             }
+            if (lane == 0) trace_mark(p, cid, crank, team, jm, 8);
         }
         // ---- (8) the head merges the lists, cuts, draws and tests ----
         if ((int)crank == head) {
@@ -1818,6 +1847,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_local_kernel(Params p, LLayo
             }
             ++hph;
             team_sync(team);
+            if (tt == 0) trace_mark(p, cid, crank, team, jm, 9);
             if (ls.abort_) break;
             if (tt == 0) {
                 int rd = 0;
@@ -1905,6 +1935,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_local_kernel(Params p, LLayo
                 }
             }
             team_sync(team);
+            if (tt == 0) trace_mark(p, cid, crank, team, jm, 10);
             // the lists are read: acknowledge to every CTA
             if (tw == 1 && lane < CL) arrive_remote(mapa(&freeb[crank], (uint32_t)lane));
             if (tw == 0) {
@@ -1948,6 +1979,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_local_kernel(Params p, LLayo
             }
         }
         team_sync(team);  // the buffer and the local lists are free
+        if (tt == 0) trace_mark(p, cid, crank, team, jm, 11);
         if (tt == 0) {
             int nx = item + step;
             while (nx < n_items && !needs_rows(nx)) nx += step;
@@ -1987,7 +2019,11 @@ __global__ void assemble_kernel(Params p, int32_t* out_tokens, int32_t* out_coun
 // =======================================================================================
 // host side
 // =======================================================================================
-inline size_t recs_bytes(const VerifyArgs& a) { return align_up((size_t)a.B * a.K * sizeof(Rec), 256); }
+inline bool tracing() { return getenv("UNO_VERIFY_TRACE") != nullptr; }
+// the records, then (UNO_VERIFY_TRACE set) the phase-timestamp trace
+inline size_t recs_bytes(const VerifyArgs& a) {
+    return align_up((size_t)a.B * a.K * sizeof(Rec), 256) + (tracing() ? kTraceBytes : 0);
+}
 
 // the team layout for cluster size CL; top_k > 0 selects the top-k mode
 pk::Layout make_layout(int V, int CL, int top_k) {
@@ -2268,6 +2304,10 @@ uno_status verify_full_launch(const VerifyArgs& a, void* workspace, cudaStream_t
     p.u = a.u;
     p.recs = static_cast<vfull::Rec*>(workspace);
     p.status = device_status_ptr();
+    p.trace = vfull::tracing() ? reinterpret_cast<unsigned long long*>(
+                                     static_cast<unsigned char*>(workspace) +
+                                     align_up((size_t)a.B * a.K * sizeof(vfull::Rec), 256))
+                               : nullptr;
     uno_status st = UNO_OK;
     int only_redo = 0;
     if (vfull::launch_pairs(a, p, stream, st)) {

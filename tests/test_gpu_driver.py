@@ -37,9 +37,11 @@ def _run(steps, graph):
 
 
 def _oracle_y(d, s, i, gate):
+    """The oracle's projection i at step s: that step's activations, the layer's weights."""
     sh = L.shapes[i]
-    inp = W.linear_inputs(d.pool_linear_workload(s), sh)
-    return oracle.gated_lora(W.to_f64(inp["x"], "bf16"), W.to_f64(inp["w0"], "bf16"), W.to_f64(inp["a"], "bf16"),
+    x = W.linear_inputs(d.pool_linear_workload(s), sh)["x"]
+    inp = W.linear_inputs(L, sh)
+    return oracle.gated_lora(W.to_f64(x, "bf16"), W.to_f64(inp["w0"], "bf16"), W.to_f64(inp["a"], "bf16"),
                              W.to_f64(inp["b"], "bf16"), gate, float(np.float32(L.scale)))
 
 

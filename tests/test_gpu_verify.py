@@ -278,8 +278,10 @@ def test_full_vocab_ties_and_supplied_tokens():
     u = rng.random((B, K, 3), dtype=np.float32)
     for top_p in (1.0, 0.9, 0.3):
         _check_full(P, Q, u, 1.0, top_p, "bf16")
+    # every token tied: the cut keeps the lowest ids (top_p * V is kept away from an integer,
+    # where the cut itself would sit on its threshold)
     const = np.zeros((B, K, V), np.float32)
-    _check_full(W.bf16_bits(const), W.bf16_bits(const), u, 1.0, 0.5, "bf16")
+    _check_full(W.bf16_bits(const), W.bf16_bits(const), u, 1.0, 0.3001, "bf16")
     drafts = rng.integers(0, V, (B, K)).astype(np.int32)
     pos0 = rng.integers(0, V, B).astype(np.int32)
     gpu, _, _ = _check_full(P, Q, u, 1.0, 0.9, "bf16", drafts=drafts, pos0=pos0)
