@@ -1,8 +1,9 @@
-// verify.cu — dispatch of the block verify. The item path (verify_full.cu: one thread-block
-// cluster per block position, rows resident in shared memory) takes every top-k-off batch and
-// the top-k batches it supports (bf16 rows whose length is a multiple of 8, 16-byte aligned,
-// k <= 256); the streaming path (verify_topk.cu) takes the other top-k batches.
-// UNO_VERIFY_TOPK=stream sends every top-k batch to the streaming path.
+// verify.cu — dispatch of the block verify. Top-k batches go to the streaming path
+// (verify_topk.cu: every row read once by independent CTAs, per-warp exact top-k lists
+// merged per row); top-k-off batches to the item path (verify_full.cu: one thread-block
+// cluster per block position, rows resident in shared memory). UNO_VERIFY_TOPK=local or
+// =window sends the top-k batches the item path supports (bf16 rows whose length is a
+// multiple of 8, 16-byte aligned, k <= 256) to its cluster kernels instead.
 #include <algorithm>
 #include <cstdlib>
 #include <cstring>
@@ -11,9 +12,9 @@
 
 namespace uno {
 
-static bool topk_stream_forced() {
+static bool topk_cluster_selected() {
     const char* e = getenv("UNO_VERIFY_TOPK");
-    return e && strcmp(e, "stream") == 0;
+    return e && (strcmp(e, "local") == 0 || strcmp(e, "window") == 0);
 }
 
 size_t verify_workspace_bytes(const VerifyArgs& a) {
@@ -27,7 +28,7 @@ uno_status verify_launch(const VerifyArgs& a, void* workspace, size_t workspace_
     if (a.B == 0) return UNO_OK;
     bool taken = false;
     if (a.top_k == 0) return verify_full_launch(a, workspace, stream, true, &taken);
-    if (!topk_stream_forced()) {
+    if (topk_cluster_selected()) {
         const uno_status s = verify_full_launch(a, workspace, stream, false, &taken);
         if (s != UNO_OK || taken) return s;
     }

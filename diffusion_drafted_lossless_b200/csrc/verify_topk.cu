@@ -6,18 +6,23 @@
 // sampler settings from the uno-qwen3-8B model card, "Evaluation protocol" (temperature
 // 1.0, top-k 50, top-p 0.95, block 16).
 //
-// Three launches, none of which waits on another CTA:
+// Two launches, neither of which waits on another CTA:
 //   1. stream: the logit rows (verifier rows 0..K-1 and drafter rows 1..K-1 of every
 //      sequence) are read once with 16-byte coalesced loads; every warp keeps the exact
-//      top-k of its own run of the row in shared memory and writes it out;
-//   2. finish: one warp per row merges the row's lists, applies softmax and top-p in fp64
-//      and stores the survivors sorted by token id;
-//   3. sequence: one CTA per sequence runs draft sampling, acceptance, the longest
-//      accepted prefix and the residual resample, one warp per block position.
+//      top-k of its own run of the row (among the elements at or above a sampled guess)
+//      and writes it out. bf16 rows that are 16-byte aligned take the persistent row
+//      kernel; the rest one CTA per row segment (or the TMA-fed variant);
+//   2. finish: one CTA per sequence; a warp per row merges the row's lists into its exact
+//      top-k (redoing the row when the guess could have hidden part of it), applies softmax
+//      and top-p in fp64 and stores the survivors sorted by token id; the CTA then runs
+//      draft sampling, acceptance, the longest accepted prefix and the residual resample,
+//      one warp per block position.
 #include <cuda_bf16.h>
 
 #include <cstdlib>
 #include <cstring>
+#include <type_traits>
+#include <algorithm>
 
 #include "select.cuh"
 #include "verify_common.cuh"
@@ -32,15 +37,6 @@ constexpr int kGuessPerWarp = 8; // sample maxima each warp contributes to the g
 template <int KCAP>
 constexpr int cap_entries() { return KCAP + 576; }
 
-// warps per CTA of the row-finishing kernel and its shared memory per warp
-template <int KCAP>
-struct FinishCfg;
-template <>
-struct FinishCfg<64> { static constexpr int WARPS = 4; };
-template <>
-struct FinishCfg<256> { static constexpr int WARPS = 2; };
-template <>
-struct FinishCfg<1024> { static constexpr int WARPS = 1; };
 
 struct Params {
     VerifyArgs a;
@@ -760,56 +756,12 @@ constexpr size_t finish_bytes_per_warp(int lists_per_row) {
     return (size_t)lists_per_row * KCAP * 8 + 2 * KCAP * 8 + 256 * 4 + 32;
 }
 
-template <typename T, int KCAP>
-__global__ void __launch_bounds__(FinishCfg<KCAP>::WARPS * 32)
-finish_kernel(Params p, int n_rows) {
-    constexpr int FW = FinishCfg<KCAP>::WARPS;
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t grow = (int64_t)blockIdx.x * FW + warp;
-    if (grow >= n_rows) return;
-    const VerifyArgs& a = p.a;
-    const int k = a.top_k, L = p.lists_per_row;
-    unsigned char* base = smem_raw + warp * finish_bytes_per_warp<KCAP>(L);
-    uint64_t* cand = reinterpret_cast<uint64_t*>(base);      // [L * KCAP], ascending id
-    uint64_t* sb = cand + (size_t)L * KCAP;                  // [np] (value desc, id asc)
-    double* w = reinterpret_cast<double*>(sb + KCAP);        // [KCAP]
-    uint32_t* hist = reinterpret_cast<uint32_t*>(sb + 2 * KCAP);
-    WarpSlot* ws = reinterpret_cast<WarpSlot*>(hist + 256);
-    uint32_t* bound = reinterpret_cast<uint32_t*>(ws + 1);
-
-    // gather the row's lists in (segment, warp) order: ascending token id overall
-    int n = 0;
-    uint32_t G = 0u;  // the largest guess any list was taken with
-    for (int l = 0; l < L; ++l) {
-        const int64_t list = grow * L + l;
-        const int cnt = __ldcg(p.counts + list);
-        G = max(G, __ldcg(p.guesses + list));
-        const uint64_t* src = p.lists + list * KCAP;
-        for (int j = lane; j < cnt; j += 32) cand[n + j] = __ldcg(src + j);
-        n += cnt;
-    }
-    __syncwarp();
-    if (n > k) {
-        const uint64_t T2 = warp_select(cand, n, k, hist, lane);
-        uint64_t mn;
-        n = warp_compact(cand, n, T2, lane, &mn);
-    }
-    // exact iff the k-th value is >= every guess: then every element that can be in the
-    // top-k was >= its warp's guess and so was a candidate
-    uint32_t kmin = 0xFFFFFFFFu;
-    for (int j = lane; j < n; j += 32) kmin = min(kmin, candidate_key(cand[j]));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) kmin = min(kmin, __shfl_xor_sync(kFullMask, kmin, o));
-    if (n < k || kmin < G) {
-        // the streaming guess left fewer than k candidates: redo this row exactly
-        const int b = (int)(grow / p.rows_per_seq), r = (int)(grow % p.rows_per_seq);
-        const bool isP = r < a.K;
-        const int pos = isP ? r : r - a.K + 1;
-        const T* row = reinterpret_cast<const T*>(isP ? a.P : a.Q) + ((int64_t)b * a.K + pos) * a.V;
-        n = warp_exact_row<T, fallback_cap<KCAP>()>(row, a.V, cand, hist, ws, bound, k, lane);
-    }
-    // cand[0..n): the row's top-k (any order). Sort by (value desc, id asc) for top-p.
+// The row's top-k cand[0..n) (any order) -> its survivor record: sorted by (value desc, id
+// asc) into sb, fp64 softmax weights w relative to the largest value, the top-p cut (the
+// shortest prefix of that order whose mass reaches top_p), and the survivors sorted by id
+// (reusing cand) with their weights and total. One warp.
+__device__ __forceinline__ void write_survivors(const VerifyArgs& a, uint64_t* cand, int n, uint64_t* sb, double* w,
+                                                RecView rec, int lane) {
     const double Td = (double)a.temperature;
     int np = 1;
     while (np < n) np <<= 1;
@@ -846,7 +798,6 @@ finish_kernel(Params p, int n_rows) {
         ib[j] = j < c ? ((uint64_t)(0xFFFFFFFFu - candidate_id(sb[j])) << 32) | (uint64_t)j : 0ull;
     __syncwarp();
     warp_sort_desc(ib, np2, lane);
-    RecView rec = rec_view(p.recs, p.kcap, grow);
     double z = 0.0;
     for (int j = lane; j < c; j += 32) {
         const uint64_t e = ib[j];
@@ -862,16 +813,296 @@ finish_kernel(Params p, int n_rows) {
     }
 }
 
-// ---------------------------------------------------------------------------------------
-// Kernel 3: one CTA per sequence: draft sampling, acceptance, longest accepted prefix,
-// residual resample.
-// ---------------------------------------------------------------------------------------
-constexpr int kSeqWarps = 8;
+// Finish row `grow` (one warp): gather its lists, select the exact top-k (redoing the row
+// exactly when the streaming guess could have hidden part of it) and write the survivor
+// record. `base` is the warp's finish_bytes_per_warp(L) bytes of shared memory.
+template <typename T, int KCAP>
+__device__ void finish_row(const Params& p, int64_t grow, unsigned char* base, int lane) {
+    const VerifyArgs& a = p.a;
+    const int k = a.top_k, L = p.lists_per_row;
+    uint64_t* cand = reinterpret_cast<uint64_t*>(base);      // [L * KCAP], ascending id
+    uint64_t* sb = cand + (size_t)L * KCAP;                  // [np] (value desc, id asc)
+    double* w = reinterpret_cast<double*>(sb + KCAP);        // [KCAP]
+    uint32_t* hist = reinterpret_cast<uint32_t*>(sb + 2 * KCAP);
+    WarpSlot* ws = reinterpret_cast<WarpSlot*>(hist + 256);
+    uint32_t* bound = reinterpret_cast<uint32_t*>(ws + 1);
 
-__global__ void __launch_bounds__(kSeqWarps * 32)
-sequence_kernel(Params p, size_t region_bytes) {
+    // gather the row's lists in (segment, warp) order: ascending token id overall. Every
+    // list's count and guess is loaded at once (lane l: lists l, l + 32, ...), then every
+    // entry, so the gather costs two dependent rounds of loads whatever the list count.
+    int n = 0;
+    uint32_t G = 0u;  // the largest guess any list was taken with
+    for (int l0 = 0; l0 < L; l0 += 32) {
+        const int l = l0 + lane;
+        const int64_t list = grow * L + l;
+        const int cnt = l < L ? __ldcg(p.counts + list) : 0;
+        if (l < L) G = max(G, __ldcg(p.guesses + list));
+        const int incl = warp_inclusive_scan(cnt, lane);
+        const int tot = __shfl_sync(kFullMask, incl, 31);
+        const int excl = incl - cnt;
+        for (int e0 = 0; e0 < tot; e0 += 32) {
+            const int e = e0 + lane;
+            // the list holding entry e: the number of lists whose inclusive count is <= e
+            int li = 0;
+#pragma unroll
+            for (int b = 16; b > 0; b >>= 1)
+                if (__shfl_sync(kFullMask, incl, li + b - 1) <= e) li += b;
+            const int first = __shfl_sync(kFullMask, excl, li & 31);
+            if (e < tot) cand[n + e] = __ldcg(p.lists + (grow * L + l0 + li) * KCAP + (e - first));
+        }
+        n += tot;
+    }
+    for (int o = 16; o > 0; o >>= 1) G = max(G, __shfl_xor_sync(kFullMask, G, o));
+    __syncwarp();
+    if (n > k) {
+        const uint64_t T2 = warp_select(cand, n, k, hist, lane);
+        uint64_t mn;
+        n = warp_compact(cand, n, T2, lane, &mn);
+    }
+    // exact iff the k-th value is >= every guess: then every element that can be in the
+    // top-k was >= its warp's guess and so was a candidate
+    uint32_t kmin = 0xFFFFFFFFu;
+    for (int j = lane; j < n; j += 32) kmin = min(kmin, candidate_key(cand[j]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) kmin = min(kmin, __shfl_xor_sync(kFullMask, kmin, o));
+    if (n < k || kmin < G) {
+        // the streaming guess left fewer than k candidates: redo this row exactly
+        const int b = (int)(grow / p.rows_per_seq), r = (int)(grow % p.rows_per_seq);
+        const bool isP = r < a.K;
+        const int pos = isP ? r : r - a.K + 1;
+        const T* row = reinterpret_cast<const T*>(isP ? a.P : a.Q) + ((int64_t)b * a.K + pos) * a.V;
+        n = warp_exact_row<T, fallback_cap<KCAP>()>(row, a.V, cand, hist, ws, bound, k, lane);
+    }
+    // cand[0..n): the row's top-k (any order)
+    write_survivors(a, cand, n, sb, w, rec_view(p.recs, p.kcap, grow), lane);
+}
+
+// ---------------------------------------------------------------------------------------
+// Kernel 2: one CTA per sequence. Warp w (of the first fw) finishes rows w, w + fw, ... of
+// the sequence: merges their lists into the exact top-k, applies softmax and top-p in fp64
+// and writes each survivor record sorted by token id; then the CTA runs the sequence's
+// draft sampling, acceptance, longest accepted prefix and residual resample.
+// ---------------------------------------------------------------------------------------
+constexpr int kFinWarps = 32;
+
+template <typename T, int KCAP>
+__global__ void __launch_bounds__(kFinWarps * 32)
+finish_seq_kernel(Params p, int fw, size_t smem_bytes) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    sequence_verify<kSeqWarps>(p.a, p.recs, p.kcap, blockIdx.x, p.rows_per_seq, smem_raw, region_bytes);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int b = blockIdx.x;
+    if (warp < fw) {
+        unsigned char* base = smem_raw + (size_t)warp * finish_bytes_per_warp<KCAP>(p.lists_per_row);
+        for (int r = warp; r < p.rows_per_seq; r += fw) finish_row<T, KCAP>(p, (int64_t)b * p.rows_per_seq + r, base, lane);
+    }
+    __syncthreads();  // every record of the sequence is written (and visible to the block)
+    sequence_verify<kFinWarps>(p.a, p.recs, KCAP, b, p.rows_per_seq, smem_raw, smem_bytes);
+}
+
+// ---------------------------------------------------------------------------------------
+// Kernel 1 (bf16 rows, 16-byte aligned, V a multiple of 8, k <= 256): persistent over rows.
+// kRowsCtasPerSm CTAs of kRowsWarps warps per SM take the rows in turn, so no SM idles
+// through a last partial wave. Each warp streams its 1/kRowsWarps run of the row with
+// 16-byte register loads one group of kGroup chunks ahead (a chunk is 32 lanes x 8
+// elements, a group gives each lane 64 elements to test); a group costs a few packed
+// bf16x2 maxima and one vote. A lane whose chunk holds an element at or above the
+// threshold only records the chunk (one 16-byte shared store); once 32 chunks are recorded
+// the warp unpacks them together into its candidate buffer (cut to its exact top-k, packed
+// value/id order, when more might not fit; after a cut, later elements of the run are kept
+// only when strictly above the k-th value). The threshold starts at a guess g: every warp
+// offers the four largest lane maxima of its first group, and g is the m-th largest of
+// those 32 offers, m = 3 lambda + 4 with lambda the expected number of the row's top-k
+// among the sampled elements. g exceeds the row's k-th value only with negligible
+// probability on exchangeable data; the finish kernel checks every row (its k-th value
+// must be >= g, so that every element that can be in the top-k was a candidate) and redoes
+// the rare failures exactly. The next row's first group is loaded before this row's lists
+// are written, so the warp's loads stay in flight across rows. No CTA waits for another.
+// ---------------------------------------------------------------------------------------
+constexpr int kRowsWarps = 8;
+constexpr int kRowsCtasPerSm = 2;
+constexpr int kGroup = 8;                        // chunks per group
+constexpr int kHitSlots = 32 + 32 * kGroup;      // recorded chunks: < 32 carried + one group
+constexpr uint32_t kNegInfPair = 0xFF80FF80u;    // two bf16 -inf
+
+template <int KCAP>
+constexpr int rows_cap() { return KCAP + 320; }  // a flush of 32 chunks (<= 256 elements) fits after a cut
+
+// shared memory: recorded chunks [warp][kHitSlots] (16 bytes + id each), candidate buffers
+// [warp][rows_cap], histograms [warp][256]
+template <int KCAP>
+constexpr size_t rows_smem_bytes() {
+    return (size_t)kRowsWarps * ((size_t)kHitSlots * (16 + 4) + (size_t)rows_cap<KCAP>() * 8 + 256 * 4);
+}
+
+__device__ __forceinline__ __nv_bfloat162 bf2_of(uint32_t w) { return *reinterpret_cast<const __nv_bfloat162*>(&w); }
+__device__ __forceinline__ __nv_bfloat162 bf2_max4(const uint4& v) {
+    return __hmax2(__hmax2(bf2_of(v.x), bf2_of(v.y)), __hmax2(bf2_of(v.z), bf2_of(v.w)));
+}
+
+template <int KCAP>
+__global__ void __launch_bounds__(kRowsWarps * 32, kRowsCtasPerSm)
+stream_rows_kernel(Params p, int n_items) {
+    constexpr int CAP = rows_cap<KCAP>();
+    constexpr int CH = 256;  // elements per chunk
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    uint4* hvs = reinterpret_cast<uint4*>(smem_raw);
+    uint64_t* wbuf = reinterpret_cast<uint64_t*>(hvs + kRowsWarps * kHitSlots);
+    uint32_t* hids = reinterpret_cast<uint32_t*>(wbuf + kRowsWarps * CAP);
+    uint32_t* whist = hids + kRowsWarps * kHitSlots;
+    __shared__ WarpSlot s_slot[kRowsWarps];
+    __shared__ uint32_t s_top[kRowsWarps * 4];
+    __shared__ int s_nsample[kRowsWarps];
+    __shared__ float s_guess;
+
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const VerifyArgs& a = p.a;
+    const int k = a.top_k, V = a.V;
+    const int V8 = V >> 3;
+    const int nchunks = (V + CH - 1) / CH;
+    uint4* hv = hvs + warp * kHitSlots;
+    uint32_t* hid = hids + warp * kHitSlots;
+    uint64_t* buf = wbuf + warp * CAP;
+    uint32_t* hist = whist + warp * 256;
+    WarpSlot* ws = &s_slot[warp];
+
+    // the warp's chunk run [c0, c1) of a row
+    auto run_of = [&](int& c0, int& c1) {
+        c0 = nchunks * warp / kRowsWarps;
+        c1 = nchunks * (warp + 1) / kRowsWarps;
+    };
+    auto row_of = [&](int grow) -> const __nv_bfloat16* {
+        const int b = grow / p.rows_per_seq, r = grow % p.rows_per_seq;
+        const bool isP = r < a.K;
+        const int pos = isP ? r : r - a.K + 1;
+        return reinterpret_cast<const __nv_bfloat16*>(isP ? a.P : a.Q) + ((int64_t)b * a.K + pos) * V;
+    };
+    // chunk c of the run: this lane's 8 elements, or two -inf pairs past the run or the row
+    auto load = [&](const uint4* r4, int c, int c1) -> uint4 {
+        const int idx = c * 32 + lane;
+        return (c < c1 && idx < V8) ? ld_stream_v4(r4 + idx) : make_uint4(kNegInfPair, kNegInfPair, kNegInfPair, kNegInfPair);
+    };
+
+    int item = blockIdx.x;
+    int c0 = 0, c1 = 0;
+    uint4 cur[kGroup];
+    const uint4* r4 = nullptr;
+    if (item < n_items) {
+        run_of(c0, c1);
+        r4 = reinterpret_cast<const uint4*>(row_of(item));
+#pragma unroll
+        for (int u = 0; u < kGroup; ++u) cur[u] = load(r4, c0 + u, c1);
+    }
+    for (; item < n_items; item += gridDim.x) {
+        const int grow = item;
+        if (lane == 0) {
+            ws->count = 0;
+            ws->have_k = 0;
+            ws->thr = -INFINITY;
+        }
+        // ---- the guess, from every warp's first group ----
+        {
+            float lm = -INFINITY;
+            int nv = 0;
+#pragma unroll
+            for (int u = 0; u < kGroup; ++u) {
+                const int c = c0 + u;
+                if (c < c1 && c * 32 + lane < V8) {
+                    const __nv_bfloat162 m2 = bf2_max4(cur[u]);
+                    lm = fmaxf(lm, fmaxf(__low2float(m2), __high2float(m2)));
+                    nv += 8;
+                }
+            }
+            uint32_t key = nv > 0 ? float_key(lm) : 0u;
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                uint32_t mx = key;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(kFullMask, mx, o));
+                if (lane == 0) s_top[warp * 4 + t] = mx;
+                const unsigned owner = __ballot_sync(kFullMask, key == mx);
+                if (lane == __ffs(owner) - 1) key = 0u;
+            }
+            nv = warp_sum(nv);
+            if (lane == 0) s_nsample[warp] = nv;
+            __syncthreads();
+            if (warp == 0) {
+                int ns = 0;
+                for (int w = 0; w < kRowsWarps; ++w) ns += s_nsample[w];
+                const uint32_t sorted = warp_sort32_desc(s_top[lane], lane);
+                const int m = (int)(3.0 * k * (double)ns / (double)V) + 4;
+                uint32_t g = 0u;
+                const uint32_t gm = __shfl_sync(kFullMask, sorted, (m - 1) & 31);
+                if (m <= 32 && ns < V) g = gm;
+                if (lane == 0) s_guess = key_float(g < 0x007FFFFFu ? 0x007FFFFFu : g);
+            }
+            __syncthreads();
+        }
+        const float guess = s_guess;
+        __nv_bfloat162 lo2 = __float2bfloat162_rn(guess);  // the guess is a bf16 value (or -inf)
+        int nh = 0;
+        // ---- stream the run ----
+        int c = c0;
+        while (true) {
+            if (nh >= 32) {  // unpack the recorded chunks (the next group's loads are not out yet)
+                __syncwarp();
+                warp_flush_hits<__nv_bfloat16, CAP>(hv, hid, nh, 8, guess, buf, hist, ws, k, lane);
+                nh = 0;
+                const float th = ws->have_k ? ws->thr : -INFINITY;
+                lo2 = __float2bfloat162_rn(fmaxf(guess, th));
+            }
+            const bool more = c + kGroup < c1;
+            uint4 nxt[kGroup];
+            if (more) {
+#pragma unroll
+                for (int u = 0; u < kGroup; ++u) nxt[u] = load(r4, c + kGroup + u, c1);
+            }
+            __nv_bfloat162 mu[kGroup];
+#pragma unroll
+            for (int u = 0; u < kGroup; ++u) mu[u] = bf2_max4(cur[u]);
+            __nv_bfloat162 gm2 = mu[0];
+#pragma unroll
+            for (int u = 1; u < kGroup; ++u) gm2 = __hmax2(gm2, mu[u]);
+            if (__any_sync(kFullMask, __hge2_mask(gm2, lo2) != 0u)) {
+#pragma unroll
+                for (int u = 0; u < kGroup; ++u) {
+                    const int cc = c + u;
+                    const bool f = cc < c1 && cc * 32 + lane < V8 && __hge2_mask(mu[u], lo2) != 0u;
+                    const unsigned bal = __ballot_sync(kFullMask, f);
+                    if (f) {
+                        const int pos = nh + __popc(bal & ((1u << lane) - 1u));
+                        hv[pos] = cur[u];
+                        hid[pos] = (uint32_t)(cc * CH + lane * 8);
+                    }
+                    nh += __popc(bal);
+                }
+            }
+            if (!more) break;
+#pragma unroll
+            for (int u = 0; u < kGroup; ++u) cur[u] = nxt[u];
+            c += kGroup;
+        }
+        // ---- the warp's list: its exact top-k among the candidates ----
+        __syncwarp();
+        if (nh > 0) warp_flush_hits<__nv_bfloat16, CAP>(hv, hid, nh, 8, guess, buf, hist, ws, k, lane);
+        if (ws->count > k) warp_shrink_packed(buf, hist, ws, k, lane);
+        const int64_t list = (int64_t)grow * kRowsWarps + warp;
+        uint64_t* out = p.lists + list * KCAP;
+        const int cnt = ws->count;
+        for (int j = lane; j < cnt; j += 32) out[j] = buf[j];
+        if (lane == 0) {
+            p.counts[list] = cnt;
+            p.guesses[list] = float_key(guess);
+        }
+        __syncwarp();
+        // ---- the next row's first group ----
+        const int next = item + gridDim.x;
+        if (next < n_items) {
+            run_of(c0, c1);
+            r4 = reinterpret_cast<const uint4*>(row_of(next));
+#pragma unroll
+            for (int u = 0; u < kGroup; ++u) cur[u] = load(r4, c0 + u, c1);
+        }
+    }
 }
 
 inline int num_sms() {
@@ -892,12 +1123,27 @@ struct Layout {
     size_t off_lists, off_counts, off_guesses, off_recs, total;
 };
 
-inline int choose_segments(int V) {
-    static int forced = -1;
-    if (forced < 0) {
-        const char* e = getenv("UNO_VERIFY_SEGMENTS");
-        forced = e ? atoi(e) : 0;
-    }
+// The streaming kernel a batch takes: UNO_VERIFY_STREAM=warps (one CTA per row segment,
+// any dtype and alignment) or =tma (TMA-fed, 16-byte aligned rows) select one; by default
+// bf16 rows that are 16-byte aligned with V a multiple of 8 and k <= 256 take the
+// persistent row-segment kernel, the rest the per-segment CTAs.
+enum class StreamKind { kRows, kWarps, kTma };
+inline StreamKind stream_kind(const VerifyArgs& a) {
+    const bool aligned = ((reinterpret_cast<uintptr_t>(a.P) | reinterpret_cast<uintptr_t>(a.Q)) & 15u) == 0;
+    const size_t esz = a.dtype == UNO_BF16 ? 2 : 4;
+    const bool rows_aligned = aligned && ((size_t)a.V * esz) % 16 == 0;
+    const char* sel = getenv("UNO_VERIFY_STREAM");
+    if (sel && strcmp(sel, "warps") == 0) return StreamKind::kWarps;
+    if (sel && strcmp(sel, "tma") == 0) return rows_aligned ? StreamKind::kTma : StreamKind::kWarps;
+    return (a.dtype == UNO_BF16 && rows_aligned && a.top_k <= 256) ? StreamKind::kRows : StreamKind::kWarps;
+}
+
+// Segments per row: the persistent kernel takes whole rows; the per-segment CTAs one each
+// unless UNO_VERIFY_SEGMENTS=s forces s.
+inline int choose_segments(int V, StreamKind kind) {
+    if (kind == StreamKind::kRows) return 1;
+    int forced = 0;
+    if (const char* e = getenv("UNO_VERIFY_SEGMENTS")) forced = atoi(e);
     int S = forced > 0 ? forced : 1;
     int nchunks = (V + 255) / 256;
     if (S > nchunks) S = nchunks;
@@ -908,7 +1154,10 @@ inline int choose_segments(int V) {
 inline Layout layout(const VerifyArgs& a) {
     Layout L{};
     L.kcap = a.top_k <= 64 ? 64 : (a.top_k <= 256 ? 256 : 1024);
-    L.S = choose_segments(a.V);
+    L.S = choose_segments(a.V, stream_kind(a));
+    // a finishing warp holds a row's lists in shared memory: fewer segments where they
+    // would not fit
+    while (L.S > 1 && ((size_t)L.S * 8 * L.kcap * 8 + 2 * (size_t)L.kcap * 8 + 256 * 4 + 32) > 220 * 1024) --L.S;
     L.rows_per_seq = 2 * a.K - 1;
     // sized for the streaming kernel with the most warps; the launch sets the actual count
     L.lists_per_row = L.S * (kTmaWarps > kStreamWarps ? kTmaWarps : kStreamWarps);
@@ -942,41 +1191,47 @@ uno_status launch_t(const VerifyArgs& a, const Layout& L, unsigned char* ws, cud
     p.recs = ws + L.off_recs;
     p.kcap = KCAP;
     const int n_rows = a.B * L.rows_per_seq;
-    const bool rows_aligned = ((reinterpret_cast<uintptr_t>(a.P) | reinterpret_cast<uintptr_t>(a.Q)) & 15u) == 0 &&
-                              ((size_t)a.V * sizeof(T)) % 16 == 0;
-    // The register-load streaming kernel is the default; the TMA-fed persistent kernel is
-    // selected with UNO_VERIFY_STREAM=tma (it needs 16-byte aligned rows).
-    const char* sel = getenv("UNO_VERIFY_STREAM");
-    const bool use_tma = sel && strcmp(sel, "tma") == 0 && rows_aligned && tma_smem_bytes<KCAP>() <= 227 * 1024;
-    p.lists_per_row = L.S * (use_tma ? kTmaWarps : kStreamWarps);
-    static bool a1 = false, a2 = false, a3 = false;
+    const StreamKind kind = stream_kind(a);
+    const bool use_tma = kind == StreamKind::kTma && tma_smem_bytes<KCAP>() <= 227 * 1024;
+    const bool use_rows = kind == StreamKind::kRows && std::is_same<T, __nv_bfloat16>::value && KCAP <= 256;
+    p.lists_per_row = L.S * (use_tma ? kTmaWarps : (use_rows ? kRowsWarps : kStreamWarps));
+    static bool a1 = false, a2 = false;
     const size_t smem1 = (size_t)kStreamWarps * cap_entries<KCAP>() * 8 + (size_t)kStreamWarps * 256 * 4;
-    constexpr int FW = FinishCfg<KCAP>::WARPS;
-    const size_t smem2 = FW * finish_bytes_per_warp<KCAP>(p.lists_per_row);
-    const size_t region3 = (size_t)kSeqWarps * 2 * 12 * KCAP;
-    const size_t smem3 = region3 < 200 * 1024 ? region3 : 200 * 1024;
-    if (smem2 > 227 * 1024) return set_error(UNO_ERR_UNSUPPORTED, "verify: too many segments for top_k %d", a.top_k);
+    // the finish: as many warps finishing rows at once as their lists fit in shared memory
+    // (the kernel's static shared memory takes the rest of the 227 KB)
+    constexpr size_t kFinSmem = 220 * 1024;
+    const size_t per_warp = finish_bytes_per_warp<KCAP>(p.lists_per_row);
+    if (per_warp > kFinSmem) return set_error(UNO_ERR_UNSUPPORTED, "verify: too many segments for top_k %d", a.top_k);
+    const int fw = (int)std::min<size_t>(kFinWarps, kFinSmem / per_warp);
+    const size_t smem2 = std::max<size_t>((size_t)fw * per_warp, (size_t)2 * 12 * KCAP);
 
     uno_status s;
-    if ((s = set_smem(stream_kernel<T, KCAP>, smem1, a1, "cudaFuncSetAttribute(verify stream)")) != UNO_OK) return s;
-    if ((s = set_smem(finish_kernel<T, KCAP>, 227 * 1024, a2, "cudaFuncSetAttribute(verify finish)")) != UNO_OK) return s;
-    if ((s = set_smem(sequence_kernel, 200 * 1024, a3, "cudaFuncSetAttribute(verify sequence)")) != UNO_OK) return s;
-    if (use_tma) {
+    if ((s = set_smem(finish_seq_kernel<T, KCAP>, kFinSmem, a2, "cudaFuncSetAttribute(verify finish)")) != UNO_OK)
+        return s;
+    const int n_items = n_rows * L.S;
+    if (use_rows) {
+        if constexpr (KCAP <= 256) {
+            static bool a0 = false;
+            constexpr size_t smem0 = rows_smem_bytes<KCAP>();
+            if ((s = set_smem(stream_rows_kernel<KCAP>, smem0, a0, "cudaFuncSetAttribute(verify rows)")) != UNO_OK)
+                return s;
+            const int grid = std::min(n_rows, num_sms() * kRowsCtasPerSm);
+            stream_rows_kernel<KCAP><<<(unsigned)grid, kRowsWarps * 32, smem0, stream>>>(p, n_rows);
+        }
+    } else if (use_tma) {
         static bool a0 = false;
         const size_t smem0 = tma_smem_bytes<KCAP>();
         if ((s = set_smem(stream_tma_kernel<T, KCAP>, smem0, a0, "cudaFuncSetAttribute(verify stream tma)")) != UNO_OK)
             return s;
-        const int n_items = n_rows * L.S;
         const int grid = n_items < num_sms() * kTmaCtasPerSm ? n_items : num_sms() * kTmaCtasPerSm;
         stream_tma_kernel<T, KCAP><<<(unsigned)grid, kTmaWarps * 32, smem0, stream>>>(p, n_items, device_status_ptr());
     } else {
+        if ((s = set_smem(stream_kernel<T, KCAP>, smem1, a1, "cudaFuncSetAttribute(verify stream)")) != UNO_OK) return s;
         stream_kernel<T, KCAP><<<(unsigned)(n_rows * L.S), kStreamWarps * 32, smem1, stream>>>(p);
     }
     if ((s = check_cuda(cudaGetLastError(), "launch(verify stream)")) != UNO_OK) return s;
-    finish_kernel<T, KCAP><<<(unsigned)((n_rows + FW - 1) / FW), FW * 32, smem2, stream>>>(p, n_rows);
-    if ((s = check_cuda(cudaGetLastError(), "launch(verify finish)")) != UNO_OK) return s;
-    sequence_kernel<<<(unsigned)a.B, kSeqWarps * 32, smem3, stream>>>(p, smem3);
-    return check_cuda(cudaGetLastError(), "launch(verify sequence)");
+    finish_seq_kernel<T, KCAP><<<(unsigned)a.B, kFinWarps * 32, smem2, stream>>>(p, fw, smem2);
+    return check_cuda(cudaGetLastError(), "launch(verify finish)");
 }
 
 }  // namespace vtopk

@@ -177,12 +177,16 @@ def test_threshold_guess_fallback():
         _check(P, Q, u, 1.0, k, 0.95, "bf16")
 
 
-@pytest.mark.parametrize("env", [{"UNO_VERIFY_TOPK": "stream"}, {"UNO_VERIFY_TOPK": "stream", "UNO_VERIFY_STREAM": "tma"}],
-                         ids=["stream", "stream_tma"])
-def test_streaming_path_parity(env):
-    """The streaming top-k path (selected for every top-k batch by UNO_VERIFY_TOPK=stream;
-    by default it serves the batches the cluster kernel does not take) and its TMA-fed
-    variant give the oracle's result; run in a subprocess so that the selection is clean."""
+@pytest.mark.parametrize("env", [{"UNO_VERIFY_STREAM": "warps"}, {"UNO_VERIFY_STREAM": "tma"},
+                                 {"UNO_VERIFY_STREAM": "warps", "UNO_VERIFY_SEGMENTS": "3"},
+                                 {"UNO_VERIFY_TOPK": "local"}],
+                         ids=["stream_warps", "stream_tma", "stream_warps_s3", "cluster_local"])
+def test_alternate_topk_paths_parity(env):
+    """The top-k tests on the other top-k paths: the streaming kernel with one CTA per row
+    segment (UNO_VERIFY_STREAM=warps, the path of fp32 and unaligned rows), its TMA-fed
+    variant (UNO_VERIFY_STREAM=tma) and the cluster kernel with per-CTA lists
+    (UNO_VERIFY_TOPK=local, with the streaming path for the batches it does not take); run
+    in a subprocess so that the selection is clean."""
     import os
     import subprocess
     import sys
@@ -210,16 +214,15 @@ TOPK_CLUSTER_CASES = [
 @pytest.mark.parametrize("case", TOPK_CLUSTER_CASES, ids=[f"B{c[0]}K{c[1]}V{c[2]}k{c[4]}p{c[5]}" for c in TOPK_CLUSTER_CASES])
 def test_topk_cluster_kernel(case, cl, mode, monkeypatch):
     """The cluster kernels' top-k modes against the oracle, for every cluster size that fits:
-    "local" (k <= 128: every CTA takes its slice's exact top-k, a head CTA merges the lists)
-    and "window" (the row's k-th value from per-value counts over its 256 largest values,
+    "local" (k <= 128: every CTA takes its slice's exact top-k, a head CTA merges the lists,
+    selected by UNO_VERIFY_TOPK=local) and "window" (the row's k-th value from per-value counts over its 256 largest values,
     selected by UNO_VERIFY_TOPK=window; it also serves 128 < k <= 256). UNO_VERIFY_FULL=cluster
     makes any other path an error."""
     B, K, V, T, k, p = case
     from diffusion_drafted_lossless_b200._lib import UnoError
     monkeypatch.setenv("UNO_VERIFY_FULL", "cluster")
     monkeypatch.setenv("UNO_VERIFY_FULL_CLUSTER", str(cl))
-    if mode == "window":
-        monkeypatch.setenv("UNO_VERIFY_TOPK", "window")
+    monkeypatch.setenv("UNO_VERIFY_TOPK", mode)
     P, Q, u = _inputs(B, K, V, "bf16", seed=zlib.crc32(str((case, cl)).encode()) % 10007)
     try:
         _check(P, Q, u, T, k, p, "bf16")
@@ -412,10 +415,11 @@ def test_pos0_entries_below_zero_draw_from_p0(top_k):
 
 
 @pytest.mark.parametrize("k", [1, 50, 128])
-def test_topk_outlier_slices_go_to_the_generic_kernel(k):
+def test_topk_outlier_slices_go_to_the_generic_kernel(k, monkeypatch):
     """A few huge logits put the largest values of their slice far above the rest, so that
     slice holds fewer than k tokens among its 256 largest values: the cluster kernel hands
-    those items to the generic kernel, and every result must still be the oracle's."""
+    those items to the generic kernel, and every result must still be the oracle's. The
+    streaming path (the default) gets the same rows."""
     B, K, V = 3, 4, 40000
     rng = np.random.default_rng(46 + k)
     base = rng.standard_normal((B, K, V)).astype(np.float32)
@@ -424,4 +428,6 @@ def test_topk_outlier_slices_go_to_the_generic_kernel(k):
     P = W.bf16_bits(base)
     Q = W.bf16_bits((0.8 * base + 0.6 * rng.standard_normal((B, K, V))).astype(np.float32))
     u = rng.random((B, K, 3), dtype=np.float32)
+    _check(P, Q, u, 1.0, k, 0.9, "bf16")
+    monkeypatch.setenv("UNO_VERIFY_TOPK", "local")
     _check(P, Q, u, 1.0, k, 0.9, "bf16")
