@@ -1995,6 +1995,1040 @@ __global__ void __launch_bounds__(kThreads, 1) topk_local_kernel(Params p, LLayo
 }  // namespace pk
 
 // =======================================================================================
+// Row streaming (bf16 rows, V a multiple of 8, 16-byte aligned, top-k off): two persistent
+// kernels, each reading every logit once.
+//
+// row_kernel, one row per CTA at a time (the verifier rows and the drafter rows i >= 1).
+// Streaming the row it takes the largest value M, counts exactly how many tokens hold each
+// of the kWin largest order keys from an anchor a little above a sampled maximum (one count
+// array per warp), and sums the weight exp((x - F) / T) of every element below that window
+// (F its lowest value) in fp32 (ex2.approx) into an fp64 total, with a rigorous bound E on
+// that sum's error: the measured ex2 error, the three roundings of the argument and the
+// fp32 partial sums. Z = sum over the window of count * exp(v / T - M / T) in fp64 plus the
+// rescaled rest sum, known to within E. The top-p cut (the value at which the mass from the
+// top first reaches top_p * Z, and how many of the tokens at that value it keeps, lowest
+// ids first) is decided from the window's counts for top_p * (Z - E) and top_p * (Z + E):
+// when both give the same cut it is the exact one, and every mass the item pass needs (the
+// survivors lie inside the window) is a count times an fp64 weight. Otherwise (the bound
+// straddles a token boundary, the cut lies below the window, the row has no cut, an element
+// lies above the window, the window would reach non-positive values, a non-finite weight)
+// the CTA recounts the row exactly: counts per (sign, magnitude) for the kMagWin magnitudes
+// below the largest and an fp64 weight for every tinier element. A row whose cut cannot be decided that way (or whose
+// largest value is not finite) sends its item to the generic kernel.
+//
+// item_kernel_rs, one item per CTA at a time: streams the item's rows again, each warp its
+// run of chunks in id order, and sums per group of chunks the masses the draws walk (the
+// draw row's survivors, the verifier's survivors, the residual max(0, p - q)) and |p - q|.
+// A draw finds the group holding its target from those sums and rescans that group alone.
+// Tokens at a cut value survive by rank among the row's tokens at that value (the row
+// record holds how many precede each warp's run).
+// =======================================================================================
+namespace rs {
+
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+constexpr int kCtasPerSm = 2;         // item pass
+constexpr int kRowCtasPerSm = 3;      // row pass
+constexpr int kGroup = 4;             // chunks per group of the row pass (a chunk: 32 lanes x 8 elements)
+constexpr int kCh = 256;              // elements per chunk
+constexpr int kWin = 320;             // counted keys: the anchor and the kWin - 1 below it
+constexpr int kAbove = 96;            // the anchor: this many keys above the sampled maximum
+constexpr int kLutMax = 512;          // tabulated survivor weights per row
+constexpr int kMagWin = 2048;         // recount: counted magnitudes (both signs) from the largest down
+constexpr double kEx2Err = 0x1p-22;   // bound on ex2.approx.ftz.f32's relative error (2^-22.7 measured)
+constexpr double kU = 0x1p-24;        // fp32 unit roundoff
+constexpr double kLn2 = 0.6931471805599453;
+
+// A row's statistics (written by row_kernel, read by item_kernel_rs).
+struct RowRec {
+    double zmax;              // largest logit / T
+    double S;                 // surviving mass, relative to zmax
+    uint32_t kM;              // order key of the largest value
+    uint32_t kc;              // order key of the cut value: smaller keys do not survive
+    int cut;                  // 0: every token survives
+    int tie_t;                // tokens at the cut value that survive (the first tie_t by id)
+    int tie_before[kWarps];   // tokens at the cut value before each warp's run
+    int lut_n;                // lut[j]: weight of key kM - j, for j < lut_n (0 where absent)
+    int state;                // kDone, or kRedo (the item goes to the generic kernel)
+    double lut[kLutMax];
+};
+
+typedef unsigned long long f2;
+__device__ __forceinline__ f2 pk(float lo, float hi) {
+    f2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float lo_of(f2 v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float hi_of(f2 v) { return __uint_as_float((uint32_t)(v >> 32)); }
+__device__ __forceinline__ f2 add2(f2 a, f2 b) {
+    f2 d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ f2 sub2(f2 a, f2 b) {
+    f2 d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ f2 mul2(f2 a, f2 b) {
+    f2 d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float ex2f(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float bfv(uint32_t h16) { return __uint_as_float(h16 << 16); }
+__device__ __forceinline__ f2 widen(uint32_t w) { return pk(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)); }
+__device__ __forceinline__ __nv_bfloat162 bf2(uint32_t w) { return *reinterpret_cast<const __nv_bfloat162*>(&w); }
+// 16-bit order key of a bf16 value and back
+__device__ __forceinline__ uint32_t okey(uint32_t h) { return (h & 0x8000u) ? (~h & 0xFFFFu) : (h | 0x8000u); }
+__device__ __forceinline__ uint32_t obits(uint32_t k) { return (k & 0x8000u) ? (k & 0x7FFFu) : (~k & 0xFFFFu); }
+
+// rows of the item space: r < n_items the verifier row of item r, else the drafter row of
+// item r - n_items
+__device__ __forceinline__ bool row_needed(const Params& p, int r) {
+    const int n = p.B * p.K;
+    if (r < n) return !trivial_item(p, r / p.K, r % p.K);
+    return (r - n) % p.K > 0;
+}
+__device__ __forceinline__ const uint4* row_ptr(const Params& p, int r) {
+    const int n = p.B * p.K;
+    const __nv_bfloat16* base = r < n ? static_cast<const __nv_bfloat16*>(p.P) + (int64_t)r * p.V
+                                      : static_cast<const __nv_bfloat16*>(p.Q) + (int64_t)(r - n) * p.V;
+    return reinterpret_cast<const uint4*>(base);
+}
+
+// the warp's run of chunks
+__device__ __forceinline__ void warp_run(int V, int warp, int& c0, int& c1) {
+    const int nchunks = (V + kCh - 1) / kCh;
+    c0 = nchunks * warp / kWarps;
+    c1 = nchunks * (warp + 1) / kWarps;
+}
+
+// UNO_VERIFY_TRACE (profiling aid): phase timestamps of CTA 0's first 32 rows / items
+// (kernel 0: rows, 1: items), and counters of recounted rows (slot 0) and generic items (1)
+__device__ __forceinline__ void rs_mark(const Params& p, int kernel, int j, int e) {
+    if (p.trace != nullptr && blockIdx.x == 0 && threadIdx.x == 0 && j < 32) {
+        unsigned long long t;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        p.trace[((kernel * 2) * 32 + j) * 16 + e] = t;
+    }
+}
+__device__ __forceinline__ void rs_count(const Params& p, int slot) {
+    if (p.trace != nullptr && threadIdx.x == 0) atomicAdd(&p.trace[(15 * 2 * 32) * 16 + slot], 1ull);
+}
+
+__device__ __forceinline__ double cta_sum(double v, double* red) {
+    v = warp_sum_f64(v);
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    double t = 0.0;
+    for (int w = 0; w < kWarps; ++w) t += red[w];  // the same order in every thread
+    return t;
+}
+
+struct RowShared {
+    uint32_t hw[kWarps][kWin + 1];  // per-warp counts of the window keys (anchor - d); the last slot takes
+                                    // counted values above the anchor (the window is then void)
+    uint32_t hc[kWin];           // their sum
+    double wd[kWin];             // weight of window key d (where present), relative to zmax
+    uint32_t hr[2 * kMagWin];    // recount: counts of (sign, magnitude largest - d)
+    float fmax[kWarps];
+    double dz[kWarps], db[kWarps], red[kWarps];
+    int ties[kWarps];
+    int d_cut, tie_t, ok;
+    double S;
+};
+
+// The recount's bins in value order: VC over the positive magnitudes (largest first), VC2
+// over the negative ones (smallest first).
+struct VC {
+    const uint32_t* hr;
+    __device__ uint32_t operator[](int v) const { return hr[v]; }
+};
+struct VC2 {
+    const uint32_t* hr;
+    __device__ uint32_t operator[](int v) const { return hr[2 * kMagWin - 1 - v]; }
+};
+
+// The cut for `target` over bins [0, n) of masses cnt[d] * w[d] in value order (one warp,
+// every lane gets the answer): the first bin at which the running mass reaches the target
+// and how many of its tokens are kept (the fewest, at least one, that bring it there).
+// Returns false if the bins' total does not reach the target.
+template <typename C, typename W>
+__device__ bool warp_cut(C cnt, W w, int n, double target, int lane, int& dcut, long long& t, double& cb) {
+    const int per = (n + 31) / 32;
+    double s = 0.0;
+    for (int j = 0; j < per; ++j) {
+        const int d = lane * per + j;
+        if (d < n && cnt[d]) s += (double)cnt[d] * w(d);
+    }
+    const double incl = warp_scan_f64(s, lane);
+    const unsigned hit = __ballot_sync(kFullMask, s > 0.0 && incl >= target);
+    if (!hit) return false;
+    const int L = __ffs(hit) - 1;
+    double c = __shfl_sync(kFullMask, incl - s, L);
+    int found = -1;
+    for (int j = 0; j < per && found < 0; ++j) {
+        const int d = L * per + j;
+        if (d >= n || !cnt[d]) continue;
+        const double m = (double)cnt[d] * w(d);
+        if (c + m >= target) found = d;
+        else c += m;
+    }
+    if (found < 0) return false;  // rounding between the two summation orders
+    const double wk = w(found);
+    const long long kc = cnt[found];
+    long long tt = (long long)ceil((target - c) / wk);
+    if (tt < 1) tt = 1;
+    if (tt > kc) tt = kc;
+    while (tt > 1 && c + (double)(tt - 1) * wk >= target) --tt;
+    while (tt < kc && c + (double)tt * wk < target) ++tt;
+    dcut = found;
+    t = tt;
+    cb = c;
+    return true;
+}
+
+__global__ void __launch_bounds__(kThreads, kRowCtasPerSm) row_kernel(Params p, RowRec* rows) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    RowShared& sh = *reinterpret_cast<RowShared*>(smem_raw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int V = p.V, V8 = V >> 3;
+    int c0, c1;
+    warp_run(V, warp, c0, c1);
+    const int n_rows = 2 * p.B * p.K;
+    const double T = p.T;
+    const float cT = (float)(1.4426950408889634 / T);  // log2(e) / T
+
+    int jr = 0;  // rows this CTA has taken (trace)
+    for (int r = blockIdx.x; r < n_rows; r += gridDim.x) {
+        if (!row_needed(p, r)) continue;  // the same in every thread
+        const uint4* r4 = row_ptr(p, r);
+        RowRec& out = rows[r];
+        const int jm = jr++;
+        rs_mark(p, 0, jm, 0);
+        for (int j = lane; j <= kWin; j += 32) sh.hw[warp][j] = 0u;
+        auto valid = [&](int c) { return c < c1 && c * 32 + lane < V8; };
+        uint4 cur[kGroup];
+#pragma unroll
+        for (int u = 0; u < kGroup; ++u) cur[u] = valid(c0 + u) ? ld_stream_v4(r4 + (c0 + u) * 32 + lane) : make_uint4(0, 0, 0, 0);
+
+        // ---- the anchor: kAbove keys above the largest value of every warp's first group ----
+        {
+            float lm = -INFINITY;
+#pragma unroll
+            for (int u = 0; u < kGroup; ++u) {
+                if (!valid(c0 + u)) continue;
+                const uint4 v = cur[u];
+                const __nv_bfloat162 m2 = __hmax2(__hmax2(bf2(v.x), bf2(v.y)), __hmax2(bf2(v.z), bf2(v.w)));
+                lm = fmaxf(lm, fmaxf(__low2float(m2), __high2float(m2)));
+            }
+            lm = warp_max(lm);
+            if (lane == 0) sh.fmax[warp] = lm;
+        }
+        __syncthreads();
+        float smax = -INFINITY;
+        for (int w = 0; w < kWarps; ++w) smax = fmaxf(smax, sh.fmax[w]);
+        uint32_t A15 = 0x7F80u, F15 = 0x7F80u;  // no window: every element to the rest sum
+        bool fast = false;
+        if (smax < INFINITY && smax > -INFINITY) {
+            const uint32_t akey = min(okey(__float_as_uint(smax) >> 16) + (uint32_t)kAbove, 0xFF7Fu);
+            if (akey >= 0x8000u + (uint32_t)kWin) {  // the window's lowest value is positive
+                fast = true;
+                A15 = akey - 0x8000u;
+                F15 = A15 - (uint32_t)(kWin - 1);
+            }
+        }
+        const float Fv = bfv(F15);
+        const __nv_bfloat162 F2 = bf2(F15 | (F15 << 16));
+        const f2 Ff = pk(Fv, Fv), C2 = pk(cT, cT);
+
+        rs_mark(p, 0, jm, 1);
+        // ---- stream the row ----
+        __nv_bfloat162 mx2 = __floats2bfloat162_rn(-INFINITY, -INFINITY);
+        double zr = 0.0;  // rest weights exp((x - F) / T)
+        float zb = 0.f;   // rest weights times |their ex2 argument| (for the error bound)
+        uint32_t* hwp = sh.hw[warp];
+        int c = c0;
+        while (true) {
+            const bool more = c + kGroup < c1;
+            uint4 nxt[kGroup];
+            if (more) {
+#pragma unroll
+                for (int u = 0; u < kGroup; ++u)
+                    nxt[u] = valid(c + kGroup + u) ? ld_stream_v4(r4 + (c + kGroup + u) * 32 + lane) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < kGroup; ++u) {
+                if (!valid(c + u)) continue;
+                const uint32_t w4[4] = {cur[u].x, cur[u].y, cur[u].z, cur[u].w};
+                f2 acc = pk(0.f, 0.f);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t wq = w4[q];
+                    const uint32_t m = __hge2_mask(bf2(wq), F2);  // x >= F: counted (0xFFFF per half)
+                    mx2 = __hmax2(mx2, bf2(wq));
+                    const f2 a = mul2(sub2(widen(wq), Ff), C2);
+                    const bool in0 = (m & 0xFFFFu) != 0u, in1 = (m >> 16) != 0u;
+                    const float x0 = ex2f(lo_of(a)), x1 = ex2f(hi_of(a));
+                    const float e0 = in0 ? 0.f : x0, e1 = in1 ? 0.f : x1;
+                    // counted values above the anchor land in the last slot (and M shows them)
+                    const uint32_t d0 = min(A15 - (wq & 0xFFFFu), (uint32_t)kWin);
+                    const uint32_t d1 = min(A15 - (wq >> 16), (uint32_t)kWin);
+                    if (in0) atomicAdd(&hwp[d0], 1u);
+                    if (in1) atomicAdd(&hwp[d1], 1u);
+                    acc = add2(acc, pk(e0, e1));
+                    zb = fmaf(e0, fabsf(lo_of(a)), zb);
+                    zb = fmaf(e1, fabsf(hi_of(a)), zb);
+                }
+                zr += (double)lo_of(acc) + (double)hi_of(acc);
+            }
+            if (!more) break;
+#pragma unroll
+            for (int u = 0; u < kGroup; ++u) cur[u] = nxt[u];
+            c += kGroup;
+        }
+        rs_mark(p, 0, jm, 2);
+        {
+            float lm = fmaxf(__low2float(mx2), __high2float(mx2));
+            lm = warp_max(lm);
+            zr = warp_sum_f64(zr);
+            const double zbd = warp_sum_f64((double)zb);
+            __syncthreads();  // every thread has read the anchor's maxima
+            if (lane == 0) {
+                sh.fmax[warp] = lm;
+                sh.dz[warp] = zr;
+                sh.db[warp] = zbd;
+            }
+        }
+        __syncthreads();
+        float M = -INFINITY;
+        double ZR = 0.0, ZB = 0.0;
+        for (int w = 0; w < kWarps; ++w) {
+            M = fmaxf(M, sh.fmax[w]);
+            ZR += sh.dz[w];
+            ZB += sh.db[w];
+        }
+        if (M == 0.f) M = 0.f;  // +0
+        // a value above the anchor was not counted: the window is void
+        const int OVF = fast && (__float_as_uint(M) >> 16) > A15;
+        const bool finite_max = M < INFINITY && M > -INFINITY;
+        const double zmax = (double)M / T;
+        const uint32_t kM = okey(__float_as_uint(M) >> 16);
+        bool exact = fast && !OVF && p.cut && finite_max && ZR < INFINITY && ZB < INFINITY;  // NaN fails
+
+        // ---- the window's masses, Z within E, and the cut ----
+        if (exact) {
+            double zw = 0.0;
+            for (int d = tid; d < kWin; d += kThreads) {
+                uint32_t cnt = 0;
+                for (int w = 0; w < kWarps; ++w) cnt += sh.hw[w][d];
+                sh.hc[d] = cnt;
+                const double wv = cnt ? exp((double)bfv(A15 - (uint32_t)d) / T - zmax) : 0.0;
+                sh.wd[d] = wv;
+                zw += (double)cnt * wv;
+            }
+            zw = cta_sum(zw, sh.red);
+            const double fz = exp((double)Fv / T - zmax);
+            const double Zr = ZR * fz;
+            const double Z = zw + Zr;
+            const double E = 1.01 * ((kEx2Err + 3.0 * kU) * ZR + 3.0 * kU * kLn2 * ZB) * fz + 1e-14 * Z;
+            if (warp == 0) {
+                int d_lo = -1, d_hi = -2;
+                long long t_lo = 0, t_hi = -1;
+                double cb_lo = 0.0, cb_hi = 0.0;
+                auto wwin = [&](int d) { return sh.wd[d]; };
+                const bool a = warp_cut(sh.hc, wwin, kWin, p.top_p * (Z - E), lane, d_lo, t_lo, cb_lo);
+                const bool b = warp_cut(sh.hc, wwin, kWin, p.top_p * (Z + E), lane, d_hi, t_hi, cb_hi);
+                if (lane == 0) {
+                    sh.ok = a && b && d_lo == d_hi && t_lo == t_hi;
+                    sh.d_cut = d_hi;
+                    sh.tie_t = (int)t_hi;
+                    sh.S = cb_hi + (double)t_hi * sh.wd[max(d_hi, 0)];
+                }
+            }
+            __syncthreads();
+            exact = sh.ok;
+        }
+        rs_mark(p, 0, jm, 3);
+        if (exact) {
+            const int dcut = sh.d_cut;
+            const int d0 = (int)(A15 - (__float_as_uint(M) >> 16));  // the largest value's bin
+            const int lut_n = dcut - d0 + 1;
+            for (int j = tid; j < lut_n; j += kThreads) out.lut[j] = sh.wd[d0 + j];
+            if (tid == 0) {
+                out.zmax = zmax;
+                out.S = sh.S;
+                out.kM = kM;
+                out.kc = (A15 - (uint32_t)dcut) | 0x8000u;
+                out.cut = 1;
+                out.tie_t = sh.tie_t;
+                int before = 0;
+                for (int w = 0; w < kWarps; ++w) {
+                    out.tie_before[w] = before;
+                    before += (int)sh.hw[w][dcut];
+                }
+                out.lut_n = lut_n;
+                out.state = kDone;
+            }
+            __syncthreads();  // the window counts are reused by the next row
+            continue;
+        }
+
+        // ---- exact recount ----
+        rs_count(p, 0);
+        if (!finite_max) {
+            if (tid == 0) out.state = kRedo;
+            __syncthreads();
+            continue;
+        }
+        // the largest magnitude (pass 1), then counts per (sign, magnitude) for the kMagWin
+        // magnitudes below it and fp64 weights for the tinier ones (pass 2)
+        for (int d = tid; d < 2 * kMagWin; d += kThreads) sh.hr[d] = 0u;
+        uint32_t am = 0u;
+        for (int cb = c0; cb < c1; cb += kGroup) {
+            uint4 vv[kGroup];
+#pragma unroll
+            for (int u = 0; u < kGroup; ++u) vv[u] = valid(cb + u) ? ld_stream_v4(r4 + (cb + u) * 32 + lane) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int u = 0; u < kGroup; ++u) {
+                const uint32_t w4[4] = {vv[u].x, vv[u].y, vv[u].z, vv[u].w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) am = max(am, max(w4[q] & 0x7FFFu, (w4[q] >> 16) & 0x7FFFu));
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) am = max(am, __shfl_xor_sync(kFullMask, am, o));
+        if (lane == 0) sh.ties[warp] = (int)am;
+        __syncthreads();
+        uint32_t atop = 0u;
+        for (int w = 0; w < kWarps; ++w) atop = max(atop, (uint32_t)sh.ties[w]);
+        double zo = 0.0;
+        for (int cb = c0; cb < c1; cb += kGroup) {
+            uint4 vv[kGroup];
+#pragma unroll
+            for (int u = 0; u < kGroup; ++u) vv[u] = valid(cb + u) ? ld_stream_v4(r4 + (cb + u) * 32 + lane) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int u = 0; u < kGroup; ++u) {
+                if (!valid(cb + u)) continue;
+                const uint32_t w4[4] = {vv[u].x, vv[u].y, vv[u].z, vv[u].w};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const uint32_t h = (w4[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
+                    const uint32_t d = atop - (h & 0x7FFFu);
+                    if (d < (uint32_t)kMagWin) atomicAdd(&sh.hr[(h >> 15) * kMagWin + d], 1u);
+                    else zo += exp((double)bfv(h) / T - zmax);
+                }
+            }
+        }
+        __syncthreads();
+        // value order: positive magnitudes from the top, the tiny ones, negative magnitudes
+        // from the bottom; virtual bin v < kMagWin is (+, d = v), v >= kMagWin (-, d = 2 kMagWin - 1 - v)
+        auto vcnt = [&](int v) -> uint32_t {
+            return v < kMagWin ? sh.hr[v] : sh.hr[kMagWin + (2 * kMagWin - 1 - v)];
+        };
+        auto vbits = [&](int v) -> uint32_t {
+            return v < kMagWin ? atop - (uint32_t)v : 0x8000u | (atop - (uint32_t)(2 * kMagWin - 1 - v));
+        };
+        auto vw = [&](int v) -> double { return (atop >= (uint32_t)(v < kMagWin ? v : 2 * kMagWin - 1 - v)) ? exp((double)bfv(vbits(v)) / T - zmax) : 0.0; };
+        double zp = 0.0, zn = 0.0;  // masses of the positive and the negative bins
+        for (int v = tid; v < 2 * kMagWin; v += kThreads) {
+            const uint32_t cnt = vcnt(v);
+            if (!cnt) continue;
+            const double m = (double)cnt * vw(v);
+            if (v < kMagWin) zp += m;
+            else zn += m;
+        }
+        rs_mark(p, 0, jm, 4);
+        zp = cta_sum(zp, sh.red);
+        zn = cta_sum(zn, sh.red);
+        zo = cta_sum(zo, sh.red);
+        const double Z = zp + zo + zn;
+        if (warp == 0) {
+            int v = -1;
+            long long tt = 0;
+            double cb = 0.0;
+            bool ok = Z > 0.0 && Z < INFINITY;
+            if (ok && p.cut) {
+                const double target = p.top_p * Z;
+                VC vc{sh.hr};
+                if (warp_cut(vc, vw, kMagWin, target, lane, v, tt, cb)) {
+                    // the cut among the positive magnitudes
+                } else if (target <= zp + zo) {
+                    ok = false;  // among the tiniest magnitudes: the generic kernel decides
+                } else {
+                    // among the negative magnitudes (virtual bins kMagWin ..)
+                    auto vw2 = [&](int x) { return vw(x + kMagWin); };
+                    VC2 vc2{sh.hr};
+                    ok = warp_cut(vc2, vw2, kMagWin, target - zp - zo, lane, v, tt, cb);
+                    if (ok) {
+                        v += kMagWin;
+                        cb += zp + zo;
+                    }
+                }
+                // +0 and -0 are one value under two keys: leave such a cut to the generic kernel
+                if (ok && (vbits(v) & 0x7FFFu) == 0u) ok = false;
+            }
+            if (lane == 0) {
+                sh.ok = ok;
+                sh.d_cut = v;
+                sh.tie_t = (int)tt;
+                sh.S = p.cut ? (ok ? cb + (double)tt * vw(v) : 0.0) : Z;
+            }
+        }
+        __syncthreads();
+        if (!sh.ok) {
+            if (tid == 0) out.state = kRedo;
+            rs_count(p, 1);
+            __syncthreads();
+            continue;
+        }
+        const int dcut = sh.d_cut;
+        const uint32_t kc = p.cut ? okey(vbits(dcut)) : 0u;
+        // tokens at the cut value in each warp's run
+        if (p.cut) {
+            int cnt = 0;
+            for (int cb = c0; cb < c1; cb += kGroup) {
+                uint4 vv[kGroup];
+#pragma unroll
+                for (int u = 0; u < kGroup; ++u) vv[u] = valid(cb + u) ? ld_stream_v4(r4 + (cb + u) * 32 + lane) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                for (int u = 0; u < kGroup; ++u) {
+                    if (!valid(cb + u)) continue;
+                    const uint32_t w4[4] = {vv[u].x, vv[u].y, vv[u].z, vv[u].w};
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) cnt += okey((w4[e >> 1] >> (16 * (e & 1))) & 0xFFFFu) == kc;
+                }
+            }
+            cnt = warp_sum(cnt);
+            if (lane == 0) sh.ties[warp] = cnt;
+        }
+        const int lut_n = p.cut ? (int)min((uint32_t)kLutMax, kM - kc + 1u) : kLutMax;
+        for (int j = tid; j < lut_n; j += kThreads)
+            out.lut[j] = kM >= (uint32_t)j ? exp((double)bfv(obits(kM - (uint32_t)j)) / T - zmax) : 0.0;
+        __syncthreads();
+        if (tid == 0) {
+            out.zmax = zmax;
+            out.S = sh.S;
+            out.kM = kM;
+            out.kc = kc;
+            out.cut = p.cut;
+            out.tie_t = sh.tie_t;
+            int before = 0;
+            for (int w = 0; w < kWarps; ++w) {
+                out.tie_before[w] = before;
+                before += p.cut ? sh.ties[w] : 0;
+            }
+            out.lut_n = lut_n;
+            out.state = kDone;
+        }
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// item pass
+// ---------------------------------------------------------------------------------------
+struct RowView {
+    double zmax, iS, S;
+    uint32_t kM, kc;
+    int cut, tie_t, tie_before, lut_n;
+    const double* lut;  // shared memory
+};
+
+// survivor weight of value bits h (relative to zmax) if it survives by value alone, or is
+// at the cut value (the caller ranks those); 0 otherwise
+__device__ __noinline__ double weight_far(uint32_t h, double T, double zmax) { return exp((double)bfv(h) / T - zmax); }
+__device__ __forceinline__ double weight_of(const RowView& R, uint32_t h, double T) {
+    const uint32_t j = R.kM - okey(h);
+    return j < (uint32_t)R.lut_n ? R.lut[j] : weight_far(h, T, R.zmax);
+}
+
+// the 8-bit masks of this lane's 8 elements strictly above / equal to the cut value
+__device__ __forceinline__ void cut_masks(const uint4& v, const RowView& R, uint32_t& gt, uint32_t& eq) {
+    gt = 0u;
+    eq = 0u;
+    if (!R.cut) {
+        gt = 0xFFu;
+        return;
+    }
+    const uint32_t cb = obits(R.kc);
+    const __nv_bfloat162 c2 = bf2(cb | (cb << 16));
+    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint32_t g = __hgt2_mask(bf2(w4[q]), c2), e = __heq2_mask(bf2(w4[q]), c2);
+        gt |= ((g & 1u) << (2 * q)) | (((g >> 16) & 1u) << (2 * q + 1));
+        eq |= ((e & 1u) << (2 * q)) | (((e >> 16) & 1u) << (2 * q + 1));
+    }
+    // +0 and -0 compare equal as bf16 but the cut is never at zero (those go to the generic kernel)
+}
+
+// Keep the ties (eq) this lane holds whose rank among the row's tokens at the cut value is
+// below tie_t; seen: ties before this chunk in the warp's run (updated; the same in all lanes).
+__device__ __forceinline__ uint32_t rank_ties(uint32_t eq, const RowView& R, int& seen, int lane) {
+    const int ce = __popc(eq);
+    const int incl = warp_inclusive_scan(ce, lane);
+    const int base = R.tie_before + seen + incl - ce;
+    seen += __shfl_sync(kFullMask, incl, 31);
+    int keep = R.tie_t - base;
+    if (keep <= 0) return 0u;
+    uint32_t kept = 0u, m = eq;
+    while (m && keep > 0) {
+        const uint32_t bit = m & (0u - m);
+        kept |= bit;
+        m ^= bit;
+        --keep;
+    }
+    return kept;
+}
+
+constexpr int kIG = 4;              // chunks per group of the item pass
+constexpr int kMaxIGroups = 128;    // its groups per warp run (V <= kWarps * kMaxIGroups * kIG * kCh)
+constexpr int kQueue = 32 + 4 * 32;  // word pairs queued per warp: < 32 carried + one chunk
+
+struct ItemShared {
+    double lut[2][kLutMax];
+    double gs[kWarps][kMaxIGroups][3];   // per group: draw row, verifier survivors, residual
+    int gseen[kWarps][kMaxIGroups][2];   // ties seen before the group (verifier, drafter)
+    uint4 queue[kWarps][kQueue];         // word pairs with a kept token: (verifier, drafter, masks, first id)
+    double wt[kWarps][3];                // per warp run: the totals of gs
+    int ng[kWarps];                      // groups per warp run
+    double red[kWarps];
+    int sel_w, sel_g, mode;
+    double sel_c;
+    int tok_found;
+};
+
+// survivor masks of one chunk for both rows (ties ranked)
+__device__ __forceinline__ void chunk_survivors(const uint4& vp, const uint4& vq, bool two, const RowView& P,
+                                                const RowView& Q, int& seen_p, int& seen_q, int lane, uint32_t& sp,
+                                                uint32_t& sq) {
+    uint32_t gp, ep, gq = 0u, eq = 0u;
+    cut_masks(vp, P, gp, ep);
+    if (two) cut_masks(vq, Q, gq, eq);
+    if (__any_sync(kFullMask, ep != 0u)) gp |= rank_ties(ep, P, seen_p, lane);
+    if (two && __any_sync(kFullMask, eq != 0u)) gq |= rank_ties(eq, Q, seen_q, lane);
+    sp = gp;
+    sq = gq;
+}
+
+// the per-element masses of one chunk for the draw modes (0: draw row, 1: verifier, 2: residual)
+__device__ __forceinline__ void chunk_masses(const uint4& vp, const uint4& vq, uint32_t mp, uint32_t mq, bool two,
+                                             const RowView& P, const RowView& Q, double T, int mode, double (&x)[8]) {
+    const uint32_t wp4[4] = {vp.x, vp.y, vp.z, vp.w};
+    const uint32_t wq4[4] = {vq.x, vq.y, vq.z, vq.w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const double wp = (mp >> e) & 1u ? weight_of(P, (wp4[e >> 1] >> (16 * (e & 1))) & 0xFFFFu, T) : 0.0;
+        const double wq = (mq >> e) & 1u ? weight_of(Q, (wq4[e >> 1] >> (16 * (e & 1))) & 0xFFFFu, T) : 0.0;
+        double v;
+        if (mode == 1) v = wp;
+        else if (mode == 0) v = two ? wq : wp;
+        else {
+            const double dl = wp * P.iS - wq * Q.iS;
+            v = dl > 0.0 ? dl : 0.0;
+        }
+        x[e] = v;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, kCtasPerSm) item_kernel_rs(Params p, const RowRec* rows) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    ItemShared& sh = *reinterpret_cast<ItemShared*>(smem_raw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int V = p.V, V8 = V >> 3;
+    int c0, c1;
+    warp_run(V, warp, c0, c1);
+    const int n_items = p.B * p.K;
+    const double T = p.T;
+
+    int ji = 0;  // items this CTA has taken (trace)
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+        const int b = item / p.K, i = item % p.K;
+        if (trivial_item(p, b, i)) {
+            if (tid == 0) write_trivial(p, item, b);
+            continue;
+        }
+        const int jm = ji++;
+        rs_mark(p, 1, jm, 0);
+        const bool two = i > 0;
+        const RowRec& rp = rows[item];
+        const RowRec& rq = rows[n_items + item];
+        if (rp.state != kDone || (two && rq.state != kDone)) {
+            if (tid == 0) p.recs[item].state = kRedo;
+            continue;
+        }
+        RowView P, Q;
+        auto view = [&](const RowRec& rr, int slot, RowView& R) {
+            R.zmax = rr.zmax;
+            R.S = rr.S;
+            R.iS = 1.0 / rr.S;
+            R.kM = rr.kM;
+            R.kc = rr.kc;
+            R.cut = rr.cut;
+            R.tie_t = rr.tie_t;
+            R.tie_before = rr.tie_before[warp];
+            R.lut_n = rr.lut_n;
+            R.lut = sh.lut[slot];
+            for (int j = tid; j < rr.lut_n; j += kThreads) sh.lut[slot][j] = rr.lut[j];
+        };
+        __syncthreads();  // the previous item is done with the tables
+        view(rp, 0, P);
+        if (two) view(rq, 1, Q);
+        else Q = P;
+        __syncthreads();
+        rs_mark(p, 1, jm, 1);
+
+        const uint4* p4 = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.P) + (int64_t)item * V);
+        const uint4* q4 = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.Q) + (int64_t)item * V);
+        auto valid = [&](int c) { return c < c1 && c * 32 + lane < V8; };
+        auto ldp = [&](int c) { return valid(c) ? ld_stream_v4(p4 + c * 32 + lane) : make_uint4(0, 0, 0, 0); };
+        auto ldq = [&](int c) { return (two && valid(c)) ? ld_stream_v4(q4 + c * 32 + lane) : make_uint4(0, 0, 0, 0); };
+
+        // ---- per-group masses in id order (the next group's loads in flight) ----
+        // Word pairs (two tokens of each row) holding a token at or above a row's cut value
+        // are queued in id order with the masks of those tokens; 32 queued pairs are weighed
+        // at a time, one per lane, tokens at the cut value ranked among the row's as they come.
+        const uint32_t cbp = P.cut ? obits(P.kc) : 0u, cbq = Q.cut ? obits(Q.kc) : 0u;
+        const __nv_bfloat162 cp2 = bf2(cbp | (cbp << 16)), cq2 = bf2(cbq | (cbq << 16));
+        uint4* qu = sh.queue[warp];
+        int seen_p = 0, seen_q = 0, g = 0, nq = 0;
+        double acc_d = 0.0, acc_v = 0.0, acc_r = 0.0;  // this lane's masses of the current group
+        // tokens at a cut value in entries of lower lanes and before element e: kept while their
+        // rank is below tie_t (m: the row's 2-bit mask of this entry, updated)
+        auto rank2 = [&](uint32_t w, uint32_t& m, uint32_t cb, const RowView& R, int& seen) {
+            const uint32_t t0 = (m & 1u) && (w & 0xFFFFu) == cb, t1 = ((m >> 1) & 1u) && (w >> 16) == cb;
+            const unsigned any = __ballot_sync(kFullMask, t0 | t1);
+            if (!any) return;
+            const int c = (int)(t0 + t1);
+            const int incl = warp_inclusive_scan(c, lane);
+            const int r0 = R.tie_before + seen + incl - c;
+            if (t0 && r0 >= R.tie_t) m &= ~1u;
+            if (t1 && r0 + (int)t0 >= R.tie_t) m &= ~2u;
+            seen += __shfl_sync(kFullMask, incl, 31);
+        };
+        // weigh queue entries [off, off + n) (n <= 32): one per lane
+        auto weigh = [&](int off, int n) {
+            const uint4 e = lane < n ? qu[off + lane] : make_uint4(0u, 0u, 0u, 0u);
+            uint32_t mp = e.z & 3u, mq = (e.z >> 2) & 3u;
+            if (P.cut) rank2(e.x, mp, cbp, P, seen_p);
+            if (two && Q.cut) rank2(e.y, mq, cbq, Q, seen_q);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const double wp = (mp >> h) & 1u ? weight_of(P, (e.x >> (16 * h)) & 0xFFFFu, T) : 0.0;
+                const double wq = (mq >> h) & 1u ? weight_of(Q, (e.y >> (16 * h)) & 0xFFFFu, T) : 0.0;
+                acc_v += wp;
+                acc_d += two ? wq : wp;
+                const double dl = wp * P.iS - wq * Q.iS;
+                acc_r += dl > 0.0 ? dl : 0.0;
+            }
+        };
+        double tw[3] = {0.0, 0.0, 0.0};
+        if (c0 < c1) {
+            uint4 cp[kIG], cq[kIG];
+#pragma unroll
+            for (int u = 0; u < kIG; ++u) {
+                cp[u] = ldp(c0 + u);
+                cq[u] = ldq(c0 + u);
+            }
+            for (int c = c0;; c += kIG, ++g) {
+                const bool more = c + kIG < c1;
+                uint4 np[kIG], nq4[kIG];
+                if (more) {
+#pragma unroll
+                    for (int u = 0; u < kIG; ++u) {
+                        np[u] = ldp(c + kIG + u);
+                        nq4[u] = ldq(c + kIG + u);
+                    }
+                }
+                if (lane == 0) {
+                    sh.gseen[warp][g][0] = seen_p;
+                    sh.gseen[warp][g][1] = seen_q;
+                }
+#pragma unroll
+                for (int u = 0; u < kIG; ++u) {
+                    if (c + u >= c1) continue;  // the same in every lane
+                    // this lane's word pairs with a token at or above a row's cut value
+                    const uint32_t wp4[4] = {cp[u].x, cp[u].y, cp[u].z, cp[u].w};
+                    const uint32_t wq4[4] = {cq[u].x, cq[u].y, cq[u].z, cq[u].w};
+                    uint32_t mk[4];
+                    int cnt = 0;
+                    const bool ok = valid(c + u);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t a = P.cut ? (__hge2_mask(bf2(wp4[q]), cp2) >> 15) & 3u : 3u;
+                        const uint32_t b2 = two ? (Q.cut ? (__hge2_mask(bf2(wq4[q]), cq2) >> 15) & 3u : 3u) : 0u;
+                        mk[q] = ok ? (a | (b2 << 2)) : 0u;
+                        cnt += mk[q] != 0u;
+                    }
+                    const int incl = warp_inclusive_scan(cnt, lane);
+                    int pos = nq + incl - cnt;
+                    const uint32_t id0 = (uint32_t)((c + u) * kCh + lane * 8);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        if (mk[q]) qu[pos++] = make_uint4(wp4[q], wq4[q], mk[q], id0 + 2 * q);
+                    nq += __shfl_sync(kFullMask, incl, 31);
+                    __syncwarp();
+                    // weigh whole rounds of 32; the rest moves to the front
+                    int done = 0;
+                    for (; nq - done >= 32; done += 32) weigh(done, 32);
+                    if (done > 0) {
+                        const int rest = nq - done;
+                        const uint4 v = lane < rest ? qu[done + lane] : make_uint4(0u, 0u, 0u, 0u);
+                        __syncwarp();
+                        if (lane < rest) qu[lane] = v;
+                        __syncwarp();
+                        nq = rest;
+                    }
+                }
+                // the group's last queued tokens, then its masses
+                if (nq > 0) {
+                    weigh(0, nq);
+                    nq = 0;
+                }
+                __syncwarp();
+                const double sd = warp_sum_f64(acc_d), sv = warp_sum_f64(acc_v), sr = warp_sum_f64(acc_r);
+                acc_d = acc_v = acc_r = 0.0;
+                tw[0] += sd;
+                tw[1] += sv;
+                tw[2] += sr;
+                if (lane == 0) {
+                    sh.gs[warp][g][0] = sd;
+                    sh.gs[warp][g][1] = sv;
+                    sh.gs[warp][g][2] = sr;
+                }
+                if (!more) {
+                    ++g;
+                    break;
+                }
+#pragma unroll
+                for (int u = 0; u < kIG; ++u) {
+                    cp[u] = np[u];
+                    cq[u] = nq4[u];
+                }
+            }
+        }
+        if (lane == 0) {
+            sh.ng[warp] = g;
+            for (int k = 0; k < 3; ++k) sh.wt[warp][k] = tw[k];
+        }
+        __syncthreads();
+        rs_mark(p, 1, jm, 2);
+
+        // ---- draws: the group holding the target, then the token within it ----
+        // The first token whose running mass (id order) exceeds the target; if rounding
+        // leaves no crossing, the last token with positive mass; -1 if there is none.
+        auto draw = [&](int mode, double target) -> int {
+            if (warp == 0) {
+                // the warp run, then (lanes over its groups) the group
+                double cacc = 0.0, clast = 0.0;
+                int sw = -1, lw = -1;
+                for (int w = 0; w < kWarps; ++w) {
+                    const double m = sh.wt[w][mode];
+                    if (!(m > 0.0)) continue;
+                    lw = w;
+                    clast = cacc;
+                    if (cacc + m > target) {
+                        sw = w;
+                        break;
+                    }
+                    cacc += m;
+                }
+                const bool last_mode = sw < 0;
+                const int w = last_mode ? lw : sw;
+                double base = last_mode ? clast : cacc;
+                int sg = -1;
+                if (w >= 0) {
+                    const int n = sh.ng[w];
+                    const int per = (n + 31) / 32;
+                    double s = 0.0;
+                    int lastg = -1;
+                    for (int j = 0; j < per; ++j) {
+                        const int gg = lane * per + j;
+                        if (gg < n && sh.gs[w][gg][mode] > 0.0) {
+                            s += sh.gs[w][gg][mode];
+                            lastg = gg;
+                        }
+                    }
+                    const double incl = warp_scan_f64(s, lane);
+                    const unsigned hit = last_mode ? 0u : __ballot_sync(kFullMask, s > 0.0 && base + incl > target);
+                    int L;
+                    if (hit) {
+                        L = __ffs(hit) - 1;
+                    } else {  // the last lane with mass
+                        const unsigned any = __ballot_sync(kFullMask, s > 0.0);
+                        L = any ? 31 - __clz(any) : -1;
+                    }
+                    if (L >= 0) {
+                        double cg = base + __shfl_sync(kFullMask, incl - s, L);
+                        int pick = -1;
+                        const int lg = __shfl_sync(kFullMask, lastg, L);
+                        for (int j = 0; j < per && pick < 0 && hit; ++j) {
+                            const int gg = L * per + j;
+                            if (gg >= n) break;
+                            const double m = sh.gs[w][gg][mode];
+                            if (!(m > 0.0)) continue;
+                            if (cg + m > target) pick = gg;
+                            else cg += m;
+                        }
+                        if (pick < 0) {  // no crossing (rounding, or past the end): the last group with mass
+                            pick = lg;
+                            cg = base + __shfl_sync(kFullMask, incl - s, L);
+                            for (int j = 0; j < per; ++j) {
+                                const int gg = L * per + j;
+                                if (gg >= pick) break;
+                                const double m = sh.gs[w][gg][mode];
+                                if (m > 0.0) cg += m;
+                            }
+                            sh.mode = 1;
+                        } else {
+                            sh.mode = last_mode;
+                        }
+                        sg = pick;
+                        base = cg;
+                    }
+                }
+                if (lane == 0) {
+                    sh.sel_w = sg >= 0 ? w : -1;
+                    sh.sel_g = sg;
+                    sh.sel_c = base;
+                    sh.tok_found = -1;
+                }
+            }
+            __syncthreads();
+            const int sw = sh.sel_w;
+            if (sw < 0) return -1;
+            if (warp == sw) {
+                const bool last_mode = sh.mode;
+                const int sg = sh.sel_g;
+                int seen_pp = sh.gseen[sw][sg][0], seen_qq = sh.gseen[sw][sg][1];
+                double carry = sh.sel_c;
+                int res = -1, lastpos = -1;
+                const int cs = c0 + sg * kIG;
+                uint4 gp[kIG], gq[kIG];
+#pragma unroll
+                for (int u = 0; u < kIG; ++u) {
+                    gp[u] = ldp(cs + u);
+                    gq[u] = ldq(cs + u);
+                }
+#pragma unroll
+                for (int u = 0; u < kIG; ++u) {
+                    const int cc = cs + u;
+                    if (cc >= c1 || res >= 0) continue;  // the same in every lane
+                    uint32_t mp, mq;
+                    chunk_survivors(gp[u], gq[u], two, P, Q, seen_pp, seen_qq, lane, mp, mq);
+                    if (!valid(cc)) mp = mq = 0u;
+                    double x[8];
+                    chunk_masses(gp[u], gq[u], mp, mq, two, P, Q, T, mode, x);
+                    double lsum = 0.0;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) lsum += x[e];
+                    const double incl = warp_scan_f64(lsum, lane);
+                    const double before = carry + incl - lsum;
+                    const unsigned hit = last_mode ? 0u : __ballot_sync(kFullMask, lsum > 0.0 && carry + incl > target);
+                    if (hit) {
+                        const int L = __ffs(hit) - 1;
+                        int pos = -1;
+                        if (lane == L) {
+                            double cc2 = before;
+                            for (int e = 0; e < 8 && pos < 0; ++e) {
+                                if (x[e] > 0.0 && cc2 + x[e] > target) pos = e;
+                                cc2 += x[e];
+                            }
+                            if (pos < 0)  // rounding: the lane's last positive element
+                                for (int e = 7; e >= 0 && pos < 0; --e)
+                                    if (x[e] > 0.0) pos = e;
+                        }
+                        pos = __shfl_sync(kFullMask, pos, L);
+                        res = cc * kCh + L * 8 + pos;
+                    }
+                    unsigned posm = 0u;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) posm |= (x[e] > 0.0 ? 1u : 0u) << e;
+                    const unsigned anyp = __ballot_sync(kFullMask, posm != 0u);
+                    if (anyp) {
+                        const int L = 31 - __clz(anyp);
+                        const int e = 31 - __clz(__shfl_sync(kFullMask, posm, L));
+                        lastpos = cc * kCh + L * 8 + e;
+                    }
+                    carry += __shfl_sync(kFullMask, incl, 31);
+                }
+                if (res < 0) res = lastpos;
+                if (lane == 0) sh.tok_found = res;
+            }
+            __syncthreads();
+            const int out = sh.tok_found;
+            __syncthreads();
+            return out;
+        };
+
+        const float* u = p.u + (int64_t)item * 3;
+        Rec rec;
+        rec.state = kDone;
+        rec.pad = 0.0;
+        int tok;
+        if (!two) tok = pos0_given(p, b) ? p.pos0[b] : draw(0, (double)u[0] * P.S);
+        else tok = p.drafts ? p.drafts[item] : draw(0, (double)u[0] * Q.S);
+        rs_mark(p, 1, jm, 3);
+        rec.tok = tok;
+        rec.res = -1;
+        rec.acc = 1;
+        rec.tv = 0.0;
+        rec.p = 0.0;
+        rec.q = 0.0;
+        // P(tok) and Q(tok): value, survival (a token at the cut value is ranked by the count
+        // of those before it, one pass by the whole CTA)
+        {
+            const bool in = tok >= 0 && tok < V;
+            double pr[2] = {0.0, 0.0};
+            for (int rr = 0; rr < (two ? 2 : 1); ++rr) {
+                const RowView& R = rr == 0 ? P : Q;
+                const uint4* r4 = rr == 0 ? p4 : q4;
+                uint32_t h = 0u;
+                int state = 0;  // 0: not a survivor, 1: survivor, 2: at the cut value (rank it)
+                if (in) {
+                    h = reinterpret_cast<const uint16_t*>(r4)[tok];
+                    if (!R.cut) state = 1;
+                    else {
+                        const uint32_t k = okey(h);
+                        state = k > R.kc ? 1 : (k == R.kc ? 2 : 0);
+                    }
+                }
+                if (state == 2) {
+                    const uint32_t cbits = obits(R.kc);
+                    int cnt = 0;
+                    for (int v = tid; v < tok; v += kThreads) cnt += reinterpret_cast<const uint16_t*>(r4)[v] == cbits;
+                    const double tot = cta_sum((double)cnt, sh.red);
+                    state = tot < (double)R.tie_t ? 1 : 0;
+                }
+                if (state == 1) pr[rr] = weight_of(R, h, T) * R.iS;
+            }
+            rec.p = pr[0];
+            rec.q = pr[1];
+        }
+        rs_mark(p, 1, jm, 4);
+        if (two) {
+            rec.acc = (double)u[1] * rec.q < rec.p;
+            double R = 0.0;
+            for (int w = 0; w < kWarps; ++w) R += sh.wt[w][2];
+            rec.tv = R;  // TV(p, q) = sum of max(0, p - q), both distributions summing to 1
+            rec.res = R > 0.0 ? draw(2, (double)u[2] * R) : draw(1, (double)u[2] * P.S);
+        }
+        rs_mark(p, 1, jm, 5);
+        if (tid == 0) p.recs[item] = rec;
+    }
+}
+
+}  // namespace rs
+
+// =======================================================================================
 // per sequence: the longest accepted prefix and the outputs
 // =======================================================================================
 __global__ void assemble_kernel(Params p, int32_t* out_tokens, int32_t* out_count, int32_t* out_next, float* out_p,
@@ -2268,6 +3302,49 @@ bool launch_local(const VerifyArgs& a, const Params& p, cudaStream_t stream, uno
     return true;
 }
 
+// The row-streaming path takes bf16 rows, 16-byte aligned, V a multiple of 8 (and at most
+// the groups its item pass keeps sums for), top-k off; UNO_VERIFY_FULL=generic or =cluster
+// selects another path.
+bool rs_applies(const VerifyArgs& a) {
+    const char* mode = getenv("UNO_VERIFY_FULL");
+    if (mode && (strcmp(mode, "generic") == 0 || strcmp(mode, "cluster") == 0)) return false;
+    const int64_t vmax = (int64_t)rs::kWarps * rs::kMaxIGroups * rs::kIG * rs::kCh;
+    return a.top_k == 0 && a.dtype == UNO_BF16 && a.V % 8 == 0 && (int64_t)a.V <= vmax &&
+           ((reinterpret_cast<uintptr_t>(a.P) | reinterpret_cast<uintptr_t>(a.Q)) & 15u) == 0;
+}
+
+int num_sms();
+
+uno_status launch_rs(const VerifyArgs& a, const Params& p, rs::RowRec* rows, cudaStream_t stream) {
+    static std::mutex mu;
+    static bool ready[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return set_error(UNO_ERR_CUDA, "verify: no device");
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!ready[dev]) {
+            uno_status s;
+            if ((s = check_cuda(cudaFuncSetAttribute(rs::row_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                     (int)sizeof(rs::RowShared)),
+                                "cudaFuncSetAttribute(verify rows)")) != UNO_OK)
+                return s;
+            if ((s = check_cuda(cudaFuncSetAttribute(rs::item_kernel_rs, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                     (int)sizeof(rs::ItemShared)),
+                                "cudaFuncSetAttribute(verify items)")) != UNO_OK)
+                return s;
+            ready[dev] = true;
+        }
+    }
+    const int items = a.B * a.K;
+    const int slots = num_sms() * rs::kCtasPerSm;
+    rs::row_kernel<<<(unsigned)std::min(2 * items, num_sms() * rs::kRowCtasPerSm), rs::kThreads, sizeof(rs::RowShared),
+                     stream>>>(p, rows);
+    uno_status s = check_cuda(cudaGetLastError(), "launch(verify rows)");
+    if (s != UNO_OK) return s;
+    rs::item_kernel_rs<<<(unsigned)std::min(items, slots), rs::kThreads, sizeof(rs::ItemShared), stream>>>(p, rows);
+    return check_cuda(cudaGetLastError(), "launch(verify items)");
+}
+
 int num_sms() {
     static int n = 0;
     if (n == 0) {
@@ -2281,7 +3358,12 @@ int num_sms() {
 
 }  // namespace vfull
 
-size_t verify_full_workspace_bytes(const VerifyArgs& a) { return vfull::recs_bytes(a); }
+// the records, then (top-k off) the row records of the row-streaming path
+size_t verify_full_workspace_bytes(const VerifyArgs& a) {
+    size_t n = align_up(vfull::recs_bytes(a), 256);
+    if (a.top_k == 0) n += (size_t)2 * a.B * a.K * sizeof(vfull::rs::RowRec);
+    return n;
+}
 
 // The item path: pair_kernel where it applies, the generic kernel for the rest, then the
 // per-sequence assembly. With allow_generic false (top-k on: the streaming path serves the
@@ -2310,7 +3392,12 @@ uno_status verify_full_launch(const VerifyArgs& a, void* workspace, cudaStream_t
                                : nullptr;
     uno_status st = UNO_OK;
     int only_redo = 0;
-    if (vfull::launch_pairs(a, p, stream, st)) {
+    if (vfull::rs_applies(a)) {
+        auto* rows = reinterpret_cast<vfull::rs::RowRec*>(static_cast<unsigned char*>(workspace) +
+                                                          align_up(vfull::recs_bytes(a), 256));
+        if ((st = vfull::launch_rs(a, p, rows, stream)) != UNO_OK) return st;
+        only_redo = 1;
+    } else if (vfull::launch_pairs(a, p, stream, st)) {
         if (st != UNO_OK) return st;
         only_redo = 1;
     } else if (!allow_generic) {

@@ -48,7 +48,17 @@ struct Params {
     uint32_t* guesses;   // [rows * lists_per_row] ordered key of the guess each list was taken with
     unsigned char* recs;
     int kcap;
+    unsigned long long* trace;  // UNO_VERIFY_TRACE: phase timestamps of the finish (profiling aid), or NULL
 };
+
+// finish kernel, CTA 0: slot (warp, event)
+__device__ __forceinline__ void fin_mark(const Params& p, int warp, int e) {
+    if (p.trace != nullptr && blockIdx.x == 0 && (threadIdx.x & 31) == 0) {
+        unsigned long long t;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        p.trace[warp * 8 + e] = t;
+    }
+}
 
 template <typename T>
 struct KeyBits;
@@ -854,6 +864,7 @@ __device__ void finish_row(const Params& p, int64_t grow, unsigned char* base, i
     }
     for (int o = 16; o > 0; o >>= 1) G = max(G, __shfl_xor_sync(kFullMask, G, o));
     __syncwarp();
+    fin_mark(p, threadIdx.x >> 5, 1);
     if (n > k) {
         const uint64_t T2 = warp_select(cand, n, k, hist, lane);
         uint64_t mn;
@@ -873,8 +884,10 @@ __device__ void finish_row(const Params& p, int64_t grow, unsigned char* base, i
         const T* row = reinterpret_cast<const T*>(isP ? a.P : a.Q) + ((int64_t)b * a.K + pos) * a.V;
         n = warp_exact_row<T, fallback_cap<KCAP>()>(row, a.V, cand, hist, ws, bound, k, lane);
     }
+    fin_mark(p, threadIdx.x >> 5, 2);
     // cand[0..n): the row's top-k (any order)
     write_survivors(a, cand, n, sb, w, rec_view(p.recs, p.kcap, grow), lane);
+    fin_mark(p, threadIdx.x >> 5, 3);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -891,12 +904,15 @@ finish_seq_kernel(Params p, int fw, size_t smem_bytes) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int b = blockIdx.x;
+    fin_mark(p, warp, 0);
     if (warp < fw) {
         unsigned char* base = smem_raw + (size_t)warp * finish_bytes_per_warp<KCAP>(p.lists_per_row);
         for (int r = warp; r < p.rows_per_seq; r += fw) finish_row<T, KCAP>(p, (int64_t)b * p.rows_per_seq + r, base, lane);
     }
     __syncthreads();  // every record of the sequence is written (and visible to the block)
+    fin_mark(p, warp, 4);
     sequence_verify<kFinWarps>(p.a, p.recs, KCAP, b, p.rows_per_seq, smem_raw, smem_bytes);
+    fin_mark(p, warp, 5);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -1120,7 +1136,7 @@ inline int num_sms() {
 
 struct Layout {
     int kcap, S, rows_per_seq, lists_per_row;
-    size_t off_lists, off_counts, off_guesses, off_recs, total;
+    size_t off_lists, off_counts, off_guesses, off_recs, off_trace, total;
 };
 
 // The streaming kernel a batch takes: UNO_VERIFY_STREAM=warps (one CTA per row segment,
@@ -1167,6 +1183,8 @@ inline Layout layout(const VerifyArgs& a) {
     L.off_guesses = align_up(L.off_counts + rows * L.lists_per_row * 4, 256);
     L.off_recs = align_up(L.off_guesses + rows * L.lists_per_row * 4, 256);
     L.total = align_up(L.off_recs + rows * rec_bytes(L.kcap), 256);
+    L.off_trace = L.total;
+    if (getenv("UNO_VERIFY_TRACE")) L.total += 32 * 8 * 8;
     return L;
 }
 
@@ -1189,6 +1207,7 @@ uno_status launch_t(const VerifyArgs& a, const Layout& L, unsigned char* ws, cud
     p.counts = reinterpret_cast<int32_t*>(ws + L.off_counts);
     p.guesses = reinterpret_cast<uint32_t*>(ws + L.off_guesses);
     p.recs = ws + L.off_recs;
+    p.trace = getenv("UNO_VERIFY_TRACE") ? reinterpret_cast<unsigned long long*>(ws + L.off_trace) : nullptr;
     p.kcap = KCAP;
     const int n_rows = a.B * L.rows_per_seq;
     const StreamKind kind = stream_kind(a);

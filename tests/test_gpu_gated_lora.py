@@ -216,11 +216,14 @@ def test_withheld_adapter_flags_time_out(monkeypatch):
     assert _lib.uno_read_device_status() == _lib.UNO_OK
 
 
-def test_tma_store_epilogue(monkeypatch):
-    """UNO_LORA_EPI=tma: bf16 output tiles staged in shared memory (64-byte swizzle) and
-    written by TMA stores. Ragged M (the stores leave rows past M out), every tile width,
-    several tiles per CTA, and two calls in a row."""
-    monkeypatch.setenv("UNO_LORA_EPI", "tma")
+@pytest.mark.parametrize("epi", ["tma", "rows"])
+def test_output_epilogues(epi, monkeypatch):
+    """Both bf16 epilogues: output tiles staged in shared memory (64-byte swizzle) and written
+    by TMA stores (the default), and per-lane row stores (UNO_LORA_EPI=rows). Ragged M (the
+    stores leave rows past M out), every tile width, several tiles per CTA, and two calls in
+    a row."""
+    if epi == "rows":
+        monkeypatch.setenv("UNO_LORA_EPI", "rows")
     for M, d_in, d_out, r in [(300, 1024, 512, 64), (1000, 768, 1024, 256), (129, 256, 640, 128),
                               (1024, 4096, 4096, 128), (2048, 2560, 640, 64), (5, 128, 64, 24)]:
         w = W.GatedLoraWorkload("t", 23 + M + r, M=M, block=8, rank=r, scale=2.0,
