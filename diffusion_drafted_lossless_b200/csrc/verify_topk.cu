@@ -49,7 +49,15 @@ struct Params {
     unsigned char* recs;
     int kcap;
     unsigned long long* trace;  // UNO_VERIFY_TRACE: phase timestamps of the finish (profiling aid), or NULL
+    uint32_t* seq_done;         // [B] rows finished per sequence (zeroed by the streaming kernel)
 };
+
+// Zero the per-sequence counters of the finish kernel (CTA 0 of the streaming kernel, which
+// runs before it in the stream).
+__device__ __forceinline__ void zero_seq_counters(const Params& p) {
+    if (blockIdx.x == 0)
+        for (int i = threadIdx.x; i < p.a.B; i += blockDim.x) p.seq_done[i] = 0u;
+}
 
 // finish kernel, CTA 0: slot (warp, event)
 __device__ __forceinline__ void fin_mark(const Params& p, int warp, int e) {
@@ -288,6 +296,7 @@ __device__ __noinline__ int stream_full_bf16(const uint4* lp, int cb, int cf, ui
 template <typename T, int KCAP>
 __global__ void __launch_bounds__(kStreamWarps * 32, 3)
 stream_kernel(Params p) {
+    zero_seq_counters(p);
     using Ops = LaneOps<T>;
     constexpr int VEC = Elem<T>::VEC;
     constexpr int CAP = cap_entries<KCAP>();
@@ -556,6 +565,7 @@ __device__ __noinline__ void warp_flush_hits(const uint4* hv, const uint32_t* hi
 template <typename T, int KCAP>
 __global__ void __launch_bounds__(kTmaWarps * 32, kTmaCtasPerSm)
 stream_tma_kernel(Params p, int n_items, uint32_t* status) {
+    zero_seq_counters(p);
     using Ops = LaneOps<T>;
     constexpr int VEC = Elem<T>::VEC;
     constexpr int CAP = tma_cap<KCAP>();
@@ -766,12 +776,13 @@ constexpr size_t finish_bytes_per_warp(int lists_per_row) {
     return (size_t)lists_per_row * KCAP * 8 + 2 * KCAP * 8 + 256 * 4 + 32;
 }
 
-// The row's top-k cand[0..n) (any order) -> its survivor record: sorted by (value desc, id
-// asc) into sb, fp64 softmax weights w relative to the largest value, the top-p cut (the
-// shortest prefix of that order whose mass reaches top_p), and the survivors sorted by id
-// (reusing cand) with their weights and total. One warp.
-__device__ __forceinline__ void write_survivors(const VerifyArgs& a, uint64_t* cand, int n, uint64_t* sb, double* w,
-                                                RecView rec, int lane) {
+// The row's top-k cand[0..n), in ascending id order -> its survivor record. Sorted copy sb
+// (value desc, id asc) gives the fp64 softmax weights relative to the largest value and the
+// top-p cut (the shortest prefix of that order whose mass reaches top_p); the survivors are
+// then taken from cand in id order (values above the cut value, and the first of the ties at
+// it), so no second sort is needed. One warp.
+__device__ __forceinline__ void write_survivors_ids(const VerifyArgs& a, uint64_t* cand, int n, uint64_t* sb, double* w,
+                                                    RecView rec, int lane) {
     const double Td = (double)a.temperature;
     int np = 1;
     while (np < n) np <<= 1;
@@ -800,26 +811,36 @@ __device__ __forceinline__ void write_survivors(const VerifyArgs& a, uint64_t* c
         }
         if (c < 0) c = n;
     }
-    // survivors sb[0..c) sorted by id (key: ~id << 32 | position), reusing cand
-    int np2 = 1;
-    while (np2 < c) np2 <<= 1;
-    uint64_t* ib = cand;
-    for (int j = lane; j < np2; j += 32)
-        ib[j] = j < c ? ((uint64_t)(0xFFFFFFFFu - candidate_id(sb[j])) << 32) | (uint64_t)j : 0ull;
-    __syncwarp();
-    warp_sort_desc(ib, np2, lane);
+    // the cut key and how many of its ties survive (those in sb[0..c))
+    const uint32_t kc = c > 0 ? candidate_key(sb[c - 1]) : 0xFFFFFFFFu;
+    int above = 0;
+    for (int j = lane; j < c; j += 32) above += candidate_key(sb[j]) > kc;
+    above = warp_sum(above);
+    const int tkeep = c - above;
+    int out = 0, ties = 0;
     double z = 0.0;
-    for (int j = lane; j < c; j += 32) {
-        const uint64_t e = ib[j];
-        const double wj = w[(uint32_t)(e & 0xFFFFFFFFu)];
-        rec.id[j] = (int32_t)(0xFFFFFFFFu - (uint32_t)(e >> 32));
-        rec.w[j] = wj;
-        z += wj;
+    for (int b0 = 0; b0 < n; b0 += 32) {
+        const int j = b0 + lane;
+        const uint64_t x = j < n ? cand[j] : 0ull;
+        const uint32_t key = candidate_key(x);
+        const bool tie = j < n && key == kc;
+        const unsigned tb = __ballot_sync(kFullMask, tie);
+        const bool keep = j < n && (key > kc || (tie && ties + __popc(tb & ((1u << lane) - 1u)) < tkeep));
+        const unsigned kb = __ballot_sync(kFullMask, keep);
+        if (keep) {
+            const int o = out + __popc(kb & ((1u << lane) - 1u));
+            const double wj = exp((double)key_float(key) / Td - zmax);  // the same weight as in w
+            rec.id[o] = (int32_t)candidate_id(x);
+            rec.w[o] = wj;
+            z += wj;
+        }
+        out += __popc(kb);
+        ties += __popc(tb);
     }
     z = warp_sum_f64(z);
     if (lane == 0) {
         *rec.Z = z;
-        *rec.n = c;
+        *rec.n = out;
     }
 }
 
@@ -865,18 +886,21 @@ __device__ void finish_row(const Params& p, int64_t grow, unsigned char* base, i
     for (int o = 16; o > 0; o >>= 1) G = max(G, __shfl_xor_sync(kFullMask, G, o));
     __syncwarp();
     fin_mark(p, threadIdx.x >> 5, 1);
+    // the exact top-k in id order: radix selection over the value keys, ties to the lower id
+    const int n_all = n;
     if (n > k) {
-        const uint64_t T2 = warp_select(cand, n, k, hist, lane);
-        uint64_t mn;
-        n = warp_compact(cand, n, T2, lane, &mn);
+        uint32_t tau;
+        int need;
+        warp_select_key<KeyBits<T>::value>(cand, n, k, hist, lane, tau, need);
+        n = warp_compact_key<KeyBits<T>::value>(cand, n, tau, need, lane);
     }
-    // exact iff the k-th value is >= every guess: then every element that can be in the
-    // top-k was >= its warp's guess and so was a candidate
     uint32_t kmin = 0xFFFFFFFFu;
     for (int j = lane; j < n; j += 32) kmin = min(kmin, candidate_key(cand[j]));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) kmin = min(kmin, __shfl_xor_sync(kFullMask, kmin, o));
-    if (n < k || kmin < G) {
+    // exact iff the k-th value is >= every guess: then every element that can be in the
+    // top-k was >= its warp's guess and so was a candidate
+    if (n_all < k || kmin < G) {
         // the streaming guess left fewer than k candidates: redo this row exactly
         const int b = (int)(grow / p.rows_per_seq), r = (int)(grow % p.rows_per_seq);
         const bool isP = r < a.K;
@@ -885,33 +909,54 @@ __device__ void finish_row(const Params& p, int64_t grow, unsigned char* base, i
         n = warp_exact_row<T, fallback_cap<KCAP>()>(row, a.V, cand, hist, ws, bound, k, lane);
     }
     fin_mark(p, threadIdx.x >> 5, 2);
-    // cand[0..n): the row's top-k (any order)
-    write_survivors(a, cand, n, sb, w, rec_view(p.recs, p.kcap, grow), lane);
+    // cand[0..n): the row's top-k in id order
+    write_survivors_ids(a, cand, n, sb, w, rec_view(p.recs, p.kcap, grow), lane);
     fin_mark(p, threadIdx.x >> 5, 3);
 }
 
 // ---------------------------------------------------------------------------------------
-// Kernel 2: one CTA per sequence. Warp w (of the first fw) finishes rows w, w + fw, ... of
-// the sequence: merges their lists into the exact top-k, applies softmax and top-p in fp64
-// and writes each survivor record sorted by token id; then the CTA runs the sequence's
-// draft sampling, acceptance, longest accepted prefix and residual resample.
+// Kernel 2: warp w of CTA c finishes row c fw + w: merges its lists into the exact top-k,
+// applies softmax and top-p in fp64 and writes the survivor record sorted by token id. The
+// CTA then adds its rows to each of their sequences' counters (after a fence); the CTA that
+// completes a sequence runs its draft sampling, acceptance, longest accepted prefix and
+// residual resample. Spreading the rows over many CTAs keeps every SM busy; no CTA waits for
+// another.
 // ---------------------------------------------------------------------------------------
-constexpr int kFinWarps = 32;
+constexpr int kFinWarps = 16;
 
 template <typename T, int KCAP>
 __global__ void __launch_bounds__(kFinWarps * 32)
-finish_seq_kernel(Params p, int fw, size_t smem_bytes) {
+finish_seq_kernel(Params p, int fw, int n_rows, size_t smem_bytes) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
+    __shared__ int s_done[kFinWarps], s_nd;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int b = blockIdx.x;
+    const int rps = p.rows_per_seq;
+    const int64_t r0 = (int64_t)blockIdx.x * fw, r1 = min(r0 + fw, (int64_t)n_rows);
     fin_mark(p, warp, 0);
-    if (warp < fw) {
+    if (warp < fw && r0 + warp < r1) {
         unsigned char* base = smem_raw + (size_t)warp * finish_bytes_per_warp<KCAP>(p.lists_per_row);
-        for (int r = warp; r < p.rows_per_seq; r += fw) finish_row<T, KCAP>(p, (int64_t)b * p.rows_per_seq + r, base, lane);
+        finish_row<T, KCAP>(p, r0 + warp, base, lane);
+        __threadfence();  // the record is visible to the CTA that verifies its sequence
     }
-    __syncthreads();  // every record of the sequence is written (and visible to the block)
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int nd = 0;
+        for (int64_t r = r0; r < r1;) {
+            const int b = (int)(r / rps);
+            const int64_t e = min(r1, (int64_t)(b + 1) * rps);
+            const unsigned add = (unsigned)(e - r);
+            if (atomicAdd(&p.seq_done[b], add) + add == (unsigned)rps) s_done[nd++] = b;
+            r = e;
+        }
+        s_nd = nd;
+        if (nd) __threadfence();
+    }
+    __syncthreads();
     fin_mark(p, warp, 4);
-    sequence_verify<kFinWarps>(p.a, p.recs, KCAP, b, p.rows_per_seq, smem_raw, smem_bytes);
+    for (int j = 0; j < s_nd; ++j) {
+        sequence_verify<kFinWarps>(p.a, p.recs, KCAP, s_done[j], rps, smem_raw, smem_bytes);
+        __syncthreads();
+    }
     fin_mark(p, warp, 5);
 }
 
@@ -958,6 +1003,7 @@ __device__ __forceinline__ __nv_bfloat162 bf2_max4(const uint4& v) {
 template <int KCAP>
 __global__ void __launch_bounds__(kRowsWarps * 32, kRowsCtasPerSm)
 stream_rows_kernel(Params p, int n_items) {
+    zero_seq_counters(p);
     constexpr int CAP = rows_cap<KCAP>();
     constexpr int CH = 256;  // elements per chunk
     extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -1136,7 +1182,7 @@ inline int num_sms() {
 
 struct Layout {
     int kcap, S, rows_per_seq, lists_per_row;
-    size_t off_lists, off_counts, off_guesses, off_recs, off_trace, total;
+    size_t off_lists, off_counts, off_guesses, off_recs, off_seq, off_trace, total;
 };
 
 // The streaming kernel a batch takes: UNO_VERIFY_STREAM=warps (one CTA per row segment,
@@ -1182,7 +1228,8 @@ inline Layout layout(const VerifyArgs& a) {
     L.off_counts = align_up(rows * L.lists_per_row * L.kcap * 8, 256);
     L.off_guesses = align_up(L.off_counts + rows * L.lists_per_row * 4, 256);
     L.off_recs = align_up(L.off_guesses + rows * L.lists_per_row * 4, 256);
-    L.total = align_up(L.off_recs + rows * rec_bytes(L.kcap), 256);
+    L.off_seq = align_up(L.off_recs + rows * rec_bytes(L.kcap), 256);
+    L.total = align_up(L.off_seq + (size_t)a.B * 4, 256);
     L.off_trace = L.total;
     if (getenv("UNO_VERIFY_TRACE")) L.total += 32 * 8 * 8;
     return L;
@@ -1207,6 +1254,7 @@ uno_status launch_t(const VerifyArgs& a, const Layout& L, unsigned char* ws, cud
     p.counts = reinterpret_cast<int32_t*>(ws + L.off_counts);
     p.guesses = reinterpret_cast<uint32_t*>(ws + L.off_guesses);
     p.recs = ws + L.off_recs;
+    p.seq_done = reinterpret_cast<uint32_t*>(ws + L.off_seq);
     p.trace = getenv("UNO_VERIFY_TRACE") ? reinterpret_cast<unsigned long long*>(ws + L.off_trace) : nullptr;
     p.kcap = KCAP;
     const int n_rows = a.B * L.rows_per_seq;
@@ -1249,7 +1297,7 @@ uno_status launch_t(const VerifyArgs& a, const Layout& L, unsigned char* ws, cud
         stream_kernel<T, KCAP><<<(unsigned)(n_rows * L.S), kStreamWarps * 32, smem1, stream>>>(p);
     }
     if ((s = check_cuda(cudaGetLastError(), "launch(verify stream)")) != UNO_OK) return s;
-    finish_seq_kernel<T, KCAP><<<(unsigned)a.B, kFinWarps * 32, smem2, stream>>>(p, fw, smem2);
+    finish_seq_kernel<T, KCAP><<<(unsigned)((n_rows + fw - 1) / fw), kFinWarps * 32, smem2, stream>>>(p, fw, n_rows, smem2);
     return check_cuda(cudaGetLastError(), "launch(verify finish)");
 }
 
