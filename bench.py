@@ -43,7 +43,7 @@ UNIT = "rows/s"
 WORKLOAD = "uno_step_b64_k16_v151936_qwen3_8b"
 LINEARS = W.QWEN3_8B
 VERIFY = W.SERVING_VERIFY
-LAUNCHES_PER_STEP = 7 + 3 + 2  # 7 projections (one kernel each) + verify (cluster items, generic items, assembly) + TV (mask, rows)
+LAUNCHES_PER_STEP = 7 + 2 + 2  # 7 projections (one kernel each) + verify (row streaming, finish) + TV (mask, rows)
 
 
 def peaks():
@@ -502,33 +502,27 @@ def run_uno(args):
     # the headline: B * K / t_verify (the verify's mean time inside the timed steps)
     value = whole_job_rate(rows, world, ph["block_verify"])
     gemm_fl = sum(gemm_flops(L["shape"], LINEARS.M, LINEARS.rank, st.n_gated) for L in st.lin)
-    # the dominant kernel: the TV kernel is one launch per step (plus a 1-block mask count);
-    # the linears are 7 launches (one per projection), the verify 3
-    per_launch = {"gated_lora_linears": ph["gated_lora_linears"] / 7, "block_verify": ph["block_verify"],
-                  "tv_loss": ph["tv_loss"]}
-    dominant = max(per_launch, key=per_launch.get)
-    if dominant == "gated_lora_linears":
-        ach = gemm_fl / (ph[dominant] * 1e-3) / 1e12
-        roof = {"kernel": "gated_lora_linear (mean of the 7 projections)", "bound": "tensor", "achieved": ach,
-                "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops"],
-                "traffic": None, "algorithmic_per_launch": gemm_fl / 7}
-    elif dominant == "block_verify":
-        ach = verify_bytes(v) / (ph[dominant] * 1e-3) / 1e9
-        roof = {"kernel": "block_verify", "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": ach / pk["hbm_gbs"], "traffic": None, "algorithmic_per_launch": verify_bytes(v)}
-    else:
-        ach = tv_bytes(rows, v.V) / (ph[dominant] * 1e-3) / 1e9
-        roof = {"kernel": "tv_loss", "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": ach / pk["hbm_gbs"], "traffic": profiled_traffic("tv_loss"),
-                "algorithmic_per_launch": tv_bytes(rows, v.V)}
+    # The roofline of the metric's kernel: the value is B * K over the verify's time, and the
+    # verify is the streaming kernel (about 80% of it) and the per-sequence finish kernel, both
+    # inside one library call; its algorithmic bytes are the logit rows it must read once.
+    # The other phases' fractions (the projections against the tensor peak, the TV loss
+    # against HBM) are in "phases".
+    ach = verify_bytes(v) / (ph["block_verify"] * 1e-3) / 1e9
+    roof = {"kernel": "block_verify (row-streaming top-k kernel + per-sequence finish kernel, one call)",
+            "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": ach / pk["hbm_gbs"],
+            "traffic": profiled_traffic("block_verify"), "algorithmic_per_launch": verify_bytes(v)}
     roof["peak_source"] = pk["source"]
+    gl_tf = gemm_fl / (ph["gated_lora_linears"] * 1e-3) / 1e12
+    vb_gbs = verify_bytes(v) / (ph["block_verify"] * 1e-3) / 1e9
+    tv_gbs = tv_bytes(rows, v.V) / (ph["tv_loss"] * 1e-3) / 1e9
     phases = {
-        "gated_lora_linears": {"ms": ph["gated_lora_linears"],
-                               "tflops": gemm_fl / (ph["gated_lora_linears"] * 1e-3) / 1e12},
-        "block_verify": {"ms": ph["block_verify"],
-                         "gbs": verify_bytes(v) / (ph["block_verify"] * 1e-3) / 1e9,
+        "gated_lora_linears": {"ms": ph["gated_lora_linears"], "tflops": gl_tf,
+                               "frac": gl_tf / (pk["bf16_tflops_sustained"] or pk["bf16_tflops"]),
+                               "peak": "bf16 sustained (the projections run back to back inside the step)"},
+        "block_verify": {"ms": ph["block_verify"], "gbs": vb_gbs, "frac": vb_gbs / pk["hbm_gbs"],
                          "rows_per_s": rows / (ph["block_verify"] * 1e-3)},
-        "tv_loss": {"ms": ph["tv_loss"], "gbs": tv_bytes(rows, v.V) / (ph["tv_loss"] * 1e-3) / 1e9},
+        "tv_loss": {"ms": ph["tv_loss"], "gbs": tv_gbs, "frac": tv_gbs / pk["hbm_gbs"],
+                    "traffic": profiled_traffic("tv_loss")},
     }
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
