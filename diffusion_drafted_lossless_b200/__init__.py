@@ -7,6 +7,7 @@ stream); `workloads` holds the seeded synthetic inputs.
 """
 from ._lib import (  # noqa: F401
     UNO_BF16, UNO_F32, UNO_OK, UnoError, load, uno_block_noise, uno_block_verify, uno_block_verify_workspace_size,
+    uno_block_verify_min_workspace_size,
     uno_gated_lora_linear, uno_gated_lora_linear_workspace_size, uno_read_device_status, uno_tv_loss,
     uno_tv_loss_workspace_size, uno_version,
 )

@@ -23,7 +23,8 @@ UNO_BF16, UNO_F32 = 0, 1
 EXPORTED = (
     "uno_status_string", "uno_last_error_string", "uno_version", "uno_read_device_status",
     "uno_gated_lora_linear_workspace_size", "uno_gated_lora_linear",
-    "uno_block_verify_workspace_size", "uno_block_verify", "uno_block_verify_noalloc",
+    "uno_block_verify_workspace_size", "uno_block_verify_min_workspace_size", "uno_block_verify",
+    "uno_block_verify_noalloc",
     "uno_tv_loss_workspace_size", "uno_tv_loss", "uno_block_noise",
 )
 
@@ -59,6 +60,8 @@ def load(path: str | os.PathLike | None = None) -> ctypes.CDLL:
                                           _vp, _vp, _sz, _vp]
     lib.uno_block_verify_workspace_size.restype = _sz
     lib.uno_block_verify_workspace_size.argtypes = [_i32, _i32, _i32, _i32, _f32, ctypes.c_int]
+    lib.uno_block_verify_min_workspace_size.restype = _sz
+    lib.uno_block_verify_min_workspace_size.argtypes = [_i32, _i32, _i32, _i32, _f32, ctypes.c_int]
     lib.uno_block_verify.argtypes = [_vp, _vp, ctypes.c_int, _i32, _i32, _i32, _f32, _i32, _f32,
                                      _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
     lib.uno_block_verify_noalloc.argtypes = [_vp, _vp, ctypes.c_int, _i32, _i32, _i32, _f32, _i32, _f32,
@@ -147,6 +150,10 @@ def uno_gated_lora_linear(x, w0, lora_a, lora_b, row_gate, scale, y, workspace=N
 # ---------------------------------------------------------------------------------------
 def uno_block_verify_workspace_size(B, K, V, top_k, top_p, dtype=UNO_BF16) -> int:
     return int(load().uno_block_verify_workspace_size(B, K, V, top_k, top_p, dtype))
+
+
+def uno_block_verify_min_workspace_size(B, K, V, top_k, top_p, dtype=UNO_BF16) -> int:
+    return int(load().uno_block_verify_min_workspace_size(B, K, V, top_k, top_p, dtype))
 
 
 def uno_block_verify(verifier_logits, drafter_logits, temperature, top_k, top_p, uniforms,

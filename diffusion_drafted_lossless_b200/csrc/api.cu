@@ -161,7 +161,14 @@ static uno_status verify_args(VerifyArgs& a, const void* P, const void* Q, uno_d
 size_t uno_block_verify_workspace_size(int32_t B, int32_t K, int32_t V, int32_t top_k, float top_p, uno_dtype dtype) {
     VerifyArgs a;
     if (verify_args(a, nullptr, nullptr, dtype, B, K, V, 1.0f, top_k, top_p) != UNO_OK) return 0;
-    return verify_workspace_bytes(a);
+    return verify_workspace_bytes(a, false);
+}
+
+size_t uno_block_verify_min_workspace_size(int32_t B, int32_t K, int32_t V, int32_t top_k, float top_p,
+                                           uno_dtype dtype) {
+    VerifyArgs a;
+    if (verify_args(a, nullptr, nullptr, dtype, B, K, V, 1.0f, top_k, top_p) != UNO_OK) return 0;
+    return verify_workspace_bytes(a, true);
 }
 
 uno_status uno_block_verify(const void* verifier_logits, const void* drafter_logits, uno_dtype dtype, int32_t B,
@@ -189,7 +196,7 @@ uno_status uno_block_verify(const void* verifier_logits, const void* drafter_log
     a.out_p = out_p_tok;
     a.out_q = out_q_tok;
     a.out_tv = out_tv;
-    s = check_workspace(workspace, workspace_bytes, verify_workspace_bytes(a));
+    s = check_workspace(workspace, workspace_bytes, verify_workspace_bytes(a, true));
     if (s != UNO_OK) return s;
     return verify_launch(a, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }

@@ -55,7 +55,7 @@ extern "C" uno_status uno_block_verify_noalloc(const void* verifier_logits, cons
                                                int32_t* out_tokens, int32_t* out_count, int32_t* out_next_token,
                                                float* out_p_tok, float* out_q_tok, float* out_tv,
                                                uno_stream_t stream) {
-    const size_t need = uno_block_verify_workspace_size(B, K, V, top_k, top_p, dtype);
+    const size_t need = uno_block_verify_min_workspace_size(B, K, V, top_k, top_p, dtype);
     if (need > (size_t)UNO_NOALLOC_SCRATCH_BYTES)
         return uno::set_error(UNO_ERR_UNSUPPORTED,
                               "uno_block_verify_noalloc: this batch needs %zu bytes of scratch; the fixed array "

@@ -24,10 +24,11 @@ struct VerifyArgs {
     float* out_tv;
 };
 
-// Bytes of workspace the verify needs for these arguments (0 if B == 0).
-size_t verify_workspace_bytes(const VerifyArgs& a);
+// Bytes of workspace the verify uses for these arguments (0 if B == 0): the fastest path's,
+// or (minimal) the least it accepts.
+size_t verify_workspace_bytes(const VerifyArgs& a, bool minimal);
 
-// Enqueue the verify on `stream`; the workspace is at least verify_workspace_bytes(a).
+// Enqueue the verify on `stream`; the workspace is at least verify_workspace_bytes(a, true).
 uno_status verify_launch(const VerifyArgs& a, void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 }  // namespace uno

@@ -293,8 +293,8 @@ __device__ void sequence_verify(const VerifyArgs& a, unsigned char* recs, int kc
 
 size_t verify_topk_workspace_bytes(const VerifyArgs& a);
 uno_status verify_topk_launch(const VerifyArgs& a, void* workspace, cudaStream_t stream);
-size_t verify_full_workspace_bytes(const VerifyArgs& a);
-uno_status verify_full_launch(const VerifyArgs& a, void* workspace, cudaStream_t stream, bool allow_generic,
-                              bool* taken);
+size_t verify_full_workspace_bytes(const VerifyArgs& a, bool with_lists);
+uno_status verify_full_launch(const VerifyArgs& a, void* workspace, size_t workspace_bytes, cudaStream_t stream,
+                              bool allow_generic, bool* taken);
 
 }  // namespace uno

@@ -2028,13 +2028,16 @@ namespace rs {
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kCtasPerSm = 2;         // item pass
-constexpr int kRowCtasPerSm = 3;      // row pass
+constexpr int kRowCtasPerSm = 3;      // row pass (UNO_VERIFY_ROW_CTAS=2: two, with more registers each)
 constexpr int kGroup = 4;             // chunks per group of the row pass (a chunk: 32 lanes x 8 elements)
 constexpr int kCh = 256;              // elements per chunk
 constexpr int kWin = 320;             // counted keys: the anchor and the kWin - 1 below it
 constexpr int kAbove = 96;            // the anchor: this many keys above the sampled maximum
 constexpr int kLutMax = 512;          // tabulated survivor weights per row
 constexpr int kMagWin = 2048;         // recount: counted magnitudes (both signs) from the largest down
+constexpr int kListCap = 4096;        // candidate list entries per warp run (beyond: the row has no list)
+constexpr int kStage = 512;           // staged entries per warp before a list flush
+constexpr int kMaxListV = 196608;     // list path: V up to this (the item pass's bitmap size)
 constexpr double kEx2Err = 0x1p-22;   // bound on ex2.approx.ftz.f32's relative error (2^-22.7 measured)
 constexpr double kU = 0x1p-24;        // fp32 unit roundoff
 constexpr double kLn2 = 0.6931471805599453;
@@ -2050,6 +2053,11 @@ struct RowRec {
     int tie_before[kWarps];   // tokens at the cut value before each warp's run
     int lut_n;                // lut[j]: weight of key kM - j, for j < lut_n (0 where absent)
     int state;                // kDone, or kRedo (the item goes to the generic kernel)
+    int list_ok;              // the candidate lists hold every survivor (window path, no overflow)
+    uint32_t A15;             // the window's anchor (bf16 bits): an entry's window bin is A15 - its bits
+    int dcut;                 // the cut value's window bin (list path)
+    int list_n[kWarps];       // entries in each warp run's list
+    int theta;                // list path: a token at the cut value survives when its id is below theta
     double lut[kLutMax];
 };
 
@@ -2118,6 +2126,15 @@ __device__ __forceinline__ void rs_mark(const Params& p, int kernel, int j, int 
         p.trace[((kernel * 2) * 32 + j) * 16 + e] = t;
     }
 }
+// (kernel 0: rows, 1: items, 2: list items; the end time of each CTA at 6144 + CTA for rows,
+// 7168 + CTA for list items)
+__device__ __forceinline__ void rs_end(const Params& p, int base) {
+    if (p.trace != nullptr && threadIdx.x == 0 && blockIdx.x < 1024) {
+        unsigned long long t;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        p.trace[base + blockIdx.x] = t;
+    }
+}
 __device__ __forceinline__ void rs_count(const Params& p, int slot) {
     if (p.trace != nullptr && threadIdx.x == 0) atomicAdd(&p.trace[(15 * 2 * 32) * 16 + slot], 1ull);
 }
@@ -2138,10 +2155,13 @@ struct RowShared {
     uint32_t hc[kWin];           // their sum
     double wd[kWin];             // weight of window key d (where present), relative to zmax
     uint32_t hr[2 * kMagWin];    // recount: counts of (sign, magnitude largest - d)
+    uint32_t stage[kWarps][kStage];  // counted elements ((id - c0 256) << 16 | bits) on their way to the list
     float fmax[kWarps];
     double dz[kWarps], db[kWarps], red[kWarps];
     int ties[kWarps];
-    int d_cut, tie_t, ok;
+    int ln[kWarps];              // entries each warp's list has taken
+    int next[2];                 // the next row (alternate rows use alternate slots)
+    int d_cut, tie_t, ok, theta;
     double S;
 };
 
@@ -2195,7 +2215,53 @@ __device__ bool warp_cut(C cnt, W w, int n, double target, int lane, int& dcut, 
     return true;
 }
 
-__global__ void __launch_bounds__(kThreads, kRowCtasPerSm) row_kernel(Params p, RowRec* rows) {
+constexpr int kLT = 128;  // entries per list tile: lane l holds entries 4l .. 4l + 3 (one 16-byte load)
+constexpr int kLB = 8;    // tiles per batch: the 16-byte loads each lane has in flight
+
+// The id of the kk-th entry (0-based, id order) of a warp's list of n entries whose bits are
+// hcut (entries: (id - id0) << 16 | bits); INT_MAX if there are not that many.
+__device__ int find_tie(const uint32_t* list, int n, uint32_t hcut, int kk, int id0, int lane) {
+    int cnt = 0;
+    for (int t0 = 0; t0 < n; t0 += kLT * kLB) {
+        uint4 v[kLB];
+#pragma unroll
+        for (int u = 0; u < kLB; ++u) {
+            const int j = t0 + u * kLT + lane * 4;
+            v[u] = j < n ? __ldcg(reinterpret_cast<const uint4*>(list + j)) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < kLB; ++u) {
+            const int j = t0 + u * kLT + lane * 4;
+            const uint32_t e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+            uint32_t tie = 0u;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) tie |= (uint32_t)(j + k < n && (e[k] & 0xFFFFu) == hcut) << k;
+            const int nt = __popc(tie);
+            const int tot = (int)__reduce_add_sync(kFullMask, (unsigned)nt);
+            if (cnt + tot > kk) {  // the same in every lane
+                const int incl = warp_inclusive_scan(nt, lane);
+                const int r = kk - cnt;  // its rank among this tile's ties
+                const bool mine = incl > r && incl - nt <= r;
+                int id = 0;
+                if (mine) {
+                    int q = r - (incl - nt);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        if ((tie >> k) & 1u) {
+                            if (q == 0) id = id0 + (int)(e[k] >> 16);
+                            --q;
+                        }
+                }
+                return __shfl_sync(kFullMask, id, __ffs(__ballot_sync(kFullMask, mine)) - 1);
+            }
+            cnt += tot;
+        }
+    }
+    return INT_MAX;
+}
+
+template <int CPS>
+__global__ void __launch_bounds__(kThreads, CPS) row_kernel(Params p, RowRec* rows, uint32_t* lists, uint32_t* ctr) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     RowShared& sh = *reinterpret_cast<RowShared*>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -2207,8 +2273,15 @@ __global__ void __launch_bounds__(kThreads, kRowCtasPerSm) row_kernel(Params p, 
     const float cT = (float)(1.4426950408889634 / T);  // log2(e) / T
 
     int jr = 0;  // rows this CTA has taken (trace)
-    for (int r = blockIdx.x; r < n_rows; r += gridDim.x) {
-        if (!row_needed(p, r)) continue;  // the same in every thread
+    // rows are taken from a counter (after each CTA's first, blockIdx.x): a row that needs the
+    // recount holds up only the CTA that has it
+    int par = 0;
+    for (int r = blockIdx.x; r < n_rows; r = sh.next[par], par ^= 1) {
+        if (tid == 0) sh.next[par] = gridDim.x + (int)atomicAdd(ctr, 1u);  // read after this row's last barrier
+        if (!row_needed(p, r)) {  // the same in every thread
+            __syncthreads();
+            continue;
+        }
         const uint4* r4 = row_ptr(p, r);
         RowRec& out = rows[r];
         const int jm = jr++;
@@ -2251,10 +2324,26 @@ __global__ void __launch_bounds__(kThreads, kRowCtasPerSm) row_kernel(Params p, 
 
         rs_mark(p, 0, jm, 1);
         // ---- stream the row ----
+        // Every counted element (x >= F) goes, in id order, to the warp's stage as
+        // (id - c0 256) << 16 | bits; each flush of the stage counts its entries' window bins
+        // and appends them to the warp's candidate list.
         __nv_bfloat162 mx2 = __floats2bfloat162_rn(-INFINITY, -INFINITY);
         double zr = 0.0;  // rest weights exp((x - F) / T)
         float zb = 0.f;   // rest weights times |their ex2 argument| (for the error bound)
         uint32_t* hwp = sh.hw[warp];
+        uint32_t* stg = sh.stage[warp];
+        uint32_t* gl = lists ? lists + ((int64_t)r * kWarps + warp) * kListCap : nullptr;
+        int lq = 0, gn = 0;  // staged entries, entries this warp's list has taken (both warp-uniform)
+        auto flush = [&](int n) {  // the first n staged entries (n <= 256)
+            __syncwarp();
+            for (int j = lane; j < n; j += 32) {
+                const uint32_t s = stg[j];
+                atomicAdd(&hwp[min(A15 - (s & 0xFFFFu), (uint32_t)kWin)], 1u);  // above the anchor: last slot
+                if (gl != nullptr && gn + n <= kListCap) gl[gn + j] = s;
+            }
+            gn += n;
+            __syncwarp();
+        };
         int c = c0;
         while (true) {
             const bool more = c + kGroup < c1;
@@ -2266,33 +2355,57 @@ __global__ void __launch_bounds__(kThreads, kRowCtasPerSm) row_kernel(Params p, 
             }
 #pragma unroll
             for (int u = 0; u < kGroup; ++u) {
-                if (!valid(c + u)) continue;
+                if (c + u >= c1) continue;  // the same in every lane
+                const bool ok = valid(c + u);
                 const uint32_t w4[4] = {cur[u].x, cur[u].y, cur[u].z, cur[u].w};
-                f2 acc = pk(0.f, 0.f);
+                uint32_t cm = 0u;  // this lane's counted elements (bit e: element e of its 8)
+                if (ok) {
+                    f2 acc = pk(0.f, 0.f);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint32_t wq = w4[q];
-                    const uint32_t m = __hge2_mask(bf2(wq), F2);  // x >= F: counted (0xFFFF per half)
-                    mx2 = __hmax2(mx2, bf2(wq));
-                    const f2 a = mul2(sub2(widen(wq), Ff), C2);
-                    const bool in0 = (m & 0xFFFFu) != 0u, in1 = (m >> 16) != 0u;
-                    const float x0 = ex2f(lo_of(a)), x1 = ex2f(hi_of(a));
-                    const float e0 = in0 ? 0.f : x0, e1 = in1 ? 0.f : x1;
-                    // counted values above the anchor land in the last slot (and M shows them)
-                    const uint32_t d0 = min(A15 - (wq & 0xFFFFu), (uint32_t)kWin);
-                    const uint32_t d1 = min(A15 - (wq >> 16), (uint32_t)kWin);
-                    if (in0) atomicAdd(&hwp[d0], 1u);
-                    if (in1) atomicAdd(&hwp[d1], 1u);
-                    acc = add2(acc, pk(e0, e1));
-                    zb = fmaf(e0, fabsf(lo_of(a)), zb);
-                    zb = fmaf(e1, fabsf(hi_of(a)), zb);
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t wq = w4[q];
+                        const uint32_t m = __hge2_mask(bf2(wq), F2);  // x >= F: counted (0xFFFF per half)
+                        mx2 = __hmax2(mx2, bf2(wq));
+                        const f2 a = mul2(sub2(widen(wq), Ff), C2);
+                        const bool in0 = (m & 0xFFFFu) != 0u, in1 = (m >> 16) != 0u;
+                        const float x0 = ex2f(lo_of(a)), x1 = ex2f(hi_of(a));
+                        const float e0 = in0 ? 0.f : x0, e1 = in1 ? 0.f : x1;
+                        cm |= ((m & 1u) | ((m >> 15) & 2u)) << (2 * q);
+                        acc = add2(acc, pk(e0, e1));
+                        zb = fmaf(e0, fabsf(lo_of(a)), zb);
+                        zb = fmaf(e1, fabsf(hi_of(a)), zb);
+                    }
+                    zr += (double)lo_of(acc) + (double)hi_of(acc);
                 }
-                zr += (double)lo_of(acc) + (double)hi_of(acc);
+                // this chunk's counted elements, in id order (lane, element), to the stage
+                const int cnt = __popc(cm);
+                const int incl = warp_inclusive_scan(cnt, lane);
+                const int tot = __shfl_sync(kFullMask, incl, 31);
+                if (tot) {
+                    int pos = lq + incl - cnt;
+                    const uint32_t base = (uint32_t)((c + u - c0) * kCh + lane * 8) << 16;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        if ((cm >> e) & 1u)
+                            stg[pos++] = __byte_perm(w4[e >> 1], base + ((uint32_t)e << 16), (e & 1) ? 0x7632u : 0x7610u);
+                    lq += tot;
+                    if (lq >= 256) {  // (lq < 512: the rest moves from [256, lq) to the front)
+                        flush(256);
+                        for (int j = lane; j < lq - 256; j += 32) stg[j] = stg[256 + j];
+                        __syncwarp();
+                        lq -= 256;
+                    }
+                }
             }
             if (!more) break;
 #pragma unroll
             for (int u = 0; u < kGroup; ++u) cur[u] = nxt[u];
             c += kGroup;
+        }
+        if (lq > 0) flush(lq);
+        if (lane == 0) {
+            out.list_n[warp] = gn;
+            sh.ln[warp] = gn;
         }
         rs_mark(p, 0, jm, 2);
         {
@@ -2376,6 +2489,34 @@ __global__ void __launch_bounds__(kThreads, kRowCtasPerSm) row_kernel(Params p, 
                 }
                 out.lut_n = lut_n;
                 out.state = kDone;
+                out.A15 = A15;
+                out.dcut = dcut;
+            }
+            // The lists are complete when every warp's fits. Then the tie at the cut of rank
+            // tie_t (id order), the first that does not survive, is found in its warp's list:
+            // a tie survives exactly when its id is below that tie's id (theta).
+            int lok = lists != nullptr && V <= kMaxListV;
+            for (int w = 0; w < kWarps; ++w) lok &= sh.ln[w] <= kListCap;
+            if (lok) {
+                const int tt = sh.tie_t;
+                int wb = -1, kk = 0, before = 0;
+                for (int w = 0; w < kWarps; ++w) {
+                    const int cw = (int)sh.hw[w][dcut];
+                    if (wb < 0 && tt < before + cw) {
+                        wb = w;
+                        kk = tt - before;
+                    }
+                    before += cw;
+                }
+                if (warp == (wb < 0 ? 0 : wb)) {
+                    const int th = wb < 0 ? INT_MAX : find_tie(gl, gn, A15 - (uint32_t)dcut, kk, c0 * kCh, lane);
+                    if (lane == 0) sh.theta = th;
+                }
+            }
+            __syncthreads();
+            if (tid == 0) {
+                out.list_ok = lok;
+                out.theta = lok ? sh.theta : INT_MAX;
             }
             __syncthreads();  // the window counts are reused by the next row
             continue;
@@ -2383,6 +2524,7 @@ __global__ void __launch_bounds__(kThreads, kRowCtasPerSm) row_kernel(Params p, 
 
         // ---- exact recount ----
         rs_count(p, 0);
+        if (tid == 0) out.list_ok = 0;
         if (!finite_max) {
             if (tid == 0) out.state = kRedo;
             __syncthreads();
@@ -2530,6 +2672,7 @@ __global__ void __launch_bounds__(kThreads, kRowCtasPerSm) row_kernel(Params p, 
         }
         __syncthreads();
     }
+    rs_end(p, 6144);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -2665,6 +2808,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) item_kernel_rs(Params p,
             if (tid == 0) p.recs[item].state = kRedo;
             continue;
         }
+        if (rp.list_ok && (!two || rq.list_ok)) continue;  // item_list_kernel decides it
         RowView P, Q;
         auto view = [&](const RowRec& rr, int slot, RowView& R) {
             R.zmax = rr.zmax;
@@ -3026,6 +3170,374 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) item_kernel_rs(Params p,
     }
 }
 
+
+// ---------------------------------------------------------------------------------------
+// item pass over the candidate lists (items whose rows both took the window path)
+// ---------------------------------------------------------------------------------------
+// The survivors of a row are the entries of its lists with a bin below the cut bin, and the
+// first tie_t of those at it (in id order: the lists are in id order, warp run by warp run).
+// Warp w works on list segment w of both rows, which covers the same ids [c0 256, c1 256)
+// in both: the drafter's survivors go to a bitmap of their ids and a compact array of their
+// bins (id order), which the verifier's survivors look up to weigh max(0, p - q).
+constexpr int kBitWords = kMaxListV / 32;
+struct ListShared {
+    double lut[2][kLutMax];
+    uint32_t qbits[kBitWords];               // drafter survivors by id
+    uint16_t wpre[kBitWords];                // drafter survivors before each bitmap word (within its warp run)
+    uint16_t qd[kWarps][kListCap];           // drafter survivors' bins, id order, per warp run
+    double ws[kWarps][3];                    // per warp run: draw-row mass, verifier mass, residual mass
+    double sel_c;
+    int sel_w, tok_found, last_mode;
+    int next[2];  // the next item (alternate items use alternate slots)
+};
+
+// A list entry is (id - id0) << 16 | bits for a counted element of the warp run starting at
+// token id0; its window bin is A15 - bits. It survives when its bin is below the cut bin, or
+// at it with an id below theta.
+struct ListRow {
+    const uint32_t* list;   // this warp's segment
+    int n, dcut, theta, d0, a15, id0;
+    double iS, S;
+    const double* lut;
+    __device__ __forceinline__ int bin(uint32_t e) const { return a15 - (int)(e & 0xFFFFu); }
+    __device__ __forceinline__ int id(uint32_t e) const { return id0 + (int)(e >> 16); }
+    __device__ __forceinline__ bool survives(uint32_t e) const {
+        const int d = bin(e);
+        return d < dcut || (d == dcut && id(e) < theta);
+    }
+    __device__ __forceinline__ double weight(uint32_t e) const { return lut[bin(e) - d0]; }
+};
+
+// a batch of kLB tiles of a segment from entry t0 (entries past n read as 0; the segment's
+// kListCap entries are all in the workspace)
+__device__ __forceinline__ void load_batch(const ListRow& R, int t0, uint4 (&v)[kLB], int lane) {
+#pragma unroll
+    for (int u = 0; u < kLB; ++u) {
+        const int j = t0 + u * kLT + lane * 4;
+        v[u] = j < R.n ? __ldcg(reinterpret_cast<const uint4*>(R.list + j)) : make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+
+// the survivors among a lane's 4 entries of a tile (bit k: entry k); j: the first one's index
+__device__ __forceinline__ uint32_t tile_keep(const uint4& v, int j, const ListRow& R, uint32_t (&e)[4]) {
+    e[0] = v.x;
+    e[1] = v.y;
+    e[2] = v.z;
+    e[3] = v.w;
+    uint32_t keep = 0u;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) keep |= (uint32_t)(j + k < R.n && R.survives(e[k])) << k;
+    return keep;
+}
+
+__global__ void __launch_bounds__(kThreads, 2) item_list_kernel(Params p, const RowRec* rows, const uint32_t* lists,
+                                                                 uint32_t* ctr) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    ListShared& sh = *reinterpret_cast<ListShared*>(smem_raw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int V = p.V;
+    int c0, c1;
+    warp_run(V, warp, c0, c1);
+    const int w0 = c0 * (kCh / 32), w1 = c1 * (kCh / 32);  // this warp run's bitmap words
+    const int n_items = p.B * p.K;
+    int jr = 0;  // items this CTA has taken (trace)
+
+    // items are taken from a counter (after each CTA's first, blockIdx.x)
+    int par = 0;
+    for (int item = blockIdx.x; item < n_items; item = sh.next[par], par ^= 1) {
+        if (tid == 0) sh.next[par] = gridDim.x + (int)atomicAdd(ctr, 1u);  // read after this item's last barrier
+        const int b = item / p.K, i = item % p.K;
+        const bool two = i > 0;
+        const RowRec& rp = rows[item];
+        const RowRec& rq = rows[n_items + item];
+        // trivial items: the row-reading pass writes them; items without lists: item_kernel_rs
+        if (trivial_item(p, b, i) || rp.state != kDone || !rp.list_ok ||
+            (two && (rq.state != kDone || !rq.list_ok))) {
+            __syncthreads();
+            continue;
+        }
+        __syncthreads();  // the previous item is done with the shared tables
+        const int jm = jr++;
+        rs_mark(p, 2, jm, 0);
+        auto view = [&](const RowRec& rr, int r, int slot) {
+            ListRow R;
+            R.list = lists + ((int64_t)r * kWarps + warp) * kListCap;
+            R.n = rr.list_n[warp];
+            R.dcut = rr.dcut;
+            R.theta = rr.theta;
+            R.d0 = (int)(rr.A15 - (obits(rr.kM) & 0x7FFFu));
+            R.a15 = (int)rr.A15;
+            R.id0 = c0 * kCh;
+            R.S = rr.S;
+            R.iS = 1.0 / rr.S;
+            R.lut = sh.lut[slot];
+            for (int j = tid; j < rr.lut_n; j += kThreads) sh.lut[slot][j] = rr.lut[j];
+            return R;
+        };
+        const ListRow P = view(rp, item, 0);
+        const ListRow Q = two ? view(rq, n_items + item, 1) : P;
+        for (int j = w0 + lane; j < w1; j += 32) sh.qbits[j] = 0u;
+        __syncthreads();
+
+        // ---- the drafter's survivors: bitmap, bins in id order, mass ----
+        double sq = 0.0;
+        if (two) {
+            int nq = 0;
+            double sqk[4] = {0.0, 0.0, 0.0, 0.0};
+            for (int t0 = 0; t0 < Q.n; t0 += kLT * kLB) {
+                uint4 v[kLB];
+                load_batch(Q, t0, v, lane);
+#pragma unroll
+                for (int u = 0; u < kLB; ++u) {
+                    if (t0 + u * kLT >= Q.n) break;  // the same in every lane
+                    uint32_t e[4];
+                    const uint32_t keep = tile_keep(v[u], t0 + u * kLT + lane * 4, Q, e);
+                    const int c = __popc(keep);
+                    const int incl = warp_inclusive_scan(c, lane);
+                    int pos = nq + incl - c;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const bool s = (keep >> k) & 1u;
+                        const uint32_t id = (uint32_t)Q.id(e[k]);
+                        const int d = Q.bin(e[k]);
+                        if (s) {
+                            atomicOr(&sh.qbits[id >> 5], 1u << (id & 31u));
+                            sh.qd[warp][pos] = (uint16_t)d;
+                        }
+                        pos += s;
+                        const double w = Q.lut[s ? d - Q.d0 : 0];
+                        sqk[k] += s ? w : 0.0;
+                    }
+                    nq += __shfl_sync(kFullMask, incl, 31);
+                }
+            }
+            sq = (sqk[0] + sqk[1]) + (sqk[2] + sqk[3]);
+            __syncwarp();
+            // survivors before each word of this warp run
+            const int nw = w1 - w0, per = (nw + 31) / 32;
+            int cnt = 0;
+            for (int k = 0; k < per; ++k) {
+                const int wd = w0 + lane * per + k;
+                if (wd < w1) cnt += __popc(sh.qbits[wd]);
+            }
+            int run = warp_inclusive_scan(cnt, lane) - cnt;
+            for (int k = 0; k < per; ++k) {
+                const int wd = w0 + lane * per + k;
+                if (wd < w1) {
+                    sh.wpre[wd] = (uint16_t)run;
+                    run += __popc(sh.qbits[wd]);
+                }
+            }
+            __syncwarp();
+        }
+        rs_mark(p, 2, jm, 1);
+        // weight of a verifier survivor's drafter twin (0 if the drafter does not keep the id)
+        auto q_of = [&](uint32_t id) -> double {
+            const uint32_t word = sh.qbits[id >> 5], bit = 1u << (id & 31u);
+            if (!(word & bit)) return 0.0;
+            const int k = sh.wpre[id >> 5] + __popc(word & (bit - 1u));
+            return Q.lut[(int)sh.qd[warp][k] - Q.d0];
+        };
+        // a survivor's mass under draw mode (0: the draw row, 1: verifier, 2: residual)
+        auto mass = [&](int mode, const ListRow& R, uint32_t e) -> double {
+            const double w = R.weight(e);
+            if (mode != 2) return w;
+            const double dl = w * P.iS - q_of((uint32_t)R.id(e)) * Q.iS;
+            return dl > 0.0 ? dl : 0.0;
+        };
+
+        // ---- the verifier's survivors: mass and residual mass ----
+        // (branch-free, one accumulator per entry slot: the four lookups of a lane overlap)
+        double sp = 0.0, sr = 0.0;
+        {
+            double spk[4] = {0.0, 0.0, 0.0, 0.0}, srk[4] = {0.0, 0.0, 0.0, 0.0};
+            for (int t0 = 0; t0 < P.n; t0 += kLT * kLB) {
+                uint4 v[kLB];
+                load_batch(P, t0, v, lane);
+#pragma unroll
+                for (int u = 0; u < kLB; ++u) {
+                    if (t0 + u * kLT >= P.n) break;
+                    uint32_t e[4];
+                    const uint32_t keep = tile_keep(v[u], t0 + u * kLT + lane * 4, P, e);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const bool s = (keep >> k) & 1u;
+                        const double wp = P.lut[s ? P.bin(e[k]) - P.d0 : 0];
+                        spk[k] += s ? wp : 0.0;
+                        if (two) {
+                            const uint32_t id = (uint32_t)P.id(e[k]);
+                            const uint32_t word = sh.qbits[id >> 5], bit = 1u << (id & 31u);
+                            const bool has = s && (word & bit);
+                            const int kq = has ? sh.wpre[id >> 5] + __popc(word & (bit - 1u)) : 0;
+                            const int qb = sh.qd[warp][kq];
+                            const double wq = Q.lut[has ? qb - Q.d0 : 0];
+                            const double dl = wp * P.iS - (has ? wq : 0.0) * Q.iS;
+                            srk[k] += (s && dl > 0.0) ? dl : 0.0;
+                        }
+                    }
+                }
+            }
+            sp = (spk[0] + spk[1]) + (spk[2] + spk[3]);
+            sr = (srk[0] + srk[1]) + (srk[2] + srk[3]);
+        }
+        sq = warp_sum_f64(sq);
+        sp = warp_sum_f64(sp);
+        sr = warp_sum_f64(sr);
+        if (lane == 0) {
+            sh.ws[warp][0] = two ? sq : sp;
+            sh.ws[warp][1] = sp;
+            sh.ws[warp][2] = sr;
+        }
+        __syncthreads();
+        rs_mark(p, 2, jm, 2);
+
+        // ---- draws: the warp run holding the target, then the token in its segment ----
+        // The first token whose running mass (id order) exceeds the target; if rounding leaves
+        // no crossing, the last token with positive mass; -1 if there is none.
+        auto draw = [&](int mode, double target) -> int {
+            if (tid == 0) {
+                double cacc = 0.0, clast = 0.0;
+                int sw = -1, lw = -1;
+                for (int w = 0; w < kWarps; ++w) {
+                    const double m = sh.ws[w][mode];
+                    if (!(m > 0.0)) continue;
+                    lw = w;
+                    clast = cacc;
+                    if (cacc + m > target) {
+                        sw = w;
+                        break;
+                    }
+                    cacc += m;
+                }
+                sh.last_mode = sw < 0;
+                sh.sel_w = sw < 0 ? lw : sw;
+                sh.sel_c = sw < 0 ? clast : cacc;
+                sh.tok_found = -1;
+            }
+            __syncthreads();
+            if (warp == sh.sel_w) {
+                const bool last_mode = sh.last_mode;
+                const ListRow R = (mode == 0 && two) ? Q : P;  // (a copy: both stay in registers)
+                // the masses of a lane's 4 entries of tile u (0 for those that do not survive)
+                auto tile_mass = [&](const uint4& vu, int j, double (&x)[4], uint32_t (&e)[4]) {
+                    const uint32_t keep = tile_keep(vu, j, R, e);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) x[k] = ((keep >> k) & 1u) ? mass(mode, R, e[k]) : 0.0;
+                };
+                double carry = sh.sel_c;
+                int res = -1;
+                // the tile holding the crossing from whole-tile masses (independent reductions),
+                // then the token inside it
+                for (int t0 = 0; t0 < R.n && res < 0 && !last_mode; t0 += kLT * kLB) {
+                    uint4 v[kLB];
+                    load_batch(R, t0, v, lane);
+                    double T[kLB];
+#pragma unroll
+                    for (int u = 0; u < kLB; ++u) {
+                        double x[4];
+                        uint32_t e[4];
+                        tile_mass(v[u], t0 + u * kLT + lane * 4, x, e);
+                        T[u] = (x[0] + x[1]) + (x[2] + x[3]);
+                    }
+#pragma unroll
+                    for (int u = 0; u < kLB; ++u) T[u] = warp_sum_f64(T[u]);
+#pragma unroll
+                    for (int u = 0; u < kLB; ++u) {
+                        if (res >= 0 || !(T[u] > 0.0)) continue;  // the same in every lane
+                        if (carry + T[u] > target) {
+                            double x[4];
+                            uint32_t e[4];
+                            tile_mass(v[u], t0 + u * kLT + lane * 4, x, e);
+                            const double s = (x[0] + x[1]) + (x[2] + x[3]);
+                            const double incl = warp_scan_f64(s, lane);
+                            const unsigned hit = __ballot_sync(kFullMask, s > 0.0 && carry + incl > target);
+                            if (hit) {
+                                int cross = -1, lastk = -1;
+                                double run = carry + (incl - s);
+#pragma unroll
+                                for (int k = 0; k < 4; ++k)
+                                    if (x[k] > 0.0) {
+                                        run += x[k];
+                                        lastk = R.id(e[k]);
+                                        if (cross < 0 && run > target) cross = lastk;
+                                    }
+                                if (cross < 0) cross = lastk;
+                                res = __shfl_sync(kFullMask, cross, __ffs(hit) - 1);
+                            }
+                        }
+                        carry += T[u];
+                    }
+                }
+                if (res < 0) {
+                    // no crossing (rounding, or the target at the total): the last token with mass
+                    for (int t0 = 0; t0 < R.n; t0 += kLT * kLB) {
+                        uint4 v[kLB];
+                        load_batch(R, t0, v, lane);
+#pragma unroll
+                        for (int u = 0; u < kLB; ++u) {
+                            double x[4];
+                            uint32_t e[4];
+                            tile_mass(v[u], t0 + u * kLT + lane * 4, x, e);
+                            int lastk = -1;
+#pragma unroll
+                            for (int k = 0; k < 4; ++k)
+                                if (x[k] > 0.0) lastk = R.id(e[k]);
+                            const unsigned pos = __ballot_sync(kFullMask, lastk >= 0);
+                            if (pos) res = __shfl_sync(kFullMask, lastk, 31 - __clz(pos));
+                        }
+                    }
+                }
+                if (lane == 0) sh.tok_found = res;
+            }
+            __syncthreads();
+            const int out = sh.tok_found;
+            __syncthreads();
+            return out;
+        };
+
+        const float* u = p.u + (int64_t)item * 3;
+        double Rm = 0.0;  // TV(p, q) = sum of max(0, p - q), both distributions summing to 1
+        for (int w = 0; w < kWarps; ++w) Rm += sh.ws[w][2];
+        Rec rec;
+        rec.state = kDone;
+        rec.pad = 0.0;
+        rec.res = -1;
+        rec.tv = two ? Rm : 0.0;
+        const bool given = !two ? pos0_given(p, b) : p.drafts != nullptr;
+        int tok = !given ? -1 : (!two ? p.pos0[b] : p.drafts[item]);
+        // the draws (one call site keeps the code small): s = 0 the token, unless it is given;
+        // s = 1 the residual draw (two rows), from p itself if max(0, p - q) has no mass
+        for (int s = 0; s < 2; ++s) {
+            if (s == 0 && given) continue;
+            if (s == 1 && !two) break;
+            const int mode = s == 0 ? 0 : (Rm > 0.0 ? 2 : 1);
+            const double target = s == 0 ? (double)u[0] * (two ? Q.S : P.S) : (double)u[2] * (Rm > 0.0 ? Rm : P.S);
+            const int got = draw(mode, target);
+            if (s == 0) tok = got;
+            else rec.res = got;
+        }
+        rs_mark(p, 2, jm, 3);
+        rec.tok = tok;
+        // p(tok), q(tok) from the logits: survivors by the same rule as the lists'
+        auto prob = [&](const ListRow& R, int r) -> double {
+            if (tok < 0 || tok >= V) return 0.0;
+            const __nv_bfloat16* row = r < n_items ? static_cast<const __nv_bfloat16*>(p.P) + (int64_t)r * V
+                                                   : static_cast<const __nv_bfloat16*>(p.Q) + (int64_t)(r - n_items) * V;
+            const uint32_t h = reinterpret_cast<const uint16_t*>(row)[tok];
+            if (h & 0x8000u) return 0.0;  // negative: below the window (whose floor is positive)
+            const int d = R.a15 - (int)h;
+            if (d < 0 || d > R.dcut || (d == R.dcut && tok >= R.theta)) return 0.0;
+            return R.lut[d - R.d0] * R.iS;
+        };
+        rec.p = prob(P, item);
+        rec.q = two ? prob(Q, n_items + item) : 0.0;
+        rec.acc = two ? (double)u[1] * rec.q < rec.p : 1;
+        if (tid == 0) p.recs[item] = rec;
+        rs_mark(p, 2, jm, 4);
+    }
+    rs_end(p, 7168);
+}
+
 }  // namespace rs
 
 // =======================================================================================
@@ -3315,7 +3827,8 @@ bool rs_applies(const VerifyArgs& a) {
 
 int num_sms();
 
-uno_status launch_rs(const VerifyArgs& a, const Params& p, rs::RowRec* rows, cudaStream_t stream) {
+uno_status launch_rs(const VerifyArgs& a, const Params& p, rs::RowRec* rows, uint32_t* ctr, uint32_t* lists,
+                     cudaStream_t stream) {
     static std::mutex mu;
     static bool ready[64] = {};
     int dev = 0;
@@ -3324,7 +3837,11 @@ uno_status launch_rs(const VerifyArgs& a, const Params& p, rs::RowRec* rows, cud
         std::lock_guard<std::mutex> lock(mu);
         if (!ready[dev]) {
             uno_status s;
-            if ((s = check_cuda(cudaFuncSetAttribute(rs::row_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            if ((s = check_cuda(cudaFuncSetAttribute(rs::row_kernel<rs::kRowCtasPerSm>,
+                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(rs::RowShared)),
+                                "cudaFuncSetAttribute(verify rows)")) != UNO_OK)
+                return s;
+            if ((s = check_cuda(cudaFuncSetAttribute(rs::row_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                      (int)sizeof(rs::RowShared)),
                                 "cudaFuncSetAttribute(verify rows)")) != UNO_OK)
                 return s;
@@ -3332,15 +3849,33 @@ uno_status launch_rs(const VerifyArgs& a, const Params& p, rs::RowRec* rows, cud
                                                      (int)sizeof(rs::ItemShared)),
                                 "cudaFuncSetAttribute(verify items)")) != UNO_OK)
                 return s;
+            if ((s = check_cuda(cudaFuncSetAttribute(rs::item_list_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                     (int)sizeof(rs::ListShared)),
+                                "cudaFuncSetAttribute(verify list items)")) != UNO_OK)
+                return s;
             ready[dev] = true;
         }
     }
     const int items = a.B * a.K;
     const int slots = num_sms() * rs::kCtasPerSm;
-    rs::row_kernel<<<(unsigned)std::min(2 * items, num_sms() * rs::kRowCtasPerSm), rs::kThreads, sizeof(rs::RowShared),
-                     stream>>>(p, rows);
-    uno_status s = check_cuda(cudaGetLastError(), "launch(verify rows)");
+    // UNO_VERIFY_LISTS=off: every item weighed from the logits by item_kernel_rs
+    const char* lm = getenv("UNO_VERIFY_LISTS");
+    if (lists == nullptr || a.V > rs::kMaxListV || (lm && strcmp(lm, "off") == 0)) lists = nullptr;
+    uno_status s = check_cuda(cudaMemsetAsync(ctr, 0, 2 * sizeof(uint32_t), stream), "verify: counters");
     if (s != UNO_OK) return s;
+    const char* rc = getenv("UNO_VERIFY_ROW_CTAS");
+    if (rc && strcmp(rc, "2") == 0)
+        rs::row_kernel<2><<<(unsigned)std::min(2 * items, num_sms() * 2), rs::kThreads, sizeof(rs::RowShared), stream>>>(
+            p, rows, lists, ctr);
+    else
+        rs::row_kernel<rs::kRowCtasPerSm><<<(unsigned)std::min(2 * items, num_sms() * rs::kRowCtasPerSm), rs::kThreads,
+                                            sizeof(rs::RowShared), stream>>>(p, rows, lists, ctr);
+    if ((s = check_cuda(cudaGetLastError(), "launch(verify rows)")) != UNO_OK) return s;
+    if (lists != nullptr) {
+        rs::item_list_kernel<<<(unsigned)std::min(items, 2 * num_sms()), rs::kThreads, sizeof(rs::ListShared), stream>>>(
+            p, rows, lists, ctr + 1);
+        if ((s = check_cuda(cudaGetLastError(), "launch(verify list items)")) != UNO_OK) return s;
+    }
     rs::item_kernel_rs<<<(unsigned)std::min(items, slots), rs::kThreads, sizeof(rs::ItemShared), stream>>>(p, rows);
     return check_cuda(cudaGetLastError(), "launch(verify items)");
 }
@@ -3358,18 +3893,28 @@ int num_sms() {
 
 }  // namespace vfull
 
-// the records, then (top-k off) the row records of the row-streaming path
-size_t verify_full_workspace_bytes(const VerifyArgs& a) {
+// the row records of the row-streaming path and its two work counters
+inline size_t rs_rows_bytes(const VerifyArgs& a) {
+    return align_up((size_t)2 * a.B * a.K * sizeof(vfull::rs::RowRec) + 2 * sizeof(uint32_t), 256);
+}
+
+// the records, then (top-k off) the row records of the row-streaming path and, with
+// with_lists, the rows' candidate lists (without them every item is weighed from the logits)
+size_t verify_full_workspace_bytes(const VerifyArgs& a, bool with_lists) {
     size_t n = align_up(vfull::recs_bytes(a), 256);
-    if (a.top_k == 0) n += (size_t)2 * a.B * a.K * sizeof(vfull::rs::RowRec);
+    if (a.top_k == 0) {
+        n += rs_rows_bytes(a);
+        if (with_lists && a.V <= vfull::rs::kMaxListV)
+            n += (size_t)2 * a.B * a.K * vfull::rs::kWarps * vfull::rs::kListCap * 4;
+    }
     return n;
 }
 
 // The item path: pair_kernel where it applies, the generic kernel for the rest, then the
 // per-sequence assembly. With allow_generic false (top-k on: the streaming path serves the
 // cases pair_kernel does not take) nothing is launched unless pair_kernel takes the batch.
-uno_status verify_full_launch(const VerifyArgs& a, void* workspace, cudaStream_t stream, bool allow_generic,
-                              bool* taken) {
+uno_status verify_full_launch(const VerifyArgs& a, void* workspace, size_t workspace_bytes, cudaStream_t stream,
+                              bool allow_generic, bool* taken) {
     vfull::Params p{};
     p.P = a.P;
     p.Q = a.Q;
@@ -3393,9 +3938,13 @@ uno_status verify_full_launch(const VerifyArgs& a, void* workspace, cudaStream_t
     uno_status st = UNO_OK;
     int only_redo = 0;
     if (vfull::rs_applies(a)) {
-        auto* rows = reinterpret_cast<vfull::rs::RowRec*>(static_cast<unsigned char*>(workspace) +
-                                                          align_up(vfull::recs_bytes(a), 256));
-        if ((st = vfull::launch_rs(a, p, rows, stream)) != UNO_OK) return st;
+        unsigned char* w8 = static_cast<unsigned char*>(workspace) + align_up(vfull::recs_bytes(a), 256);
+        auto* rows = reinterpret_cast<vfull::rs::RowRec*>(w8);
+        auto* ctr = reinterpret_cast<uint32_t*>(w8 + (size_t)2 * a.B * a.K * sizeof(vfull::rs::RowRec));
+        auto* lists = workspace_bytes >= verify_full_workspace_bytes(a, true)
+                          ? reinterpret_cast<uint32_t*>(w8 + rs_rows_bytes(a))
+                          : nullptr;
+        if ((st = vfull::launch_rs(a, p, rows, ctr, lists, stream)) != UNO_OK) return st;
         only_redo = 1;
     } else if (vfull::launch_pairs(a, p, stream, st)) {
         if (st != UNO_OK) return st;

@@ -178,10 +178,17 @@ uno_status uno_gated_lora_linear(const void* x, const void* w0, const void* lora
  *
  * Logits must be finite. Limits (else UNO_ERR_UNSUPPORTED): 1 <= K <= 32, 1 <= V < 2^31,
  * B >= 0 (B = 0 does nothing), B * K * V < 2^40.
- * Workspace: uno_block_verify_workspace_size(B, K, V, top_k, top_p, dtype) bytes.
+ * Workspace: uno_block_verify_workspace_size(B, K, V, top_k, top_p, dtype) bytes, the size
+ * the fastest path uses. With top_k off and bf16 logits that includes each row's candidate
+ * list (every token whose logit is near enough to the row's largest to be in the nucleus,
+ * 128 KiB per row); a workspace of at least uno_block_verify_min_workspace_size(...) bytes
+ * is also accepted, and the call then weighs every item from the logits instead (slower,
+ * same results). The two sizes are equal when top_k is on.
  * ====================================================================================== */
 size_t uno_block_verify_workspace_size(int32_t B, int32_t K, int32_t V, int32_t top_k,
                                        float top_p, uno_dtype dtype);
+size_t uno_block_verify_min_workspace_size(int32_t B, int32_t K, int32_t V, int32_t top_k,
+                                           float top_p, uno_dtype dtype);
 
 uno_status uno_block_verify(const void* verifier_logits, const void* drafter_logits,
                             uno_dtype dtype, int32_t B, int32_t K, int32_t V,
@@ -210,8 +217,9 @@ uno_status uno_block_verify(const void* verifier_logits, const void* drafter_log
  * zero); calls that can overlap on the GPU race on it, so order them on one stream or
  * synchronise between them.
  *
+ * It uses the candidate lists when the array holds them, and otherwise the smaller workspace.
  * Errors: as uno_block_verify, plus UNO_ERR_UNSUPPORTED when the batch needs more scratch
- * than the array holds (uno_block_verify_workspace_size(...) > UNO_NOALLOC_SCRATCH_BYTES;
+ * than the array holds (uno_block_verify_min_workspace_size(...) > UNO_NOALLOC_SCRATCH_BYTES;
  * the 64 x 16 x 151936 top-k 50 batch needs about 9.4 MiB).
  * ====================================================================================== */
 #define UNO_NOALLOC_SCRATCH_BYTES (16u << 20)

@@ -28,7 +28,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported(lib):
     names = declared_functions()
-    assert len(names) == 12, names
+    assert len(names) == 13, names
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(_lib.EXPORTED)
@@ -77,6 +77,15 @@ def test_verify_workspace_sizes(lib):
     assert lib.uno_block_verify_workspace_size(0, 16, 151936, 50, 0.95, _lib.UNO_BF16) == 0
     assert lib.uno_block_verify_workspace_size(4, 40, 1000, 0, 1.0, _lib.UNO_BF16) == 0  # unsupported
     assert lib.uno_block_verify_workspace_size(2, 8, 1000, 0, 1.0, _lib.UNO_F32) > 0
+    # top-k on: one size; top-k off with bf16 rows: the fastest path adds a 128 KiB
+    # candidate list per row (two rows per item) to the smallest workspace accepted
+    for B, K, V, k in ((64, 16, 151936, 50), (3, 5, 700, 1)):
+        assert (lib.uno_block_verify_min_workspace_size(B, K, V, k, 0.95, _lib.UNO_BF16)
+                == lib.uno_block_verify_workspace_size(B, K, V, k, 0.95, _lib.UNO_BF16))
+    full = lib.uno_block_verify_workspace_size(256, 8, 166144, 0, 0.95, _lib.UNO_BF16)
+    small = lib.uno_block_verify_min_workspace_size(256, 8, 166144, 0, 0.95, _lib.UNO_BF16)
+    assert full - small == 2 * 256 * 8 * (128 << 10)
+    assert lib.uno_block_verify_min_workspace_size(0, 8, 166144, 0, 0.95, _lib.UNO_BF16) == 0
 
 
 def test_lora_validation(lib):

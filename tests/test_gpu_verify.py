@@ -272,6 +272,50 @@ def test_full_vocab_parity(case):
     _check_full(P, Q, u, T, p, dtype)
 
 
+@pytest.mark.parametrize("case", [c for c in FULL_CASES if c[0] == "bf16"],
+                         ids=[f"B{c[1]}K{c[2]}V{c[3]}p{c[5]}" for c in FULL_CASES if c[0] == "bf16"])
+def test_full_vocab_parity_without_lists(case, monkeypatch):
+    """UNO_VERIFY_LISTS=off: the row pass records no candidate lists, so every item is weighed
+    from the logits by the row-streaming item kernel instead of from its rows' lists; both
+    give the oracle's results."""
+    monkeypatch.setenv("UNO_VERIFY_LISTS", "off")
+    dtype, B, K, V, T, p = case
+    P, Q, u = _inputs(B, K, V, dtype, seed=zlib.crc32(str(case).encode()) % 10007)
+    _check_full(P, Q, u, T, p, dtype)
+
+
+def test_full_vocab_smallest_workspace():
+    """A workspace of uno_block_verify_min_workspace_size bytes (no room for the candidate
+    lists) is accepted and gives the same outputs as the full workspace; one byte less is
+    rejected."""
+    from diffusion_drafted_lossless_b200 import _lib
+    from tests.gpu_util import dev
+    B, K, V = 3, 6, 20000
+    P, Q, u = _inputs(B, K, V, "bf16", seed=46)
+    outs = []
+    for size in (_lib.uno_block_verify_workspace_size(B, K, V, 0, 0.95),
+                 _lib.uno_block_verify_min_workspace_size(B, K, V, 0, 0.95)):
+        ws = torch.empty(size, dtype=torch.uint8, device="cuda")
+        t = torch.empty((B, K), dtype=torch.int32, device="cuda")
+        c = torch.empty((B,), dtype=torch.int32, device="cuda")
+        nx = torch.empty((B,), dtype=torch.int32, device="cuda")
+        pt = torch.empty((B, K), dtype=torch.float32, device="cuda")
+        _lib.uno_block_verify(dev(P, "bf16"), dev(Q, "bf16"), 1.0, 0, 0.95, torch.from_numpy(u).cuda(), t, c, nx,
+                              out_p_tok=pt, workspace=ws)
+        torch.cuda.synchronize()
+        outs.append((t.cpu().numpy(), c.cpu().numpy(), nx.cpu().numpy(), pt.cpu().numpy()))
+    for a, b in zip(outs[0][:3], outs[1][:3]):
+        np.testing.assert_array_equal(a, b)
+    np.testing.assert_allclose(outs[0][3], outs[1][3], rtol=1e-6, atol=0)
+    ws = torch.empty(_lib.uno_block_verify_min_workspace_size(B, K, V, 0, 0.95) - 256, dtype=torch.uint8,
+                     device="cuda")
+    t = torch.empty((B, K), dtype=torch.int32, device="cuda")
+    c = torch.empty((B,), dtype=torch.int32, device="cuda")
+    with pytest.raises(Exception):
+        _lib.uno_block_verify(dev(P, "bf16"), dev(Q, "bf16"), 1.0, 0, 0.95, torch.from_numpy(u).cuda(), t, c,
+                              workspace=ws)
+
+
 def test_full_vocab_ties_and_supplied_tokens():
     B, K, V = 3, 5, 4000
     rng = np.random.default_rng(41)
