@@ -2155,7 +2155,7 @@ struct RowShared {
     uint32_t hc[kWin];           // their sum
     double wd[kWin];             // weight of window key d (where present), relative to zmax
     uint32_t hr[2 * kMagWin];    // recount: counts of (sign, magnitude largest - d)
-    uint32_t stage[kWarps][kStage];  // counted elements ((id - c0 256) << 16 | bits) on their way to the list
+    uint32_t stage[kWarps][kStage];  // counted elements (bits << 16 | (0xFFFF - (id - c0 256))) on their way to the list
     float fmax[kWarps];
     double dz[kWarps], db[kWarps], red[kWarps];
     int ties[kWarps];
@@ -2219,7 +2219,7 @@ constexpr int kLT = 128;  // entries per list tile: lane l holds entries 4l .. 4
 constexpr int kLB = 8;    // tiles per batch: the 16-byte loads each lane has in flight
 
 // The id of the kk-th entry (0-based, id order) of a warp's list of n entries whose bits are
-// hcut (entries: (id - id0) << 16 | bits); INT_MAX if there are not that many.
+// hcut (entries: bits << 16 | (0xFFFF - (id - id0))); INT_MAX if there are not that many.
 __device__ int find_tie(const uint32_t* list, int n, uint32_t hcut, int kk, int id0, int lane) {
     int cnt = 0;
     for (int t0 = 0; t0 < n; t0 += kLT * kLB) {
@@ -2235,7 +2235,7 @@ __device__ int find_tie(const uint32_t* list, int n, uint32_t hcut, int kk, int 
             const uint32_t e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
             uint32_t tie = 0u;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) tie |= (uint32_t)(j + k < n && (e[k] & 0xFFFFu) == hcut) << k;
+            for (int k = 0; k < 4; ++k) tie |= (uint32_t)(j + k < n && (e[k] >> 16) == hcut) << k;
             const int nt = __popc(tie);
             const int tot = (int)__reduce_add_sync(kFullMask, (unsigned)nt);
             if (cnt + tot > kk) {  // the same in every lane
@@ -2248,7 +2248,7 @@ __device__ int find_tie(const uint32_t* list, int n, uint32_t hcut, int kk, int 
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
                         if ((tie >> k) & 1u) {
-                            if (q == 0) id = id0 + (int)(e[k] >> 16);
+                            if (q == 0) id = id0 + 0xFFFF - (int)(e[k] & 0xFFFFu);
                             --q;
                         }
                 }
@@ -2325,8 +2325,9 @@ __global__ void __launch_bounds__(kThreads, CPS) row_kernel(Params p, RowRec* ro
         rs_mark(p, 0, jm, 1);
         // ---- stream the row ----
         // Every counted element (x >= F) goes, in id order, to the warp's stage as
-        // (id - c0 256) << 16 | bits; each flush of the stage counts its entries' window bins
-        // and appends them to the warp's candidate list.
+        // bits << 16 | (0xFFFF - (id - c0 256)) (so one unsigned comparison with a per-row
+        // threshold tells a survivor); each flush of the stage counts its entries' window
+        // bins and appends them to the warp's candidate list.
         __nv_bfloat162 mx2 = __floats2bfloat162_rn(-INFINITY, -INFINITY);
         double zr = 0.0;  // rest weights exp((x - F) / T)
         float zb = 0.f;   // rest weights times |their ex2 argument| (for the error bound)
@@ -2338,7 +2339,7 @@ __global__ void __launch_bounds__(kThreads, CPS) row_kernel(Params p, RowRec* ro
             __syncwarp();
             for (int j = lane; j < n; j += 32) {
                 const uint32_t s = stg[j];
-                atomicAdd(&hwp[min(A15 - (s & 0xFFFFu), (uint32_t)kWin)], 1u);  // above the anchor: last slot
+                atomicAdd(&hwp[min(A15 - (s >> 16), (uint32_t)kWin)], 1u);  // above the anchor: last slot
                 if (gl != nullptr && gn + n <= kListCap) gl[gn + j] = s;
             }
             gn += n;
@@ -2383,11 +2384,11 @@ __global__ void __launch_bounds__(kThreads, CPS) row_kernel(Params p, RowRec* ro
                 const int tot = __shfl_sync(kFullMask, incl, 31);
                 if (tot) {
                     int pos = lq + incl - cnt;
-                    const uint32_t base = (uint32_t)((c + u - c0) * kCh + lane * 8) << 16;
+                    const uint32_t base = 0xFFFFu - (uint32_t)((c + u - c0) * kCh + lane * 8);
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
                         if ((cm >> e) & 1u)
-                            stg[pos++] = __byte_perm(w4[e >> 1], base + ((uint32_t)e << 16), (e & 1) ? 0x7632u : 0x7610u);
+                            stg[pos++] = __byte_perm(w4[e >> 1], base - (uint32_t)e, (e & 1) ? 0x3254u : 0x1054u);
                     lq += tot;
                     if (lq >= 256) {  // (lq < 512: the rest moves from [256, lq) to the front)
                         flush(256);
@@ -2495,7 +2496,7 @@ __global__ void __launch_bounds__(kThreads, CPS) row_kernel(Params p, RowRec* ro
             // The lists are complete when every warp's fits. Then the tie at the cut of rank
             // tie_t (id order), the first that does not survive, is found in its warp's list:
             // a tie survives exactly when its id is below that tie's id (theta).
-            int lok = lists != nullptr && V <= kMaxListV;
+            int lok = lists != nullptr && V <= kMaxListV && lut_n <= 255;  // (table indices fit a byte)
             for (int w = 0; w < kWarps; ++w) lok &= sh.ln[w] <= kListCap;
             if (lok) {
                 const int tt = sh.tie_t;
@@ -3172,62 +3173,57 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) item_kernel_rs(Params p,
 
 
 // ---------------------------------------------------------------------------------------
-// item pass over the candidate lists (items whose rows both took the window path)
+// item pass over the candidate lists (items whose rows both have complete lists)
 // ---------------------------------------------------------------------------------------
-// The survivors of a row are the entries of its lists with a bin below the cut bin, and the
-// first tie_t of those at it (in id order: the lists are in id order, warp run by warp run).
-// Warp w works on list segment w of both rows, which covers the same ids [c0 256, c1 256)
-// in both: the drafter's survivors go to a bitmap of their ids and a compact array of their
-// bins (id order), which the verifier's survivors look up to weigh max(0, p - q).
+// Warp w works on list segment w of both rows, which covers the same ids [c0 256, c1 256) in
+// both. A list entry is bits << 16 | (0xFFFF - (id - id0)) (id0 = c0 256, bits the logit's
+// bf16 bits, positive); it survives when it is above the row's threshold: its value above
+// the cut value, or at it with an id below theta. The drafter's survivors go to a bitmap of
+// their ids and a byte array of their table indices (id order, found through per-word
+// prefix counts), which the verifier's survivors look up to weigh max(0, p - q). Each pass
+// also keeps every 128-entry tile's masses, so a draw reads one tile of one segment.
 constexpr int kBitWords = kMaxListV / 32;
+constexpr int kMaxTiles = kListCap / kLT;
+
 struct ListShared {
-    double lut[2][kLutMax];
+    double lut[2][kLutMax];                  // weights by table index (hM - bits): verifier, drafter
+    double tm[kWarps][kMaxTiles][3];         // per tile: drafter mass, verifier mass, residual mass
     uint32_t qbits[kBitWords];               // drafter survivors by id
     uint16_t wpre[kBitWords];                // drafter survivors before each bitmap word (within its warp run)
-    uint16_t qd[kWarps][kListCap];           // drafter survivors' bins, id order, per warp run
-    double ws[kWarps][3];                    // per warp run: draw-row mass, verifier mass, residual mass
+    uint8_t qd[kWarps][kListCap];            // drafter survivors' table indices, id order, per warp run
+    double ws[kWarps][3];                    // per warp run: the tiles' masses summed in order
     double sel_c;
-    int sel_w, tok_found, last_mode;
-    int next[2];  // the next item (alternate items use alternate slots)
+    int sel_w, tok_found;
+    int next[2];                             // the next item (alternate items use alternate slots)
 };
 
-// A list entry is (id - id0) << 16 | bits for a counted element of the warp run starting at
-// token id0; its window bin is A15 - bits. It survives when its bin is below the cut bin, or
-// at it with an id below theta.
 struct ListRow {
     const uint32_t* list;   // this warp's segment
-    int n, dcut, theta, d0, a15, id0;
+    int n;                  // its entries
+    uint32_t thr;           // survivors: entries above thr
+    int hM;                 // bits of the row's largest value (table index = hM - bits)
+    int idtop;              // id0 + 0xFFFF (id = idtop - low half)
+    int hcut, theta;        // the cut value's bits; ties survive below theta
     double iS, S;
-    const double* lut;
-    __device__ __forceinline__ int bin(uint32_t e) const { return a15 - (int)(e & 0xFFFFu); }
-    __device__ __forceinline__ int id(uint32_t e) const { return id0 + (int)(e >> 16); }
-    __device__ __forceinline__ bool survives(uint32_t e) const {
-        const int d = bin(e);
-        return d < dcut || (d == dcut && id(e) < theta);
-    }
-    __device__ __forceinline__ double weight(uint32_t e) const { return lut[bin(e) - d0]; }
+    __device__ __forceinline__ int tix(uint32_t e) const { return hM - (int)(e >> 16); }
+    __device__ __forceinline__ int id(uint32_t e) const { return idtop - (int)(e & 0xFFFFu); }
 };
 
-// a batch of kLB tiles of a segment from entry t0 (entries past n read as 0; the segment's
-// kListCap entries are all in the workspace)
+// a batch of kLB tiles of a segment from entry t0 (entries past n read as 0, which never
+// survives: thr >= 2^16 - 1)
 __device__ __forceinline__ void load_batch(const ListRow& R, int t0, uint4 (&v)[kLB], int lane) {
 #pragma unroll
     for (int u = 0; u < kLB; ++u) {
         const int j = t0 + u * kLT + lane * 4;
-        v[u] = j < R.n ? __ldcg(reinterpret_cast<const uint4*>(R.list + j)) : make_uint4(0u, 0u, 0u, 0u);
+        uint4 x = make_uint4(0u, 0u, 0u, 0u);
+        if (j < R.n) {
+            x = __ldcg(reinterpret_cast<const uint4*>(R.list + j));
+            if (j + 1 >= R.n) x.y = 0u;
+            if (j + 2 >= R.n) x.z = 0u;
+            if (j + 3 >= R.n) x.w = 0u;
+        }
+        v[u] = x;
     }
-}
-
-// the survivors among a lane's 4 entries of a tile (bit k: entry k); j: the first one's index
-__device__ __forceinline__ uint32_t tile_keep(const uint4& v, int j, const ListRow& R, uint32_t (&e)[4]) {
-    e[0] = v.x;
-    e[1] = v.y;
-    e[2] = v.z;
-    e[3] = v.w;
-    uint32_t keep = 0u;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) keep |= (uint32_t)(j + k < R.n && R.survives(e[k])) << k;
-    return keep;
 }
 
 __global__ void __launch_bounds__(kThreads, 2) item_list_kernel(Params p, const RowRec* rows, const uint32_t* lists,
@@ -3263,14 +3259,14 @@ __global__ void __launch_bounds__(kThreads, 2) item_list_kernel(Params p, const 
             ListRow R;
             R.list = lists + ((int64_t)r * kWarps + warp) * kListCap;
             R.n = rr.list_n[warp];
-            R.dcut = rr.dcut;
+            R.hM = (int)(obits(rr.kM) & 0x7FFFu);
+            R.idtop = c0 * kCh + 0xFFFF;
+            R.hcut = (int)(rr.A15 - (uint32_t)rr.dcut);
             R.theta = rr.theta;
-            R.d0 = (int)(rr.A15 - (obits(rr.kM) & 0x7FFFu));
-            R.a15 = (int)rr.A15;
-            R.id0 = c0 * kCh;
+            const long long trel = min(max((long long)rr.theta - (long long)c0 * kCh, 0ll), 0x10000ll);
+            R.thr = (uint32_t)(((long long)R.hcut << 16) + 0xFFFF - trel);
             R.S = rr.S;
             R.iS = 1.0 / rr.S;
-            R.lut = sh.lut[slot];
             for (int j = tid; j < rr.lut_n; j += kThreads) sh.lut[slot][j] = rr.lut[j];
             return R;
         };
@@ -3279,39 +3275,41 @@ __global__ void __launch_bounds__(kThreads, 2) item_list_kernel(Params p, const 
         for (int j = w0 + lane; j < w1; j += 32) sh.qbits[j] = 0u;
         __syncthreads();
 
-        // ---- the drafter's survivors: bitmap, bins in id order, mass ----
-        double sq = 0.0;
+        // ---- the drafter's survivors: bitmap, table indices in id order, tile masses ----
         if (two) {
-            int nq = 0;
-            double sqk[4] = {0.0, 0.0, 0.0, 0.0};
+            int nq = 0, tile = 0;
             for (int t0 = 0; t0 < Q.n; t0 += kLT * kLB) {
                 uint4 v[kLB];
                 load_batch(Q, t0, v, lane);
 #pragma unroll
                 for (int u = 0; u < kLB; ++u) {
                     if (t0 + u * kLT >= Q.n) break;  // the same in every lane
-                    uint32_t e[4];
-                    const uint32_t keep = tile_keep(v[u], t0 + u * kLT + lane * 4, Q, e);
+                    const uint32_t e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+                    uint32_t keep = 0u;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) keep |= (uint32_t)(e[k] > Q.thr) << k;
                     const int c = __popc(keep);
                     const int incl = warp_inclusive_scan(c, lane);
                     int pos = nq + incl - c;
+                    double m = 0.0;
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
                         const bool s = (keep >> k) & 1u;
                         const uint32_t id = (uint32_t)Q.id(e[k]);
-                        const int d = Q.bin(e[k]);
+                        const int ti = Q.tix(e[k]);
                         if (s) {
                             atomicOr(&sh.qbits[id >> 5], 1u << (id & 31u));
-                            sh.qd[warp][pos] = (uint16_t)d;
+                            sh.qd[warp][pos] = (uint8_t)ti;
                         }
                         pos += s;
-                        const double w = Q.lut[s ? d - Q.d0 : 0];
-                        sqk[k] += s ? w : 0.0;
+                        m += s ? sh.lut[1][s ? ti : 0] : 0.0;
                     }
+                    m = warp_sum_f64(m);
+                    if (lane == 0) sh.tm[warp][tile][0] = m;
+                    ++tile;
                     nq += __shfl_sync(kFullMask, incl, 31);
                 }
             }
-            sq = (sqk[0] + sqk[1]) + (sqk[2] + sqk[3]);
             __syncwarp();
             // survivors before each word of this warp run
             const int nw = w1 - w0, per = (nw + 31) / 32;
@@ -3331,75 +3329,69 @@ __global__ void __launch_bounds__(kThreads, 2) item_list_kernel(Params p, const 
             __syncwarp();
         }
         rs_mark(p, 2, jm, 1);
-        // weight of a verifier survivor's drafter twin (0 if the drafter does not keep the id)
-        auto q_of = [&](uint32_t id) -> double {
+        // the drafter's weight of a verifier survivor's id (0 if the drafter does not keep it;
+        // s false: not a survivor, and the entry may be padding, whose id is out of range)
+        auto q_of = [&](uint32_t e, bool s) -> double {
+            const uint32_t id = s ? (uint32_t)P.id(e) : (uint32_t)(c0 * kCh);
             const uint32_t word = sh.qbits[id >> 5], bit = 1u << (id & 31u);
-            if (!(word & bit)) return 0.0;
-            const int k = sh.wpre[id >> 5] + __popc(word & (bit - 1u));
-            return Q.lut[(int)sh.qd[warp][k] - Q.d0];
-        };
-        // a survivor's mass under draw mode (0: the draw row, 1: verifier, 2: residual)
-        auto mass = [&](int mode, const ListRow& R, uint32_t e) -> double {
-            const double w = R.weight(e);
-            if (mode != 2) return w;
-            const double dl = w * P.iS - q_of((uint32_t)R.id(e)) * Q.iS;
-            return dl > 0.0 ? dl : 0.0;
+            const bool has = s && (word & bit);
+            const int kq = has ? sh.wpre[id >> 5] + __popc(word & (bit - 1u)) : 0;
+            const double wq = sh.lut[1][sh.qd[warp][kq]];
+            return has ? wq : 0.0;
         };
 
-        // ---- the verifier's survivors: mass and residual mass ----
-        // (branch-free, one accumulator per entry slot: the four lookups of a lane overlap)
-        double sp = 0.0, sr = 0.0;
+        // ---- the verifier's survivors: tile masses and residual masses (branch-free) ----
         {
-            double spk[4] = {0.0, 0.0, 0.0, 0.0}, srk[4] = {0.0, 0.0, 0.0, 0.0};
+            int tile = 0;
             for (int t0 = 0; t0 < P.n; t0 += kLT * kLB) {
                 uint4 v[kLB];
                 load_batch(P, t0, v, lane);
 #pragma unroll
                 for (int u = 0; u < kLB; ++u) {
                     if (t0 + u * kLT >= P.n) break;
-                    uint32_t e[4];
-                    const uint32_t keep = tile_keep(v[u], t0 + u * kLT + lane * 4, P, e);
+                    const uint32_t e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+                    double mp = 0.0, mr = 0.0;
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        const bool s = (keep >> k) & 1u;
-                        const double wp = P.lut[s ? P.bin(e[k]) - P.d0 : 0];
-                        spk[k] += s ? wp : 0.0;
+                        const bool s = e[k] > P.thr;
+                        const double wp = sh.lut[0][s ? P.tix(e[k]) : 0];
+                        mp += s ? wp : 0.0;
                         if (two) {
-                            const uint32_t id = (uint32_t)P.id(e[k]);
-                            const uint32_t word = sh.qbits[id >> 5], bit = 1u << (id & 31u);
-                            const bool has = s && (word & bit);
-                            const int kq = has ? sh.wpre[id >> 5] + __popc(word & (bit - 1u)) : 0;
-                            const int qb = sh.qd[warp][kq];
-                            const double wq = Q.lut[has ? qb - Q.d0 : 0];
-                            const double dl = wp * P.iS - (has ? wq : 0.0) * Q.iS;
-                            srk[k] += (s && dl > 0.0) ? dl : 0.0;
+                            const double dl = wp * P.iS - q_of(e[k], s) * Q.iS;
+                            mr += (s && dl > 0.0) ? dl : 0.0;
                         }
                     }
+                    mp = warp_sum_f64(mp);
+                    if (two) mr = warp_sum_f64(mr);
+                    if (lane == 0) {
+                        sh.tm[warp][tile][1] = mp;
+                        sh.tm[warp][tile][2] = mr;
+                    }
+                    ++tile;
                 }
             }
-            sp = (spk[0] + spk[1]) + (spk[2] + spk[3]);
-            sr = (srk[0] + srk[1]) + (srk[2] + srk[3]);
-        }
-        sq = warp_sum_f64(sq);
-        sp = warp_sum_f64(sp);
-        sr = warp_sum_f64(sr);
-        if (lane == 0) {
-            sh.ws[warp][0] = two ? sq : sp;
-            sh.ws[warp][1] = sp;
-            sh.ws[warp][2] = sr;
+            __syncwarp();
+            if (lane < 3) {  // the warp run's masses: its tiles' in order
+                const int nt = (lane == 0 ? Q.n : P.n) + kLT - 1;
+                double s = 0.0;
+                if (lane != 2 || two)
+                    for (int u = 0; u < nt / kLT; ++u) s += sh.tm[warp][u][lane];
+                sh.ws[warp][lane] = s;
+            }
         }
         __syncthreads();
         rs_mark(p, 2, jm, 2);
 
-        // ---- draws: the warp run holding the target, then the token in its segment ----
-        // The first token whose running mass (id order) exceeds the target; if rounding leaves
-        // no crossing, the last token with positive mass; -1 if there is none.
-        auto draw = [&](int mode, double target) -> int {
+        // ---- draws: the warp run, then the tile, holding the target; then the token ----
+        // col 0: the drafter's survivors, 1: the verifier's, 2: the residual. The first token
+        // whose running mass (id order) exceeds the target; if rounding leaves no crossing,
+        // the last token with positive mass; -1 if there is none.
+        auto draw = [&](int col, double target) -> int {
             if (tid == 0) {
                 double cacc = 0.0, clast = 0.0;
                 int sw = -1, lw = -1;
                 for (int w = 0; w < kWarps; ++w) {
-                    const double m = sh.ws[w][mode];
+                    const double m = sh.ws[w][col];
                     if (!(m > 0.0)) continue;
                     lw = w;
                     clast = cacc;
@@ -3409,83 +3401,65 @@ __global__ void __launch_bounds__(kThreads, 2) item_list_kernel(Params p, const 
                     }
                     cacc += m;
                 }
-                sh.last_mode = sw < 0;
                 sh.sel_w = sw < 0 ? lw : sw;
                 sh.sel_c = sw < 0 ? clast : cacc;
                 sh.tok_found = -1;
             }
             __syncthreads();
             if (warp == sh.sel_w) {
-                const bool last_mode = sh.last_mode;
-                const ListRow R = (mode == 0 && two) ? Q : P;  // (a copy: both stay in registers)
-                // the masses of a lane's 4 entries of tile u (0 for those that do not survive)
-                auto tile_mass = [&](const uint4& vu, int j, double (&x)[4], uint32_t (&e)[4]) {
-                    const uint32_t keep = tile_keep(vu, j, R, e);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) x[k] = ((keep >> k) & 1u) ? mass(mode, R, e[k]) : 0.0;
-                };
+                const ListRow R = col == 0 ? Q : P;  // (a copy: both stay in registers)
+                const int nt = (R.n + kLT - 1) / kLT;
                 double carry = sh.sel_c;
-                int res = -1;
-                // the tile holding the crossing from whole-tile masses (independent reductions),
-                // then the token inside it
-                for (int t0 = 0; t0 < R.n && res < 0 && !last_mode; t0 += kLT * kLB) {
-                    uint4 v[kLB];
-                    load_batch(R, t0, v, lane);
-                    double T[kLB];
-#pragma unroll
-                    for (int u = 0; u < kLB; ++u) {
-                        double x[4];
-                        uint32_t e[4];
-                        tile_mass(v[u], t0 + u * kLT + lane * 4, x, e);
-                        T[u] = (x[0] + x[1]) + (x[2] + x[3]);
+                int tf = -1, tl = -1;  // the tile with the crossing; the last tile with mass
+                for (int u = 0; u < nt; ++u) {
+                    const double m = sh.tm[warp][u][col];
+                    if (!(m > 0.0)) continue;
+                    tl = u;
+                    if (carry + m > target) {
+                        tf = u;
+                        break;
                     }
-#pragma unroll
-                    for (int u = 0; u < kLB; ++u) T[u] = warp_sum_f64(T[u]);
-#pragma unroll
-                    for (int u = 0; u < kLB; ++u) {
-                        if (res >= 0 || !(T[u] > 0.0)) continue;  // the same in every lane
-                        if (carry + T[u] > target) {
-                            double x[4];
-                            uint32_t e[4];
-                            tile_mass(v[u], t0 + u * kLT + lane * 4, x, e);
-                            const double s = (x[0] + x[1]) + (x[2] + x[3]);
-                            const double incl = warp_scan_f64(s, lane);
-                            const unsigned hit = __ballot_sync(kFullMask, s > 0.0 && carry + incl > target);
-                            if (hit) {
-                                int cross = -1, lastk = -1;
-                                double run = carry + (incl - s);
-#pragma unroll
-                                for (int k = 0; k < 4; ++k)
-                                    if (x[k] > 0.0) {
-                                        run += x[k];
-                                        lastk = R.id(e[k]);
-                                        if (cross < 0 && run > target) cross = lastk;
-                                    }
-                                if (cross < 0) cross = lastk;
-                                res = __shfl_sync(kFullMask, cross, __ffs(hit) - 1);
-                            }
-                        }
-                        carry += T[u];
-                    }
+                    carry += m;
                 }
-                if (res < 0) {
-                    // no crossing (rounding, or the target at the total): the last token with mass
-                    for (int t0 = 0; t0 < R.n; t0 += kLT * kLB) {
-                        uint4 v[kLB];
-                        load_batch(R, t0, v, lane);
-#pragma unroll
-                        for (int u = 0; u < kLB; ++u) {
-                            double x[4];
-                            uint32_t e[4];
-                            tile_mass(v[u], t0 + u * kLT + lane * 4, x, e);
-                            int lastk = -1;
-#pragma unroll
-                            for (int k = 0; k < 4; ++k)
-                                if (x[k] > 0.0) lastk = R.id(e[k]);
-                            const unsigned pos = __ballot_sync(kFullMask, lastk >= 0);
-                            if (pos) res = __shfl_sync(kFullMask, lastk, 31 - __clz(pos));
-                        }
+                int res = -1;
+                const int u = tf >= 0 ? tf : tl;
+                if (u >= 0) {
+                    const int j = u * kLT + lane * 4;
+                    uint4 x4 = make_uint4(0u, 0u, 0u, 0u);
+                    if (j < R.n) {
+                        x4 = __ldcg(reinterpret_cast<const uint4*>(R.list + j));
+                        if (j + 1 >= R.n) x4.y = 0u;
+                        if (j + 2 >= R.n) x4.z = 0u;
+                        if (j + 3 >= R.n) x4.w = 0u;
                     }
+                    const uint32_t e[4] = {x4.x, x4.y, x4.z, x4.w};
+                    double x[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const bool s = e[k] > R.thr;
+                        const double w = sh.lut[col == 0 ? 1 : 0][s ? R.tix(e[k]) : 0];
+                        double m = s ? w : 0.0;
+                        if (col == 2) {
+                            const double dl = w * P.iS - q_of(e[k], s) * Q.iS;
+                            m = (s && dl > 0.0) ? dl : 0.0;
+                        }
+                        x[k] = m;
+                    }
+                    const double s = (x[0] + x[1]) + (x[2] + x[3]);
+                    const double incl = warp_scan_f64(s, lane);
+                    int cross = -1, lastk = -1;
+                    double run = carry + (incl - s);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        if (x[k] > 0.0) {
+                            run += x[k];
+                            lastk = R.id(e[k]);
+                            if (cross < 0 && run > target) cross = lastk;
+                        }
+                    const unsigned hit = tf >= 0 ? __ballot_sync(kFullMask, cross >= 0) : 0u;
+                    const unsigned pos = __ballot_sync(kFullMask, lastk >= 0);
+                    if (hit) res = __shfl_sync(kFullMask, cross, __ffs(hit) - 1);
+                    else if (pos) res = __shfl_sync(kFullMask, lastk, 31 - __clz(pos));
                 }
                 if (lane == 0) sh.tok_found = res;
             }
@@ -3510,27 +3484,26 @@ __global__ void __launch_bounds__(kThreads, 2) item_list_kernel(Params p, const 
         for (int s = 0; s < 2; ++s) {
             if (s == 0 && given) continue;
             if (s == 1 && !two) break;
-            const int mode = s == 0 ? 0 : (Rm > 0.0 ? 2 : 1);
+            const int col = s == 0 ? (two ? 0 : 1) : (Rm > 0.0 ? 2 : 1);
             const double target = s == 0 ? (double)u[0] * (two ? Q.S : P.S) : (double)u[2] * (Rm > 0.0 ? Rm : P.S);
-            const int got = draw(mode, target);
+            const int got = draw(col, target);
             if (s == 0) tok = got;
             else rec.res = got;
         }
         rs_mark(p, 2, jm, 3);
         rec.tok = tok;
         // p(tok), q(tok) from the logits: survivors by the same rule as the lists'
-        auto prob = [&](const ListRow& R, int r) -> double {
+        auto prob = [&](const ListRow& R, int r, int slot) -> double {
             if (tok < 0 || tok >= V) return 0.0;
             const __nv_bfloat16* row = r < n_items ? static_cast<const __nv_bfloat16*>(p.P) + (int64_t)r * V
                                                    : static_cast<const __nv_bfloat16*>(p.Q) + (int64_t)(r - n_items) * V;
-            const uint32_t h = reinterpret_cast<const uint16_t*>(row)[tok];
-            if (h & 0x8000u) return 0.0;  // negative: below the window (whose floor is positive)
-            const int d = R.a15 - (int)h;
-            if (d < 0 || d > R.dcut || (d == R.dcut && tok >= R.theta)) return 0.0;
-            return R.lut[d - R.d0] * R.iS;
+            const int h = (int)reinterpret_cast<const uint16_t*>(row)[tok];
+            if (h & 0x8000) return 0.0;  // negative: below the window (whose floor is positive)
+            if (h < R.hcut || (h == R.hcut && tok >= R.theta) || h > R.hM) return 0.0;
+            return sh.lut[slot][R.hM - h] * R.iS;
         };
-        rec.p = prob(P, item);
-        rec.q = two ? prob(Q, n_items + item) : 0.0;
+        rec.p = prob(P, item, 0);
+        rec.q = two ? prob(Q, n_items + item, 1) : 0.0;
         rec.acc = two ? (double)u[1] * rec.q < rec.p : 1;
         if (tid == 0) p.recs[item] = rec;
         rs_mark(p, 2, jm, 4);
