@@ -2127,7 +2127,7 @@ __device__ __forceinline__ void rs_mark(const Params& p, int kernel, int j, int 
     }
 }
 // (kernel 0: rows, 1: items, 2: list items; the end time of each CTA at 6144 + CTA for rows,
-// 7168 + CTA for list items)
+// 7168 + CTA for list items, 8192 + CTA for items)
 __device__ __forceinline__ void rs_end(const Params& p, int base) {
     if (p.trace != nullptr && threadIdx.x == 0 && blockIdx.x < 1024) {
         unsigned long long t;
@@ -2655,8 +2655,36 @@ __global__ void __launch_bounds__(kThreads, CPS) row_kernel(Params p, RowRec* ro
         const int lut_n = p.cut ? (int)min((uint32_t)kLutMax, kM - kc + 1u) : kLutMax;
         for (int j = tid; j < lut_n; j += kThreads)
             out.lut[j] = kM >= (uint32_t)j ? exp((double)bfv(obits(kM - (uint32_t)j)) / T - zmax) : 0.0;
+        // The candidate lists hold every element at or above the window's floor F, so they
+        // serve the list item pass when the cut value is at or above F (the recount only
+        // decided what the bounded sums could not); theta as on the window path.
+        __syncthreads();  // every warp's tie count has landed
+        const uint32_t hcut = p.cut ? obits(kc) : 0u;
+        int lok = p.cut && fast && lists != nullptr && V <= kMaxListV && lut_n <= 255 && !(hcut & 0x8000u) &&
+                  hcut >= F15;
+        for (int w = 0; w < kWarps; ++w) lok &= sh.ln[w] <= kListCap;
+        if (lok) {
+            const int tt = sh.tie_t;
+            int wb = -1, kk = 0, before = 0;
+            for (int w = 0; w < kWarps; ++w) {
+                const int cw = sh.ties[w];
+                if (wb < 0 && tt < before + cw) {
+                    wb = w;
+                    kk = tt - before;
+                }
+                before += cw;
+            }
+            if (warp == (wb < 0 ? 0 : wb)) {
+                const int th = wb < 0 ? INT_MAX : find_tie(gl, gn, hcut, kk, c0 * kCh, lane);
+                if (lane == 0) sh.theta = th;
+            }
+        }
         __syncthreads();
         if (tid == 0) {
+            out.list_ok = lok;
+            out.theta = lok ? sh.theta : INT_MAX;
+            out.A15 = A15;
+            out.dcut = (int)(A15 - hcut);
             out.zmax = zmax;
             out.S = sh.S;
             out.kM = kM;
@@ -3169,6 +3197,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) item_kernel_rs(Params p,
         rs_mark(p, 1, jm, 5);
         if (tid == 0) p.recs[item] = rec;
     }
+    rs_end(p, 8192);
 }
 
 

@@ -12,11 +12,11 @@
 //      top-k of its own run of the row (among the elements at or above a sampled guess)
 //      and writes it out. bf16 rows that are 16-byte aligned take the persistent row
 //      kernel; the rest one CTA per row segment (or the TMA-fed variant);
-//   2. finish: one CTA per sequence; a warp per row merges the row's lists into its exact
-//      top-k (redoing the row when the guess could have hidden part of it), applies softmax
-//      and top-p in fp64 and stores the survivors sorted by token id; the CTA then runs
-//      draft sampling, acceptance, the longest accepted prefix and the residual resample,
-//      one warp per block position.
+//   2. finish: CTAs of 16 warps, a warp per row, merge each row's lists into its exact
+//      top-k (redoing the row when the guess could have hidden part of it), apply softmax
+//      and top-p in fp64 and store the survivors sorted by token id; the CTA that completes
+//      a sequence's rows (per-sequence counters) then runs its draft sampling, acceptance,
+//      longest accepted prefix and residual resample, one warp per block position.
 #include <cuda_bf16.h>
 
 #include <cstdlib>
