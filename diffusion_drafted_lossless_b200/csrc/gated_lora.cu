@@ -59,7 +59,7 @@ struct Params {
     int kt0, kt1;                 // K tiles of (X, W0) and of (T, B)
     int m_tiles;                  // 128-row tiles (T flags, tickets)
     int m_units;                  // row units of the work items: 128 x CG rows
-    int splits, per;              // adapter items: m_tiles x splits, `per` K tiles each
+    int splits, per;              // adapter items: m_units x splits, `per` K tiles each (one T partial each)
     int n_adapter, n_items;       // adapter items, all items
     int n_tiles;                  // column tiles of the output
     int ksplit, kper;             // output items per tile (split over K), K tiles of (X, W0) each
@@ -69,14 +69,12 @@ struct Params {
     uint32_t cb;                  // TMEM columns of one accumulator
     void* y;                      // [M, N] bf16 or fp32
     int out_f32;
-    float* tpart;                 // [splits][M][r] fp32 partials (splits > 1)
     float* ypart;                 // [ksplit][M][N] fp32 partials of the output (ksplit > 1)
     unsigned long long* otickets; // [m_tiles * n_tiles]: (epoch << 16) | output partials stored
-    __nv_bfloat16* t;             // [M][r] bf16 T
+    __nv_bfloat16* t;             // [splits][M][r] bf16 T partials (their sum is T)
     const float* gate;            // [M] or NULL (all zero)
     float scale;
-    unsigned long long* flags;    // [m_tiles]: the epoch once row tile m's T is written
-    unsigned long long* tickets;  // [m_tiles]: (epoch << 16) | partials stored
+    unsigned long long* flags;    // [m_tiles][splits]: the epoch once row tile m's T partial s is written
     unsigned long long* header;   // [5]: the next execution's epoch and exit counter (see Header)
     unsigned long long host_tag;  // lower bound for this execution's epoch (fresh per host call), < 2^48
     uint32_t flag_polls;          // polls of a T flag before the wait gives up
@@ -283,7 +281,7 @@ __device__ __forceinline__ Item decode(const Params& p, int item) {
         it.s = js % p.ksplit;
         it.j = js / p.ksplit;
         it.kb = it.s * p.kper;
-        it.ke = it.s == p.ksplit - 1 ? p.kt0 + p.kt1 : it.kb + p.kper;
+        it.ke = it.s == p.ksplit - 1 ? p.kt0 + p.splits * p.kt1 : it.kb + p.kper;
     }
     return it;
 }
@@ -424,24 +422,29 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
                         *abort_flag = 1;
                         break;
                     }
-                    // rows past M have no T (their loads are zero-filled): nothing to wait for
-                    if (!w.adapter && kt == p.kt0 && m0 < p.M && !wait_flag(&p.flags[m0 / BM], epoch, p.flag_polls)) {
+                    // the (T, B) K tiles run over T's partials in turn: partial ts, its K tile tk
+                    const bool tpart = !w.adapter && kt >= p.kt0;
+                    const int ts = tpart ? (kt - p.kt0) / p.kt1 : 0, tk = tpart ? kt - p.kt0 - ts * p.kt1 : 0;
+                    // rows past M have no T (their loads are zero-filled or not stored): nothing to wait for
+                    if (tpart && tk == 0 && m0 < p.M &&
+                        !wait_flag(&p.flags[(m0 / BM) * p.splits + ts], epoch, p.flag_polls)) {
                         *abort_flag = 1;
                         break;
                     }
                     if (*abort_flag) break;
                     unsigned char* a = sA + (size_t)s * A_BYTES;
                     unsigned char* b = sB + (size_t)s * p.b_bytes;
-                    const CUtensorMap* ma = w.adapter || kt < p.kt0 ? &tX : &tT;
-                    const CUtensorMap* mb = w.adapter ? &tA : (kt < p.kt0 ? &tW0 : &tB);
-                    const int kx = (w.adapter || kt < p.kt0 ? kt : kt - p.kt0) * BK;
+                    const CUtensorMap* ma = tpart ? &tT : &tX;
+                    const CUtensorMap* mb = w.adapter ? &tA : (tpart ? &tB : &tW0);
+                    const int kx = (tpart ? tk : kt) * BK;
+                    const int ma_row = tpart ? ts * p.M + m0 : m0;  // partial ts's rows follow the earlier partials
                     if (leader) mbar_arrive_expect_tx(&full[s], CG * A_BYTES + (uint32_t)nrows * 128u);
                     if constexpr (CG == 2) {
                         const uint32_t bar = lead_full0 + (uint32_t)s * 8u;
-                        tma_load_2d_pair(a, ma, kx, m0, bar);
+                        tma_load_2d_pair(a, ma, kx, ma_row, bar);
                         tma_load_2d_pair(b, mb, kx, n0, bar);
                     } else {
-                        tma_load_2d(a, ma, kx, m0, &full[s]);
+                        tma_load_2d(a, ma, kx, ma_row, &full[s]);
                         tma_load_2d(b, mb, kx, n0, &full[s]);
                     }
                 }
@@ -529,8 +532,8 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
                     tmem_ld32(taddr + (uint32_t)c0, r);
                     if (row >= p.M || c0 >= p.r) continue;
                     const int ncol = min(32, p.r - c0);  // a multiple of 8
-                    if (p.splits == 1) {
-                        __nv_bfloat16* dst = p.t + (size_t)row * p.r + c0;
+                    {
+                        __nv_bfloat16* dst = p.t + ((size_t)w.j * p.M + row) * p.r + c0;
                         for (int j = 0; j < ncol; j += 8) {
                             __nv_bfloat162 h0 = __floats2bfloat162_rn(gs * __uint_as_float(r[j]), gs * __uint_as_float(r[j + 1]));
                             __nv_bfloat162 h1 = __floats2bfloat162_rn(gs * __uint_as_float(r[j + 2]), gs * __uint_as_float(r[j + 3]));
@@ -540,12 +543,6 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
                                 make_uint4(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),
                                            *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
                         }
-                    } else {
-                        float* dst = p.tpart + ((size_t)w.j * p.M + row) * p.r + c0;
-                        for (int j = 0; j < ncol; j += 4)
-                            *reinterpret_cast<float4*>(dst + j) =
-                                make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
-                                            __uint_as_float(r[j + 3]));
                     }
                 }
             } else if (ok) {
@@ -674,45 +671,14 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
                 named_sync_epilogue();
             }
             if (w.adapter) {
-                // publish this CTA's 128 rows of T (all four warps take every barrier)
+                // publish this CTA's 128 rows of T partial w.j (all four warps take every barrier)
                 const int tile = m0 / BM;
                 asm volatile("fence.proxy.async.global;" ::: "memory");
                 __threadfence();
                 named_sync_epilogue();
-                if (p.splits > 1) {
-                    if (et == 0)
-                        s_last = (ok && !*abort_flag && m0 < p.M) ? take_ticket(&p.tickets[tile], epoch, p.splits) : 0;
-                    named_sync_epilogue();
-                    if (s_last) {
-                        // sum the partials of these 128 rows into T
-                        const int r4 = p.r / 4;
-                        for (int idx = et; idx < BM * r4; idx += kEpiThreads) {
-                            const int rr = m0 + idx / r4, c = (idx % r4) * 4;
-                            if (rr >= p.M) continue;
-                            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                            for (int s = 0; s < p.splits; ++s) {
-                                const float4 v = __ldcg(reinterpret_cast<const float4*>(
-                                    p.tpart + ((size_t)s * p.M + rr) * p.r + c));
-                                acc.x += v.x;
-                                acc.y += v.y;
-                                acc.z += v.z;
-                                acc.w += v.w;
-                            }
-                            const float gs = p.gate ? p.scale * p.gate[rr] : 0.f;
-                            __nv_bfloat162 h0 = __floats2bfloat162_rn(gs * acc.x, gs * acc.y);
-                            __nv_bfloat162 h1 = __floats2bfloat162_rn(gs * acc.z, gs * acc.w);
-                            *reinterpret_cast<uint2*>(p.t + (size_t)rr * p.r + c) =
-                                make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
-                        }
-                        asm volatile("fence.proxy.async.global;" ::: "memory");
-                        __threadfence();
-                    }
-                    named_sync_epilogue();
-                    if (et == 0 && s_last && !p.withhold_flags)
-                        asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(&p.flags[tile]), "l"(epoch) : "memory");
-                } else if (et == 0 && ok && m0 < p.M && !p.withhold_flags) {
-                    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(&p.flags[tile]), "l"(epoch) : "memory");
-                }
+                if (et == 0 && ok && m0 < p.M && !p.withhold_flags)
+                    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(&p.flags[tile * p.splits + w.j]), "l"(epoch)
+                                 : "memory");
             }
         }
         if (p.epi_tma && lane == 0) bulk_wait_all();  // this warp's output stores have completed
@@ -795,8 +761,10 @@ struct Plan {
     uint32_t b_bytes, epi_off;
     size_t smem;
     // workspace offsets
-    size_t header, flags, tickets, t, tpart, ypart, otickets, x, w0, a, b, total;
+    size_t header, flags, t, ypart, otickets, x, w0, a, b, total;
 };
+
+int num_sms_cached();
 
 Plan make_plan(int64_t M, int64_t d_in, int64_t d_out, int64_t rank, uno_dtype dtype) {
     Plan P{};
@@ -829,10 +797,28 @@ Plan make_plan(int64_t M, int64_t d_in, int64_t d_out, int64_t rank, uno_dtype d
     while (P.cb < w) P.cb <<= 1;
     P.kt0 = (int)(d_in / BK);
     P.kt1 = (int)((rank + BK - 1) / BK);
-    // One adapter item per row unit: its time is set by streaming the unit's rows of X and
-    // all of A through the SM, not by its MMAs, and summing split partials back in one CTA
-    // costs more than it saves (the split path stays for UNO_LORA_SPLITS=n).
+    // The adapter product X A^T of a row unit is split over K into `splits` items, each of
+    // which writes its own bf16 partial of T; the output tiles run the (T, B) K tiles once
+    // per partial, so no partial is ever summed on its own. An adapter item streams the
+    // unit's rows of X and all of A through one SM, so one item per row unit can take longer
+    // than the output tiles it feeds (the narrow k/v projections): the split is the smallest
+    // that brings an item's operand bytes under half of those of an SM's output work,
+    // without adding a wave of items. UNO_LORA_SPLITS=n fixes it.
     int splits = 1;
+    {
+        const int sms = num_sms_cached();
+        const int64_t out_items = (int64_t)P.m_units * ((d_out + P.BN - 1) / P.BN);
+        const int64_t waves = (out_items + sms - 1) / sms;
+        const double out_bytes = (double)waves * (P.kt0 + P.kt1) * (A_BYTES + (double)P.BN / P.CG * 128.0);
+        const double ad_row = A_BYTES + (double)P.rb / P.CG * 128.0;
+        while (splits < 8) {
+            const int per = (P.kt0 + splits - 1) / splits;
+            if ((double)per * ad_row <= 0.5 * out_bytes) break;
+            const int next = splits + 1;
+            if (out_items <= sms && (int64_t)P.m_units * next + out_items > sms) break;
+            splits = next;
+        }
+    }
     if (const char* e = getenv("UNO_LORA_SPLITS")) splits = atoi(e);
     splits = splits < 1 ? 1 : (splits > P.kt0 ? P.kt0 : splits);
     P.per = (P.kt0 + splits - 1) / splits;
@@ -874,10 +860,8 @@ Plan make_plan(int64_t M, int64_t d_in, int64_t d_out, int64_t rank, uno_dtype d
         return o;
     };
     P.header = take(sizeof(unsigned long long) * 5);
-    P.flags = take((size_t)P.m_tiles * 8);
-    P.tickets = take((size_t)P.m_tiles * 8);
-    P.t = take((size_t)M * rank * 2);
-    P.tpart = P.splits > 1 ? take((size_t)P.splits * M * rank * 4) : 0;
+    P.flags = take((size_t)P.m_tiles * P.splits * 8);
+    P.t = take((size_t)P.splits * M * rank * 2);
     P.ypart = P.ksplit > 1 ? take((size_t)P.ksplit * M * d_out * 4) : 0;
     P.otickets = P.ksplit > 1 ? take((size_t)P.m_tiles * P.n_tiles * 8) : 0;
     if (dtype == UNO_F32) {
@@ -996,7 +980,7 @@ uno_status gated_lora_launch(const GatedLoraArgs& g, void* workspace, cudaStream
     if ((s = make_tmap(&maps[0], x, M, din, BM)) != UNO_OK) return s;              // X
     if ((s = make_tmap(&maps[1], w0, dout, din, P.BN / cg)) != UNO_OK) return s;   // W0
     if ((s = make_tmap(&maps[2], a, r, din, P.rb / cg)) != UNO_OK) return s;       // A
-    if ((s = make_tmap(&maps[3], t, M, r, BM)) != UNO_OK) return s;                // T
+    if ((s = make_tmap(&maps[3], t, (int64_t)P.splits * M, r, BM)) != UNO_OK) return s;  // T partials
     if ((s = make_tmap(&maps[4], b, dout, r, P.BN / cg)) != UNO_OK) return s;      // B
     if (P.epi_tma) {
         if ((s = make_tmap_store(&maps[5], g.y, M, dout)) != UNO_OK) return s;     // Y (stores)
@@ -1026,12 +1010,10 @@ uno_status gated_lora_launch(const GatedLoraArgs& g, void* workspace, cudaStream
     p.cb = (uint32_t)P.cb;
     p.y = g.y;
     p.out_f32 = g.dtype == UNO_F32;
-    p.tpart = P.splits > 1 ? reinterpret_cast<float*>(ws + P.tpart) : nullptr;
     p.t = t;
     p.gate = g.gate;
     p.scale = g.scale;
     p.flags = reinterpret_cast<unsigned long long*>(ws + P.flags);
-    p.tickets = reinterpret_cast<unsigned long long*>(ws + P.tickets);
     p.header = reinterpret_cast<unsigned long long*>(ws + P.header);
     p.host_tag = next_epoch();
     // UNO_LORA_TEST_WITHHOLD_FLAGS=1 (tests of the failure path only): the adapter items keep

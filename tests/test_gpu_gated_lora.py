@@ -171,8 +171,9 @@ def test_calls_back_to_back_on_one_workspace():
 
 @pytest.mark.parametrize("splits", ["3", "64"])
 def test_split_adapter_path(monkeypatch, splits):
-    """The adapter product split over K (partials summed by the item that completes a row
-    tile) gives the same result; 64 splits exceed the K tiles and are clamped."""
+    """The adapter product split over K into bf16 partials of T, each run through the output
+    tiles' (T, B) K tiles in turn, gives the oracle's result; 64 splits exceed the K tiles
+    and are clamped."""
     monkeypatch.setenv("UNO_LORA_SPLITS", splits)
     for M, d_in, d_out, r in [(300, 1024, 256, 64), (1000, 768, 1024, 256), (129, 256, 640, 128)]:
         w = W.GatedLoraWorkload("t", 5 + M, M=M, block=8, rank=r, scale=2.0,
