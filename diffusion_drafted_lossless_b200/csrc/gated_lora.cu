@@ -81,6 +81,7 @@ struct Params {
     int epi_tma;                  // bf16 output tiles leave through shared memory and TMA stores
     uint32_t epi_off;             // byte offset of the epilogue staging buffers in dynamic smem
     int withhold_flags;           // test switch: adapter items do not publish T (every wait on it runs out)
+    long long* trace;             // UNO_LORA_TRACE (profiling aid): per-K-step SM clocks of three CTAs, or NULL
     uint32_t* status;
 };
 
@@ -335,6 +336,14 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t bar) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+// UNO_LORA_TRACE: SM clock at event e (0: loads issued, 1: stage landed, 2: MMAs committed)
+// of K step g, for CTAs 0, 20 and 100
+__device__ __forceinline__ void gl_mark(const Params& p, int e, uint32_t g) {
+    if (p.trace == nullptr || g >= 512) return;
+    const int slot = blockIdx.x == 0 ? 0 : (blockIdx.x == 20 ? 1 : (blockIdx.x == 100 ? 2 : -1));
+    if (slot >= 0) p.trace[(slot * 6 + e) * 512 + g] = clock64();
+}
+
 // CG = 1: one CTA computes a 128 x N tile. CG = 2: the two CTAs of a cluster compute a
 // 256 x N tile with one MMA stream issued by the leader (rank 0): each CTA holds its 128
 // rows of A and half of the N rows of B, and its own 128-lane accumulator.
@@ -410,43 +419,60 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
         if (lane == 0) {
             // ---- TMA producer (each CTA loads its own rows of A and its half of B) ----
             const uint32_t lead_full0 = CG == 2 ? map_to_rank(&full[0], 0) : 0u;
-            uint32_t g = 0;  // K steps issued by this CTA, across items
+            // (the parameters the loop reads, in registers: every asm statement below clobbers memory)
+            const int kt0 = p.kt0, kt1 = p.kt1, M = p.M, splits = p.splits, rb = p.rb;
+            const uint32_t bbytes = p.b_bytes, polls = p.flag_polls;
+            unsigned long long* const flags = p.flags;
+            uint32_t g = 0;       // K steps issued by this CTA, across items
+            int s = 0;            // their stage: g mod ST
+            uint32_t ph = 0;      // and its pass over the ring, mod 2
             for (int item = unit0; item < p.n_items && !*abort_flag; item += units) {
                 const Item w = decode(p, item);
                 const int m0 = w.m * BM * CG + (int)rank * BM;
-                const int nrows = w.adapter ? p.rb : BN;  // B rows of the whole (pair) tile
+                const int nrows = w.adapter ? rb : BN;  // B rows of the whole (pair) tile
                 const int n0 = w.adapter ? (int)rank * (nrows / CG) : w.j * BN + (int)rank * (BN / CG);
+                const uint32_t tx = CG * A_BYTES + (uint32_t)nrows * 128u;
+                int ts = 0, tk = 0;  // the (T, B) K tiles run over T's partials in turn: partial ts, its K tile tk
                 for (int kt = w.kb; kt < w.ke; ++kt, ++g) {
-                    const int s = (int)(g % ST);
-                    if (g >= (uint32_t)ST && !mbar_wait(&empty[s], ((g / ST) & 1) ^ 1)) {
+                    gl_mark(p, 5, g);
+                    if (g >= (uint32_t)ST && !mbar_wait(&empty[s], ph ^ 1u)) {
                         *abort_flag = 1;
                         break;
                     }
-                    // the (T, B) K tiles run over T's partials in turn: partial ts, its K tile tk
-                    const bool tpart = !w.adapter && kt >= p.kt0;
-                    const int ts = tpart ? (kt - p.kt0) / p.kt1 : 0, tk = tpart ? kt - p.kt0 - ts * p.kt1 : 0;
+                    const bool tpart = !w.adapter && kt >= kt0;
                     // rows past M have no T (their loads are zero-filled or not stored): nothing to wait for
-                    if (tpart && tk == 0 && m0 < p.M &&
-                        !wait_flag(&p.flags[(m0 / BM) * p.splits + ts], epoch, p.flag_polls)) {
+                    if (tpart && tk == 0 && m0 < M && !wait_flag(&flags[(m0 / BM) * splits + ts], epoch, polls)) {
                         *abort_flag = 1;
                         break;
                     }
                     if (*abort_flag) break;
                     unsigned char* a = sA + (size_t)s * A_BYTES;
-                    unsigned char* b = sB + (size_t)s * p.b_bytes;
+                    unsigned char* b = sB + (size_t)s * bbytes;
                     const CUtensorMap* ma = tpart ? &tT : &tX;
                     const CUtensorMap* mb = w.adapter ? &tA : (tpart ? &tB : &tW0);
                     const int kx = (tpart ? tk : kt) * BK;
-                    const int ma_row = tpart ? ts * p.M + m0 : m0;  // partial ts's rows follow the earlier partials
-                    if (leader) mbar_arrive_expect_tx(&full[s], CG * A_BYTES + (uint32_t)nrows * 128u);
+                    const int ma_row = tpart ? ts * M + m0 : m0;  // partial ts's rows follow the earlier partials
+                    if (tpart && ++tk == kt1) {
+                        tk = 0;
+                        ++ts;
+                    }
+                    const int st = s;
+                    if (++s == ST) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                    gl_mark(p, 3, g);
+                    if (leader) mbar_arrive_expect_tx(&full[st], tx);
                     if constexpr (CG == 2) {
-                        const uint32_t bar = lead_full0 + (uint32_t)s * 8u;
+                        const uint32_t bar = lead_full0 + (uint32_t)st * 8u;
                         tma_load_2d_pair(a, ma, kx, ma_row, bar);
                         tma_load_2d_pair(b, mb, kx, n0, bar);
                     } else {
-                        tma_load_2d(a, ma, kx, ma_row, &full[s]);
-                        tma_load_2d(b, mb, kx, n0, &full[s]);
+                        tma_load_2d(a, ma, kx, ma_row, &full[st]);
+                        gl_mark(p, 4, g);
+                        tma_load_2d(b, mb, kx, n0, &full[st]);
                     }
+                    gl_mark(p, 0, g);
                 }
             }
             // on abort: wait (bounded) for the loads that no MMA will consume
@@ -458,7 +484,11 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
     } else if (warp == 1) {
         if (lane == 0 && leader) {
             // ---- MMA issuer (one thread of the leader CTA) ----
+            const uint32_t cb = p.cb, rb = (uint32_t)p.rb, bbytes = p.b_bytes;
+            const uint64_t da0 = smem_desc_sw128(smem_u32(sA)), db0 = smem_desc_sw128(smem_u32(sB));
             uint32_t g = 0, li = 0;
+            int s = 0;        // stage of K step g
+            uint32_t ph = 0;  // its pass over the ring, mod 2
             for (int item = unit0; item < p.n_items && !*abort_flag; item += units, ++li) {
                 const Item w = decode(p, item);
                 const int buf = li & 1;
@@ -467,29 +497,37 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
                     break;
                 }
                 tmem_fence_after();
-                const uint32_t d = tmem + (uint32_t)buf * p.cb;
-                const uint32_t idesc = instr_desc_bf16(BM * CG, w.adapter ? p.rb : BN);
+                const uint32_t d = tmem + (uint32_t)buf * cb;
+                const uint32_t idesc = instr_desc_bf16(BM * CG, w.adapter ? (int)rb : BN);
                 bool ok = true;
                 for (int kt = w.kb; kt < w.ke; ++kt, ++g) {
-                    const int s = (int)(g % ST);
-                    if (!wait_or_abort(&full[s], (g / ST) & 1, abort_flag)) {
+                    if (!wait_or_abort(&full[s], ph, abort_flag)) {
                         ok = false;
                         break;
                     }
+                    gl_mark(p, 1, g);
                     tmem_fence_after();
-                    const uint32_t a0 = smem_u32(sA + (size_t)s * A_BYTES), b0 = smem_u32(sB + (size_t)s * p.b_bytes);
+                    // descriptors of this stage's tiles: the start-address field (address >> 4)
+                    // of the ring's base plus the stage offset (no carry: shared addresses < 2^18)
+                    const uint64_t da = da0 + (uint64_t)(((uint32_t)s * A_BYTES) >> 4);
+                    const uint64_t db = db0 + (uint64_t)(((uint32_t)s * bbytes) >> 4);
 #pragma unroll
                     for (int kk = 0; kk < BK / UMMA_K; ++kk) {
-                        const uint32_t off = kk * UMMA_K * 2;  // bytes along K within the 128-byte row
+                        const uint64_t off = (uint64_t)((kk * UMMA_K * 2) >> 4);  // 32 bytes along K per step
                         const uint32_t acc = (kt > w.kb || kk > 0) ? 1u : 0u;
                         if constexpr (CG == 2)
-                            umma_bf16_pair(d, smem_desc_sw128(a0 + off), smem_desc_sw128(b0 + off), idesc, acc);
+                            umma_bf16_pair(d, da + off, db + off, idesc, acc);
                         else
-                            umma_bf16(d, smem_desc_sw128(a0 + off), smem_desc_sw128(b0 + off), idesc, acc);
+                            umma_bf16(d, da + off, db + off, idesc, acc);
                     }
                     // the stage is free (in both CTAs) once these MMAs have read it
                     if constexpr (CG == 2) umma_commit_pair(&empty[s]);
                     else umma_commit(&empty[s]);
+                    gl_mark(p, 2, g);
+                    if (++s == ST) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
                 if (!ok) {
                     *abort_flag = 1;
@@ -761,7 +799,7 @@ struct Plan {
     uint32_t b_bytes, epi_off;
     size_t smem;
     // workspace offsets
-    size_t header, flags, t, ypart, otickets, x, w0, a, b, total;
+    size_t header, flags, t, ypart, otickets, x, w0, a, b, trace, total;
 };
 
 int num_sms_cached();
@@ -781,8 +819,19 @@ Plan make_plan(int64_t M, int64_t d_in, int64_t d_out, int64_t rank, uno_dtype d
     if (P.CG == 2) {
         P.BN = 256;
     } else {
-        P.BN = 256;
-        while (P.BN > 64 && (int64_t)P.m_tiles * ((d_out + P.BN - 1) / P.BN) < 120) P.BN >>= 1;
+        // A K step takes about as long at every tile width (its operand loads set the pace),
+        // so the width is the one with the fewest waves of items over the SMs, the wider on a
+        // tie (ranked by waves x (1 + BN / 1024)); two adapter items per row tile count too.
+        const int sms = num_sms_cached();
+        double best = 0.0;
+        for (int bn = 256; bn >= 64; bn >>= 1) {
+            const int64_t items = (int64_t)P.m_tiles * ((d_out + bn - 1) / bn + 2);
+            const double cost = (double)((items + sms - 1) / sms) * (1.0 + bn / 1024.0);
+            if (bn == 256 || cost < best) {
+                best = cost;
+                P.BN = bn;
+            }
+        }
         // UNO_LORA_BN (64, 128 or 256) fixes the tile width, for measurements
         if (const char* e = getenv("UNO_LORA_BN")) {
             const int bn = atoi(e);
@@ -799,26 +848,12 @@ Plan make_plan(int64_t M, int64_t d_in, int64_t d_out, int64_t rank, uno_dtype d
     P.kt1 = (int)((rank + BK - 1) / BK);
     // The adapter product X A^T of a row unit is split over K into `splits` items, each of
     // which writes its own bf16 partial of T; the output tiles run the (T, B) K tiles once
-    // per partial, so no partial is ever summed on its own. An adapter item streams the
-    // unit's rows of X and all of A through one SM, so one item per row unit can take longer
-    // than the output tiles it feeds (the narrow k/v projections): the split is the smallest
-    // that brings an item's operand bytes under half of those of an SM's output work,
-    // without adding a wave of items. UNO_LORA_SPLITS=n fixes it.
-    int splits = 1;
-    {
-        const int sms = num_sms_cached();
-        const int64_t out_items = (int64_t)P.m_units * ((d_out + P.BN - 1) / P.BN);
-        const int64_t waves = (out_items + sms - 1) / sms;
-        const double out_bytes = (double)waves * (P.kt0 + P.kt1) * (A_BYTES + (double)P.BN / P.CG * 128.0);
-        const double ad_row = A_BYTES + (double)P.rb / P.CG * 128.0;
-        while (splits < 8) {
-            const int per = (P.kt0 + splits - 1) / splits;
-            if ((double)per * ad_row <= 0.5 * out_bytes) break;
-            const int next = splits + 1;
-            if (out_items <= sms && (int64_t)P.m_units * next + out_items > sms) break;
-            splits = next;
-        }
-    }
+    // per partial, so no partial is ever summed on its own. Two partials measured fastest
+    // on every Qwen3-8B and looped-3B projection (an adapter item streams the unit's rows of
+    // X and all of A through one SM; halving that keeps it off the output tiles' critical
+    // path, while more partials add (T, B) K tiles to every output tile, or a wave of items).
+    // UNO_LORA_SPLITS=n fixes it.
+    int splits = P.kt0 >= 2 ? 2 : 1;
     if (const char* e = getenv("UNO_LORA_SPLITS")) splits = atoi(e);
     splits = splits < 1 ? 1 : (splits > P.kt0 ? P.kt0 : splits);
     P.per = (P.kt0 + splits - 1) / splits;
@@ -870,6 +905,7 @@ Plan make_plan(int64_t M, int64_t d_in, int64_t d_out, int64_t rank, uno_dtype d
         P.a = take((size_t)rank * d_in * 2);
         P.b = take((size_t)d_out * rank * 2);
     }
+    P.trace = getenv("UNO_LORA_TRACE") ? take((size_t)3 * 6 * 512 * 8) : 0;
     P.total = off;
     return P;
 }
@@ -1029,6 +1065,7 @@ uno_status gated_lora_launch(const GatedLoraArgs& g, void* workspace, cudaStream
             p.flag_polls = 4096;
         }
     p.status = device_status_ptr();
+    p.trace = getenv("UNO_LORA_TRACE") ? reinterpret_cast<long long*>(ws + P.trace) : nullptr;
     if (P.CG == 2) return launch_t<256, 2>(maps, p, P, stream);
     switch (P.BN) {
         case 64: return launch_t<64, 1>(maps, p, P, stream);
