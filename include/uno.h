@@ -30,18 +30,22 @@
  *   - Device pointers must be 16-byte aligned (uno_block_noise: 4-byte aligned).
  *   - bf16 is IEEE-754 binary32 truncated to its upper 16 bits (1-8-7), stored as uint16.
  *
- * Kernel variants (environment, read at each call, UNO_VERIFY_SEGMENTS at the first; every
- * variant computes the same result up to floating-point summation order, and the defaults
- * are the fastest measured ones)
+ * Kernel variants (environment, read at each call; every variant computes the same result
+ * up to floating-point summation order, and the defaults are the fastest measured ones)
  *   UNO_LORA_CG=2            gated LoRA on CTA pairs (256-row tiles, cta_group::2)
- *   UNO_LORA_SPLITS=n        adapter product X A^T split over K into n partials
+ *   UNO_LORA_BN=64|128|256   gated LoRA output tile width
+ *   UNO_LORA_SPLITS=n        adapter product X A^T split over K into n bf16 partials of T
  *   UNO_LORA_KSPLIT=n        output tiles split over K into n fp32 partials
- *   UNO_VERIFY_STREAM=tma    top-k verify rows streamed by bulk copies into shared memory
- *   UNO_VERIFY_SEGMENTS=n    top-k verify: CTAs per row in the streaming pass (1 to 8)
- *   UNO_VERIFY_FULL=rows     full-vocabulary verify: one CTA per row (no cluster form);
+ *   UNO_LORA_EPI=rows        output tiles stored by lanes (no shared-memory staging)
+ *   UNO_VERIFY_STREAM=warps|tma  top-k verify: per-segment streaming CTAs (register or bulk-copy fed)
+ *   UNO_VERIFY_SEGMENTS=n    top-k verify with UNO_VERIFY_STREAM=warps: CTAs per row (1 to 8)
+ *   UNO_VERIFY_TOPK=local|window  top-k verify on the cluster kernels
+ *   UNO_VERIFY_FULL=generic  full-vocabulary verify: one CTA per item, fp64 exp per token;
  *                  =cluster  the cluster form or UNO_ERR_UNSUPPORTED
- *   UNO_VERIFY_FULL_CLUSTER=c  full-vocabulary verify: clusters of c CTAs (1, 2, 4, 8, 16)
- *   UNO_TV_KERNEL=rows       TV loss: one CTA per row (no cluster form)
+ *   UNO_VERIFY_FULL_CLUSTER=c  full-vocabulary cluster form: clusters of c CTAs
+ *   UNO_VERIFY_LISTS=off     full-vocabulary verify without candidate lists
+ *   UNO_VERIFY_ROW_CTAS=2    full-vocabulary row pass: two CTAs per SM
+ *   UNO_TV_KERNEL=rows|teams TV loss: one CTA per row / two teams per CTA
  *   UNO_TV_CLUSTER=c         TV loss: clusters of c CTAs
  * A workspace must be sized under the same settings as the call that uses it.
  */
