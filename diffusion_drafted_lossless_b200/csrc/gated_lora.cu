@@ -65,7 +65,8 @@ struct Params {
     int ksplit, kper;             // output items per tile (split over K), K tiles of (X, W0) each
     int rb;                       // adapter accumulator width: r rounded up to 16 x CG
     int stages;                   // shared-memory ring depth
-    uint32_t b_bytes;             // bytes of one B-operand stage (max(BN, rb) rows)
+    uint32_t b_bytes;             // bytes of one B-operand K slab (max(BN, rb) rows of 64 elements)
+    int ws;                       // K slabs per main K step (1 or 2: X/W0/A loads are 3-D boxes of ws slabs)
     uint32_t cb;                  // TMEM columns of one accumulator
     void* y;                      // [M, N] bf16 or fp32
     int out_f32;
@@ -93,6 +94,16 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
             smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+
+// a 3-D box (x fastest): here 64 columns x rows x K slabs of a row-major matrix, landing in
+// shared memory slab after slab
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
         : "memory");
 }
 
@@ -362,8 +373,10 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
     // 128-byte swizzled tiles need 1024-byte aligned shared-memory addresses
     unsigned char* smem = smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u);
     const int ST = p.stages;
+    const int WS = CG == 1 ? p.ws : 1;                 // K slabs per main K step
+    const uint32_t a_stage = (uint32_t)WS * A_BYTES;  // bytes of a stage's A tiles
     unsigned char* sA = smem;
-    unsigned char* sB = smem + (size_t)ST * A_BYTES;
+    unsigned char* sB = smem + (size_t)ST * a_stage;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int* abort_flag = &s_abort;
@@ -421,7 +434,7 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
             const uint32_t lead_full0 = CG == 2 ? map_to_rank(&full[0], 0) : 0u;
             // (the parameters the loop reads, in registers: every asm statement below clobbers memory)
             const int kt0 = p.kt0, kt1 = p.kt1, M = p.M, splits = p.splits, rb = p.rb;
-            const uint32_t bbytes = p.b_bytes, polls = p.flag_polls;
+            const uint32_t bbytes = (uint32_t)WS * p.b_bytes, polls = p.flag_polls;
             unsigned long long* const flags = p.flags;
             uint32_t g = 0;       // K steps issued by this CTA, across items
             int s = 0;            // their stage: g mod ST
@@ -431,7 +444,7 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
                 const int m0 = w.m * BM * CG + (int)rank * BM;
                 const int nrows = w.adapter ? rb : BN;  // B rows of the whole (pair) tile
                 const int n0 = w.adapter ? (int)rank * (nrows / CG) : w.j * BN + (int)rank * (BN / CG);
-                const uint32_t tx = CG * A_BYTES + (uint32_t)nrows * 128u;
+                const uint32_t tx1 = CG * A_BYTES + (uint32_t)nrows * 128u;  // bytes of one K slab
                 int ts = 0, tk = 0;  // the (T, B) K tiles run over T's partials in turn: partial ts, its K tile tk
                 for (int kt = w.kb; kt < w.ke; ++kt, ++g) {
                     gl_mark(p, 5, g);
@@ -446,7 +459,7 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
                         break;
                     }
                     if (*abort_flag) break;
-                    unsigned char* a = sA + (size_t)s * A_BYTES;
+                    unsigned char* a = sA + (size_t)s * a_stage;
                     unsigned char* b = sB + (size_t)s * bbytes;
                     const CUtensorMap* ma = tpart ? &tT : &tX;
                     const CUtensorMap* mb = w.adapter ? &tA : (tpart ? &tB : &tW0);
@@ -462,15 +475,21 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
                         ph ^= 1u;
                     }
                     gl_mark(p, 3, g);
-                    if (leader) mbar_arrive_expect_tx(&full[st], tx);
+                    if (leader) mbar_arrive_expect_tx(&full[st], tpart ? tx1 : (uint32_t)WS * tx1);
                     if constexpr (CG == 2) {
                         const uint32_t bar = lead_full0 + (uint32_t)st * 8u;
                         tma_load_2d_pair(a, ma, kx, ma_row, bar);
                         tma_load_2d_pair(b, mb, kx, n0, bar);
                     } else {
-                        tma_load_2d(a, ma, kx, ma_row, &full[st]);
-                        gl_mark(p, 4, g);
-                        tma_load_2d(b, mb, kx, n0, &full[st]);
+                        if (tpart) {
+                            tma_load_2d(a, ma, kx, ma_row, &full[st]);
+                            gl_mark(p, 4, g);
+                            tma_load_2d(b, mb, kx, n0, &full[st]);
+                        } else {  // X, W0 and A are 3-D maps: WS K slabs in one box each
+                            tma_load_3d(a, ma, 0, ma_row, kt * WS, &full[st]);
+                            gl_mark(p, 4, g);
+                            tma_load_3d(b, mb, 0, n0, kt * WS, &full[st]);
+                        }
                     }
                     gl_mark(p, 0, g);
                 }
@@ -484,7 +503,8 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
     } else if (warp == 1) {
         if (lane == 0 && leader) {
             // ---- MMA issuer (one thread of the leader CTA) ----
-            const uint32_t cb = p.cb, rb = (uint32_t)p.rb, bbytes = p.b_bytes;
+            const uint32_t cb = p.cb, rb = (uint32_t)p.rb, bbytes = (uint32_t)WS * p.b_bytes;
+            const int kt0 = p.kt0;
             const uint64_t da0 = smem_desc_sw128(smem_u32(sA)), db0 = smem_desc_sw128(smem_u32(sB));
             uint32_t g = 0, li = 0;
             int s = 0;        // stage of K step g
@@ -509,16 +529,23 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
                     tmem_fence_after();
                     // descriptors of this stage's tiles: the start-address field (address >> 4)
                     // of the ring's base plus the stage offset (no carry: shared addresses < 2^18)
-                    const uint64_t da = da0 + (uint64_t)(((uint32_t)s * A_BYTES) >> 4);
+                    const uint64_t da = da0 + (uint64_t)(((uint32_t)s * a_stage) >> 4);
                     const uint64_t db = db0 + (uint64_t)(((uint32_t)s * bbytes) >> 4);
+                    // a main step holds WS K slabs (slab j of B at j x its box rows x 128 bytes);
+                    // a (T, B) step one
+                    const int slabs = (!w.adapter && kt >= kt0) ? 1 : WS;
+                    const uint32_t bslab = ((w.adapter ? rb : (uint32_t)BN) / CG * 128u) >> 4;
+                    for (int sl = 0; sl < slabs; ++sl) {
 #pragma unroll
-                    for (int kk = 0; kk < BK / UMMA_K; ++kk) {
-                        const uint64_t off = (uint64_t)((kk * UMMA_K * 2) >> 4);  // 32 bytes along K per step
-                        const uint32_t acc = (kt > w.kb || kk > 0) ? 1u : 0u;
-                        if constexpr (CG == 2)
-                            umma_bf16_pair(d, da + off, db + off, idesc, acc);
-                        else
-                            umma_bf16(d, da + off, db + off, idesc, acc);
+                        for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+                            const uint64_t off = (uint64_t)((kk * UMMA_K * 2) >> 4);  // 32 bytes along K per step
+                            const uint32_t acc = (kt > w.kb || sl > 0 || kk > 0) ? 1u : 0u;
+                            const uint64_t oa = off + (uint64_t)sl * (A_BYTES >> 4), ob = off + (uint64_t)sl * bslab;
+                            if constexpr (CG == 2)
+                                umma_bf16_pair(d, da + oa, db + ob, idesc, acc);
+                            else
+                                umma_bf16(d, da + oa, db + ob, idesc, acc);
+                        }
                     }
                     // the stage is free (in both CTAs) once these MMAs have read it
                     if constexpr (CG == 2) umma_commit_pair(&empty[s]);
@@ -774,6 +801,22 @@ uno_status make_tmap(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols
     return UNO_OK;
 }
 
+// row-major [rows, cols] bf16 matrix (cols a multiple of 64) seen as 64 columns x rows x
+// cols / 64 K slabs: a box of 64 columns x box_rows rows x slabs, 128-byte swizzle
+uno_status make_tmap3(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols, int box_rows, int slabs) {
+    auto fn = encode_fn();
+    if (!fn) return set_error(UNO_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    cuuint64_t gdim[3] = {(cuuint64_t)BK, (cuuint64_t)rows, (cuuint64_t)(cols / BK)};
+    cuuint64_t gstride[2] = {(cuuint64_t)cols * 2, (cuuint64_t)BK * 2};
+    cuuint32_t box[3] = {(cuuint32_t)BK, (cuuint32_t)box_rows, (cuuint32_t)slabs};
+    cuuint32_t estride[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), gdim, gstride, box, estride,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return set_error(UNO_ERR_CUDA, "cuTensorMapEncodeTiled (3-D) failed (%d)", (int)r);
+    return UNO_OK;
+}
+
 // row-major [rows, cols] bf16 output, 32 x 32 boxes with 64-byte swizzle (the epilogue's
 // staging layout)
 uno_status make_tmap_store(CUtensorMap* m, void* ptr, int64_t rows, int64_t cols) {
@@ -793,7 +836,7 @@ uno_status make_tmap_store(CUtensorMap* m, void* ptr, int64_t rows, int64_t cols
 
 // The launch plan of one call (also sizes the workspace).
 struct Plan {
-    int CG, BN, rb, cb, m_tiles, m_units, n_tiles, kt0, kt1, splits, per, n_adapter, n_items, stages;
+    int CG, BN, rb, cb, m_tiles, m_units, n_tiles, kt0, kt1, splits, per, n_adapter, n_items, stages, ws;
     int ksplit, kper;
     int epi_tma;
     uint32_t b_bytes, epi_off;
@@ -844,7 +887,14 @@ Plan make_plan(int64_t M, int64_t d_in, int64_t d_out, int64_t rank, uno_dtype d
     const int w = P.BN > P.rb ? P.BN : P.rb;  // N of the widest MMA
     P.cb = 32;
     while (P.cb < w) P.cb <<= 1;
-    P.kt0 = (int)(d_in / BK);
+    // Main K steps of WS = 2 slabs of 64 (one 3-D TMA box per operand): a stage lands about
+    // every thousand SM clocks whatever its bytes (a per-load cost, measured with
+    // UNO_LORA_TRACE at 24 to 48 KB per stage), so two slabs per load nearly halve the count
+    // of loads. UNO_LORA_WIDE=0 keeps one slab per step; CTA pairs keep one.
+    P.ws = (P.CG == 1 && (d_in / BK) % 2 == 0) ? 2 : 1;
+    if (const char* e = getenv("UNO_LORA_WIDE"))
+        if (atoi(e) == 0) P.ws = 1;
+    P.kt0 = (int)(d_in / BK) / P.ws;
     P.kt1 = (int)((rank + BK - 1) / BK);
     // The adapter product X A^T of a row unit is split over K into `splits` items, each of
     // which writes its own bf16 partial of T; the output tiles run the (T, B) K tiles once
@@ -879,14 +929,14 @@ Plan make_plan(int64_t M, int64_t d_in, int64_t d_out, int64_t rank, uno_dtype d
     if (const char* e = getenv("UNO_LORA_EPI"))
         if (strcmp(e, "rows") == 0) P.epi_tma = 0;
     const uint32_t epi_bytes = P.epi_tma ? 4u * 4096u : 0u;
-    P.stages = (int)((kSmemBudget - 1024 - epi_bytes) / (A_BYTES + P.b_bytes));
+    P.stages = (int)((kSmemBudget - 1024 - epi_bytes) / ((uint32_t)P.ws * (A_BYTES + P.b_bytes)));
     if (P.stages > kMaxStages) P.stages = kMaxStages;
     // UNO_LORA_STAGES=n (2 up to what fits) shortens the ring, for measurements
     if (const char* e = getenv("UNO_LORA_STAGES")) {
         const int st = atoi(e);
         if (st >= 2 && st < P.stages) P.stages = st;
     }
-    P.epi_off = (uint32_t)align_up((size_t)P.stages * (A_BYTES + P.b_bytes), 1024);
+    P.epi_off = (uint32_t)align_up((size_t)P.stages * P.ws * (A_BYTES + P.b_bytes), 1024);
     P.smem = (size_t)P.epi_off + epi_bytes + 1024;
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -1013,9 +1063,15 @@ uno_status gated_lora_launch(const GatedLoraArgs& g, void* workspace, cudaStream
     __nv_bfloat16* t = reinterpret_cast<__nv_bfloat16*>(ws + P.t);
     CUtensorMap maps[6];
     const int cg = P.CG;
-    if ((s = make_tmap(&maps[0], x, M, din, BM)) != UNO_OK) return s;              // X
-    if ((s = make_tmap(&maps[1], w0, dout, din, P.BN / cg)) != UNO_OK) return s;   // W0
-    if ((s = make_tmap(&maps[2], a, r, din, P.rb / cg)) != UNO_OK) return s;       // A
+    if (cg == 1) {  // X, W0, A: boxes of P.ws K slabs
+        if ((s = make_tmap3(&maps[0], x, M, din, BM, P.ws)) != UNO_OK) return s;
+        if ((s = make_tmap3(&maps[1], w0, dout, din, P.BN, P.ws)) != UNO_OK) return s;
+        if ((s = make_tmap3(&maps[2], a, r, din, P.rb, P.ws)) != UNO_OK) return s;
+    } else {
+        if ((s = make_tmap(&maps[0], x, M, din, BM)) != UNO_OK) return s;              // X
+        if ((s = make_tmap(&maps[1], w0, dout, din, P.BN / cg)) != UNO_OK) return s;   // W0
+        if ((s = make_tmap(&maps[2], a, r, din, P.rb / cg)) != UNO_OK) return s;       // A
+    }
     if ((s = make_tmap(&maps[3], t, (int64_t)P.splits * M, r, BM)) != UNO_OK) return s;  // T partials
     if ((s = make_tmap(&maps[4], b, dout, r, P.BN / cg)) != UNO_OK) return s;      // B
     if (P.epi_tma) {
@@ -1043,6 +1099,7 @@ uno_status gated_lora_launch(const GatedLoraArgs& g, void* workspace, cudaStream
     p.rb = P.rb;
     p.stages = P.stages;
     p.b_bytes = P.b_bytes;
+    p.ws = P.ws;
     p.cb = (uint32_t)P.cb;
     p.y = g.y;
     p.out_f32 = g.dtype == UNO_F32;
