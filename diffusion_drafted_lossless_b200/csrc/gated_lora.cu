@@ -321,6 +321,13 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
         : "memory");
 }
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, int x, int y, int z, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
 __device__ __forceinline__ void umma_bf16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                                uint32_t accumulate) {
     asm volatile(
@@ -373,7 +380,7 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
     // 128-byte swizzled tiles need 1024-byte aligned shared-memory addresses
     unsigned char* smem = smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u);
     const int ST = p.stages;
-    const int WS = CG == 1 ? p.ws : 1;                 // K slabs per main K step
+    const int WS = p.ws;                               // K slabs per main K step
     const uint32_t a_stage = (uint32_t)WS * A_BYTES;  // bytes of a stage's A tiles
     unsigned char* sA = smem;
     unsigned char* sB = smem + (size_t)ST * a_stage;
@@ -478,8 +485,13 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
                     if (leader) mbar_arrive_expect_tx(&full[st], tpart ? tx1 : (uint32_t)WS * tx1);
                     if constexpr (CG == 2) {
                         const uint32_t bar = lead_full0 + (uint32_t)st * 8u;
-                        tma_load_2d_pair(a, ma, kx, ma_row, bar);
-                        tma_load_2d_pair(b, mb, kx, n0, bar);
+                        if (tpart) {
+                            tma_load_2d_pair(a, ma, kx, ma_row, bar);
+                            tma_load_2d_pair(b, mb, kx, n0, bar);
+                        } else {
+                            tma_load_3d_pair(a, ma, 0, ma_row, kt * WS, bar);
+                            tma_load_3d_pair(b, mb, 0, n0, kt * WS, bar);
+                        }
                     } else {
                         if (tpart) {
                             tma_load_2d(a, ma, kx, ma_row, &full[st]);
@@ -850,13 +862,17 @@ int num_sms_cached();
 Plan make_plan(int64_t M, int64_t d_in, int64_t d_out, int64_t rank, uno_dtype dtype) {
     Plan P{};
     P.m_tiles = (int)((M + BM - 1) / BM);
-    // Single-CTA 128 x BN tiles. The CTA-pair form (256 x 256 tiles, one MMA stream over two
-    // SMs, each loading half of B) is selected with UNO_LORA_CG=2; on the Qwen3-8B and
-    // looped-3B shapes it measured no faster, so it is not the default.
-    P.CG = 1;
+    // The CTA-pair form (256 x 256 tiles, one MMA stream over two SMs, each loading half of
+    // B: a third less operand traffic per FLOP) when there are enough of its tiles to fill
+    // the GPU (64 pairs or more); otherwise single-CTA 128 x BN tiles. With two K slabs per
+    // load the pair form measured 12-18% faster on the Qwen3-8B q/o/gate/up/down and the
+    // looped-3B gate/up/down projections, and slower on the narrow k/v ones and at M = 256.
+    // UNO_LORA_CG=1 or 2 fixes it.
+    const bool pair_ok = M >= 2 * BM && d_out % 256 == 0;
+    P.CG = pair_ok && ((M + 2 * BM - 1) / (2 * BM)) * (d_out / 256) >= 64 ? 2 : 1;
     if (const char* e = getenv("UNO_LORA_CG")) {
         const int c = atoi(e);
-        if (c == 1 || (c == 2 && M >= 2 * BM && d_out % 256 == 0)) P.CG = c;
+        if (c == 1 || (c == 2 && pair_ok)) P.CG = c;
     }
     P.m_units = (int)((M + (int64_t)BM * P.CG - 1) / ((int64_t)BM * P.CG));
     if (P.CG == 2) {
@@ -890,8 +906,8 @@ Plan make_plan(int64_t M, int64_t d_in, int64_t d_out, int64_t rank, uno_dtype d
     // Main K steps of WS = 2 slabs of 64 (one 3-D TMA box per operand): a stage lands about
     // every thousand SM clocks whatever its bytes (a per-load cost, measured with
     // UNO_LORA_TRACE at 24 to 48 KB per stage), so two slabs per load nearly halve the count
-    // of loads. UNO_LORA_WIDE=0 keeps one slab per step; CTA pairs keep one.
-    P.ws = (P.CG == 1 && (d_in / BK) % 2 == 0) ? 2 : 1;
+    // of loads. UNO_LORA_WIDE=0 keeps one slab per step.
+    P.ws = (d_in / BK) % 2 == 0 ? 2 : 1;
     if (const char* e = getenv("UNO_LORA_WIDE"))
         if (atoi(e) == 0) P.ws = 1;
     P.kt0 = (int)(d_in / BK) / P.ws;
@@ -1063,15 +1079,10 @@ uno_status gated_lora_launch(const GatedLoraArgs& g, void* workspace, cudaStream
     __nv_bfloat16* t = reinterpret_cast<__nv_bfloat16*>(ws + P.t);
     CUtensorMap maps[6];
     const int cg = P.CG;
-    if (cg == 1) {  // X, W0, A: boxes of P.ws K slabs
-        if ((s = make_tmap3(&maps[0], x, M, din, BM, P.ws)) != UNO_OK) return s;
-        if ((s = make_tmap3(&maps[1], w0, dout, din, P.BN, P.ws)) != UNO_OK) return s;
-        if ((s = make_tmap3(&maps[2], a, r, din, P.rb, P.ws)) != UNO_OK) return s;
-    } else {
-        if ((s = make_tmap(&maps[0], x, M, din, BM)) != UNO_OK) return s;              // X
-        if ((s = make_tmap(&maps[1], w0, dout, din, P.BN / cg)) != UNO_OK) return s;   // W0
-        if ((s = make_tmap(&maps[2], a, r, din, P.rb / cg)) != UNO_OK) return s;       // A
-    }
+    // X, W0, A: boxes of P.ws K slabs (each CTA of a pair loads half of the B rows)
+    if ((s = make_tmap3(&maps[0], x, M, din, BM, P.ws)) != UNO_OK) return s;
+    if ((s = make_tmap3(&maps[1], w0, dout, din, P.BN / cg, P.ws)) != UNO_OK) return s;
+    if ((s = make_tmap3(&maps[2], a, r, din, P.rb / cg, P.ws)) != UNO_OK) return s;
     if ((s = make_tmap(&maps[3], t, (int64_t)P.splits * M, r, BM)) != UNO_OK) return s;  // T partials
     if ((s = make_tmap(&maps[4], b, dout, r, P.BN / cg)) != UNO_OK) return s;      // B
     if (P.epi_tma) {
