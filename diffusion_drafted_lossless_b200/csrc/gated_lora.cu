@@ -67,6 +67,8 @@ struct Params {
     int stages;                   // shared-memory ring depth
     uint32_t b_bytes;             // bytes of one B-operand K slab (max(BN, rb) rows of 64 elements)
     int ws;                       // K slabs per main K step (1 or 2: X/W0/A loads are 3-D boxes of ws slabs)
+    int tws;                      // K slabs per (T, B) step; T and B are 3-D maps when r is a multiple of 64
+    int t3d;
     uint32_t cb;                  // TMEM columns of one accumulator
     void* y;                      // [M, N] bf16 or fp32
     int out_f32;
@@ -381,6 +383,7 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
     unsigned char* smem = smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u);
     const int ST = p.stages;
     const int WS = p.ws;                               // K slabs per main K step
+    const int TWS = p.tws, t3d = p.t3d;                // K slabs per (T, B) step; 3-D maps for T and B
     const uint32_t a_stage = (uint32_t)WS * A_BYTES;  // bytes of a stage's A tiles
     unsigned char* sA = smem;
     unsigned char* sB = smem + (size_t)ST * a_stage;
@@ -470,7 +473,8 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
                     unsigned char* b = sB + (size_t)s * bbytes;
                     const CUtensorMap* ma = tpart ? &tT : &tX;
                     const CUtensorMap* mb = w.adapter ? &tA : (tpart ? &tB : &tW0);
-                    const int kx = (tpart ? tk : kt) * BK;
+                    const int kx = (tpart ? tk * TWS : kt) * BK;  // (2-D (T, B) loads)
+                    const int kz = tpart ? tk * TWS : kt * WS;      // (3-D loads: the first K slab)
                     const int ma_row = tpart ? ts * M + m0 : m0;  // partial ts's rows follow the earlier partials
                     if (tpart && ++tk == kt1) {
                         tk = 0;
@@ -482,25 +486,28 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
                         ph ^= 1u;
                     }
                     gl_mark(p, 3, g);
-                    if (leader) mbar_arrive_expect_tx(&full[st], tpart ? tx1 : (uint32_t)WS * tx1);
+                    if (leader) mbar_arrive_expect_tx(&full[st], (uint32_t)(tpart ? TWS : WS) * tx1);
+                    // every operand is a 3-D map (64 columns x rows x K slabs, several slabs per
+                    // box), except T and B when r is not a multiple of 64
+                    const bool two_d = tpart && !t3d;
                     if constexpr (CG == 2) {
                         const uint32_t bar = lead_full0 + (uint32_t)st * 8u;
-                        if (tpart) {
+                        if (two_d) {
                             tma_load_2d_pair(a, ma, kx, ma_row, bar);
                             tma_load_2d_pair(b, mb, kx, n0, bar);
                         } else {
-                            tma_load_3d_pair(a, ma, 0, ma_row, kt * WS, bar);
-                            tma_load_3d_pair(b, mb, 0, n0, kt * WS, bar);
+                            tma_load_3d_pair(a, ma, 0, ma_row, kz, bar);
+                            tma_load_3d_pair(b, mb, 0, n0, kz, bar);
                         }
                     } else {
-                        if (tpart) {
+                        if (two_d) {
                             tma_load_2d(a, ma, kx, ma_row, &full[st]);
                             gl_mark(p, 4, g);
                             tma_load_2d(b, mb, kx, n0, &full[st]);
-                        } else {  // X, W0 and A are 3-D maps: WS K slabs in one box each
-                            tma_load_3d(a, ma, 0, ma_row, kt * WS, &full[st]);
+                        } else {
+                            tma_load_3d(a, ma, 0, ma_row, kz, &full[st]);
                             gl_mark(p, 4, g);
-                            tma_load_3d(b, mb, 0, n0, kt * WS, &full[st]);
+                            tma_load_3d(b, mb, 0, n0, kz, &full[st]);
                         }
                     }
                     gl_mark(p, 0, g);
@@ -545,7 +552,7 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
                     const uint64_t db = db0 + (uint64_t)(((uint32_t)s * bbytes) >> 4);
                     // a main step holds WS K slabs (slab j of B at j x its box rows x 128 bytes);
                     // a (T, B) step one
-                    const int slabs = (!w.adapter && kt >= kt0) ? 1 : WS;
+                    const int slabs = (!w.adapter && kt >= kt0) ? TWS : WS;
                     const uint32_t bslab = ((w.adapter ? rb : (uint32_t)BN) / CG * 128u) >> 4;
                     for (int sl = 0; sl < slabs; ++sl) {
 #pragma unroll
@@ -848,7 +855,7 @@ uno_status make_tmap_store(CUtensorMap* m, void* ptr, int64_t rows, int64_t cols
 
 // The launch plan of one call (also sizes the workspace).
 struct Plan {
-    int CG, BN, rb, cb, m_tiles, m_units, n_tiles, kt0, kt1, splits, per, n_adapter, n_items, stages, ws;
+    int CG, BN, rb, cb, m_tiles, m_units, n_tiles, kt0, kt1, splits, per, n_adapter, n_items, stages, ws, tws, t3d;
     int ksplit, kper;
     int epi_tma;
     uint32_t b_bytes, epi_off;
@@ -911,7 +918,10 @@ Plan make_plan(int64_t M, int64_t d_in, int64_t d_out, int64_t rank, uno_dtype d
     if (const char* e = getenv("UNO_LORA_WIDE"))
         if (atoi(e) == 0) P.ws = 1;
     P.kt0 = (int)(d_in / BK) / P.ws;
-    P.kt1 = (int)((rank + BK - 1) / BK);
+    // (T, B) steps: two slabs when r is a multiple of 128 (and main steps take two)
+    P.t3d = rank % BK == 0;
+    P.tws = (P.t3d && P.ws == 2 && (rank / BK) % 2 == 0) ? 2 : 1;
+    P.kt1 = (int)((rank + BK - 1) / BK) / P.tws;
     // The adapter product X A^T of a row unit is split over K into `splits` items, each of
     // which writes its own bf16 partial of T; the output tiles run the (T, B) K tiles once
     // per partial, so no partial is ever summed on its own. Two partials measured fastest
@@ -1083,8 +1093,13 @@ uno_status gated_lora_launch(const GatedLoraArgs& g, void* workspace, cudaStream
     if ((s = make_tmap3(&maps[0], x, M, din, BM, P.ws)) != UNO_OK) return s;
     if ((s = make_tmap3(&maps[1], w0, dout, din, P.BN / cg, P.ws)) != UNO_OK) return s;
     if ((s = make_tmap3(&maps[2], a, r, din, P.rb / cg, P.ws)) != UNO_OK) return s;
-    if ((s = make_tmap(&maps[3], t, (int64_t)P.splits * M, r, BM)) != UNO_OK) return s;  // T partials
-    if ((s = make_tmap(&maps[4], b, dout, r, P.BN / cg)) != UNO_OK) return s;      // B
+    if (P.t3d) {  // T partials, B: boxes of P.tws K slabs
+        if ((s = make_tmap3(&maps[3], t, (int64_t)P.splits * M, r, BM, P.tws)) != UNO_OK) return s;
+        if ((s = make_tmap3(&maps[4], b, dout, r, P.BN / cg, P.tws)) != UNO_OK) return s;
+    } else {
+        if ((s = make_tmap(&maps[3], t, (int64_t)P.splits * M, r, BM)) != UNO_OK) return s;  // T partials
+        if ((s = make_tmap(&maps[4], b, dout, r, P.BN / cg)) != UNO_OK) return s;      // B
+    }
     if (P.epi_tma) {
         if ((s = make_tmap_store(&maps[5], g.y, M, dout)) != UNO_OK) return s;     // Y (stores)
     } else {
@@ -1111,6 +1126,8 @@ uno_status gated_lora_launch(const GatedLoraArgs& g, void* workspace, cudaStream
     p.stages = P.stages;
     p.b_bytes = P.b_bytes;
     p.ws = P.ws;
+    p.tws = P.tws;
+    p.t3d = P.t3d;
     p.cb = (uint32_t)P.cb;
     p.y = g.y;
     p.out_f32 = g.dtype == UNO_F32;
