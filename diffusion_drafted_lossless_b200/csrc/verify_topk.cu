@@ -932,6 +932,9 @@ finish_seq_kernel(Params p, int fw, int n_rows, size_t smem_bytes) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int rps = p.rows_per_seq;
     const int64_t r0 = (int64_t)blockIdx.x * fw, r1 = min(r0 + fw, (int64_t)n_rows);
+    // launched as a programmatic dependent of the streaming kernel: its CTAs may start while
+    // the last rows stream; the lists are read only after that grid has completed
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     fin_mark(p, warp, 0);
     if (warp < fw && r0 + warp < r1) {
         unsigned char* base = smem_raw + (size_t)warp * finish_bytes_per_warp<KCAP>(p.lists_per_row);
@@ -1165,6 +1168,8 @@ stream_rows_kernel(Params p, int n_items) {
             for (int u = 0; u < kGroup; ++u) cur[u] = load(r4, c0 + u, c1);
         }
     }
+    // this CTA's rows are written: the finish kernel may be scheduled
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 inline int num_sms() {
@@ -1297,8 +1302,19 @@ uno_status launch_t(const VerifyArgs& a, const Layout& L, unsigned char* ws, cud
         stream_kernel<T, KCAP><<<(unsigned)(n_rows * L.S), kStreamWarps * 32, smem1, stream>>>(p);
     }
     if ((s = check_cuda(cudaGetLastError(), "launch(verify stream)")) != UNO_OK) return s;
-    finish_seq_kernel<T, KCAP><<<(unsigned)((n_rows + fw - 1) / fw), kFinWarps * 32, smem2, stream>>>(p, fw, n_rows, smem2);
-    return check_cuda(cudaGetLastError(), "launch(verify finish)");
+    // a programmatic dependent launch (UNO_VERIFY_PDL=0: an ordinary one)
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[1];
+    cfg.gridDim = dim3((unsigned)((n_rows + fw - 1) / fw));
+    cfg.blockDim = dim3(kFinWarps * 32);
+    cfg.dynamicSmemBytes = smem2;
+    cfg.stream = stream;
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    const char* pe = getenv("UNO_VERIFY_PDL");
+    cfg.numAttrs = (pe && strcmp(pe, "0") == 0) ? 0 : 1;
+    return check_cuda(cudaLaunchKernelEx(&cfg, finish_seq_kernel<T, KCAP>, p, fw, n_rows, smem2), "launch(verify finish)");
 }
 
 }  // namespace vtopk
