@@ -32,14 +32,16 @@
  *
  * Kernel variants (environment, read at each call; every variant computes the same result
  * up to floating-point summation order, and the defaults are the fastest measured ones)
- *   UNO_LORA_CG=2            gated LoRA on CTA pairs (256-row tiles, cta_group::2)
+ *   UNO_LORA_CG=1|2          gated LoRA on single CTAs / CTA pairs (256-row tiles, cta_group::2)
  *   UNO_LORA_BN=64|128|256   gated LoRA output tile width
  *   UNO_LORA_SPLITS=n        adapter product X A^T split over K into n bf16 partials of T
  *   UNO_LORA_KSPLIT=n        output tiles split over K into n fp32 partials
  *   UNO_LORA_EPI=rows        output tiles stored by lanes (no shared-memory staging)
+ *   UNO_LORA_WIDE=0          one K slab per TMA load (default: two)
  *   UNO_VERIFY_STREAM=warps|tma  top-k verify: per-segment streaming CTAs (register or bulk-copy fed)
  *   UNO_VERIFY_SEGMENTS=n    top-k verify with UNO_VERIFY_STREAM=warps: CTAs per row (1 to 8)
  *   UNO_VERIFY_TOPK=local|window  top-k verify on the cluster kernels
+ *   UNO_VERIFY_PDL=0         top-k verify: the finish kernel launched after the streaming one ends
  *   UNO_VERIFY_FULL=generic  full-vocabulary verify: one CTA per item, fp64 exp per token;
  *                  =cluster  the cluster form or UNO_ERR_UNSUPPORTED
  *   UNO_VERIFY_FULL_CLUSTER=c  full-vocabulary cluster form: clusters of c CTAs
