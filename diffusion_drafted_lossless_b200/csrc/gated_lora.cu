@@ -390,6 +390,17 @@ lora_gemm_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int* abort_flag = &s_abort;
+    if constexpr (CG == 2) {
+        // the pair form needs its two-CTA cluster: a launch that arrives without it (a
+        // profiler may run a cooperative cluster launch as single CTAs) records an error and
+        // returns before any cta_group::2 instruction (the test is uniform over the grid)
+        uint32_t nct;
+        asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(nct));
+        if (nct != 2u) {
+            if (threadIdx.x == 0 && blockIdx.x == 0) record_device_status(p.status, (uint32_t)UNO_ERR_UNSUPPORTED);
+            return;
+        }
+    }
     const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
     const bool leader = rank == 0;
     const int unit0 = blockIdx.x / CG, units = gridDim.x / CG;  // this CTA's pair and the pair count
@@ -1047,12 +1058,15 @@ uno_status launch_t(const CUtensorMap (&maps)[6], Params& p, const Plan& P, cuda
     cfg.gridDim = dim3((unsigned)(units * CG));
     // Ask for a cooperative launch (every CTA resident, as the waits on T assume); where the
     // runtime does not take it together with clusters, the grid is sized to what is
-    // resident at once, which an otherwise idle GPU runs in full.
+    // resident at once, which an otherwise idle GPU runs in full. UNO_LORA_COOP=0 leaves the
+    // attribute out (Nsight Compute runs a cooperative launch with clusters as single CTAs).
+    const char* coop_env = getenv("UNO_LORA_COOP");
+    const bool coop = !(coop_env && coop_env[0] == '0');
     attrs[n_attr].id = cudaLaunchAttributeCooperative;
     attrs[n_attr].val.cooperative = 1;
-    cfg.numAttrs = n_attr + 1;
+    cfg.numAttrs = coop ? n_attr + 1 : n_attr;
     cudaError_t e = cudaLaunchKernelEx(&cfg, lora_gemm_kernel<BN, CG>, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], p);
-    if (e != cudaSuccess) {
+    if (e != cudaSuccess && coop) {
         cudaGetLastError();
         cfg.numAttrs = n_attr;
         e = cudaLaunchKernelEx(&cfg, lora_gemm_kernel<BN, CG>, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], p);

@@ -38,6 +38,8 @@
  *   UNO_LORA_KSPLIT=n        output tiles split over K into n fp32 partials
  *   UNO_LORA_EPI=rows        output tiles stored by lanes (no shared-memory staging)
  *   UNO_LORA_WIDE=0          one K slab per TMA load (default: two)
+ *   UNO_LORA_COOP=0          gated LoRA launched without the cooperative attribute (for
+ *                            profilers that run cooperative cluster launches as single CTAs)
  *   UNO_VERIFY_STREAM=warps|tma  top-k verify: per-segment streaming CTAs (register or bulk-copy fed)
  *   UNO_VERIFY_SEGMENTS=n    top-k verify with UNO_VERIFY_STREAM=warps: CTAs per row (1 to 8)
  *   UNO_VERIFY_TOPK=local|window  top-k verify on the cluster kernels
@@ -89,7 +91,8 @@ int uno_version(void);
 
 /*
  * Device status word: kernels whose bounded waits time out record UNO_ERR_TIMEOUT there
- * instead of trapping. This call synchronises the current device, returns the word in
+ * instead of trapping; the CTA-pair gated LoRA kernel records UNO_ERR_UNSUPPORTED there
+ * and does nothing when it finds itself launched without its two-CTA clusters. This call synchronises the current device, returns the word in
  * *code (UNO_OK if no kernel recorded anything since the last read) and clears it.
  * There is one word per device, shared by every stream and host thread that uses the
  * library on that device: a timeout recorded by any call since the last read is reported
