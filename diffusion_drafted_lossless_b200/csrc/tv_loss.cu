@@ -13,12 +13,14 @@
 // a thread-block cluster of CL CTAs owns one (teacher, student) row pair at a time, each
 // CTA holding a 1/CL slice of both rows in shared memory, so every logit is read from HBM
 // exactly once. The slices arrive by bulk copies (mbarrier completion) issued one row
-// ahead, so the next row streams in while this one is computed. Per row: slice maxima ->
-// cluster max; exp of both rows, keeping exp(student) in shared memory -> cluster sums;
-// p, q, sum |p - q| and sum q s, overwriting the kept exp with sign(q - p) folded into its
-// spare bits -> cluster sums; gradient from the kept values. Cluster-wide reductions read
-// every CTA's per-warp partials through distributed shared memory after a cluster barrier.
-// That is 3 exponentials per element pair and 6 bytes of HBM traffic per element pair.
+// ahead, so the next row streams in while this one is computed. Per row: warp maxima and
+// exps of both rows, keeping exp(student) in shared memory -> cluster reduction of the
+// (max, sum) pairs; A = sum of q over q > p and P = sum of p over q > p -> cluster
+// reduction; gradient. Each reduction is a per-warp st.async of its partial into every CTA
+// of the cluster. Rows overlap: row i's second reduction is in flight while the warps take
+// row i + 1's maxima and exps, and row i + 1's first while they write row i's gradient
+// (which recomputes exp(student), since row i + 1's exps have replaced it). That is 4
+// exponentials per element pair and 6 bytes of HBM traffic per element pair.
 //
 // rows_kernel (fp32 rows, unaligned rows, rows too long for the cluster's shared memory):
 // one CTA per token row. Pass 1 streams both rows from HBM once and keeps per-thread
@@ -279,7 +281,10 @@ __host__ __device__ inline size_t header_bytes(int ncta) {
 }
 // Elements of a row slice: a multiple of 8 (16-byte bulk copies and 8-element units).
 inline int64_t slice_elems(int64_t V, int cl) { return ((V + cl - 1) / cl + 7) / 8 * 8; }
-inline size_t smem_bytes(int64_t n, int ncta) { return header_bytes(ncta) + (size_t)n * (2 * 2 * 2 + 4); }
+// two (teacher, student) buffers, and with `keep` exp(student) of the current row in fp32
+inline size_t smem_bytes(int64_t n, int ncta, bool keep) {
+    return header_bytes(ncta) + (size_t)n * (2 * 2 * 2 + (keep ? 4 : 0));
+}
 
 __device__ __forceinline__ uint32_t cluster_rank() {
     uint32_t r;
@@ -372,6 +377,7 @@ __device__ __forceinline__ f2 mul2(f2 a, f2 b) {
 // the two bf16 values of a 32-bit word, widened (exact)
 __device__ __forceinline__ f2 widen(uint32_t w) { return pk(bf16_lo(w), bf16_hi(w)); }
 
+template <bool KEEP>
 __global__ void __launch_bounds__(kThreads, 1) cluster_kernel(Params p, int64_t n) {
     extern __shared__ __align__(128) unsigned char smem[];
     const TVArgs& a = p.a;
@@ -384,8 +390,9 @@ __global__ void __launch_bounds__(kThreads, 1) cluster_kernel(Params p, int64_t 
     float2* slots1 = reinterpret_cast<float2*>(smem + 64 + (size_t)ncta * kWarps * 16);  // [ncta][kWarps]
     const size_t hdr = header_bytes((int)ncta);
     uint16_t* inbuf = reinterpret_cast<uint16_t*>(smem + hdr);  // [2][teacher, student][n]
+    // (KEEP) unit u keeps its 8 exps at es[u*4 ..+4) and es[half + u*4 ..+4)
     float* es = reinterpret_cast<float*>(smem + hdr + (size_t)n * 8);
-    const int half = (int)(n / 2);  // unit u keeps its 8 exps at es[u*4 ..+4) and es[half + u*4 ..+4)
+    const int half = (int)(n / 2);
     const int64_t N = a.N, V = a.V;
     const int64_t lo = (int64_t)rank * n;
     const int cnt = (int)max((int64_t)0, min(n, V - lo));  // elements of this CTA's slice
@@ -406,18 +413,28 @@ __global__ void __launch_bounds__(kThreads, 1) cluster_kernel(Params p, int64_t 
         }
     };
 
-    bool more_rows = false;  // the current row is not this cluster's last
-    // Cluster-wide reductions of this row's per-warp partials (every lane of the warp
-    // passes the same value): each warp stores its partial into slot [rank][warp] of every
-    // CTA of the cluster; once all have landed, every warp combines them. The next row's
-    // phase of a reduction is armed before this CTA sends anything that lets another CTA
-    // reach it.
+    // Cluster-wide reductions of a row's per-warp partials (every lane of the warp passes the
+    // same value): each warp stores its partial into slot [rank][warp] of every CTA of the
+    // cluster (st.async, counted in bytes on that CTA's barrier); once all have landed, every
+    // warp combines them. Rows overlap (see the compute loop), yet one slot array and one
+    // barrier per reduction suffice, because of the order of the sends: a warp sends its
+    // partial of reduction 1 for row i only after reading the slots of reduction 0 for row
+    // i, and its partial of reduction 0 for row i + 1 only after reading the slots of
+    // reduction 1 for row i; so no CTA can send a row's partial into slots that another CTA
+    // is still reading, or count it on a barrier phase that is still open. Thread 0 arms a
+    // barrier's next phase right after its own wait, before it sends anything further.
+    // After a failed wait the later reduction waits are skipped (the call reports an error).
+    auto wait_red = [&](uint64_t* bar, uint32_t parity) {
+        if (!failed) wait(bar, parity);
+    };
     // 0: (max t, sum exp(t - max t), max s, sum exp(s - max s)) -> row maxima and sums
-    auto reduce0 = [&](float4 part, uint32_t parity) -> float4 {
+    auto send0 = [&](float4 part) {
         if ((uint32_t)lane < ncta)
             st_async_v4(map_rank(&slots0[rank * kWarps + warp], lane), map_rank(&red[0], lane), part.x, part.y,
                         part.z, part.w);
-        wait(&red[0], parity);
+    };
+    auto recv0 = [&](uint32_t parity, bool arm_next) -> float4 {
+        wait_red(&red[0], parity);
         float Mt = -INFINITY, Ms = -INFINITY;
         for (uint32_t j = lane; j < ncta * kWarps; j += 32) {
             const float4 w = slots0[j];
@@ -432,21 +449,23 @@ __global__ void __launch_bounds__(kThreads, 1) cluster_kernel(Params p, int64_t 
             if (w.y > 0.f) Zt += w.y * ex2((w.x - Mt) * kLog2e);
             if (w.w > 0.f) Zs += w.w * ex2((w.z - Ms) * kLog2e);
         }
-        if (tid == 0 && more_rows) mbar_arrive_expect_tx(&red[0], red0_bytes);
+        if (tid == 0 && arm_next) mbar_arrive_expect_tx(&red[0], red0_bytes);
         return make_float4(Mt, warp_sum(Zt), Ms, warp_sum(Zs));
     };
     // 1: (A, P) sums
-    auto reduce1 = [&](float2 part, uint32_t parity) -> float2 {
+    auto send1 = [&](float2 part) {
         if ((uint32_t)lane < ncta)
             st_async_v2(map_rank(&slots1[rank * kWarps + warp], lane), map_rank(&red[1], lane), part.x, part.y);
-        wait(&red[1], parity);
+    };
+    auto recv1 = [&](uint32_t parity, bool arm_next) -> float2 {
+        wait_red(&red[1], parity);
         float x = 0.f, y = 0.f;
         for (uint32_t j = lane; j < ncta * kWarps; j += 32) {
             const float2 w = slots1[j];
             x += w.x;
             y += w.y;
         }
-        if (tid == 0 && more_rows) mbar_arrive_expect_tx(&red[1], red1_bytes);
+        if (tid == 0 && arm_next) mbar_arrive_expect_tx(&red[1], red1_bytes);
         return make_float2(warp_sum(x), warp_sum(y));
     };
 
@@ -503,17 +522,22 @@ __global__ void __launch_bounds__(kThreads, 1) cluster_kernel(Params p, int64_t 
         __syncwarp();
     } else {
         // ---------------- compute warps ----------------
+        // Rows overlap: row i's reduction 1 is in flight while the warps take row i + 1's
+        // maxima and exps, and row i + 1's reduction 0 while they write row i's gradient:
+        //   [combine 0 (i)] [A, P (i); send 1 (i)] [maxima, exps (i + 1)]
+        //   [combine 1 (i); send 0 (i + 1)] [gradient (i)] ...
+        // Row i + 1's exps overwrite the kept exp(student) of row i, so the gradient pass
+        // recomputes exp(student) (4 exponentials per element pair).
         double tv_sum = 0.0;  // this cluster's masked TV (rank 0, thread 0)
-        uint32_t rows_done = 0, it = 0;
-        for (int64_t r = first; r < N; r += step, ++it) {
-            const int b = it & 1;
-            const uint32_t par = it & 1;
-            more_rows = r + step < N;
-            if (cnt > 0) wait(&full[b], (it >> 1) & 1);
+        uint32_t rows_done = 0;
+        const f2 L2E = pk(kLog2e, kLog2e);
+        // maxima and exps of the row in buffer b: this warp's (max t, sum, max s, sum), with
+        // exp(s - warp max) kept; lt, ls are the warp maxima x log2(e) (0 for a warp with no
+        // elements: its sums are 0 and it never reads its factors)
+        float mt = -INFINITY, ms = -INFINITY, lt = 0.f, ls = 0.f;
+        auto maxima_exps = [&](int b) -> float4 {
             const uint16_t* tin = inbuf + (size_t)b * 2 * n;
             const uint16_t* sin = tin + n;
-
-            // ---- this warp's maxima (exps are taken relative to them) ----
             __nv_bfloat162 mt2 = __floats2bfloat162_rn(-INFINITY, -INFINITY), ms2 = mt2;
             for (int u = tid; u < units; u += kWarps * 32) {
                 const uint4 wt = lds128(tin + u * 8), ws = lds128(sin + u * 8);
@@ -524,13 +548,11 @@ __global__ void __launch_bounds__(kThreads, 1) cluster_kernel(Params p, int64_t 
                     ms2 = __hmax2(ms2, *reinterpret_cast<const __nv_bfloat162*>(&as4[j]));
                 }
             }
-            const float mt = warp_max(fmaxf(__low2float(mt2), __high2float(mt2)));
-            const float ms = warp_max(fmaxf(__low2float(ms2), __high2float(ms2)));
-            // a warp with no elements uses 0 (its sums are 0 and it never reads its factors)
-            const float lt = (mt == -INFINITY ? 0.f : mt) * kLog2e, ls = (ms == -INFINITY ? 0.f : ms) * kLog2e;
-            const f2 L2E = pk(kLog2e, kLog2e), NLT = pk(-lt, -lt), NLS = pk(-ls, -ls);
-
-            // ---- sums of exp(x - warp max); exp(s - warp max) kept ----
+            mt = warp_max(fmaxf(__low2float(mt2), __high2float(mt2)));
+            ms = warp_max(fmaxf(__low2float(ms2), __high2float(ms2)));
+            lt = (mt == -INFINITY ? 0.f : mt) * kLog2e;
+            ls = (ms == -INFINITY ? 0.f : ms) * kLog2e;
+            const f2 NLT = pk(-lt, -lt), NLS = pk(-ls, -ls);
             f2 zt2 = pk(0.f, 0.f), zs2 = zt2;
             for (int u = tid; u < units; u += kWarps * 32) {
                 const uint4 wt = lds128(tin + u * 8), ws = lds128(sin + u * 8);
@@ -544,50 +566,82 @@ __global__ void __launch_bounds__(kThreads, 1) cluster_kernel(Params p, int64_t 
                     e[2 * j + 1] = ex2(hi_of(xs));
                     zs2 = add2(zs2, pk(e[2 * j], e[2 * j + 1]));
                 }
-                *reinterpret_cast<float4*>(es + u * 4) = make_float4(e[0], e[1], e[2], e[3]);
-                *reinterpret_cast<float4*>(es + half + u * 4) = make_float4(e[4], e[5], e[6], e[7]);
+                if constexpr (KEEP) {
+                    *reinterpret_cast<float4*>(es + u * 4) = make_float4(e[0], e[1], e[2], e[3]);
+                    *reinterpret_cast<float4*>(es + half + u * 4) = make_float4(e[4], e[5], e[6], e[7]);
+                }
             }
-            const float4 st = reduce0(make_float4(mt, warp_sum(lo_of(zt2) + hi_of(zt2)), ms,
-                                                  warp_sum(lo_of(zs2) + hi_of(zs2))), par);
+            return make_float4(mt, warp_sum(lo_of(zt2) + hi_of(zt2)), ms, warp_sum(lo_of(zs2) + hi_of(zs2)));
+        };
+
+        if (first < N) {
+            if (cnt > 0) wait(&full[0], 0);
+            send0(maxima_exps(0));
+        }
+        uint32_t it = 0;
+        for (int64_t r = first; r < N; r += step, ++it) {
+            const int b = it & 1;
+            const uint32_t par = it & 1;
+            const bool more = r + step < N;
+            const uint16_t* tin = inbuf + (size_t)b * 2 * n;
+            const uint16_t* sin = tin + n;
+            // this row's warp maxima (the next row's maxima_exps replaces them)
+            const float rmt = mt, rms = ms, rlt = lt, rls = ls;
+
+            const float4 st = recv0(par, more);
             const float Mt = st.x, Zt = st.y, Ms = st.z, Zs = st.w;
-            // p = exp(t - wmt) * at, q = kept exp(s - wms) * as: this warp's maxima folded
-            // into at, as (the same arithmetic for both rows: identical rows give p == q).
+            // p = exp(t - wmt) * at, q = exp(s - wms) * as: this warp's maxima folded into at,
+            // as (the same arithmetic for both rows: identical rows give p == q).
             // q > p is decided in the log domain, exact up to the rounding of one threshold:
             //   q > p  <=>  s - t > K = (Ms + ln Zs) - (Mt + ln Zt)
             // (Ms - Mt is exact; Zs / Zt is near 1 in practice, so its log is accurate to ~1e-7)
-            const float at = mt == -INFINITY ? 0.f : ex2(lt - Mt * kLog2e) / Zt;
-            const float as = ms == -INFINITY ? 0.f : ex2(ls - Ms * kLog2e) / Zs;
+            const float at = rmt == -INFINITY ? 0.f : ex2(rlt - Mt * kLog2e) / Zt;
+            const float as = rms == -INFINITY ? 0.f : ex2(rls - Ms * kLog2e) / Zs;
             const float K = (Ms - Mt) + logf(Zs / Zt);
+            const f2 NLT = pk(-rlt, -rlt), NLS = pk(-rls, -rls);
 
             // ---- A = sum of q over q > p, P = sum of p over q > p ----
             // TV = A - P and sum_v q_v sign(q_v - p_v) / 2 = A - 1/2 (both rows sum to 1)
             float Araw = 0.f, Praw = 0.f;
             for (int u = tid; u < units; u += kWarps * 32) {
                 const uint4 wt = lds128(tin + u * 8), ws = lds128(sin + u * 8);
-                const float4 k0 = *reinterpret_cast<const float4*>(es + u * 4);
-                const float4 k1 = *reinterpret_cast<const float4*>(es + half + u * 4);
                 const uint32_t at4[4] = {wt.x, wt.y, wt.z, wt.w}, as4[4] = {ws.x, ws.y, ws.z, ws.w};
-                const float qe[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+                float qe[8];
+                if constexpr (KEEP) {
+                    const float4 k0 = *reinterpret_cast<const float4*>(es + u * 4);
+                    const float4 k1 = *reinterpret_cast<const float4*>(es + half + u * 4);
+                    qe[0] = k0.x, qe[1] = k0.y, qe[2] = k0.z, qe[3] = k0.w;
+                    qe[4] = k1.x, qe[5] = k1.y, qe[6] = k1.z, qe[7] = k1.w;
+                }
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    const f2 t2 = widen(at4[j]);
-                    const f2 dl = sub2(widen(as4[j]), t2);
-                    const f2 xt = fma2(t2, L2E, NLT);
+                    const f2 t2 = widen(at4[j]), s2 = widen(as4[j]);
+                    const f2 dl = sub2(s2, t2);
+                    const f2 xt = fma2(t2, L2E, NLT), xs = fma2(s2, L2E, NLS);
                     if (lo_of(dl) > K) {
-                        Araw += qe[2 * j];
+                        Araw += KEEP ? qe[2 * j] : ex2(lo_of(xs));
                         Praw += ex2(lo_of(xt));
                     }
                     if (hi_of(dl) > K) {
-                        Araw += qe[2 * j + 1];
+                        Araw += KEEP ? qe[2 * j + 1] : ex2(hi_of(xs));
                         Praw += ex2(hi_of(xt));
                     }
                 }
             }
-            const float2 ap = reduce1(make_float2(warp_sum(Araw * as), warp_sum(Praw * at)), par);
+            send1(make_float2(warp_sum(Araw * as), warp_sum(Praw * at)));
+
+            // ---- the next row's maxima and exps, while reduction 1 is in flight ----
+            float4 next_part = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (more) {
+                if (cnt > 0) wait(&full[b ^ 1], ((it + 1) >> 1) & 1);
+                next_part = maxima_exps(b ^ 1);
+            }
+            const float2 ap = recv1(par, more);
             const float Af = ap.x, Pf = ap.y;
+            if (more) send0(next_part);
             const bool on = a.mask == nullptr || a.mask[r] != 0;
 
-            // ---- gradient: f q (s - c) = f q (1 - A) where q > p, -f q A elsewhere ----
+            // ---- gradient: f q (1 - A) where q > p, -f q A elsewhere ----
             // written as bf16 in place of the teacher slice (each unit by the thread that read
             // it); the producer warp streams the slice out once every warp is done
             if (G != nullptr) {
@@ -599,16 +653,15 @@ __global__ void __launch_bounds__(kThreads, 1) cluster_kernel(Params p, int64_t 
                     uint4 o = make_uint4(0u, 0u, 0u, 0u);
                     if (grad_on) {
                         const uint4 wt = lds128(tin + u * 8), ws = lds128(sin + u * 8);
-                        const float4 k0 = *reinterpret_cast<const float4*>(es + u * 4);
-                        const float4 k1 = *reinterpret_cast<const float4*>(es + half + u * 4);
                         const uint32_t at4[4] = {wt.x, wt.y, wt.z, wt.w}, as4[4] = {ws.x, ws.y, ws.z, ws.w};
-                        const f2 qe[4] = {pk(k0.x, k0.y), pk(k0.z, k0.w), pk(k1.x, k1.y), pk(k1.z, k1.w)};
                         uint32_t ow[4];
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
-                            const f2 dl = sub2(widen(as4[j]), widen(at4[j]));
+                            const f2 s2 = widen(as4[j]);
+                            const f2 dl = sub2(s2, widen(at4[j]));
+                            const f2 xs = fma2(s2, L2E, NLS);
                             const f2 fac = pk(lo_of(dl) > K ? kp : kn, hi_of(dl) > K ? kp : kn);
-                            const f2 g = mul2(qe[j], fac);
+                            const f2 g = mul2(pk(ex2(lo_of(xs)), ex2(hi_of(xs))), fac);
                             __nv_bfloat162 hv = __floats2bfloat162_rn(lo_of(g), hi_of(g));
                             ow[j] = *reinterpret_cast<uint32_t*>(&hv);
                         }
@@ -650,10 +703,12 @@ __global__ void __launch_bounds__(kThreads, 1) cluster_kernel(Params p, int64_t 
 // A team waits for its cluster reductions and its copies while the other team computes, so
 // those latencies overlap instead of adding up. Each team holds one (teacher, student) slice
 // pair (the gradient replaces the teacher slice and is streamed out by the team's leader,
-// who then brings in the team's next row); exp(student) is recomputed where it is needed
-// rather than kept (5 exponentials per element pair instead of 3), which is what lets two
-// row pairs fit in shared memory. Reductions: each warp stores its partial into slot
-// [rank][warp] of every CTA of the cluster and arrives on that CTA's barrier.
+// who then brings in the team's next row). KEEP: exp(student) of the team's row is kept in
+// fp32 beside its slices (3 exponentials per element pair, 12 bytes of shared memory per
+// element and team, so clusters of 16 at a 152k vocabulary); otherwise it is recomputed
+// where it is needed (5 exponentials per element pair, 4 bytes per element and team).
+// Reductions: each warp stores its partial into slot [rank][warp] of every CTA of the
+// cluster and arrives on that CTA's barrier.
 // ---------------------------------------------------------------------------------------
 constexpr int kTeams = 2;
 constexpr int kTeamWarps = 8;
@@ -661,9 +716,12 @@ constexpr int kTeamThreads = kTeamWarps * 32;
 constexpr int kTeamKernelThreads = kTeams * kTeamThreads;
 constexpr int kMaxCL = 16;
 
-__host__ __device__ inline size_t team_slice_bytes(int64_t n) { return ((size_t)n * 4 + 127) / 128 * 128; }
-__host__ __device__ inline size_t team_bytes(int64_t n) {
-    return team_slice_bytes(n) + (size_t)kMaxCL * kTeamWarps * (16 + 8);
+// a team's (teacher, student) slices, and with `keep` its exp(student) in fp32
+__host__ __device__ inline size_t team_slice_bytes(int64_t n, bool keep) {
+    return ((size_t)n * (keep ? 8 : 4) + 127) / 128 * 128;
+}
+__host__ __device__ inline size_t team_bytes(int64_t n, bool keep) {
+    return team_slice_bytes(n, keep) + (size_t)kMaxCL * kTeamWarps * (16 + 8);
 }
 
 __device__ __forceinline__ void team_sync(int team) {
@@ -694,6 +752,7 @@ __device__ __forceinline__ bool wait_cluster(uint64_t* bar, uint32_t parity) {
     return false;
 }
 
+template <bool KEEP>
 __global__ void __launch_bounds__(kTeamKernelThreads, 1) team_kernel(Params p, int64_t n) {
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t bars[kTeams][3];  // slices landed, reduction 0, reduction 1
@@ -704,10 +763,13 @@ __global__ void __launch_bounds__(kTeamKernelThreads, 1) team_kernel(Params p, i
     const int team = threadIdx.x / kTeamThreads, tt = threadIdx.x % kTeamThreads;
     const int tw = tt >> 5, lane = tt & 31;
     const uint32_t rank = cluster_rank(), ncta = cluster_size();
-    unsigned char* base = smem + (size_t)team * team_bytes(n);
+    unsigned char* base = smem + (size_t)team * team_bytes(n, KEEP);
     uint16_t* tin = reinterpret_cast<uint16_t*>(base);  // teacher slice, then the gradient
     uint16_t* sin = tin + n;                            // student slice
-    float4* s0 = reinterpret_cast<float4*>(base + team_slice_bytes(n));  // [kMaxCL][kTeamWarps]
+    // (KEEP) unit u's 8 values of exp(s - warp max) at es[u*4 ..+4) and es[half + u*4 ..+4)
+    float* es = reinterpret_cast<float*>(base + (size_t)n * 4);
+    const int half = (int)(n / 2);
+    float4* s0 = reinterpret_cast<float4*>(base + team_slice_bytes(n, KEEP));  // [kMaxCL][kTeamWarps]
     float2* s1 = reinterpret_cast<float2*>(s0 + kMaxCL * kTeamWarps);     // [kMaxCL][kTeamWarps]
     uint64_t* full = &bars[team][0];
     uint64_t* red0 = &bars[team][1];
@@ -774,11 +836,18 @@ __global__ void __launch_bounds__(kTeamKernelThreads, 1) team_kernel(Params p, i
         for (int u = tt; u < units; u += kTeamThreads) {
             const uint4 wt = lds128(tin + u * 8), ws = lds128(sin + u * 8);
             const uint32_t at4[4] = {wt.x, wt.y, wt.z, wt.w}, as4[4] = {ws.x, ws.y, ws.z, ws.w};
+            float e[8];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const f2 xt = fma2(widen(at4[j]), L2E, NLT), xs = fma2(widen(as4[j]), L2E, NLS);
                 zt2 = add2(zt2, pk(ex2(lo_of(xt)), ex2(hi_of(xt))));
-                zs2 = add2(zs2, pk(ex2(lo_of(xs)), ex2(hi_of(xs))));
+                e[2 * j] = ex2(lo_of(xs));
+                e[2 * j + 1] = ex2(hi_of(xs));
+                zs2 = add2(zs2, pk(e[2 * j], e[2 * j + 1]));
+            }
+            if constexpr (KEEP) {
+                *reinterpret_cast<float4*>(es + u * 4) = make_float4(e[0], e[1], e[2], e[3]);
+                *reinterpret_cast<float4*>(es + half + u * 4) = make_float4(e[4], e[5], e[6], e[7]);
             }
         }
         const float zt = warp_sum(lo_of(zt2) + hi_of(zt2)), zs = warp_sum(lo_of(zs2) + hi_of(zs2));
@@ -814,17 +883,24 @@ __global__ void __launch_bounds__(kTeamKernelThreads, 1) team_kernel(Params p, i
         for (int u = tt; u < units; u += kTeamThreads) {
             const uint4 wt = lds128(tin + u * 8), ws = lds128(sin + u * 8);
             const uint32_t at4[4] = {wt.x, wt.y, wt.z, wt.w}, as4[4] = {ws.x, ws.y, ws.z, ws.w};
+            float qe[8];
+            if constexpr (KEEP) {
+                const float4 k0 = *reinterpret_cast<const float4*>(es + u * 4);
+                const float4 k1 = *reinterpret_cast<const float4*>(es + half + u * 4);
+                qe[0] = k0.x, qe[1] = k0.y, qe[2] = k0.z, qe[3] = k0.w;
+                qe[4] = k1.x, qe[5] = k1.y, qe[6] = k1.z, qe[7] = k1.w;
+            }
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const f2 t2 = widen(at4[j]), s2 = widen(as4[j]);
                 const f2 dl = sub2(s2, t2);
                 const f2 xt = fma2(t2, L2E, NLT), xs = fma2(s2, L2E, NLS);
                 if (lo_of(dl) > K) {
-                    Araw += ex2(lo_of(xs));
+                    Araw += KEEP ? qe[2 * j] : ex2(lo_of(xs));
                     Praw += ex2(lo_of(xt));
                 }
                 if (hi_of(dl) > K) {
-                    Araw += ex2(hi_of(xs));
+                    Araw += KEEP ? qe[2 * j + 1] : ex2(hi_of(xs));
                     Praw += ex2(hi_of(xt));
                 }
             }
@@ -855,6 +931,13 @@ __global__ void __launch_bounds__(kTeamKernelThreads, 1) team_kernel(Params p, i
                 if (grad_on) {
                     const uint4 wt = lds128(tin + u * 8), ws = lds128(sin + u * 8);
                     const uint32_t at4[4] = {wt.x, wt.y, wt.z, wt.w}, as4[4] = {ws.x, ws.y, ws.z, ws.w};
+                    float qe[8];
+                    if constexpr (KEEP) {
+                        const float4 k0 = *reinterpret_cast<const float4*>(es + u * 4);
+                        const float4 k1 = *reinterpret_cast<const float4*>(es + half + u * 4);
+                        qe[0] = k0.x, qe[1] = k0.y, qe[2] = k0.z, qe[3] = k0.w;
+                        qe[4] = k1.x, qe[5] = k1.y, qe[6] = k1.z, qe[7] = k1.w;
+                    }
                     uint32_t ow[4];
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
@@ -862,7 +945,8 @@ __global__ void __launch_bounds__(kTeamKernelThreads, 1) team_kernel(Params p, i
                         const f2 dl = sub2(s2, widen(at4[j]));
                         const f2 xs = fma2(s2, L2E, NLS);
                         const f2 fac = pk(lo_of(dl) > K ? kp : kn, hi_of(dl) > K ? kp : kn);
-                        const f2 g = mul2(pk(ex2(lo_of(xs)), ex2(hi_of(xs))), fac);
+                        const f2 qv = KEEP ? pk(qe[2 * j], qe[2 * j + 1]) : pk(ex2(lo_of(xs)), ex2(hi_of(xs)));
+                        const f2 g = mul2(qv, fac);
                         __nv_bfloat162 hv = __floats2bfloat162_rn(lo_of(g), hi_of(g));
                         ow[j] = *reinterpret_cast<uint32_t*>(&hv);
                     }
@@ -932,33 +1016,100 @@ struct DeviceInfo {
 std::mutex g_mu;
 DeviceInfo g_dev[64];
 
-// Cluster size for rows of V bf16 elements: UNO_TV_CLUSTER if set (1, 2, 4, 8 or 16) and
-// its slices fit, else the smallest whose slices fit in one CTA's shared memory; 0 when none
-// fits.
-int choose_cluster(int64_t V, int smem_optin) {
-    auto need = [&](int c) { return tvk::cl::smem_bytes(tvk::cl::slice_elems(V, c), c); };
-    if (const char* e = getenv("UNO_TV_CLUSTER")) {
-        const int c = atoi(e);
-        if ((c == 1 || c == 2 || c == 4 || c == 8 || c == 16) && need(c) <= (size_t)smem_optin) return c;
+// Co-resident clusters of the cluster kernel at cluster size c (cached per device).
+int cluster_capacity(DeviceInfo& di, int c, bool keep, int64_t n) {
+    cudaLaunchConfig_t q = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)c;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    q.blockDim = dim3(tvk::cl::kThreads);
+    q.dynamicSmemBytes = tvk::cl::smem_bytes(n, c, keep);
+    q.attrs = attr;
+    q.numAttrs = 1;
+    q.gridDim = dim3((unsigned)c);
+    auto key = std::make_pair(c + (keep ? 32 : 0), q.dynamicSmemBytes);
+    auto found = di.max_clusters.find(key);
+    if (found != di.max_clusters.end()) return found->second;
+    int maxc = 0;
+    if (cudaOccupancyMaxActiveClusters(&maxc, keep ? tvk::cl::cluster_kernel<true> : tvk::cl::cluster_kernel<false>,
+                                       &q) != cudaSuccess) {
+        cudaGetLastError();
+        maxc = 0;
     }
-    for (int c = 1; c <= 16; c *= 2)
-        if (need(c) <= (size_t)smem_optin) return c;
-    return 0;
+    di.max_clusters[key] = maxc;
+    return maxc;
 }
 
-// The two-team kernel: the smallest cluster size whose two slice pairs per CTA fit
-// (UNO_TV_CLUSTER forces one that fits).
+// Cluster form for N rows of V bf16 elements: a cluster size c (1 to 8, or 16) whose slices
+// fit in one CTA's shared memory, with exp(student) kept (12 bytes per element) or
+// recomputed (8 bytes per element, 5 exponentials per element pair instead of 4, so a
+// smaller c fits). Among those that fit, the one with the least estimated time: the rows
+// each co-resident cluster takes in turn x the slice each CTA works through, x 1.02 when
+// exp(student) is kept (its shared-memory traffic measured costlier than the extra
+// exponentials: at V = 151936, clusters of 8 took 0.438 ms per 1024 rows keeping it and
+// 0.430 ms recomputing it; clusters of 6, which only the recomputing form fits, 0.361 ms:
+// no more than 15 clusters of 8 are co-resident, 120 of the 148 SMs). UNO_TV_CLUSTER=c
+// forces c where it fits; UNO_TV_KEEP=0 forces the recomputing form and UNO_TV_KEEP=1 the
+// keeping one. Returns c = 0 when none fits.
+std::pair<int, bool> choose_cluster(DeviceInfo& di, int64_t N, int64_t V) {
+    int forced = 0;
+    if (const char* e = getenv("UNO_TV_CLUSTER")) forced = atoi(e);
+    const char* ke = getenv("UNO_TV_KEEP");
+    const bool allow_keep = !(ke && ke[0] == '0'), allow_recompute = !(ke && ke[0] == '1');
+    std::pair<int, bool> best{0, false};
+    double best_cost = 0.0;
+    static const int kSizes[] = {1, 2, 3, 4, 5, 6, 7, 8, 16};
+    // pass 0: the forced size only (if any); pass 1: every size
+    for (int pass = forced != 0 ? 0 : 1; pass < 2 && best.first == 0; ++pass) {
+        for (int c : kSizes) {
+            if (pass == 0 && c != forced) continue;
+            const int64_t n = tvk::cl::slice_elems(V, c);
+            for (int k = 0; k < 2; ++k) {
+                const bool keep = k == 0;
+                if ((keep && !allow_keep) || (!keep && !allow_recompute)) continue;
+                if (tvk::cl::smem_bytes(n, c, keep) > (size_t)di.smem_optin) continue;
+                const int maxc = cluster_capacity(di, c, keep, n);
+                if (maxc <= 0) continue;
+                const double cost = (double)((N + maxc - 1) / maxc) * (double)n * (keep ? 1.02 : 1.0);
+                if (best.first == 0 || cost < best_cost) {
+                    best = {c, keep};
+                    best_cost = cost;
+                }
+            }
+        }
+    }
+    return best;
+}
+
+// The two-team kernel: the smallest cluster size whose two teams' slices fit, keeping
+// exp(student) where some cluster size lets it fit (UNO_TV_CLUSTER forces a size, and
+// UNO_TV_KEEP=0 recomputes exp(student) instead).
 bool launch_teams(const tvk::Params& p, cudaStream_t stream, uno_status& st, DeviceInfo& di) {
     const TVArgs& a = p.a;
     const size_t room = (size_t)di.smem_optin - 256;  // the kernel's static shared memory
-    auto fits = [&](int c) { return 2 * tvk::cl::team_bytes(tvk::cl::slice_elems(a.V, c)) <= room; };
-    int c = 0;
+    auto fits = [&](int c, bool keep) {
+        return 2 * tvk::cl::team_bytes(tvk::cl::slice_elems(a.V, c), keep) <= room;
+    };
+    int forced = 0;
     if (const char* e = getenv("UNO_TV_CLUSTER")) {
         const int f = atoi(e);
-        if ((f == 1 || f == 2 || f == 4 || f == 8 || f == 16) && fits(f)) c = f;
+        if (f == 1 || f == 2 || f == 4 || f == 8 || f == 16) forced = f;
     }
-    for (int t = 1; t <= 16 && c == 0; t *= 2)
-        if (fits(t)) c = t;
+    const char* ke = getenv("UNO_TV_KEEP");
+    const bool allow_keep = !(ke && ke[0] == '0');
+    int c = 0;
+    bool keep = false;
+    for (int pass = allow_keep ? 0 : 1; pass < 2 && c == 0; ++pass) {
+        keep = pass == 0;
+        if (forced != 0) {
+            if (fits(forced, keep)) c = forced;
+        } else {
+            for (int t = 1; t <= 16 && c == 0; t *= 2)
+                if (fits(t, keep)) c = t;
+        }
+    }
     if (c == 0) return false;
     const int64_t n = tvk::cl::slice_elems(a.V, c);
     cudaLaunchConfig_t cfg = {};
@@ -968,11 +1119,12 @@ bool launch_teams(const tvk::Params& p, cudaStream_t stream, uno_status& st, Dev
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.blockDim = dim3(tvk::cl::kTeamKernelThreads);
-    cfg.dynamicSmemBytes = 2 * tvk::cl::team_bytes(n);
+    cfg.dynamicSmemBytes = 2 * tvk::cl::team_bytes(n, keep);
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    auto key = std::make_pair(-c, cfg.dynamicSmemBytes);
+    auto kernel = keep ? tvk::cl::team_kernel<true> : tvk::cl::team_kernel<false>;
+    auto key = std::make_pair(-(c + (keep ? 32 : 0)), cfg.dynamicSmemBytes);
     auto found = di.max_clusters.find(key);
     int maxc = 0;
     if (found != di.max_clusters.end()) {
@@ -980,7 +1132,7 @@ bool launch_teams(const tvk::Params& p, cudaStream_t stream, uno_status& st, Dev
     } else {
         cudaLaunchConfig_t q = cfg;
         q.gridDim = dim3((unsigned)c);
-        if (cudaOccupancyMaxActiveClusters(&maxc, tvk::cl::team_kernel, &q) != cudaSuccess) {
+        if (cudaOccupancyMaxActiveClusters(&maxc, kernel, &q) != cudaSuccess) {
             cudaGetLastError();
             maxc = 0;
         }
@@ -989,7 +1141,7 @@ bool launch_teams(const tvk::Params& p, cudaStream_t stream, uno_status& st, Dev
     if (maxc <= 0) return false;
     const int64_t clusters = std::min<int64_t>((a.N + 1) / 2, (int64_t)maxc);
     cfg.gridDim = dim3((unsigned)(clusters * c));
-    st = check_cuda(cudaLaunchKernelEx(&cfg, tvk::cl::team_kernel, p, n), "launch(tv teams)");
+    st = check_cuda(cudaLaunchKernelEx(&cfg, kernel, p, n), "launch(tv teams)");
     return true;
 }
 
@@ -1012,13 +1164,21 @@ bool launch_cluster(const tvk::Params& p, cudaStream_t stream, uno_status& st) {
     if (!di.ready) {
         if (cudaDeviceGetAttribute(&di.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
             return false;
-        if (cudaFuncSetAttribute(tvk::cl::cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(tvk::cl::cluster_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  di.smem_optin) != cudaSuccess ||
-            cudaFuncSetAttribute(tvk::cl::cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+            cudaFuncSetAttribute(tvk::cl::cluster_kernel<true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
                 cudaSuccess ||
-            cudaFuncSetAttribute(tvk::cl::team_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(tvk::cl::cluster_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 di.smem_optin) != cudaSuccess ||
+            cudaFuncSetAttribute(tvk::cl::cluster_kernel<false>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(tvk::cl::team_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  di.smem_optin - 256) != cudaSuccess ||
-            cudaFuncSetAttribute(tvk::cl::team_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+            cudaFuncSetAttribute(tvk::cl::team_kernel<false>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(tvk::cl::team_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 di.smem_optin - 256) != cudaSuccess ||
+            cudaFuncSetAttribute(tvk::cl::team_kernel<true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
                 cudaSuccess) {
             cudaGetLastError();
             return false;
@@ -1026,9 +1186,12 @@ bool launch_cluster(const tvk::Params& p, cudaStream_t stream, uno_status& st) {
         di.ready = true;
     }
     if (teams) return launch_teams(p, stream, st, di);
-    const int c = choose_cluster(a.V, di.smem_optin);
+    const std::pair<int, bool> choice = choose_cluster(di, a.N, a.V);
+    const int c = choice.first;
+    const bool keep = choice.second;
     if (c == 0) return false;
     const int64_t n = tvk::cl::slice_elems(a.V, c);
+    const int maxc = cluster_capacity(di, c, keep, n);
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1036,28 +1199,15 @@ bool launch_cluster(const tvk::Params& p, cudaStream_t stream, uno_status& st) {
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.blockDim = dim3(tvk::cl::kThreads);
-    cfg.dynamicSmemBytes = tvk::cl::smem_bytes(n, c);
+    cfg.dynamicSmemBytes = tvk::cl::smem_bytes(n, c, keep);
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    auto key = std::make_pair(c, cfg.dynamicSmemBytes);
-    auto found = di.max_clusters.find(key);
-    int maxc = 0;
-    if (found != di.max_clusters.end()) {
-        maxc = found->second;
-    } else {
-        cudaLaunchConfig_t q = cfg;
-        q.gridDim = dim3((unsigned)c);
-        if (cudaOccupancyMaxActiveClusters(&maxc, tvk::cl::cluster_kernel, &q) != cudaSuccess) {
-            cudaGetLastError();
-            maxc = 0;
-        }
-        di.max_clusters[key] = maxc;
-    }
-    if (maxc <= 0) return false;
     const int64_t clusters = std::min<int64_t>(a.N, (int64_t)maxc);
     cfg.gridDim = dim3((unsigned)(clusters * c));
-    st = check_cuda(cudaLaunchKernelEx(&cfg, tvk::cl::cluster_kernel, p, n), "launch(tv cluster)");
+    st = check_cuda(cudaLaunchKernelEx(&cfg, keep ? tvk::cl::cluster_kernel<true> : tvk::cl::cluster_kernel<false>,
+                                       p, n),
+                    "launch(tv cluster)");
     return true;
 }
 

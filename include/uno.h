@@ -50,7 +50,8 @@
  *   UNO_VERIFY_LISTS=off     full-vocabulary verify without candidate lists
  *   UNO_VERIFY_ROW_CTAS=2    full-vocabulary row pass: two CTAs per SM
  *   UNO_TV_KERNEL=rows|teams TV loss: one CTA per row / two teams per CTA
- *   UNO_TV_CLUSTER=c         TV loss: clusters of c CTAs
+ *   UNO_TV_CLUSTER=c         TV loss: clusters of c CTAs (1 to 8, or 16)
+ *   UNO_TV_KEEP=0|1          TV loss: exp(student) recomputed / kept in shared memory
  * A workspace must be sized under the same settings as the call that uses it.
  */
 #ifndef UNO_H

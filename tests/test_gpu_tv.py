@@ -70,12 +70,19 @@ def test_tv_parity(N, V, dtype):
     ({"UNO_TV_CLUSTER": "16"}, 5, 151936),   # a larger cluster than needed
     ({"UNO_TV_CLUSTER": "16"}, 3, 64),       # half of the CTAs hold an empty slice
     ({"UNO_TV_CLUSTER": "16"}, 4, 1000),     # ragged last slice
-    ({"UNO_TV_CLUSTER": "2"}, 300, 151936),  # does not fit: falls back to the default size
+    ({"UNO_TV_CLUSTER": "2"}, 300, 151936),  # does not fit: falls back to the chosen size
+    ({"UNO_TV_CLUSTER": "6", "UNO_TV_KEEP": "0"}, 50, 151936),  # exp(student) recomputed
+    ({"UNO_TV_CLUSTER": "8", "UNO_TV_KEEP": "1"}, 40, 151936),  # exp(student) kept
+    ({"UNO_TV_KEEP": "1"}, 7, 5000),
+    ({"UNO_TV_CLUSTER": "3", "UNO_TV_KEEP": "0"}, 9, 4000),      # ragged slices at a size of 3
     ({"UNO_TV_KERNEL": "rows"}, 6, 151936),  # the per-row kernel on bf16 rows
     ({"UNO_TV_KERNEL": "teams"}, 37, 151936),  # the two-team kernel: many rows per team
     ({"UNO_TV_KERNEL": "teams"}, 5, 1000),
     ({"UNO_TV_KERNEL": "teams", "UNO_TV_CLUSTER": "16"}, 9, 4000),  # CTAs with empty slices
     ({"UNO_TV_KERNEL": "teams"}, 3, 166144),
+    ({"UNO_TV_KERNEL": "teams", "UNO_TV_KEEP": "0"}, 37, 151936),  # exp(student) recomputed
+    ({"UNO_TV_KERNEL": "teams", "UNO_TV_KEEP": "0"}, 5, 1000),
+    ({"UNO_TV_KERNEL": "teams", "UNO_TV_CLUSTER": "8"}, 11, 151936),  # keep does not fit at 8
 ])
 def test_tv_kernel_variants(monkeypatch, env, N, V):
     """Every kernel variant and cluster size gives the oracle's result."""
