@@ -881,20 +881,29 @@ Plan make_plan(int64_t M, int64_t d_in, int64_t d_out, int64_t rank, uno_dtype d
     Plan P{};
     P.m_tiles = (int)((M + BM - 1) / BM);
     // The CTA-pair form (256 x 256 tiles, one MMA stream over two SMs, each loading half of
-    // B: a third less operand traffic per FLOP) when there are enough of its tiles to fill
-    // the GPU (64 pairs or more); otherwise single-CTA 128 x BN tiles. With two K slabs per
-    // load the pair form measured 12-18% faster on the Qwen3-8B q/o/gate/up/down and the
-    // looped-3B gate/up/down projections, and slower on the narrow k/v ones and at M = 256.
-    // UNO_LORA_CG=1 or 2 fixes it.
-    const bool pair_ok = M >= 2 * BM && d_out % 256 == 0;
-    P.CG = pair_ok && ((M + 2 * BM - 1) / (2 * BM)) * (d_out / 256) >= 64 ? 2 : 1;
+    // B: a third less operand traffic per FLOP) when there are 32 or more of its tiles;
+    // otherwise single-CTA 128 x BN tiles. With two K slabs per load the pair form measured
+    // 12-18% faster on the Qwen3-8B q/o/gate/up/down and the looped-3B gate/up/down
+    // projections (64 pair tiles or more), 11% faster on the looped-3B gate/up at M = 256
+    // (43 pair tiles), and slower on the narrow k/v ones and on q/k/v/o/down at M = 256 (8 to
+    // 16 pair tiles). Narrower pair tiles (UNO_LORA_BN=64 or 128 with UNO_LORA_CG=2) measured
+    // slower than single CTAs on every narrow projection (Qwen3-8B k: 37.7 against 31.6 us).
+    // UNO_LORA_CG=1 or 2 fixes the form.
+    const bool pair_ok = M >= 2 * BM && d_out % 64 == 0;
+    const int64_t pair_tiles = d_out % 256 == 0 ? ((M + 2 * BM - 1) / (2 * BM)) * (d_out / 256) : 0;
+    P.CG = pair_ok && pair_tiles >= 32 ? 2 : 1;
     if (const char* e = getenv("UNO_LORA_CG")) {
         const int c = atoi(e);
         if (c == 1 || (c == 2 && pair_ok)) P.CG = c;
     }
     P.m_units = (int)((M + (int64_t)BM * P.CG - 1) / ((int64_t)BM * P.CG));
     if (P.CG == 2) {
-        P.BN = 256;
+        P.BN = d_out % 256 == 0 ? 256 : d_out % 128 == 0 ? 128 : 64;
+        // UNO_LORA_BN (64, 128 or 256, dividing d_out) fixes the pair tile width, for measurements
+        if (const char* e = getenv("UNO_LORA_BN")) {
+            const int bn = atoi(e);
+            if ((bn == 64 || bn == 128 || bn == 256) && d_out % bn == 0) P.BN = bn;
+        }
     } else {
         // A K step takes about as long at every tile width (its operand loads set the pace),
         // so the width is the one with the fewest waves of items over the SMs, the wider on a
@@ -1165,7 +1174,14 @@ uno_status gated_lora_launch(const GatedLoraArgs& g, void* workspace, cudaStream
         }
     p.status = device_status_ptr();
     p.trace = getenv("UNO_LORA_TRACE") ? reinterpret_cast<long long*>(ws + P.trace) : nullptr;
-    if (P.CG == 2) return launch_t<256, 2>(maps, p, P, stream);
+    if (P.CG == 2) {
+        switch (P.BN) {
+            case 64: return launch_t<64, 2>(maps, p, P, stream);
+            case 128: return launch_t<128, 2>(maps, p, P, stream);
+            case 256: return launch_t<256, 2>(maps, p, P, stream);
+        }
+        return set_error(UNO_ERR_UNSUPPORTED, "pair tile width %d", P.BN);
+    }
     switch (P.BN) {
         case 64: return launch_t<64, 1>(maps, p, P, stream);
         case 128: return launch_t<128, 1>(maps, p, P, stream);

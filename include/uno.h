@@ -33,7 +33,7 @@
  * Kernel variants (environment, read at each call; every variant computes the same result
  * up to floating-point summation order, and the defaults are the fastest measured ones)
  *   UNO_LORA_CG=1|2          gated LoRA on single CTAs / CTA pairs (256-row tiles, cta_group::2)
- *   UNO_LORA_BN=64|128|256   gated LoRA output tile width
+ *   UNO_LORA_BN=64|128|256   gated LoRA output tile width (with UNO_LORA_CG=2: pair tile width)
  *   UNO_LORA_SPLITS=n        adapter product X A^T split over K into n bf16 partials of T
  *   UNO_LORA_KSPLIT=n        output tiles split over K into n fp32 partials
  *   UNO_LORA_EPI=rows        output tiles stored by lanes (no shared-memory staging)

@@ -184,10 +184,12 @@ def test_split_adapter_path(monkeypatch, splits):
 
 
 @pytest.mark.parametrize("env", [{"UNO_LORA_CG": "2"}, {"UNO_LORA_CG": "2", "UNO_LORA_SPLITS": "3"},
+                                 {"UNO_LORA_CG": "2", "UNO_LORA_BN": "128"}, {"UNO_LORA_CG": "2", "UNO_LORA_BN": "64"},
                                  {"UNO_LORA_CG": "1"}])
 def test_cta_pair_and_single_forms(monkeypatch, env):
-    """The CTA-pair form (256-row tiles, one MMA stream over two SMs) and the single-CTA
-    form give the oracle's result on ragged shapes (M not a multiple of 256, rank 8/24/256)."""
+    """The CTA-pair form (256-row tiles of 256, 128 or 64 columns, one MMA stream over two
+    SMs) and the single-CTA form give the oracle's result on ragged shapes (M not a multiple
+    of 256, rank 8/24/256)."""
     for k, v in env.items():
         monkeypatch.setenv(k, v)
     for M, d_in, d_out, r in [(300, 1024, 512, 64), (1000, 768, 1024, 256), (257, 256, 768, 8),
