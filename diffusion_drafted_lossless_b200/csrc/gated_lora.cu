@@ -968,9 +968,10 @@ Plan make_plan(int64_t M, int64_t d_in, int64_t d_out, int64_t rank, uno_dtype d
     P.ksplit = (P.kt0 + P.kper - 1) / P.kper;  // every split has K tiles of (X, W0); the last also (T, B)
     P.n_items = P.n_adapter + P.m_units * P.n_tiles * P.ksplit;
     P.b_bytes = (uint32_t)(w / P.CG) * 128u;
-    // bf16 output tiles leave through 16 KB of shared-memory staging boxes and TMA stores
-    // (measured 2-5 % faster than per-lane row stores on the Qwen3-8B and looped-3B shapes);
-    // UNO_LORA_EPI=rows selects the row stores, which fp32 outputs, split K and CTA pairs use
+    // bf16 output tiles of single CTAs leave through 16 KB of shared-memory staging boxes and
+    // TMA stores (measured 2-5 % faster than per-lane row stores on the Qwen3-8B and looped-3B
+    // shapes; on CTA pairs the two measured the same, within 0.5 %, so pairs keep the row
+    // stores); UNO_LORA_EPI=rows selects the row stores, which fp32 outputs and split K use
     P.epi_tma = dtype == UNO_BF16 && P.ksplit == 1 && P.CG == 1;
     if (const char* e = getenv("UNO_LORA_EPI"))
         if (strcmp(e, "rows") == 0) P.epi_tma = 0;
