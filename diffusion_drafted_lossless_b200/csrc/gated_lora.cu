@@ -38,6 +38,9 @@
 #include <chrono>
 #include <cstdlib>
 #include <cstring>
+#include <map>
+#include <mutex>
+#include <utility>
 
 #include "gated_lora.cuh"
 
@@ -1055,13 +1058,28 @@ uno_status launch_t(const CUtensorMap (&maps)[6], Params& p, const Plan& P, cuda
     ++n_attr;
     cfg.numAttrs = n_attr;
     // resident units (CTAs or CTA pairs): an output tile may wait for its row unit's T
+    // (the occupancy query costs tens of microseconds of host time: cached per device and
+    // shared-memory size)
     int resident = 0;
     {
-        cudaLaunchConfig_t q = cfg;
-        q.gridDim = dim3(CG);
-        uno_status s = check_cuda(cudaOccupancyMaxActiveClusters(&resident, lora_gemm_kernel<BN, CG>, &q),
-                                  "cudaOccupancyMaxActiveClusters(gated lora)");
-        if (s != UNO_OK) return s;
+        static std::mutex mu;
+        static std::map<std::pair<int, size_t>, int> cache;
+        int dev = 0;
+        cudaGetDevice(&dev);
+        const auto key = std::make_pair(dev, (size_t)P.smem);
+        std::lock_guard<std::mutex> lock(mu);
+        const auto found = cache.find(key);
+        if (found != cache.end()) {
+            resident = found->second;
+        } else {
+            cudaLaunchConfig_t q = cfg;
+            q.gridDim = dim3(CG);
+            q.numAttrs = 1;  // the cluster shape alone
+            uno_status s = check_cuda(cudaOccupancyMaxActiveClusters(&resident, lora_gemm_kernel<BN, CG>, &q),
+                                      "cudaOccupancyMaxActiveClusters(gated lora)");
+            if (s != UNO_OK) return s;
+            cache[key] = resident;
+        }
     }
     if (resident < 1) return set_error(UNO_ERR_CUDA, "gated lora kernel does not fit on the GPU");
     const int units = p.n_items < resident ? p.n_items : resident;
