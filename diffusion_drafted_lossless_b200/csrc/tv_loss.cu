@@ -7,20 +7,25 @@
 //   mean = sum_{masked} TV / N_mask
 //   dmean/dstudent_v = q_v (s_v - sum_w q_w s_w) / N_mask,  s = 1/2 sign(q - p)
 //
-// Two kernels compute the same thing.
+// Three kernels compute the same thing.
 //
 // cluster_kernel (bf16 rows whose length is a multiple of 8 elements, the common case):
 // a thread-block cluster of CL CTAs owns one (teacher, student) row pair at a time, each
 // CTA holding a 1/CL slice of both rows in shared memory, so every logit is read from HBM
 // exactly once. The slices arrive by bulk copies (mbarrier completion) issued one row
 // ahead, so the next row streams in while this one is computed. Per row: warp maxima and
-// exps of both rows, keeping exp(student) in shared memory -> cluster reduction of the
-// (max, sum) pairs; A = sum of q over q > p and P = sum of p over q > p -> cluster
-// reduction; gradient. Each reduction is a per-warp st.async of its partial into every CTA
-// of the cluster. Rows overlap: row i's second reduction is in flight while the warps take
-// row i + 1's maxima and exps, and row i + 1's first while they write row i's gradient
-// (which recomputes exp(student), since row i + 1's exps have replaced it). That is 4
-// exponentials per element pair and 6 bytes of HBM traffic per element pair.
+// exps of both rows -> cluster reduction of the (max, sum) pairs; A = sum of q over q > p
+// and P = sum of p over q > p -> cluster reduction; gradient. Each reduction is a per-warp
+// st.async of its partial into every CTA of the cluster. Rows overlap: row i's second
+// reduction is in flight while the warps take row i + 1's maxima and exps, and row i + 1's
+// first while they write row i's gradient. exp(student) is either kept in shared memory
+// from the exp pass to the A, P pass (KEEP: 4 exponentials per element pair, 12 bytes of
+// shared memory per element) or recomputed there too (5 exponentials, 8 bytes, so a
+// smaller cluster fits: clusters of 6 at a 152k vocabulary). 6 bytes of HBM traffic per
+// element pair either way.
+//
+// team_kernel: the cluster kernel's computation with two teams of warps per CTA on
+// alternate rows (a variant; see its own comment).
 //
 // rows_kernel (fp32 rows, unaligned rows, rows too long for the cluster's shared memory):
 // one CTA per token row. Pass 1 streams both rows from HBM once and keeps per-thread
