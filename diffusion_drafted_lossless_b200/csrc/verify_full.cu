@@ -2079,6 +2079,11 @@ __device__ __forceinline__ f2 sub2(f2 a, f2 b) {
     asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
 }
+__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
+    f2 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
 __device__ __forceinline__ f2 mul2(f2 a, f2 b) {
     f2 d;
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
@@ -2330,7 +2335,9 @@ __global__ void __launch_bounds__(kThreads, CPS) row_kernel(Params p, RowRec* ro
         // bins and appends them to the warp's candidate list.
         __nv_bfloat162 mx2 = __floats2bfloat162_rn(-INFINITY, -INFINITY);
         double zr = 0.0;  // rest weights exp((x - F) / T)
-        float zb = 0.f;   // rest weights times |their ex2 argument| (for the error bound)
+        // rest weights times their ex2 argument, which is negative for every rest element: the
+        // error bound's sum of weights times |argument| is minus this (counted elements add 0)
+        f2 zb2 = pk(0.f, 0.f);
         uint32_t* hwp = sh.hw[warp];
         uint32_t* stg = sh.stage[warp];
         uint32_t* gl = lists ? lists + ((int64_t)r * kWarps + warp) * kListCap : nullptr;
@@ -2362,20 +2369,26 @@ __global__ void __launch_bounds__(kThreads, CPS) row_kernel(Params p, RowRec* ro
                 uint32_t cm = 0u;  // this lane's counted elements (bit e: element e of its 8)
                 if (ok) {
                     f2 acc = pk(0.f, 0.f);
+                    uint32_t mq[4];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         const uint32_t wq = w4[q];
                         const uint32_t m = __hge2_mask(bf2(wq), F2);  // x >= F: counted (0xFFFF per half)
+                        mq[q] = m;
                         mx2 = __hmax2(mx2, bf2(wq));
                         const f2 a = mul2(sub2(widen(wq), Ff), C2);
                         const bool in0 = (m & 0xFFFFu) != 0u, in1 = (m >> 16) != 0u;
                         const float x0 = ex2f(lo_of(a)), x1 = ex2f(hi_of(a));
-                        const float e0 = in0 ? 0.f : x0, e1 = in1 ? 0.f : x1;
-                        cm |= ((m & 1u) | ((m >> 15) & 2u)) << (2 * q);
-                        acc = add2(acc, pk(e0, e1));
-                        zb = fmaf(e0, fabsf(lo_of(a)), zb);
-                        zb = fmaf(e1, fabsf(hi_of(a)), zb);
+                        const f2 e = pk(in0 ? 0.f : x0, in1 ? 0.f : x1);
+                        acc = add2(acc, e);
+                        zb2 = fma2(e, a, zb2);
                     }
+                    // bit 2q, 2q + 1: the halves of word q. One byte of each half (0x00 or
+                    // 0xFF), four to a word, then each byte's low bit moved to bit 24 + its
+                    // index by one multiply (the partial products do not overlap)
+                    const uint32_t b0 = __byte_perm(mq[0], mq[1], 0x6420u) & 0x01010101u;
+                    const uint32_t b1 = __byte_perm(mq[2], mq[3], 0x6420u) & 0x01010101u;
+                    cm = ((b0 * 0x01020408u) >> 24) | (((b1 * 0x01020408u) >> 24) << 4);
                     zr += (double)lo_of(acc) + (double)hi_of(acc);
                 }
                 // this chunk's counted elements, in id order (lane, element), to the stage
@@ -2413,7 +2426,7 @@ __global__ void __launch_bounds__(kThreads, CPS) row_kernel(Params p, RowRec* ro
             float lm = fmaxf(__low2float(mx2), __high2float(mx2));
             lm = warp_max(lm);
             zr = warp_sum_f64(zr);
-            const double zbd = warp_sum_f64((double)zb);
+            const double zbd = warp_sum_f64(-((double)lo_of(zb2) + (double)hi_of(zb2)));
             __syncthreads();  // every thread has read the anchor's maxima
             if (lane == 0) {
                 sh.fmax[warp] = lm;
