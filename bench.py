@@ -3,7 +3,11 @@
 One step = one pass of the whole hot path over one batch of 64 sequences x block 16
 (V = 151936, Qwen3-8B shapes):
   1. the seven row-gated LoRA projections of one decoder layer (q, k, v, o, gate, up,
-     down) at M = 64 x 16 = 1024 rows, rank 128, position 0 of each block ungated;
+     down) at M = 64 x 16 = 1024 rows, rank 128, position 0 of each block ungated; k and v
+     share their input, so they run as one call over the concatenated weights (W0 and A
+     stacked, B block-diagonal: each adapter still acts only on its own outputs, and the
+     outputs are bit-identical to two calls); the FLOPs counted are the seven projections'
+     own;
   2. the lossless block verify over the [64, 16, 151936] verifier / drafter logits
      (bf16, T = 1, top-k 50, top-p 0.95; drafter correlated with the verifier, rho 0.8);
   3. the TV self-distillation loss and its gradient over the same 1024 logit rows
@@ -43,7 +47,7 @@ UNIT = "rows/s"
 WORKLOAD = "uno_step_b64_k16_v151936_qwen3_8b"
 LINEARS = W.QWEN3_8B
 VERIFY = W.SERVING_VERIFY
-LAUNCHES_PER_STEP = 7 + 2 + 2  # 7 projections (one kernel each) + verify (row streaming, finish) + TV (mask, rows)
+LAUNCHES_PER_STEP = 6 + 2 + 2  # 6 projection calls (k and v as one) + verify (row streaming, finish) + TV (mask, rows)
 
 
 def peaks():
@@ -113,6 +117,27 @@ class Step:
                              dtype=torch.uint8, device=dev)
             self.lin.append(dict(shape=sh, x=xs[sh.d_in], w0=t(inp["w0"]), a=t(inp["a"]), b=t(inp["b"]),
                                  g=torch.from_numpy(inp["gate"]).to(dev), y=y, ws=ws))
+        # the calls a step makes: k and v as one call over [W0_k; W0_v], [A_k; A_v] and
+        # diag(B_k, B_v) (rank 2r), whose output holds k's columns, then v's
+        by = {L["shape"].name: L for L in self.lin}
+        self.calls = []
+        for L in self.lin:
+            name = L["shape"].name
+            if name == "v" and "k" in by:
+                continue
+            if name == "k" and "v" in by:
+                K_, V_ = by["k"], by["v"]
+                dk, dv, r = K_["shape"].d_out, V_["shape"].d_out, w.rank
+                bf_ = torch.zeros((dk + dv, 2 * r), dtype=bf, device=dev)
+                bf_[:dk, :r] = K_["b"]
+                bf_[dk:, r:] = V_["b"]
+                self.calls.append(dict(x=K_["x"], w0=torch.cat([K_["w0"], V_["w0"]], 0).contiguous(),
+                                       a=torch.cat([K_["a"], V_["a"]], 0).contiguous(), b=bf_, g=K_["g"],
+                                       y=torch.empty((w.M, dk + dv), dtype=bf, device=dev),
+                                       ws=torch.empty(_lib.uno_gated_lora_linear_workspace_size(
+                                           w.M, K_["shape"].d_in, dk + dv, 2 * r), dtype=torch.uint8, device=dev)))
+                continue
+            self.calls.append(L)
         self.n_gated = int((W.row_gate(w.M, w.block) > 0).sum())
         self.x_host = {k: v.cpu() for k, v in xs.items()}
         v = VERIFY
@@ -132,7 +157,7 @@ class Step:
         self.tws = torch.empty(_lib.uno_tv_loss_workspace_size(n, v.V), dtype=torch.uint8, device=dev)
 
     def linears(self):
-        for L in self.lin:
+        for L in self.calls:
             self.lib.uno_gated_lora_linear(L["x"], L["w0"], L["a"], L["b"], L["g"], LINEARS.scale, L["y"],
                                            workspace=L["ws"])
 
@@ -164,7 +189,7 @@ class Step:
         self.hu = self.u.cpu().pin_memory()
         # every result of the step: the seven projection outputs, the verify's tokens, counts
         # and correction tokens, the per-token TV, the mean TV and the TV gradient
-        self.d_out = [L["y"] for L in self.lin] + [self.tokens, self.count, self.next, self.tv, self.mean, self.grad]
+        self.d_out = [L["y"] for L in self.calls] + [self.tokens, self.count, self.next, self.tv, self.mean, self.grad]
         self.h_out = [pinned_like(t) for t in self.d_out]
         self.h2d = sum(t.numel() * t.element_size() for t in list(self.hx.values()) + [self.hP, self.hQ, self.hu])
         self.d2h = sum(t.numel() * t.element_size() for t in self.h_out)

@@ -884,17 +884,17 @@ Plan make_plan(int64_t M, int64_t d_in, int64_t d_out, int64_t rank, uno_dtype d
     Plan P{};
     P.m_tiles = (int)((M + BM - 1) / BM);
     // The CTA-pair form (256 x 256 tiles, one MMA stream over two SMs, each loading half of
-    // B: a third less operand traffic per FLOP) when there are 32 or more of its tiles;
+    // B: a third less operand traffic per FLOP) when there are 40 or more of its tiles;
     // otherwise single-CTA 128 x BN tiles. With two K slabs per load the pair form measured
     // 12-18% faster on the Qwen3-8B q/o/gate/up/down and the looped-3B gate/up/down
     // projections (64 pair tiles or more), 11% faster on the looped-3B gate/up at M = 256
-    // (43 pair tiles), and slower on the narrow k/v ones and on q/k/v/o/down at M = 256 (8 to
-    // 16 pair tiles). Narrower pair tiles (UNO_LORA_BN=64 or 128 with UNO_LORA_CG=2) measured
+    // (43 pair tiles), and slower on the narrow k/v ones, on q/k/v/o/down at M = 256 (8 to
+    // 16 pair tiles) and on Qwen3-8B k and v as one call (32 pair tiles: 42.0 against 39.7 us). Narrower pair tiles (UNO_LORA_BN=64 or 128 with UNO_LORA_CG=2) measured
     // slower than single CTAs on every narrow projection (Qwen3-8B k: 37.7 against 31.6 us).
     // UNO_LORA_CG=1 or 2 fixes the form.
     const bool pair_ok = M >= 2 * BM && d_out % 64 == 0;
     const int64_t pair_tiles = d_out % 256 == 0 ? ((M + 2 * BM - 1) / (2 * BM)) * (d_out / 256) : 0;
-    P.CG = pair_ok && pair_tiles >= 32 ? 2 : 1;
+    P.CG = pair_ok && pair_tiles >= 40 ? 2 : 1;
     if (const char* e = getenv("UNO_LORA_CG")) {
         const int c = atoi(e);
         if (c == 1 || (c == 2 && pair_ok)) P.CG = c;

@@ -235,3 +235,23 @@ def test_output_epilogues(epi, monkeypatch):
         ref = _ref(inp)
         for _ in range(2):
             assert _rel(_run(inp, M, d_in, d_out, r), ref) <= TOL, (M, d_in, d_out, r)
+
+def test_k_and_v_as_one_call():
+    """k and v of the Qwen3-8B layer as one call over [W0_k; W0_v], [A_k; A_v] and
+    diag(B_k, B_v) (rank 2r): the output's column halves equal the two separate calls bit
+    for bit (the zero blocks of B add exact zeros) and the oracle on sampled rows."""
+    wl = W.QWEN3_8B
+    sh = {s.name: s for s in wl.shapes}
+    ik, iv = W.linear_inputs(wl, sh["k"]), W.linear_inputs(wl, sh["v"])
+    M, d_in, dk, r = wl.M, sh["k"].d_in, sh["k"].d_out, wl.rank
+    iv = dict(iv, x=ik["x"], gate=ik["gate"])  # the same input rows and gate
+    yk = _run(ik, M, d_in, dk, r)
+    yv = _run(iv, M, d_in, dk, r)
+    bf = np.zeros((2 * dk, 2 * r), dtype=ik["b"].dtype)
+    bf[:dk, :r] = ik["b"]
+    bf[dk:, r:] = iv["b"]
+    fused = dict(ik, w0=np.concatenate([ik["w0"], iv["w0"]]), a=np.concatenate([ik["a"], iv["a"]]), b=bf)
+    y = _run(fused, M, d_in, 2 * dk, 2 * r)
+    assert np.array_equal(y[:, :dk], yk) and np.array_equal(y[:, dk:], yv)
+    rows = _tile_rows(M, 7)
+    assert _rel(y[rows], _ref(fused, rows)) <= TOL
