@@ -329,6 +329,29 @@ def oracle_sample(n_seq=2, threads=None):
 
 
 # ---------------------------------------------------------------------------------------
+def fuse_kv(lw, rank):
+    """A layer's projection calls with k and v as one: (shape, W0, A, B) for k and for v
+    become one call over [W0_k; W0_v], [A_k; A_v] and diag(B_k, B_v) at rank 2 rank (they
+    share their input rows and gate; each adapter acts only on its own outputs)."""
+    import torch
+    by = {c[0].name: c for c in lw}
+    if "k" not in by or "v" not in by or by["k"][0].d_in != by["v"][0].d_in:
+        return lw
+    (sk, wk, ak, bk), (sv, wv, av, bv) = by["k"], by["v"]
+    b = torch.zeros((sk.d_out + sv.d_out, 2 * rank), dtype=bk.dtype, device=bk.device)
+    b[:sk.d_out, :rank] = bk
+    b[sk.d_out:, rank:] = bv
+    kv = (W.LinearShape("kv", sk.d_in, sk.d_out + sv.d_out), torch.cat([wk, wv], 0).contiguous(),
+          torch.cat([ak, av], 0).contiguous(), b)
+    out = []
+    for c in lw:
+        if c[0].name == "k":
+            out.append(kv)
+        elif c[0].name != "v":
+            out.append(c)
+    return out
+
+
 def measure_configs(torch, dev, lib, pk, reduce):
     """The other single-GPU configurations of the path, each timed with CUDA events after
     warm-up (inputs resident in HBM, larger than L2): the looped 3B-class step (7 gated
@@ -369,10 +392,12 @@ def measure_configs(torch, dev, lib, pk, reduce):
             seed = 8000 + 10 * l + i
             lw.append((sh, normal((sh.d_out, sh.d_in), w.w_sigma, seed), normal((w.rank, sh.d_in), w.w_sigma, seed + 3000),
                        normal((sh.d_out, w.rank), w.w_sigma, seed + 6000)))
-        layers.append(lw)
-    ys = {sh.name: torch.empty((M, sh.d_out), dtype=bf, device=dev) for sh in w.shapes}
-    wss = {sh.name: torch.empty(lib.uno_gated_lora_linear_workspace_size(M, sh.d_in, sh.d_out, w.rank),
-                                dtype=torch.uint8, device=dev) for sh in w.shapes}
+        layers.append(fuse_kv(lw, w.rank))
+    calls = [c[0] for c in layers[0]]  # the call shapes (k and v as one), the same in every layer
+    ranks = {c[0].name: c[2].shape[0] for c in layers[0]}
+    ys = {sh.name: torch.empty((M, sh.d_out), dtype=bf, device=dev) for sh in calls}
+    wss = {sh.name: torch.empty(lib.uno_gated_lora_linear_workspace_size(M, sh.d_in, sh.d_out, ranks[sh.name]),
+                                dtype=torch.uint8, device=dev) for sh in calls}
 
     def looped():
         for _ in range(W.LOOPED_3B_LOOPS):
@@ -385,15 +410,16 @@ def measure_configs(torch, dev, lib, pk, reduce):
     out["looped_3b_linears_m2048_x44"] = {"ms": ms, "tflops": fl / (ms * 1e-3) / 1e12,
                                           "frac": fl / (ms * 1e-3) / 1e12 / pk["bf16_tflops_sustained"],
                                           "peak": "bf16_tflops_sustained (a seconds-long loop)",
-                                          "launches": 7 * W.LOOPED_3B_LAYERS * W.LOOPED_3B_LOOPS}
+                                          "launches": len(calls) * W.LOOPED_3B_LAYERS * W.LOOPED_3B_LOOPS}
     # ---- one-loop drafting: the draft rows leave after the first loop; the verify rows (the
     # gate-0 rows, laid out first) go through the second loop alone, a prefix of the batch ----
     n_verify = M - n_gated
     gate_vf = torch.cat([torch.zeros(n_verify), torch.ones(n_gated)]).to(dev)
     gate_v = torch.zeros(n_verify, device=dev)
-    ys_v = {sh.name: torch.empty((n_verify, sh.d_out), dtype=bf, device=dev) for sh in w.shapes}
-    wss_v = {sh.name: torch.empty(lib.uno_gated_lora_linear_workspace_size(n_verify, sh.d_in, sh.d_out, w.rank),
-                                  dtype=torch.uint8, device=dev) for sh in w.shapes}
+    ys_v = {sh.name: torch.empty((n_verify, sh.d_out), dtype=bf, device=dev) for sh in calls}
+    wss_v = {sh.name: torch.empty(lib.uno_gated_lora_linear_workspace_size(n_verify, sh.d_in, sh.d_out,
+                                                                           ranks[sh.name]),
+                                  dtype=torch.uint8, device=dev) for sh in calls}
 
     def one_loop():
         for lw in layers:
@@ -411,7 +437,7 @@ def measure_configs(torch, dev, lib, pk, reduce):
         "ms": ms1, "tflops": fl1 / (ms1 * 1e-3) / 1e12,
         "frac": fl1 / (ms1 * 1e-3) / 1e12 / pk["bf16_tflops_sustained"],
         "saving_vs_two_loops": 1.0 - ms1 / ms, "verify_rows": n_verify,
-        "launches": 7 * W.LOOPED_3B_LAYERS * 2}
+        "launches": len(calls) * W.LOOPED_3B_LAYERS * 2}
     del layers, xs, ys, wss, ys_v, wss_v
     v = W.LOOPED_VERIFY
     P = normal((v.B, v.K, v.V), v.sigma, 9001)
@@ -591,7 +617,8 @@ def run_uno(args):
                        "seq_len": v.K, "parallelism": f"dp{world}",
                        "value": "B*K / mean verify time inside the timed steps (each step: 7 projections, "
                                 "verify, TV loss)",
-                       "linears": "Qwen3-8B layer: q,k,v,o,gate,up,down at M=1024, rank 128, scale 2",
+                       "linears": "Qwen3-8B layer: q,k,v,o,gate,up,down at M=1024, rank 128, scale 2; k and v as "
+                                  "one call over their concatenated weights",
                        "verify": "T=1, top-k 50, top-p 0.95, drafts sampled in-kernel",
                        "tv": "1024 rows x 151936, teacher=verifier, student=drafter logits",
                        "l2": "no flush: every input (logits 622 MB, weights 380 MB) exceeds L2 or is read once"},
